@@ -1,0 +1,175 @@
+/*
+ * hcadsa.h -- C ABI of the hybrid sparse attention forward (HCA + MLA-DSA) on
+ * NVIDIA B200 (sm_100a).  Library: sparse_attention_hca_b200/libhcadsa.so.
+ *
+ * The method, as the pages state it:
+ *   "Baidu open-sourced a brand-new pretraining model, still focusing on
+ *   efficiency with Flash" (blog.mirrorspeed.com), section "Hybrid sparse
+ *   attention, 1/7 full context access"; the same section of "Baidu
+ *   Open-Sources ERNIE 5.5 Flash Base: Efficient 280B MoE for Agents"
+ *   (besthub.dev, "Core Architectural Innovations", item 1); and the ai-club.cn
+ *   article, section "混合注意力（MLA + HCA）" (512-wide HCA heads, 256-wide
+ *   MLA heads).  HCA layers compress every 128 tokens into one cache entry and
+ *   attend over the compressed entries plus a short recent raw window; MLA
+ *   layers use DSA: an indexer scores earlier positions per query and
+ *   attention runs over the top-k positions only.
+ *
+ * Conventions for every call:
+ *   - All tensor pointers are DEVICE pointers owned by the caller; the library
+ *     never allocates, frees or retains them.  Tensors are dense, row-major,
+ *     last dimension contiguous.  bf16 tensors hold raw bfloat16 bit patterns.
+ *   - Every tensor pointer must be 16-byte aligned (HCADSA_ERR_ALIGN otherwise).
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *     default stream) and only enqueue kernels; they are thread-safe.
+ *   - Errors the host can see (null pointers, shapes, alignment, unsupported
+ *     sizes, short workspace, launch failures) are returned before anything is
+ *     enqueued.  Errors only the device can see (a bounded wait that expired,
+ *     an index out of range) are recorded in a per-device error word that
+ *     hcadsa_check_device_error() reads and clears.
+ *   - Query row r of batch b sits at absolute position t = q_offset + r.
+ *     Prefill: q_offset = 0, Lq = L.  Decode: Lq = 1, q_offset = t.
+ */
+#ifndef HCADSA_H_
+#define HCADSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t hcadsa_bf16; /* bfloat16 bit pattern */
+typedef void* hcadsa_stream;  /* cudaStream_t */
+
+typedef enum {
+  HCADSA_OK = 0,
+  HCADSA_ERR_NULL = -1,          /* a required pointer is NULL */
+  HCADSA_ERR_SHAPE = -2,         /* sizes inconsistent with each other */
+  HCADSA_ERR_ALIGN = -3,         /* a pointer is not 16-byte aligned */
+  HCADSA_ERR_UNSUPPORTED = -4,   /* valid but not implemented (e.g. head dim) */
+  HCADSA_ERR_WORKSPACE = -5,     /* workspace missing or too small */
+  HCADSA_ERR_CUDA = -6,          /* a CUDA runtime/driver call failed */
+  HCADSA_ERR_TIMEOUT = -7,       /* device: a bounded wait expired */
+  HCADSA_ERR_DEVICE_BOUNDS = -8  /* device: an index input was out of range */
+} hcadsa_status;
+
+/* Library version (major*10000 + minor*100 + patch). */
+int hcadsa_version(void);
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* hcadsa_status_string(hcadsa_status status);
+
+/*
+ * Synchronises `stream`, then returns and clears the device error word of the
+ * current device (HCADSA_OK if no kernel recorded an error).  Returns
+ * HCADSA_ERR_CUDA if the synchronisation itself failed.
+ */
+hcadsa_status hcadsa_check_device_error(hcadsa_stream stream);
+
+/*
+ * HCA block compression.  Source: mirrorspeed / besthub sections cited above
+ * ("every 128 tokens are compressed into one cache entry").  Compressor form
+ * (the pages leave it open): entry j of head h, channel c is
+ *     acc = 0; for i in 0..blk-1: acc = fma(w[i], X[b, blk*j + i, h, c], acc)
+ *     Xc[b, j, h, c] = bf16_round_nearest_even(acc)
+ * with fp32 accumulation in ascending i, applied to K and V with the same w.
+ * Only complete blocks are compressed: n_c = floor(L / blk) entries.
+ *
+ *   K, V   : [B, L, Hkv, d] bf16              (read)
+ *   w      : [blk] fp32                        (read)
+ *   Kc, Vc : [B, L/blk, Hkv, d] bf16           (written)
+ *   d must be a multiple of 8; 1 <= blk <= 1024.
+ */
+hcadsa_status hca_compress_kv(const hcadsa_bf16* K, const hcadsa_bf16* V, const float* w, hcadsa_bf16* Kc,
+                              hcadsa_bf16* Vc, int B, int L, int Hkv, int d, int blk, hcadsa_stream stream);
+
+/*
+ * Size in bytes of the workspace hca_attn_fwd needs for these sizes (0 when it
+ * needs none: prefill-shaped calls).  Decode-shaped calls (few query tokens
+ * over many keys) split the keys across thread blocks and combine partial
+ * softmax results through this workspace.
+ */
+size_t hca_attn_fwd_workspace_size(int B, int Lq, int q_offset, int Hq, int Hkv, int d, int n_c, int blk,
+                                   int W);
+
+/*
+ * HCA attention forward.  Source: the sections cited above ("attention is
+ * computed only on the compressed entries plus a recent short uncompressed
+ * window"; 512-wide heads).  Visible set of a query at position t (reading of
+ * the pages, which do not say how the two parts meet):
+ *     raw window  s in [max(0, t-W+1), t]
+ *     entries     j in [0, n_c(t)),  n_c(t) = max(0, floor((t-W+1)/blk))
+ * i.e. an entry is visible once every token it summarises lies before the
+ * window.  One softmax over the union, scores = scale * <q, k>:
+ *     O[b,r,h,:] = sum_k softmax_k(score) * v_k,   lse = log sum_k exp(score)
+ * Query head h reads K/V head h / (Hq/Hkv).
+ *
+ *   Q        : [B, Lq, Hq, d] bf16
+ *   Kc, Vc   : [B, n_c, Hkv, d] bf16   compressed entries (may be NULL iff n_c == 0)
+ *   Kw, Vw   : [B, n_w, Hkv, d] bf16   raw tokens; row i holds position win_start + i
+ *              (prefill: Kw = K, win_start = 0, n_w = L)
+ *   O        : [B, Lq, Hq, d] bf16     (written)
+ *   lse      : [B, Lq, Hq] fp32 natural-log log-sum-exp, or NULL
+ *   workspace: hca_attn_fwd_workspace_size(...) bytes (NULL allowed when that is 0)
+ * Requirements: d == 512; Hq % Hkv == 0 and (Hq/Hkv) divides 128; every query
+ * must have its window inside [win_start, win_start + n_w) and n_c(t) <= n_c.
+ */
+hcadsa_status hca_attn_fwd(const hcadsa_bf16* Q, const hcadsa_bf16* Kc, const hcadsa_bf16* Vc, int n_c,
+                           const hcadsa_bf16* Kw, const hcadsa_bf16* Vw, int win_start, int n_w, hcadsa_bf16* O,
+                           float* lse, int B, int Lq, int q_offset, int Hq, int Hkv, int d, int blk, int W,
+                           float scale, void* workspace, size_t workspace_bytes, hcadsa_stream stream);
+
+/*
+ * Size in bytes of the workspace dsa_index_topk needs: the int32 indexer score
+ * rows plus per-row selection state.
+ */
+size_t dsa_index_topk_workspace_size(int B, int Lq, int q_offset, int Lk, int k);
+
+/*
+ * DSA indexer + per-query top-k.  Source: mirrorspeed / besthub sections cited
+ * above ("a lightweight indexer ... scores historical positions for each
+ * query ... core attention is computed only on the top-k positions with the
+ * highest scores").  Indexer form (left open by the pages):
+ *     score[t, s] = sum_j w_idx[j] * sum_c q_idx[b, r, j, c] * k_idx[b, s, c]
+ * exact in int32.  Candidates of a query at t are the positions s <= t with
+ * s < Lk (its own position included).  The k candidates with the largest
+ * (score, -s) are kept -- equal scores go to the lower position -- and written
+ * in ascending position order, padded with -1 when fewer than k exist.
+ *
+ *   q_idx : [B, Lq, H_idx, d_idx] int8
+ *   k_idx : [B, Lk, d_idx] int8          (one key shared by the indexer heads)
+ *   w_idx : [H_idx] int32  (device)
+ *   idx   : [B, Lq, k] int32             (written)
+ *   ws    : workspace of dsa_index_topk_workspace_size(...) bytes
+ * Requirements: H_idx == 4, d_idx == 64, 1 <= k <= 4096, |w_idx| small enough
+ * that every score fits in [-2^30, 2^30] (checked on the device).
+ */
+hcadsa_status dsa_index_topk(const int8_t* q_idx, const int8_t* k_idx, const int32_t* w_idx, int32_t* idx,
+                             void* ws, size_t ws_bytes, int B, int Lq, int q_offset, int Lk, int H_idx, int d_idx,
+                             int k, hcadsa_stream stream);
+
+/*
+ * DSA sparse attention forward.  Source: mirrorspeed / besthub sections cited
+ * above, and the ai-club.cn section for the 256-wide MLA heads.  All Hq query
+ * heads read one shared K/V head (the MLA latent reading) and share the index
+ * row of their query:
+ *     O[b,r,h,:] = sum_{s in idx[b,r]} softmax_s(scale * <Q[b,r,h], K[b,s]>) V[b,s]
+ * Entries < 0 in idx are padding; the order of entries does not matter.
+ *
+ *   Q   : [B, Lq, Hq, d] bf16
+ *   K, V: [B, Lk, d] bf16
+ *   idx : [B, Lq, k] int32, entries in [0, Lk) or < 0
+ *   O   : [B, Lq, Hq, d] bf16 (written); lse: [B, Lq, Hq] fp32 or NULL
+ * Requirements: d == 256, Hq == 64, 1 <= k.  An entry >= Lk is skipped and
+ * recorded as HCADSA_ERR_DEVICE_BOUNDS.
+ */
+hcadsa_status dsa_sparse_attn_fwd(const hcadsa_bf16* Q, const hcadsa_bf16* K, const hcadsa_bf16* V,
+                                  const int32_t* idx, hcadsa_bf16* O, float* lse, int B, int Lq, int Lk, int Hq,
+                                  int d, int k, float scale, hcadsa_stream stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HCADSA_H_ */

@@ -1,0 +1,193 @@
+"""Python binding of libhcadsa.so: hybrid sparse attention forward (HCA + MLA-DSA) on B200.
+
+Thin argument marshalling over the C ABI declared in include/hcadsa.h: every step of
+the computation runs in the library's CUDA kernels.  PyTorch supplies device memory
+and the current CUDA stream.  There is no fallback: if the library is missing or the
+tensors are not on a CUDA device, the calls raise.
+
+Functions (same names as the C ABI):
+    hca_compress_kv(K, V, w, blk=128)                 -> (Kc, Vc)
+    hca_attn_fwd(Q, Kc, Vc, Kw, Vw, ...)              -> O  (or (O, lse))
+    dsa_index_topk(q_idx, k_idx, w_idx, k, ...)       -> idx
+    dsa_sparse_attn_fwd(Q, K, V, idx, ...)            -> O  (or (O, lse))
+    hcadsa_check_device_error()                       -> raises on a recorded device error
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import threading
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libhcadsa.so")
+
+_lock = threading.Lock()
+_lib = None
+
+STATUS = {
+    0: "HCADSA_OK", -1: "HCADSA_ERR_NULL", -2: "HCADSA_ERR_SHAPE", -3: "HCADSA_ERR_ALIGN",
+    -4: "HCADSA_ERR_UNSUPPORTED", -5: "HCADSA_ERR_WORKSPACE", -6: "HCADSA_ERR_CUDA",
+    -7: "HCADSA_ERR_TIMEOUT", -8: "HCADSA_ERR_DEVICE_BOUNDS",
+}
+
+
+class HcaDsaError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {STATUS.get(status, status)}")
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded C library (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise ImportError(f"{LIB_PATH} is missing; build it with "
+                                  "`python -m sparse_attention_hca_b200.build`")
+            L = ctypes.CDLL(LIB_PATH)
+            P, I, F, S = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+            L.hcadsa_version.restype = I
+            L.hcadsa_status_string.argtypes = [I]
+            L.hcadsa_status_string.restype = ctypes.c_char_p
+            L.hcadsa_check_device_error.argtypes = [P]
+            L.hcadsa_check_device_error.restype = I
+            L.hca_compress_kv.argtypes = [P, P, P, P, P, I, I, I, I, I, P]
+            L.hca_compress_kv.restype = I
+            L.hca_attn_fwd_workspace_size.argtypes = [I] * 9
+            L.hca_attn_fwd_workspace_size.restype = S
+            L.hca_attn_fwd.argtypes = [P, P, P, I, P, P, I, I, P, P, I, I, I, I, I, I, I, I, F, P, S, P]
+            L.hca_attn_fwd.restype = I
+            L.dsa_index_topk_workspace_size.argtypes = [I, I, I, I, I]
+            L.dsa_index_topk_workspace_size.restype = S
+            L.dsa_index_topk.argtypes = [P, P, P, P, P, S, I, I, I, I, I, I, I, P]
+            L.dsa_index_topk.restype = I
+            L.dsa_sparse_attn_fwd.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, F, P]
+            L.dsa_sparse_attn_fwd.restype = I
+            _lib = L
+    return _lib
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(status: int, what: str):
+    if status != 0:
+        raise HcaDsaError(status, what)
+
+
+def _need(t, dtype, name):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _bf16(t):
+    return t.view(torch.int16) if t is not None else None
+
+
+def hcadsa_check_device_error(stream=None):
+    """Synchronises the stream and raises if a kernel recorded a device-side error."""
+    _check(lib().hcadsa_check_device_error(_stream(stream)), "device")
+
+
+def hca_compress_kv(K, V, w, blk: int = 128, *, Kc=None, Vc=None, stream=None):
+    """K, V: [B, L, Hkv, d] bf16; w: [blk] fp32 -> Kc, Vc: [B, L // blk, Hkv, d] bf16."""
+    for t, n in ((K, "K"), (V, "V")):
+        _need(t, torch.bfloat16, n)
+    _need(w, torch.float32, "w")
+    B, L, Hkv, d = K.shape
+    if V.shape != K.shape or w.numel() != blk:
+        raise ValueError("shape mismatch")
+    shape = (B, L // blk, Hkv, d)
+    Kc = torch.empty(shape, dtype=torch.bfloat16, device=K.device) if Kc is None else Kc
+    Vc = torch.empty(shape, dtype=torch.bfloat16, device=K.device) if Vc is None else Vc
+    st = lib().hca_compress_kv(_ptr(K), _ptr(V), _ptr(w), _ptr(Kc), _ptr(Vc), B, L, Hkv, d, blk,
+                               _stream(stream))
+    _check(st, "hca_compress_kv")
+    return Kc, Vc
+
+
+def hca_attn_fwd(Q, Kc, Vc, Kw, Vw, *, win_start: int = 0, q_offset: int = 0, blk: int = 128,
+                 W: int = 128, scale: float | None = None, O=None, lse=None, return_lse=False,
+                 workspace=None, stream=None):
+    """Q: [B, Lq, Hq, d]; Kc/Vc: [B, n_c, Hkv, d] (or None); Kw/Vw: [B, n_w, Hkv, d]."""
+    _need(Q, torch.bfloat16, "Q")
+    _need(Kw, torch.bfloat16, "Kw")
+    _need(Vw, torch.bfloat16, "Vw")
+    B, Lq, Hq, d = Q.shape
+    n_w, Hkv = Kw.shape[1], Kw.shape[2]
+    n_c = 0 if Kc is None else Kc.shape[1]
+    if n_c:
+        _need(Kc, torch.bfloat16, "Kc")
+        _need(Vc, torch.bfloat16, "Vc")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    O = torch.empty_like(Q) if O is None else O
+    if return_lse and lse is None:
+        lse = torch.empty((B, Lq, Hq), dtype=torch.float32, device=Q.device)
+    L = lib()
+    ws_bytes = L.hca_attn_fwd_workspace_size(B, Lq, q_offset, Hq, Hkv, d, n_c, blk, W)
+    if ws_bytes and workspace is None:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=Q.device)
+    st = L.hca_attn_fwd(_ptr(Q), _ptr(Kc) if n_c else None, _ptr(Vc) if n_c else None, n_c, _ptr(Kw),
+                        _ptr(Vw), win_start, n_w, _ptr(O), _ptr(lse), B, Lq, q_offset, Hq, Hkv, d, blk, W,
+                        float(scale), _ptr(workspace), ws_bytes, _stream(stream))
+    _check(st, "hca_attn_fwd")
+    return (O, lse) if return_lse else O
+
+
+def dsa_index_topk_workspace_size(B, Lq, q_offset, Lk, k) -> int:
+    return lib().dsa_index_topk_workspace_size(B, Lq, q_offset, Lk, k)
+
+
+def dsa_index_topk(q_idx, k_idx, w_idx, k: int, *, q_offset: int = 0, idx=None, workspace=None,
+                   stream=None):
+    """q_idx: [B, Lq, 4, 64] int8; k_idx: [B, Lk, 64] int8; w_idx: [4] int32 -> idx [B, Lq, k] int32."""
+    _need(q_idx, torch.int8, "q_idx")
+    _need(k_idx, torch.int8, "k_idx")
+    _need(w_idx, torch.int32, "w_idx")
+    B, Lq, H_idx, d_idx = q_idx.shape
+    Lk = k_idx.shape[1]
+    idx = torch.empty((B, Lq, k), dtype=torch.int32, device=q_idx.device) if idx is None else idx
+    ws_bytes = dsa_index_topk_workspace_size(B, Lq, q_offset, Lk, k)
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=q_idx.device)
+    st = lib().dsa_index_topk(_ptr(q_idx), _ptr(k_idx), _ptr(w_idx), _ptr(idx), _ptr(workspace),
+                              workspace.numel() * workspace.element_size(), B, Lq, q_offset, Lk, H_idx,
+                              d_idx, k, _stream(stream))
+    _check(st, "dsa_index_topk")
+    return idx
+
+
+def dsa_sparse_attn_fwd(Q, K, V, idx, *, scale: float | None = None, O=None, lse=None,
+                        return_lse=False, stream=None):
+    """Q: [B, Lq, 64, 256]; K, V: [B, Lk, 256]; idx: [B, Lq, k] int32 -> O [B, Lq, 64, 256]."""
+    _need(Q, torch.bfloat16, "Q")
+    _need(K, torch.bfloat16, "K")
+    _need(V, torch.bfloat16, "V")
+    _need(idx, torch.int32, "idx")
+    B, Lq, Hq, d = Q.shape
+    Lk = K.shape[1]
+    k = idx.shape[-1]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    O = torch.empty_like(Q) if O is None else O
+    if return_lse and lse is None:
+        lse = torch.empty((B, Lq, Hq), dtype=torch.float32, device=Q.device)
+    st = lib().dsa_sparse_attn_fwd(_ptr(Q), _ptr(K), _ptr(V), _ptr(idx), _ptr(O), _ptr(lse), B, Lq, Lk,
+                                   Hq, d, k, float(scale), _stream(stream))
+    _check(st, "dsa_sparse_attn_fwd")
+    return (O, lse) if return_lse else O

@@ -1,0 +1,31 @@
+// host_common.h -- host-side helpers shared by the launchers: status mapping,
+// argument checks, TMA tensor-map encoding, the per-device error word.
+#pragma once
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "../../include/hcadsa.h"
+
+namespace hcadsa {
+
+// Address of the device error word for the current device (set up on first use).
+// Returns nullptr if the CUDA runtime call failed.
+int* device_error_ptr();
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline cudaStream_t as_stream(hcadsa_stream s) { return reinterpret_cast<cudaStream_t>(s); }
+
+// Encodes a tiled bf16 tensor map with 128-byte swizzle over a tensor of rank `rank`
+// (dims[0] innermost, element counts; strides_bytes[i] = byte stride of dim i+1).
+// Returns false if the driver rejects it.
+bool encode_tmap_bf16(CUtensorMap* map, int rank, void* base, const uint64_t* dims,
+                      const uint64_t* strides_bytes, const uint32_t* box, bool swizzle128);
+
+inline hcadsa_status launch_status() {
+  return cudaGetLastError() == cudaSuccess ? HCADSA_OK : HCADSA_ERR_CUDA;
+}
+
+}  // namespace hcadsa

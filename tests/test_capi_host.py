@@ -1,0 +1,100 @@
+"""C-ABI checks that need no GPU: the library loads, exports every function the
+header declares, and rejects invalid arguments with the documented status codes
+before touching any device memory."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "hcadsa.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from sparse_attention_hca_b200 import build
+
+    build.build()
+    import sparse_attention_hca_b200 as m
+
+    return m.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\*?\s*([a-z][a-z0-9_]+)\s*\(", text, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_the_four_calls():
+    names = declared_functions()
+    for n in ("hca_compress_kv", "hca_attn_fwd", "dsa_index_topk", "dsa_sparse_attn_fwd",
+              "hcadsa_check_device_error", "hcadsa_status_string"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for n in declared_functions():
+        assert hasattr(lib, n), n
+
+
+def test_status_strings_and_version(lib):
+    assert lib.hcadsa_version() >= 100
+    for code in range(0, -9, -1):
+        s = lib.hcadsa_status_string(code).decode()
+        assert s.startswith("HCADSA_")
+    assert b"unknown" in lib.hcadsa_status_string(-99)
+
+
+FAKE = ctypes.c_void_p(1 << 20)      # never dereferenced: every call below fails its checks first
+MISALIGNED = ctypes.c_void_p((1 << 20) + 8)
+
+
+def test_compress_argument_errors(lib):
+    f = lib.hca_compress_kv
+    assert f(None, FAKE, FAKE, FAKE, FAKE, 1, 256, 1, 512, 128, None) == -1
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 256, 0, 512, 128, None) == -2
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 256, 1, 500, 128, None) == -4
+    assert f(FAKE, MISALIGNED, FAKE, FAKE, FAKE, 1, 256, 1, 512, 128, None) == -3
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 100, 1, 512, 128, None) == 0   # no complete block: nothing to do
+
+
+def test_hca_attn_argument_errors(lib):
+    f = lib.hca_attn_fwd
+    args = dict(Q=FAKE, Kc=FAKE, Vc=FAKE, n_c=8, Kw=FAKE, Vw=FAKE, ws=0, n_w=1024, O=FAKE, lse=None, B=1,
+                Lq=1024, q0=0, Hq=16, Hkv=1, d=512, blk=128, W=128, scale=0.04, wsp=None, wsb=0, s=None)
+
+    def call(**kw):
+        a = dict(args, **kw)
+        return f(*a.values())
+
+    assert call(Q=None) == -1
+    assert call(Hkv=3) == -2             # 16 % 3
+    assert call(d=256) == -4
+    assert call(Hq=48, Hkv=1) == -4      # group 48 does not divide 128
+    assert call(O=MISALIGNED) == -3
+    assert call(n_w=1000) == -2          # window of the last query not stored
+    assert call(n_c=6) == -2             # entries of the last query not stored
+    assert call(Lq=0) == 0
+
+
+def test_dsa_argument_errors(lib):
+    t = lib.dsa_index_topk
+    assert t(None, FAKE, FAKE, FAKE, FAKE, 1 << 30, 1, 64, 0, 64, 4, 64, 16, None) == -1
+    assert t(FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 30, 1, 64, 0, 64, 8, 64, 16, None) == -4
+    assert t(FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 30, 1, 64, 0, 64, 4, 64, 0, None) == -2
+    assert t(FAKE, FAKE, FAKE, FAKE, None, 0, 1, 4096, 0, 4096, 4, 64, 16, None) == -5
+    assert t(FAKE, FAKE, FAKE, FAKE, FAKE, 16, 1, 4096, 0, 4096, 4, 64, 16, None) == -5
+    a = lib.dsa_sparse_attn_fwd
+    assert a(FAKE, FAKE, FAKE, FAKE, None, None, 1, 8, 8, 64, 256, 16, 0.06, None) == -1
+    assert a(FAKE, FAKE, FAKE, FAKE, FAKE, None, 1, 8, 8, 32, 256, 16, 0.06, None) == -4
+    assert a(FAKE, FAKE, FAKE, FAKE, FAKE, None, 1, 8, 8, 64, 512, 16, 0.06, None) == -4
+    assert a(FAKE, FAKE, MISALIGNED, FAKE, FAKE, None, 1, 8, 8, 64, 256, 16, 0.06, None) == -3
+
+
+def test_workspace_size_queries(lib):
+    assert lib.dsa_index_topk_workspace_size(1, 32768, 0, 32768, 2048) == 32768 * 32768 * 4
+    assert lib.dsa_index_topk_workspace_size(2, 1, 1048575, 1048576, 2048) == 2 * 1048576 * 4
+    assert lib.hca_attn_fwd_workspace_size(1, 32768, 0, 16, 1, 512, 256, 128, 128) == 0

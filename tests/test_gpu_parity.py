@@ -1,0 +1,327 @@
+"""GPU parity: the CUDA library (through its C ABI) against the CPU oracle.
+
+Bars: compression and top-k bit-exact; attention outputs (bf16) within max-abs 2e-2
+and mean-abs 2e-3 of the fp64 oracle, plus a relative RMS error <= 1e-2 (the absolute
+bars alone would accept an all-zero output at sigma = 1/sqrt(d)).  Inputs come from
+the seeded generators in synth; every expected value comes from the oracle.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+
+pytestmark = pytest.mark.gpu
+
+MAX_ABS, MEAN_ABS, REL_RMS = 2e-2, 2e-3, 1e-2
+
+
+@pytest.fixture(scope="module")
+def hd():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from sparse_attention_hca_b200 import build
+
+    build.build()
+    import sparse_attention_hca_b200 as m
+
+    oracle.build()
+    return m
+
+
+def bits(x: torch.Tensor) -> np.ndarray:
+    return x.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def check_attn(gpu: torch.Tensor, ref: np.ndarray, what: str, value_scale: float = 1.0):
+    """value_scale: standard deviation of V when it is not O(1) (stress inputs with sigma > 1);
+    the absolute bars are stated for O(1) values and scale with it, the relative bar does not."""
+    g = gpu.detach().float().cpu().numpy().astype(np.float64).reshape(ref.shape)
+    err = np.abs(g - ref)
+    rel = math.sqrt(float((err ** 2).sum()) / max(float((ref ** 2).sum()), 1e-300))
+    msg = f"{what}: max_abs={err.max():.3e} mean_abs={err.mean():.3e} rel_rms={rel:.3e}"
+    s = max(1.0, value_scale)
+    assert err.max() <= MAX_ABS * s and err.mean() <= MEAN_ABS * s and rel <= REL_RMS, msg
+    return msg
+
+
+def no_device_error(hd):
+    hd.hcadsa_check_device_error()
+
+
+# ------------------------------------------------------------------ compression
+
+@pytest.mark.parametrize("cfg", [
+    synth.HCA_TINY,
+    synth.HCA_32K,
+    synth.HcaConfig("ragged_L1000_hkv2", B=2, L=1000, Hq=4, Hkv=2),
+])
+def test_compress_bit_exact(hd, cfg):
+    inp = synth.hca_inputs(cfg)
+    Kc, Vc = hd.hca_compress_kv(inp["K"].cuda(), inp["V"].cuda(), inp["w"].cuda(), cfg.blk)
+    no_device_error(hd)
+    w = inp["w"].numpy()
+    assert np.array_equal(bits(Kc), oracle.hca_compress(bits(inp["K"]), w, cfg.blk))
+    assert np.array_equal(bits(Vc), oracle.hca_compress(bits(inp["V"]), w, cfg.blk))
+
+
+def test_compress_block_one_is_identity(hd):
+    cfg = synth.HcaConfig("blk1", B=1, L=77, Hq=1, Hkv=1, d=64, blk=1)
+    inp = synth.hca_inputs(cfg)
+    one = torch.ones(1, dtype=torch.float32, device="cuda")
+    Kc, _ = hd.hca_compress_kv(inp["K"].cuda(), inp["V"].cuda(), one, 1)
+    assert torch.equal(Kc.cpu(), inp["K"])
+
+
+# ------------------------------------------------------------------ HCA attention
+
+def _hca_gpu_and_oracle(hd, cfg, rows=None, W=None):
+    W = cfg.W if W is None else W
+    inp = synth.hca_inputs(cfg)
+    Kd, Vd, Qd = inp["K"].cuda(), inp["V"].cuda(), inp["Q"].cuda()
+    Kc, Vc = hd.hca_compress_kv(Kd, Vd, inp["w"].cuda(), cfg.blk)
+    O, lse = hd.hca_attn_fwd(Qd, Kc, Vc, Kd, Vd, blk=cfg.blk, W=W, return_lse=True)
+    no_device_error(hd)
+    w = inp["w"].numpy()
+    Kc_o = oracle.hca_compress(bits(inp["K"]), w, cfg.blk)
+    Vc_o = oracle.hca_compress(bits(inp["V"]), w, cfg.blk)
+    ref, ref_lse = oracle.hca_attn(bits(inp["Q"]), Kc_o, Vc_o, bits(inp["K"]), bits(inp["V"]), blk=cfg.blk,
+                                   W=W, rows=rows, with_lse=True)
+    Of = O.reshape(cfg.B * cfg.L, cfg.Hq, cfg.d)
+    lf = lse.reshape(cfg.B * cfg.L, cfg.Hq)
+    if rows is not None:
+        r = torch.as_tensor(rows, device="cuda")
+        Of, lf = Of[r], lf[r]
+    return Of, lf, ref, ref_lse
+
+
+def test_hca_tiny_all_rows(hd):
+    O, lse, ref, ref_lse = _hca_gpu_and_oracle(hd, synth.HCA_TINY)
+    print(check_attn(O, ref, "hca tiny"))
+    np.testing.assert_allclose(lse.cpu().numpy(), ref_lse, atol=2e-3, rtol=0)
+
+
+@pytest.mark.parametrize("cfg,W", [
+    (synth.HcaConfig("stress_sigma1_L1003_hq16", B=1, L=1003, Hq=16, Hkv=1, sigma=1.0), 128),
+    (synth.HcaConfig("stress_sigma1_L700_hq8_hkv2_B2", B=2, L=700, Hq=8, Hkv=2, sigma=1.0), 128),
+    (synth.HcaConfig("wide_window_L300", B=1, L=300, Hq=16, Hkv=1, sigma=1.0), 512),
+    (synth.HcaConfig("sharp_L600_blk64_W96", B=1, L=600, Hq=16, Hkv=1, blk=64, W=96, sigma=2.0), 96),
+])
+def test_hca_stress(hd, cfg, W):
+    O, lse, ref, ref_lse = _hca_gpu_and_oracle(hd, cfg, W=W)
+    print(check_attn(O, ref, cfg.name, value_scale=cfg.sigma or 1.0))
+    np.testing.assert_allclose(lse.cpu().numpy(), ref_lse, atol=2e-2, rtol=0)
+
+
+def _sample_rows(L, B=1, extra=()):
+    toks = {0, 1, 2, 126, 127, 128, 129, 254, 255, 256, 257, 383, 384, 1000, 4095, 4096, L // 2, L - 2, L - 1}
+    toks |= set(extra)
+    toks = sorted(t for t in toks if 0 <= t < L)
+    return np.array([b * L + t for b in range(B) for t in toks], np.int64)
+
+
+def test_hca_32k_sampled(hd):
+    cfg = synth.HCA_32K
+    rows = _sample_rows(cfg.L, extra=(8191, 16384, 32000))
+    O, lse, ref, ref_lse = _hca_gpu_and_oracle(hd, cfg, rows=rows)
+    print(check_attn(O, ref, "hca 32k sampled"))
+
+
+def test_hca_131k_sampled(hd):
+    cfg = synth.HCA_131K
+    rows = _sample_rows(cfg.L, extra=(65536, 100000, 131000))
+    O, lse, ref, ref_lse = _hca_gpu_and_oracle(hd, cfg, rows=rows)
+    print(check_attn(O, ref, "hca 131k sampled"))
+
+
+@pytest.mark.parametrize("B,t", [(2, 5000), (3, 130)])
+def test_hca_decode_form(hd, B, t):
+    """One query token per sequence at position t over [entries | window buffer]."""
+    d, Hq, blk, W = 512, 16, 128, 128
+    n_c = (t + 1) // blk
+    Kc = synth.normal_bf16((B, n_c, 1, d), 1.0, 7, "K")
+    Vc = synth.normal_bf16((B, n_c, 1, d), 1.0, 7, "V")
+    ws = max(0, t - W + 1)
+    Kw = synth.normal_bf16((B, t + 1 - ws, 1, d), 1.0, 8, "K")
+    Vw = synth.normal_bf16((B, t + 1 - ws, 1, d), 1.0, 8, "V")
+    Q = synth.normal_bf16((B, 1, Hq, d), 1.0, 9, "Q")
+    O = hd.hca_attn_fwd(Q.cuda(), Kc.cuda(), Vc.cuda(), Kw.cuda(), Vw.cuda(), win_start=ws, q_offset=t, blk=blk, W=W)
+    no_device_error(hd)
+    ref = oracle.hca_attn(bits(Q), bits(Kc), bits(Vc), bits(Kw), bits(Vw), win_start=ws, q_offset=t, blk=blk, W=W)
+    print(check_attn(O.reshape(B, Hq, d), ref, f"hca decode t={t}"))
+
+
+# ------------------------------------------------------------------ DSA indexer + top-k
+
+def _dsa_cfg(name, L, B=1, k=2048, sigma=None):
+    return synth.DsaConfig(name, B=B, L=L, Hq=64, k=k, sigma=sigma)
+
+
+@pytest.mark.parametrize("L,k,B", [(3000, 2048, 1), (700, 64, 2), (200, 16, 1), (130, 200, 1)])
+def test_topk_bit_exact_all_rows(hd, L, k, B):
+    cfg = _dsa_cfg("topk", L, B=B, k=k)
+    inp = synth.dsa_inputs(cfg)
+    idx = hd.dsa_index_topk(inp["q_idx"].cuda(), inp["k_idx"].cuda(), inp["w_idx"].cuda(), k)
+    no_device_error(hd)
+    ref = oracle.dsa_topk(inp["q_idx"].numpy(), inp["k_idx"].numpy(), inp["w_idx"].numpy(), k)
+    assert np.array_equal(idx.cpu().numpy().reshape(B * L, k), ref)
+
+
+def test_topk_heavy_ties(hd):
+    L, k = 2500, 300
+    g = torch.Generator().manual_seed(5)
+    q = torch.randint(-1, 2, (1, L, 4, 64), generator=g).to(torch.int8)
+    kk = torch.randint(-1, 2, (1, L, 64), generator=g).to(torch.int8)
+    w = torch.tensor([1, 1, 2, 1], dtype=torch.int32)
+    idx = hd.dsa_index_topk(q.cuda(), kk.cuda(), w.cuda(), k)
+    ref = oracle.dsa_topk(q.numpy(), kk.numpy(), w.numpy(), k)
+    assert np.array_equal(idx.cpu().numpy().reshape(L, k), ref)
+
+
+def test_topk_all_equal_scores(hd):
+    L, k = 600, 100
+    q = torch.zeros(1, L, 4, 64, dtype=torch.int8)
+    kk = synth.dsa_inputs(_dsa_cfg("x", L))["k_idx"]
+    idx = hd.dsa_index_topk(q.cuda(), kk.cuda(), torch.tensor([1, 2, 3, 4], dtype=torch.int32).cuda(), k)
+    exp = np.array([list(range(min(k, t + 1))) + [-1] * (k - min(k, t + 1)) for t in range(L)], np.int32)
+    assert np.array_equal(idx.cpu().numpy().reshape(L, k), exp)
+
+
+def test_topk_wide_weights_and_extreme_int8(hd):
+    L, k = 900, 50
+    g = torch.Generator().manual_seed(6)
+    q = torch.randint(-128, 128, (1, L, 4, 64), generator=g).to(torch.int8)
+    kk = torch.randint(-128, 128, (1, L, 64), generator=g).to(torch.int8)
+    w = torch.tensor([7, -3, 100, 1], dtype=torch.int32)
+    idx = hd.dsa_index_topk(q.cuda(), kk.cuda(), w.cuda(), k)
+    ref = oracle.dsa_topk(q.numpy(), kk.numpy(), w.numpy(), k)
+    assert np.array_equal(idx.cpu().numpy().reshape(L, k), ref)
+
+
+@pytest.mark.parametrize("B,t", [(2, 70000), (1, 3000)])
+def test_topk_decode_form(hd, B, t):
+    """Lq = 1 at position t (streaming scorer; t + 1 > shared-memory row capacity for 70000)."""
+    Lk = t + 1
+    g = torch.Generator().manual_seed(t)
+    q = torch.randint(-8, 9, (B, 1, 4, 64), generator=g).to(torch.int8)
+    kk = torch.randint(-8, 9, (B, Lk, 64), generator=g).to(torch.int8)
+    w = torch.tensor([1, 4, 2, 3], dtype=torch.int32)
+    idx = hd.dsa_index_topk(q.cuda(), kk.cuda(), w.cuda(), 2048, q_offset=t)
+    no_device_error(hd)
+    ref = oracle.dsa_topk(q.numpy(), kk.numpy(), w.numpy(), 2048, q_offset=t)
+    assert np.array_equal(idx.cpu().numpy().reshape(B, 2048), ref)
+
+
+def test_topk_32k_sampled_rows(hd):
+    cfg = synth.DSA_32K
+    inp = synth.dsa_inputs(cfg)
+    idx = hd.dsa_index_topk(inp["q_idx"].cuda(), inp["k_idx"].cuda(), inp["w_idx"].cuda(), cfg.k)
+    no_device_error(hd)
+    rows = _sample_rows(cfg.L, extra=(2046, 2047, 2048, 2049, 12345, 30000))
+    ref = oracle.dsa_topk(inp["q_idx"].numpy(), inp["k_idx"].numpy(), inp["w_idx"].numpy(), cfg.k, rows=rows)
+    got = idx.reshape(cfg.L, cfg.k)[torch.as_tensor(rows, device="cuda")].cpu().numpy()
+    assert np.array_equal(got, ref)
+
+
+# ------------------------------------------------------------------ DSA sparse attention
+
+def _dsa_attn_case(hd, cfg, rows, sigma_tag=""):
+    """GPU attention fed the ORACLE's index rows for the sampled queries."""
+    inp = synth.dsa_inputs(cfg)
+    idx_o = oracle.dsa_topk(inp["q_idx"].numpy(), inp["k_idx"].numpy(), inp["w_idx"].numpy(), cfg.k, rows=rows)
+    Qs = inp["Q"].reshape(cfg.B * cfg.L, 1, cfg.Hq, cfg.d)[torch.as_tensor(rows)]   # one query per sequence row
+    # every sampled row becomes its own "token" of a batch-1 call over the key sequence of its batch
+    outs = []
+    for b in range(cfg.B):
+        sel = (rows // cfg.L) == b
+        if not sel.any():
+            continue
+        q_b = Qs[torch.as_tensor(np.nonzero(sel)[0])].reshape(1, -1, cfg.Hq, cfg.d)
+        O = hd.dsa_sparse_attn_fwd(q_b.cuda(), inp["K"][b:b + 1].cuda(), inp["V"][b:b + 1].cuda(),
+                                   torch.as_tensor(idx_o[sel]).reshape(1, -1, cfg.k).cuda())
+        outs.append(O.reshape(-1, cfg.Hq, cfg.d))
+    no_device_error(hd)
+    ref = oracle.dsa_attn(bits(inp["Q"]), bits(inp["K"]), bits(inp["V"]), idx_o, rows=rows)
+    return torch.cat(outs), ref
+
+
+@pytest.mark.parametrize("L,k,sigma", [(3000, 2048, None), (2000, 256, 1.0), (300, 2048, 1.0), (500, 100, 2.0)])
+def test_dsa_attn_against_oracle(hd, L, k, sigma):
+    cfg = _dsa_cfg("dsa", L, k=k, sigma=sigma)
+    rows = _sample_rows(L, extra=(k - 1, k, k + 1, L - 3))
+    O, ref = _dsa_attn_case(hd, cfg, rows)
+    print(check_attn(O, ref, f"dsa L={L} k={k} sigma={sigma}", value_scale=sigma or 1.0))
+
+
+def test_dsa_pipeline_32k_sampled(hd):
+    """Indexer -> top-k -> sparse attention, all on the GPU at the 32K configuration."""
+    cfg = synth.DSA_32K
+    inp = synth.dsa_inputs(cfg)
+    dev = {k: v.cuda() for k, v in inp.items()}
+    idx = hd.dsa_index_topk(dev["q_idx"], dev["k_idx"], dev["w_idx"], cfg.k)
+    O = hd.dsa_sparse_attn_fwd(dev["Q"], dev["K"], dev["V"], idx)
+    no_device_error(hd)
+    rows = _sample_rows(cfg.L, extra=(2047, 2048, 20000))
+    idx_o = oracle.dsa_topk(inp["q_idx"].numpy(), inp["k_idx"].numpy(), inp["w_idx"].numpy(), cfg.k, rows=rows)
+    r = torch.as_tensor(rows, device="cuda")
+    assert np.array_equal(idx.reshape(cfg.L, cfg.k)[r].cpu().numpy(), idx_o)
+    ref = oracle.dsa_attn(bits(inp["Q"]), bits(inp["K"]), bits(inp["V"]), idx_o, rows=rows)
+    print(check_attn(O.reshape(cfg.L, cfg.Hq, cfg.d)[r], ref, "dsa 32k pipeline"))
+
+
+def test_dsa_padding_and_order(hd):
+    """Index rows with -1 padding in arbitrary places and shuffled order."""
+    cfg = _dsa_cfg("pad", 400, k=64, sigma=1.0)
+    inp = synth.dsa_inputs(cfg)
+    rng = np.random.default_rng(3)
+    idx = np.full((cfg.L, cfg.k), -1, np.int32)
+    for t in range(cfg.L):
+        n = min(cfg.k, t + 1, int(rng.integers(1, cfg.k + 1)))
+        sel = rng.choice(t + 1, size=n, replace=False)
+        pos = rng.choice(cfg.k, size=n, replace=False)
+        idx[t, pos] = sel
+    O = hd.dsa_sparse_attn_fwd(inp["Q"].cuda(), inp["K"].cuda(), inp["V"].cuda(),
+                               torch.as_tensor(idx).reshape(1, cfg.L, cfg.k).cuda())
+    no_device_error(hd)
+    ref = oracle.dsa_attn(bits(inp["Q"]), bits(inp["K"]), bits(inp["V"]), idx)
+    print(check_attn(O, ref, "dsa padded/shuffled"))
+
+
+def test_dsa_decode_1m_sampled_batch(hd):
+    """The 1M-context decode shape for 2 of the 32 sequences (each sequence is independent)."""
+    cfg = synth.DECODE_1M
+    B, t, Lk = 2, cfg.t, cfg.t + 1
+    g = 11
+    q_idx = synth.randint((B, 1, 4, 64), -8, 8, g, "q_idx", torch.int8)
+    k_idx = synth.randint((B, Lk, 64), -8, 8, g, "k_idx", torch.int8)
+    w_idx = synth.randint((4,), 1, 4, g, "w_idx", torch.int32)
+    Q = synth.normal_bf16((B, 1, 64, 256), 1.0, g, "Q")
+    K = synth.normal_bf16((B, Lk, 256), 1.0, g, "K")
+    V = synth.normal_bf16((B, Lk, 256), 1.0, g, "V")
+    idx = hd.dsa_index_topk(q_idx.cuda(), k_idx.cuda(), w_idx.cuda(), cfg.k, q_offset=t)
+    O = hd.dsa_sparse_attn_fwd(Q.cuda(), K.cuda(), V.cuda(), idx)
+    no_device_error(hd)
+    idx_o = oracle.dsa_topk(q_idx.numpy(), k_idx.numpy(), w_idx.numpy(), cfg.k, q_offset=t)
+    assert np.array_equal(idx.cpu().numpy().reshape(B, cfg.k), idx_o)
+    ref = oracle.dsa_attn(bits(Q), bits(K), bits(V), idx_o)
+    print(check_attn(O.reshape(B, 64, 256), ref, "dsa decode 1M"))
+
+
+def test_hca_decode_1m_sampled_batch(hd):
+    cfg = synth.DECODE_1M
+    B, t = 2, cfg.t
+    n_c = cfg.n_c
+    g = 12
+    Kc = synth.normal_bf16((B, n_c, 1, 512), 1.0, g, "K")
+    Vc = synth.normal_bf16((B, n_c, 1, 512), 1.0, g, "V")
+    ws = t - cfg.W + 1
+    Kw = synth.normal_bf16((B, cfg.W, 1, 512), 1.0, g + 1, "K")
+    Vw = synth.normal_bf16((B, cfg.W, 1, 512), 1.0, g + 1, "V")
+    Q = synth.normal_bf16((B, 1, 16, 512), 1.0, g, "Q")
+    O = hd.hca_attn_fwd(Q.cuda(), Kc.cuda(), Vc.cuda(), Kw.cuda(), Vw.cuda(), win_start=ws, q_offset=t)
+    no_device_error(hd)
+    ref = oracle.hca_attn(bits(Q), bits(Kc), bits(Vc), bits(Kw), bits(Vw), win_start=ws, q_offset=t)
+    print(check_attn(O.reshape(B, 16, 512), ref, "hca decode 1M"))
