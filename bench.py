@@ -1,0 +1,486 @@
+"""Benchmark: hybrid sparse attention prefill, one HCA layer + one MLA-DSA layer per step.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--no-decode]
+
+Step = the whole hot path over one batch of synthetic input (L = 32768 tokens):
+  HCA layer : hca_compress_kv (K, V -> 128:1 entries) + hca_attn_fwd (16 query heads, 1 K/V
+              head, d = 512, window 128)
+  DSA layer : dsa_index_topk (int8 indexer, 4 heads x 64, top-2048) + dsa_sparse_attn_fwd
+              (64 heads, shared K/V head, d = 256)
+value = tokens per second through both layers, summed over ranks (each rank runs its own
+sequence: weak scaling, no data-path collective).  Inputs (Q alone is 1.5 GiB) are larger
+than the 126 MB L2, so no flush is needed between steps.  A decode block (batch 32 at
+position 1,048,575) is measured after the timed loop and reported beside the headline.
+
+--impl reference times the CPU oracle (the only reference this method has) on a bounded
+row sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+L = 32768
+HCA = synth.HCA_32K
+DSA = synth.DSA_32K
+DEC = synth.DECODE_1M
+METRIC = "prefill attention tokens/s and TFLOP/s (% of B200 BF16 peak) per HCA / DSA layer"
+WORKLOAD = "hca_prefill_L32768_hq16_hkv1_d512 + dsa_prefill_L32768_h64_d256_k2048 (B=1 per rank)"
+
+
+# ----------------------------------------------------------------------------- work accounting
+
+def hca_visible_keys_per_head(L, W=128, blk=128):
+    tot = 0
+    for t in range(L):
+        s = t - W + 1
+        tot += (s // blk if s > 0 else 0) + (t - max(0, s) + 1)
+    return tot
+
+
+def dsa_keys_per_head(L, k=2048):
+    return sum(min(t + 1, k) for t in range(L))
+
+
+HCA_KEYS = hca_visible_keys_per_head(L)                   # 8,331,711
+DSA_KEYS = dsa_keys_per_head(L)                           # 65,012,736
+HCA_FLOP = 4.0 * HCA.d * HCA.Hq * HCA_KEYS                # algorithmic: QK^T + PV
+DSA_FLOP = 4.0 * DSA.d * DSA.Hq * DSA_KEYS
+COMPRESS_BYTES = 2 * (L * HCA.Hkv * HCA.d * 2) + 2 * ((L // 128) * HCA.Hkv * HCA.d * 2) + 128 * 4
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]), "src": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "src": "fallback"}
+
+
+def kernel_source_hash(name):
+    p = os.path.join(ROOT, "sparse_attention_hca_b200", "csrc", name)
+    h = hashlib.sha256()
+    for f in (p, os.path.join(ROOT, "sparse_attention_hca_b200", "csrc", "ptx.cuh")):
+        h.update(open(f, "rb").read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(summary_file, source_file):
+    """DRAM bytes per launch from a committed ncu summary, only if the kernel is unchanged since."""
+    p = os.path.join(ROOT, "profiles", summary_file)
+    if not os.path.exists(p):
+        return None
+    text = open(p).read()
+    m = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    h = re.search(r"kernel_source_sha256_16:\s*([0-9a-f]+)", text)
+    if not m or not h or h.group(1) != kernel_source_hash(source_file):
+        return None
+    return float(m.group(1))
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.dev = device_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{device_index}.csv")
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.fh, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.fh.close()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+# ----------------------------------------------------------------------------- our arm
+
+def make_inputs(device, seed):
+    """Bench inputs drawn on the device with torch's generator (same laws as synth, other values)."""
+    g = torch.Generator(device=device)
+
+    def normal(shape, sigma, tid):
+        g.manual_seed(seed * 1000 + tid)
+        return (torch.randn(*shape, generator=g, device=device) * sigma).to(torch.bfloat16)
+
+    def ints(shape, lo, hi, tid, dtype):
+        g.manual_seed(seed * 1000 + tid)
+        return torch.randint(lo, hi + 1, shape, generator=g, device=device, dtype=torch.int64).to(dtype)
+
+    sh, sd = 1 / math.sqrt(HCA.d), 1 / math.sqrt(DSA.d)
+    g.manual_seed(seed * 1000 + 4)
+    w = torch.rand(HCA.blk, generator=g, device=device) * (2.0 / HCA.blk)
+    return {
+        "hQ": normal((1, L, HCA.Hq, HCA.d), sh, 1), "hK": normal((1, L, HCA.Hkv, HCA.d), sh, 2),
+        "hV": normal((1, L, HCA.Hkv, HCA.d), sh, 3), "w": w,
+        "dQ": normal((1, L, DSA.Hq, DSA.d), sd, 11), "dK": normal((1, L, DSA.d), sd, 12),
+        "dV": normal((1, L, DSA.d), sd, 13),
+        "q_idx": ints((1, L, 4, 64), -8, 8, 15, torch.int8), "k_idx": ints((1, L, 64), -8, 8, 16, torch.int8),
+        "w_idx": ints((4,), 1, 4, 17, torch.int32),
+    }
+
+
+class Step:
+    """Pre-allocated outputs/workspace; run() enqueues the 5 kernels of one step."""
+
+    N_KERNELS = 5
+
+    def __init__(self, hd, x, device):
+        self.hd, self.x = hd, x
+        self.Kc = torch.empty((1, L // 128, 1, HCA.d), dtype=torch.bfloat16, device=device)
+        self.Vc = torch.empty_like(self.Kc)
+        self.hO = torch.empty_like(x["hQ"])
+        self.dO = torch.empty_like(x["dQ"])
+        self.idx = torch.empty((1, L, DSA.k), dtype=torch.int32, device=device)
+        ws = hd.dsa_index_topk_workspace_size(1, L, 0, L, DSA.k)
+        self.ws = torch.empty(ws, dtype=torch.uint8, device=device)
+
+    def run(self, ev=None):
+        hd, x = self.hd, self.x
+        if ev: ev[0].record()
+        hd.hca_compress_kv(x["hK"], x["hV"], x["w"], 128, Kc=self.Kc, Vc=self.Vc)
+        if ev: ev[1].record()
+        hd.hca_attn_fwd(x["hQ"], self.Kc, self.Vc, x["hK"], x["hV"], O=self.hO)
+        if ev: ev[2].record()
+        hd.dsa_index_topk(x["q_idx"], x["k_idx"], x["w_idx"], DSA.k, idx=self.idx, workspace=self.ws)
+        if ev: ev[3].record()
+        hd.dsa_sparse_attn_fwd(x["dQ"], x["dK"], x["dV"], self.idx, O=self.dO)
+        if ev: ev[4].record()
+
+
+def run_decode(hd, device, iters=5):
+    """Batch 32 single-token queries at t = 1,048,575: HCA layer and DSA layer, HBM-bound."""
+    B, t = DEC.B, DEC.t
+    g = torch.Generator(device=device)
+    g.manual_seed(777)
+    n_c = DEC.n_c
+    Kc = torch.randn(B, n_c, 1, 512, generator=g, device=device).to(torch.bfloat16)
+    Vc = torch.randn(B, n_c, 1, 512, generator=g, device=device).to(torch.bfloat16)
+    Kw = torch.randn(B, DEC.W, 1, 512, generator=g, device=device).to(torch.bfloat16)
+    Vw = torch.randn(B, DEC.W, 1, 512, generator=g, device=device).to(torch.bfloat16)
+    hQ = torch.randn(B, 1, 16, 512, generator=g, device=device).to(torch.bfloat16)
+    Lk = t + 1
+    k_idx = torch.randint(-8, 9, (B, Lk, 64), generator=g, device=device, dtype=torch.int8)
+    q_idx = torch.randint(-8, 9, (B, 1, 4, 64), generator=g, device=device, dtype=torch.int8)
+    w_idx = torch.randint(1, 5, (4,), generator=g, device=device, dtype=torch.int32)
+    K = torch.empty(B, Lk, 256, dtype=torch.bfloat16, device=device)
+    V = torch.empty(B, Lk, 256, dtype=torch.bfloat16, device=device)
+    for b in range(B):
+        K[b].normal_(generator=g)
+        V[b].normal_(generator=g)
+    dQ = torch.randn(B, 1, 64, 256, generator=g, device=device).to(torch.bfloat16)
+    hO = torch.empty_like(hQ)
+    dO = torch.empty_like(dQ)
+    idx = torch.empty(B, 1, DEC.k, dtype=torch.int32, device=device)
+    ws = torch.empty(hd.dsa_index_topk_workspace_size(B, 1, t, Lk, DEC.k), dtype=torch.uint8, device=device)
+    ws_start = t - DEC.W + 1
+
+    def step(ev=None):
+        if ev: ev[0].record()
+        hd.hca_attn_fwd(hQ, Kc, Vc, Kw, Vw, win_start=ws_start, q_offset=t, O=hO)
+        if ev: ev[1].record()
+        hd.dsa_index_topk(q_idx, k_idx, w_idx, DEC.k, q_offset=t, idx=idx, workspace=ws)
+        if ev: ev[2].record()
+        hd.dsa_sparse_attn_fwd(dQ, K, V, idx, O=dO)
+        if ev: ev[3].record()
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(iters)]
+    for i in range(iters):
+        step(evs[i])
+    torch.cuda.synchronize()
+    hca_ms = statistics.median(e[0].elapsed_time(e[1]) for e in evs)
+    idx_ms = statistics.median(e[1].elapsed_time(e[2]) for e in evs)
+    att_ms = statistics.median(e[2].elapsed_time(e[3]) for e in evs)
+    hca_bytes = B * ((n_c + DEC.W) * 512 * 2 * 2 + 16 * 512 * 2 * 2)
+    dsa_idx_bytes = B * Lk * 64
+    dsa_att_bytes = B * (DEC.k * 256 * 2 * 2 + 64 * 256 * 2 * 2)
+    out = {
+        "workload": "decode_B32_t1048575 (HCA 16h d512 over 8191 entries + 128 window; DSA 64h d256 top-2048 of 1M)",
+        "hca_us": hca_ms * 1e3, "hca_gbs": hca_bytes / hca_ms / 1e6,
+        "dsa_index_topk_us": idx_ms * 1e3, "dsa_index_gbs": dsa_idx_bytes / idx_ms / 1e6,
+        "dsa_attn_us": att_ms * 1e3, "dsa_attn_gbs": dsa_att_bytes / att_ms / 1e6,
+        "step_us": (hca_ms + idx_ms + att_ms) * 1e3,
+    }
+    del Kc, Vc, K, V, k_idx, ws
+    torch.cuda.empty_cache()
+    return out
+
+
+def e2e_measure(hd, x, device, steps):
+    """Same step through the C ABI with host buffers: H2D of every input from pinned memory and
+    D2H of both layer outputs inside the timed region."""
+    host = {k: v.cpu().pin_memory() for k, v in x.items()}
+    dev = {k: torch.empty_like(v) for k, v in x.items()}
+    stp = Step(hd, dev, device)
+    out_h = torch.empty(x["hQ"].shape, dtype=torch.bfloat16).pin_memory()
+    out_d = torch.empty(x["dQ"].shape, dtype=torch.bfloat16).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = out_h.numel() * 2 + out_d.numel() * 2
+
+    def one():
+        for k in host:
+            dev[k].copy_(host[k], non_blocking=True)
+        stp.run()
+        out_h.copy_(stp.hO, non_blocking=True)
+        out_d.copy_(stp.dO, non_blocking=True)
+
+    one()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        one()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    del dev, stp
+    return ms, h2d, d2h
+
+
+def cpu_sample(seconds_budget=20.0, n_hca=48, n_dsa=6):
+    """Times the oracle on a bounded sample of query tokens spread over [0, L)."""
+    import numpy as np
+
+    import oracle
+
+    oracle.build()
+    inp_h = synth.hca_inputs(synth.HcaConfig("s", B=1, L=L, Hq=1, Hkv=1))   # K, V full; Q unused
+    rng = np.random.default_rng(1)
+    bits = lambda t: t.contiguous().view(torch.int16).numpy().view(np.uint16)  # noqa: E731
+    Kh, Vh = bits(inp_h["K"]), bits(inp_h["V"])
+    w = inp_h["w"].numpy()
+    t0 = time.perf_counter()
+    Kc, Vc = oracle.hca_compress(Kh, w, 128), oracle.hca_compress(Vh, w, 128)
+    t_comp = time.perf_counter() - t0
+    toks_h = np.linspace(0, L - 1, n_hca).astype(np.int64)
+    Qh = bits(synth.normal_bf16((1, n_hca, HCA.Hq, HCA.d), 1 / math.sqrt(512), 5, "Q"))
+    t0 = time.perf_counter()
+    for i, t in enumerate(toks_h):
+        oracle.hca_attn(Qh[:, i:i + 1], Kc, Vc, Kh, Vh, q_offset=int(t))
+    t_hca = (time.perf_counter() - t0) / n_hca
+    di = synth.dsa_inputs(synth.DsaConfig("s", B=1, L=L, Hq=1))
+    toks_d = np.linspace(0, L - 1, n_dsa).astype(np.int64)
+    Qd = bits(synth.normal_bf16((1, n_dsa, DSA.Hq, DSA.d), 1 / 16, 6, "Q"))
+    qi = di["q_idx"].numpy()
+    t0 = time.perf_counter()
+    for i, t in enumerate(toks_d):
+        idx = oracle.dsa_topk(qi[:, t:t + 1], di["k_idx"].numpy(), di["w_idx"].numpy(), DSA.k, q_offset=int(t))
+        oracle.dsa_attn(Qd[:, i:i + 1], bits(di["K"]), bits(di["V"]), idx)
+    t_dsa = (time.perf_counter() - t0) / n_dsa
+    per_token = t_comp / L + t_hca + t_dsa   # mean cost of one token through both layers
+    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+    return {
+        "value": 1.0 / per_token, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+        "sample": (f"{n_hca} HCA rows and {n_dsa} DSA rows (top-k + attention) at positions spread evenly over "
+                   f"[0, {L}) plus full compression; per-token cost averaged and inverted"),
+        "sample_seconds": t_comp + t_hca * n_hca + t_dsa * n_dsa,
+    }
+
+
+def ours(args):
+    import sparse_attention_hca_b200 as hd
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=device)
+    hd.lib()
+    x = make_inputs(device, seed=synth.SEED + rank)
+    st = Step(hd, x, device)
+    for _ in range(args.warmup):
+        st.run()
+    torch.cuda.synchronize()
+    hd.hcadsa_check_device_error()
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record()
+    for i in range(args.steps):
+        st.run(evs[i])
+    t_end.record()
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    clk = clocks.stop()
+    hd.hcadsa_check_device_error()
+    ms_total = t_start.elapsed_time(t_end)
+    if dist:
+        tt = torch.tensor([ms_total], device=device)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms_total = float(tt.item())
+    ms_step = ms_total / args.steps
+    k_ms = [sum(e[i].elapsed_time(e[i + 1]) for e in evs) / args.steps for i in range(4)]
+    comp_ms, hca_ms, idx_ms, dsa_ms = k_ms
+    peaks = load_peaks()
+    hca_tf = HCA_FLOP / (hca_ms * 1e-3) / 1e12
+    dsa_tf = DSA_FLOP / (dsa_ms * 1e-3) / 1e12
+    peak_s = peaks["bf16_tflops_sustained"]
+
+    decode = None
+    e2e = None
+    if rank == 0 and not args.no_decode:
+        decode = run_decode(hd, device)
+        hd.hcadsa_check_device_error()
+    e2e_ms, h2d, d2h = e2e_measure(hd, x, device, steps=max(2, min(args.steps, 4)))
+    if dist:
+        tt = torch.tensor([e2e_ms], device=device)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e_ms = float(tt.item())
+    e2e = {"value": world * L / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+           "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_sample()
+    traffic = profiled_traffic("dsa_sparse_attn_fwd_L32768.md", "dsa_attn.cu")
+    line = {
+        "metric": METRIC,
+        "value": world * L / (ms_step * 1e-3),
+        "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded; Q/K/V ~N(0,1)/sqrt(d) bf16, int8 indexer U[-8,8], weights U[1,4], w~U(0,2/128))",
+        "config": {"workload": WORKLOAD, "global_batch": world, "seq_len": L, "parallelism": f"replicas{world}",
+                   "l2": "inputs larger than L2 (1.5 GiB of Q per step), no flush"},
+        "layers": {
+            "hca": {"compress_us": comp_ms * 1e3, "compress_gbs": COMPRESS_BYTES / (comp_ms * 1e-3) / 1e9,
+                    "attn_ms": hca_ms, "attn_tflops": hca_tf, "attn_pct_bf16_sustained": 100 * hca_tf / peak_s,
+                    "layer_tokens_per_s": L / ((comp_ms + hca_ms) * 1e-3)},
+            "dsa": {"index_topk_ms": idx_ms, "attn_ms": dsa_ms, "attn_tflops": dsa_tf,
+                    "attn_pct_bf16_sustained": 100 * dsa_tf / peak_s,
+                    "layer_tokens_per_s": L / ((idx_ms + dsa_ms) * 1e-3)},
+            "algorithmic_flop": {"hca_attn": HCA_FLOP, "dsa_attn": DSA_FLOP},
+        },
+        "roofline": {"kernel": "dsa_sparse_attn_fwd", "bound": "tensor", "achieved": dsa_tf,
+                     "peak": peak_s, "unit": "TFLOP/s", "frac": dsa_tf / peak_s,
+                     "peak_kind": f"bf16_tflops_sustained ({peaks['src']})",
+                     "frac_of_burst_peak": dsa_tf / peaks["bf16_tflops"], "traffic": traffic,
+                     "units_per_launch": f"{DSA_KEYS} visible keys x 64 heads x 4*256 flop"},
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": Step.N_KERNELS * args.steps,
+        "clocks": clk,
+        "decode": decode,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    per = []
+    cpu = None
+    for _ in range(args.warmup):
+        cpu_sample(n_hca=4, n_dsa=1)
+    for _ in range(args.steps):
+        cpu = cpu_sample(n_hca=16, n_dsa=2)
+        per.append(cpu["value"])
+    v = statistics.median(per)
+    cpu["value"] = v
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * L / v, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "global_batch": 1, "seq_len": L, "parallelism": "host cores"},
+        "cpu_baseline": cpu,
+        "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+    if args.impl == "reference":
+        reference(args)
+    else:
+        ours(args)
+
+
+if __name__ == "__main__":
+    main()
