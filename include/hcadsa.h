@@ -150,6 +150,30 @@ hcadsa_status dsa_index_topk(const int8_t* q_idx, const int8_t* k_idx, const int
                              int k, hcadsa_stream stream);
 
 /*
+ * DSA indexer + top-k without any device allocation by anyone.  The pages have no
+ * counterpart: this is a library convenience for callers that cannot allocate device
+ * memory -- code that must not call cudaMalloc/cudaFree on its hot path (those calls can
+ * stall the device), plugins hosted by a framework that owns all device memory, or callers
+ * with no workspace allocator at all.  Same arguments, computation and result as
+ * dsa_index_topk, minus the workspace: the int32 score rows go to a fixed scratch array of
+ * dsa_index_topk_noalloc_max_scratch_bytes() bytes (64 MiB) compiled into the library.
+ * Every GPU that loads the library holds that array until the process exits.
+ *   - Calls whose score rows need more than that (dsa_index_topk_workspace_size(...) >
+ *     the maximum) return HCADSA_ERR_WORKSPACE before anything is enqueued.  Example limits:
+ *     prefill up to 4096 x 4096, or decode (Lq = 1) of 16 sequences at 1M keys.
+ *   - The first call on each device looks up the array's device address (one
+ *     cudaGetSymbolAddress, no allocation); make that first call before any stream capture.
+ *   - All calls share the one array and it keeps the last call's scores.  Nothing in it needs
+ *     clearing (every score a call reads is written earlier in the same call), but calls whose
+ *     kernels overlap on the GPU (different streams, or several host threads) race on it:
+ *     serialise them.
+ */
+size_t dsa_index_topk_noalloc_max_scratch_bytes(void);
+hcadsa_status dsa_index_topk_noalloc(const int8_t* q_idx, const int8_t* k_idx, const int32_t* w_idx, int32_t* idx,
+                                     int B, int Lq, int q_offset, int Lk, int H_idx, int d_idx, int k,
+                                     hcadsa_stream stream);
+
+/*
  * DSA sparse attention forward.  Source: mirrorspeed / besthub sections cited
  * above, and the ai-club.cn section for the 256-wide MLA heads.  All Hq query
  * heads read one shared K/V head (the MLA latent reading) and share the index

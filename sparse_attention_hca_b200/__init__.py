@@ -65,6 +65,10 @@ def lib() -> ctypes.CDLL:
             L.dsa_index_topk_workspace_size.restype = S
             L.dsa_index_topk.argtypes = [P, P, P, P, P, S, I, I, I, I, I, I, I, P]
             L.dsa_index_topk.restype = I
+            L.dsa_index_topk_noalloc_max_scratch_bytes.argtypes = []
+            L.dsa_index_topk_noalloc_max_scratch_bytes.restype = S
+            L.dsa_index_topk_noalloc.argtypes = [P, P, P, P, I, I, I, I, I, I, I, P]
+            L.dsa_index_topk_noalloc.restype = I
             L.dsa_sparse_attn_fwd.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, F, P]
             L.dsa_sparse_attn_fwd.restype = I
             _lib = L
@@ -169,6 +173,22 @@ def dsa_index_topk(q_idx, k_idx, w_idx, k: int, *, q_offset: int = 0, idx=None, 
                               workspace.numel() * workspace.element_size(), B, Lq, q_offset, Lk, H_idx,
                               d_idx, k, _stream(stream))
     _check(st, "dsa_index_topk")
+    return idx
+
+
+def dsa_index_topk_noalloc(q_idx, k_idx, w_idx, k: int, *, q_offset: int = 0, idx=None, stream=None):
+    """dsa_index_topk for callers that cannot allocate device memory: the score rows go to a
+    fixed 64 MiB array inside the library (see include/hcadsa.h for its limits and sharing).
+    The output tensor is still the caller's; pass ``idx`` to avoid allocating it here."""
+    _need(q_idx, torch.int8, "q_idx")
+    _need(k_idx, torch.int8, "k_idx")
+    _need(w_idx, torch.int32, "w_idx")
+    B, Lq, H_idx, d_idx = q_idx.shape
+    Lk = k_idx.shape[1]
+    idx = torch.empty((B, Lq, k), dtype=torch.int32, device=q_idx.device) if idx is None else idx
+    st = lib().dsa_index_topk_noalloc(_ptr(q_idx), _ptr(k_idx), _ptr(w_idx), _ptr(idx), B, Lq, q_offset, Lk,
+                                      H_idx, d_idx, k, _stream(stream))
+    _check(st, "dsa_index_topk_noalloc")
     return idx
 
 

@@ -18,6 +18,8 @@
 //                             and the output is ascending.
 #include <cuda_bf16.h>
 
+#include <mutex>
+
 #include "host_common.h"
 #include "ptx.cuh"
 
@@ -458,5 +460,84 @@ extern "C" hcadsa_status dsa_index_topk(const int8_t* q_idx, const int8_t* k_idx
     return HCADSA_ERR_CUDA;
   select_kernel<<<(unsigned)(B * Lq), kSelThreads, smem, s>>>(need_scores ? static_cast<int32_t*>(ws) : nullptr,
                                                               idx, Lq, q_offset, Lk, k, stride);
+  return launch_status();
+}
+
+// ---------------------------------------------------------------------------------------------
+// dsa_index_topk_noalloc: the same indexer + top-k for callers that cannot allocate device
+// memory.  The score rows live in a fixed array compiled into this library instead of a
+// caller-provided workspace.
+// ---------------------------------------------------------------------------------------------
+namespace hcadsa {
+namespace {
+
+// Built-in score scratch: 16,777,216 int32 scores = 64 MiB per device, resident from the
+// moment the library's device code is loaded on a GPU until the process exits.
+constexpr size_t kNoAllocScratchBytes = size_t(64) << 20;
+static __device__ __align__(256) int32_t g_noalloc_scores[kNoAllocScratchBytes / sizeof(int32_t)];
+
+// Device address of g_noalloc_scores for the current device, looked up once per device.
+// The name g_noalloc_scores is only a host-side stand-in in host code; kernels must be given
+// the address that cudaGetSymbolAddress returns for the device they run on.
+int32_t* noalloc_scratch_for_current_device() {
+  static std::mutex mu;
+  static int32_t* ptr_by_device[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!ptr_by_device[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scores) != cudaSuccess || !p) return nullptr;
+    ptr_by_device[dev] = static_cast<int32_t*>(p);
+  }
+  return ptr_by_device[dev];
+}
+
+}  // namespace
+}  // namespace hcadsa
+
+extern "C" size_t dsa_index_topk_noalloc_max_scratch_bytes(void) { return hcadsa::kNoAllocScratchBytes; }
+
+extern "C" hcadsa_status dsa_index_topk_noalloc(const int8_t* q_idx, const int8_t* k_idx, const int32_t* w_idx,
+                                                int32_t* idx, int B, int Lq, int q_offset, int Lk, int H_idx,
+                                                int d_idx, int k, hcadsa_stream stream) {
+  using namespace hcadsa;
+  if (!q_idx || !k_idx || !w_idx || !idx) return HCADSA_ERR_NULL;
+  if (B < 0 || Lq < 0 || Lk < 0 || q_offset < 0 || k <= 0) return HCADSA_ERR_SHAPE;
+  if (H_idx != kHIdx || d_idx != kDIdx || k > 4096) return HCADSA_ERR_UNSUPPORTED;
+  if ((long long)q_offset + Lq > 2147483647LL - 1 || (long long)B * Lq > 2147483647LL) return HCADSA_ERR_UNSUPPORTED;
+  if (!aligned16(q_idx) || !aligned16(k_idx) || !aligned16(w_idx) || !aligned16(idx)) return HCADSA_ERR_ALIGN;
+  if (B == 0 || Lq == 0) return HCADSA_OK;
+  const bool need_scores = (long long)q_offset + Lq > k && Lk > k;
+  const long long stride = score_row_stride(Lq, q_offset, Lk);
+  // size check first: a call that does not fit is refused before any CUDA call
+  if (need_scores && dsa_index_topk_workspace_size(B, Lq, q_offset, Lk, k) > kNoAllocScratchBytes)
+    return HCADSA_ERR_WORKSPACE;
+  cudaStream_t s = as_stream(stream);
+  int32_t* scores = nullptr;
+  if (need_scores) {
+    scores = noalloc_scratch_for_current_device();
+    if (!scores) return HCADSA_ERR_CUDA;
+    if (Lq >= 64) {
+      dim3 grid((unsigned)((stride + kKeyTilesPerCta * kKTile - 1) / (kKeyTilesPerCta * kKTile)),
+                (unsigned)((Lq + kQTile - 1) / kQTile), (unsigned)B);
+      if (grid.y > 65535u || grid.z > 65535u) return HCADSA_ERR_UNSUPPORTED;
+      const int smem_tiled = kQTile * kARow + 2 * kKTile * kBRow;
+      if (cudaFuncSetAttribute(score_tiled_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_tiled) !=
+          cudaSuccess)
+        return HCADSA_ERR_CUDA;
+      score_tiled_kernel<<<grid, 256, smem_tiled, s>>>(q_idx, k_idx, w_idx, scores, Lq, q_offset, Lk, stride);
+    } else {
+      dim3 grid((unsigned)((stride + kStreamThreads * kKeysPerThread - 1) / (kStreamThreads * kKeysPerThread)),
+                (unsigned)(B * Lq));
+      if (grid.y > 65535u) return HCADSA_ERR_UNSUPPORTED;
+      score_stream_kernel<<<grid, kStreamThreads, 0, s>>>(q_idx, k_idx, w_idx, scores, Lq, q_offset, Lk, stride);
+    }
+    if (cudaGetLastError() != cudaSuccess) return HCADSA_ERR_CUDA;
+  }
+  const int smem = kSelSmemCap * (int)sizeof(int);
+  if (cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return HCADSA_ERR_CUDA;
+  select_kernel<<<(unsigned)(B * Lq), kSelThreads, smem, s>>>(scores, idx, Lq, q_offset, Lk, k, stride);
   return launch_status();
 }
