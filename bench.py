@@ -465,6 +465,38 @@ def reference(args):
     }), flush=True)
 
 
+def only_kernel(args):
+    """Runs one library kernel alone at sequence length --seq-len (profiling driver): W warm-up
+    and K timed launches; prints a small JSON record (not the benchmark contract line)."""
+    import sparse_attention_hca_b200 as hd
+
+    global L
+    L = args.seq_len
+    device = torch.device("cuda", 0)
+    x = make_inputs(device, seed=synth.SEED)
+    st = Step(hd, x, device)
+    st.run()
+    torch.cuda.synchronize()
+    fn = {
+        "compress": lambda: hd.hca_compress_kv(x["hK"], x["hV"], x["w"], 128, Kc=st.Kc, Vc=st.Vc),
+        "hca_attn": lambda: hd.hca_attn_fwd(x["hQ"], st.Kc, st.Vc, x["hK"], x["hV"], O=st.hO),
+        "index_topk": lambda: hd.dsa_index_topk(x["q_idx"], x["k_idx"], x["w_idx"], DSA.k, idx=st.idx,
+                                                workspace=st.ws),
+        "dsa_attn": lambda: hd.dsa_sparse_attn_fwd(x["dQ"], x["dK"], x["dV"], st.idx, O=st.dO),
+    }[args.only]
+    for _ in range(args.warmup):
+        fn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    hd.hcadsa_check_device_error()
+    print(json.dumps({"kernel": args.only, "seq_len": L, "ms_per_launch": e0.elapsed_time(e1) / max(1, args.steps)}))
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -473,7 +505,12 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--only", choices=["compress", "hca_attn", "index_topk", "dsa_attn"],
+                    help="profiling driver: run one kernel alone at --seq-len")
+    ap.add_argument("--seq-len", type=int, default=L)
     args = ap.parse_args()
+    if args.only:
+        return only_kernel(args)
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
     if args.impl == "reference":

@@ -61,6 +61,12 @@ int hcadsa_version(void);
 const char* hcadsa_status_string(hcadsa_status status);
 
 /*
+ * Message of the last CUDA runtime error this thread saw inside the library (after a call
+ * returned HCADSA_ERR_CUDA); "" if none.  Static thread-local storage, never NULL.
+ */
+const char* hcadsa_last_error_string(void);
+
+/*
  * Synchronises `stream`, then returns and clears the device error word of the
  * current device (HCADSA_OK if no kernel recorded an error).  Returns
  * HCADSA_ERR_CUDA if the synchronisation itself failed.

@@ -53,6 +53,8 @@ def lib() -> ctypes.CDLL:
             L.hcadsa_version.restype = I
             L.hcadsa_status_string.argtypes = [I]
             L.hcadsa_status_string.restype = ctypes.c_char_p
+            L.hcadsa_last_error_string.argtypes = []
+            L.hcadsa_last_error_string.restype = ctypes.c_char_p
             L.hcadsa_check_device_error.argtypes = [P]
             L.hcadsa_check_device_error.restype = I
             L.hca_compress_kv.argtypes = [P, P, P, P, P, I, I, I, I, I, P]
@@ -86,6 +88,8 @@ def _stream(stream=None):
 
 def _check(status: int, what: str):
     if status != 0:
+        if status == -6:
+            what = f"{what} ({lib().hcadsa_last_error_string().decode(errors='replace')})"
         raise HcaDsaError(status, what)
 
 

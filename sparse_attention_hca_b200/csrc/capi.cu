@@ -2,6 +2,7 @@
 // and the host helpers the launchers share (TMA tensor-map encoding).
 #include <cudaTypedefs.h>
 
+#include <cstdio>
 #include <mutex>
 
 #include "host_common.h"
@@ -62,7 +63,15 @@ bool encode_tmap_bf16(CUtensorMap* map, int rank, void* base, const uint64_t* di
   return r == CUDA_SUCCESS;
 }
 
+thread_local char t_last_error[256] = "";
+
+void record_cuda_error(cudaError_t e) {
+  snprintf(t_last_error, sizeof(t_last_error), "%s: %s", cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
 }  // namespace hcadsa
+
+extern "C" const char* hcadsa_last_error_string(void) { return hcadsa::t_last_error; }
 
 extern "C" int hcadsa_version(void) { return 100; }
 

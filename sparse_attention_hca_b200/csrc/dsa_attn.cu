@@ -1,4 +1,4 @@
-// dsa_attn.cu -- DSA sparse attention forward on sm_100a (tcgen05 + TMEM).
+// dsa_attn.cu -- DSA sparse attention forward on sm_100a (tcgen05 + TMEM + TMA gather).
 //
 // Method: the mirrorspeed page, section "Hybrid sparse attention, 1/7 full context
 // access": in the MLA layers "the core attention is computed only on the top-k
@@ -6,21 +6,33 @@
 // section "混合注意力（MLA + HCA）").  All 64 query heads of a token share one K/V
 // head (the MLA latent reading) and the token's index row.
 //
-// Kernel design (one CTA per query token):
-//   * The 64 heads of a token are too few rows for a full-rate M=128 tcgen05 tile, so
-//     the contraction is transposed: the 128 gathered keys of a tile are M.
+// Kernel design (persistent: one CTA per SM walks query tokens tok = blockIdx.x + i*gridDim.x):
+//   * The 64 heads of a token are too few rows for a full-rate M=128 tcgen05 tile, so the
+//     contraction is transposed: the 128 gathered keys of a tile are M.
 //       S^T[key, head]  = K_g (A, K-major, 128 x 256)  *  Q^T (B, K-major, 64 heads)
 //       O^T[dv, head]  += V_g^T (A, MN-major, 2 x 128 dv) * P^T (B, MN-major, 64 heads)
-//     TMEM: O^T halves [0,64), [64,128); S^T double buffer [128,192), [192,256).
-//   * Producer warps (one thread per key row) gather K and V rows with cp.async into
-//     128B-swizzled 16 KB chunks of an 8-slot ring; the MMA warp consumes K_0, K_1, V_0,
-//     K_2, V_1, ... in exactly the order they were loaded.
-//   * Softmax warps: one thread per key (TMEM lane) holding its 64 head scores; per-head
-//     maxima come from a warp reduce-scatter (62 shuffles) plus a 4-warp combine in shared
-//     memory; lazy rescale (reference max moves only when exceeded by 2^8); P^T rows are
-//     written to shared memory as bf16 and handed to the tensor core after a proxy fence.
-//     Row sums are kept per thread and reduced once at the end.
+//     TMEM: O^T double-buffered per token [0,128) / [128,256) so one token's epilogue
+//     overlaps the next token's MMAs; S^T double-buffered per tile [256,320) / [320,384).
+//   * Warps 0-2 gather K and V rows with cp.async: one warp instruction moves one whole
+//     512-byte row (lane l -> 16 bytes of 64-column chunk l/8), written 128B-swizzled into a
+//     ring of 8 x 16 KB chunk slots; a tile's K (or V) occupies 4 consecutive slots, loaded in
+//     exactly the order warp 4 consumes them: K_0, K_1, V_0, K_2, V_1, ...  Completion is
+//     tracked with cp.async.mbarrier.arrive.noinc; the MMA thread issues a proxy fence after
+//     each wait so the tensor core sees the generic-proxy writes.  (Measured on B200: this
+//     reaches ~105 GB/s per SM from L2, TMA tile::gather4 of 4 x 128 B rows ~16 GB/s.)
+//     Q (32 KB, TMA) is reloaded per token once the previous token's last S^T MMA is done.
+//   * Warp 3, lane 0 issues every MMA.  Warps 4-7: softmax (one thread per key = TMEM lane,
+//     64 head scores each).  The first tile of a token sets the per-head reference max by a
+//     warp reduce-scatter + 4-warp combine; later tiles only check their scores against it and
+//     redo the reduction (and rescale O^T) when some score exceeds it by 2^8.  P^T rows go to
+//     shared memory; then the token's epilogue (normalise O^T, store O).
+//   * Index rows may hold padding (< 0) anywhere; a 128-entry tile without any valid entry
+//     is skipped, other invalid entries read row 0 and are masked.
+//   * Barrier phases continue across tokens: s_full/p_ready/pv_done are indexed by a global
+//     tile counter, q_full/q_empty/o_full/o_empty by a counter of tokens with work.
 #include <cuda_bf16.h>
+
+#include <mutex>
 
 #include "host_common.h"
 #include "ptx.cuh"
@@ -36,15 +48,16 @@ constexpr int kRingSlots = 8;
 constexpr int kQChunkBytes = kH * 128;     // 64 heads x 64 bf16
 constexpr int kQBytes = 4 * kQChunkBytes;  // 32 KB
 constexpr int kPBytes = kKeyTile * 128;    // 128 keys x 64 heads bf16
-constexpr int kMaxK = 4096;
+constexpr int kMaxK = 4096;                // 32 tiles: one bit per tile in a 32-bit mask
 constexpr int kSmemBytes = kQBytes + kRingSlots * kChunkBytes + 2 * kPBytes + 1024;
-constexpr int kProducerWarps = 4;
-constexpr int kSoftmaxWarps = 4;
-constexpr int kThreads = 32 * (kProducerWarps + 1 + kSoftmaxWarps);  // 288
-constexpr int kMmaWarp = kProducerWarps;                            // warp 4
-constexpr int kSoftmaxWarp0 = kProducerWarps + 1;                   // warps 5..8
+// 8 warps = 2 per SM sub-partition, so each thread may use up to 255 registers (each
+// sub-partition has a 16K-entry register file; a third warp there would cap it near 168).
+constexpr int kProducerWarps = 3;
+constexpr int kMmaWarp = 3;
+constexpr int kSoftmaxWarp0 = 4;
+constexpr int kThreads = 32 * 8;
+constexpr uint32_t kTmemS = 256;  // S^T buffers at columns 256 and 320
 constexpr float kLazyRescale = 8.0f;
-constexpr int kInFlight = 3;  // cp.async groups a producer thread keeps in flight
 
 struct Params {
   const uint16_t* K;
@@ -53,38 +66,57 @@ struct Params {
   uint16_t* O;
   float* lse;
   int* err;
-  int Lq, Lk, k;
+  int n_tok, Lq, Lk, k;
   float scale_log2;
 };
 
 struct __align__(8) Barriers {
-  uint64_t q_full;
+  uint64_t q_full, q_empty;
   uint64_t full[kRingSlots];
   uint64_t empty[kRingSlots];
   uint64_t s_full[2];
   uint64_t p_ready[2];
   uint64_t pv_done;
-  uint64_t o_full;  // one-shot: every PV of the work item has completed
+  uint64_t o_full[2];
+  uint64_t o_empty[2];
 };
 
 struct SoftShared {
-  float wred[kSoftmaxWarps][kH];
-  float m_ref[kH];
-  float alpha[kH];
-  float l_tot[kH];
+  float wred[4][kH];
+  __align__(16) float m_ref[kH];
+  __align__(16) float alpha[kH];  // rescale factors; 1/l in the epilogue
 };
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool valid) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(valid ? 16 : 0)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
+__device__ __forceinline__ bool idx_ok(int s, int Lk) { return s >= 0 && s < Lk; }
 
-__device__ __forceinline__ void softmax_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+// Arrives on bar once every cp.async this thread issued so far has landed (no pending-count bump).
+__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+// Bit j set iff tile j (entries [128j, 128j+128) of the row) holds a valid entry.  Whole warp.
+__device__ __forceinline__ uint32_t tile_mask_of_row(const int32_t* row, int k, int Lk, int lane) {
+  uint32_t mask = 0;
+  const int n_tiles = (k + kKeyTile - 1) / kKeyTile;
+  const bool vec = (k & 3) == 0;  // rows start 16-byte aligned
+  for (int j = 0; j < n_tiles; ++j) {
+    const int e = j * kKeyTile + lane * 4;
+    bool any = false;
+    if (vec && e + 3 < k) {
+      const int4 v = *reinterpret_cast<const int4*>(row + e);
+      any = idx_ok(v.x, Lk) | idx_ok(v.y, Lk) | idx_ok(v.z, Lk) | idx_ok(v.w, Lk);
+    } else {
+      for (int q = 0; q < 4; ++q)
+        if (e + q < k) any |= idx_ok(row[e + q], Lk);
+    }
+    if (__any_sync(0xffffffffu, any)) mask |= 1u << j;
+  }
+  return mask;
+}
 
 // Warp reduce-scatter of 64 per-lane values: afterwards lane l holds, in v[0] and v[1],
 // the reduction over all 32 lanes of heads 2l and 2l+1.
@@ -109,6 +141,21 @@ __device__ __forceinline__ void warp_reduce_scatter64(float (&v)[64], int lane) 
   reduce_scatter_stage<kMax, 4>(v, lane);
 }
 
+__device__ __forceinline__ void softmax_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+// Named barrier over the 128 softmax threads that also ORs a predicate across them.
+__device__ __forceinline__ bool softmax_bar_or(bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, 1, 128, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)pred)
+      : "memory");
+  return r != 0;
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
     dsa_attn_kernel(const __grid_constant__ CUtensorMap map_q, const Params p) {
   extern __shared__ uint8_t smem_raw[];
@@ -119,322 +166,394 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ Barriers bar;
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_flag;
-  __shared__ int s_idx[kMaxK];
-  __shared__ int s_nvalid;
-  __shared__ int s_wcount[kThreads / 32];
   __shared__ SoftShared ss;
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int row = blockIdx.x;  // flat b * Lq + r
-  const int b = row / p.Lq;
-
-  // ---- stable compaction of the valid index entries (all threads)
-  {
-    const int32_t* irow = p.idx + (size_t)row * p.k;
-    const int per = (p.k + kThreads - 1) / kThreads;
-    const int i0 = threadIdx.x * per;
-    int cnt = 0;
-    for (int i = i0; i < min(i0 + per, p.k); ++i) {
-      const int s = irow[i];
-      if (s >= p.Lk) raise_device_error(p.err, kErrDeviceBounds);
-      cnt += (s >= 0 && s < p.Lk);
-    }
-    int x = cnt;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, x, o);
-      if (lane >= o) x += y;
-    }
-    if (lane == 31) s_wcount[warp] = x;
-    __syncthreads();
-    int before = 0;
-    for (int w = 0; w < warp; ++w) before += s_wcount[w];
-    int pos = before + x - cnt;
-    for (int i = i0; i < min(i0 + per, p.k); ++i) {
-      const int s = irow[i];
-      if (s >= 0 && s < p.Lk) s_idx[pos++] = s;
-    }
-    if (threadIdx.x == kThreads - 1) s_nvalid = before + x;
-  }
   if (threadIdx.x == 0) {
     mbar_init(&bar.q_full, 1);
+    mbar_init(&bar.q_empty, 1);
     for (int s = 0; s < kRingSlots; ++s) {
       mbar_init(&bar.full[s], kProducerWarps * 32);
       mbar_init(&bar.empty[s], 1);
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bar.s_full[s], 1);
-      mbar_init(&bar.p_ready[s], kSoftmaxWarps * 32);
+      mbar_init(&bar.p_ready[s], 128);
+      mbar_init(&bar.o_full[s], 1);
+      mbar_init(&bar.o_empty[s], 128);
     }
     mbar_init(&bar.pv_done, 1);
-    mbar_init(&bar.o_full, 1);
     abort_flag = 0;
     fence_mbarrier_init();
   }
   if (warp == kMmaWarp) {
-    tmem_alloc(&tmem_base_sh, 256);
+    tmem_alloc(&tmem_base_sh, 512);
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
-  const int n_valid = s_nvalid;
-  const int J = (n_valid + kKeyTile - 1) / kKeyTile;
+  const int Lk = p.Lk, k = p.k;
 
   if (warp < kProducerWarps) {
-    // ------------------------------------------------------------ gather producers
-    const int i = threadIdx.x;  // key row within a tile
-    if (i == 0 && J > 0) {
-      mbar_arrive_expect_tx(&bar.q_full, kQBytes);
-      for (int c = 0; c < 4; ++c) tma_load_3d(sQ + c * kQChunkBytes, &map_q, &bar.q_full, c * 64, 0, row);
-    }
-    const uint16_t* Kb = p.K + (size_t)b * p.Lk * kD;
-    const uint16_t* Vb = p.V + (size_t)b * p.Lk * kD;
+    // ------------------------------------------------------------ producers (cp.async rows)
     const uint32_t ring = smem_u32(sRing);
-    int slot = 0;
-    int pending_slot[kInFlight + 1] = {};  // FIFO of slots whose copies are not yet signalled
+    const uint16_t* Kg = p.K;
+    const uint16_t* Vg = p.V;
+    int slot = 0;  // always 0 or 4: a tile half takes 4 consecutive slots of the 8
     uint32_t phase = 0;
-    int n_pending = 0, pending_head = 0;
+    int it = 0;  // tokens with work so far
     bool ok = true;
-    auto issue_chunk = [&](const uint16_t* base, int tile, int c) {
-      const int key = tile * kKeyTile + i;
-      const bool valid = key < n_valid;
-      const uint16_t* src = base + (size_t)(valid ? s_idx[key] : 0) * kD + c * 64;
-      const uint32_t dst = ring + slot * kChunkBytes + i * 128;
-#pragma unroll
-      for (int piece = 0; piece < 8; ++piece)
-        cp_async16(dst + ((piece ^ (i & 7)) << 4), src + piece * 8, valid);
-      cp_async_commit();
-    };
-    auto retire_oldest = [&]() {
-      fence_proxy_async_smem();
-      mbar_arrive(&bar.full[pending_slot[pending_head]]);
-      pending_head = (pending_head + 1) % (kInFlight + 1);
-      --n_pending;
-    };
-    for (int step = 0; step <= J && ok; ++step) {
-      for (int part = 0; part < 2 && ok; ++part) {
-        // part 0: K chunks of tile `step`; part 1: V chunks of tile `step - 1`
-        const int tile = part == 0 ? step : step - 1;
-        if (tile < 0 || tile >= J) continue;
-        for (int c = 0; c < 4; ++c) {
-          ok = mbar_wait(&bar.empty[slot], phase ^ 1, &abort_flag, p.err);
-          if (!ok) break;
-          issue_chunk(part == 0 ? Kb : Vb, tile, c);
-          pending_slot[(pending_head + n_pending) % (kInFlight + 1)] = slot;
-          ++n_pending;
-          if (n_pending > kInFlight) {
-            cp_async_wait<kInFlight>();
-            retire_oldest();
-          }
-          if (++slot == kRingSlots) { slot = 0; phase ^= 1; }
+    const int chunk = lane >> 3, piece = lane & 7;
+    for (int tok = blockIdx.x; tok < p.n_tok && ok; tok += gridDim.x) {
+      const int32_t* row = p.idx + (size_t)tok * k;
+      const uint32_t mask = tile_mask_of_row(row, k, Lk, lane);
+      if (!mask) continue;
+      const int J = __popc(mask);
+      const size_t kv_row0 = (size_t)(tok / p.Lq) * Lk;  // first K/V row of this token's batch
+      // warp w gathers tile rows w, w+3, w+6, ...: lane l holds the K/V row of the warp's
+      // l-th row (ra) and (32+l)-th row (rb)
+      const int n_rows_w = (kKeyTile - warp + kProducerWarps - 1) / kProducerWarps;  // 43, 43, 42
+      int ra_prev = 0, rb_prev = 0, ra_cur = 0, rb_cur = 0;
+      uint32_t m = mask;
+      for (int step = 0; step <= J && ok; ++step) {
+        if (step < J) {
+          const int j = __ffs(m) - 1;
+          m &= m - 1;
+          const int ea = j * kKeyTile + warp + kProducerWarps * lane;
+          const int eb = j * kKeyTile + warp + kProducerWarps * (32 + lane);
+          const int sa = ea < k ? row[ea] : -1;
+          const int sb = (32 + lane < n_rows_w && eb < k) ? row[eb] : -1;
+          ra_cur = idx_ok(sa, Lk) ? sa : 0;
+          rb_cur = idx_ok(sb, Lk) ? sb : 0;
         }
+        for (int part = 0; part < 2 && ok; ++part) {
+          const bool is_k = part == 0;
+          if (is_k ? step >= J : step < 1) continue;
+          const int ra = is_k ? ra_cur : ra_prev, rb = is_k ? rb_cur : rb_prev;
+          const uint16_t* base = (is_k ? Kg : Vg) + kv_row0 * kD + lane * 8;
+          for (int c = 0; c < 4 && ok; ++c)
+            ok = mbar_wait(&bar.empty[slot + c], phase ^ 1, &abort_flag, p.err);
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) break;
+          const uint32_t dst0 = ring + (slot + chunk) * kChunkBytes;
+#pragma unroll 4
+          for (int i = 0; i < n_rows_w; ++i) {
+            const int trow = warp + kProducerWarps * i;  // row of the tile
+            const int src_row = __shfl_sync(0xffffffffu, i < 32 ? ra : rb, i & 31);
+            cp_async16(dst0 + trow * 128 + ((piece ^ (trow & 7)) << 4), base + (size_t)src_row * kD);
+          }
+#pragma unroll
+          for (int c = 0; c < 4; ++c) cp_async_arrive_noinc(&bar.full[slot + c]);
+          slot += 4;
+          if (slot == kRingSlots) { slot = 0; phase ^= 1; }
+          if (is_k && step == 0 && warp == 0) {
+            // Q of this token (after its first K tile is in flight), once the previous token's
+            // last S^T MMA no longer reads the buffer
+            ok = __all_sync(0xffffffffu, mbar_wait(&bar.q_empty, (it & 1) ^ 1, &abort_flag, p.err));
+            if (ok && lane == 0) {
+              mbar_arrive_expect_tx(&bar.q_full, kQBytes);
+              for (int c = 0; c < 4; ++c) tma_load_3d(sQ + c * kQChunkBytes, &map_q, &bar.q_full, c * 64, 0, tok);
+            }
+          }
+        }
+        ra_prev = ra_cur;
+        rb_prev = rb_cur;
       }
+      ++it;
     }
-    cp_async_wait<0>();
-    while (n_pending > 0) retire_oldest();
+    cp_async_wait_all();
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0 && J > 0) {
-      bool ok = mbar_wait(&bar.q_full, 0, &abort_flag, p.err);
-      tc_fence_after();
-      int slot = 0;
-      uint32_t phase = 0;
-      const uint32_t sQa = smem_u32(sQ), sRa = smem_u32(sRing), sPa = smem_u32(sP);
-      const uint32_t idesc_s = idesc_bf16_f32(128, kH, false, false);
-      const uint32_t idesc_o = idesc_bf16_f32(128, kH, true, true);
-      for (int step = 0; ok && step <= J; ++step) {
-        if (step < J) {
-          const uint32_t tS = tmem + 128 + (step & 1) * kH;
-          for (int c = 0; c < 4 && ok; ++c) {
-            ok = mbar_wait(&bar.full[slot], phase, &abort_flag, p.err);
-            if (!ok) break;
-            tc_fence_after();
+    int slot = 0;
+    uint32_t phase = 0;
+    int it = 0;
+    uint32_t g = 0;  // global tile counter
+    bool ok = true;
+    const uint32_t sQa = smem_u32(sQ), sRa = smem_u32(sRing), sPa = smem_u32(sP);
+    const uint32_t idesc_s = idesc_bf16_f32(128, kH, false, false);
+    const uint32_t idesc_o = idesc_bf16_f32(128, kH, true, true);
+    for (int tok = blockIdx.x; tok < p.n_tok && ok; tok += gridDim.x) {
+      const int32_t* row = p.idx + (size_t)tok * k;
+      const uint32_t mask = tile_mask_of_row(row, k, Lk, lane);
+      if (!mask) continue;
+      const int J = __popc(mask);
+      const int ob = it & 1;
+      if (lane == 0) {
+        ok = mbar_wait(&bar.q_full, it & 1, &abort_flag, p.err);
+        tc_fence_after();
+        for (int step = 0; step <= J && ok; ++step) {
+          if (step < J) {
+            const uint32_t gs = g + step;
+            const uint32_t tS = tmem + kTmemS + (gs & 1) * kH;
+            for (int c = 0; c < 4 && ok; ++c) {
+              ok = mbar_wait(&bar.full[slot], phase, &abort_flag, p.err);
+              if (!ok) break;
+              fence_proxy_async_smem();  // cp.async (generic proxy) writes -> tensor core reads
+              tc_fence_after();
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              const uint64_t da = smem_desc_sw128(sRa + slot * kChunkBytes + k * 32, 16, 1024);
-              const uint64_t db = smem_desc_sw128(sQa + c * kQChunkBytes + k * 32, 16, 1024);
-              mma_ss(tS, da, db, idesc_s, (c | k) != 0);
+              for (int kk = 0; kk < 4; ++kk) {
+                const uint64_t da = smem_desc_sw128(sRa + slot * kChunkBytes + kk * 32, 16, 1024);
+                const uint64_t db = smem_desc_sw128(sQa + c * kQChunkBytes + kk * 32, 16, 1024);
+                mma_ss(tS, da, db, idesc_s, (c | kk) != 0);
+              }
+              mma_commit(&bar.empty[slot]);
+              if (++slot == kRingSlots) { slot = 0; phase ^= 1; }
             }
-            mma_commit(&bar.empty[slot]);
-            if (++slot == kRingSlots) { slot = 0; phase ^= 1; }
+            if (!ok) break;
+            mma_commit(&bar.s_full[gs & 1]);
+            if (step == J - 1) mma_commit(&bar.q_empty);
           }
-          if (!ok) break;
-          mma_commit(&bar.s_full[step & 1]);
-        }
-        if (step >= 1) {
-          const int j = step - 1;
-          ok = mbar_wait(&bar.p_ready[j & 1], (j >> 1) & 1, &abort_flag, p.err);
-          if (!ok) break;
-          tc_fence_after();
-          const uint32_t pbase = sPa + (j & 1) * kPBytes;
-          for (int hv = 0; hv < 2 && ok; ++hv) {
-            // V chunks 2hv, 2hv+1 sit in consecutive slots (slot is even here)
-            ok = mbar_wait(&bar.full[slot], phase, &abort_flag, p.err) &&
-                 mbar_wait(&bar.full[slot + 1], phase, &abort_flag, p.err);
+          if (step >= 1) {
+            const int j = step - 1;
+            const uint32_t gj = g + j;
+            if (j == 0) {  // O^T buffer ob must have been drained by the epilogue of token it-2
+              ok = mbar_wait(&bar.o_empty[ob], ((it >> 1) & 1) ^ 1, &abort_flag, p.err);
+              if (!ok) break;
+            }
+            ok = mbar_wait(&bar.p_ready[gj & 1], (gj >> 1) & 1, &abort_flag, p.err);
             if (!ok) break;
             tc_fence_after();
-            for (int kk = 0; kk < kKeyTile / 16; ++kk) {
-              const uint64_t da = smem_desc_sw128(sRa + slot * kChunkBytes + kk * 2048, kChunkBytes, 1024);
-              const uint64_t db = smem_desc_sw128(pbase + kk * 2048, kPBytes, 1024);
-              mma_ss(tmem + hv * kH, da, db, idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+            const uint32_t pbase = sPa + (gj & 1) * kPBytes;
+            for (int hv = 0; hv < 2 && ok; ++hv) {
+              // V chunks 2hv, 2hv+1 sit in consecutive slots (slot is even here)
+              ok = mbar_wait(&bar.full[slot], phase, &abort_flag, p.err) &&
+                   mbar_wait(&bar.full[slot + 1], phase, &abort_flag, p.err);
+              if (!ok) break;
+              fence_proxy_async_smem();
+              tc_fence_after();
+              for (int kk = 0; kk < kKeyTile / 16; ++kk) {
+                const uint64_t da = smem_desc_sw128(sRa + slot * kChunkBytes + kk * 2048, kChunkBytes, 1024);
+                const uint64_t db = smem_desc_sw128(pbase + kk * 2048, kPBytes, 1024);
+                mma_ss(tmem + ob * 128 + hv * kH, da, db, idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+              }
+              mma_commit(&bar.empty[slot]);
+              mma_commit(&bar.empty[slot + 1]);
+              slot += 2;
+              if (slot == kRingSlots) { slot = 0; phase ^= 1; }
             }
-            mma_commit(&bar.empty[slot]);
-            mma_commit(&bar.empty[slot + 1]);
-            slot += 2;
-            if (slot == kRingSlots) { slot = 0; phase ^= 1; }
+            if (!ok) break;
+            mma_commit(&bar.pv_done);
+            if (j == J - 1) mma_commit(&bar.o_full[ob]);
           }
-          if (!ok) break;
-          mma_commit(&bar.pv_done);
-          if (j == J - 1) mma_commit(&bar.o_full);
         }
       }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      slot = __shfl_sync(0xffffffffu, slot, 0);
+      phase = __shfl_sync(0xffffffffu, phase, 0);
+      g += J;
+      ++it;
     }
   } else {
     // ------------------------------------------------------------ softmax + epilogue
     const int sw = warp - kSoftmaxWarp0;  // 0..3
     const int quarter = warp & 3;         // TMEM lane quarter this warp may access
-    const int key_lane = quarter * 32 + lane;
+    const int kl = quarter * 32 + lane;   // key lane of a tile / d_v row of O^T
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const int tid = sw * 32 + lane;       // 0..127
-    float lpart[kH];
-#pragma unroll
-    for (int h = 0; h < kH; ++h) lpart[h] = 0.0f;
-    if (tid < kH) ss.m_ref[tid] = -INFINITY;
-    softmax_bar();
+    int it = 0;
+    uint32_t g = 0;
     bool ok = true;
     // No early exit in this loop: the four softmax warps meet at named barriers, so after an
     // abort every thread keeps walking the same barrier sequence (waits then fail fast).
-    for (int j = 0; j < J; ++j) {
-      ok = mbar_wait(&bar.s_full[j & 1], (j >> 1) & 1, &abort_flag, p.err) && ok;
-      tc_fence_after();
-      const bool valid = j * kKeyTile + key_lane < n_valid;
-      const uint32_t tS = tmem + lane_off + 128 + (j & 1) * kH;
-      float red[kH];
-      {
-        uint32_t u[32];
-        tmem_ld32(tS, u);
-        tmem_wait_ld();
-#pragma unroll
-        for (int h = 0; h < 32; ++h) red[h] = valid ? __uint_as_float(u[h]) * p.scale_log2 : -INFINITY;
-        tmem_ld32(tS + 32, u);
-        tmem_wait_ld();
-#pragma unroll
-        for (int h = 0; h < 32; ++h) red[32 + h] = valid ? __uint_as_float(u[h]) * p.scale_log2 : -INFINITY;
+    for (int tok = blockIdx.x; tok < p.n_tok; tok += gridDim.x) {
+      const int32_t* row = p.idx + (size_t)tok * k;
+      const uint32_t mask = tile_mask_of_row(row, k, Lk, lane);
+      uint16_t* obase = p.O + (size_t)tok * kH * kD;
+      if (!mask) {  // no valid entry: O = 0, lse = -inf
+        for (int e = tid; e < kH * kD / 8; e += 128) reinterpret_cast<uint4*>(obase)[e] = make_uint4(0, 0, 0, 0);
+        if (p.lse && tid < kH) p.lse[(size_t)tok * kH + tid] = -INFINITY;
+        continue;
       }
-      warp_reduce_scatter64<true>(red, lane);
-      ss.wred[sw][2 * lane] = red[0];
-      ss.wred[sw][2 * lane + 1] = red[1];
-      softmax_bar();
-      if (tid < kH) {
-        const float mt = fmaxf(fmaxf(ss.wred[0][tid], ss.wred[1][tid]), fmaxf(ss.wred[2][tid], ss.wred[3][tid]));
-        const float mo = ss.m_ref[tid];
-        float alpha = 1.0f, mn = mo;
-        if (mo == -INFINITY) {
-          mn = mt;
-        } else if (mt > mo + kLazyRescale) {
-          mn = mt;
-          alpha = fast_exp2(mo - mt);
-        }
-        ss.m_ref[tid] = mn;
-        ss.alpha[tid] = alpha;
-      }
-      softmax_bar();
-      bool rescale = false;
-#pragma unroll 8
-      for (int h = 0; h < kH; ++h) rescale |= ss.alpha[h] != 1.0f;
-      if (rescale) {
-        // O^T must hold every PV up to tile j-1 before it is rescaled
-        ok = mbar_wait(&bar.pv_done, (j - 1) & 1, &abort_flag, p.err) && ok;
+      const int J = __popc(mask);
+      const int ob = it & 1;
+      if (tid < kH) ss.m_ref[tid] = -INFINITY;
+      float lpart[kH];
+#pragma unroll
+      for (int h = 0; h < kH; ++h) lpart[h] = 0.0f;
+      uint32_t m = mask;
+      for (int jj = 0; jj < J; ++jj) {
+        const int j = __ffs(m) - 1;
+        m &= m - 1;
+        const uint32_t gs = g + jj;
+        const int e = j * kKeyTile + kl;
+        const int s_idx = e < k ? row[e] : -1;
+        const bool valid = idx_ok(s_idx, Lk);
+        if (s_idx >= Lk) raise_device_error(p.err, kErrDeviceBounds);
+        ok = mbar_wait(&bar.s_full[gs & 1], (gs >> 1) & 1, &abort_flag, p.err) && ok;
         tc_fence_after();
+        const uint32_t tS = tmem + lane_off + kTmemS + (gs & 1) * kH;
+        // Does any score of this tile exceed its head's reference max by more than 2^8?  The
+        // first tile of a token always runs the reduction (its reference is still -inf).
+        bool over = jj == 0;
+        if (!over) {
+          uint32_t u0[32], u1[32];
+          tmem_ld32_nowait(tS, u0);
+          tmem_ld32_nowait(tS + 32, u1);
+          tmem_wait_ld_regs2(u0, u1);
+          if (valid) {
+#pragma unroll
+            for (int c8 = 0; c8 < 16; ++c8) {
+              const float4 mr = *reinterpret_cast<const float4*>(&ss.m_ref[c8 * 4]);
+              const float r4[4] = {mr.x, mr.y, mr.z, mr.w};
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                const int h = c8 * 4 + q;
+                const float sc = __uint_as_float(h < 32 ? u0[h] : u1[h - 32]) * p.scale_log2;
+                over |= sc > r4[q] + kLazyRescale;
+              }
+            }
+          }
+        }
+        if (softmax_bar_or(over)) {
+          float red[kH];
+          {
+            uint32_t u0[32], u1[32];
+            tmem_ld32_nowait(tS, u0);
+            tmem_ld32_nowait(tS + 32, u1);
+            tmem_wait_ld_regs2(u0, u1);
+#pragma unroll
+            for (int h = 0; h < 32; ++h) {
+              red[h] = valid ? __uint_as_float(u0[h]) * p.scale_log2 : -INFINITY;
+              red[32 + h] = valid ? __uint_as_float(u1[h]) * p.scale_log2 : -INFINITY;
+            }
+          }
+          warp_reduce_scatter64<true>(red, lane);
+          ss.wred[sw][2 * lane] = red[0];
+          ss.wred[sw][2 * lane + 1] = red[1];
+          softmax_bar();
+          bool resc = false;
+          if (tid < kH) {
+            const float mt = fmaxf(fmaxf(ss.wred[0][tid], ss.wred[1][tid]), fmaxf(ss.wred[2][tid], ss.wred[3][tid]));
+            const float mo = ss.m_ref[tid];
+            float alpha = 1.0f, mn = mo;
+            if (mo == -INFINITY) {
+              mn = mt;
+            } else if (mt > mo + kLazyRescale) {
+              mn = mt;
+              alpha = fast_exp2(mo - mt);
+              resc = true;
+            }
+            ss.m_ref[tid] = mn;
+            ss.alpha[tid] = alpha;
+          }
+          if (softmax_bar_or(resc)) {
+            // O^T must hold every PV of this token up to tile jj-1 before it is rescaled
+            ok = mbar_wait(&bar.pv_done, (gs - 1) & 1, &abort_flag, p.err) && ok;
+            tc_fence_after();
+#pragma unroll
+            for (int hv = 0; hv < 2; ++hv) {
+#pragma unroll
+              for (int c = 0; c < 2; ++c) {
+                uint32_t u[32];
+                const uint32_t tO = tmem + lane_off + ob * 128 + hv * kH + c * 32;
+                tmem_ld32_nowait(tO, u);
+                tmem_wait_ld_regs(u);
+#pragma unroll
+                for (int h = 0; h < 32; ++h) u[h] = __float_as_uint(__uint_as_float(u[h]) * ss.alpha[c * 32 + h]);
+                tmem_st32(tO, u);
+              }
+            }
+            tmem_wait_st();
+#pragma unroll
+            for (int h = 0; h < kH; ++h) lpart[h] *= ss.alpha[h];
+          }
+        }
+        // P^T row of this key: 64 heads, bf16, 128B-swizzled (scores re-read from TMEM)
+        uint8_t* prow = sP + (gs & 1) * kPBytes + kl * 128;
+        {
+          uint32_t u0[32], u1[32];
+          tmem_ld32_nowait(tS, u0);
+          tmem_ld32_nowait(tS + 32, u1);
+          tmem_wait_ld_regs2(u0, u1);
+#pragma unroll
+          for (int c8 = 0; c8 < 8; ++c8) {
+            const float4 ma = *reinterpret_cast<const float4*>(&ss.m_ref[c8 * 8]);
+            const float4 mb = *reinterpret_cast<const float4*>(&ss.m_ref[c8 * 8 + 4]);
+            const float mr[8] = {ma.x, ma.y, ma.z, ma.w, mb.x, mb.y, mb.z, mb.w};
+            uint32_t w4[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const int h = c8 * 8 + 2 * q;
+              const uint32_t s0 = h < 32 ? u0[h] : u1[h - 32];
+              const uint32_t s1 = h + 1 < 32 ? u0[h + 1] : u1[h + 1 - 32];
+              float p0 = 0.0f, p1 = 0.0f;
+              if (valid) {
+                p0 = fast_exp2(fmaf(__uint_as_float(s0), p.scale_log2, -mr[2 * q]));
+                p1 = fast_exp2(fmaf(__uint_as_float(s1), p.scale_log2, -mr[2 * q + 1]));
+              }
+              lpart[h] += p0;
+              lpart[h + 1] += p1;
+              w4[q] = pack_bf16x2(p0, p1);
+            }
+            *reinterpret_cast<uint4*>(prow + ((c8 ^ (kl & 7)) << 4)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+          }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(&bar.p_ready[gs & 1]);
+      }
+      // ---- epilogue of this token
+      warp_reduce_scatter64<false>(lpart, lane);
+      ss.wred[sw][2 * lane] = lpart[0];
+      ss.wred[sw][2 * lane + 1] = lpart[1];
+      softmax_bar();
+      if (tid < kH) {  // per-head row sum -> 1/l (kept in ss.alpha) and log-sum-exp
+        const float l = ss.wred[0][tid] + ss.wred[1][tid] + ss.wred[2][tid] + ss.wred[3][tid];
+        ss.alpha[tid] = 1.0f / l;
+        if (p.lse) p.lse[(size_t)tok * kH + tid] = (ss.m_ref[tid] + __log2f(l)) * 0.69314718055994531f;
+      }
+      softmax_bar();
+      ok = mbar_wait(&bar.o_full[ob], (it >> 1) & 1, &abort_flag, p.err) && ok;
+      tc_fence_after();
+      {
+        __nv_bfloat16* ob16 = reinterpret_cast<__nv_bfloat16*>(obase);
 #pragma unroll
         for (int hv = 0; hv < 2; ++hv) {
+          const int dv = hv * 128 + kl;  // this lane's d_v row of O^T
+          uint32_t u0[32], u1[32];
+          tmem_ld32_nowait(tmem + lane_off + ob * 128 + hv * kH, u0);
+          tmem_ld32_nowait(tmem + lane_off + ob * 128 + hv * kH + 32, u1);
+          tmem_wait_ld_regs2(u0, u1);
 #pragma unroll
-          for (int c = 0; c < 2; ++c) {
-            uint32_t u[32];
-            const uint32_t tO = tmem + lane_off + hv * kH + c * 32;
-            tmem_ld32(tO, u);
-            tmem_wait_ld();
+          for (int h4 = 0; h4 < 16; ++h4) {
+            const float4 il = *reinterpret_cast<const float4*>(&ss.alpha[h4 * 4]);
+            const float inv[4] = {il.x, il.y, il.z, il.w};
 #pragma unroll
-            for (int h = 0; h < 32; ++h) u[h] = __float_as_uint(__uint_as_float(u[h]) * ss.alpha[c * 32 + h]);
-            tmem_st32(tO, u);
-          }
-        }
-        tmem_wait_st();
-#pragma unroll
-        for (int h = 0; h < kH; ++h) lpart[h] *= ss.alpha[h];
-      }
-      // P^T row of this key: 64 heads, bf16, 128B-swizzled (scores re-read from TMEM)
-      uint8_t* prow = sP + (j & 1) * kPBytes + key_lane * 128;
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        uint32_t u[32];
-        tmem_ld32(tS + hh * 32, u);
-        tmem_wait_ld();
-#pragma unroll
-        for (int c8 = 0; c8 < 4; ++c8) {
-          uint32_t w4[4];
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const int hl = c8 * 8 + 2 * q, h = hh * 32 + hl;
-            float p0 = 0.0f, p1 = 0.0f;
-            if (valid) {
-              p0 = fast_exp2(__uint_as_float(u[hl]) * p.scale_log2 - ss.m_ref[h]);
-              p1 = fast_exp2(__uint_as_float(u[hl + 1]) * p.scale_log2 - ss.m_ref[h + 1]);
+            for (int q = 0; q < 4; ++q) {
+              const int h = h4 * 4 + q;
+              const float o = __uint_as_float(h < 32 ? u0[h] : u1[h - 32]) * inv[q];
+              ob16[(size_t)h * kD + dv] = __float2bfloat16_rn(o);
             }
-            lpart[h] += p0;
-            lpart[h + 1] += p1;
-            w4[q] = pack_bf16x2(p0, p1);
           }
-          const int chunk = hh * 4 + c8;
-          *reinterpret_cast<uint4*>(prow + ((chunk ^ (key_lane & 7)) << 4)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
         }
       }
-      fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(&bar.p_ready[j & 1]);
-    }
-    // ---- final: row sums, normalisation, store
-    // pv_done may be two phases behind here, so its parity cannot be trusted: use o_full
-    if (ok && J > 0) ok = mbar_wait(&bar.o_full, 0, &abort_flag, p.err);
-    warp_reduce_scatter64<false>(lpart, lane);
-    ss.wred[sw][2 * lane] = lpart[0];
-    ss.wred[sw][2 * lane + 1] = lpart[1];
-    softmax_bar();
-    if (tid < kH) ss.l_tot[tid] = ss.wred[0][tid] + ss.wred[1][tid] + ss.wred[2][tid] + ss.wred[3][tid];
-    softmax_bar();
-    if (ok) {
-      tc_fence_after();
-      uint16_t* obase = p.O + (size_t)row * kH * kD;
-#pragma unroll
-      for (int hv = 0; hv < 2; ++hv) {
-        const int dv = hv * 128 + key_lane;  // this lane's d_v row of O^T
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          uint32_t u[32];
-          if (J > 0) {
-            tmem_ld32(tmem + lane_off + hv * kH + c * 32, u);
-            tmem_wait_ld();
-          }
-#pragma unroll
-          for (int h = 0; h < 32; ++h) {
-            const float l = ss.l_tot[c * 32 + h];
-            const float o = (J > 0 && l > 0.0f) ? __uint_as_float(u[h]) / l : 0.0f;
-            reinterpret_cast<__nv_bfloat16*>(obase)[(size_t)(c * 32 + h) * kD + dv] = __float2bfloat16_rn(o);
-          }
-        }
-      }
-      if (p.lse && tid < kH) {
-        const float l = ss.l_tot[tid];
-        p.lse[(size_t)row * kH + tid] = l > 0.0f ? (ss.m_ref[tid] + __log2f(l)) * 0.69314718055994531f : -INFINITY;
-      }
+      mbar_arrive(&bar.o_empty[ob]);
+      softmax_bar();  // wred / m_ref are rewritten by the next token
+      g += J;
+      ++it;
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == kMmaWarp) tmem_dealloc(tmem, 256);
+  if (warp == kMmaWarp) tmem_dealloc(tmem, 512);
+}
+
+int num_sms_current_device() {
+  static std::mutex mu;
+  static int cache[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!cache[dev]) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    cache[dev] = n;
+  }
+  return cache[dev];
 }
 
 }  // namespace
@@ -451,12 +570,14 @@ extern "C" hcadsa_status dsa_sparse_attn_fwd(const hcadsa_bf16* Q, const hcadsa_
       (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
     return HCADSA_ERR_ALIGN;
   if (B == 0 || Lq == 0) return HCADSA_OK;
-  if ((long long)B * Lq > 2147483647LL) return HCADSA_ERR_UNSUPPORTED;
+  if ((long long)B * Lq > 2147483647LL || (long long)B * Lk > 2147483647LL) return HCADSA_ERR_UNSUPPORTED;
   CUtensorMap mq;
-  const uint64_t dims[3] = {(uint64_t)kD, (uint64_t)kH, (uint64_t)B * Lq};
-  const uint64_t strides[2] = {(uint64_t)kD * 2, (uint64_t)kH * kD * 2};
-  const uint32_t box[3] = {64, (uint32_t)kH, 1};
-  if (!encode_tmap_bf16(&mq, 3, const_cast<hcadsa_bf16*>(Q), dims, strides, box, true)) return HCADSA_ERR_CUDA;
+  {
+    const uint64_t dims[3] = {(uint64_t)kD, (uint64_t)kH, (uint64_t)B * Lq};
+    const uint64_t strides[2] = {(uint64_t)kD * 2, (uint64_t)kH * kD * 2};
+    const uint32_t box[3] = {64, (uint32_t)kH, 1};
+    if (!encode_tmap_bf16(&mq, 3, const_cast<hcadsa_bf16*>(Q), dims, strides, box, true)) return HCADSA_ERR_CUDA;
+  }
   Params p;
   p.K = K;
   p.V = V;
@@ -464,12 +585,16 @@ extern "C" hcadsa_status dsa_sparse_attn_fwd(const hcadsa_bf16* Q, const hcadsa_
   p.O = O;
   p.lse = lse;
   p.err = device_error_ptr();
+  p.n_tok = B * Lq;
   p.Lq = Lq;
   p.Lk = Lk;
   p.k = k;
   p.scale_log2 = scale * 1.4426950408889634f;
   if (cudaFuncSetAttribute(dsa_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) != cudaSuccess)
     return HCADSA_ERR_CUDA;
-  dsa_attn_kernel<<<(unsigned)(B * Lq), kThreads, kSmemBytes, as_stream(stream)>>>(mq, p);
+  const int sms = num_sms_current_device();
+  if (sms <= 0) return HCADSA_ERR_CUDA;
+  const int grid = p.n_tok < sms ? p.n_tok : sms;
+  dsa_attn_kernel<<<grid, kThreads, kSmemBytes, as_stream(stream)>>>(mq, p);
   return launch_status();
 }

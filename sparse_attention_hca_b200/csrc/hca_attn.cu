@@ -288,8 +288,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       float mx = -INFINITY;
       for (int c0 = 0; c0 < kt.n; c0 += 32) {
         uint32_t v[32];
-        tmem_ld32(tS + c0, v);
-        tmem_wait_ld();
+        tmem_ld32_nowait(tS + c0, v);
+        tmem_wait_ld_regs(v);
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
           const int col = c0 + i;
@@ -313,8 +313,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         l_run *= alpha;
         for (int oc = 0; oc < kDHalf; oc += 32) {
           uint32_t v[32];
-          tmem_ld32(tmem + lane_off + oc, v);
-          tmem_wait_ld();
+          tmem_ld32_nowait(tmem + lane_off + oc, v);
+          tmem_wait_ld_regs(v);
 #pragma unroll
           for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * alpha);
           tmem_st32(tmem + lane_off + oc, v);
@@ -325,8 +325,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool any_visible = m_ref != -INFINITY;
       for (int c0 = 0; c0 < kt.n; c0 += 32) {
         uint32_t v[32];
-        tmem_ld32(tS + c0, v);
-        tmem_wait_ld();
+        tmem_ld32_nowait(tS + c0, v);
+        tmem_wait_ld_regs(v);
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
@@ -352,8 +352,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint16_t* orow = p.O + ((size_t)((size_t)b * p.Lq + tok) * p.Hq + h) * kD + half * kDHalf;
       for (int oc = 0; oc < kDHalf; oc += 32) {
         uint32_t v[32];
-        tmem_ld32(tmem + lane_off + oc, v);
-        tmem_wait_ld();
+        tmem_ld32_nowait(tmem + lane_off + oc, v);
+        tmem_wait_ld_regs(v);
         if (row_valid) {
           uint4 packed[4];
           uint32_t* pw = reinterpret_cast<uint32_t*>(packed);

@@ -24,8 +24,14 @@ inline cudaStream_t as_stream(hcadsa_stream s) { return reinterpret_cast<cudaStr
 bool encode_tmap_bf16(CUtensorMap* map, int rank, void* base, const uint64_t* dims,
                       const uint64_t* strides_bytes, const uint32_t* box, bool swizzle128);
 
+// Records the message of a failed CUDA call for hcadsa_last_error_string().
+void record_cuda_error(cudaError_t e);
+
 inline hcadsa_status launch_status() {
-  return cudaGetLastError() == cudaSuccess ? HCADSA_OK : HCADSA_ERR_CUDA;
+  const cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) return HCADSA_OK;
+  record_cuda_error(e);
+  return HCADSA_ERR_CUDA;
 }
 
 }  // namespace hcadsa
