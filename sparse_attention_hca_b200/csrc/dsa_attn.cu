@@ -13,7 +13,7 @@
 //       O^T[dv, head]  += V_g^T (A, MN-major, 2 x 128 dv) * P^T (B, MN-major, 64 heads)
 //     TMEM: O^T double-buffered per token [0,128) / [128,256) so one token's epilogue
 //     overlaps the next token's MMAs; S^T double-buffered per tile [256,320) / [320,384).
-//   * Warps 0-2 gather K and V rows with cp.async: one warp instruction moves one whole
+//   * Warps 0-5 gather K and V rows with cp.async: one warp instruction moves one whole
 //     512-byte row (lane l -> 16 bytes of 64-column chunk l/8), written 128B-swizzled into a
 //     ring of 8 x 16 KB chunk slots; a tile's K (or V) occupies 4 consecutive slots, loaded in
 //     exactly the order warp 4 consumes them: K_0, K_1, V_0, K_2, V_1, ...  Completion is
@@ -21,13 +21,16 @@
 //     each wait so the tensor core sees the generic-proxy writes.  (Measured on B200: this
 //     reaches ~105 GB/s per SM from L2, TMA tile::gather4 of 4 x 128 B rows ~16 GB/s.)
 //     Q (32 KB, TMA) is reloaded per token once the previous token's last S^T MMA is done.
-//   * Warp 3, lane 0 issues every MMA.  Warps 4-7: softmax (one thread per key = TMEM lane,
-//     64 head scores each).  The first tile of a token sets the per-head reference max by a
+//   * Warp 6, lane 0 issues every MMA.  Warps 7-10: softmax (one thread per key = TMEM lane,
+//     64 head scores each; per-head row sums reduced across the warp every tile).  The first tile of a token sets the per-head reference max by a
 //     warp reduce-scatter + 4-warp combine; later tiles only check their scores against it and
 //     redo the reduction (and rescale O^T) when some score exceeds it by 2^8.  P^T rows go to
 //     shared memory; then the token's epilogue (normalise O^T, store O).
 //   * Index rows may hold padding (< 0) anywhere; a 128-entry tile without any valid entry
-//     is skipped, other invalid entries read row 0 and are masked.
+//     is skipped, other invalid entries read row 0 and are masked.  Index rows are staged in
+//     shared memory (double buffer): the softmax warps prefetch token i+2's row with cp.async
+//     as soon as the producer and MMA warps have released the buffer token i used, so no
+//     role waits on the index tensor in HBM.
 //   * Barrier phases continue across tokens: s_full/p_ready/pv_done are indexed by a global
 //     tile counter, q_full/q_empty/o_full/o_empty by a counter of tokens with work.
 #include <cuda_bf16.h>
@@ -44,18 +47,20 @@ constexpr int kD = 256;
 constexpr int kH = 64;
 constexpr int kKeyTile = 128;
 constexpr int kChunkBytes = 128 * 128;     // 128 rows x 64 bf16
-constexpr int kRingSlots = 8;
+constexpr int kRingSlots = 8;  // even: a V pair (2hv, 2hv+1) never wraps
 constexpr int kQChunkBytes = kH * 128;     // 64 heads x 64 bf16
 constexpr int kQBytes = 4 * kQChunkBytes;  // 32 KB
 constexpr int kPBytes = kKeyTile * 128;    // 128 keys x 64 heads bf16
 constexpr int kMaxK = 4096;                // 32 tiles: one bit per tile in a 32-bit mask
-constexpr int kSmemBytes = kQBytes + kRingSlots * kChunkBytes + 2 * kPBytes + 1024;
-// 8 warps = 2 per SM sub-partition, so each thread may use up to 255 registers (each
-// sub-partition has a 16K-entry register file; a third warp there would cap it near 168).
-constexpr int kProducerWarps = 3;
-constexpr int kMmaWarp = 3;
-constexpr int kSoftmaxWarp0 = 4;
-constexpr int kThreads = 32 * 8;
+constexpr int kIdxBytes = kMaxK * 4;  // one index row
+constexpr int kSmemBytes = kQBytes + kRingSlots * kChunkBytes + 2 * kPBytes + 2 * kIdxBytes + 1024;
+// Gather throughput scales with the number of producer warps.  11 warps put 3 on some SM
+// sub-partitions (16K-entry register file each), which caps a thread at 168 registers; the
+// softmax keeps its per-head row sums reduced across the warp (2 per lane) to fit.
+constexpr int kProducerWarps = 6;
+constexpr int kMmaWarp = kProducerWarps;
+constexpr int kSoftmaxWarp0 = kProducerWarps + 1;
+constexpr int kThreads = 32 * (kProducerWarps + 1 + 4);
 constexpr uint32_t kTmemS = 256;  // S^T buffers at columns 256 and 320
 constexpr float kLazyRescale = 8.0f;
 
@@ -79,6 +84,8 @@ struct __align__(8) Barriers {
   uint64_t pv_done;
   uint64_t o_full[2];
   uint64_t o_empty[2];
+  uint64_t idx_full[2];   // index row of a token landed (128 softmax-thread cp.async arrivals)
+  uint64_t idx_empty[2];  // producers (3 warps) and MMA warp are done with the row
 };
 
 struct SoftShared {
@@ -98,24 +105,25 @@ __device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
 }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
-// Bit j set iff tile j (entries [128j, 128j+128) of the row) holds a valid entry.  Whole warp.
+// Bit j set iff tile j (entries [128j, 128j+128) of the row) holds a valid entry.  Whole warp;
+// `row` is the shared-memory copy of the index row.
 __device__ __forceinline__ uint32_t tile_mask_of_row(const int32_t* row, int k, int Lk, int lane) {
   uint32_t mask = 0;
   const int n_tiles = (k + kKeyTile - 1) / kKeyTile;
-  const bool vec = (k & 3) == 0;  // rows start 16-byte aligned
   for (int j = 0; j < n_tiles; ++j) {
-    const int e = j * kKeyTile + lane * 4;
     bool any = false;
-    if (vec && e + 3 < k) {
-      const int4 v = *reinterpret_cast<const int4*>(row + e);
-      any = idx_ok(v.x, Lk) | idx_ok(v.y, Lk) | idx_ok(v.z, Lk) | idx_ok(v.w, Lk);
-    } else {
-      for (int q = 0; q < 4; ++q)
-        if (e + q < k) any |= idx_ok(row[e + q], Lk);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int e = j * kKeyTile + lane * 4 + q;
+      if (e < k) any |= idx_ok(row[e], Lk);
     }
     if (__any_sync(0xffffffffu, any)) mask |= 1u << j;
   }
   return mask;
+}
+
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
 }
 
 // Warp reduce-scatter of 64 per-lane values: afterwards lane l holds, in v[0] and v[1],
@@ -156,6 +164,16 @@ __device__ __forceinline__ bool softmax_bar_or(bool pred) {
   return r != 0;
 }
 
+// Softmax threads: once the producers and the MMA warp released buffer `buf` (used by local
+// token i), fetch the index row of token `next` into it with cp.async.
+__device__ __forceinline__ void refill_idx_row(const Params& p, Barriers& bar, uint32_t sIdx_a, int buf, int i,
+                                               int next, int tid, volatile int& abort_flag, bool& ok) {
+  if (next >= p.n_tok) return;
+  ok = mbar_wait(&bar.idx_empty[buf], (i >> 1) & 1, &abort_flag, p.err) && ok;
+  for (int e = tid; e < p.k; e += 128) cp_async4(sIdx_a + (buf * kMaxK + e) * 4, p.idx + (size_t)next * p.k + e);
+  cp_async_arrive_noinc(&bar.idx_full[buf]);
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
     dsa_attn_kernel(const __grid_constant__ CUtensorMap map_q, const Params p) {
   extern __shared__ uint8_t smem_raw[];
@@ -163,6 +181,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sQ = smem;
   uint8_t* sRing = smem + kQBytes;
   uint8_t* sP = sRing + kRingSlots * kChunkBytes;
+  int32_t* sIdx = reinterpret_cast<int32_t*>(sP + 2 * kPBytes);  // [2][kMaxK]
   __shared__ Barriers bar;
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_flag;
@@ -183,6 +202,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bar.o_empty[s], 128);
     }
     mbar_init(&bar.pv_done, 1);
+    for (int s2 = 0; s2 < 2; ++s2) {
+      mbar_init(&bar.idx_full[s2], 128);
+      mbar_init(&bar.idx_empty[s2], kProducerWarps + 1);
+    }
     abort_flag = 0;
     fence_mbarrier_init();
   }
@@ -201,15 +224,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t ring = smem_u32(sRing);
     const uint16_t* Kg = p.K;
     const uint16_t* Vg = p.V;
-    int slot = 0;  // always 0 or 4: a tile half takes 4 consecutive slots of the 8
-    uint32_t phase = 0;
+    uint32_t q = 0;  // chunks issued so far: slot q % kRingSlots, phase (q / kRingSlots) & 1
     int it = 0;  // tokens with work so far
     bool ok = true;
     const int chunk = lane >> 3, piece = lane & 7;
-    for (int tok = blockIdx.x; tok < p.n_tok && ok; tok += gridDim.x) {
-      const int32_t* row = p.idx + (size_t)tok * k;
+    int i = 0;   // tokens of this CTA so far (index-row buffer i & 1)
+    for (int tok = blockIdx.x; tok < p.n_tok && ok; tok += gridDim.x, ++i) {
+      const int buf = i & 1;
+      ok = __all_sync(0xffffffffu, mbar_wait(&bar.idx_full[buf], (i >> 1) & 1, &abort_flag, p.err));
+      if (!ok) break;
+      const int32_t* row = sIdx + buf * kMaxK;
       const uint32_t mask = tile_mask_of_row(row, k, Lk, lane);
-      if (!mask) continue;
+      if (!mask) {
+        if (lane == 0) mbar_arrive(&bar.idx_empty[buf]);
+        continue;
+      }
       const int J = __popc(mask);
       const size_t kv_row0 = (size_t)(tok / p.Lq) * Lk;  // first K/V row of this token's batch
       // warp w gathers tile rows w, w+3, w+6, ...: lane l holds the K/V row of the warp's
@@ -233,11 +262,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (is_k ? step >= J : step < 1) continue;
           const int ra = is_k ? ra_cur : ra_prev, rb = is_k ? rb_cur : rb_prev;
           const uint16_t* base = (is_k ? Kg : Vg) + kv_row0 * kD + lane * 8;
-          for (int c = 0; c < 4 && ok; ++c)
-            ok = mbar_wait(&bar.empty[slot + c], phase ^ 1, &abort_flag, p.err);
+          for (int c = 0; c < 4 && ok; ++c) {
+            const uint32_t qc = q + c;
+            ok = mbar_wait(&bar.empty[qc % kRingSlots], ((qc / kRingSlots) & 1) ^ 1, &abort_flag, p.err);
+          }
           ok = __all_sync(0xffffffffu, ok);
           if (!ok) break;
-          const uint32_t dst0 = ring + (slot + chunk) * kChunkBytes;
+          const uint32_t dst0 = ring + ((q + chunk) % kRingSlots) * kChunkBytes;
 #pragma unroll 4
           for (int i = 0; i < n_rows_w; ++i) {
             const int trow = warp + kProducerWarps * i;  // row of the tile
@@ -245,9 +276,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             cp_async16(dst0 + trow * 128 + ((piece ^ (trow & 7)) << 4), base + (size_t)src_row * kD);
           }
 #pragma unroll
-          for (int c = 0; c < 4; ++c) cp_async_arrive_noinc(&bar.full[slot + c]);
-          slot += 4;
-          if (slot == kRingSlots) { slot = 0; phase ^= 1; }
+          for (int c = 0; c < 4; ++c) cp_async_arrive_noinc(&bar.full[(q + c) % kRingSlots]);
+          q += 4;
           if (is_k && step == 0 && warp == 0) {
             // Q of this token (after its first K tile is in flight), once the previous token's
             // last S^T MMA no longer reads the buffer
@@ -261,22 +291,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         ra_prev = ra_cur;
         rb_prev = rb_cur;
       }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar.idx_empty[buf]);  // this warp read its last row index
       ++it;
     }
     cp_async_wait_all();
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
-    int slot = 0;
-    uint32_t phase = 0;
+    uint32_t q = 0;  // chunks consumed so far (same sequence as the producers)
     int it = 0;
     uint32_t g = 0;  // global tile counter
     bool ok = true;
     const uint32_t sQa = smem_u32(sQ), sRa = smem_u32(sRing), sPa = smem_u32(sP);
     const uint32_t idesc_s = idesc_bf16_f32(128, kH, false, false);
     const uint32_t idesc_o = idesc_bf16_f32(128, kH, true, true);
-    for (int tok = blockIdx.x; tok < p.n_tok && ok; tok += gridDim.x) {
-      const int32_t* row = p.idx + (size_t)tok * k;
-      const uint32_t mask = tile_mask_of_row(row, k, Lk, lane);
+    int i = 0;
+    for (int tok = blockIdx.x; tok < p.n_tok && ok; tok += gridDim.x, ++i) {
+      const int buf = i & 1;
+      ok = __all_sync(0xffffffffu, mbar_wait(&bar.idx_full[buf], (i >> 1) & 1, &abort_flag, p.err));
+      if (!ok) break;
+      const uint32_t mask = tile_mask_of_row(sIdx + buf * kMaxK, k, Lk, lane);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar.idx_empty[buf]);  // only the mask was needed
       if (!mask) continue;
       const int J = __popc(mask);
       const int ob = it & 1;
@@ -288,7 +324,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t gs = g + step;
             const uint32_t tS = tmem + kTmemS + (gs & 1) * kH;
             for (int c = 0; c < 4 && ok; ++c) {
-              ok = mbar_wait(&bar.full[slot], phase, &abort_flag, p.err);
+              const uint32_t slot = q % kRingSlots;
+              ok = mbar_wait(&bar.full[slot], (q / kRingSlots) & 1, &abort_flag, p.err);
               if (!ok) break;
               fence_proxy_async_smem();  // cp.async (generic proxy) writes -> tensor core reads
               tc_fence_after();
@@ -299,7 +336,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mma_ss(tS, da, db, idesc_s, (c | kk) != 0);
               }
               mma_commit(&bar.empty[slot]);
-              if (++slot == kRingSlots) { slot = 0; phase ^= 1; }
+              ++q;
             }
             if (!ok) break;
             mma_commit(&bar.s_full[gs & 1]);
@@ -317,7 +354,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_after();
             const uint32_t pbase = sPa + (gj & 1) * kPBytes;
             for (int hv = 0; hv < 2 && ok; ++hv) {
-              // V chunks 2hv, 2hv+1 sit in consecutive slots (slot is even here)
+              // V chunks 2hv, 2hv+1 sit in consecutive slots (q is even here and the ring size is
+              // even, so the pair never wraps)
+              const uint32_t slot = q % kRingSlots;
+              const uint32_t phase = (q / kRingSlots) & 1;
               ok = mbar_wait(&bar.full[slot], phase, &abort_flag, p.err) &&
                    mbar_wait(&bar.full[slot + 1], phase, &abort_flag, p.err);
               if (!ok) break;
@@ -330,8 +370,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
               mma_commit(&bar.empty[slot]);
               mma_commit(&bar.empty[slot + 1]);
-              slot += 2;
-              if (slot == kRingSlots) { slot = 0; phase ^= 1; }
+              q += 2;
             }
             if (!ok) break;
             mma_commit(&bar.pv_done);
@@ -340,8 +379,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       ok = __shfl_sync(0xffffffffu, ok, 0);
-      slot = __shfl_sync(0xffffffffu, slot, 0);
-      phase = __shfl_sync(0xffffffffu, phase, 0);
+      q = __shfl_sync(0xffffffffu, q, 0);
       g += J;
       ++it;
     }
@@ -357,21 +395,33 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     // No early exit in this loop: the four softmax warps meet at named barriers, so after an
     // abort every thread keeps walking the same barrier sequence (waits then fail fast).
-    for (int tok = blockIdx.x; tok < p.n_tok; tok += gridDim.x) {
-      const int32_t* row = p.idx + (size_t)tok * k;
+    const uint32_t sIdx_a = smem_u32(sIdx);
+    // index rows of this CTA's first two tokens
+    for (int i0 = 0; i0 < 2; ++i0) {
+      const int t0 = blockIdx.x + i0 * gridDim.x;
+      if (t0 < p.n_tok) {
+        for (int e = tid; e < k; e += 128) cp_async4(sIdx_a + (i0 * kMaxK + e) * 4, p.idx + (size_t)t0 * k + e);
+        cp_async_arrive_noinc(&bar.idx_full[i0]);
+      }
+    }
+    int i = 0;
+    for (int tok = blockIdx.x; tok < p.n_tok; tok += gridDim.x, ++i) {
+      const int buf = i & 1;
+      ok = mbar_wait(&bar.idx_full[buf], (i >> 1) & 1, &abort_flag, p.err) && ok;
+      const int32_t* row = sIdx + buf * kMaxK;
       const uint32_t mask = tile_mask_of_row(row, k, Lk, lane);
       uint16_t* obase = p.O + (size_t)tok * kH * kD;
       if (!mask) {  // no valid entry: O = 0, lse = -inf
         for (int e = tid; e < kH * kD / 8; e += 128) reinterpret_cast<uint4*>(obase)[e] = make_uint4(0, 0, 0, 0);
         if (p.lse && tid < kH) p.lse[(size_t)tok * kH + tid] = -INFINITY;
+        softmax_bar();  // every softmax thread has read the row before it is refilled
+        refill_idx_row(p, bar, sIdx_a, buf, i, tok + 2 * gridDim.x, tid, abort_flag, ok);
         continue;
       }
       const int J = __popc(mask);
       const int ob = it & 1;
       if (tid < kH) ss.m_ref[tid] = -INFINITY;
-      float lpart[kH];
-#pragma unroll
-      for (int h = 0; h < kH; ++h) lpart[h] = 0.0f;
+      float lsum0 = 0.0f, lsum1 = 0.0f;  // row sums of heads 2*lane, 2*lane+1 over this warp's keys
       uint32_t m = mask;
       for (int jj = 0; jj < J; ++jj) {
         const int j = __ffs(m) - 1;
@@ -384,39 +434,61 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = mbar_wait(&bar.s_full[gs & 1], (gs >> 1) & 1, &abort_flag, p.err) && ok;
         tc_fence_after();
         const uint32_t tS = tmem + lane_off + kTmemS + (gs & 1) * kH;
-        // Does any score of this tile exceed its head's reference max by more than 2^8?  The
-        // first tile of a token always runs the reduction (its reference is still -inf).
+        uint8_t* prow = sP + (gs & 1) * kPBytes + kl * 128;
+        uint32_t u0[32], u1[32];  // scores, then p (fp32 bits)
+        tmem_ld32_nowait(tS, u0);
+        tmem_ld32_nowait(tS + 32, u1);
+        tmem_wait_ld_regs2(u0, u1);
+        // Speculative pass: P against the current per-head reference max, and whether any score
+        // exceeds it by more than 2^8 (then the tile is redone after a reduction).  The first
+        // tile of a token always takes the reduction path (its reference is still -inf).
         bool over = jj == 0;
         if (!over) {
-          uint32_t u0[32], u1[32];
-          tmem_ld32_nowait(tS, u0);
-          tmem_ld32_nowait(tS + 32, u1);
-          tmem_wait_ld_regs2(u0, u1);
-          if (valid) {
 #pragma unroll
-            for (int c8 = 0; c8 < 16; ++c8) {
-              const float4 mr = *reinterpret_cast<const float4*>(&ss.m_ref[c8 * 4]);
-              const float r4[4] = {mr.x, mr.y, mr.z, mr.w};
+          for (int c8 = 0; c8 < 8; ++c8) {
+            const float4 ma = *reinterpret_cast<const float4*>(&ss.m_ref[c8 * 8]);
+            const float4 mb = *reinterpret_cast<const float4*>(&ss.m_ref[c8 * 8 + 4]);
+            const float mr[8] = {ma.x, ma.y, ma.z, ma.w, mb.x, mb.y, mb.z, mb.w};
+            uint32_t w4[4];
 #pragma unroll
-              for (int q = 0; q < 4; ++q) {
-                const int h = c8 * 4 + q;
-                const float sc = __uint_as_float(h < 32 ? u0[h] : u1[h - 32]) * p.scale_log2;
-                over |= sc > r4[q] + kLazyRescale;
-              }
+            for (int qq = 0; qq < 4; ++qq) {
+              const int h = c8 * 8 + 2 * qq;
+              uint32_t& r0 = h < 32 ? u0[h] : u1[h - 32];
+              uint32_t& r1 = h + 1 < 32 ? u0[h + 1] : u1[h + 1 - 32];
+              const float x0 = fmaf(__uint_as_float(r0), p.scale_log2, -mr[2 * qq]);
+              const float x1 = fmaf(__uint_as_float(r1), p.scale_log2, -mr[2 * qq + 1]);
+              over |= valid && (x0 > kLazyRescale || x1 > kLazyRescale);
+              const float p0 = valid ? fast_exp2(x0) : 0.0f;
+              const float p1 = valid ? fast_exp2(x1) : 0.0f;
+              r0 = __float_as_uint(p0);
+              r1 = __float_as_uint(p1);
+              w4[qq] = pack_bf16x2(p0, p1);
             }
+            *reinterpret_cast<uint4*>(prow + ((c8 ^ (kl & 7)) << 4)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
           }
         }
-        if (softmax_bar_or(over)) {
+        if (!softmax_bar_or(over)) {
+          float pv[kH];
+#pragma unroll
+          for (int h = 0; h < 32; ++h) {
+            pv[h] = __uint_as_float(u0[h]);
+            pv[32 + h] = __uint_as_float(u1[h]);
+          }
+          warp_reduce_scatter64<false>(pv, lane);
+          lsum0 += pv[0];
+          lsum1 += pv[1];
+        } else {
+          // reduction path: new per-head reference, rescale O^T if it moved, P from scratch
           float red[kH];
           {
-            uint32_t u0[32], u1[32];
-            tmem_ld32_nowait(tS, u0);
-            tmem_ld32_nowait(tS + 32, u1);
-            tmem_wait_ld_regs2(u0, u1);
+            uint32_t t0[32], t1[32];
+            tmem_ld32_nowait(tS, t0);
+            tmem_ld32_nowait(tS + 32, t1);
+            tmem_wait_ld_regs2(t0, t1);
 #pragma unroll
             for (int h = 0; h < 32; ++h) {
-              red[h] = valid ? __uint_as_float(u0[h]) * p.scale_log2 : -INFINITY;
-              red[32 + h] = valid ? __uint_as_float(u1[h]) * p.scale_log2 : -INFINITY;
+              red[h] = valid ? __uint_as_float(t0[h]) * p.scale_log2 : -INFINITY;
+              red[32 + h] = valid ? __uint_as_float(t1[h]) * p.scale_log2 : -INFINITY;
             }
           }
           warp_reduce_scatter64<true>(red, lane);
@@ -456,14 +528,9 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
             }
             tmem_wait_st();
-#pragma unroll
-            for (int h = 0; h < kH; ++h) lpart[h] *= ss.alpha[h];
+            lsum0 *= ss.alpha[2 * lane];
+            lsum1 *= ss.alpha[2 * lane + 1];
           }
-        }
-        // P^T row of this key: 64 heads, bf16, 128B-swizzled (scores re-read from TMEM)
-        uint8_t* prow = sP + (gs & 1) * kPBytes + kl * 128;
-        {
-          uint32_t u0[32], u1[32];
           tmem_ld32_nowait(tS, u0);
           tmem_ld32_nowait(tS + 32, u1);
           tmem_wait_ld_regs2(u0, u1);
@@ -474,30 +541,38 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float mr[8] = {ma.x, ma.y, ma.z, ma.w, mb.x, mb.y, mb.z, mb.w};
             uint32_t w4[4];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const int h = c8 * 8 + 2 * q;
+            for (int qq = 0; qq < 4; ++qq) {
+              const int h = c8 * 8 + 2 * qq;
               const uint32_t s0 = h < 32 ? u0[h] : u1[h - 32];
               const uint32_t s1 = h + 1 < 32 ? u0[h + 1] : u1[h + 1 - 32];
               float p0 = 0.0f, p1 = 0.0f;
               if (valid) {
-                p0 = fast_exp2(fmaf(__uint_as_float(s0), p.scale_log2, -mr[2 * q]));
-                p1 = fast_exp2(fmaf(__uint_as_float(s1), p.scale_log2, -mr[2 * q + 1]));
+                p0 = fast_exp2(fmaf(__uint_as_float(s0), p.scale_log2, -mr[2 * qq]));
+                p1 = fast_exp2(fmaf(__uint_as_float(s1), p.scale_log2, -mr[2 * qq + 1]));
               }
-              lpart[h] += p0;
-              lpart[h + 1] += p1;
-              w4[q] = pack_bf16x2(p0, p1);
+              (h < 32 ? u0[h] : u1[h - 32]) = __float_as_uint(p0);
+              (h + 1 < 32 ? u0[h + 1] : u1[h + 1 - 32]) = __float_as_uint(p1);
+              w4[qq] = pack_bf16x2(p0, p1);
             }
             *reinterpret_cast<uint4*>(prow + ((c8 ^ (kl & 7)) << 4)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
           }
+          float pv[kH];
+#pragma unroll
+          for (int h = 0; h < 32; ++h) {
+            pv[h] = __uint_as_float(u0[h]);
+            pv[32 + h] = __uint_as_float(u1[h]);
+          }
+          warp_reduce_scatter64<false>(pv, lane);
+          lsum0 += pv[0];
+          lsum1 += pv[1];
         }
         fence_proxy_async_smem();
         tc_fence_before();
         mbar_arrive(&bar.p_ready[gs & 1]);
       }
       // ---- epilogue of this token
-      warp_reduce_scatter64<false>(lpart, lane);
-      ss.wred[sw][2 * lane] = lpart[0];
-      ss.wred[sw][2 * lane + 1] = lpart[1];
+      ss.wred[sw][2 * lane] = lsum0;
+      ss.wred[sw][2 * lane + 1] = lsum1;
       softmax_bar();
       if (tid < kH) {  // per-head row sum -> 1/l (kept in ss.alpha) and log-sum-exp
         const float l = ss.wred[0][tid] + ss.wred[1][tid] + ss.wred[2][tid] + ss.wred[3][tid];
@@ -531,7 +606,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_before();
       mbar_arrive(&bar.o_empty[ob]);
-      softmax_bar();  // wred / m_ref are rewritten by the next token
+      softmax_bar();  // wred / m_ref are rewritten by the next token; the row has been read
+      refill_idx_row(p, bar, sIdx_a, buf, i, tok + 2 * gridDim.x, tid, abort_flag, ok);
       g += J;
       ++it;
     }
