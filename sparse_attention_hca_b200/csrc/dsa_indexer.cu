@@ -220,62 +220,94 @@ __global__ void __launch_bounds__(kStreamThreads) score_stream_kernel(const int8
 }
 
 // ------------------------------------------------------------------ selection
+//
+// One thread block per query row.  The row is staged in shared memory (when it fits) with
+// coalesced 16-byte loads; then thread t owns the contiguous segment [t*E, t*E + E) of it,
+// E odd so the 32 lanes of a warp read 32 different banks.  Radix select on u = score - min:
+// 8-bit digits from the top, each counted into a per-warp histogram (contention only within a
+// warp), summed, and the bin holding the k-th largest found by one warp.  The compaction then
+// needs a single block scan of packed (count > threshold, count == threshold) pairs: a thread's
+// output position is (greater elements before it) + min(equal elements before it, equal
+// elements to take), so ties go to the lowest positions and the output is ascending.
 constexpr int kSelThreads = 512;
-constexpr int kSelItems = 4;                 // consecutive elements per thread per chunk
-constexpr int kSelChunk = kSelThreads * kSelItems;
-constexpr int kRadixBits = 11;
-constexpr int kRadixBins = 1 << kRadixBits;  // 2048
-constexpr int kSelSmemCap = 40960;           // row entries staged in shared memory (160 KB)
+constexpr int kSelWarps = kSelThreads / 32;
+constexpr int kDigitBits = 8;
+constexpr int kDigitBins = 1 << kDigitBits;
+constexpr int kSelSmemCap = 40960;  // row entries staged in shared memory (160 KB)
 
 struct SelShared {
-  unsigned int hist[kRadixBins];
-  int warp_tot[kSelThreads / 32];
-  int warp_tot2[kSelThreads / 32];
+  unsigned int hist[kSelWarps][kDigitBins];
+  unsigned long long scan_warp[kSelWarps];
+  int red_a[kSelWarps], red_b[kSelWarps];
   int bcast[4];
 };
 
-// Block-wide exclusive prefix sum of one int per thread; returns the exclusive prefix
+// Block-wide exclusive prefix sum of a 64-bit value per thread; returns the exclusive prefix
 // and writes the block total to *total.
-__device__ __forceinline__ int block_exclusive_scan(int v, int* warp_tot, int* total) {
+__device__ __forceinline__ unsigned long long block_exclusive_scan64(unsigned long long v, SelShared& sh,
+                                                                     unsigned long long* total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  int x = v;
+  unsigned long long x = v;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    const unsigned long long y = __shfl_up_sync(0xffffffffu, x, o);
     if (lane >= o) x += y;
   }
-  if (lane == 31) warp_tot[warp] = x;
+  if (lane == 31) sh.scan_warp[warp] = x;
   __syncthreads();
   if (warp == 0) {
-    int t = lane < kSelThreads / 32 ? warp_tot[lane] : 0;
+    unsigned long long t = lane < kSelWarps ? sh.scan_warp[lane] : 0ull;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, t, o);
+      const unsigned long long y = __shfl_up_sync(0xffffffffu, t, o);
       if (lane >= o) t += y;
     }
-    if (lane < kSelThreads / 32) warp_tot[lane] = t;  // inclusive
+    if (lane < kSelWarps) sh.scan_warp[lane] = t;  // inclusive
   }
   __syncthreads();
-  const int warp_excl = warp == 0 ? 0 : warp_tot[warp - 1];
-  *total = warp_tot[kSelThreads / 32 - 1];
-  __syncthreads();
-  return warp_excl + x - v;
+  const unsigned long long before = warp == 0 ? 0ull : sh.scan_warp[warp - 1];
+  *total = sh.scan_warp[kSelWarps - 1];
+  return before + x - v;
 }
 
-template <bool kInSmem>
-__device__ __forceinline__ int load_score(const int* row_smem, const int* row_gmem, int i) {
-  return kInSmem ? row_smem[i] : __ldcg(row_gmem + i);
+// Stages row_g[c0, c0 + len) into row_s[0, len) with coalesced 16-byte loads (c0 % 4 == 0).
+__device__ __forceinline__ void stage_chunk(const int* __restrict__ row_g, int* row_s, int c0, int len) {
+  const int tid = threadIdx.x;
+  const int n4 = len >> 2;
+  const int4* src4 = reinterpret_cast<const int4*>(row_g + c0);  // 16-byte aligned: c0 % 4 == 0
+  constexpr int kUnroll = 8;
+  for (int base = tid; base < n4; base += kSelThreads * kUnroll) {
+    int4 v[kUnroll];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const int i4 = base + u * kSelThreads;
+      v[u] = i4 < n4 ? __ldcg(src4 + i4) : make_int4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const int i4 = base + u * kSelThreads;
+      if (i4 < n4) reinterpret_cast<int4*>(row_s)[i4] = v[u];
+    }
+  }
+  for (int i = (n4 << 2) + tid; i < len; i += kSelThreads) row_s[i] = __ldcg(row_g + c0 + i);
 }
 
+// kInSmem: the whole row is staged in row_s; otherwise the passes read global memory (strided,
+// coalesced) and the ordered compaction walks the row in chunks staged through row_s.
 template <bool kInSmem>
 __device__ void select_row(const int* __restrict__ row_g, int* row_s, int n, int k, int32_t* __restrict__ out,
                            SelShared& sh) {
-  const int tid = threadIdx.x;
-  // ---- stage + min/max
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (kInSmem) {
+    stage_chunk(row_g, row_s, 0, n);
+    __syncthreads();
+  }
+  auto at = [&](int i) { return kInSmem ? row_s[i] : __ldcg(row_g + i); };
+
+  // ---- min / max (strided: coalesced in global memory, conflict-free in shared memory)
   int mn = INT_MAX, mx = INT_MIN;
   for (int i = tid; i < n; i += kSelThreads) {
-    const int v = __ldcg(row_g + i);
-    if (kInSmem) row_s[i] = v;
+    const int v = at(i);
     mn = min(mn, v);
     mx = max(mx, v);
   }
@@ -284,60 +316,73 @@ __device__ void select_row(const int* __restrict__ row_g, int* row_s, int n, int
     mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, o));
     mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
   }
-  if ((tid & 31) == 0) {
-    sh.warp_tot[tid >> 5] = mn;
-    sh.warp_tot2[tid >> 5] = mx;
+  if (lane == 0) {
+    sh.red_a[warp] = mn;
+    sh.red_b[warp] = mx;
   }
   __syncthreads();
-  if (tid == 0) {
-    int a = INT_MAX, c = INT_MIN;
-    for (int i = 0; i < kSelThreads / 32; ++i) {
-      a = min(a, sh.warp_tot[i]);
-      c = max(c, sh.warp_tot2[i]);
+  if (warp == 0) {
+    int a = lane < kSelWarps ? sh.red_a[lane] : INT_MAX, c = lane < kSelWarps ? sh.red_b[lane] : INT_MIN;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      a = min(a, __shfl_xor_sync(0xffffffffu, a, o));
+      c = max(c, __shfl_xor_sync(0xffffffffu, c, o));
     }
-    sh.bcast[0] = a;
-    sh.bcast[1] = c;
+    if (lane == 0) {
+      sh.bcast[0] = a;
+      sh.bcast[1] = c;
+    }
   }
   __syncthreads();
   const int vmin = sh.bcast[0];
   const unsigned range = (unsigned)sh.bcast[1] - (unsigned)vmin;
-  __syncthreads();
 
   // ---- radix select on u = score - vmin (unsigned, order preserving)
   int nbits = range == 0 ? 0 : 32 - __clz((int)range);
   unsigned prefix = 0, pmask = 0;
-  int remaining = k;  // rank (1-based from the top) still to locate among prefix matches
+  int remaining = k;  // rank (1 = largest) still to locate among the prefix matches
   while (nbits > 0) {
-    const int dbits = nbits < kRadixBits ? nbits : kRadixBits;
+    const int dbits = nbits < kDigitBits ? nbits : kDigitBits;
     const int lo = nbits - dbits;
     const unsigned dmask = (1u << dbits) - 1u;
-    for (int i = tid; i < (1 << dbits); i += kSelThreads) sh.hist[i] = 0;
-    __syncthreads();
+    unsigned int* hw = sh.hist[warp];
+    for (int b = lane; b < kDigitBins; b += 32) hw[b] = 0;
+    __syncwarp();
     for (int i = tid; i < n; i += kSelThreads) {
-      const unsigned u = (unsigned)load_score<kInSmem>(row_s, row_g, i) - (unsigned)vmin;
-      if ((u & pmask) == prefix) atomicAdd(&sh.hist[(u >> lo) & dmask], 1u);
+      const unsigned u = (unsigned)at(i) - (unsigned)vmin;
+      if ((u & pmask) == prefix) atomicAdd(&hw[(u >> lo) & dmask], 1u);
     }
     __syncthreads();
-    // find the bin holding the remaining-th largest: scan bins from the top
-    const int nb = 1 << dbits;
-    const int per = (nb + kSelThreads - 1) / kSelThreads;  // bins per thread (<= 4)
-    const int top = nb - 1 - tid * per;                   // this thread covers bins top, top-1, ...
-    int cnt = 0;
-    for (int q = 0; q < per; ++q)
-      if (top - q >= 0) cnt += (int)sh.hist[top - q];
-    int tot;
-    const int above = block_exclusive_scan(cnt, sh.warp_tot, &tot);  // elements in higher bins
-    if (above < remaining && above + cnt >= remaining) {
-      int acc = above;
-      for (int q = 0; q < per; ++q) {
-        const int bin = top - q;
-        const int c = (int)sh.hist[bin];
-        if (acc + c >= remaining) {
-          sh.bcast[2] = bin;
-          sh.bcast[3] = remaining - acc;
-          break;
+    if (warp == 0) {
+      // lane l owns bins 255 - 8l - q, q = 0..7: counts from the top down
+      int cnt[8];
+      int lane_tot = 0;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const int bin = kDigitBins - 1 - (lane * 8 + q);
+        int c = 0;
+        for (int w = 0; w < kSelWarps; ++w) c += (int)sh.hist[w][bin];
+        cnt[q] = c;
+        lane_tot += c;
+      }
+      int incl = lane_tot;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      const int above = incl - lane_tot;  // elements in higher bins than this lane's
+      if (above < remaining && incl >= remaining) {
+        int acc = above;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          if (acc + cnt[q] >= remaining) {
+            sh.bcast[2] = kDigitBins - 1 - (lane * 8 + q);
+            sh.bcast[3] = remaining - acc;
+            break;
+          }
+          acc += cnt[q];
         }
-        acc += c;
       }
     }
     __syncthreads();
@@ -345,47 +390,49 @@ __device__ void select_row(const int* __restrict__ row_g, int* row_s, int n, int
     pmask |= dmask << lo;
     remaining = sh.bcast[3];
     nbits = lo;
-    __syncthreads();
+    __syncthreads();  // histograms are cleared again by the next pass
   }
-  const unsigned thr = prefix;   // u of the k-th largest
-  const int need_eq = remaining; // how many elements equal to thr are taken (lowest positions)
+  const unsigned thr = prefix;    // u of the k-th largest
+  const int need_eq = remaining;  // elements equal to thr that are kept (lowest positions first)
 
-  // ---- ordered compaction
-  int written = 0, eq_seen = 0;
-  for (int base = 0; base < n && written < k; base += kSelChunk) {
-    const int i0 = base + tid * kSelItems;
-    unsigned u[kSelItems];
-    int n_eq = 0;
-#pragma unroll
-    for (int q = 0; q < kSelItems; ++q) {
-      const int i = i0 + q;
-      u[q] = i < n ? (unsigned)load_score<kInSmem>(row_s, row_g, i) - (unsigned)vmin : 0u;
-      if (i < n && u[q] == thr) ++n_eq;
+  // ---- ordered compaction: per chunk, one scan of packed (greater, equal) counts; thread t owns
+  // the contiguous segment [t*E, t*E + E) of the chunk, E odd so a warp hits 32 banks
+  const int chunk = kInSmem ? n : kSelSmemCap;
+  int written_gt = 0, eq_seen = 0;
+  for (int c0 = 0; c0 < n; c0 += chunk) {
+    const int len = min(chunk, n - c0);
+    if (!kInSmem) {
+      __syncthreads();  // previous chunk fully consumed
+      stage_chunk(row_g, row_s, c0, len);
+      __syncthreads();
     }
-    int eq_tot;
-    const int eq_before = eq_seen + block_exclusive_scan(n_eq, sh.warp_tot, &eq_tot);
-    bool take[kSelItems];
-    int n_take = 0, eq_rank = eq_before;
-#pragma unroll
-    for (int q = 0; q < kSelItems; ++q) {
-      const int i = i0 + q;
-      bool t = false;
-      if (i < n) {
-        if (u[q] > thr) t = true;
-        else if (u[q] == thr) t = (eq_rank++ < need_eq);
+    const int E = ((len + kSelThreads - 1) / kSelThreads) | 1;
+    const int s0 = min(tid * E, len), s1 = min(s0 + E, len);
+    int gt = 0, eq = 0;
+    for (int i = s0; i < s1; ++i) {
+      const unsigned u = (unsigned)row_s[i] - (unsigned)vmin;
+      gt += u > thr;
+      eq += u == thr;
+    }
+    unsigned long long tot;
+    const unsigned long long before =
+        block_exclusive_scan64(((unsigned long long)gt << 32) | (unsigned)eq, sh, &tot);
+    const int gt_before = written_gt + (int)(before >> 32);
+    const int eq_before = eq_seen + (int)(before & 0xffffffffu);
+    int pos = gt_before + min(eq_before, need_eq);
+    int eq_rank = eq_before;
+    for (int i = s0; i < s1; ++i) {
+      const unsigned u = (unsigned)row_s[i] - (unsigned)vmin;
+      if (u > thr) {
+        out[pos++] = c0 + i;
+      } else if (u == thr) {
+        if (eq_rank < need_eq) out[pos++] = c0 + i;
+        ++eq_rank;
       }
-      take[q] = t;
-      n_take += t;
     }
-    int take_tot;
-    int pos = written + block_exclusive_scan(n_take, sh.warp_tot, &take_tot);
-#pragma unroll
-    for (int q = 0; q < kSelItems; ++q)
-      if (take[q] && pos < k) out[pos++] = i0 + q;
-    written += take_tot;
-    eq_seen += eq_tot;
+    written_gt += (int)(tot >> 32);
+    eq_seen += (int)(tot & 0xffffffffu);
   }
-  for (int i = written + tid; i < k; i += kSelThreads) out[i] = -1;
 }
 
 __global__ void __launch_bounds__(kSelThreads) select_kernel(const int32_t* __restrict__ scores,
@@ -405,7 +452,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const int32_t* __re
   if (n <= kSelSmemCap)
     select_row<true>(row_g, sel_row, n, k, out, sh);
   else
-    select_row<false>(row_g, nullptr, n, k, out, sh);
+    select_row<false>(row_g, sel_row, n, k, out, sh);  // sel_row stages compaction chunks
 }
 
 }  // namespace
