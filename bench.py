@@ -94,6 +94,24 @@ def profiled_traffic(summary_file, source_file):
     return float(m.group(1))
 
 
+# ----------------------------------------------------------------------------- multi-rank plumbing
+
+def max_over_ranks(x: float, dist=None, device="cpu") -> float:
+    """Max of a per-rank scalar (device time in ms) over all ranks; identity on one rank."""
+    if dist is None:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(ms_per_step_max: float, world: int, tokens_per_rank: int = None) -> float:
+    """Whole-job tokens/s: every rank runs its own sequence (weak scaling), so the job moves
+    world * tokens_per_rank tokens per step, paced by the slowest rank."""
+    tokens = L if tokens_per_rank is None else tokens_per_rank
+    return world * tokens / (ms_per_step_max * 1e-3)
+
+
 # ----------------------------------------------------------------------------- clocks
 
 class ClockSampler:
@@ -292,43 +310,45 @@ def e2e_measure(hd, x, device, steps):
     return ms, h2d, d2h
 
 
-def cpu_sample(seconds_budget=20.0, n_hca=48, n_dsa=6):
-    """Times the oracle on a bounded sample of query tokens spread over [0, L)."""
+def cpu_sample(n_hca=4096, n_dsa=1024):
+    """Times the oracle (plain C, OpenMP over query rows) on a bounded sample of the workload:
+    full compression, HCA attention for n_hca query tokens and DSA top-k + attention for
+    n_dsa query tokens, positions spread evenly over [0, L).  Each function runs once over all
+    its sampled rows, so OpenMP spreads them over the host cores.  Returns tokens/s through
+    both layers (inverse of the mean per-token cost)."""
     import numpy as np
 
     import oracle
 
     oracle.build()
-    inp_h = synth.hca_inputs(synth.HcaConfig("s", B=1, L=L, Hq=1, Hkv=1))   # K, V full; Q unused
-    rng = np.random.default_rng(1)
     bits = lambda t: t.contiguous().view(torch.int16).numpy().view(np.uint16)  # noqa: E731
-    Kh, Vh = bits(inp_h["K"]), bits(inp_h["V"])
-    w = inp_h["w"].numpy()
+    hx = synth.hca_inputs(HCA)                   # same shapes and laws as the GPU workload
+    Kh, Vh, Qh = bits(hx["K"]), bits(hx["V"]), bits(hx["Q"])
+    w = hx["w"].numpy()
     t0 = time.perf_counter()
-    Kc, Vc = oracle.hca_compress(Kh, w, 128), oracle.hca_compress(Vh, w, 128)
+    Kc, Vc = oracle.hca_compress(Kh, w, HCA.blk), oracle.hca_compress(Vh, w, HCA.blk)
     t_comp = time.perf_counter() - t0
-    toks_h = np.linspace(0, L - 1, n_hca).astype(np.int64)
-    Qh = bits(synth.normal_bf16((1, n_hca, HCA.Hq, HCA.d), 1 / math.sqrt(512), 5, "Q"))
+    rows_h = np.linspace(0, L - 1, n_hca).astype(np.int64)
     t0 = time.perf_counter()
-    for i, t in enumerate(toks_h):
-        oracle.hca_attn(Qh[:, i:i + 1], Kc, Vc, Kh, Vh, q_offset=int(t))
-    t_hca = (time.perf_counter() - t0) / n_hca
-    di = synth.dsa_inputs(synth.DsaConfig("s", B=1, L=L, Hq=1))
-    toks_d = np.linspace(0, L - 1, n_dsa).astype(np.int64)
-    Qd = bits(synth.normal_bf16((1, n_dsa, DSA.Hq, DSA.d), 1 / 16, 6, "Q"))
-    qi = di["q_idx"].numpy()
+    oracle.hca_attn(Qh, Kc, Vc, Kh, Vh, blk=HCA.blk, W=HCA.W, rows=rows_h)
+    t_hca = time.perf_counter() - t0
+    dc = synth.DsaConfig("s", B=1, L=L, Hq=1)    # indexer inputs and K/V (Q drawn per sample)
+    di = synth.dsa_inputs(dc)
+    rows_d = np.linspace(0, L - 1, n_dsa).astype(np.int64)
+    Qd = bits(synth.normal_bf16((1, n_dsa, DSA.Hq, DSA.d), 1 / math.sqrt(DSA.d), synth.SEED, "Q"))
     t0 = time.perf_counter()
-    for i, t in enumerate(toks_d):
-        idx = oracle.dsa_topk(qi[:, t:t + 1], di["k_idx"].numpy(), di["w_idx"].numpy(), DSA.k, q_offset=int(t))
-        oracle.dsa_attn(Qd[:, i:i + 1], bits(di["K"]), bits(di["V"]), idx)
-    t_dsa = (time.perf_counter() - t0) / n_dsa
-    per_token = t_comp / L + t_hca + t_dsa   # mean cost of one token through both layers
-    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+    idx = oracle.dsa_topk(di["q_idx"].numpy(), di["k_idx"].numpy(), di["w_idx"].numpy(), DSA.k, rows=rows_d)
+    oracle.dsa_attn(Qd, bits(di["K"]), bits(di["V"]), idx)
+    t_dsa = time.perf_counter() - t0
+    per_token = t_comp / L + t_hca / n_hca + t_dsa / n_dsa
+    cores = int(os.environ.get("OMP_NUM_THREADS", "0")) or (
+        len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count())
     return {
         "value": 1.0 / per_token, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-        "sample": (f"{n_hca} HCA rows and {n_dsa} DSA rows (top-k + attention) at positions spread evenly over "
-                   f"[0, {L}) plus full compression; per-token cost averaged and inverted"),
-        "sample_seconds": t_comp + t_hca * n_hca + t_dsa * n_dsa,
+        "sample": (f"full compression of the L={L} sequence; HCA attention (16 heads) for {n_hca} and DSA "
+                   f"top-{DSA.k} + attention (64 heads) for {n_dsa} query tokens spread evenly over [0, {L}); "
+                   f"tokens/s = 1 / (compress/L + HCA per row + DSA per row)"),
+        "sample_seconds": t_comp + t_hca + t_dsa,
     }
 
 
@@ -371,11 +391,7 @@ def ours(args):
         dist.barrier()
     clk = clocks.stop()
     hd.hcadsa_check_device_error()
-    ms_total = t_start.elapsed_time(t_end)
-    if dist:
-        tt = torch.tensor([ms_total], device=device)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms_total = float(tt.item())
+    ms_total = max_over_ranks(t_start.elapsed_time(t_end), dist, device)
     ms_step = ms_total / args.steps
     k_ms = [sum(e[i].elapsed_time(e[i + 1]) for e in evs) / args.steps for i in range(4)]
     comp_ms, hca_ms, idx_ms, dsa_ms = k_ms
@@ -390,11 +406,8 @@ def ours(args):
         decode = run_decode(hd, device)
         hd.hcadsa_check_device_error()
     e2e_ms, h2d, d2h = e2e_measure(hd, x, device, steps=max(2, min(args.steps, 4)))
-    if dist:
-        tt = torch.tensor([e2e_ms], device=device)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_ms = float(tt.item())
-    e2e = {"value": world * L / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+    e2e_ms = max_over_ranks(e2e_ms, dist, device)
+    e2e = {"value": job_throughput(e2e_ms, world), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
            "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
 
     cpu = None
@@ -403,7 +416,7 @@ def ours(args):
     traffic = profiled_traffic("dsa_sparse_attn_fwd_L32768.md", "dsa_attn.cu")
     line = {
         "metric": METRIC,
-        "value": world * L / (ms_step * 1e-3),
+        "value": job_throughput(ms_step, world),
         "unit": "tokens/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms_step,
@@ -449,9 +462,9 @@ def reference(args):
     per = []
     cpu = None
     for _ in range(args.warmup):
-        cpu_sample(n_hca=4, n_dsa=1)
+        cpu_sample(n_hca=256, n_dsa=32)
     for _ in range(args.steps):
-        cpu = cpu_sample(n_hca=16, n_dsa=2)
+        cpu = cpu_sample(n_hca=1024, n_dsa=128)
         per.append(cpu["value"])
     v = statistics.median(per)
     cpu["value"] = v

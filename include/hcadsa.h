@@ -74,6 +74,16 @@ const char* hcadsa_last_error_string(void);
 hcadsa_status hcadsa_check_device_error(hcadsa_stream stream);
 
 /*
+ * Self-test of the device-side failure path (no counterpart on the pages): launches one
+ * block that waits on a barrier nothing arrives on, with a limit of `timeout_us`
+ * microseconds (1 .. 10^7).  The wait gives up, records HCADSA_ERR_TIMEOUT in the device
+ * error word and the kernel returns normally; a following hcadsa_check_device_error()
+ * reports it.  Every wait inside the library's kernels uses the same bounded mechanism
+ * (limit 2 s), so a lost arrival turns into an error status instead of a hung GPU.
+ */
+hcadsa_status hcadsa_selftest_bounded_wait(unsigned timeout_us, hcadsa_stream stream);
+
+/*
  * HCA block compression.  Source: mirrorspeed / besthub sections cited above
  * ("every 128 tokens are compressed into one cache entry").  Compressor form
  * (the pages leave it open): entry j of head h, channel c is

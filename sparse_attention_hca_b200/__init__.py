@@ -55,6 +55,8 @@ def lib() -> ctypes.CDLL:
             L.hcadsa_status_string.restype = ctypes.c_char_p
             L.hcadsa_last_error_string.argtypes = []
             L.hcadsa_last_error_string.restype = ctypes.c_char_p
+            L.hcadsa_selftest_bounded_wait.argtypes = [ctypes.c_uint, P]
+            L.hcadsa_selftest_bounded_wait.restype = I
             L.hcadsa_check_device_error.argtypes = [P]
             L.hcadsa_check_device_error.restype = I
             L.hca_compress_kv.argtypes = [P, P, P, P, P, I, I, I, I, I, P]

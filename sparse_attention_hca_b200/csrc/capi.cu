@@ -6,6 +6,7 @@
 #include <mutex>
 
 #include "host_common.h"
+#include "ptx.cuh"
 
 namespace hcadsa {
 namespace {
@@ -65,6 +66,20 @@ bool encode_tmap_bf16(CUtensorMap* map, int rank, void* base, const uint64_t* di
 
 thread_local char t_last_error[256] = "";
 
+// Waits on an mbarrier that nothing ever arrives on, with a short limit: exercises the bounded
+// wait every kernel uses, which must give up, record HCADSA_ERR_TIMEOUT and return.
+__global__ void bounded_wait_selftest_kernel(int* err, unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbarrier_init();
+  }
+  __syncthreads();
+  mbar_wait_for(&bar, 0, &abort_flag, err, limit_ns);
+}
+
 void record_cuda_error(cudaError_t e) {
   snprintf(t_last_error, sizeof(t_last_error), "%s: %s", cudaGetErrorName(e), cudaGetErrorString(e));
 }
@@ -72,6 +87,15 @@ void record_cuda_error(cudaError_t e) {
 }  // namespace hcadsa
 
 extern "C" const char* hcadsa_last_error_string(void) { return hcadsa::t_last_error; }
+
+extern "C" hcadsa_status hcadsa_selftest_bounded_wait(unsigned timeout_us, hcadsa_stream stream) {
+  using namespace hcadsa;
+  if (timeout_us == 0 || timeout_us > 10000000u) return HCADSA_ERR_SHAPE;
+  int* err = device_error_ptr();
+  if (!err) return HCADSA_ERR_CUDA;
+  bounded_wait_selftest_kernel<<<1, 32, 0, as_stream(stream)>>>(err, 1000ull * timeout_us);
+  return launch_status();
+}
 
 extern "C" int hcadsa_version(void) { return 100; }
 

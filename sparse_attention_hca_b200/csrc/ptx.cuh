@@ -65,14 +65,15 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
 // Wait until the phase with the given parity has completed.  Returns false (and
 // raises the timeout error + the CTA abort flag) if it has not after kWaitLimitNs,
 // or if another thread of the CTA already aborted.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int* err) {
+__device__ __forceinline__ bool mbar_wait_for(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int* err,
+                                              unsigned long long limit_ns) {
   if (mbar_test(bar, parity)) return true;
   const unsigned long long t0 = global_timer_ns();
   uint32_t spins = 0;
   while (!mbar_test(bar, parity)) {
     if ((++spins & 255u) == 0) {
       if (*abort_flag) return false;
-      if (global_timer_ns() - t0 > kWaitLimitNs) {
+      if (global_timer_ns() - t0 > limit_ns) {
         raise_device_error(err, kErrTimeout);
         *abort_flag = 1;
         return false;
@@ -80,6 +81,10 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     }
   }
   return true;
+}
+
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int* err) {
+  return mbar_wait_for(bar, parity, abort_flag, err, kWaitLimitNs);
 }
 
 // ------------------------------------------------------------------ TMA
