@@ -4,11 +4,15 @@
 // the pages -- "Hybrid sparse attention, 1/7 full context access" on the mirrorspeed
 // page -- only say that 128 tokens become one entry).
 //
-// The work is a pure HBM stream: each thread owns 8 adjacent channels of one block
-// and walks its blk rows in order, so one warp reads 512 contiguous bytes per row
-// and the FMA order per channel is exactly the sequential chain.  Loads for 16 rows
-// are issued before their FMAs to keep enough bytes in flight per SM.
+// The work is a pure HBM stream.  Persistent CTAs walk work units (tensor, batch, block,
+// 256-channel column group).  One thread streams each unit's rows into a 3-stage ring of
+// shared-memory boxes (TMA, up to 128 rows x 256 channels = 64 KB per box) so plenty of
+// bytes are in flight per SM; four warps then run the sequential FMA chains from shared
+// memory, two channels per thread, rows in ascending order -- exactly the fixed
+// accumulation order, so results are bit-identical to a plain loop.
 #include <cuda_bf16.h>
+
+#include <mutex>
 
 #include "host_common.h"
 #include "ptx.cuh"
@@ -16,72 +20,105 @@
 namespace hcadsa {
 namespace {
 
-constexpr int kMaxThreads = 128;
-constexpr int kRowsInFlight = 16;
+constexpr int kCols = 256;            // channels per work unit (TMA box width)
+constexpr int kBoxRows = 128;         // rows per TMA box
+constexpr int kStages = 3;
+constexpr int kBoxBytes = kCols * kBoxRows * 2;  // 64 KB
+constexpr int kConsumerWarps = 4;     // 128 threads x 2 channels = 256 channels
+constexpr int kThreads = 32 * (kConsumerWarps + 1);
+constexpr int kSmemBytes = kStages * kBoxBytes + 128;
 
-__device__ __forceinline__ float bf16_lo(uint32_t u) { return __uint_as_float(u << 16); }
-__device__ __forceinline__ float bf16_hi(uint32_t u) { return __uint_as_float(u & 0xFFFF0000u); }
+struct Params {
+  const float* w;
+  uint16_t* Kc;
+  uint16_t* Vc;
+  int* err;
+  int B, L, row_elems, n_c, blk, col_groups, n_units;
+};
 
-__device__ __forceinline__ uint4 ld_stream(const uint4* p) { return __ldg(p); }
-
-// grid: x = B * n_c blocks, y = column groups of blockDim.x*8 channels, z = 2 (K, V)
-__global__ void __launch_bounds__(kMaxThreads) hca_compress_kernel(const uint16_t* __restrict__ K,
-                                                                const uint16_t* __restrict__ V,
-                                                                const float* __restrict__ w,
-                                                                uint16_t* __restrict__ Kc,
-                                                                uint16_t* __restrict__ Vc, int L, int row_elems,
-                                                                int n_c, int blk) {
+__global__ void __launch_bounds__(kThreads, 1)
+    hca_compress_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v,
+                        const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+  __shared__ uint64_t full[kStages], empty[kStages];
   __shared__ float sw[1024];
-  for (int i = threadIdx.x; i < blk; i += blockDim.x) sw[i] = w[i];
+  __shared__ int abort_flag;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  for (int i = threadIdx.x; i < p.blk; i += kThreads) sw[i] = p.w[i];
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kConsumerWarps * 32);
+    }
+    abort_flag = 0;
+    fence_mbarrier_init();
+  }
   __syncthreads();
+  const int boxes_per_unit = (p.blk + kBoxRows - 1) / kBoxRows;
 
-  const int col = (blockIdx.y * blockDim.x + threadIdx.x) * 8;
-  if (col >= row_elems) return;
-  const int b = blockIdx.x / n_c, j = blockIdx.x % n_c;
-  const uint16_t* src = (blockIdx.z == 0 ? K : V) + ((size_t)b * L + (size_t)blk * j) * row_elems + col;
-  uint16_t* dst = (blockIdx.z == 0 ? Kc : Vc) + ((size_t)b * n_c + j) * row_elems + col;
+  if (warp == kConsumerWarps) {
+    // ------------------------------------------------------------ producer (one thread)
+    if (lane == 0) {
+      uint32_t q = 0;  // boxes issued: stage q % kStages, phase (q / kStages) & 1
+      for (int u = blockIdx.x; u < p.n_units; u += gridDim.x) {
+        const int cg = u % p.col_groups;
+        const int rest = u / p.col_groups;
+        const int tensor = rest & 1;
+        const int bj = rest >> 1;  // b * n_c + j
+        const int b = bj / p.n_c, j = bj % p.n_c;
+        const int row0 = b * p.L + j * p.blk;
+        for (int bx = 0; bx < boxes_per_unit; ++bx, ++q) {
+          const uint32_t st = q % kStages;
+          if (!mbar_wait(&empty[st], ((q / kStages) & 1) ^ 1, &abort_flag, p.err)) return;
+          mbar_arrive_expect_tx(&full[st], kBoxBytes);
+          tma_load_2d(ring + st * kBoxBytes, tensor ? &map_v : &map_k, &full[st], cg * kCols, row0 + bx * kBoxRows);
+        }
+      }
+    }
+    return;
+  }
 
-  float acc[8];
-#pragma unroll
-  for (int c = 0; c < 8; ++c) acc[c] = 0.0f;
-
-  int i = 0;
-  for (; i + kRowsInFlight <= blk; i += kRowsInFlight) {
-    uint4 x[kRowsInFlight];
-#pragma unroll
-    for (int u = 0; u < kRowsInFlight; ++u)
-      x[u] = ld_stream(reinterpret_cast<const uint4*>(src + (size_t)(i + u) * row_elems));
-#pragma unroll
-    for (int u = 0; u < kRowsInFlight; ++u) {
-      const float wi = sw[i + u];
-      acc[0] = fmaf(wi, bf16_lo(x[u].x), acc[0]);
-      acc[1] = fmaf(wi, bf16_hi(x[u].x), acc[1]);
-      acc[2] = fmaf(wi, bf16_lo(x[u].y), acc[2]);
-      acc[3] = fmaf(wi, bf16_hi(x[u].y), acc[3]);
-      acc[4] = fmaf(wi, bf16_lo(x[u].z), acc[4]);
-      acc[5] = fmaf(wi, bf16_hi(x[u].z), acc[5]);
-      acc[6] = fmaf(wi, bf16_lo(x[u].w), acc[6]);
-      acc[7] = fmaf(wi, bf16_hi(x[u].w), acc[7]);
+  // -------------------------------------------------------------- consumers: FMA chains
+  const int col = threadIdx.x * 2;  // 2 channels of the unit's 256
+  uint32_t q = 0;
+  for (int u = blockIdx.x; u < p.n_units; u += gridDim.x) {
+    const int cg = u % p.col_groups;
+    const int rest = u / p.col_groups;
+    const int tensor = rest & 1;
+    const int bj = rest >> 1;
+    float a0 = 0.0f, a1 = 0.0f;
+    for (int bx = 0; bx < boxes_per_unit; ++bx, ++q) {
+      const uint32_t st = q % kStages;
+      if (!mbar_wait(&full[st], (q / kStages) & 1, &abort_flag, p.err)) return;
+      const uint32_t* box = reinterpret_cast<const uint32_t*>(ring + st * kBoxBytes) + threadIdx.x;
+      const int rows = min(kBoxRows, p.blk - bx * kBoxRows);
+      const float* wr = sw + bx * kBoxRows;
+#pragma unroll 8
+      for (int i = 0; i < rows; ++i) {
+        const uint32_t x = box[i * (kCols / 2)];
+        a0 = fmaf(wr[i], __uint_as_float(x << 16), a0);
+        a1 = fmaf(wr[i], __uint_as_float(x & 0xFFFF0000u), a1);
+      }
+      mbar_arrive(&empty[st]);
+    }
+    const int gcol = cg * kCols + col;
+    if (gcol < p.row_elems) {
+      uint16_t* dst = (tensor ? p.Vc : p.Kc) + (size_t)bj * p.row_elems + gcol;
+      *reinterpret_cast<uint32_t*>(dst) = pack_bf16x2(a0, a1);
     }
   }
-  for (; i < blk; ++i) {
-    const uint4 x = ld_stream(reinterpret_cast<const uint4*>(src + (size_t)i * row_elems));
-    const float wi = sw[i];
-    acc[0] = fmaf(wi, bf16_lo(x.x), acc[0]);
-    acc[1] = fmaf(wi, bf16_hi(x.x), acc[1]);
-    acc[2] = fmaf(wi, bf16_lo(x.y), acc[2]);
-    acc[3] = fmaf(wi, bf16_hi(x.y), acc[3]);
-    acc[4] = fmaf(wi, bf16_lo(x.z), acc[4]);
-    acc[5] = fmaf(wi, bf16_hi(x.z), acc[5]);
-    acc[6] = fmaf(wi, bf16_lo(x.w), acc[6]);
-    acc[7] = fmaf(wi, bf16_hi(x.w), acc[7]);
-  }
-  uint4 out;
-  out.x = pack_bf16x2(acc[0], acc[1]);
-  out.y = pack_bf16x2(acc[2], acc[3]);
-  out.z = pack_bf16x2(acc[4], acc[5]);
-  out.w = pack_bf16x2(acc[6], acc[7]);
-  *reinterpret_cast<uint4*>(dst) = out;
+}
+
+int num_sms() {
+  static std::mutex mu;
+  static int cache[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!cache[dev] && cudaDeviceGetAttribute(&cache[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return 0;
+  return cache[dev];
 }
 
 }  // namespace
@@ -99,12 +136,37 @@ extern "C" hcadsa_status hca_compress_kv(const hcadsa_bf16* K, const hcadsa_bf16
   const int n_c = L / blk;
   if (B == 0 || n_c == 0) return HCADSA_OK;
   const long long row_elems = (long long)Hkv * d;
-  if ((long long)B * n_c > 2147483647LL || row_elems > (1LL << 30)) return HCADSA_ERR_UNSUPPORTED;
-  const long long groups8 = row_elems / 8;
-  const int threads = (int)(groups8 >= kMaxThreads ? kMaxThreads : ((groups8 + 31) / 32) * 32);
-  const long long col_blocks = (groups8 + threads - 1) / threads;
-  if (col_blocks > 65535) return HCADSA_ERR_UNSUPPORTED;
-  dim3 grid((unsigned)(B * n_c), (unsigned)col_blocks, 2);
-  hca_compress_kernel<<<grid, threads, 0, as_stream(stream)>>>(K, V, w, Kc, Vc, L, (int)row_elems, n_c, blk);
+  const long long rows = (long long)B * L;
+  if (row_elems > (1LL << 24) || rows > 2147483647LL) return HCADSA_ERR_UNSUPPORTED;
+  const long long col_groups = (row_elems + kCols - 1) / kCols;
+  const long long n_units = 2LL * B * n_c * col_groups;
+  if (n_units > 2147483647LL) return HCADSA_ERR_UNSUPPORTED;
+  // [rows, row_elems] bf16, box = 128 rows x 256 channels, no swizzle; box parts past the last
+  // row or the last channel are zero-filled and never stored
+  CUtensorMap mk, mv;
+  const uint64_t dims[2] = {(uint64_t)row_elems, (uint64_t)rows};
+  const uint64_t strides[1] = {(uint64_t)row_elems * 2};
+  const uint32_t box[2] = {(uint32_t)kCols, (uint32_t)kBoxRows};
+  if (!encode_tmap_bf16(&mk, 2, const_cast<hcadsa_bf16*>(K), dims, strides, box, false)) return HCADSA_ERR_CUDA;
+  if (!encode_tmap_bf16(&mv, 2, const_cast<hcadsa_bf16*>(V), dims, strides, box, false)) return HCADSA_ERR_CUDA;
+  Params p;
+  p.w = w;
+  p.Kc = Kc;
+  p.Vc = Vc;
+  p.err = device_error_ptr();
+  p.B = B;
+  p.L = L;
+  p.row_elems = (int)row_elems;
+  p.n_c = n_c;
+  p.blk = blk;
+  p.col_groups = (int)col_groups;
+  p.n_units = (int)n_units;
+  if (cudaFuncSetAttribute(hca_compress_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) !=
+      cudaSuccess)
+    return HCADSA_ERR_CUDA;
+  const int sms = num_sms();
+  if (sms <= 0) return HCADSA_ERR_CUDA;
+  const int grid = (int)(n_units < sms ? n_units : sms);
+  hca_compress_kernel<<<grid, kThreads, kSmemBytes, as_stream(stream)>>>(mk, mv, p);
   return launch_status();
 }
