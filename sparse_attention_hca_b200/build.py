@@ -64,7 +64,8 @@ def build(force: bool = False, verbose: bool = False) -> str:
     if failed:
         raise RuntimeError("nvcc failed while building libhcadsa.so")
     tmp = LIB + f".tmp{os.getpid()}"
-    subprocess.run([nvcc(), "-shared", *objs, "-o", tmp, "-lcudart", "-lcuda"], check=True)
+    subprocess.run([nvcc(), "-gencode", "arch=compute_100a,code=sm_100a", "-shared", *objs, "-o", tmp, "-lcudart", "-lcuda"],
+                   check=True)
     os.replace(tmp, LIB)
     return LIB
 
