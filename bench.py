@@ -206,13 +206,15 @@ class Step:
         self.idx = torch.empty((1, L, DSA.k), dtype=torch.int32, device=device)
         ws = hd.dsa_index_topk_workspace_size(1, L, 0, L, DSA.k)
         self.ws = torch.empty(ws, dtype=torch.uint8, device=device)
+        hws = hd.lib().hca_attn_fwd_workspace_size(1, L, 0, HCA.Hq, HCA.Hkv, HCA.d, L // 128, 128, 128)
+        self.hws = torch.empty(max(hws, 16), dtype=torch.uint8, device=device)
 
     def run(self, ev=None):
         hd, x = self.hd, self.x
         if ev: ev[0].record()
         hd.hca_compress_kv(x["hK"], x["hV"], x["w"], 128, Kc=self.Kc, Vc=self.Vc)
         if ev: ev[1].record()
-        hd.hca_attn_fwd(x["hQ"], self.Kc, self.Vc, x["hK"], x["hV"], O=self.hO)
+        hd.hca_attn_fwd(x["hQ"], self.Kc, self.Vc, x["hK"], x["hV"], O=self.hO, workspace=self.hws)
         if ev: ev[2].record()
         hd.dsa_index_topk(x["q_idx"], x["k_idx"], x["w_idx"], DSA.k, idx=self.idx, workspace=self.ws)
         if ev: ev[3].record()
@@ -246,10 +248,12 @@ def run_decode(hd, device, iters=5):
     idx = torch.empty(B, 1, DEC.k, dtype=torch.int32, device=device)
     ws = torch.empty(hd.dsa_index_topk_workspace_size(B, 1, t, Lk, DEC.k), dtype=torch.uint8, device=device)
     ws_start = t - DEC.W + 1
+    hws = hd.lib().hca_attn_fwd_workspace_size(B, 1, t, 16, 1, 512, n_c, 128, DEC.W)
+    hws = torch.empty(max(hws, 16), dtype=torch.uint8, device=device)
 
     def step(ev=None):
         if ev: ev[0].record()
-        hd.hca_attn_fwd(hQ, Kc, Vc, Kw, Vw, win_start=ws_start, q_offset=t, O=hO)
+        hd.hca_attn_fwd(hQ, Kc, Vc, Kw, Vw, win_start=ws_start, q_offset=t, O=hO, workspace=hws)
         if ev: ev[1].record()
         hd.dsa_index_topk(q_idx, k_idx, w_idx, DEC.k, q_offset=t, idx=idx, workspace=ws)
         if ev: ev[2].record()
@@ -494,7 +498,7 @@ def only_kernel(args):
     torch.cuda.synchronize()
     fn = {
         "compress": lambda: hd.hca_compress_kv(x["hK"], x["hV"], x["w"], 128, Kc=st.Kc, Vc=st.Vc),
-        "hca_attn": lambda: hd.hca_attn_fwd(x["hQ"], st.Kc, st.Vc, x["hK"], x["hV"], O=st.hO),
+        "hca_attn": lambda: hd.hca_attn_fwd(x["hQ"], st.Kc, st.Vc, x["hK"], x["hV"], O=st.hO, workspace=st.hws),
         "index_topk": lambda: hd.dsa_index_topk(x["q_idx"], x["k_idx"], x["w_idx"], DSA.k, idx=st.idx,
                                                 workspace=st.ws),
         "dsa_attn": lambda: hd.dsa_sparse_attn_fwd(x["dQ"], x["dK"], x["dV"], st.idx, O=st.dO),

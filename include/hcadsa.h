@@ -101,10 +101,15 @@ hcadsa_status hca_compress_kv(const hcadsa_bf16* K, const hcadsa_bf16* V, const 
                               hcadsa_bf16* Vc, int B, int L, int Hkv, int d, int blk, hcadsa_stream stream);
 
 /*
- * Size in bytes of the workspace hca_attn_fwd needs for these sizes (0 when it
- * needs none: prefill-shaped calls).  Decode-shaped calls (few query tokens
- * over many keys) split the keys across thread blocks and combine partial
- * softmax results through this workspace.
+ * Size in bytes of the workspace hca_attn_fwd needs for these sizes on the current
+ * device (0 if the sizes are invalid or unsupported; the call then reports why).
+ * The kernel computes each probability tile P once, for the first half of the
+ * 512-wide value dimension, and keeps it in this workspace (bf16, plus one fp32
+ * rescale factor per row and key tile) for the second half:
+ *     min(#tiles, #SMs) * J_max * (128*128*2 + 128*4) bytes,
+ * where #tiles = B * Hkv * ceil(Lq / (128 / (Hq/Hkv))) and J_max = ceil(n_c(t_last)/128)
+ * + floor((128/(Hq/Hkv) + W + 126) / 128) key tiles.  The workspace holds no state
+ * between calls; concurrent calls need separate workspaces.
  */
 size_t hca_attn_fwd_workspace_size(int B, int Lq, int q_offset, int Hq, int Hkv, int d, int n_c, int blk,
                                    int W);
@@ -127,7 +132,8 @@ size_t hca_attn_fwd_workspace_size(int B, int Lq, int q_offset, int Hq, int Hkv,
  *              (prefill: Kw = K, win_start = 0, n_w = L)
  *   O        : [B, Lq, Hq, d] bf16     (written)
  *   lse      : [B, Lq, Hq] fp32 natural-log log-sum-exp, or NULL
- *   workspace: hca_attn_fwd_workspace_size(...) bytes (NULL allowed when that is 0)
+ *   workspace: at least hca_attn_fwd_workspace_size(...) bytes of device memory, 16-byte
+ *              aligned (HCADSA_ERR_WORKSPACE if NULL or smaller, HCADSA_ERR_ALIGN if misaligned)
  * Requirements: d == 512; Hq % Hkv == 0 and (Hq/Hkv) divides 128; every query
  * must have its window inside [win_start, win_start + n_w) and n_c(t) <= n_c.
  */

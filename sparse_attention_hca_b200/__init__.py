@@ -150,8 +150,11 @@ def hca_attn_fwd(Q, Kc, Vc, Kw, Vw, *, win_start: int = 0, q_offset: int = 0, bl
         lse = torch.empty((B, Lq, Hq), dtype=torch.float32, device=Q.device)
     L = lib()
     ws_bytes = L.hca_attn_fwd_workspace_size(B, Lq, q_offset, Hq, Hkv, d, n_c, blk, W)
-    if ws_bytes and workspace is None:
-        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=Q.device)
+    if workspace is None:
+        if ws_bytes:
+            workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=Q.device)
+    else:
+        ws_bytes = workspace.numel() * workspace.element_size()
     st = L.hca_attn_fwd(_ptr(Q), _ptr(Kc) if n_c else None, _ptr(Vc) if n_c else None, n_c, _ptr(Kw),
                         _ptr(Vw), win_start, n_w, _ptr(O), _ptr(lse), B, Lq, q_offset, Hq, Hkv, d, blk, W,
                         float(scale), _ptr(workspace), ws_bytes, _stream(stream))

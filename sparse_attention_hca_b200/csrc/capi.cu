@@ -35,8 +35,17 @@ int* device_error_ptr() {
   return g_error_ptr[dev];
 }
 
-bool encode_tmap_bf16(CUtensorMap* map, int rank, void* base, const uint64_t* dims, const uint64_t* strides_bytes,
-                      const uint32_t* box, bool swizzle128) {
+bool encode_tmap_bf16_swizzle(CUtensorMap* map, int rank, void* base, const uint64_t* dims,
+                              const uint64_t* strides_bytes, const uint32_t* box, int swizzle_bytes) {
+  CUtensorMapSwizzle sw;
+  switch (swizzle_bytes) {
+    case 0: sw = CU_TENSOR_MAP_SWIZZLE_NONE; break;
+    case 32: sw = CU_TENSOR_MAP_SWIZZLE_32B; break;
+    case 64: sw = CU_TENSOR_MAP_SWIZZLE_64B; break;
+    case 128: sw = CU_TENSOR_MAP_SWIZZLE_128B; break;
+    default: return false;
+  }
+  if (rank < 1 || rank > 5) return false;
   {
     std::lock_guard<std::mutex> lock(g_mu);
     if (!g_encode) {
@@ -58,10 +67,14 @@ bool encode_tmap_bf16(CUtensorMap* map, int rank, void* base, const uint64_t* di
     if (i + 1 < rank) st[i] = strides_bytes[i];
   }
   const CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, base, d, st, bx, es,
-                              CU_TENSOR_MAP_INTERLEAVE_NONE,
-                              swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
-                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                              CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+bool encode_tmap_bf16(CUtensorMap* map, int rank, void* base, const uint64_t* dims, const uint64_t* strides_bytes,
+                      const uint32_t* box, bool swizzle128) {
+  return encode_tmap_bf16_swizzle(map, rank, base, dims, strides_bytes, box, swizzle128 ? 128 : 0);
 }
 
 thread_local char t_last_error[256] = "";

@@ -7,30 +7,36 @@
 // section "混合注意力（MLA + HCA）").  Visible set of a query at t (this library's
 // reading): raw positions [max(0,t-W+1), t] and entries j < n_c(t) = max(0,(t-W+1)/blk).
 //
-// Kernel design (persistent: a CTA walks row tiles T = blockIdx.x + i*gridDim.x and runs the
-// two 256-wide halves of d_v of each tile back to back as two work items):
+// Kernel design (persistent: a CTA walks row tiles T = blockIdx.x + i*gridDim.x):
 //   * A row tile = 128 rows = (128/g) consecutive tokens x the g query heads sharing one K/V
 //     head, so every K/V tile is shared by the whole tile and the window band of 128/g
 //     tokens spans only 128/g + W - 1 keys.
-//   * d = 512 makes a 128 x 512 fp32 O accumulator fill all of TMEM, so a work item keeps O
-//     for one half of d_v: TMEM = O half [0,256) + two S buffers [256,384), [384,512).  Each
-//     item recomputes S = Q K^T (1.5x the algorithmic MMA work); Q is loaded once per tile.
-//   * warp 0: TMA producer (Q per tile, then K chunks and V chunks through a 5-slot ring of
-//     16 KB stages, in exactly the order the MMA warp consumes them; key tiles of at most
-//     32 keys use 32-row boxes); warp 1: TMEM allocation and the single MMA-issuing thread;
-//     warps 2-5: softmax, one thread per row (TMEM lane), then the item's epilogue.  The next
-//     item's S MMAs run while the epilogue drains O.
-//   * S_j = Q K_j^T accumulates over eight 64-wide d chunks (SS MMA, K-major operands,
-//     128B swizzle).  Softmax converts S_j to P_j (bf16) in place in TMEM and PV runs as
-//     a TS MMA (A = P from TMEM, B = V chunk, MN-major).  Online softmax with a lazy
-//     rescale: the reference max only moves when the tile max exceeds it by 2^8.
+//   * d = 512 makes a 128 x 512 fp32 O accumulator fill all of TMEM, so O is built one
+//     256-wide half of d_v at a time: TMEM = O half [0,256) + two S buffers [256,384),
+//     [384,512).  Phase A of a tile computes S_j = Q K_j^T, the online softmax and
+//     O[:, 0:256] += P_j V_j[:, 0:256]; it also writes each P_j (bf16) and the rescale
+//     factor it applied to a per-CTA scratch (L2-resident).  Phase B reloads those P_j into
+//     TMEM and runs only O[:, 256:512] += P_j V_j[:, 256:512] with the same rescales, so the
+//     second half costs no QK^T and no exponentials, and Q's buffer is free to take the
+//     next tile's Q while phase B runs.
+//   * warp 0: TMA producer (Q per tile; K chunks and V chunks through a 5-slot ring of 16 KB
+//     stages, in exactly the order the MMA warp consumes them; key tiles of at most 32 keys
+//     use 32-row boxes); warp 1: TMEM allocation and the single MMA-issuing thread;
+//     warps 2-5: softmax, one thread per row (TMEM lane), and the epilogues, which stage O
+//     through shared memory (64-byte swizzle, two 8 KB buffers) into TMA tensor stores.
+//   * S_j accumulates over eight 64-wide d chunks (SS MMA, K-major operands, 128B swizzle).
+//     P_j is written in place over S_j in TMEM and PV runs as a TS MMA (A = P from TMEM,
+//     B = V chunk, MN-major).  Online softmax with a lazy rescale: the reference max only
+//     moves when the tile max exceeds it by 2^8.
 //   * Key tiles: compressed entries [0, n_c(t_last)) in tiles of 128, then the window
 //     band [max(0, t_first-W+1), t_last] in tiles of 128; per-row visibility is one
 //     column interval per tile.
-//   * Barrier phases run on across work items: s_full / p_ready / pv_done are per S buffer
-//     and follow a key-tile counter that never resets, o_full / o_empty follow the item
-//     counter, q_full / q_empty the row-tile counter.  MMAs on different accumulators are
-//     not ordered, so an S buffer is rewritten only after the PV that read its P completed.
+//   * Barrier phases run on across tiles: p_ready / pv_done are per S buffer and follow a
+//     key-tile counter that never resets (phase A and phase B tiles both count); s_full is per
+//     S buffer too but only phase-A tiles complete it, so its consumer keeps one parity bit per
+//     buffer; o_full / o_empty follow the O-half counter, q_full / q_empty the row-tile counter.
+//     MMAs on different accumulators are not ordered, so an S buffer is rewritten (by QK^T
+//     or by a P reload) only after the PV that read its previous P has completed.
 #include <cuda_bf16.h>
 
 #include <mutex>
@@ -51,23 +57,30 @@ constexpr int kSmallChunkBytes = kSmallRows * 128;
 constexpr int kQChunks = kD / 64;      // 8
 constexpr int kVChunks = kDHalf / 64;  // 4
 constexpr int kQBytes = kQChunks * kChunkBytes;
-constexpr int kSmemBytes = kQBytes + kStages * kChunkBytes + 1024;
+constexpr int kOutCols = 32;                  // O columns per staged store
+constexpr int kOutBufBytes = 128 * kOutCols * 2;  // 8 KB
+constexpr int kSmemBytes = kQBytes + kStages * kChunkBytes + 2 * kOutBufBytes + 1024;
 constexpr int kThreads = 192;
 constexpr float kLazyRescale = 8.0f;  // log2 units
+// per-CTA scratch per key tile: P (128 rows x 128 keys bf16) + one fp32 rescale factor per row
+constexpr size_t kScratchPBytes = 128 * kKeyTile * 2;
+constexpr size_t kScratchTileBytes = kScratchPBytes + 128 * 4;
 
 struct Params {
   int Lq, q_offset, Hq, Hkv, g, TT, n_c, win_start, W, blk;
   int n_tiles;      // token tiles per (b, kv head)
   int total_tiles;  // B * Hkv * n_tiles
+  int J_max;        // key tiles of the longest row tile (scratch capacity)
   float scale_log2;
-  uint16_t* O;
   float* lse;
+  uint8_t* scratch;  // gridDim.x * J_max * kScratchTileBytes
   int* err;
 };
 
-// Q, then K and V over {compressed entries, window} x {128-row box, 32-row box}.
+// Q and O, then K and V over {compressed entries, window} x {128-row box, 32-row box}.
 struct Maps {
   CUtensorMap q;
+  CUtensorMap o;            // box 32 columns x 128 rows, 64-byte swizzle (stores)
   CUtensorMap kv[2][2][2];  // [0 = K, 1 = V][0 = compressed, 1 = window][0 = 128 rows, 1 = 32 rows]
 };
 
@@ -78,6 +91,11 @@ __device__ __forceinline__ int n_compressed(int t, int W, int blk) {
 __device__ __forceinline__ int window_start(int t, int W) {
   const int s = t - W + 1;
   return s > 0 ? s : 0;
+}
+
+__device__ __forceinline__ void softmax_bar_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_group_read1() {
+  asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
 }
 
 struct KeyTile {
@@ -128,15 +146,48 @@ struct __align__(8) Barriers {
   uint64_t s_full[2];
   uint64_t p_ready[2];
   uint64_t pv_done[2];  // the PV that read P from S buffer i has completed
-  uint64_t o_full;      // every PV of the work item has completed
+  uint64_t o_full;      // every PV of the current O half has completed
   uint64_t o_empty;     // the epilogue has read O
 };
+
+// One thread's row of P_j in the scratch: key tile j owns kScratchTileBytes; inside it the
+// 16-byte unit c16 (8 keys) of row r is unit c16*128 + r, so a warp's 32 rows are one
+// contiguous 512-byte run; the 128 rescale factors follow the P units.
+__device__ __forceinline__ uint4* scratch_p(uint8_t* base, int j, int r) {
+  return reinterpret_cast<uint4*>(base + (size_t)j * kScratchTileBytes) + r;
+}
+__device__ __forceinline__ float* scratch_alpha(uint8_t* base, int j, int r) {
+  return reinterpret_cast<float*>(base + (size_t)j * kScratchTileBytes + kScratchPBytes) + r;
+}
+
+// Loads row r of P_j (n keys) from the scratch into 16 registers of 8 keys each.
+__device__ __forceinline__ void load_p_row(uint4 (&pr)[16], float& alpha, uint8_t* base, int j, int n, int r) {
+  const uint4* src = scratch_p(base, j, r);
+#pragma unroll
+  for (int c = 0; c < 16; ++c)
+    pr[c] = c * 8 < n ? __ldcg(src + c * 128) : make_uint4(0u, 0u, 0u, 0u);
+  alpha = __ldcg(scratch_alpha(base, j, r));
+}
+
+// Multiplies this thread's row of the O half by alpha.
+__device__ __forceinline__ void rescale_o(uint32_t t_row, float alpha) {
+  for (int oc = 0; oc < kDHalf; oc += 32) {
+    uint32_t v[32];
+    tmem_ld32_nowait(t_row + oc, v);
+    tmem_wait_ld_regs(v);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * alpha);
+    tmem_st32(t_row + oc, v);
+  }
+  tmem_wait_st();
+}
 
 __global__ void __launch_bounds__(kThreads, 1) hca_attn_kernel(const __grid_constant__ Maps maps, const Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;
   uint8_t* sRing = smem + kQBytes;
+  uint8_t* sOut = sRing + kStages * kChunkBytes;
   __shared__ Barriers bar;
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_flag;
@@ -172,41 +223,61 @@ __global__ void __launch_bounds__(kThreads, 1) hca_attn_kernel(const __grid_cons
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       tma_prefetch_desc(&maps.q);
-      uint32_t q = 0;       // ring chunks issued: slot q % kStages, phase (q / kStages) & 1
-      uint32_t tcount = 0;  // row tiles started
+      uint32_t q = 0;  // ring chunks issued: slot q % kStages, phase (q / kStages) & 1
       bool ok = true;
+      auto load_chunk = [&](const CUtensorMap* m, bool small, int col, int hk, int row0, int b) {
+        const uint32_t slot = q % kStages;
+        ok = mbar_wait(&bar.empty[slot], ((q / kStages) & 1) ^ 1, &abort_flag, p.err);
+        if (ok) {
+          mbar_arrive_expect_tx(&bar.full[slot], small ? kSmallChunkBytes : kChunkBytes);
+          tma_load_4d(sRing + slot * kChunkBytes, m, &bar.full[slot], col, hk, row0, b);
+        }
+        ++q;
+      };
+      auto load_v = [&](const TileSet& ts, int j, int col0) {
+        const KeyTile kt = ts.get(j);
+        const int small = kt.n <= kSmallRows ? 1 : 0;
+        const int row0 = kt.window ? kt.start - p.win_start : kt.start;
+        for (int c = 0; ok && c < kVChunks; ++c)
+          load_chunk(&maps.kv[1][kt.window][small], small, col0 + c * 64, ts.hk, row0, ts.b);
+      };
+      if (blockIdx.x < p.total_tiles) {
+        TileSet t0;
+        t0.init(blockIdx.x, p);
+        mbar_arrive_expect_tx(&bar.q_full, kQBytes);
+        for (int c = 0; c < kQChunks; ++c)
+          tma_load_4d(sQ + c * kChunkBytes, &maps.q, &bar.q_full, c * 64, t0.hk * p.g, t0.tok0, t0.b);
+      }
+      uint32_t tcount = 0;
       for (int T = blockIdx.x; ok && T < p.total_tiles; T += gridDim.x, ++tcount) {
         TileSet ts;
         ts.init(T, p);
-        // Q of this tile, once the previous tile's last S MMA has read the buffer
-        ok = mbar_wait(&bar.q_empty, (tcount & 1) ^ 1, &abort_flag, p.err);
-        if (!ok) break;
-        mbar_arrive_expect_tx(&bar.q_full, kQBytes);
-        for (int c = 0; c < kQChunks; ++c)
-          tma_load_4d(sQ + c * kChunkBytes, &maps.q, &bar.q_full, c * 64, ts.hk * p.g, ts.tok0, ts.b);
-        for (int half = 0; ok && half < 2; ++half) {
-          for (int step = 0; ok && step <= ts.J; ++step) {
-            // step s: the K chunks of key tile s, then the V chunks (this half) of key tile s-1
-            for (int part = 0; ok && part < 2; ++part) {
-              const int is_v = part;
-              const int j = step - is_v;
-              if (j < 0 || j >= ts.J) continue;
-              const KeyTile kt = ts.get(j);
-              const int small = kt.n <= kSmallRows ? 1 : 0;
-              const CUtensorMap* m = &maps.kv[is_v][kt.window][small];
-              const int row0 = kt.window ? kt.start - p.win_start : kt.start;
-              const int n_ch = is_v ? kVChunks : kQChunks;
-              const int col0 = is_v ? half * kDHalf : 0;
-              for (int c = 0; c < n_ch; ++c, ++q) {
-                const uint32_t slot = q % kStages;
-                ok = mbar_wait(&bar.empty[slot], ((q / kStages) & 1) ^ 1, &abort_flag, p.err);
-                if (!ok) break;
-                mbar_arrive_expect_tx(&bar.full[slot], small ? kSmallChunkBytes : kChunkBytes);
-                tma_load_4d(sRing + slot * kChunkBytes, m, &bar.full[slot], col0 + c * 64, ts.hk, row0, ts.b);
-              }
-            }
+        if (ts.J > p.J_max) break;
+        // phase A: step s loads the K chunks of key tile s, then the first-half V chunks of tile s-1
+        for (int step = 0; ok && step <= ts.J; ++step) {
+          if (step < ts.J) {
+            const KeyTile kt = ts.get(step);
+            const int small = kt.n <= kSmallRows ? 1 : 0;
+            const int row0 = kt.window ? kt.start - p.win_start : kt.start;
+            for (int c = 0; ok && c < kQChunks; ++c)
+              load_chunk(&maps.kv[0][kt.window][small], small, c * 64, ts.hk, row0, ts.b);
           }
+          if (ok && step >= 1) load_v(ts, step - 1, 0);
         }
+        if (!ok) break;
+        // the next tile's Q, once this tile's last S MMA has read the buffer
+        const int Tn = T + gridDim.x;
+        if (Tn < p.total_tiles) {
+          TileSet tn;
+          tn.init(Tn, p);
+          ok = mbar_wait(&bar.q_empty, tcount & 1, &abort_flag, p.err);
+          if (!ok) break;
+          mbar_arrive_expect_tx(&bar.q_full, kQBytes);
+          for (int c = 0; c < kQChunks; ++c)
+            tma_load_4d(sQ + c * kChunkBytes, &maps.q, &bar.q_full, c * 64, tn.hk * p.g, tn.tok0, tn.b);
+        }
+        // phase B: second-half V chunks
+        for (int j = 0; ok && j < ts.J; ++j) load_v(ts, j, kDHalf);
       }
     }
   } else if (warp == 1) {
@@ -215,76 +286,100 @@ __global__ void __launch_bounds__(kThreads, 1) hca_attn_kernel(const __grid_cons
       const uint32_t sQa = smem_u32(sQ), sRa = smem_u32(sRing);
       uint32_t q = 0;       // ring chunks consumed
       uint32_t tcount = 0;  // row tiles
-      uint32_t g = 0;       // key tiles of all earlier work items
-      uint32_t it = 0;      // work items
+      uint32_t g = 0;       // key tiles of all earlier phases
+      uint32_t it = 0;      // O halves
       bool ok = true;
+      const uint32_t idesc_pv = idesc_bf16_f32(128, 64, false, true);
+      // PV of key tile j (global counter gj) into the O half; V chunks from the ring
+      auto pv = [&](const KeyTile& kt, int j, uint32_t gj) {
+        const uint32_t tP = tmem + kDHalf + (gj & 1) * kKeyTile;
+        for (int c = 0; ok && c < kVChunks; ++c, ++q) {
+          const uint32_t slot = q % kStages;
+          ok = mbar_wait(&bar.full[slot], (q / kStages) & 1, &abort_flag, p.err);
+          if (!ok) break;
+          tc_fence_after();
+          for (int kk = 0; kk < kt.n / 16; ++kk) {
+            const uint64_t db = smem_desc_sw128(sRa + slot * kChunkBytes + kk * 2048, kChunkBytes, 1024);
+            mma_ts(tmem + c * 64, tP + kk * 8, db, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(&bar.empty[slot]);
+        }
+      };
       for (int T = blockIdx.x; ok && T < p.total_tiles; T += gridDim.x, ++tcount) {
         TileSet ts;
         ts.init(T, p);
+        if (ts.J > p.J_max) {
+          raise_device_error(p.err, kErrDeviceBounds);
+          break;
+        }
         ok = mbar_wait(&bar.q_full, tcount & 1, &abort_flag, p.err);
         if (!ok) break;
         tc_fence_after();
-        for (int half = 0; ok && half < 2; ++half, ++it) {
-          for (int step = 0; ok && step <= ts.J; ++step) {
-            if (step < ts.J) {
-              const uint32_t gs = g + step;
-              const KeyTile kt = ts.get(step);
-              const uint32_t tS = tmem + kDHalf + (gs & 1) * kKeyTile;
-              const uint32_t idesc = idesc_bf16_f32(128, kt.n, false, false);
-              // S buffer gs&1 holds P_{gs-2}, the TMEM operand of PV_{gs-2}
-              if (gs >= 2) {
-                ok = mbar_wait(&bar.pv_done[gs & 1], ((gs >> 1) - 1) & 1, &abort_flag, p.err);
-                if (!ok) break;
-                tc_fence_after();
-              }
-              for (int c = 0; ok && c < kQChunks; ++c, ++q) {
-                const uint32_t slot = q % kStages;
-                ok = mbar_wait(&bar.full[slot], (q / kStages) & 1, &abort_flag, p.err);
-                if (!ok) break;
-                tc_fence_after();
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                  const uint64_t da = smem_desc_sw128(sQa + c * kChunkBytes + k * 32, 16, 1024);
-                  const uint64_t db = smem_desc_sw128(sRa + slot * kChunkBytes + k * 32, 16, 1024);
-                  mma_ss(tS, da, db, idesc, (c | k) != 0);
-                }
-                mma_commit(&bar.empty[slot]);
-              }
-              if (!ok) break;
-              mma_commit(&bar.s_full[gs & 1]);
-              if (half == 1 && step == ts.J - 1) mma_commit(&bar.q_empty);
-            }
-            if (step >= 1) {
-              const int j = step - 1;
-              const uint32_t gj = g + j;
-              const KeyTile kt = ts.get(j);
-              if (j == 0) {  // the previous item's epilogue must have read O
-                ok = mbar_wait(&bar.o_empty, (it & 1) ^ 1, &abort_flag, p.err);
-                if (!ok) break;
-              }
-              ok = mbar_wait(&bar.p_ready[gj & 1], (gj >> 1) & 1, &abort_flag, p.err);
+        // ---- phase A: step s issues QK_s, then PV_{s-1} (first half of d_v)
+        for (int step = 0; ok && step <= ts.J; ++step) {
+          if (step < ts.J) {
+            const uint32_t gs = g + step;
+            const KeyTile kt = ts.get(step);
+            const uint32_t tS = tmem + kDHalf + (gs & 1) * kKeyTile;
+            const uint32_t idesc = idesc_bf16_f32(128, kt.n, false, false);
+            if (gs >= 2) {  // S buffer gs&1 holds P_{gs-2}, the TMEM operand of PV_{gs-2}
+              ok = mbar_wait(&bar.pv_done[gs & 1], ((gs >> 1) - 1) & 1, &abort_flag, p.err);
               if (!ok) break;
               tc_fence_after();
-              const uint32_t tP = tmem + kDHalf + (gj & 1) * kKeyTile;
-              const uint32_t idesc = idesc_bf16_f32(128, 64, false, true);
-              for (int c = 0; ok && c < kVChunks; ++c, ++q) {
-                const uint32_t slot = q % kStages;
-                ok = mbar_wait(&bar.full[slot], (q / kStages) & 1, &abort_flag, p.err);
-                if (!ok) break;
-                tc_fence_after();
-                for (int kk = 0; kk < kt.n / 16; ++kk) {
-                  const uint64_t db = smem_desc_sw128(sRa + slot * kChunkBytes + kk * 2048, kChunkBytes, 1024);
-                  mma_ts(tmem + c * 64, tP + kk * 8, db, idesc, (j > 0 || kk > 0) ? 1u : 0u);
-                }
-                mma_commit(&bar.empty[slot]);
-              }
-              if (!ok) break;
-              mma_commit(&bar.pv_done[gj & 1]);
-              if (j == ts.J - 1) mma_commit(&bar.o_full);
             }
+            for (int c = 0; ok && c < kQChunks; ++c, ++q) {
+              const uint32_t slot = q % kStages;
+              ok = mbar_wait(&bar.full[slot], (q / kStages) & 1, &abort_flag, p.err);
+              if (!ok) break;
+              tc_fence_after();
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                const uint64_t da = smem_desc_sw128(sQa + c * kChunkBytes + k * 32, 16, 1024);
+                const uint64_t db = smem_desc_sw128(sRa + slot * kChunkBytes + k * 32, 16, 1024);
+                mma_ss(tS, da, db, idesc, (c | k) != 0);
+              }
+              mma_commit(&bar.empty[slot]);
+            }
+            if (!ok) break;
+            mma_commit(&bar.s_full[gs & 1]);
+            if (step == ts.J - 1) mma_commit(&bar.q_empty);
           }
-          g += ts.J;
+          if (step >= 1) {
+            const int j = step - 1;
+            const uint32_t gj = g + j;
+            if (j == 0) {  // the previous O half's epilogue must have read O
+              ok = mbar_wait(&bar.o_empty, (it & 1) ^ 1, &abort_flag, p.err);
+              if (!ok) break;
+            }
+            ok = mbar_wait(&bar.p_ready[gj & 1], (gj >> 1) & 1, &abort_flag, p.err);
+            if (!ok) break;
+            tc_fence_after();
+            pv(ts.get(j), j, gj);
+            if (!ok) break;
+            mma_commit(&bar.pv_done[gj & 1]);
+            if (j == ts.J - 1) mma_commit(&bar.o_full);
+          }
         }
+        if (!ok) break;
+        g += ts.J;
+        ++it;
+        // ---- phase B: PV only (second half of d_v), P reloaded into TMEM by the softmax warps
+        for (int j = 0; ok && j < ts.J; ++j) {
+          const uint32_t gj = g + j;
+          if (j == 0) {
+            ok = mbar_wait(&bar.o_empty, (it & 1) ^ 1, &abort_flag, p.err);
+            if (!ok) break;
+          }
+          ok = mbar_wait(&bar.p_ready[gj & 1], (gj >> 1) & 1, &abort_flag, p.err);
+          if (!ok) break;
+          tc_fence_after();
+          pv(ts.get(j), j, gj);
+          if (!ok) break;
+          mma_commit(&bar.pv_done[gj & 1]);
+          if (j == ts.J - 1) mma_commit(&bar.o_full);
+        }
+        g += ts.J;
+        ++it;
       }
     }
   } else {
@@ -292,125 +387,188 @@ __global__ void __launch_bounds__(kThreads, 1) hca_attn_kernel(const __grid_cons
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;  // row of the tile == TMEM lane
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-    uint32_t g = 0, it = 0;
+    const bool store_issuer = r == 0;
+    uint8_t* scratch = p.scratch + (size_t)blockIdx.x * p.J_max * kScratchTileBytes;
+    uint32_t g = 0, it = 0, ec = 0;  // key tiles, O halves, staged stores
+    // s_full[b] completes once per phase-A key tile on S buffer b (phase B issues no QK^T), so
+    // its parity is tracked per buffer here rather than derived from the key-tile counter
+    uint32_t s_par = 0;
     bool ok = true;
+
+    // O half (TMEM) -> bf16 -> two 8 KB staging buffers -> TMA tensor store; then release O
+    auto epilogue = [&](const TileSet& ts, int col0, float inv_l) {
+      ok = mbar_wait(&bar.o_full, it & 1, &abort_flag, p.err);
+      if (!ok) return;
+      tc_fence_after();
+      for (int oc = 0; oc < kDHalf; oc += kOutCols, ++ec) {
+        uint32_t v[32];
+        tmem_ld32_nowait(tmem + lane_off + oc, v);
+        tmem_wait_ld_regs(v);
+        if (oc + kOutCols == kDHalf) {  // last read of O
+          tc_fence_before();
+          mbar_arrive(&bar.o_empty);
+        }
+        uint4 packed[4];
+        uint32_t* pw = reinterpret_cast<uint32_t*>(packed);
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          pw[i] = pack_bf16x2(__uint_as_float(v[2 * i]) * inv_l, __uint_as_float(v[2 * i + 1]) * inv_l);
+        uint8_t* buf = sOut + (ec & 1) * kOutBufBytes;
+        if (store_issuer && ec >= 2) bulk_wait_group_read1();  // the store from this buffer has read it
+        softmax_bar_sync();
+#pragma unroll
+        for (int i = 0; i < 4; ++i)  // 64-byte swizzle: 16-byte unit i of row r at unit i ^ ((r >> 1) & 3)
+          *reinterpret_cast<uint4*>(buf + r * 64 + ((i ^ ((r >> 1) & 3)) * 16)) = packed[i];
+        fence_proxy_async_smem();
+        softmax_bar_sync();
+        if (store_issuer) {
+          tma_store_4d(&maps.o, buf, col0 + oc, ts.hk * p.g, ts.tok0, ts.b);
+          bulk_commit_group();
+        }
+      }
+      ++it;
+    };
+
     for (int T = blockIdx.x; ok && T < p.total_tiles; T += gridDim.x) {
       TileSet ts;
       ts.init(T, p);
+      if (ts.J > p.J_max) break;
       const int tok = ts.tok0 + r / p.g;  // relative token index
       const int h = ts.hk * p.g + r % p.g;
       const bool row_valid = tok < p.Lq;
       const int t = p.q_offset + min(tok, p.Lq - 1);
       const int nc_t = n_compressed(t, p.W, p.blk);
       const int ws_t = window_start(t, p.W);
-      for (int half = 0; ok && half < 2; ++half, ++it) {
-        float m_ref = -INFINITY, l_run = 0.0f;
-        for (int j = 0; ok && j < ts.J; ++j) {
-          const uint32_t gs = g + j;
-          const KeyTile kt = ts.get(j);
-          int lo, hi;
-          if (kt.window) {
-            lo = max(ws_t, kt.start) - kt.start;
-            hi = min(t + 1, kt.start + kt.n) - kt.start;
-          } else {
-            lo = 0;
-            hi = min(nc_t, kt.start + kt.n) - kt.start;
+      float m_ref = -INFINITY, l_run = 0.0f;
+      // ---- phase A
+      for (int j = 0; ok && j < ts.J; ++j) {
+        const uint32_t gs = g + j;
+        const KeyTile kt = ts.get(j);
+        int lo, hi;
+        if (kt.window) {
+          lo = max(ws_t, kt.start) - kt.start;
+          hi = min(t + 1, kt.start + kt.n) - kt.start;
+        } else {
+          lo = 0;
+          hi = min(nc_t, kt.start + kt.n) - kt.start;
+        }
+        if (!row_valid) hi = lo;  // padding rows see nothing
+        const uint32_t tS = tmem + lane_off + kDHalf + (gs & 1) * kKeyTile;
+        ok = mbar_wait(&bar.s_full[gs & 1], (s_par >> (gs & 1)) & 1, &abort_flag, p.err);
+        if (!ok) break;
+        s_par ^= 1u << (gs & 1);
+        tc_fence_after();
+        // pass 1: tile max over this row's visible columns
+        float mx = -INFINITY;
+        for (int c0 = 0; c0 < kt.n; c0 += 32) {
+          uint32_t v[32];
+          tmem_ld32_nowait(tS + c0, v);
+          tmem_wait_ld_regs(v);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const int col = c0 + i;
+            if (col >= lo && col < hi) mx = fmaxf(mx, __uint_as_float(v[i]));
           }
-          if (!row_valid) hi = lo;  // padding rows see nothing
-          const uint32_t tS = tmem + lane_off + kDHalf + (gs & 1) * kKeyTile;
-          ok = mbar_wait(&bar.s_full[gs & 1], (gs >> 1) & 1, &abort_flag, p.err);
+        }
+        const float m_tile = mx * p.scale_log2;  // -inf stays -inf
+        bool need = false;
+        if (m_ref == -INFINITY) {
+          m_ref = m_tile;
+        } else if (m_tile > m_ref + kLazyRescale) {
+          need = true;
+        }
+        float alpha = 1.0f;
+        if (__any_sync(0xffffffffu, need)) {
+          // O must hold every PV of this half up to key tile j-1 (j >= 1 here) before the rescale
+          const uint32_t gp = gs - 1;
+          ok = mbar_wait(&bar.pv_done[gp & 1], (gp >> 1) & 1, &abort_flag, p.err);
           if (!ok) break;
           tc_fence_after();
-          // pass 1: tile max over this row's visible columns
-          float mx = -INFINITY;
-          for (int c0 = 0; c0 < kt.n; c0 += 32) {
-            uint32_t v[32];
-            tmem_ld32_nowait(tS + c0, v);
-            tmem_wait_ld_regs(v);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              const int col = c0 + i;
-              if (col >= lo && col < hi) mx = fmaxf(mx, __uint_as_float(v[i]));
-            }
-          }
-          const float m_tile = mx * p.scale_log2;  // -inf stays -inf
-          bool need = false;
-          if (m_ref == -INFINITY) {
+          if (need) {
+            alpha = fast_exp2(m_ref - m_tile);
             m_ref = m_tile;
-          } else if (m_tile > m_ref + kLazyRescale) {
-            need = true;
           }
-          if (__any_sync(0xffffffffu, need)) {
-            // O must hold every PV of this item up to key tile j-1 (j >= 1 here) before the rescale
-            const uint32_t gp = gs - 1;
-            ok = mbar_wait(&bar.pv_done[gp & 1], (gp >> 1) & 1, &abort_flag, p.err);
-            if (!ok) break;
-            tc_fence_after();
-            const float alpha = need ? fast_exp2(m_ref - m_tile) : 1.0f;
-            if (need) m_ref = m_tile;
-            l_run *= alpha;
-            for (int oc = 0; oc < kDHalf; oc += 32) {
-              uint32_t v[32];
-              tmem_ld32_nowait(tmem + lane_off + oc, v);
-              tmem_wait_ld_regs(v);
+          l_run *= alpha;
+          rescale_o(tmem + lane_off, alpha);
+        }
+        *scratch_alpha(scratch, j, r) = alpha;
+        // pass 2: P = exp2(s*scale*log2e - m_ref) as bf16, in place over S and into the scratch
+        const bool any_visible = m_ref != -INFINITY;
+        uint4* prow = scratch_p(scratch, j, r);
+        for (int c0 = 0; c0 < kt.n; c0 += 32) {
+          uint32_t v[32];
+          tmem_ld32_nowait(tS + c0, v);
+          tmem_wait_ld_regs(v);
+          uint32_t pk[16];
 #pragma unroll
-              for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * alpha);
-              tmem_st32(tmem + lane_off + oc, v);
-            }
-            tmem_wait_st();
+          for (int i = 0; i < 16; ++i) {
+            const int c = c0 + 2 * i;
+            float p0 = 0.0f, p1 = 0.0f;
+            if (any_visible && c >= lo && c < hi) p0 = fast_exp2(__uint_as_float(v[2 * i]) * p.scale_log2 - m_ref);
+            if (any_visible && c + 1 >= lo && c + 1 < hi)
+              p1 = fast_exp2(__uint_as_float(v[2 * i + 1]) * p.scale_log2 - m_ref);
+            l_run += p0 + p1;
+            pk[i] = pack_bf16x2(p0, p1);
           }
-          // pass 2: P = exp2(s*scale*log2e - m_ref) as bf16, in place over S
-          const bool any_visible = m_ref != -INFINITY;
-          for (int c0 = 0; c0 < kt.n; c0 += 32) {
-            uint32_t v[32];
-            tmem_ld32_nowait(tS + c0, v);
-            tmem_wait_ld_regs(v);
+          tmem_st16(tS + c0 / 2, pk);
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+            __stcg(prow + (c0 / 8 + u) * 128, make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]));
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&bar.p_ready[gs & 1]);
+      }
+      if (!ok) break;
+      const float inv_l = l_run > 0.0f ? 1.0f / l_run : 0.0f;
+      if (p.lse && row_valid)
+        p.lse[((size_t)ts.b * p.Lq + tok) * p.Hq + h] = (m_ref + __log2f(l_run)) * 0.69314718055994531f;
+      epilogue(ts, 0, inv_l);
+      if (!ok) break;
+      g += ts.J;
+      // ---- phase B: reload P_j into the S buffers, apply the same rescales
+      for (int j = 0; ok && j < ts.J; ++j) {
+        const uint32_t gs = g + j;
+        const KeyTile kt = ts.get(j);
+        uint4 pr[16];
+        float alpha;
+        load_p_row(pr, alpha, scratch, j, kt.n, r);
+        if (gs >= 2) {  // S buffer gs&1 is free once PV_{gs-2} has read its P
+          ok = mbar_wait(&bar.pv_done[gs & 1], ((gs >> 1) - 1) & 1, &abort_flag, p.err);
+          if (!ok) break;
+          tc_fence_after();
+        }
+        if (__any_sync(0xffffffffu, alpha != 1.0f)) {
+          const uint32_t gp = gs - 1;
+          ok = mbar_wait(&bar.pv_done[gp & 1], (gp >> 1) & 1, &abort_flag, p.err);
+          if (!ok) break;
+          tc_fence_after();
+          rescale_o(tmem + lane_off, alpha);
+        }
+        const uint32_t tS = tmem + lane_off + kDHalf + (gs & 1) * kKeyTile;
+#pragma unroll
+        for (int c0 = 0; c0 < kKeyTile; c0 += 32) {
+          if (c0 < kt.n) {
             uint32_t pk[16];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const int c = c0 + 2 * i;
-              float p0 = 0.0f, p1 = 0.0f;
-              if (any_visible && c >= lo && c < hi) p0 = fast_exp2(__uint_as_float(v[2 * i]) * p.scale_log2 - m_ref);
-              if (any_visible && c + 1 >= lo && c + 1 < hi)
-                p1 = fast_exp2(__uint_as_float(v[2 * i + 1]) * p.scale_log2 - m_ref);
-              l_run += p0 + p1;
-              pk[i] = pack_bf16x2(p0, p1);
+            for (int u = 0; u < 4; ++u) {
+              pk[4 * u] = pr[c0 / 8 + u].x;
+              pk[4 * u + 1] = pr[c0 / 8 + u].y;
+              pk[4 * u + 2] = pr[c0 / 8 + u].z;
+              pk[4 * u + 3] = pr[c0 / 8 + u].w;
             }
             tmem_st16(tS + c0 / 2, pk);
           }
-          tmem_wait_st();
-          tc_fence_before();
-          mbar_arrive(&bar.p_ready[gs & 1]);
         }
-        if (!ok) break;
-        // ---- epilogue of the item: O half -> bf16 -> global, then hand O back to the MMA warp
-        ok = mbar_wait(&bar.o_full, it & 1, &abort_flag, p.err);
-        if (!ok) break;
-        tc_fence_after();
-        const float inv_l = l_run > 0.0f ? 1.0f / l_run : 0.0f;
-        uint16_t* orow = p.O + ((size_t)((size_t)ts.b * p.Lq + tok) * p.Hq + h) * kD + half * kDHalf;
-        for (int oc = 0; oc < kDHalf; oc += 32) {
-          uint32_t v[32];
-          tmem_ld32_nowait(tmem + lane_off + oc, v);
-          tmem_wait_ld_regs(v);
-          if (row_valid) {
-            uint4 packed[4];
-            uint32_t* pw = reinterpret_cast<uint32_t*>(packed);
-#pragma unroll
-            for (int i = 0; i < 16; ++i)
-              pw[i] = pack_bf16x2(__uint_as_float(v[2 * i]) * inv_l, __uint_as_float(v[2 * i + 1]) * inv_l);
-            uint4* dst = reinterpret_cast<uint4*>(orow + oc);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) dst[i] = packed[i];
-          }
-        }
+        tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(&bar.o_empty);
-        if (half == 0 && p.lse && row_valid)
-          p.lse[((size_t)ts.b * p.Lq + tok) * p.Hq + h] = (m_ref + __log2f(l_run)) * 0.69314718055994531f;
-        g += ts.J;
+        mbar_arrive(&bar.p_ready[gs & 1]);
       }
+      if (!ok) break;
+      epilogue(ts, kDHalf, inv_l);
+      g += ts.J;
     }
+    if (store_issuer) bulk_wait_group0();
   }
 
   tc_fence_before();
@@ -418,11 +576,12 @@ __global__ void __launch_bounds__(kThreads, 1) hca_attn_kernel(const __grid_cons
   if (warp == 1) tmem_dealloc(tmem, 512);
 }
 
-bool make_map_4d(CUtensorMap* m, const void* base, int d, int heads, int rows, int B, int box_heads, int box_rows) {
+bool make_map_4d(CUtensorMap* m, const void* base, int d, int heads, int rows, int B, int box_cols, int box_heads,
+                 int box_rows, int swizzle) {
   const uint64_t dims[4] = {(uint64_t)d, (uint64_t)heads, (uint64_t)rows, (uint64_t)B};
   const uint64_t strides[3] = {(uint64_t)d * 2, (uint64_t)heads * d * 2, (uint64_t)rows * heads * d * 2};
-  const uint32_t box[4] = {64, (uint32_t)box_heads, (uint32_t)box_rows, 1};
-  return encode_tmap_bf16(m, 4, const_cast<void*>(base), dims, strides, box, true);
+  const uint32_t box[4] = {(uint32_t)box_cols, (uint32_t)box_heads, (uint32_t)box_rows, 1};
+  return encode_tmap_bf16_swizzle(m, 4, const_cast<void*>(base), dims, strides, box, swizzle);
 }
 
 int num_sms() {
@@ -436,13 +595,49 @@ int num_sms() {
   return cache[dev];
 }
 
+// Launch geometry shared by the workspace query and the launch: HCADSA_ERR_UNSUPPORTED for
+// shapes the kernel does not take, HCADSA_ERR_CUDA if the device cannot be queried.
+struct Geometry {
+  int g, TT, n_tiles, total_tiles, grid, J_max;
+  size_t scratch_bytes;
+};
+
+hcadsa_status geometry(Geometry* G, int B, int Lq, int q_offset, int Hq, int Hkv, int d, int blk, int W) {
+  if (B <= 0 || Lq <= 0 || q_offset < 0 || Hq <= 0 || Hkv <= 0 || blk <= 0 || W <= 0 || Hq % Hkv != 0)
+    return HCADSA_ERR_SHAPE;
+  const int g = Hq / Hkv;
+  if (d != kD || g > 128 || 128 % g != 0) return HCADSA_ERR_UNSUPPORTED;
+  const long long t_last = (long long)q_offset + Lq - 1;
+  if (t_last > 2147483647LL - 256) return HCADSA_ERR_UNSUPPORTED;
+  const int TT = 128 / g;
+  const long long n_tiles = (Lq + TT - 1) / TT;
+  const long long total = (long long)B * Hkv * n_tiles;
+  if (total > 2147483647LL) return HCADSA_ERR_UNSUPPORTED;
+  const long long nc_last = t_last - W + 1 > 0 ? (t_last - W + 1) / blk : 0;
+  // a tile's window band spans at most TT + W - 1 positions
+  const long long J_max = (nc_last + kKeyTile - 1) / kKeyTile + ((long long)TT + W - 2 + kKeyTile) / kKeyTile;
+  if (J_max > (1 << 20)) return HCADSA_ERR_UNSUPPORTED;
+  const int sms = num_sms();
+  if (sms <= 0) return HCADSA_ERR_CUDA;
+  G->g = g;
+  G->TT = TT;
+  G->n_tiles = (int)n_tiles;
+  G->total_tiles = (int)total;
+  G->grid = (int)(total < sms ? total : sms);
+  G->J_max = (int)J_max;
+  G->scratch_bytes = (size_t)G->grid * (size_t)J_max * kScratchTileBytes;
+  return HCADSA_OK;
+}
+
 }  // namespace
 }  // namespace hcadsa
 
 extern "C" size_t hca_attn_fwd_workspace_size(int B, int Lq, int q_offset, int Hq, int Hkv, int d, int n_c, int blk,
                                               int W) {
-  (void)B; (void)Lq; (void)q_offset; (void)Hq; (void)Hkv; (void)d; (void)n_c; (void)blk; (void)W;
-  return 0;
+  (void)n_c;
+  hcadsa::Geometry G;
+  if (hcadsa::geometry(&G, B, Lq, q_offset, Hq, Hkv, d, blk, W) != HCADSA_OK) return 0;
+  return G.scratch_bytes;
 }
 
 extern "C" hcadsa_status hca_attn_fwd(const hcadsa_bf16* Q, const hcadsa_bf16* Kc, const hcadsa_bf16* Vc, int n_c,
@@ -451,7 +646,6 @@ extern "C" hcadsa_status hca_attn_fwd(const hcadsa_bf16* Q, const hcadsa_bf16* K
                                       int d, int blk, int W, float scale, void* workspace, size_t workspace_bytes,
                                       hcadsa_stream stream) {
   using namespace hcadsa;
-  (void)workspace; (void)workspace_bytes;
   if (!Q || !Kw || !Vw || !O) return HCADSA_ERR_NULL;
   if (n_c > 0 && (!Kc || !Vc)) return HCADSA_ERR_NULL;
   if (B < 0 || Lq < 0 || q_offset < 0 || Hq <= 0 || Hkv <= 0 || n_c < 0 || n_w < 0 || win_start < 0 || blk <= 0 ||
@@ -470,19 +664,22 @@ extern "C" hcadsa_status hca_attn_fwd(const hcadsa_bf16* Q, const hcadsa_bf16* K
   const long long ws_first = t_first - W + 1 > 0 ? t_first - W + 1 : 0;
   const long long nc_last = t_last - W + 1 > 0 ? (t_last - W + 1) / blk : 0;
   if (ws_first < win_start || t_last - win_start >= n_w || nc_last > n_c) return HCADSA_ERR_SHAPE;
-  const int TT = 128 / g;
-  const long long n_tiles = (Lq + TT - 1) / TT;
-  if ((long long)B * Hkv * n_tiles > 2147483647LL) return HCADSA_ERR_UNSUPPORTED;
+  Geometry G;
+  const hcadsa_status gs = geometry(&G, B, Lq, q_offset, Hq, Hkv, d, blk, W);
+  if (gs != HCADSA_OK) return gs;
+  if (!workspace || workspace_bytes < G.scratch_bytes) return HCADSA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return HCADSA_ERR_ALIGN;
 
   Maps maps;
-  if (!make_map_4d(&maps.q, Q, kD, Hq, Lq, B, g, TT)) return HCADSA_ERR_CUDA;
+  if (!make_map_4d(&maps.q, Q, kD, Hq, Lq, B, 64, g, G.TT, 128)) return HCADSA_ERR_CUDA;
+  if (!make_map_4d(&maps.o, O, kD, Hq, Lq, B, kOutCols, g, G.TT, 64)) return HCADSA_ERR_CUDA;
   for (int small = 0; small < 2; ++small) {
     const int rows = small ? kSmallRows : 128;
-    if (!make_map_4d(&maps.kv[0][1][small], Kw, kD, Hkv, n_w, B, 1, rows)) return HCADSA_ERR_CUDA;
-    if (!make_map_4d(&maps.kv[1][1][small], Vw, kD, Hkv, n_w, B, 1, rows)) return HCADSA_ERR_CUDA;
+    if (!make_map_4d(&maps.kv[0][1][small], Kw, kD, Hkv, n_w, B, 64, 1, rows, 128)) return HCADSA_ERR_CUDA;
+    if (!make_map_4d(&maps.kv[1][1][small], Vw, kD, Hkv, n_w, B, 64, 1, rows, 128)) return HCADSA_ERR_CUDA;
     if (n_c > 0) {
-      if (!make_map_4d(&maps.kv[0][0][small], Kc, kD, Hkv, n_c, B, 1, rows)) return HCADSA_ERR_CUDA;
-      if (!make_map_4d(&maps.kv[1][0][small], Vc, kD, Hkv, n_c, B, 1, rows)) return HCADSA_ERR_CUDA;
+      if (!make_map_4d(&maps.kv[0][0][small], Kc, kD, Hkv, n_c, B, 64, 1, rows, 128)) return HCADSA_ERR_CUDA;
+      if (!make_map_4d(&maps.kv[1][0][small], Vc, kD, Hkv, n_c, B, 64, 1, rows, 128)) return HCADSA_ERR_CUDA;
     } else {  // no query sees an entry: these maps are never read
       maps.kv[0][0][small] = maps.kv[0][1][small];
       maps.kv[1][0][small] = maps.kv[1][1][small];
@@ -494,22 +691,20 @@ extern "C" hcadsa_status hca_attn_fwd(const hcadsa_bf16* Q, const hcadsa_bf16* K
   p.Hq = Hq;
   p.Hkv = Hkv;
   p.g = g;
-  p.TT = TT;
+  p.TT = G.TT;
   p.n_c = n_c;
   p.win_start = win_start;
   p.W = W;
   p.blk = blk;
-  p.n_tiles = (int)n_tiles;
-  p.total_tiles = (int)((long long)B * Hkv * n_tiles);
+  p.n_tiles = G.n_tiles;
+  p.total_tiles = G.total_tiles;
+  p.J_max = G.J_max;
   p.scale_log2 = scale * 1.4426950408889634f;
-  p.O = O;
   p.lse = lse;
+  p.scratch = static_cast<uint8_t*>(workspace);
   p.err = device_error_ptr();
   if (cudaFuncSetAttribute(hca_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) != cudaSuccess)
     return HCADSA_ERR_CUDA;
-  const int sms = num_sms();
-  if (sms <= 0) return HCADSA_ERR_CUDA;
-  const int grid = p.total_tiles < sms ? p.total_tiles : sms;
-  hca_attn_kernel<<<grid, kThreads, kSmemBytes, as_stream(stream)>>>(maps, p);
+  hca_attn_kernel<<<G.grid, kThreads, kSmemBytes, as_stream(stream)>>>(maps, p);
   return launch_status();
 }

@@ -24,6 +24,10 @@ inline cudaStream_t as_stream(hcadsa_stream s) { return reinterpret_cast<cudaStr
 bool encode_tmap_bf16(CUtensorMap* map, int rank, void* base, const uint64_t* dims,
                       const uint64_t* strides_bytes, const uint32_t* box, bool swizzle128);
 
+// Same, with the swizzle span given in bytes: 0 (none), 32, 64 or 128.
+bool encode_tmap_bf16_swizzle(CUtensorMap* map, int rank, void* base, const uint64_t* dims,
+                              const uint64_t* strides_bytes, const uint32_t* box, int swizzle_bytes);
+
 // Records the message of a failed CUDA call for hcadsa_last_error_string().
 void record_cuda_error(cudaError_t e);
 

@@ -116,6 +116,49 @@ def test_hca_stress(hd, cfg, W):
     np.testing.assert_allclose(lse.cpu().numpy(), ref_lse, atol=2e-2, rtol=0)
 
 
+def test_hca_forced_rescales(hd):
+    """Keys whose scale grows along the sequence: later key tiles raise the running max by far
+    more than the lazy-rescale threshold, so O is rescaled in both halves of d_v."""
+    cfg = synth.HcaConfig("ramp_L1500_hq16", B=1, L=1500, Hq=16, Hkv=1, sigma=1.0)
+    inp = synth.hca_inputs(cfg)
+    ramp = 1.0 + 6.0 * torch.arange(cfg.L, dtype=torch.float32) / cfg.L
+    K = (inp["K"].float() * ramp.view(1, -1, 1, 1)).to(torch.bfloat16)
+    Kd, Vd, Qd = K.cuda(), inp["V"].cuda(), inp["Q"].cuda()
+    Kc, Vc = hd.hca_compress_kv(Kd, Vd, inp["w"].cuda(), cfg.blk)
+    O, lse = hd.hca_attn_fwd(Qd, Kc, Vc, Kd, Vd, return_lse=True)
+    O2 = hd.hca_attn_fwd(Qd, Kc, Vc, Kd, Vd)
+    no_device_error(hd)
+    assert torch.equal(O, O2)  # deterministic: no atomics, fixed accumulation order
+    w = inp["w"].numpy()
+    Kc_o = oracle.hca_compress(bits(K), w, cfg.blk)
+    Vc_o = oracle.hca_compress(bits(inp["V"]), w, cfg.blk)
+    ref, ref_lse = oracle.hca_attn(bits(inp["Q"]), Kc_o, Vc_o, bits(K), bits(inp["V"]), with_lse=True)
+    print(check_attn(O.reshape(cfg.L, cfg.Hq, cfg.d), ref, "hca forced rescales"))
+    np.testing.assert_allclose(lse.reshape(cfg.L, cfg.Hq).cpu().numpy(), ref_lse, atol=2e-2, rtol=0)
+
+
+def test_hca_workspace_size_and_check(hd):
+    """The workspace holds one probability-tile slot per key tile for each resident CTA; a
+    short workspace is rejected before launch."""
+    lib = hd.lib()
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    L, Hq = 32768, 16
+    TT = 128 // Hq
+    nc_last = (L - 1 - 128 + 1) // 128
+    J_max = -(-nc_last // 128) + (TT + 128 - 2 + 128) // 128
+    want = min(L // TT, sms) * J_max * (128 * 128 * 2 + 128 * 4)
+    assert lib.hca_attn_fwd_workspace_size(1, L, 0, Hq, 1, 512, L // 128, 128, 128) == want
+    L = 1024
+    Q = torch.zeros(1, L, Hq, 512, dtype=torch.bfloat16, device="cuda")
+    K = torch.zeros(1, L, 1, 512, dtype=torch.bfloat16, device="cuda")
+    Kc = torch.zeros(1, L // 128, 1, 512, dtype=torch.bfloat16, device="cuda")
+    need = lib.hca_attn_fwd_workspace_size(1, L, 0, Hq, 1, 512, L // 128, 128, 128)
+    assert need > 0
+    with pytest.raises(hd.HcaDsaError) as e:
+        hd.hca_attn_fwd(Q, Kc, Kc, K, K, workspace=torch.empty(need - 16, dtype=torch.uint8, device="cuda"))
+    assert e.value.status == -5
+
+
 def _sample_rows(L, B=1, extra=()):
     toks = {0, 1, 2, 126, 127, 128, 129, 254, 255, 256, 257, 383, 384, 1000, 4095, 4096, L // 2, L - 2, L - 1}
     toks |= set(extra)
