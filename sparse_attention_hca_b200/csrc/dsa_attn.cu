@@ -15,11 +15,13 @@
 //     overlaps the next token's MMAs; S^T double-buffered per tile [256,320) / [320,384).
 //   * Warps 0-5 gather K and V rows with cp.async: one warp instruction moves one whole
 //     512-byte row (lane l -> 16 bytes of 64-column chunk l/8), written 128B-swizzled into a
-//     ring of 8 x 16 KB chunk slots; a tile's K (or V) occupies 4 consecutive slots, loaded in
-//     exactly the order warp 4 consumes them: K_0, K_1, V_0, K_2, V_1, ...  Completion is
-//     tracked with cp.async.mbarrier.arrive.noinc; the MMA thread issues a proxy fence after
-//     each wait so the tensor core sees the generic-proxy writes.  (Measured on B200: this
-//     reaches ~105 GB/s per SM from L2, TMA tile::gather4 of 4 x 128 B rows ~16 GB/s.)
+//     ring of two 64 KB groups (4 chunk slots each); a group holds one K or one V tile, loaded
+//     in exactly the order warp 6 consumes them: K_0, K_1, V_0, K_2, V_1, ...  Completion is
+//     tracked with cp.async.mbarrier.arrive.noinc, one arrival per producer thread per tile, so
+//     the MMA thread waits once per tile (a wait costs the issuing thread a few hundred cycles,
+//     which only a whole tile of MMAs hides) and issues a proxy fence after it so the tensor
+//     core sees the generic-proxy writes.  (Measured on B200: this reaches ~105 GB/s per SM
+//     from L2, TMA tile::gather4 of 4 x 128 B rows ~16 GB/s.)
 //     Q (32 KB, TMA) is reloaded per token once the previous token's last S^T MMA is done.
 //   * Warp 6, lane 0 issues every MMA.  Warps 7-10: softmax (one thread per key = TMEM lane,
 //     64 head scores each; per-head row sums reduced across the warp every tile).  The first tile of a token sets the per-head reference max by a
@@ -47,7 +49,7 @@ constexpr int kD = 256;
 constexpr int kH = 64;
 constexpr int kKeyTile = 128;
 constexpr int kChunkBytes = 128 * 128;     // 128 rows x 64 bf16
-constexpr int kRingSlots = 8;  // even: a V pair (2hv, 2hv+1) never wraps
+constexpr int kRingSlots = 8;  // two groups of 4 slots: one K tile or one V tile per group
 constexpr int kQChunkBytes = kH * 128;     // 64 heads x 64 bf16
 constexpr int kQBytes = 4 * kQChunkBytes;  // 32 KB
 constexpr int kPBytes = kKeyTile * 128;    // 128 keys x 64 heads bf16
@@ -77,8 +79,8 @@ struct Params {
 
 struct __align__(8) Barriers {
   uint64_t q_full, q_empty;
-  uint64_t full[kRingSlots];
-  uint64_t empty[kRingSlots];
+  uint64_t full[2];   // ring group g holds a whole K or V tile (192 producer-thread arrivals)
+  uint64_t empty[2];  // the MMAs that read group g have completed
   uint64_t s_full[2];
   uint64_t p_ready[2];
   uint64_t pv_done;
@@ -191,7 +193,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     mbar_init(&bar.q_full, 1);
     mbar_init(&bar.q_empty, 1);
-    for (int s = 0; s < kRingSlots; ++s) {
+    for (int s = 0; s < 2; ++s) {
       mbar_init(&bar.full[s], kProducerWarps * 32);
       mbar_init(&bar.empty[s], 1);
     }
@@ -224,7 +226,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t ring = smem_u32(sRing);
     const uint16_t* Kg = p.K;
     const uint16_t* Vg = p.V;
-    uint32_t q = 0;  // chunks issued so far: slot q % kRingSlots, phase (q / kRingSlots) & 1
+    uint32_t u = 0;  // K/V tiles issued so far: ring group u & 1, phase (u >> 1) & 1
     int it = 0;  // tokens with work so far
     bool ok = true;
     const int chunk = lane >> 3, piece = lane & 7;
@@ -262,22 +264,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (is_k ? step >= J : step < 1) continue;
           const int ra = is_k ? ra_cur : ra_prev, rb = is_k ? rb_cur : rb_prev;
           const uint16_t* base = (is_k ? Kg : Vg) + kv_row0 * kD + lane * 8;
-          for (int c = 0; c < 4 && ok; ++c) {
-            const uint32_t qc = q + c;
-            ok = mbar_wait(&bar.empty[qc % kRingSlots], ((qc / kRingSlots) & 1) ^ 1, &abort_flag, p.err);
-          }
-          ok = __all_sync(0xffffffffu, ok);
+          ok = __all_sync(0xffffffffu, mbar_wait(&bar.empty[u & 1], ((u >> 1) & 1) ^ 1, &abort_flag, p.err));
           if (!ok) break;
-          const uint32_t dst0 = ring + ((q + chunk) % kRingSlots) * kChunkBytes;
+          const uint32_t dst0 = ring + ((u & 1) * 4 + chunk) * kChunkBytes;
 #pragma unroll 4
           for (int i = 0; i < n_rows_w; ++i) {
             const int trow = warp + kProducerWarps * i;  // row of the tile
             const int src_row = __shfl_sync(0xffffffffu, i < 32 ? ra : rb, i & 31);
             cp_async16(dst0 + trow * 128 + ((piece ^ (trow & 7)) << 4), base + (size_t)src_row * kD);
           }
-#pragma unroll
-          for (int c = 0; c < 4; ++c) cp_async_arrive_noinc(&bar.full[(q + c) % kRingSlots]);
-          q += 4;
+          cp_async_arrive_noinc(&bar.full[u & 1]);
+          ++u;
           if (is_k && step == 0 && warp == 0) {
             // Q of this token (after its first K tile is in flight), once the previous token's
             // last S^T MMA no longer reads the buffer
@@ -298,7 +295,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     cp_async_wait_all();
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
-    uint32_t q = 0;  // chunks consumed so far (same sequence as the producers)
+    uint32_t u = 0;  // K/V tiles consumed so far (same sequence as the producers)
     int it = 0;
     uint32_t g = 0;  // global tile counter
     bool ok = true;
@@ -323,22 +320,24 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (step < J) {
             const uint32_t gs = g + step;
             const uint32_t tS = tmem + kTmemS + (gs & 1) * kH;
-            for (int c = 0; c < 4 && ok; ++c) {
-              const uint32_t slot = q % kRingSlots;
-              ok = mbar_wait(&bar.full[slot], (q / kRingSlots) & 1, &abort_flag, p.err);
-              if (!ok) break;
-              fence_proxy_async_smem();  // cp.async (generic proxy) writes -> tensor core reads
-              tc_fence_after();
-#pragma unroll
-              for (int kk = 0; kk < 4; ++kk) {
-                const uint64_t da = smem_desc_sw128(sRa + slot * kChunkBytes + kk * 32, 16, 1024);
-                const uint64_t db = smem_desc_sw128(sQa + c * kQChunkBytes + kk * 32, 16, 1024);
-                mma_ss(tS, da, db, idesc_s, (c | kk) != 0);
-              }
-              mma_commit(&bar.empty[slot]);
-              ++q;
-            }
+            // one wait per K tile: every producer thread arrives once all of its row copies of
+            // the tile (all 4 chunks) have landed
+            ok = mbar_wait(&bar.full[u & 1], (u >> 1) & 1, &abort_flag, p.err);
             if (!ok) break;
+            fence_proxy_async_smem();  // cp.async (generic proxy) writes -> tensor core reads
+            tc_fence_after();
+            {
+              const uint64_t da0 = smem_desc_sw128(sRa + (u & 1) * 4 * kChunkBytes, 16, 1024);
+              const uint64_t db0 = smem_desc_sw128(sQa, 16, 1024);
+#pragma unroll
+              for (int c = 0; c < 4; ++c)
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)  // descriptor start address field is in 16-byte units
+                  mma_ss(tS, da0 + (uint64_t)((c * kChunkBytes + kk * 32) >> 4),
+                         db0 + (uint64_t)((c * kQChunkBytes + kk * 32) >> 4), idesc_s, (c | kk) != 0);
+            }
+            mma_commit(&bar.empty[u & 1]);
+            ++u;
             mma_commit(&bar.s_full[gs & 1]);
             if (step == J - 1) mma_commit(&bar.q_empty);
           }
@@ -353,33 +352,31 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!ok) break;
             tc_fence_after();
             const uint32_t pbase = sPa + (gj & 1) * kPBytes;
-            for (int hv = 0; hv < 2 && ok; ++hv) {
-              // V chunks 2hv, 2hv+1 sit in consecutive slots (q is even here and the ring size is
-              // even, so the pair never wraps)
-              const uint32_t slot = q % kRingSlots;
-              const uint32_t phase = (q / kRingSlots) & 1;
-              ok = mbar_wait(&bar.full[slot], phase, &abort_flag, p.err) &&
-                   mbar_wait(&bar.full[slot + 1], phase, &abort_flag, p.err);
-              if (!ok) break;
-              fence_proxy_async_smem();
-              tc_fence_after();
-              for (int kk = 0; kk < kKeyTile / 16; ++kk) {
-                const uint64_t da = smem_desc_sw128(sRa + slot * kChunkBytes + kk * 2048, kChunkBytes, 1024);
-                const uint64_t db = smem_desc_sw128(pbase + kk * 2048, kPBytes, 1024);
-                mma_ss(tmem + ob * 128 + hv * kH, da, db, idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
-              }
-              mma_commit(&bar.empty[slot]);
-              mma_commit(&bar.empty[slot + 1]);
-              q += 2;
-            }
+            ok = mbar_wait(&bar.full[u & 1], (u >> 1) & 1, &abort_flag, p.err);  // the whole V tile
             if (!ok) break;
+            fence_proxy_async_smem();
+            tc_fence_after();
+            {
+              // V^T chunk pair (2hv, 2hv+1): M = 128 d_v rows, the pair's slots are LBO apart
+              const uint64_t da0 = smem_desc_sw128(sRa + (u & 1) * 4 * kChunkBytes, kChunkBytes, 1024);
+              const uint64_t db0 = smem_desc_sw128(pbase, kPBytes, 1024);
+              const uint32_t acc0 = j > 0 ? 1u : 0u;
+#pragma unroll
+              for (int hv = 0; hv < 2; ++hv)
+#pragma unroll
+                for (int kk = 0; kk < kKeyTile / 16; ++kk)
+                  mma_ss(tmem + ob * 128 + hv * kH, da0 + (uint64_t)((hv * 2 * kChunkBytes + kk * 2048) >> 4),
+                         db0 + (uint64_t)((kk * 2048) >> 4), idesc_o, kk > 0 ? 1u : acc0);
+            }
+            mma_commit(&bar.empty[u & 1]);
+            ++u;
             mma_commit(&bar.pv_done);
             if (j == J - 1) mma_commit(&bar.o_full[ob]);
           }
         }
       }
       ok = __shfl_sync(0xffffffffu, ok, 0);
-      q = __shfl_sync(0xffffffffu, q, 0);
+      u = __shfl_sync(0xffffffffu, u, 0);
       g += J;
       ++it;
     }

@@ -19,14 +19,16 @@
 //     TMEM and runs only O[:, 256:512] += P_j V_j[:, 256:512] with the same rescales, so the
 //     second half costs no QK^T and no exponentials, and Q's buffer is free to take the
 //     next tile's Q while phase B runs.
-//   * warp 0: TMA producer (Q per tile; K chunks and V chunks through a 5-slot ring of 16 KB
-//     stages, in exactly the order the MMA warp consumes them; key tiles of at most 32 keys
-//     use 32-row boxes); warp 1: TMEM allocation and the single MMA-issuing thread;
+//   * warp 0: TMA producer (Q per tile; K and V in units of 128 d-columns (two 16 KB chunks)
+//     through a ring of two such groups, in exactly the order the MMA warp consumes them; key
+//     tiles of at most 32 keys use 32-row boxes); warp 1: TMEM allocation and the single
+//     MMA-issuing thread.  One barrier wait per group: a wait costs the issuing thread a few
+//     hundred cycles, which only ~500 cycles of queued MMA work (8 MMAs of N = 128) hide;
 //     warps 2-5: softmax, one thread per row (TMEM lane), and the epilogues, which stage O
 //     through shared memory (64-byte swizzle, two 8 KB buffers) into TMA tensor stores.
 //   * S_j accumulates over eight 64-wide d chunks (SS MMA, K-major operands, 128B swizzle).
 //     P_j is written in place over S_j in TMEM and PV runs as a TS MMA (A = P from TMEM,
-//     B = V chunk, MN-major).  Online softmax with a lazy rescale: the reference max only
+//     B = V, MN-major, N = 128 over the group's two chunks).  Online softmax with a lazy rescale: the reference max only
 //     moves when the tile max exceeds it by 2^8.
 //   * Key tiles: compressed entries [0, n_c(t_last)) in tiles of 128, then the window
 //     band [max(0, t_first-W+1), t_last] in tiles of 128; per-row visibility is one
@@ -51,7 +53,7 @@ constexpr int kD = 512;
 constexpr int kDHalf = 256;
 constexpr int kKeyTile = 128;
 constexpr int kSmallRows = 32;  // TMA box height for key tiles of at most 32 keys
-constexpr int kStages = 5;
+constexpr int kGroups = 2;  // ring: two groups of two 16 KB chunk slots (128 d-columns of a tile)
 constexpr int kChunkBytes = 128 * 128;  // 128 rows x 64 bf16
 constexpr int kSmallChunkBytes = kSmallRows * 128;
 constexpr int kQChunks = kD / 64;      // 8
@@ -59,7 +61,8 @@ constexpr int kVChunks = kDHalf / 64;  // 4
 constexpr int kQBytes = kQChunks * kChunkBytes;
 constexpr int kOutCols = 32;                  // O columns per staged store
 constexpr int kOutBufBytes = 128 * kOutCols * 2;  // 8 KB
-constexpr int kSmemBytes = kQBytes + kStages * kChunkBytes + 2 * kOutBufBytes + 1024;
+constexpr int kGroupBytes = 2 * kChunkBytes;
+constexpr int kSmemBytes = kQBytes + kGroups * kGroupBytes + 2 * kOutBufBytes + 1024;
 constexpr int kThreads = 192;
 constexpr float kLazyRescale = 8.0f;  // log2 units
 // per-CTA scratch per key tile: P (128 rows x 128 keys bf16) + one fp32 rescale factor per row
@@ -141,8 +144,8 @@ struct TileSet {
 
 struct __align__(8) Barriers {
   uint64_t q_full, q_empty;
-  uint64_t full[kStages];
-  uint64_t empty[kStages];
+  uint64_t full[kGroups];   // both chunks of a ring group landed
+  uint64_t empty[kGroups];  // the MMAs that read the group have completed
   uint64_t s_full[2];
   uint64_t p_ready[2];
   uint64_t pv_done[2];  // the PV that read P from S buffer i has completed
@@ -187,7 +190,7 @@ __global__ void __launch_bounds__(kThreads, 1) hca_attn_kernel(const __grid_cons
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;
   uint8_t* sRing = smem + kQBytes;
-  uint8_t* sOut = sRing + kStages * kChunkBytes;
+  uint8_t* sOut = sRing + kGroups * kGroupBytes;
   __shared__ Barriers bar;
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_flag;
@@ -196,7 +199,7 @@ __global__ void __launch_bounds__(kThreads, 1) hca_attn_kernel(const __grid_cons
   if (threadIdx.x == 0) {
     mbar_init(&bar.q_full, 1);
     mbar_init(&bar.q_empty, 1);
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < kGroups; ++s) {
       mbar_init(&bar.full[s], 1);
       mbar_init(&bar.empty[s], 1);
     }
@@ -223,23 +226,26 @@ __global__ void __launch_bounds__(kThreads, 1) hca_attn_kernel(const __grid_cons
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       tma_prefetch_desc(&maps.q);
-      uint32_t q = 0;  // ring chunks issued: slot q % kStages, phase (q / kStages) & 1
+      uint32_t u = 0;  // ring groups filled: group u & 1, phase (u >> 1) & 1
       bool ok = true;
-      auto load_chunk = [&](const CUtensorMap* m, bool small, int col, int hk, int row0, int b) {
-        const uint32_t slot = q % kStages;
-        ok = mbar_wait(&bar.empty[slot], ((q / kStages) & 1) ^ 1, &abort_flag, p.err);
+      // two 64-column chunks (columns col .. col+127 of a key tile) into the next ring group
+      auto load_unit = [&](const CUtensorMap* m, bool small, int col, int hk, int row0, int b) {
+        const uint32_t grp = u & 1;
+        ok = mbar_wait(&bar.empty[grp], ((u >> 1) & 1) ^ 1, &abort_flag, p.err);
         if (ok) {
-          mbar_arrive_expect_tx(&bar.full[slot], small ? kSmallChunkBytes : kChunkBytes);
-          tma_load_4d(sRing + slot * kChunkBytes, m, &bar.full[slot], col, hk, row0, b);
+          mbar_arrive_expect_tx(&bar.full[grp], 2 * (small ? kSmallChunkBytes : kChunkBytes));
+          uint8_t* dst = sRing + grp * kGroupBytes;
+          tma_load_4d(dst, m, &bar.full[grp], col, hk, row0, b);
+          tma_load_4d(dst + kChunkBytes, m, &bar.full[grp], col + 64, hk, row0, b);
         }
-        ++q;
+        ++u;
       };
       auto load_v = [&](const TileSet& ts, int j, int col0) {
         const KeyTile kt = ts.get(j);
         const int small = kt.n <= kSmallRows ? 1 : 0;
         const int row0 = kt.window ? kt.start - p.win_start : kt.start;
-        for (int c = 0; ok && c < kVChunks; ++c)
-          load_chunk(&maps.kv[1][kt.window][small], small, col0 + c * 64, ts.hk, row0, ts.b);
+        for (int c = 0; ok && c < kVChunks; c += 2)
+          load_unit(&maps.kv[1][kt.window][small], small, col0 + c * 64, ts.hk, row0, ts.b);
       };
       if (blockIdx.x < p.total_tiles) {
         TileSet t0;
@@ -259,8 +265,8 @@ __global__ void __launch_bounds__(kThreads, 1) hca_attn_kernel(const __grid_cons
             const KeyTile kt = ts.get(step);
             const int small = kt.n <= kSmallRows ? 1 : 0;
             const int row0 = kt.window ? kt.start - p.win_start : kt.start;
-            for (int c = 0; ok && c < kQChunks; ++c)
-              load_chunk(&maps.kv[0][kt.window][small], small, c * 64, ts.hk, row0, ts.b);
+            for (int c = 0; ok && c < kQChunks; c += 2)
+              load_unit(&maps.kv[0][kt.window][small], small, c * 64, ts.hk, row0, ts.b);
           }
           if (ok && step >= 1) load_v(ts, step - 1, 0);
         }
@@ -284,25 +290,32 @@ __global__ void __launch_bounds__(kThreads, 1) hca_attn_kernel(const __grid_cons
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t sQa = smem_u32(sQ), sRa = smem_u32(sRing);
-      uint32_t q = 0;       // ring chunks consumed
+      uint32_t u = 0;       // ring groups consumed
       uint32_t tcount = 0;  // row tiles
       uint32_t g = 0;       // key tiles of all earlier phases
       uint32_t it = 0;      // O halves
       bool ok = true;
-      const uint32_t idesc_pv = idesc_bf16_f32(128, 64, false, true);
-      // PV of key tile j (global counter gj) into the O half; V chunks from the ring
+      // N = 128: one PV MMA covers both 64-column chunks of a ring group (LBO = one slot)
+      const uint32_t idesc_pv = idesc_bf16_f32(128, 128, false, true);
+      // descriptors of the ring groups and of Q; the start-address field counts 16-byte units
+      const uint64_t dq0 = smem_desc_sw128(sQa, 16, 1024);
+      const uint64_t dk0 = smem_desc_sw128(sRa, 16, 1024);
+      const uint64_t dv0 = smem_desc_sw128(sRa, kChunkBytes, 1024);
+      constexpr uint64_t kGroupDesc = kGroupBytes >> 4;  // group offset in descriptor units
+      // PV of key tile j (global counter gj) into the O half; V from two ring groups
       auto pv = [&](const KeyTile& kt, int j, uint32_t gj) {
         const uint32_t tP = tmem + kDHalf + (gj & 1) * kKeyTile;
-        for (int c = 0; ok && c < kVChunks; ++c, ++q) {
-          const uint32_t slot = q % kStages;
-          ok = mbar_wait(&bar.full[slot], (q / kStages) & 1, &abort_flag, p.err);
+        const int nk = kt.n / 16;
+        for (int vu = 0; ok && vu < kVChunks / 2; ++vu, ++u) {
+          const uint32_t grp = u & 1;
+          ok = mbar_wait(&bar.full[grp], (u >> 1) & 1, &abort_flag, p.err);
           if (!ok) break;
           tc_fence_after();
-          for (int kk = 0; kk < kt.n / 16; ++kk) {
-            const uint64_t db = smem_desc_sw128(sRa + slot * kChunkBytes + kk * 2048, kChunkBytes, 1024);
-            mma_ts(tmem + c * 64, tP + kk * 8, db, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
-          }
-          mma_commit(&bar.empty[slot]);
+          const uint64_t db = dv0 + grp * kGroupDesc;
+          for (int kk = 0; kk < nk; ++kk)
+            mma_ts(tmem + vu * 128, tP + kk * 8, db + (uint64_t)(kk * (2048 >> 4)), idesc_pv,
+                   (j > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(&bar.empty[grp]);
         }
       };
       for (int T = blockIdx.x; ok && T < p.total_tiles; T += gridDim.x, ++tcount) {
@@ -327,18 +340,20 @@ __global__ void __launch_bounds__(kThreads, 1) hca_attn_kernel(const __grid_cons
               if (!ok) break;
               tc_fence_after();
             }
-            for (int c = 0; ok && c < kQChunks; ++c, ++q) {
-              const uint32_t slot = q % kStages;
-              ok = mbar_wait(&bar.full[slot], (q / kStages) & 1, &abort_flag, p.err);
+            for (int c = 0; ok && c < kQChunks; c += 2, ++u) {
+              const uint32_t grp = u & 1;
+              ok = mbar_wait(&bar.full[grp], (u >> 1) & 1, &abort_flag, p.err);
               if (!ok) break;
               tc_fence_after();
+              const uint64_t da = dq0 + (uint64_t)((c * kChunkBytes) >> 4);
+              const uint64_t db = dk0 + grp * kGroupDesc;
 #pragma unroll
-              for (int k = 0; k < 4; ++k) {
-                const uint64_t da = smem_desc_sw128(sQa + c * kChunkBytes + k * 32, 16, 1024);
-                const uint64_t db = smem_desc_sw128(sRa + slot * kChunkBytes + k * 32, 16, 1024);
-                mma_ss(tS, da, db, idesc, (c | k) != 0);
-              }
-              mma_commit(&bar.empty[slot]);
+              for (int cc = 0; cc < 2; ++cc)
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                  mma_ss(tS, da + (uint64_t)((cc * kChunkBytes + k * 32) >> 4),
+                         db + (uint64_t)((cc * kChunkBytes + k * 32) >> 4), idesc, (c | cc | k) != 0);
+              mma_commit(&bar.empty[grp]);
             }
             if (!ok) break;
             mma_commit(&bar.s_full[gs & 1]);
