@@ -150,7 +150,7 @@ struct __align__(8) Barriers {
   uint64_t p_ready[2];
   uint64_t pv_done[2];  // the PV that read P from S buffer i has completed
   uint64_t o_full;      // every PV of the current O half has completed
-  uint64_t o_empty;     // the epilogue has read O
+  uint64_t o_empty[2];  // the epilogue has read O columns [0,128) / [128,256)
 };
 
 // One thread's row of P_j in the scratch: key tile j owns kScratchTileBytes; inside it the
@@ -209,7 +209,8 @@ __global__ void __launch_bounds__(kThreads, 1) hca_attn_kernel(const __grid_cons
       mbar_init(&bar.pv_done[s], 1);
     }
     mbar_init(&bar.o_full, 1);
-    mbar_init(&bar.o_empty, 128);
+    mbar_init(&bar.o_empty[0], 128);
+    mbar_init(&bar.o_empty[1], 128);
     abort_flag = 0;
     fence_mbarrier_init();
   }
@@ -307,6 +308,10 @@ __global__ void __launch_bounds__(kThreads, 1) hca_attn_kernel(const __grid_cons
         const uint32_t tP = tmem + kDHalf + (gj & 1) * kKeyTile;
         const int nk = kt.n / 16;
         for (int vu = 0; ok && vu < kVChunks / 2; ++vu, ++u) {
+          if (j == 0) {  // the previous O half's epilogue must have read these 128 columns
+            ok = mbar_wait(&bar.o_empty[vu], (it & 1) ^ 1, &abort_flag, p.err);
+            if (!ok) break;
+          }
           const uint32_t grp = u & 1;
           ok = mbar_wait(&bar.full[grp], (u >> 1) & 1, &abort_flag, p.err);
           if (!ok) break;
@@ -362,10 +367,6 @@ __global__ void __launch_bounds__(kThreads, 1) hca_attn_kernel(const __grid_cons
           if (step >= 1) {
             const int j = step - 1;
             const uint32_t gj = g + j;
-            if (j == 0) {  // the previous O half's epilogue must have read O
-              ok = mbar_wait(&bar.o_empty, (it & 1) ^ 1, &abort_flag, p.err);
-              if (!ok) break;
-            }
             ok = mbar_wait(&bar.p_ready[gj & 1], (gj >> 1) & 1, &abort_flag, p.err);
             if (!ok) break;
             tc_fence_after();
@@ -381,10 +382,6 @@ __global__ void __launch_bounds__(kThreads, 1) hca_attn_kernel(const __grid_cons
         // ---- phase B: PV only (second half of d_v), P reloaded into TMEM by the softmax warps
         for (int j = 0; ok && j < ts.J; ++j) {
           const uint32_t gj = g + j;
-          if (j == 0) {
-            ok = mbar_wait(&bar.o_empty, (it & 1) ^ 1, &abort_flag, p.err);
-            if (!ok) break;
-          }
           ok = mbar_wait(&bar.p_ready[gj & 1], (gj >> 1) & 1, &abort_flag, p.err);
           if (!ok) break;
           tc_fence_after();
@@ -411,34 +408,43 @@ __global__ void __launch_bounds__(kThreads, 1) hca_attn_kernel(const __grid_cons
     bool ok = true;
 
     // O half (TMEM) -> bf16 -> two 8 KB staging buffers -> TMA tensor store; then release O
+    // O half (TMEM) -> normalised bf16 in registers, 128 columns at a time, each 128 columns
+    // released to the MMA warp as soon as they are read -> two 8 KB staging buffers -> TMA
+    // tensor stores
     auto epilogue = [&](const TileSet& ts, int col0, float inv_l) {
       ok = mbar_wait(&bar.o_full, it & 1, &abort_flag, p.err);
       if (!ok) return;
       tc_fence_after();
-      for (int oc = 0; oc < kDHalf; oc += kOutCols, ++ec) {
-        uint32_t v[32];
-        tmem_ld32_nowait(tmem + lane_off + oc, v);
-        tmem_wait_ld_regs(v);
-        if (oc + kOutCols == kDHalf) {  // last read of O
-          tc_fence_before();
-          mbar_arrive(&bar.o_empty);
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        uint32_t ob[64];
+#pragma unroll
+        for (int oc = 0; oc < 128; oc += 32) {
+          uint32_t v[32];
+          tmem_ld32_nowait(tmem + lane_off + hh * 128 + oc, v);
+          tmem_wait_ld_regs(v);
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            ob[oc / 2 + i] = pack_bf16x2(__uint_as_float(v[2 * i]) * inv_l, __uint_as_float(v[2 * i + 1]) * inv_l);
         }
-        uint4 packed[4];
-        uint32_t* pw = reinterpret_cast<uint32_t*>(packed);
+        tc_fence_before();
+        mbar_arrive(&bar.o_empty[hh]);
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
-          pw[i] = pack_bf16x2(__uint_as_float(v[2 * i]) * inv_l, __uint_as_float(v[2 * i + 1]) * inv_l);
-        uint8_t* buf = sOut + (ec & 1) * kOutBufBytes;
-        if (store_issuer && ec >= 2) bulk_wait_group_read1();  // the store from this buffer has read it
-        softmax_bar_sync();
+        for (int oc = 0; oc < 128; oc += kOutCols) {
+          uint8_t* buf = sOut + (ec & 1) * kOutBufBytes;
+          if (store_issuer && ec >= 2) bulk_wait_group_read1();  // the store from this buffer has read it
+          softmax_bar_sync();
 #pragma unroll
-        for (int i = 0; i < 4; ++i)  // 64-byte swizzle: 16-byte unit i of row r at unit i ^ ((r >> 1) & 3)
-          *reinterpret_cast<uint4*>(buf + r * 64 + ((i ^ ((r >> 1) & 3)) * 16)) = packed[i];
-        fence_proxy_async_smem();
-        softmax_bar_sync();
-        if (store_issuer) {
-          tma_store_4d(&maps.o, buf, col0 + oc, ts.hk * p.g, ts.tok0, ts.b);
-          bulk_commit_group();
+          for (int i = 0; i < 4; ++i)  // 64-byte swizzle: 16-byte unit i of row r at unit i ^ ((r >> 1) & 3)
+            *reinterpret_cast<uint4*>(buf + r * 64 + ((i ^ ((r >> 1) & 3)) * 16)) =
+                make_uint4(ob[oc / 2 + 4 * i], ob[oc / 2 + 4 * i + 1], ob[oc / 2 + 4 * i + 2], ob[oc / 2 + 4 * i + 3]);
+          fence_proxy_async_smem();
+          softmax_bar_sync();
+          if (store_issuer) {
+            tma_store_4d(&maps.o, buf, col0 + hh * 128 + oc, ts.hk * p.g, ts.tok0, ts.b);
+            bulk_commit_group();
+          }
+          ++ec;
         }
       }
       ++it;
