@@ -316,7 +316,7 @@ def e2e_measure(hd, x, device, steps):
     return ms, h2d, d2h
 
 
-def cpu_sample(n_hca=4096, n_dsa=1024):
+def cpu_sample(n_hca=12288, n_dsa=3072):
     """Times the oracle (plain C, OpenMP over query rows) on a bounded sample of the workload:
     full compression, HCA attention for n_hca query tokens and DSA top-k + attention for
     n_dsa query tokens, positions spread evenly over [0, L).  Each function runs once over all

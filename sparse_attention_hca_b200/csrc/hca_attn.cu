@@ -73,10 +73,14 @@ struct Params {
   int Lq, q_offset, Hq, Hkv, g, TT, n_c, win_start, W, blk;
   int n_tiles;      // token tiles per (b, kv head)
   int total_tiles;  // B * Hkv * n_tiles
+  int splits;       // work units per row tile (key tiles split among them; 1 = no split)
+  int total_units;  // total_tiles * splits
   int J_max;        // key tiles of the longest row tile (scratch capacity)
   float scale_log2;
   float* lse;
   uint8_t* scratch;  // gridDim.x * J_max * kScratchTileBytes
+  float* part_o;     // splits > 1: [total_units][128][512] unnormalised O of each unit
+  float2* part_ml;   // splits > 1: [total_units][128] (reference max in log2 units, row sum)
   int* err;
 };
 
@@ -107,14 +111,17 @@ struct KeyTile {
   int n;       // MMA N (multiple of 16, <= 128)
 };
 
-// The key tiles of one row tile.
+// The key tiles of one work unit: split s of row tile T (unit U = T * splits + s) takes the
+// row tile's key tiles [s*Jt/splits, (s+1)*Jt/splits).
 struct TileSet {
   int b, hk, tok0;  // batch, kv head, first token (relative to q_offset)
-  int J_c, J;       // number of compressed tiles, total tiles
+  int J_c, J;       // number of compressed tiles of the row tile, key tiles of this unit
+  int js;           // first key tile of this unit
   int nc_hi;        // entries needed by the last token
   int ws_lo;        // window start of the first token
   int t_hi;         // last valid token position
-  __device__ void init(int T, const Params& p) {
+  __device__ void init(int U, const Params& p) {
+    const int T = U / p.splits, split = U % p.splits;
     const int bh = T / p.n_tiles, tile = T % p.n_tiles;
     b = bh / p.Hkv;
     hk = bh % p.Hkv;
@@ -123,10 +130,13 @@ struct TileSet {
     nc_hi = n_compressed(t_hi, p.W, p.blk);
     ws_lo = window_start(p.q_offset + tok0, p.W);
     J_c = (nc_hi + kKeyTile - 1) / kKeyTile;
-    J = J_c + (t_hi - ws_lo + kKeyTile) / kKeyTile;
+    const int Jt = J_c + (t_hi - ws_lo + kKeyTile) / kKeyTile;
+    js = split * Jt / p.splits;
+    J = (split + 1) * Jt / p.splits - js;
   }
-  __device__ KeyTile get(int j) const {
+  __device__ KeyTile get(int jl) const {
     KeyTile kt;
+    const int j = js + jl;
     if (j < J_c) {
       kt.window = 0;
       kt.start = j * kKeyTile;
@@ -248,7 +258,7 @@ __global__ void __launch_bounds__(kThreads, 1) hca_attn_kernel(const __grid_cons
         for (int c = 0; ok && c < kVChunks; c += 2)
           load_unit(&maps.kv[1][kt.window][small], small, col0 + c * 64, ts.hk, row0, ts.b);
       };
-      if (blockIdx.x < p.total_tiles) {
+      if (blockIdx.x < p.total_units) {
         TileSet t0;
         t0.init(blockIdx.x, p);
         mbar_arrive_expect_tx(&bar.q_full, kQBytes);
@@ -256,7 +266,7 @@ __global__ void __launch_bounds__(kThreads, 1) hca_attn_kernel(const __grid_cons
           tma_load_4d(sQ + c * kChunkBytes, &maps.q, &bar.q_full, c * 64, t0.hk * p.g, t0.tok0, t0.b);
       }
       uint32_t tcount = 0;
-      for (int T = blockIdx.x; ok && T < p.total_tiles; T += gridDim.x, ++tcount) {
+      for (int T = blockIdx.x; ok && T < p.total_units; T += gridDim.x, ++tcount) {
         TileSet ts;
         ts.init(T, p);
         if (ts.J > p.J_max) break;
@@ -274,7 +284,7 @@ __global__ void __launch_bounds__(kThreads, 1) hca_attn_kernel(const __grid_cons
         if (!ok) break;
         // the next tile's Q, once this tile's last S MMA has read the buffer
         const int Tn = T + gridDim.x;
-        if (Tn < p.total_tiles) {
+        if (Tn < p.total_units) {
           TileSet tn;
           tn.init(Tn, p);
           ok = mbar_wait(&bar.q_empty, tcount & 1, &abort_flag, p.err);
@@ -323,7 +333,7 @@ __global__ void __launch_bounds__(kThreads, 1) hca_attn_kernel(const __grid_cons
           mma_commit(&bar.empty[grp]);
         }
       };
-      for (int T = blockIdx.x; ok && T < p.total_tiles; T += gridDim.x, ++tcount) {
+      for (int T = blockIdx.x; ok && T < p.total_units; T += gridDim.x, ++tcount) {
         TileSet ts;
         ts.init(T, p);
         if (ts.J > p.J_max) {
@@ -410,11 +420,31 @@ __global__ void __launch_bounds__(kThreads, 1) hca_attn_kernel(const __grid_cons
     // O half (TMEM) -> bf16 -> two 8 KB staging buffers -> TMA tensor store; then release O
     // O half (TMEM) -> normalised bf16 in registers, 128 columns at a time, each 128 columns
     // released to the MMA warp as soon as they are read -> two 8 KB staging buffers -> TMA
-    // tensor stores
-    auto epilogue = [&](const TileSet& ts, int col0, float inv_l) {
+    // tensor stores.  With split key ranges the unit's unnormalised fp32 O rows go to part_o.
+    auto epilogue = [&](const TileSet& ts, int col0, float inv_l, int U, bool row_valid) {
       ok = mbar_wait(&bar.o_full, it & 1, &abort_flag, p.err);
       if (!ok) return;
       tc_fence_after();
+      if (p.splits > 1) {
+        for (int hh = 0; hh < 2; ++hh) {
+          for (int oc = 0; oc < 128; oc += 32) {
+            uint32_t v[32];
+            tmem_ld32_nowait(tmem + lane_off + hh * 128 + oc, v);
+            tmem_wait_ld_regs(v);
+            if (row_valid) {
+              float4* dst = reinterpret_cast<float4*>(p.part_o + ((size_t)U * 128 + r) * kD + col0 + hh * 128 + oc);
+#pragma unroll
+              for (int i = 0; i < 8; ++i)
+                dst[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                                     __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+            }
+          }
+          tc_fence_before();
+          mbar_arrive(&bar.o_empty[hh]);
+        }
+        ++it;
+        return;
+      }
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
         uint32_t ob[64];
@@ -450,7 +480,7 @@ __global__ void __launch_bounds__(kThreads, 1) hca_attn_kernel(const __grid_cons
       ++it;
     };
 
-    for (int T = blockIdx.x; ok && T < p.total_tiles; T += gridDim.x) {
+    for (int T = blockIdx.x; ok && T < p.total_units; T += gridDim.x) {
       TileSet ts;
       ts.init(T, p);
       if (ts.J > p.J_max) break;
@@ -480,16 +510,15 @@ __global__ void __launch_bounds__(kThreads, 1) hca_attn_kernel(const __grid_cons
         s_par ^= 1u << (gs & 1);
         tc_fence_after();
         // pass 1: tile max over this row's visible columns
+        const uint32_t vis_n = (uint32_t)(hi - lo);  // column c is visible iff (c - lo) < vis_n
         float mx = -INFINITY;
         for (int c0 = 0; c0 < kt.n; c0 += 32) {
           uint32_t v[32];
           tmem_ld32_nowait(tS + c0, v);
           tmem_wait_ld_regs(v);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const int col = c0 + i;
-            if (col >= lo && col < hi) mx = fmaxf(mx, __uint_as_float(v[i]));
-          }
+          for (int i = 0; i < 32; ++i)
+            if ((uint32_t)(c0 + i - lo) < vis_n) mx = fmaxf(mx, __uint_as_float(v[i]));
         }
         const float m_tile = mx * p.scale_log2;  // -inf stays -inf
         bool need = false;
@@ -514,37 +543,43 @@ __global__ void __launch_bounds__(kThreads, 1) hca_attn_kernel(const __grid_cons
         }
         *scratch_alpha(scratch, j, r) = alpha;
         // pass 2: P = exp2(s*scale*log2e - m_ref) as bf16, in place over S and into the scratch
-        const bool any_visible = m_ref != -INFINITY;
+        const uint32_t vis_p = m_ref != -INFINITY ? vis_n : 0u;
         uint4* prow = scratch_p(scratch, j, r);
-        for (int c0 = 0; c0 < kt.n; c0 += 32) {
-          uint32_t v[32];
-          tmem_ld32_nowait(tS + c0, v);
-          tmem_wait_ld_regs(v);
-          uint32_t pk[16];
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const int c = c0 + 2 * i;
-            float p0 = 0.0f, p1 = 0.0f;
-            if (any_visible && c >= lo && c < hi) p0 = fast_exp2(__uint_as_float(v[2 * i]) * p.scale_log2 - m_ref);
-            if (any_visible && c + 1 >= lo && c + 1 < hi)
-              p1 = fast_exp2(__uint_as_float(v[2 * i + 1]) * p.scale_log2 - m_ref);
-            l_run += p0 + p1;
-            pk[i] = pack_bf16x2(p0, p1);
+        for (int q4 = 0; q4 < 4; ++q4) {
+          if (q4 * 32 < kt.n) {
+            uint32_t v[32];
+            tmem_ld32_nowait(tS + q4 * 32, v);
+            tmem_wait_ld_regs(v);
+            uint32_t pk[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const int c = q4 * 32 + 2 * i;
+              float p0 = 0.0f, p1 = 0.0f;
+              if ((uint32_t)(c - lo) < vis_p) p0 = fast_exp2(__uint_as_float(v[2 * i]) * p.scale_log2 - m_ref);
+              if ((uint32_t)(c + 1 - lo) < vis_p) p1 = fast_exp2(__uint_as_float(v[2 * i + 1]) * p.scale_log2 - m_ref);
+              l_run += p0 + p1;
+              pk[i] = pack_bf16x2(p0, p1);
+            }
+            tmem_st16(tS + q4 * 16, pk);
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+              __stcg(prow + (q4 * 4 + u) * 128, make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]));
           }
-          tmem_st16(tS + c0 / 2, pk);
-#pragma unroll
-          for (int u = 0; u < 4; ++u)
-            __stcg(prow + (c0 / 8 + u) * 128, make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]));
         }
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&bar.p_ready[gs & 1]);
       }
       if (!ok) break;
-      const float inv_l = l_run > 0.0f ? 1.0f / l_run : 0.0f;
-      if (p.lse && row_valid)
+      float inv_l = l_run > 0.0f ? 1.0f / l_run : 0.0f;
+      if (p.splits > 1) {  // the combine pass normalises
+        inv_l = 1.0f;
+        if (row_valid) p.part_ml[(size_t)T * 128 + r] = make_float2(m_ref, l_run);
+      } else if (p.lse && row_valid) {
         p.lse[((size_t)ts.b * p.Lq + tok) * p.Hq + h] = (m_ref + __log2f(l_run)) * 0.69314718055994531f;
-      epilogue(ts, 0, inv_l);
+      }
+      epilogue(ts, 0, inv_l, T, row_valid);
       if (!ok) break;
       g += ts.J;
       // ---- phase B: reload P_j into the S buffers, apply the same rescales
@@ -586,7 +621,7 @@ __global__ void __launch_bounds__(kThreads, 1) hca_attn_kernel(const __grid_cons
         mbar_arrive(&bar.p_ready[gs & 1]);
       }
       if (!ok) break;
-      epilogue(ts, kDHalf, inv_l);
+      epilogue(ts, kDHalf, inv_l, T, row_valid);
       g += ts.J;
     }
     if (store_issuer) bulk_wait_group0();
@@ -595,6 +630,48 @@ __global__ void __launch_bounds__(kThreads, 1) hca_attn_kernel(const __grid_cons
   tc_fence_before();
   __syncthreads();
   if (warp == 1) tmem_dealloc(tmem, 512);
+}
+
+// Split key ranges: row r of row tile T gathers its units' partial results,
+//     M = max_s m_s,  w_s = 2^(m_s - M),  O = sum_s w_s O_s / sum_s w_s l_s,
+// (m_s in log2 units, O_s and l_s relative to 2^m_s) and writes O (bf16) and lse.
+// One CTA per row tile, one warp per row at a time, 4 columns per lane per step.
+__global__ void __launch_bounds__(256) hca_combine_kernel(const Params p, uint16_t* __restrict__ O) {
+  const int T = blockIdx.x;
+  const int bh = T / p.n_tiles, tile = T % p.n_tiles;
+  const int b = bh / p.Hkv, hk = bh % p.Hkv;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  for (int r = warp; r < 128; r += 8) {
+    const int tok = tile * p.TT + r / p.g;
+    if (tok >= p.Lq) continue;
+    const int h = hk * p.g + r % p.g;
+    float M = -INFINITY;
+    for (int sp = 0; sp < p.splits; ++sp) M = fmaxf(M, p.part_ml[((size_t)T * p.splits + sp) * 128 + r].x);
+    float L = 0.0f;
+    for (int sp = 0; sp < p.splits; ++sp) {
+      const float2 ml = p.part_ml[((size_t)T * p.splits + sp) * 128 + r];
+      L += ml.y > 0.0f ? exp2f(ml.x - M) * ml.y : 0.0f;
+    }
+    const float inv_L = L > 0.0f ? 1.0f / L : 0.0f;
+    uint16_t* orow = O + (((size_t)b * p.Lq + tok) * p.Hq + h) * kD;
+    for (int c = lane * 4; c < kD; c += 128) {
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int sp = 0; sp < p.splits; ++sp) {
+        const size_t U = (size_t)T * p.splits + sp;
+        const float2 ml = p.part_ml[U * 128 + r];
+        if (!(ml.y > 0.0f)) continue;
+        const float w = exp2f(ml.x - M);
+        const float4 o = *reinterpret_cast<const float4*>(p.part_o + (U * 128 + r) * kD + c);
+        acc.x += w * o.x;
+        acc.y += w * o.y;
+        acc.z += w * o.z;
+        acc.w += w * o.w;
+      }
+      *reinterpret_cast<uint2*>(orow + c) =
+          make_uint2(pack_bf16x2(acc.x * inv_L, acc.y * inv_L), pack_bf16x2(acc.z * inv_L, acc.w * inv_L));
+    }
+    if (lane == 0 && p.lse) p.lse[((size_t)b * p.Lq + tok) * p.Hq + h] = (M + __log2f(L)) * 0.69314718055994531f;
+  }
 }
 
 bool make_map_4d(CUtensorMap* m, const void* base, int d, int heads, int rows, int B, int box_cols, int box_heads,
@@ -619,9 +696,20 @@ int num_sms() {
 // Launch geometry shared by the workspace query and the launch: HCADSA_ERR_UNSUPPORTED for
 // shapes the kernel does not take, HCADSA_ERR_CUDA if the device cannot be queried.
 struct Geometry {
-  int g, TT, n_tiles, total_tiles, grid, J_max;
-  size_t scratch_bytes;
+  int g, TT, n_tiles, total_tiles, splits, total_units, grid, J_max;
+  size_t scratch_bytes;   // probability tiles: grid * J_max * kScratchTileBytes
+  size_t part_bytes;      // splits > 1: unnormalised O rows and (max, sum) of every unit
+  size_t workspace_bytes;
 };
+
+long long host_n_compressed(long long t, int W, int blk) { return t - W + 1 > 0 ? (t - W + 1) / blk : 0; }
+long long host_window_start(long long t, int W) { return t - W + 1 > 0 ? t - W + 1 : 0; }
+// key tiles of the row tile with tokens [tok0, tok_hi] (relative to q_offset)
+long long host_tile_J(long long q_offset, long long tok0, long long tok_hi, int W, int blk) {
+  const long long t_hi = q_offset + tok_hi;
+  const long long nc = host_n_compressed(t_hi, W, blk);
+  return (nc + kKeyTile - 1) / kKeyTile + (t_hi - host_window_start(q_offset + tok0, W) + kKeyTile) / kKeyTile;
+}
 
 hcadsa_status geometry(Geometry* G, int B, int Lq, int q_offset, int Hq, int Hkv, int d, int blk, int W) {
   if (B <= 0 || Lq <= 0 || q_offset < 0 || Hq <= 0 || Hkv <= 0 || blk <= 0 || W <= 0 || Hq % Hkv != 0)
@@ -640,13 +728,32 @@ hcadsa_status geometry(Geometry* G, int B, int Lq, int q_offset, int Hq, int Hkv
   if (J_max > (1 << 20)) return HCADSA_ERR_UNSUPPORTED;
   const int sms = num_sms();
   if (sms <= 0) return HCADSA_ERR_CUDA;
+  // Few row tiles (decode: one token per sequence) leave most SMs idle: split every row tile's
+  // key tiles into `splits` units (each unit keeps at least one key tile) and combine after.
+  long long splits = 1;
+  if (2 * total <= sms) {
+    long long J_min = J_max;
+    for (long long t = 0; t < n_tiles; ++t) {
+      const long long tok0 = t * TT, tok_hi = (tok0 + TT < Lq ? tok0 + TT : Lq) - 1;
+      const long long J = host_tile_J(q_offset, tok0, tok_hi, W, blk);
+      J_min = J < J_min ? J : J_min;
+    }
+    splits = sms / total;
+    if (splits > J_min) splits = J_min;
+    if (splits > 64) splits = 64;
+    if (splits < 1) splits = 1;
+  }
   G->g = g;
   G->TT = TT;
   G->n_tiles = (int)n_tiles;
   G->total_tiles = (int)total;
-  G->grid = (int)(total < sms ? total : sms);
+  G->splits = (int)splits;
+  G->total_units = (int)(total * splits);
+  G->grid = G->total_units < sms ? G->total_units : sms;
   G->J_max = (int)J_max;
   G->scratch_bytes = (size_t)G->grid * (size_t)J_max * kScratchTileBytes;
+  G->part_bytes = splits > 1 ? (size_t)G->total_units * 128 * (kD * 4 + 8) : 0;
+  G->workspace_bytes = G->scratch_bytes + G->part_bytes;
   return HCADSA_OK;
 }
 
@@ -658,7 +765,7 @@ extern "C" size_t hca_attn_fwd_workspace_size(int B, int Lq, int q_offset, int H
   (void)n_c;
   hcadsa::Geometry G;
   if (hcadsa::geometry(&G, B, Lq, q_offset, Hq, Hkv, d, blk, W) != HCADSA_OK) return 0;
-  return G.scratch_bytes;
+  return G.workspace_bytes;
 }
 
 extern "C" hcadsa_status hca_attn_fwd(const hcadsa_bf16* Q, const hcadsa_bf16* Kc, const hcadsa_bf16* Vc, int n_c,
@@ -688,7 +795,7 @@ extern "C" hcadsa_status hca_attn_fwd(const hcadsa_bf16* Q, const hcadsa_bf16* K
   Geometry G;
   const hcadsa_status gs = geometry(&G, B, Lq, q_offset, Hq, Hkv, d, blk, W);
   if (gs != HCADSA_OK) return gs;
-  if (!workspace || workspace_bytes < G.scratch_bytes) return HCADSA_ERR_WORKSPACE;
+  if (!workspace || workspace_bytes < G.workspace_bytes) return HCADSA_ERR_WORKSPACE;
   if (!aligned16(workspace)) return HCADSA_ERR_ALIGN;
 
   Maps maps;
@@ -719,13 +826,23 @@ extern "C" hcadsa_status hca_attn_fwd(const hcadsa_bf16* Q, const hcadsa_bf16* K
   p.blk = blk;
   p.n_tiles = G.n_tiles;
   p.total_tiles = G.total_tiles;
+  p.splits = G.splits;
+  p.total_units = G.total_units;
   p.J_max = G.J_max;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.lse = lse;
   p.scratch = static_cast<uint8_t*>(workspace);
+  p.part_o = G.splits > 1 ? reinterpret_cast<float*>(p.scratch + G.scratch_bytes) : nullptr;
+  p.part_ml = G.splits > 1 ? reinterpret_cast<float2*>(p.scratch + G.scratch_bytes + (size_t)G.total_units * 128 * kD * 4)
+                           : nullptr;
   p.err = device_error_ptr();
   if (cudaFuncSetAttribute(hca_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) != cudaSuccess)
     return HCADSA_ERR_CUDA;
   hca_attn_kernel<<<G.grid, kThreads, kSmemBytes, as_stream(stream)>>>(maps, p);
+  if (G.splits > 1) {
+    const hcadsa_status st = launch_status();
+    if (st != HCADSA_OK) return st;
+    hca_combine_kernel<<<G.total_tiles, 256, 0, as_stream(stream)>>>(p, reinterpret_cast<uint16_t*>(O));
+  }
   return launch_status();
 }

@@ -197,6 +197,27 @@ def test_hca_decode_form(hd, B, t):
     print(check_attn(O.reshape(B, Hq, d), ref, f"hca decode t={t}"))
 
 
+def test_hca_split_key_ranges(hd):
+    """Few row tiles: every row tile's key tiles are split over several CTAs and the partial
+    softmax results are combined (3 query tokens per sequence, 4 sequences, lse checked)."""
+    d, Hq, blk, W, B, Lq, t0 = 512, 16, 128, 128, 4, 3, 20000
+    t_last = t0 + Lq - 1
+    n_c = (t_last + 1) // blk
+    ws = t0 - W + 1
+    Kc = synth.normal_bf16((B, n_c, 1, d), 1.0, 21, "K")
+    Vc = synth.normal_bf16((B, n_c, 1, d), 1.0, 21, "V")
+    Kw = synth.normal_bf16((B, t_last + 1 - ws, 1, d), 1.0, 22, "K")
+    Vw = synth.normal_bf16((B, t_last + 1 - ws, 1, d), 1.0, 22, "V")
+    Q = synth.normal_bf16((B, Lq, Hq, d), 1.0, 23, "Q")
+    O, lse = hd.hca_attn_fwd(Q.cuda(), Kc.cuda(), Vc.cuda(), Kw.cuda(), Vw.cuda(), win_start=ws, q_offset=t0,
+                             return_lse=True)
+    no_device_error(hd)
+    ref, ref_lse = oracle.hca_attn(bits(Q), bits(Kc), bits(Vc), bits(Kw), bits(Vw), win_start=ws, q_offset=t0,
+                                   with_lse=True)
+    print(check_attn(O.reshape(B * Lq, Hq, d), ref, "hca split key ranges"))
+    np.testing.assert_allclose(lse.reshape(B * Lq, Hq).cpu().numpy(), ref_lse, atol=2e-2, rtol=0)
+
+
 # ------------------------------------------------------------------ DSA indexer + top-k
 
 def _dsa_cfg(name, L, B=1, k=2048, sigma=None):
