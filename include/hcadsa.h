@@ -143,8 +143,11 @@ hcadsa_status hca_attn_fwd(const hcadsa_bf16* Q, const hcadsa_bf16* Kc, const hc
                            float scale, void* workspace, size_t workspace_bytes, hcadsa_stream stream);
 
 /*
- * Size in bytes of the workspace dsa_index_topk needs: the int32 indexer score
- * rows plus per-row selection state.
+ * Size in bytes of the workspace dsa_index_topk needs: the int32 indexer score rows,
+ *     B * Lq * round_up(min(q_offset + Lq, Lk), 128) * 4 bytes,
+ * plus, for few query rows over many keys (B*Lq <= 64, Lq < 64 and at least 32768 keys: the
+ * decode shape, where the selection is spread over all SMs), per row 16 + 2048*4 + 8192*8
+ * bytes of selection state (score range, histogram, candidate list).
  */
 size_t dsa_index_topk_workspace_size(int B, int Lq, int q_offset, int Lk, int k);
 
@@ -164,8 +167,9 @@ size_t dsa_index_topk_workspace_size(int B, int Lq, int q_offset, int Lk, int k)
  *   w_idx : [H_idx] int32  (device)
  *   idx   : [B, Lq, k] int32             (written)
  *   ws    : workspace of dsa_index_topk_workspace_size(...) bytes
- * Requirements: H_idx == 4, d_idx == 64, 1 <= k <= 4096, |w_idx| small enough
- * that every score fits in [-2^30, 2^30] (checked on the device).
+ * Requirements: H_idx == 4, d_idx == 64, 1 <= k <= 4096.  The caller keeps
+ * sum_j |w_idx[j]| <= 2047, so that no score (|q . k| <= 64 * 128 * 128 = 2^20 per head)
+ * overflows int32; this is not checked.
  */
 hcadsa_status dsa_index_topk(const int8_t* q_idx, const int8_t* k_idx, const int32_t* w_idx, int32_t* idx,
                              void* ws, size_t ws_bytes, int B, int Lq, int q_offset, int Lk, int H_idx, int d_idx,
@@ -180,8 +184,9 @@ hcadsa_status dsa_index_topk(const int8_t* q_idx, const int8_t* k_idx, const int
  * dsa_index_topk, minus the workspace: the int32 score rows go to a fixed scratch array of
  * dsa_index_topk_noalloc_max_scratch_bytes() bytes (64 MiB) compiled into the library.
  * Every GPU that loads the library holds that array until the process exits.
- *   - Calls whose score rows need more than that (dsa_index_topk_workspace_size(...) >
- *     the maximum) return HCADSA_ERR_WORKSPACE before anything is enqueued.  Example limits:
+ *   - Calls whose int32 score rows (B * Lq * round_up(min(q_offset + Lq, Lk), 128) * 4
+ *     bytes) exceed the maximum return HCADSA_ERR_WORKSPACE before anything is enqueued.  This
+ *     entry always selects with one thread block per query row.  Example limits:
  *     prefill up to 4096 x 4096, or decode (Lq = 1) of 16 sequences at 1M keys.
  *   - The first call on each device looks up the array's device address (one
  *     cudaGetSymbolAddress, no allocation); make that first call before any stream capture.

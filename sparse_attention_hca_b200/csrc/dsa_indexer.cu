@@ -16,6 +16,18 @@
 //                             k-th largest score over the row (staged in shared memory when it
 //                             fits), then an ordered compaction so ties go to lower positions
 //                             and the output is ascending.
+// Few query rows over very many keys (decode) would leave all but a handful of SMs idle in
+// select_kernel, so those calls select with every SM instead:
+//   * the streaming scorer also records each row's score range,
+//   * hist_kernel          -- many CTAs per row: 2048-bin histogram of the row over that range,
+//   * candidates_kernel    -- many CTAs per row: the bin b* holding the k-th largest score is
+//                             found from the histogram; every key in a bin >= b* (a superset of
+//                             the top k, at most kCandCap of them) is appended to a candidate
+//                             list,
+//   * finalize_kernel      -- one CTA per row: bitonic sort of the candidates by (score desc,
+//                             position asc), the first k positions sorted ascending.  A row
+//                             whose candidates overflow (e.g. massive ties) falls back to the
+//                             exact single-CTA select of that row.
 #include <cuda_bf16.h>
 
 #include <mutex>
@@ -42,6 +54,24 @@ __host__ __device__ inline long long score_row_stride(int Lq, int q_offset, int 
   if (n_max > Lk) n_max = Lk;
   if (n_max < 1) n_max = 1;
   return round_up(n_max, kKTile);
+}
+
+// Multi-CTA selection for few rows over many keys: per-row state after the score rows.
+constexpr int kHistBins = 2048;
+constexpr int kCandCap = 8192;
+constexpr int kSplitRowsMax = 64;       // at most this many query rows (B * Lq) ...
+constexpr long long kSplitMinKeys = 32768;  // ... each over at least this many keys (row stride)
+struct RowSel {
+  int vmin, vmax;   // score range of the row (streaming scorer)
+  int n_cand, pad;  // candidates appended (may exceed kCandCap: overflow)
+  unsigned int hist[kHistBins];
+};
+__host__ __device__ inline bool use_split_select(int B, int Lq, int q_offset, int Lk) {
+  return (long long)B * Lq <= kSplitRowsMax && Lq < 64 && score_row_stride(Lq, q_offset, Lk) >= kSplitMinKeys;
+}
+// bytes after the score rows: RowSel per row, then kCandCap (u, position) pairs per row
+__host__ __device__ inline long long split_select_bytes(int rows) {
+  return (long long)rows * ((long long)sizeof(RowSel) + (long long)kCandCap * 8);
 }
 
 __device__ __forceinline__ void cp_async16(void* dst, const void* src, bool valid) {
@@ -175,7 +205,8 @@ __global__ void __launch_bounds__(kStreamThreads) score_stream_kernel(const int8
                                                                      const int8_t* __restrict__ k_idx,
                                                                      const int32_t* __restrict__ w_idx,
                                                                      int32_t* __restrict__ scores, int Lq,
-                                                                     int q_offset, int Lk, long long row_stride) {
+                                                                     int q_offset, int Lk, long long row_stride,
+                                                                     RowSel* __restrict__ rowsel) {
   const int row = blockIdx.y;
   const int b = row / Lq, r = row % Lq;
   const int n = min(q_offset + r + 1, Lk);
@@ -192,6 +223,7 @@ __global__ void __launch_bounds__(kStreamThreads) score_stream_kernel(const int8
   const int8_t* kb = k_idx + (size_t)b * Lk * kDIdx;
   int32_t* out = scores + (size_t)row * row_stride;
   uint4 kv[kKeysPerThread][4];
+  int vmn = INT_MAX, vmx = INT_MIN;
 #pragma unroll
   for (int u = 0; u < kKeysPerThread; ++u) {
     const int s = s_base + u * kStreamThreads;
@@ -215,6 +247,19 @@ __global__ void __launch_bounds__(kStreamThreads) score_stream_kernel(const int8
         total += sw[j] * dot;
       }
       out[s] = total;
+      vmn = min(vmn, total);
+      vmx = max(vmx, total);
+    }
+  }
+  if (rowsel) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      vmn = min(vmn, __shfl_xor_sync(0xffffffffu, vmn, o));
+      vmx = max(vmx, __shfl_xor_sync(0xffffffffu, vmx, o));
+    }
+    if ((threadIdx.x & 31) == 0 && vmn <= vmx) {
+      atomicMin(&rowsel[row].vmin, vmn);
+      atomicMax(&rowsel[row].vmax, vmx);
     }
   }
 }
@@ -455,6 +500,186 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const int32_t* __re
     select_row<false>(row_g, sel_row, n, k, out, sh);  // sel_row stages compaction chunks
 }
 
+
+// ------------------------------------------------------------------ multi-CTA selection (few rows)
+
+constexpr int kSplitChunk = 16384;  // scores per CTA in hist_kernel / candidates_kernel
+
+__global__ void __launch_bounds__(256) rowsel_init_kernel(RowSel* __restrict__ rs) {
+  RowSel& r = rs[blockIdx.x];
+  if (threadIdx.x == 0) {
+    r.vmin = INT_MAX;
+    r.vmax = INT_MIN;
+    r.n_cand = 0;
+    r.pad = 0;
+  }
+  for (int i = threadIdx.x; i < kHistBins; i += 256) r.hist[i] = 0;
+}
+
+// bins of u = score - vmin: u >> shift, shift such that the whole range fits in kHistBins bins
+__device__ __forceinline__ int hist_shift(unsigned range) {
+  const int bits = range == 0u ? 0 : 32 - __clz(range);
+  return bits > 11 ? bits - 11 : 0;
+}
+
+__global__ void __launch_bounds__(256) hist_kernel(const int32_t* __restrict__ scores, RowSel* __restrict__ rs,
+                                                   int Lq, int q_offset, int Lk, int k, long long row_stride) {
+  const int row = blockIdx.y, r = row % Lq;
+  const int n = max(0, min(q_offset + r + 1, Lk));
+  const int c0 = blockIdx.x * kSplitChunk;
+  if (n <= k || c0 >= n) return;
+  __shared__ unsigned int h[kHistBins];
+  for (int i = threadIdx.x; i < kHistBins; i += 256) h[i] = 0;
+  __syncthreads();
+  const int vmin = rs[row].vmin;
+  const int sh = hist_shift((unsigned)rs[row].vmax - (unsigned)vmin);
+  const int* rowp = scores + (size_t)row * row_stride;
+  const int c1 = min(c0 + kSplitChunk, n);
+#pragma unroll 8
+  for (int i = c0 + threadIdx.x; i < c1; i += 256) atomicAdd(&h[((unsigned)__ldcg(rowp + i) - (unsigned)vmin) >> sh], 1u);
+  __syncthreads();
+  for (int b = threadIdx.x; b < kHistBins; b += 256)
+    if (h[b]) atomicAdd(&rs[row].hist[b], h[b]);
+}
+
+__global__ void __launch_bounds__(256) candidates_kernel(const int32_t* __restrict__ scores, RowSel* __restrict__ rs,
+                                                         int2* __restrict__ cand, int Lq, int q_offset, int Lk, int k,
+                                                         long long row_stride) {
+  const int row = blockIdx.y, r = row % Lq;
+  const int n = max(0, min(q_offset + r + 1, Lk));
+  const int c0 = blockIdx.x * kSplitChunk;
+  if (n <= k || c0 >= n) return;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  __shared__ int wsum[8];
+  __shared__ int bstar;
+  // thread t counts bins [kHistBins - 8(t+1), kHistBins - 8t), i.e. from the top down
+  int cnt[8], tot = 0;
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    cnt[q] = (int)rs[row].hist[kHistBins - 1 - (tid * 8 + q)];
+    tot += cnt[q];
+  }
+  int incl = tot;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) wsum[warp] = incl;
+  __syncthreads();
+  int before_warp = 0;
+  for (int w = 0; w < warp; ++w) before_warp += wsum[w];
+  incl += before_warp;
+  const int above = incl - tot;  // keys in bins above this thread's
+  if (above < k && incl >= k) {
+    int acc = above;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      if (acc + cnt[q] >= k) {
+        bstar = kHistBins - 1 - (tid * 8 + q);
+        break;
+      }
+      acc += cnt[q];
+    }
+  }
+  __syncthreads();
+  const unsigned b_lo = (unsigned)bstar;
+  const int vmin = rs[row].vmin;
+  const int sh = hist_shift((unsigned)rs[row].vmax - (unsigned)vmin);
+  const int* rowp = scores + (size_t)row * row_stride;
+  int2* cr = cand + (size_t)row * kCandCap;
+  const int c1 = min(c0 + kSplitChunk, n);
+  for (int base = c0; base < c1; base += 256) {  // warp-uniform trip count
+    const int i = base + tid;
+    unsigned u = 0;
+    bool take = false;
+    if (i < c1) {
+      u = (unsigned)__ldcg(rowp + i) - (unsigned)vmin;
+      take = (u >> sh) >= b_lo;
+    }
+    const unsigned m = __ballot_sync(0xffffffffu, take);
+    if (m) {
+      int slot = 0;
+      if (lane == __ffs(m) - 1) slot = atomicAdd(&rs[row].n_cand, __popc(m));
+      slot = __shfl_sync(0xffffffffu, slot, __ffs(m) - 1) + __popc(m & ((1u << lane) - 1u));
+      if (take && slot < kCandCap) cr[slot] = make_int2((int)u, i);
+    }
+  }
+}
+
+// Ascending bitonic sort of P (a power of two) keys in shared memory by the whole block.
+template <typename T>
+__device__ void block_bitonic_sort(T* keys, int P) {
+  for (int size = 2; size <= P; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int i = threadIdx.x; i < P / 2; i += kSelThreads) {
+        const int lo = 2 * i - (i & (stride - 1));
+        const int hi = lo + stride;
+        const bool up = (lo & size) == 0;
+        const T a = keys[lo], b = keys[hi];
+        if ((a > b) == up) {
+          keys[lo] = b;
+          keys[hi] = a;
+        }
+      }
+      __syncthreads();
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kSelThreads) finalize_kernel(const int32_t* __restrict__ scores,
+                                                               const RowSel* __restrict__ rs,
+                                                               const int2* __restrict__ cand,
+                                                               int32_t* __restrict__ idx, int Lq, int q_offset,
+                                                               int Lk, int k, long long row_stride) {
+  extern __shared__ __align__(16) int sel_row[];
+  __shared__ SelShared sh;
+  const int row = blockIdx.x, r = row % Lq;
+  const int n = max(0, min(q_offset + r + 1, Lk));
+  int32_t* out = idx + (size_t)row * k;
+  if (n <= k) {
+    for (int i = threadIdx.x; i < k; i += kSelThreads) out[i] = i < n ? i : -1;
+    return;
+  }
+  const int nc = rs[row].n_cand;
+  if (nc > kCandCap) {  // too many keys tie at the threshold bin: exact select over the whole row
+    const int* row_g = scores + (size_t)row * row_stride;
+    if (n <= kSelSmemCap)
+      select_row<true>(row_g, sel_row, n, k, out, sh);
+    else
+      select_row<false>(row_g, sel_row, n, k, out, sh);
+    return;
+  }
+  // candidates by (u desc, position asc): key = (~u) << 32 | position, ascending
+  unsigned long long* keys = reinterpret_cast<unsigned long long*>(sel_row);  // kCandCap keys
+  int P = 2;
+  while (P < nc) P <<= 1;
+  const int2* cr = cand + (size_t)row * kCandCap;
+  for (int i = threadIdx.x; i < P; i += kSelThreads) {
+    unsigned long long key = ~0ull;
+    if (i < nc) {
+      const int2 c = cr[i];
+      key = ((unsigned long long)(0xFFFFFFFFu - (unsigned)c.x) << 32) | (unsigned)c.y;
+    }
+    keys[i] = key;
+  }
+  __syncthreads();
+  block_bitonic_sort(keys, P);
+  // the first k positions, ascending
+  int* pos = reinterpret_cast<int*>(keys + kCandCap);
+  int Pk = 2;
+  while (Pk < k) Pk <<= 1;
+  for (int i = threadIdx.x; i < Pk; i += kSelThreads) pos[i] = i < k ? (int)(keys[i] & 0xFFFFFFFFull) : INT_MAX;
+  __syncthreads();
+  block_bitonic_sort(pos, Pk);
+  for (int i = threadIdx.x; i < k; i += kSelThreads) out[i] = pos[i];
+}
+
+// int32 score rows of a call (the workspace part both entry points need)
+size_t score_rows_bytes(int B, int Lq, int q_offset, int Lk) {
+  return (size_t)B * (size_t)Lq * (size_t)score_row_stride(Lq, q_offset, Lk) * sizeof(int32_t);
+}
+
 }  // namespace
 }  // namespace hcadsa
 
@@ -462,7 +687,9 @@ extern "C" size_t dsa_index_topk_workspace_size(int B, int Lq, int q_offset, int
   using namespace hcadsa;
   (void)k;
   if (B <= 0 || Lq <= 0 || Lk <= 0 || q_offset < 0) return 0;
-  return (size_t)B * (size_t)Lq * (size_t)score_row_stride(Lq, q_offset, Lk) * sizeof(int32_t);
+  size_t bytes = score_rows_bytes(B, Lq, q_offset, Lk);
+  if (use_split_select(B, Lq, q_offset, Lk)) bytes += (size_t)split_select_bytes(B * Lq);
+  return bytes;
 }
 
 extern "C" hcadsa_status dsa_index_topk(const int8_t* q_idx, const int8_t* k_idx, const int32_t* w_idx,
@@ -478,11 +705,17 @@ extern "C" hcadsa_status dsa_index_topk(const int8_t* q_idx, const int8_t* k_idx
   cudaStream_t s = as_stream(stream);
   const bool need_scores = (long long)q_offset + Lq > k && Lk > k;  // some row has more than k candidates
   const long long stride = score_row_stride(Lq, q_offset, Lk);
+  const bool split = need_scores && use_split_select(B, Lq, q_offset, Lk);
+  const int rows = B * Lq;
+  RowSel* rowsel = split ? reinterpret_cast<RowSel*>(static_cast<char*>(ws) + score_rows_bytes(B, Lq, q_offset, Lk))
+                         : nullptr;
+  int2* cand = split ? reinterpret_cast<int2*>(rowsel + rows) : nullptr;
   if (need_scores) {
     if (!ws) return HCADSA_ERR_WORKSPACE;
     if (!aligned16(ws)) return HCADSA_ERR_ALIGN;
     if (ws_bytes < dsa_index_topk_workspace_size(B, Lq, q_offset, Lk, k)) return HCADSA_ERR_WORKSPACE;
     int32_t* scores = static_cast<int32_t*>(ws);
+    if (split) rowsel_init_kernel<<<(unsigned)(B * Lq), 256, 0, s>>>(rowsel);
     if (Lq >= 64) {
       const long long n_max = stride;
       dim3 grid((unsigned)((n_max + kKeyTilesPerCta * kKTile - 1) / (kKeyTilesPerCta * kKTile)),
@@ -498,11 +731,22 @@ extern "C" hcadsa_status dsa_index_topk(const int8_t* q_idx, const int8_t* k_idx
       dim3 grid((unsigned)((n_max + kStreamThreads * kKeysPerThread - 1) / (kStreamThreads * kKeysPerThread)),
                 (unsigned)(B * Lq));
       if (grid.y > 65535u) return HCADSA_ERR_UNSUPPORTED;
-      score_stream_kernel<<<grid, kStreamThreads, 0, s>>>(q_idx, k_idx, w_idx, scores, Lq, q_offset, Lk, stride);
+      score_stream_kernel<<<grid, kStreamThreads, 0, s>>>(q_idx, k_idx, w_idx, scores, Lq, q_offset, Lk, stride,
+                                                           rowsel);
     }
     if (cudaGetLastError() != cudaSuccess) return HCADSA_ERR_CUDA;
   }
   const int smem = kSelSmemCap * (int)sizeof(int);
+  if (split) {
+    int32_t* scores = static_cast<int32_t*>(ws);
+    const dim3 grid((unsigned)((stride + kSplitChunk - 1) / kSplitChunk), (unsigned)rows);
+    hist_kernel<<<grid, 256, 0, s>>>(scores, rowsel, Lq, q_offset, Lk, k, stride);
+    candidates_kernel<<<grid, 256, 0, s>>>(scores, rowsel, cand, Lq, q_offset, Lk, k, stride);
+    if (cudaFuncSetAttribute(finalize_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+      return HCADSA_ERR_CUDA;
+    finalize_kernel<<<(unsigned)rows, kSelThreads, smem, s>>>(scores, rowsel, cand, idx, Lq, q_offset, Lk, k, stride);
+    return launch_status();
+  }
   if (cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return HCADSA_ERR_CUDA;
   select_kernel<<<(unsigned)(B * Lq), kSelThreads, smem, s>>>(need_scores ? static_cast<int32_t*>(ws) : nullptr,
@@ -558,8 +802,7 @@ extern "C" hcadsa_status dsa_index_topk_noalloc(const int8_t* q_idx, const int8_
   const bool need_scores = (long long)q_offset + Lq > k && Lk > k;
   const long long stride = score_row_stride(Lq, q_offset, Lk);
   // size check first: a call that does not fit is refused before any CUDA call
-  if (need_scores && dsa_index_topk_workspace_size(B, Lq, q_offset, Lk, k) > kNoAllocScratchBytes)
-    return HCADSA_ERR_WORKSPACE;
+  if (need_scores && score_rows_bytes(B, Lq, q_offset, Lk) > kNoAllocScratchBytes) return HCADSA_ERR_WORKSPACE;
   cudaStream_t s = as_stream(stream);
   int32_t* scores = nullptr;
   if (need_scores) {
@@ -578,7 +821,8 @@ extern "C" hcadsa_status dsa_index_topk_noalloc(const int8_t* q_idx, const int8_
       dim3 grid((unsigned)((stride + kStreamThreads * kKeysPerThread - 1) / (kStreamThreads * kKeysPerThread)),
                 (unsigned)(B * Lq));
       if (grid.y > 65535u) return HCADSA_ERR_UNSUPPORTED;
-      score_stream_kernel<<<grid, kStreamThreads, 0, s>>>(q_idx, k_idx, w_idx, scores, Lq, q_offset, Lk, stride);
+      score_stream_kernel<<<grid, kStreamThreads, 0, s>>>(q_idx, k_idx, w_idx, scores, Lq, q_offset, Lk, stride,
+                                                           nullptr);
     }
     if (cudaGetLastError() != cudaSuccess) return HCADSA_ERR_CUDA;
   }

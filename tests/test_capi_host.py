@@ -96,7 +96,10 @@ def test_dsa_argument_errors(lib):
 
 def test_workspace_size_queries(lib):
     assert lib.dsa_index_topk_workspace_size(1, 32768, 0, 32768, 2048) == 32768 * 32768 * 4
-    assert lib.dsa_index_topk_workspace_size(2, 1, 1048575, 1048576, 2048) == 2 * 1048576 * 4
+    # few rows over many keys add the multi-CTA selection state: per row 16 bytes + a 2048-bin
+    # histogram + 8192 (score, position) candidates
+    assert lib.dsa_index_topk_workspace_size(2, 1, 1048575, 1048576, 2048) == 2 * 1048576 * 4 + 2 * (
+        16 + 2048 * 4 + 8192 * 8)
     # HCA's workspace holds one probability-tile slot per resident CTA, so it is sized for the
     # current device; unsupported shapes (and a machine with no device to size for) give 0
     assert lib.hca_attn_fwd_workspace_size(1, 32768, 0, 16, 1, 256, 256, 128, 128) == 0

@@ -279,6 +279,33 @@ def test_topk_decode_form(hd, B, t):
     assert np.array_equal(idx.cpu().numpy().reshape(B, 2048), ref)
 
 
+def test_topk_decode_ties_overflow_candidates(hd):
+    """Decode shape where every score ties (q_idx = 0): the threshold bin holds all 50000 keys,
+    more than the candidate list takes, so the row falls back to the exact single-CTA select;
+    ties go to the lowest positions."""
+    B, t, k = 2, 49999, 2048
+    q = torch.zeros(B, 1, 4, 64, dtype=torch.int8)
+    kk = synth.randint((B, t + 1, 64), -8, 8, 31, "k_idx", torch.int8)
+    idx = hd.dsa_index_topk(q.cuda(), kk.cuda(), torch.tensor([1, 2, 3, 4], dtype=torch.int32).cuda(), k,
+                            q_offset=t)
+    no_device_error(hd)
+    exp = np.tile(np.arange(k, dtype=np.int32), (B, 1))
+    assert np.array_equal(idx.cpu().numpy().reshape(B, k), exp)
+
+
+def test_topk_decode_many_rows_split_select(hd):
+    """Lq = 3 rows per sequence over 40000+ keys: the multi-CTA selection path, bit-exact."""
+    B, Lq, t0, k = 3, 3, 40000, 2048
+    g = torch.Generator().manual_seed(41)
+    q = torch.randint(-8, 9, (B, Lq, 4, 64), generator=g).to(torch.int8)
+    kk = torch.randint(-8, 9, (B, t0 + Lq, 64), generator=g).to(torch.int8)
+    w = torch.tensor([2, 1, 4, 3], dtype=torch.int32)
+    idx = hd.dsa_index_topk(q.cuda(), kk.cuda(), w.cuda(), k, q_offset=t0)
+    no_device_error(hd)
+    ref = oracle.dsa_topk(q.numpy(), kk.numpy(), w.numpy(), k, q_offset=t0)
+    assert np.array_equal(idx.cpu().numpy().reshape(B * Lq, k), ref)
+
+
 def test_topk_32k_sampled_rows(hd):
     cfg = synth.DSA_32K
     inp = synth.dsa_inputs(cfg)

