@@ -53,7 +53,11 @@ constexpr int kD = 512;
 constexpr int kDHalf = 256;
 constexpr int kKeyTile = 128;
 constexpr int kSmallRows = 32;  // TMA box height for key tiles of at most 32 keys
-constexpr int kGroups = 2;  // ring: two groups of two 16 KB chunk slots (128 d-columns of a tile)
+// Ring: groups of two 16 KB chunk slots (128 d-columns of a key tile).  Two groups, plus a third
+// in the epilogue staging area when key ranges are split (those epilogues write fp32 partials
+// straight to global memory, and their K/V stream from HBM, where depth pays).
+constexpr int kGroups = 2;
+constexpr int kMaxGroups = 3;
 constexpr int kChunkBytes = 128 * 128;  // 128 rows x 64 bf16
 constexpr int kSmallChunkBytes = kSmallRows * 128;
 constexpr int kQChunks = kD / 64;      // 8
@@ -62,7 +66,8 @@ constexpr int kQBytes = kQChunks * kChunkBytes;
 constexpr int kOutCols = 32;                  // O columns per staged store
 constexpr int kOutBufBytes = 128 * kOutCols * 2;  // 8 KB
 constexpr int kGroupBytes = 2 * kChunkBytes;
-constexpr int kSmemBytes = kQBytes + kGroups * kGroupBytes + 2 * kOutBufBytes + 1024;
+constexpr int kSmemBytes = kQBytes + kMaxGroups * kGroupBytes + 1024;
+static_assert(kGroups * kGroupBytes + 2 * kOutBufBytes <= kMaxGroups * kGroupBytes, "staging fits the third group");
 constexpr int kThreads = 192;
 constexpr float kLazyRescale = 8.0f;  // log2 units
 // per-CTA scratch per key tile: P (128 rows x 128 keys bf16) + one fp32 rescale factor per row
@@ -154,8 +159,8 @@ struct TileSet {
 
 struct __align__(8) Barriers {
   uint64_t q_full, q_empty;
-  uint64_t full[kGroups];   // both chunks of a ring group landed
-  uint64_t empty[kGroups];  // the MMAs that read the group have completed
+  uint64_t full[kMaxGroups];   // both chunks of a ring group landed
+  uint64_t empty[kMaxGroups];  // the MMAs that read the group have completed
   uint64_t s_full[2];
   uint64_t p_ready[2];
   uint64_t pv_done[2];  // the PV that read P from S buffer i has completed
@@ -209,7 +214,7 @@ __global__ void __launch_bounds__(kThreads, 1) hca_attn_kernel(const __grid_cons
   if (threadIdx.x == 0) {
     mbar_init(&bar.q_full, 1);
     mbar_init(&bar.q_empty, 1);
-    for (int s = 0; s < kGroups; ++s) {
+    for (int s = 0; s < kMaxGroups; ++s) {
       mbar_init(&bar.full[s], 1);
       mbar_init(&bar.empty[s], 1);
     }
@@ -237,19 +242,22 @@ __global__ void __launch_bounds__(kThreads, 1) hca_attn_kernel(const __grid_cons
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       tma_prefetch_desc(&maps.q);
-      uint32_t u = 0;  // ring groups filled: group u & 1, phase (u >> 1) & 1
+      const uint32_t ngroups = p.splits > 1 ? kMaxGroups : kGroups;
+      uint32_t grp = 0, gph = 0;  // next ring group to fill and the phase of its use
       bool ok = true;
       // two 64-column chunks (columns col .. col+127 of a key tile) into the next ring group
       auto load_unit = [&](const CUtensorMap* m, bool small, int col, int hk, int row0, int b) {
-        const uint32_t grp = u & 1;
-        ok = mbar_wait(&bar.empty[grp], ((u >> 1) & 1) ^ 1, &abort_flag, p.err);
+        ok = mbar_wait(&bar.empty[grp], gph ^ 1, &abort_flag, p.err);
         if (ok) {
           mbar_arrive_expect_tx(&bar.full[grp], 2 * (small ? kSmallChunkBytes : kChunkBytes));
           uint8_t* dst = sRing + grp * kGroupBytes;
           tma_load_4d(dst, m, &bar.full[grp], col, hk, row0, b);
           tma_load_4d(dst + kChunkBytes, m, &bar.full[grp], col + 64, hk, row0, b);
         }
-        ++u;
+        if (++grp == ngroups) {
+          grp = 0;
+          gph ^= 1;
+        }
       };
       auto load_v = [&](const TileSet& ts, int j, int col0) {
         const KeyTile kt = ts.get(j);
@@ -301,7 +309,14 @@ __global__ void __launch_bounds__(kThreads, 1) hca_attn_kernel(const __grid_cons
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t sQa = smem_u32(sQ), sRa = smem_u32(sRing);
-      uint32_t u = 0;       // ring groups consumed
+      const uint32_t ngroups = p.splits > 1 ? kMaxGroups : kGroups;
+      uint32_t grp = 0, gph = 0;  // next ring group to consume and the phase of its use
+      auto next_group = [&]() {
+        if (++grp == ngroups) {
+          grp = 0;
+          gph ^= 1;
+        }
+      };
       uint32_t tcount = 0;  // row tiles
       uint32_t g = 0;       // key tiles of all earlier phases
       uint32_t it = 0;      // O halves
@@ -317,13 +332,12 @@ __global__ void __launch_bounds__(kThreads, 1) hca_attn_kernel(const __grid_cons
       auto pv = [&](const KeyTile& kt, int j, uint32_t gj) {
         const uint32_t tP = tmem + kDHalf + (gj & 1) * kKeyTile;
         const int nk = kt.n / 16;
-        for (int vu = 0; ok && vu < kVChunks / 2; ++vu, ++u) {
+        for (int vu = 0; ok && vu < kVChunks / 2; ++vu, next_group()) {
           if (j == 0) {  // the previous O half's epilogue must have read these 128 columns
             ok = mbar_wait(&bar.o_empty[vu], (it & 1) ^ 1, &abort_flag, p.err);
             if (!ok) break;
           }
-          const uint32_t grp = u & 1;
-          ok = mbar_wait(&bar.full[grp], (u >> 1) & 1, &abort_flag, p.err);
+          ok = mbar_wait(&bar.full[grp], gph, &abort_flag, p.err);
           if (!ok) break;
           tc_fence_after();
           const uint64_t db = dv0 + grp * kGroupDesc;
@@ -355,9 +369,8 @@ __global__ void __launch_bounds__(kThreads, 1) hca_attn_kernel(const __grid_cons
               if (!ok) break;
               tc_fence_after();
             }
-            for (int c = 0; ok && c < kQChunks; c += 2, ++u) {
-              const uint32_t grp = u & 1;
-              ok = mbar_wait(&bar.full[grp], (u >> 1) & 1, &abort_flag, p.err);
+            for (int c = 0; ok && c < kQChunks; c += 2, next_group()) {
+              ok = mbar_wait(&bar.full[grp], gph, &abort_flag, p.err);
               if (!ok) break;
               tc_fence_after();
               const uint64_t da = dq0 + (uint64_t)((c * kChunkBytes) >> 4);
