@@ -197,10 +197,17 @@ __global__ void __launch_bounds__(256) score_tiled_kernel(const int8_t* __restri
 
 // ------------------------------------------------------------------ streaming scorer (decode)
 //
-// grid.x = key blocks, grid.y = B * Lq query rows.  Each thread scores kKeysPerThread keys.
+// grid.x = key blocks of kStreamKeysPerCta, grid.y = B * Lq query rows.
 constexpr int kStreamThreads = 256;
-constexpr int kKeysPerThread = 4;
+constexpr int kStreamLoads = 8;                                          // 16-byte loads in flight per lane
+constexpr int kStreamKeysPerIter = kStreamThreads / 4 * kStreamLoads;    // 512 keys per CTA iteration
+constexpr int kStreamIters = 8;                                          // iterations per CTA
+constexpr int kStreamKeysPerCta = kStreamKeysPerIter * kStreamIters;     // 4096
 
+// Four lanes share one 64-byte key: lane l reads bytes 16*(l%4) .. +15 of key l/4 of its group
+// of 8 keys, so each warp load instruction moves 512 contiguous bytes.  A lane dots its slice
+// with the matching 16 bytes of each indexer head's query (dp4a), weights the 4 partial dots,
+// and the 4 lanes of a key add their partial totals (all int32, exact).
 __global__ void __launch_bounds__(kStreamThreads) score_stream_kernel(const int8_t* __restrict__ q_idx,
                                                                      const int8_t* __restrict__ k_idx,
                                                                      const int32_t* __restrict__ w_idx,
@@ -210,45 +217,60 @@ __global__ void __launch_bounds__(kStreamThreads) score_stream_kernel(const int8
   const int row = blockIdx.y;
   const int b = row / Lq, r = row % Lq;
   const int n = min(q_offset + r + 1, Lk);
-  __shared__ int sq[kHIdx * kDIdx / 4];
-  __shared__ int sw[kHIdx];
-  if (threadIdx.x < kHIdx * kDIdx / 4)
-    sq[threadIdx.x] = reinterpret_cast<const int*>(q_idx + (size_t)row * kHIdx * kDIdx)[threadIdx.x];
-  if (threadIdx.x < kHIdx) sw[threadIdx.x] = w_idx[threadIdx.x];
-  __syncthreads();
-  int q[kHIdx * kDIdx / 4];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int part = lane & 3;  // 16-byte slice of the key
+  int q[kHIdx][4];
+  int w[kHIdx];
+  {
+    const int4* qrow = reinterpret_cast<const int4*>(q_idx + (size_t)row * kHIdx * kDIdx);
 #pragma unroll
-  for (int i = 0; i < kHIdx * kDIdx / 4; ++i) q[i] = sq[i];
-  const int s_base = blockIdx.x * kStreamThreads * kKeysPerThread + threadIdx.x;
-  const int8_t* kb = k_idx + (size_t)b * Lk * kDIdx;
-  int32_t* out = scores + (size_t)row * row_stride;
-  uint4 kv[kKeysPerThread][4];
-  int vmn = INT_MAX, vmx = INT_MIN;
-#pragma unroll
-  for (int u = 0; u < kKeysPerThread; ++u) {
-    const int s = s_base + u * kStreamThreads;
-    if (s < n) {
-      const uint4* kp = reinterpret_cast<const uint4*>(kb + (size_t)s * kDIdx);
-#pragma unroll
-      for (int v = 0; v < 4; ++v) kv[u][v] = kp[v];
+    for (int j = 0; j < kHIdx; ++j) {
+      const int4 v = qrow[j * (kDIdx / 16) + part];
+      q[j][0] = v.x;
+      q[j][1] = v.y;
+      q[j][2] = v.z;
+      q[j][3] = v.w;
+      w[j] = w_idx[j];
     }
   }
+  const uint4* kb = reinterpret_cast<const uint4*>(k_idx + (size_t)b * Lk * kDIdx);
+  int32_t* out = scores + (size_t)row * row_stride;
+  int vmn = INT_MAX, vmx = INT_MIN;
+  const int warp_s0 = blockIdx.x * kStreamKeysPerCta + warp * (8 * kStreamLoads);
+  // key of load u in iteration it: warp_s0 + it*kStreamKeysPerIter + u*8 + lane/4
+  auto load_iter = [&](uint4 (&kv)[kStreamLoads], int it) {
 #pragma unroll
-  for (int u = 0; u < kKeysPerThread; ++u) {
-    const int s = s_base + u * kStreamThreads;
-    if (s < n) {
-      const int* kw = reinterpret_cast<const int*>(&kv[u][0]);
+    for (int u = 0; u < kStreamLoads; ++u) {
+      const int s = warp_s0 + it * kStreamKeysPerIter + u * 8 + (lane >> 2);
+      kv[u] = s < n ? __ldcs(kb + (size_t)s * 4 + part) : make_uint4(0u, 0u, 0u, 0u);
+    }
+  };
+  uint4 kv[2][kStreamLoads];
+  load_iter(kv[0], 0);
+#pragma unroll
+  for (int it = 0; it < kStreamIters; ++it) {
+    if (warp_s0 + it * kStreamKeysPerIter >= n) break;  // warp-uniform
+    if (it + 1 < kStreamIters) load_iter(kv[(it + 1) & 1], it + 1);  // next iteration's keys in flight
+#pragma unroll
+    for (int u = 0; u < kStreamLoads; ++u) {
+      const uint4 x = kv[it & 1][u];
+      const int s = warp_s0 + it * kStreamKeysPerIter + u * 8 + (lane >> 2);
       int total = 0;
 #pragma unroll
       for (int j = 0; j < kHIdx; ++j) {
-        int dot = 0;
-#pragma unroll
-        for (int i = 0; i < kDIdx / 4; ++i) dot = __dp4a(q[j * (kDIdx / 4) + i], kw[i], dot);
-        total += sw[j] * dot;
+        int dot = __dp4a(q[j][0], (int)x.x, 0);
+        dot = __dp4a(q[j][1], (int)x.y, dot);
+        dot = __dp4a(q[j][2], (int)x.z, dot);
+        dot = __dp4a(q[j][3], (int)x.w, dot);
+        total += w[j] * dot;
       }
-      out[s] = total;
-      vmn = min(vmn, total);
-      vmx = max(vmx, total);
+      total += __shfl_xor_sync(0xffffffffu, total, 1);
+      total += __shfl_xor_sync(0xffffffffu, total, 2);
+      if (part == 0 && s < n) {
+        out[s] = total;
+        vmn = min(vmn, total);
+        vmx = max(vmx, total);
+      }
     }
   }
   if (rowsel) {
@@ -257,7 +279,7 @@ __global__ void __launch_bounds__(kStreamThreads) score_stream_kernel(const int8
       vmn = min(vmn, __shfl_xor_sync(0xffffffffu, vmn, o));
       vmx = max(vmx, __shfl_xor_sync(0xffffffffu, vmx, o));
     }
-    if ((threadIdx.x & 31) == 0 && vmn <= vmx) {
+    if (lane == 0 && vmn <= vmx) {
       atomicMin(&rowsel[row].vmin, vmn);
       atomicMax(&rowsel[row].vmax, vmx);
     }
@@ -535,11 +557,66 @@ __global__ void __launch_bounds__(256) hist_kernel(const int32_t* __restrict__ s
   const int sh = hist_shift((unsigned)rs[row].vmax - (unsigned)vmin);
   const int* rowp = scores + (size_t)row * row_stride;
   const int c1 = min(c0 + kSplitChunk, n);
-#pragma unroll 8
-  for (int i = c0 + threadIdx.x; i < c1; i += 256) atomicAdd(&h[((unsigned)__ldcg(rowp + i) - (unsigned)vmin) >> sh], 1u);
+  // 4 scores per thread per load (rows are 16-byte aligned: c0 and the row stride are multiples of 128)
+  for (int base = c0; base < c1; base += 256 * 4 * 4) {
+    int4 v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int i = base + (u * 256 + threadIdx.x) * 4;
+      v[u] = i < c1 ? __ldcg(reinterpret_cast<const int4*>(rowp + i)) : make_int4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int i = base + (u * 256 + threadIdx.x) * 4;
+      const int e[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        if (i + q < c1) atomicAdd(&h[((unsigned)e[q] - (unsigned)vmin) >> sh], 1u);
+    }
+  }
   __syncthreads();
   for (int b = threadIdx.x; b < kHistBins; b += 256)
     if (h[b]) atomicAdd(&rs[row].hist[b], h[b]);
+}
+
+// The bin holding the k-th largest score of a row (bins counted from the top) and the number of
+// keys in the bins above it.  Whole block of kThreads threads; results in *bin_sh / *above_sh.
+template <int kThreads>
+__device__ __forceinline__ void threshold_bin(const unsigned int* __restrict__ hist, int k, int* wsum_sh, int* bin_sh,
+                                              int* above_sh) {
+  constexpr int kPer = kHistBins / kThreads;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  int cnt[kPer], tot = 0;
+#pragma unroll
+  for (int q = 0; q < kPer; ++q) {
+    cnt[q] = (int)hist[kHistBins - 1 - (tid * kPer + q)];
+    tot += cnt[q];
+  }
+  int incl = tot;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) wsum_sh[warp] = incl;
+  __syncthreads();
+  int before_warp = 0;
+  for (int w = 0; w < warp; ++w) before_warp += wsum_sh[w];
+  incl += before_warp;
+  const int above = incl - tot;
+  if (above < k && incl >= k) {
+    int acc = above;
+#pragma unroll
+    for (int q = 0; q < kPer; ++q) {
+      if (acc + cnt[q] >= k) {
+        *bin_sh = kHistBins - 1 - (tid * kPer + q);
+        *above_sh = acc;
+        break;
+      }
+      acc += cnt[q];
+    }
+  }
+  __syncthreads();
 }
 
 __global__ void __launch_bounds__(256) candidates_kernel(const int32_t* __restrict__ scores, RowSel* __restrict__ rs,
@@ -549,60 +626,49 @@ __global__ void __launch_bounds__(256) candidates_kernel(const int32_t* __restri
   const int n = max(0, min(q_offset + r + 1, Lk));
   const int c0 = blockIdx.x * kSplitChunk;
   if (n <= k || c0 >= n) return;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int tid = threadIdx.x, lane = tid & 31;
   __shared__ int wsum[8];
-  __shared__ int bstar;
-  // thread t counts bins [kHistBins - 8(t+1), kHistBins - 8t), i.e. from the top down
-  int cnt[8], tot = 0;
-#pragma unroll
-  for (int q = 0; q < 8; ++q) {
-    cnt[q] = (int)rs[row].hist[kHistBins - 1 - (tid * 8 + q)];
-    tot += cnt[q];
-  }
-  int incl = tot;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int y = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += y;
-  }
-  if (lane == 31) wsum[warp] = incl;
-  __syncthreads();
-  int before_warp = 0;
-  for (int w = 0; w < warp; ++w) before_warp += wsum[w];
-  incl += before_warp;
-  const int above = incl - tot;  // keys in bins above this thread's
-  if (above < k && incl >= k) {
-    int acc = above;
-#pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      if (acc + cnt[q] >= k) {
-        bstar = kHistBins - 1 - (tid * 8 + q);
-        break;
-      }
-      acc += cnt[q];
-    }
-  }
-  __syncthreads();
+  __shared__ int bstar, above_b;
+  threshold_bin<256>(rs[row].hist, k, wsum, &bstar, &above_b);
   const unsigned b_lo = (unsigned)bstar;
   const int vmin = rs[row].vmin;
   const int sh = hist_shift((unsigned)rs[row].vmax - (unsigned)vmin);
   const int* rowp = scores + (size_t)row * row_stride;
   int2* cr = cand + (size_t)row * kCandCap;
   const int c1 = min(c0 + kSplitChunk, n);
-  for (int base = c0; base < c1; base += 256) {  // warp-uniform trip count
-    const int i = base + tid;
-    unsigned u = 0;
-    bool take = false;
-    if (i < c1) {
-      u = (unsigned)__ldcg(rowp + i) - (unsigned)vmin;
-      take = (u >> sh) >= b_lo;
+  for (int base = c0; base < c1; base += 256 * 4 * 4) {  // warp-uniform trip count
+    int4 v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int i = base + (u * 256 + tid) * 4;
+      v[u] = i < c1 ? __ldcg(reinterpret_cast<const int4*>(rowp + i)) : make_int4(0, 0, 0, 0);
     }
-    const unsigned m = __ballot_sync(0xffffffffu, take);
-    if (m) {
-      int slot = 0;
-      if (lane == __ffs(m) - 1) slot = atomicAdd(&rs[row].n_cand, __popc(m));
-      slot = __shfl_sync(0xffffffffu, slot, __ffs(m) - 1) + __popc(m & ((1u << lane) - 1u));
-      if (take && slot < kCandCap) cr[slot] = make_int2((int)u, i);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int i = base + (u * 256 + tid) * 4;
+      const int e[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+      unsigned takes = 0;  // bit q: score i+q is a candidate
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        if (i + q < c1 && (((unsigned)e[q] - (unsigned)vmin) >> sh) >= b_lo) takes |= 1u << q;
+      if (!__any_sync(0xffffffffu, takes != 0)) continue;
+      // warp-aggregated append: exclusive prefix of the lanes' candidate counts
+      const int cnt = __popc(takes);
+      int incl = cnt;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      int slot0 = 0;
+      if (lane == 31) slot0 = atomicAdd(&rs[row].n_cand, incl);
+      int slot = __shfl_sync(0xffffffffu, slot0, 31) + incl - cnt;
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        if (takes & (1u << q)) {
+          if (slot < kCandCap) cr[slot] = make_int2((int)((unsigned)e[q] - (unsigned)vmin), i + q);
+          ++slot;
+        }
     }
   }
 }
@@ -650,26 +716,40 @@ __global__ void __launch_bounds__(kSelThreads) finalize_kernel(const int32_t* __
       select_row<false>(row_g, sel_row, n, k, out, sh);
     return;
   }
-  // candidates by (u desc, position asc): key = (~u) << 32 | position, ascending
-  unsigned long long* keys = reinterpret_cast<unsigned long long*>(sel_row);  // kCandCap keys
-  int P = 2;
-  while (P < nc) P <<= 1;
-  const int2* cr = cand + (size_t)row * kCandCap;
-  for (int i = threadIdx.x; i < P; i += kSelThreads) {
-    unsigned long long key = ~0ull;
-    if (i < nc) {
-      const int2 c = cr[i];
-      key = ((unsigned long long)(0xFFFFFFFFu - (unsigned)c.x) << 32) | (unsigned)c.y;
-    }
-    keys[i] = key;
+  // Keys in bins above b* are all selected; of the keys in bin b*, the (k - above) largest by
+  // (u desc, position asc).  Sort those few, then the k positions ascending.
+  __shared__ int wsum[kSelWarps];
+  __shared__ int bstar, above_b, n_tie, n_sure;
+  threshold_bin<kSelThreads>(rs[row].hist, k, wsum, &bstar, &above_b);
+  if (threadIdx.x == 0) {
+    n_tie = 0;
+    n_sure = 0;
   }
   __syncthreads();
+  const int sh_bits = hist_shift((unsigned)rs[row].vmax - (unsigned)rs[row].vmin);
+  int* pos = sel_row;                                                               // k positions (<= 4096)
+  unsigned long long* keys = reinterpret_cast<unsigned long long*>(sel_row + 4096);  // bin b*, <= kCandCap
+  const int2* cr = cand + (size_t)row * kCandCap;
+  for (int i = threadIdx.x; i < nc; i += kSelThreads) {
+    const int2 c = cr[i];
+    const int bin = (int)((unsigned)c.x >> sh_bits);
+    if (bin > bstar) {
+      pos[atomicAdd(&n_sure, 1)] = c.y;
+    } else {  // bin == bstar: every candidate is in a bin >= b*
+      keys[atomicAdd(&n_tie, 1)] = ((unsigned long long)(0xFFFFFFFFu - (unsigned)c.x) << 32) | (unsigned)c.y;
+    }
+  }
+  __syncthreads();
+  const int nt = n_tie, need = k - above_b;  // n_sure == above_b
+  int P = 2;
+  while (P < nt) P <<= 1;
+  for (int i = nt + threadIdx.x; i < P; i += kSelThreads) keys[i] = ~0ull;
+  __syncthreads();
   block_bitonic_sort(keys, P);
-  // the first k positions, ascending
-  int* pos = reinterpret_cast<int*>(keys + kCandCap);
+  for (int i = threadIdx.x; i < need; i += kSelThreads) pos[above_b + i] = (int)(keys[i] & 0xFFFFFFFFull);
   int Pk = 2;
   while (Pk < k) Pk <<= 1;
-  for (int i = threadIdx.x; i < Pk; i += kSelThreads) pos[i] = i < k ? (int)(keys[i] & 0xFFFFFFFFull) : INT_MAX;
+  for (int i = k + threadIdx.x; i < Pk; i += kSelThreads) pos[i] = INT_MAX;
   __syncthreads();
   block_bitonic_sort(pos, Pk);
   for (int i = threadIdx.x; i < k; i += kSelThreads) out[i] = pos[i];
@@ -728,8 +808,7 @@ extern "C" hcadsa_status dsa_index_topk(const int8_t* q_idx, const int8_t* k_idx
       score_tiled_kernel<<<grid, 256, smem_tiled, s>>>(q_idx, k_idx, w_idx, scores, Lq, q_offset, Lk, stride);
     } else {
       const long long n_max = stride;
-      dim3 grid((unsigned)((n_max + kStreamThreads * kKeysPerThread - 1) / (kStreamThreads * kKeysPerThread)),
-                (unsigned)(B * Lq));
+      dim3 grid((unsigned)((n_max + kStreamKeysPerCta - 1) / kStreamKeysPerCta), (unsigned)(B * Lq));
       if (grid.y > 65535u) return HCADSA_ERR_UNSUPPORTED;
       score_stream_kernel<<<grid, kStreamThreads, 0, s>>>(q_idx, k_idx, w_idx, scores, Lq, q_offset, Lk, stride,
                                                            rowsel);
@@ -818,8 +897,7 @@ extern "C" hcadsa_status dsa_index_topk_noalloc(const int8_t* q_idx, const int8_
         return HCADSA_ERR_CUDA;
       score_tiled_kernel<<<grid, 256, smem_tiled, s>>>(q_idx, k_idx, w_idx, scores, Lq, q_offset, Lk, stride);
     } else {
-      dim3 grid((unsigned)((stride + kStreamThreads * kKeysPerThread - 1) / (kStreamThreads * kKeysPerThread)),
-                (unsigned)(B * Lq));
+      dim3 grid((unsigned)((stride + kStreamKeysPerCta - 1) / kStreamKeysPerCta), (unsigned)(B * Lq));
       if (grid.y > 65535u) return HCADSA_ERR_UNSUPPORTED;
       score_stream_kernel<<<grid, kStreamThreads, 0, s>>>(q_idx, k_idx, w_idx, scores, Lq, q_offset, Lk, stride,
                                                            nullptr);

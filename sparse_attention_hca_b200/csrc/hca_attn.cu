@@ -648,15 +648,16 @@ __global__ void __launch_bounds__(kThreads, 1) hca_attn_kernel(const __grid_cons
 // Split key ranges: row r of row tile T gathers its units' partial results,
 //     M = max_s m_s,  w_s = 2^(m_s - M),  O = sum_s w_s O_s / sum_s w_s l_s,
 // (m_s in log2 units, O_s and l_s relative to 2^m_s) and writes O (bf16) and lse.
-// One CTA per row tile, one warp per row at a time, 4 columns per lane per step.
+// One warp per row (8 rows per CTA, blockIdx.y = row group), 4 columns per lane per step.
 __global__ void __launch_bounds__(256) hca_combine_kernel(const Params p, uint16_t* __restrict__ O) {
   const int T = blockIdx.x;
   const int bh = T / p.n_tiles, tile = T % p.n_tiles;
   const int b = bh / p.Hkv, hk = bh % p.Hkv;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  for (int r = warp; r < 128; r += 8) {
+  {
+    const int r = blockIdx.y * 8 + warp;
     const int tok = tile * p.TT + r / p.g;
-    if (tok >= p.Lq) continue;
+    if (tok >= p.Lq) return;
     const int h = hk * p.g + r % p.g;
     float M = -INFINITY;
     for (int sp = 0; sp < p.splits; ++sp) M = fmaxf(M, p.part_ml[((size_t)T * p.splits + sp) * 128 + r].x);
@@ -855,7 +856,10 @@ extern "C" hcadsa_status hca_attn_fwd(const hcadsa_bf16* Q, const hcadsa_bf16* K
   if (G.splits > 1) {
     const hcadsa_status st = launch_status();
     if (st != HCADSA_OK) return st;
-    hca_combine_kernel<<<G.total_tiles, 256, 0, as_stream(stream)>>>(p, reinterpret_cast<uint16_t*>(O));
+    // only row groups holding a valid token: 8 rows per CTA
+    const int valid_rows = Lq < G.TT ? Lq * g : 128;
+    hca_combine_kernel<<<dim3((unsigned)G.total_tiles, (unsigned)((valid_rows + 7) / 8)), 256, 0, as_stream(stream)>>>(
+        p, reinterpret_cast<uint16_t*>(O));
   }
   return launch_status();
 }
