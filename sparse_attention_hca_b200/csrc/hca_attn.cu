@@ -78,14 +78,16 @@ struct Params {
   int Lq, q_offset, Hq, Hkv, g, TT, n_c, win_start, W, blk;
   int n_tiles;      // token tiles per (b, kv head)
   int total_tiles;  // B * Hkv * n_tiles
-  int splits;       // work units per row tile (key tiles split among them; 1 = no split)
-  int total_units;  // total_tiles * splits
+  int splits;       // work units per row tile (key tiles split among them) ...
+  int split_extra;  // ... plus one more for the first split_extra row tiles
+  int split_mode;   // units write partial results for the combine pass
+  int total_units;  // total_tiles * splits + split_extra
   int J_max;        // key tiles of the longest row tile (scratch capacity)
   float scale_log2;
   float* lse;
   uint8_t* scratch;  // gridDim.x * J_max * kScratchTileBytes
-  float* part_o;     // splits > 1: [total_units][128][512] unnormalised O of each unit
-  float2* part_ml;   // splits > 1: [total_units][128] (reference max in log2 units, row sum)
+  float* part_o;     // split mode: [total_units][128][512] unnormalised O of each unit
+  float2* part_ml;   // split mode: [total_units][128] (reference max in log2 units, row sum)
   int* err;
 };
 
@@ -116,8 +118,11 @@ struct KeyTile {
   int n;       // MMA N (multiple of 16, <= 128)
 };
 
-// The key tiles of one work unit: split s of row tile T (unit U = T * splits + s) takes the
-// row tile's key tiles [s*Jt/splits, (s+1)*Jt/splits).
+__host__ __device__ inline int first_unit(int T, const Params& p) { return T * p.splits + min(T, p.split_extra); }
+__host__ __device__ inline int n_splits(int T, const Params& p) { return p.splits + (T < p.split_extra ? 1 : 0); }
+
+// The key tiles of one work unit: split s of row tile T (S = n_splits(T) units from
+// first_unit(T)) takes the row tile's key tiles [s*Jt/S, (s+1)*Jt/S).
 struct TileSet {
   int b, hk, tok0;  // batch, kv head, first token (relative to q_offset)
   int J_c, J;       // number of compressed tiles of the row tile, key tiles of this unit
@@ -126,7 +131,9 @@ struct TileSet {
   int ws_lo;        // window start of the first token
   int t_hi;         // last valid token position
   __device__ void init(int U, const Params& p) {
-    const int T = U / p.splits, split = U % p.splits;
+    const int big = p.split_extra * (p.splits + 1);  // units of the row tiles with an extra split
+    const int T = U < big ? U / (p.splits + 1) : p.split_extra + (U - big) / p.splits;
+    const int split = U - first_unit(T, p), S = n_splits(T, p);
     const int bh = T / p.n_tiles, tile = T % p.n_tiles;
     b = bh / p.Hkv;
     hk = bh % p.Hkv;
@@ -136,8 +143,8 @@ struct TileSet {
     ws_lo = window_start(p.q_offset + tok0, p.W);
     J_c = (nc_hi + kKeyTile - 1) / kKeyTile;
     const int Jt = J_c + (t_hi - ws_lo + kKeyTile) / kKeyTile;
-    js = split * Jt / p.splits;
-    J = (split + 1) * Jt / p.splits - js;
+    js = split * Jt / S;
+    J = (split + 1) * Jt / S - js;
   }
   __device__ KeyTile get(int jl) const {
     KeyTile kt;
@@ -242,7 +249,7 @@ __global__ void __launch_bounds__(kThreads, 1) hca_attn_kernel(const __grid_cons
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       tma_prefetch_desc(&maps.q);
-      const uint32_t ngroups = p.splits > 1 ? kMaxGroups : kGroups;
+      const uint32_t ngroups = p.split_mode ? kMaxGroups : kGroups;
       uint32_t grp = 0, gph = 0;  // next ring group to fill and the phase of its use
       bool ok = true;
       // two 64-column chunks (columns col .. col+127 of a key tile) into the next ring group
@@ -309,7 +316,7 @@ __global__ void __launch_bounds__(kThreads, 1) hca_attn_kernel(const __grid_cons
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t sQa = smem_u32(sQ), sRa = smem_u32(sRing);
-      const uint32_t ngroups = p.splits > 1 ? kMaxGroups : kGroups;
+      const uint32_t ngroups = p.split_mode ? kMaxGroups : kGroups;
       uint32_t grp = 0, gph = 0;  // next ring group to consume and the phase of its use
       auto next_group = [&]() {
         if (++grp == ngroups) {
@@ -438,7 +445,7 @@ __global__ void __launch_bounds__(kThreads, 1) hca_attn_kernel(const __grid_cons
       ok = mbar_wait(&bar.o_full, it & 1, &abort_flag, p.err);
       if (!ok) return;
       tc_fence_after();
-      if (p.splits > 1) {
+      if (p.split_mode) {
         for (int hh = 0; hh < 2; ++hh) {
           for (int oc = 0; oc < 128; oc += 32) {
             uint32_t v[32];
@@ -586,7 +593,7 @@ __global__ void __launch_bounds__(kThreads, 1) hca_attn_kernel(const __grid_cons
       }
       if (!ok) break;
       float inv_l = l_run > 0.0f ? 1.0f / l_run : 0.0f;
-      if (p.splits > 1) {  // the combine pass normalises
+      if (p.split_mode) {  // the combine pass normalises
         inv_l = 1.0f;
         if (row_valid) p.part_ml[(size_t)T * 128 + r] = make_float2(m_ref, l_run);
       } else if (p.lse && row_valid) {
@@ -660,18 +667,19 @@ __global__ void __launch_bounds__(256) hca_combine_kernel(const Params p, uint16
     if (tok >= p.Lq) return;
     const int h = hk * p.g + r % p.g;
     float M = -INFINITY;
-    for (int sp = 0; sp < p.splits; ++sp) M = fmaxf(M, p.part_ml[((size_t)T * p.splits + sp) * 128 + r].x);
+    const int U0 = first_unit(T, p), S = n_splits(T, p);
+    for (int sp = 0; sp < S; ++sp) M = fmaxf(M, p.part_ml[((size_t)U0 + sp) * 128 + r].x);
     float L = 0.0f;
-    for (int sp = 0; sp < p.splits; ++sp) {
-      const float2 ml = p.part_ml[((size_t)T * p.splits + sp) * 128 + r];
+    for (int sp = 0; sp < S; ++sp) {
+      const float2 ml = p.part_ml[((size_t)U0 + sp) * 128 + r];
       L += ml.y > 0.0f ? exp2f(ml.x - M) * ml.y : 0.0f;
     }
     const float inv_L = L > 0.0f ? 1.0f / L : 0.0f;
     uint16_t* orow = O + (((size_t)b * p.Lq + tok) * p.Hq + h) * kD;
     for (int c = lane * 4; c < kD; c += 128) {
       float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int sp = 0; sp < p.splits; ++sp) {
-        const size_t U = (size_t)T * p.splits + sp;
+      for (int sp = 0; sp < S; ++sp) {
+        const size_t U = (size_t)U0 + sp;
         const float2 ml = p.part_ml[U * 128 + r];
         if (!(ml.y > 0.0f)) continue;
         const float w = exp2f(ml.x - M);
@@ -710,9 +718,9 @@ int num_sms() {
 // Launch geometry shared by the workspace query and the launch: HCADSA_ERR_UNSUPPORTED for
 // shapes the kernel does not take, HCADSA_ERR_CUDA if the device cannot be queried.
 struct Geometry {
-  int g, TT, n_tiles, total_tiles, splits, total_units, grid, J_max;
+  int g, TT, n_tiles, total_tiles, splits, split_extra, total_units, grid, J_max;
   size_t scratch_bytes;   // probability tiles: grid * J_max * kScratchTileBytes
-  size_t part_bytes;      // splits > 1: unnormalised O rows and (max, sum) of every unit
+  size_t part_bytes;      // split mode: unnormalised O rows and (max, sum) of every unit
   size_t workspace_bytes;
 };
 
@@ -744,7 +752,7 @@ hcadsa_status geometry(Geometry* G, int B, int Lq, int q_offset, int Hq, int Hkv
   if (sms <= 0) return HCADSA_ERR_CUDA;
   // Few row tiles (decode: one token per sequence) leave most SMs idle: split every row tile's
   // key tiles into `splits` units (each unit keeps at least one key tile) and combine after.
-  long long splits = 1;
+  long long splits = 1, extra = 0;
   if (2 * total <= sms) {
     long long J_min = J_max;
     for (long long t = 0; t < n_tiles; ++t) {
@@ -752,21 +760,31 @@ hcadsa_status geometry(Geometry* G, int B, int Lq, int q_offset, int Hq, int Hkv
       const long long J = host_tile_J(q_offset, tok0, tok_hi, W, blk);
       J_min = J < J_min ? J : J_min;
     }
+    // one unit per SM: sms / total units per row tile, one more for the first sms % total
+    // (two units per SM balance the key tiles better but measured slower at B = 32, t = 1M:
+    // 148 us against 136 us, the per-unit fixed costs outweigh it)
     splits = sms / total;
-    if (splits > J_min) splits = J_min;
-    if (splits > 64) splits = 64;
-    if (splits < 1) splits = 1;
+    extra = sms % total;
+    if (splits + (extra ? 1 : 0) > J_min) {
+      splits = J_min;
+      extra = 0;
+    }
+    if (splits > 64) {
+      splits = 64;
+      extra = 0;
+    }
   }
   G->g = g;
   G->TT = TT;
   G->n_tiles = (int)n_tiles;
   G->total_tiles = (int)total;
   G->splits = (int)splits;
-  G->total_units = (int)(total * splits);
+  G->split_extra = (int)extra;
+  G->total_units = (int)(total * splits + extra);
   G->grid = G->total_units < sms ? G->total_units : sms;
   G->J_max = (int)J_max;
   G->scratch_bytes = (size_t)G->grid * (size_t)J_max * kScratchTileBytes;
-  G->part_bytes = splits > 1 ? (size_t)G->total_units * 128 * (kD * 4 + 8) : 0;
+  G->part_bytes = G->total_units > G->total_tiles ? (size_t)G->total_units * 128 * (kD * 4 + 8) : 0;
   G->workspace_bytes = G->scratch_bytes + G->part_bytes;
   return HCADSA_OK;
 }
@@ -841,19 +859,21 @@ extern "C" hcadsa_status hca_attn_fwd(const hcadsa_bf16* Q, const hcadsa_bf16* K
   p.n_tiles = G.n_tiles;
   p.total_tiles = G.total_tiles;
   p.splits = G.splits;
+  p.split_extra = G.split_extra;
+  p.split_mode = G.total_units > G.total_tiles ? 1 : 0;
   p.total_units = G.total_units;
   p.J_max = G.J_max;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.lse = lse;
   p.scratch = static_cast<uint8_t*>(workspace);
-  p.part_o = G.splits > 1 ? reinterpret_cast<float*>(p.scratch + G.scratch_bytes) : nullptr;
-  p.part_ml = G.splits > 1 ? reinterpret_cast<float2*>(p.scratch + G.scratch_bytes + (size_t)G.total_units * 128 * kD * 4)
+  p.part_o = p.split_mode ? reinterpret_cast<float*>(p.scratch + G.scratch_bytes) : nullptr;
+  p.part_ml = p.split_mode ? reinterpret_cast<float2*>(p.scratch + G.scratch_bytes + (size_t)G.total_units * 128 * kD * 4)
                            : nullptr;
   p.err = device_error_ptr();
   if (cudaFuncSetAttribute(hca_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) != cudaSuccess)
     return HCADSA_ERR_CUDA;
   hca_attn_kernel<<<G.grid, kThreads, kSmemBytes, as_stream(stream)>>>(maps, p);
-  if (G.splits > 1) {
+  if (p.split_mode) {
     const hcadsa_status st = launch_status();
     if (st != HCADSA_OK) return st;
     // only row groups holding a valid token: 8 rows per CTA

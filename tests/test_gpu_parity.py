@@ -218,6 +218,26 @@ def test_hca_split_key_ranges(hd):
     np.testing.assert_allclose(lse.reshape(B * Lq, Hq).cpu().numpy(), ref_lse, atol=2e-2, rtol=0)
 
 
+def test_hca_decode_uneven_splits(hd):
+    """32 sequences at t = 200000: the key tiles of the 32 row tiles are split over the SMs
+    unevenly (some row tiles get one more unit) and recombined."""
+    d, Hq, blk, W, B, t = 512, 16, 128, 128, 32, 200000
+    n_c = (t + 1) // blk
+    ws = t - W + 1
+    Kc = synth.normal_bf16((B, n_c, 1, d), 1.0, 51, "K")
+    Vc = synth.normal_bf16((B, n_c, 1, d), 1.0, 51, "V")
+    Kw = synth.normal_bf16((B, W, 1, d), 1.0, 52, "K")
+    Vw = synth.normal_bf16((B, W, 1, d), 1.0, 52, "V")
+    Q = synth.normal_bf16((B, 1, Hq, d), 1.0, 53, "Q")
+    O, lse = hd.hca_attn_fwd(Q.cuda(), Kc.cuda(), Vc.cuda(), Kw.cuda(), Vw.cuda(), win_start=ws, q_offset=t,
+                             return_lse=True)
+    no_device_error(hd)
+    ref, ref_lse = oracle.hca_attn(bits(Q), bits(Kc), bits(Vc), bits(Kw), bits(Vw), win_start=ws, q_offset=t,
+                                   with_lse=True)
+    print(check_attn(O.reshape(B, Hq, d), ref, "hca decode uneven splits"))
+    np.testing.assert_allclose(lse.reshape(B, Hq).cpu().numpy(), ref_lse, atol=2e-2, rtol=0)
+
+
 # ------------------------------------------------------------------ DSA indexer + top-k
 
 def _dsa_cfg(name, L, B=1, k=2048, sigma=None):
