@@ -408,56 +408,110 @@ __device__ void select_row(const int* __restrict__ row_g, int* row_s, int n, int
   int nbits = range == 0 ? 0 : 32 - __clz((int)range);
   unsigned prefix = 0, pmask = 0;
   int remaining = k;  // rank (1 = largest) still to locate among the prefix matches
-  while (nbits > 0) {
-    const int dbits = nbits < kDigitBits ? nbits : kDigitBits;
-    const int lo = nbits - dbits;
-    const unsigned dmask = (1u << dbits) - 1u;
-    unsigned int* hw = sh.hist[warp];
-    for (int b = lane; b < kDigitBins; b += 32) hw[b] = 0;
-    __syncwarp();
-    for (int i = tid; i < n; i += kSelThreads) {
-      const unsigned u = (unsigned)at(i) - (unsigned)vmin;
-      if ((u & pmask) == prefix) atomicAdd(&hw[(u >> lo) & dmask], 1u);
-    }
-    __syncthreads();
-    if (warp == 0) {
-      // lane l owns bins 255 - 8l - q, q = 0..7: counts from the top down
-      int cnt[8];
-      int lane_tot = 0;
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        const int bin = kDigitBins - 1 - (lane * 8 + q);
-        int c = 0;
-        for (int w = 0; w < kSelWarps; ++w) c += (int)sh.hist[w][bin];
-        cnt[q] = c;
-        lane_tot += c;
+  if (kInSmem) {
+    // 11-bit digits counted into one block-wide 2048-bin histogram (the per-warp histograms'
+    // storage): two passes cover the 18-bit score range of the indexer's usual inputs
+    constexpr int kBins = 2048, kPer = kBins / kSelThreads;
+    unsigned int* hb = &sh.hist[0][0];
+    while (nbits > 0) {
+      const int dbits = nbits < 11 ? nbits : 11;
+      const int lo = nbits - dbits;
+      const unsigned dmask = (1u << dbits) - 1u;
+      for (int b = tid; b < kBins; b += kSelThreads) hb[b] = 0;
+      __syncthreads();
+      for (int i = tid; i < n; i += kSelThreads) {
+        const unsigned u = (unsigned)row_s[i] - (unsigned)vmin;
+        if ((u & pmask) == prefix) atomicAdd(&hb[(u >> lo) & dmask], 1u);
       }
-      int incl = lane_tot;
+      __syncthreads();
+      // thread t owns bins kBins-1-(t*kPer+q), q < kPer: counts from the top down
+      int cnt[kPer], tot = 0;
+#pragma unroll
+      for (int q = 0; q < kPer; ++q) {
+        cnt[q] = (int)hb[kBins - 1 - (tid * kPer + q)];
+        tot += cnt[q];
+      }
+      int incl = tot;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
         const int y = __shfl_up_sync(0xffffffffu, incl, o);
         if (lane >= o) incl += y;
       }
-      const int above = incl - lane_tot;  // elements in higher bins than this lane's
+      if (lane == 31) sh.red_a[warp] = incl;
+      __syncthreads();
+      for (int w = 0; w < warp; ++w) incl += sh.red_a[w];
+      const int above = incl - tot;
       if (above < remaining && incl >= remaining) {
         int acc = above;
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
+        for (int q = 0; q < kPer; ++q) {
           if (acc + cnt[q] >= remaining) {
-            sh.bcast[2] = kDigitBins - 1 - (lane * 8 + q);
+            sh.bcast[2] = kBins - 1 - (tid * kPer + q);
             sh.bcast[3] = remaining - acc;
             break;
           }
           acc += cnt[q];
         }
       }
+      __syncthreads();
+      prefix |= (unsigned)sh.bcast[2] << lo;
+      pmask |= dmask << lo;
+      remaining = sh.bcast[3];
+      nbits = lo;
+      __syncthreads();  // red_a and the histogram are rewritten by the next pass
     }
-    __syncthreads();
-    prefix |= (unsigned)sh.bcast[2] << lo;
-    pmask |= dmask << lo;
-    remaining = sh.bcast[3];
-    nbits = lo;
-    __syncthreads();  // histograms are cleared again by the next pass
+  } else {
+    while (nbits > 0) {
+      const int dbits = nbits < kDigitBits ? nbits : kDigitBits;
+      const int lo = nbits - dbits;
+      const unsigned dmask = (1u << dbits) - 1u;
+      unsigned int* hw = sh.hist[warp];
+      for (int b = lane; b < kDigitBins; b += 32) hw[b] = 0;
+      __syncwarp();
+      for (int i = tid; i < n; i += kSelThreads) {
+        const unsigned u = (unsigned)at(i) - (unsigned)vmin;
+        if ((u & pmask) == prefix) atomicAdd(&hw[(u >> lo) & dmask], 1u);
+      }
+      __syncthreads();
+      if (warp == 0) {
+        // lane l owns bins 255 - 8l - q, q = 0..7: counts from the top down
+        int cnt[8];
+        int lane_tot = 0;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const int bin = kDigitBins - 1 - (lane * 8 + q);
+          int c = 0;
+          for (int w = 0; w < kSelWarps; ++w) c += (int)sh.hist[w][bin];
+          cnt[q] = c;
+          lane_tot += c;
+        }
+        int incl = lane_tot;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int y = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += y;
+        }
+        const int above = incl - lane_tot;  // elements in higher bins than this lane's
+        if (above < remaining && incl >= remaining) {
+          int acc = above;
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            if (acc + cnt[q] >= remaining) {
+              sh.bcast[2] = kDigitBins - 1 - (lane * 8 + q);
+              sh.bcast[3] = remaining - acc;
+              break;
+            }
+            acc += cnt[q];
+          }
+        }
+      }
+      __syncthreads();
+      prefix |= (unsigned)sh.bcast[2] << lo;
+      pmask |= dmask << lo;
+      remaining = sh.bcast[3];
+      nbits = lo;
+      __syncthreads();  // histograms are cleared again by the next pass
+    }
   }
   const unsigned thr = prefix;    // u of the k-th largest
   const int need_eq = remaining;  // elements equal to thr that are kept (lowest positions first)
