@@ -115,8 +115,8 @@ __device__ __forceinline__ uint32_t tile_mask_of_row(const int32_t* row, int k, 
   for (int j = 0; j < n_tiles; ++j) {
     bool any = false;
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int e = j * kKeyTile + lane * 4 + q;
+    for (int q = 0; q < 4; ++q) {  // consecutive lanes read consecutive words: no bank conflicts
+      const int e = j * kKeyTile + q * 32 + lane;
       if (e < k) any |= idx_ok(row[e], Lk);
     }
     if (__any_sync(0xffffffffu, any)) mask |= 1u << j;

@@ -536,9 +536,14 @@ __global__ void __launch_bounds__(kThreads, 1) hca_attn_kernel(const __grid_cons
           uint32_t v[32];
           tmem_ld32_nowait(tS + c0, v);
           tmem_wait_ld_regs(v);
+          if (__all_sync(0xffffffffu, lo <= c0 && c0 + 32 <= hi)) {  // chunk visible to every row
 #pragma unroll
-          for (int i = 0; i < 32; ++i)
-            if ((uint32_t)(c0 + i - lo) < vis_n) mx = fmaxf(mx, __uint_as_float(v[i]));
+            for (int i = 0; i < 32; ++i) mx = fmaxf(mx, __uint_as_float(v[i]));
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              if ((uint32_t)(c0 + i - lo) < vis_n) mx = fmaxf(mx, __uint_as_float(v[i]));
+          }
         }
         const float m_tile = mx * p.scale_log2;  // -inf stays -inf
         bool need = false;
@@ -572,14 +577,27 @@ __global__ void __launch_bounds__(kThreads, 1) hca_attn_kernel(const __grid_cons
             tmem_ld32_nowait(tS + q4 * 32, v);
             tmem_wait_ld_regs(v);
             uint32_t pk[16];
+            const int c0 = q4 * 32;
+            if (__all_sync(0xffffffffu, vis_p != 0u && lo <= c0 && c0 + 32 <= hi)) {  // chunk visible to every row
+              float ls = 0.0f;
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const int c = q4 * 32 + 2 * i;
-              float p0 = 0.0f, p1 = 0.0f;
-              if ((uint32_t)(c - lo) < vis_p) p0 = fast_exp2(__uint_as_float(v[2 * i]) * p.scale_log2 - m_ref);
-              if ((uint32_t)(c + 1 - lo) < vis_p) p1 = fast_exp2(__uint_as_float(v[2 * i + 1]) * p.scale_log2 - m_ref);
-              l_run += p0 + p1;
-              pk[i] = pack_bf16x2(p0, p1);
+              for (int i = 0; i < 16; ++i) {
+                const float p0 = fast_exp2(fmaf(__uint_as_float(v[2 * i]), p.scale_log2, -m_ref));
+                const float p1 = fast_exp2(fmaf(__uint_as_float(v[2 * i + 1]), p.scale_log2, -m_ref));
+                ls += p0 + p1;
+                pk[i] = pack_bf16x2(p0, p1);
+              }
+              l_run += ls;
+            } else {
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                const int c = c0 + 2 * i;
+                float p0 = 0.0f, p1 = 0.0f;
+                if ((uint32_t)(c - lo) < vis_p) p0 = fast_exp2(fmaf(__uint_as_float(v[2 * i]), p.scale_log2, -m_ref));
+                if ((uint32_t)(c + 1 - lo) < vis_p) p1 = fast_exp2(fmaf(__uint_as_float(v[2 * i + 1]), p.scale_log2, -m_ref));
+                l_run += p0 + p1;
+                pk[i] = pack_bf16x2(p0, p1);
+              }
             }
             tmem_st16(tS + q4 * 16, pk);
 #pragma unroll
