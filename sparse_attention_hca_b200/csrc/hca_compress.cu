@@ -5,9 +5,9 @@
 // page -- only say that 128 tokens become one entry).
 //
 // The work is a pure HBM stream.  Persistent CTAs walk work units (tensor, batch, block,
-// 128-channel column group).  One thread streams each unit's rows into a 6-stage ring of
-// shared-memory boxes (TMA, up to 128 rows x 128 channels = 32 KB per box) so plenty of
-// bytes are in flight per SM; two warps then run the sequential FMA chains from shared
+// 256-channel column group).  One thread streams each unit's rows into a 3-stage ring of
+// shared-memory boxes (TMA, up to 128 rows x 256 channels = 64 KB per box) so plenty of
+// bytes are in flight per SM; four warps then run the sequential FMA chains from shared
 // memory, two channels per thread, rows in ascending order -- exactly the fixed
 // accumulation order, so results are bit-identical to a plain loop.
 #include <cuda_bf16.h>
@@ -20,11 +20,11 @@
 namespace hcadsa {
 namespace {
 
-constexpr int kCols = 128;            // channels per work unit (TMA box width)
+constexpr int kCols = 256;            // channels per work unit (TMA box width)
 constexpr int kBoxRows = 128;         // rows per TMA box
-constexpr int kStages = 6;
-constexpr int kBoxBytes = kCols * kBoxRows * 2;  // 32 KB
-constexpr int kConsumerWarps = 2;     // 64 threads x 2 channels = 128 channels
+constexpr int kStages = 3;
+constexpr int kBoxBytes = kCols * kBoxRows * 2;  // 64 KB
+constexpr int kConsumerWarps = 4;     // 128 threads x 2 channels = 256 channels
 constexpr int kThreads = 32 * (kConsumerWarps + 1);
 constexpr int kSmemBytes = kStages * kBoxBytes + 128;
 
@@ -80,7 +80,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   // -------------------------------------------------------------- consumers: FMA chains
-  const int col = threadIdx.x * 2;  // 2 channels of the unit's kCols
+  const int col = threadIdx.x * 2;  // 2 channels of the unit's 256
   uint32_t q = 0;
   for (int u = blockIdx.x; u < p.n_units; u += gridDim.x) {
     const int cg = u % p.col_groups;
@@ -141,7 +141,7 @@ extern "C" hcadsa_status hca_compress_kv(const hcadsa_bf16* K, const hcadsa_bf16
   const long long col_groups = (row_elems + kCols - 1) / kCols;
   const long long n_units = 2LL * B * n_c * col_groups;
   if (n_units > 2147483647LL) return HCADSA_ERR_UNSUPPORTED;
-  // [rows, row_elems] bf16, box = 128 rows x 128 channels, no swizzle; box parts past the last
+  // [rows, row_elems] bf16, box = 128 rows x 256 channels, no swizzle; box parts past the last
   // row or the last channel are zero-filled and never stored
   CUtensorMap mk, mv;
   const uint64_t dims[2] = {(uint64_t)row_elems, (uint64_t)rows};
