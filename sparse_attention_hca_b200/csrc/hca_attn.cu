@@ -673,7 +673,8 @@ __global__ void __launch_bounds__(kThreads, 1) hca_attn_kernel(const __grid_cons
 // Split key ranges: row r of row tile T gathers its units' partial results,
 //     M = max_s m_s,  w_s = 2^(m_s - M),  O = sum_s w_s O_s / sum_s w_s l_s,
 // (m_s in log2 units, O_s and l_s relative to 2^m_s) and writes O (bf16) and lse.
-// One warp per row (8 rows per CTA, blockIdx.y = row group), 4 columns per lane per step.
+// One warp per row (8 rows per CTA, blockIdx.y = row group) and 128-column slice (blockIdx.z),
+// 4 columns per lane.
 __global__ void __launch_bounds__(256) hca_combine_kernel(const Params p, uint16_t* __restrict__ O) {
   const int T = blockIdx.x;
   const int bh = T / p.n_tiles, tile = T % p.n_tiles;
@@ -694,7 +695,8 @@ __global__ void __launch_bounds__(256) hca_combine_kernel(const Params p, uint16
     }
     const float inv_L = L > 0.0f ? 1.0f / L : 0.0f;
     uint16_t* orow = O + (((size_t)b * p.Lq + tok) * p.Hq + h) * kD;
-    for (int c = lane * 4; c < kD; c += 128) {
+    {
+      const int c = blockIdx.z * 128 + lane * 4;  // this CTA's 128-column slice of the row
       float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
       for (int sp = 0; sp < S; ++sp) {
         const size_t U = (size_t)U0 + sp;
@@ -710,7 +712,8 @@ __global__ void __launch_bounds__(256) hca_combine_kernel(const Params p, uint16
       *reinterpret_cast<uint2*>(orow + c) =
           make_uint2(pack_bf16x2(acc.x * inv_L, acc.y * inv_L), pack_bf16x2(acc.z * inv_L, acc.w * inv_L));
     }
-    if (lane == 0 && p.lse) p.lse[((size_t)b * p.Lq + tok) * p.Hq + h] = (M + __log2f(L)) * 0.69314718055994531f;
+    if (blockIdx.z == 0 && lane == 0 && p.lse)
+      p.lse[((size_t)b * p.Lq + tok) * p.Hq + h] = (M + __log2f(L)) * 0.69314718055994531f;
   }
 }
 
@@ -896,7 +899,8 @@ extern "C" hcadsa_status hca_attn_fwd(const hcadsa_bf16* Q, const hcadsa_bf16* K
     if (st != HCADSA_OK) return st;
     // only row groups holding a valid token: 8 rows per CTA
     const int valid_rows = Lq < G.TT ? Lq * g : 128;
-    hca_combine_kernel<<<dim3((unsigned)G.total_tiles, (unsigned)((valid_rows + 7) / 8)), 256, 0, as_stream(stream)>>>(
+    hca_combine_kernel<<<dim3((unsigned)G.total_tiles, (unsigned)((valid_rows + 7) / 8), kD / 128), 256, 0,
+                         as_stream(stream)>>>(
         p, reinterpret_cast<uint16_t*>(O));
   }
   return launch_status();
