@@ -191,7 +191,7 @@ __device__ __forceinline__ void load_p_row(uint4 (&pr)[16], float& alpha, uint8_
 #pragma unroll
   for (int c = 0; c < 16; ++c)
     pr[c] = c * 8 < n ? __ldcg(src + c * 128) : make_uint4(0u, 0u, 0u, 0u);
-  alpha = __ldcg(scratch_alpha(base, j, r));
+  alpha = n > 0 ? __ldcg(scratch_alpha(base, j, r)) : 1.0f;
 }
 
 // Multiplies this thread's row of the O half by alpha.
@@ -566,7 +566,9 @@ __global__ void __launch_bounds__(kThreads, 1) hca_attn_kernel(const __grid_cons
           l_run *= alpha;
           rescale_o(tmem + lane_off, alpha);
         }
-        *scratch_alpha(scratch, j, r) = alpha;
+        // rows that belong to no token (a partial last tile, decode tiles) keep nothing in the
+        // scratch: their P and O rows are never stored, so phase B leaves them unloaded
+        if (row_valid) *scratch_alpha(scratch, j, r) = alpha;
         // pass 2: P = exp2(s*scale*log2e - m_ref) as bf16, in place over S and into the scratch
         const uint32_t vis_p = m_ref != -INFINITY ? vis_n : 0u;
         uint4* prow = scratch_p(scratch, j, r);
@@ -600,9 +602,11 @@ __global__ void __launch_bounds__(kThreads, 1) hca_attn_kernel(const __grid_cons
               }
             }
             tmem_st16(tS + q4 * 16, pk);
+            if (row_valid) {
 #pragma unroll
-            for (int u = 0; u < 4; ++u)
-              __stcg(prow + (q4 * 4 + u) * 128, make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]));
+              for (int u = 0; u < 4; ++u)
+                __stcg(prow + (q4 * 4 + u) * 128, make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]));
+            }
           }
         }
         tmem_wait_st();
@@ -626,7 +630,8 @@ __global__ void __launch_bounds__(kThreads, 1) hca_attn_kernel(const __grid_cons
         const KeyTile kt = ts.get(j);
         uint4 pr[16];
         float alpha;
-        load_p_row(pr, alpha, scratch, j, kt.n, r);
+        load_p_row(pr, alpha, scratch, j, row_valid ? kt.n : 0, r);
+        if (!row_valid) alpha = 1.0f;
         if (gs >= 2) {  // S buffer gs&1 is free once PV_{gs-2} has read its P
           ok = mbar_wait(&bar.pv_done[gs & 1], ((gs >> 1) - 1) & 1, &abort_flag, p.err);
           if (!ok) break;
