@@ -129,7 +129,11 @@ extern "C" const char* hcadsa_status_string(hcadsa_status status) {
 
 extern "C" hcadsa_status hcadsa_check_device_error(hcadsa_stream stream) {
   using namespace hcadsa;
-  if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return HCADSA_ERR_CUDA;
+  const cudaError_t se = cudaStreamSynchronize(as_stream(stream));
+  if (se != cudaSuccess) {
+    record_cuda_error(se);
+    return HCADSA_ERR_CUDA;
+  }
   int* p = device_error_ptr();
   if (!p) return HCADSA_ERR_CUDA;
   int v = 0;
