@@ -32,7 +32,11 @@
 //     moves when the tile max exceeds it by 2^8.
 //   * Key tiles: compressed entries [0, n_c(t_last)) in tiles of 128, then the window
 //     band [max(0, t_first-W+1), t_last] in tiles of 128; per-row visibility is one
-//     column interval per tile.
+//     column interval per tile.  The band of 128/g tokens is 128/g + W - 1 keys long, so with
+//     W = 128 it overhangs one tile by a few keys; when those fit beside the last, partial tile
+//     of compressed entries, the two share one "merged" key tile (rows [0,16) = the band's
+//     first 16 keys, rows [16,128) = the entries) instead of costing a QK^T of their own, and
+//     that tile has two visible intervals per row.
 //   * Barrier phases run on across tiles: p_ready / pv_done are per S buffer and follow a
 //     key-tile counter that never resets (phase A and phase B tiles both count); s_full is per
 //     S buffer too but only phase-A tiles complete it, so its consumer keeps one parity bit per
@@ -53,6 +57,8 @@ constexpr int kD = 512;
 constexpr int kDHalf = 256;
 constexpr int kKeyTile = 128;
 constexpr int kSmallRows = 32;  // TMA box height for key tiles of at most 32 keys
+constexpr int kMergeWinRows = 16;                       // window keys at the head of a merged tile
+constexpr int kMergeEntRows = kKeyTile - kMergeWinRows;  // compressed entries after them
 // Ring: groups of two 16 KB chunk slots (128 d-columns of a key tile).  Two groups, plus a third
 // in the epilogue staging area when key ranges are split (those epilogues write fp32 partials
 // straight to global memory, and their K/V stream from HBM, where depth pays).
@@ -96,6 +102,7 @@ struct Maps {
   CUtensorMap q;
   CUtensorMap o;            // box 32 columns x 128 rows, 64-byte swizzle (stores)
   CUtensorMap kv[2][2][2];  // [0 = K, 1 = V][0 = compressed, 1 = window][0 = 128 rows, 1 = 32 rows]
+  CUtensorMap merge[2][2];  // [0 = K, 1 = V][0 = window 16 rows, 1 = compressed 112 rows]
 };
 
 __device__ __forceinline__ int n_compressed(int t, int W, int blk) {
@@ -113,9 +120,11 @@ __device__ __forceinline__ void bulk_wait_group_read1() {
 }
 
 struct KeyTile {
-  int window;  // 0: compressed entries, 1: raw window positions
-  int start;   // first entry / position
+  int kind;    // 0: compressed entries, 1: raw window positions, 2: merged (window keys, then entries)
+  int start;   // first entry (kinds 0, 2) / position (kind 1)
   int n;       // MMA N (multiple of 16, <= 128)
+  int wstart;  // kind 2: first window position (tile rows [0, 16))
+  int wn;      // kind 2: window keys the tile owns (<= 16; the band's later keys are in window tiles)
 };
 
 __host__ __device__ inline int first_unit(int T, const Params& p) { return T * p.splits + min(T, p.split_extra); }
@@ -130,6 +139,8 @@ struct TileSet {
   int nc_hi;        // entries needed by the last token
   int ws_lo;        // window start of the first token
   int t_hi;         // last valid token position
+  int w_part;       // keys of the band beyond its whole 128-key tiles (1..128)
+  int merged;       // 1: the band's first w_part keys share the last compressed tile
   __device__ void init(int U, const Params& p) {
     const int big = p.split_extra * (p.splits + 1);  // units of the row tiles with an extra split
     const int T = U < big ? U / (p.splits + 1) : p.split_extra + (U - big) / p.splits;
@@ -142,21 +153,34 @@ struct TileSet {
     nc_hi = n_compressed(t_hi, p.W, p.blk);
     ws_lo = window_start(p.q_offset + tok0, p.W);
     J_c = (nc_hi + kKeyTile - 1) / kKeyTile;
-    const int Jt = J_c + (t_hi - ws_lo + kKeyTile) / kKeyTile;
+    const int w_span = t_hi - ws_lo + 1;
+    const int n_wt = (w_span + kKeyTile - 1) / kKeyTile;
+    w_part = w_span - (n_wt - 1) * kKeyTile;
+    merged = J_c >= 1 && n_wt >= 2 && w_part <= kMergeWinRows && nc_hi - (J_c - 1) * kKeyTile <= kMergeEntRows;
+    const int Jt = J_c + n_wt - merged;
     js = split * Jt / S;
     J = (split + 1) * Jt / S - js;
   }
   __device__ KeyTile get(int jl) const {
     KeyTile kt;
     const int j = js + jl;
+    kt.wstart = 0;
+    kt.wn = 0;
     if (j < J_c) {
-      kt.window = 0;
+      kt.kind = merged && j == J_c - 1 ? 2 : 0;
       kt.start = j * kKeyTile;
-      const int rem = min(kKeyTile, nc_hi - kt.start);
-      kt.n = (rem + 15) & ~15;
+      const int rem = nc_hi - kt.start;
+      if (kt.kind == 2) {
+        kt.wstart = ws_lo;
+        kt.wn = w_part;
+        kt.n = kMergeWinRows + ((rem + 15) & ~15);
+      } else {
+        kt.n = (min(kKeyTile, rem) + 15) & ~15;
+      }
     } else {
-      kt.window = 1;
-      kt.start = ws_lo + (j - J_c) * kKeyTile;
+      kt.kind = 1;
+      // after a merged tile the band continues at its (w_part+1)-th key in whole tiles
+      kt.start = ws_lo + (merged ? w_part : 0) + (j - J_c) * kKeyTile;
       const int rem = min(kKeyTile, t_hi + 1 - kt.start);
       kt.n = (rem + 15) & ~15;
     }
@@ -252,14 +276,28 @@ __global__ void __launch_bounds__(kThreads, 1) hca_attn_kernel(const __grid_cons
       const uint32_t ngroups = p.split_mode ? kMaxGroups : kGroups;
       uint32_t grp = 0, gph = 0;  // next ring group to fill and the phase of its use
       bool ok = true;
-      // two 64-column chunks (columns col .. col+127 of a key tile) into the next ring group
-      auto load_unit = [&](const CUtensorMap* m, bool small, int col, int hk, int row0, int b) {
+      // two 64-column chunks (columns col .. col+127 of key tile kt; kv 0 = K, 1 = V) into the
+      // next ring group
+      auto load_unit = [&](int kv, const KeyTile& kt, int col, int hk, int b) {
         ok = mbar_wait(&bar.empty[grp], gph ^ 1, &abort_flag, p.err);
         if (ok) {
-          mbar_arrive_expect_tx(&bar.full[grp], 2 * (small ? kSmallChunkBytes : kChunkBytes));
           uint8_t* dst = sRing + grp * kGroupBytes;
-          tma_load_4d(dst, m, &bar.full[grp], col, hk, row0, b);
-          tma_load_4d(dst + kChunkBytes, m, &bar.full[grp], col + 64, hk, row0, b);
+          if (kt.kind == 2) {  // 16 window rows, then 112 entry rows: both boxes fill the slot
+            mbar_arrive_expect_tx(&bar.full[grp], 2 * kChunkBytes);
+            for (int cc = 0; cc < 2; ++cc) {
+              tma_load_4d(dst + cc * kChunkBytes, &maps.merge[kv][0], &bar.full[grp], col + cc * 64, hk,
+                          kt.wstart - p.win_start, b);
+              tma_load_4d(dst + cc * kChunkBytes + kMergeWinRows * 128, &maps.merge[kv][1], &bar.full[grp],
+                          col + cc * 64, hk, kt.start, b);
+            }
+          } else {
+            const int small = kt.n <= kSmallRows ? 1 : 0;
+            const CUtensorMap* m = &maps.kv[kv][kt.kind][small];
+            const int row0 = kt.kind ? kt.start - p.win_start : kt.start;
+            mbar_arrive_expect_tx(&bar.full[grp], 2 * (small ? kSmallChunkBytes : kChunkBytes));
+            tma_load_4d(dst, m, &bar.full[grp], col, hk, row0, b);
+            tma_load_4d(dst + kChunkBytes, m, &bar.full[grp], col + 64, hk, row0, b);
+          }
         }
         if (++grp == ngroups) {
           grp = 0;
@@ -268,10 +306,7 @@ __global__ void __launch_bounds__(kThreads, 1) hca_attn_kernel(const __grid_cons
       };
       auto load_v = [&](const TileSet& ts, int j, int col0) {
         const KeyTile kt = ts.get(j);
-        const int small = kt.n <= kSmallRows ? 1 : 0;
-        const int row0 = kt.window ? kt.start - p.win_start : kt.start;
-        for (int c = 0; ok && c < kVChunks; c += 2)
-          load_unit(&maps.kv[1][kt.window][small], small, col0 + c * 64, ts.hk, row0, ts.b);
+        for (int c = 0; ok && c < kVChunks; c += 2) load_unit(1, kt, col0 + c * 64, ts.hk, ts.b);
       };
       if (blockIdx.x < p.total_units) {
         TileSet t0;
@@ -289,10 +324,7 @@ __global__ void __launch_bounds__(kThreads, 1) hca_attn_kernel(const __grid_cons
         for (int step = 0; ok && step <= ts.J; ++step) {
           if (step < ts.J) {
             const KeyTile kt = ts.get(step);
-            const int small = kt.n <= kSmallRows ? 1 : 0;
-            const int row0 = kt.window ? kt.start - p.win_start : kt.start;
-            for (int c = 0; ok && c < kQChunks; c += 2)
-              load_unit(&maps.kv[0][kt.window][small], small, c * 64, ts.hk, row0, ts.b);
+            for (int c = 0; ok && c < kQChunks; c += 2) load_unit(0, kt, c * 64, ts.hk, ts.b);
           }
           if (ok && step >= 1) load_v(ts, step - 1, 0);
         }
@@ -515,22 +547,34 @@ __global__ void __launch_bounds__(kThreads, 1) hca_attn_kernel(const __grid_cons
       for (int j = 0; ok && j < ts.J; ++j) {
         const uint32_t gs = g + j;
         const KeyTile kt = ts.get(j);
-        int lo, hi;
-        if (kt.window) {
+        // visible columns: [lo, hi) and, in a merged tile, its window columns [lo2, hi2)
+        int lo, hi, lo2 = 0, hi2 = 0;
+        if (kt.kind == 1) {
           lo = max(ws_t, kt.start) - kt.start;
           hi = min(t + 1, kt.start + kt.n) - kt.start;
-        } else {
+        } else if (kt.kind == 0) {
           lo = 0;
           hi = min(nc_t, kt.start + kt.n) - kt.start;
+        } else {
+          lo = kMergeWinRows;
+          hi = kMergeWinRows + nc_t - kt.start;  // nc_t <= nc_hi: never past the tile's entries
+          lo2 = max(ws_t - kt.wstart, 0);
+          hi2 = min(t + 1 - kt.wstart, kt.wn);
         }
-        if (!row_valid) hi = lo;  // padding rows see nothing
+        if (!row_valid) {  // padding rows see nothing
+          hi = lo;
+          hi2 = lo2;
+        }
         const uint32_t tS = tmem + lane_off + kDHalf + (gs & 1) * kKeyTile;
         ok = mbar_wait(&bar.s_full[gs & 1], (s_par >> (gs & 1)) & 1, &abort_flag, p.err);
         if (!ok) break;
         s_par ^= 1u << (gs & 1);
         tc_fence_after();
-        // pass 1: tile max over this row's visible columns
-        const uint32_t vis_n = (uint32_t)(hi - lo);  // column c is visible iff (c - lo) < vis_n
+        // pass 1: tile max over this row's visible columns.  An interval may be empty (hi < lo:
+        // a token whose window starts past a band tile, or that needs fewer entries than a tile
+        // holds when blk < 128/g), so the widths are clamped at 0.
+        const uint32_t vis_n = hi > lo ? (uint32_t)(hi - lo) : 0u;  // c visible iff (c - lo) < vis_n
+        const uint32_t vis_n2 = hi2 > lo2 ? (uint32_t)(hi2 - lo2) : 0u;  // ... or (c - lo2) < vis_n2
         float mx = -INFINITY;
         for (int c0 = 0; c0 < kt.n; c0 += 32) {
           uint32_t v[32];
@@ -542,7 +586,8 @@ __global__ void __launch_bounds__(kThreads, 1) hca_attn_kernel(const __grid_cons
           } else {
 #pragma unroll
             for (int i = 0; i < 32; ++i)
-              if ((uint32_t)(c0 + i - lo) < vis_n) mx = fmaxf(mx, __uint_as_float(v[i]));
+              if ((uint32_t)(c0 + i - lo) < vis_n || (uint32_t)(c0 + i - lo2) < vis_n2)
+                mx = fmaxf(mx, __uint_as_float(v[i]));
           }
         }
         const float m_tile = mx * p.scale_log2;  // -inf stays -inf
@@ -571,6 +616,7 @@ __global__ void __launch_bounds__(kThreads, 1) hca_attn_kernel(const __grid_cons
         if (row_valid) *scratch_alpha(scratch, j, r) = alpha;
         // pass 2: P = exp2(s*scale*log2e - m_ref) as bf16, in place over S and into the scratch
         const uint32_t vis_p = m_ref != -INFINITY ? vis_n : 0u;
+        const uint32_t vis_p2 = m_ref != -INFINITY ? vis_n2 : 0u;
         uint4* prow = scratch_p(scratch, j, r);
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) {
@@ -595,8 +641,10 @@ __global__ void __launch_bounds__(kThreads, 1) hca_attn_kernel(const __grid_cons
               for (int i = 0; i < 16; ++i) {
                 const int c = c0 + 2 * i;
                 float p0 = 0.0f, p1 = 0.0f;
-                if ((uint32_t)(c - lo) < vis_p) p0 = fast_exp2(fmaf(__uint_as_float(v[2 * i]), p.scale_log2, -m_ref));
-                if ((uint32_t)(c + 1 - lo) < vis_p) p1 = fast_exp2(fmaf(__uint_as_float(v[2 * i + 1]), p.scale_log2, -m_ref));
+                if ((uint32_t)(c - lo) < vis_p || (uint32_t)(c - lo2) < vis_p2)
+                  p0 = fast_exp2(fmaf(__uint_as_float(v[2 * i]), p.scale_log2, -m_ref));
+                if ((uint32_t)(c + 1 - lo) < vis_p || (uint32_t)(c + 1 - lo2) < vis_p2)
+                  p1 = fast_exp2(fmaf(__uint_as_float(v[2 * i + 1]), p.scale_log2, -m_ref));
                 l_run += p0 + p1;
                 pk[i] = pack_bf16x2(p0, p1);
               }
@@ -752,11 +800,17 @@ struct Geometry {
 
 long long host_n_compressed(long long t, int W, int blk) { return t - W + 1 > 0 ? (t - W + 1) / blk : 0; }
 long long host_window_start(long long t, int W) { return t - W + 1 > 0 ? t - W + 1 : 0; }
-// key tiles of the row tile with tokens [tok0, tok_hi] (relative to q_offset)
+// key tiles of the row tile with tokens [tok0, tok_hi] (relative to q_offset); the same rule as
+// TileSet::init, merged tile included
 long long host_tile_J(long long q_offset, long long tok0, long long tok_hi, int W, int blk) {
   const long long t_hi = q_offset + tok_hi;
   const long long nc = host_n_compressed(t_hi, W, blk);
-  return (nc + kKeyTile - 1) / kKeyTile + (t_hi - host_window_start(q_offset + tok0, W) + kKeyTile) / kKeyTile;
+  const long long J_c = (nc + kKeyTile - 1) / kKeyTile;
+  const long long w_span = t_hi - host_window_start(q_offset + tok0, W) + 1;
+  const long long n_wt = (w_span + kKeyTile - 1) / kKeyTile;
+  const long long w_part = w_span - (n_wt - 1) * kKeyTile;
+  const int merged = J_c >= 1 && n_wt >= 2 && w_part <= kMergeWinRows && nc - (J_c - 1) * kKeyTile <= kMergeEntRows;
+  return J_c + n_wt - merged;
 }
 
 hcadsa_status geometry(Geometry* G, int B, int Lq, int q_offset, int Hq, int Hkv, int d, int blk, int W) {
@@ -859,6 +913,14 @@ extern "C" hcadsa_status hca_attn_fwd(const hcadsa_bf16* Q, const hcadsa_bf16* K
   Maps maps;
   if (!make_map_4d(&maps.q, Q, kD, Hq, Lq, B, 64, g, G.TT, 128)) return HCADSA_ERR_CUDA;
   if (!make_map_4d(&maps.o, O, kD, Hq, Lq, B, kOutCols, g, G.TT, 64)) return HCADSA_ERR_CUDA;
+  for (int kv = 0; kv < 2; ++kv) {
+    const hcadsa_bf16* win = kv ? Vw : Kw;
+    const hcadsa_bf16* ent = n_c > 0 ? (kv ? Vc : Kc) : win;  // no query sees an entry without n_c > 0
+    const int ent_rows = n_c > 0 ? n_c : n_w;
+    if (!make_map_4d(&maps.merge[kv][0], win, kD, Hkv, n_w, B, 64, 1, kMergeWinRows, 128)) return HCADSA_ERR_CUDA;
+    if (!make_map_4d(&maps.merge[kv][1], ent, kD, Hkv, ent_rows, B, 64, 1, kMergeEntRows, 128))
+      return HCADSA_ERR_CUDA;
+  }
   for (int small = 0; small < 2; ++small) {
     const int rows = small ? kSmallRows : 128;
     if (!make_map_4d(&maps.kv[0][1][small], Kw, kD, Hkv, n_w, B, 64, 1, rows, 128)) return HCADSA_ERR_CUDA;

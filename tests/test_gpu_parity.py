@@ -109,6 +109,13 @@ def test_hca_tiny_all_rows(hd):
     (synth.HcaConfig("stress_sigma1_L700_hq8_hkv2_B2", B=2, L=700, Hq=8, Hkv=2, sigma=1.0), 128),
     (synth.HcaConfig("wide_window_L300", B=1, L=300, Hq=16, Hkv=1, sigma=1.0), 512),
     (synth.HcaConfig("sharp_L600_blk64_W96", B=1, L=600, Hq=16, Hkv=1, blk=64, W=96, sigma=2.0), 96),
+    # one head per K/V head (128-token row tiles) with W = 64 and blk = 32: a band tile can start
+    # after a row's last key, and a compressed tile after a row's last entry (empty intervals)
+    (synth.HcaConfig("g1_W64_blk32_L4400_hq2", B=1, L=4400, Hq=2, Hkv=2, blk=32, W=64, sigma=1.0), 64),
+    # blk = 16 walks the last compressed tile through every fill (1..128 entries), so the band's
+    # overhang shares that tile (merged tiles) or not, for 8- and 16-token row tiles
+    (synth.HcaConfig("merge_blk16_L2400_hq16", B=1, L=2400, Hq=16, Hkv=1, blk=16, sigma=1.0), 128),
+    (synth.HcaConfig("merge_g8_blk16_L2400_hq16_hkv2", B=1, L=2400, Hq=16, Hkv=2, blk=16, sigma=1.0), 128),
 ])
 def test_hca_stress(hd, cfg, W):
     O, lse, ref, ref_lse = _hca_gpu_and_oracle(hd, cfg, W=W)
