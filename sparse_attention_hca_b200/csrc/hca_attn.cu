@@ -74,7 +74,9 @@ constexpr int kOutBufBytes = 128 * kOutCols * 2;  // 8 KB
 constexpr int kGroupBytes = 2 * kChunkBytes;
 constexpr int kSmemBytes = kQBytes + kMaxGroups * kGroupBytes + 1024;
 static_assert(kGroups * kGroupBytes + 2 * kOutBufBytes <= kMaxGroups * kGroupBytes, "staging fits the third group");
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;
+constexpr int kSoftmaxWarp0 = 2;   // warps 2-5: softmax and P reloads
+constexpr int kEpilogueWarp0 = 6;  // warps 6-9: O read-out and stores
 constexpr float kLazyRescale = 8.0f;  // log2 units
 // per-CTA scratch per key tile: P (128 rows x 128 keys bf16) + one fp32 rescale factor per row
 constexpr size_t kScratchPBytes = 128 * kKeyTile * 2;
@@ -197,6 +199,8 @@ struct __align__(8) Barriers {
   uint64_t pv_done[2];  // the PV that read P from S buffer i has completed
   uint64_t o_full;      // every PV of the current O half has completed
   uint64_t o_empty[2];  // the epilogue has read O columns [0,128) / [128,256)
+  uint64_t l_ready[2];  // the softmax warps have written 1/l of row tile i (mod 2)
+  uint64_t l_empty[2];  // the epilogue warps have stored both O halves of that row tile
 };
 
 // One thread's row of P_j in the scratch: key tile j owns kScratchTileBytes; inside it the
@@ -238,6 +242,7 @@ __global__ void __launch_bounds__(kThreads, 1) hca_attn_kernel(const __grid_cons
   uint8_t* sRing = smem + kQBytes;
   uint8_t* sOut = sRing + kGroups * kGroupBytes;
   __shared__ Barriers bar;
+  __shared__ float inv_l_sh[2][128];  // 1/l per row (1 in split mode), double-buffered by row tile
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_flag;
 
@@ -257,6 +262,10 @@ __global__ void __launch_bounds__(kThreads, 1) hca_attn_kernel(const __grid_cons
     mbar_init(&bar.o_full, 1);
     mbar_init(&bar.o_empty[0], 128);
     mbar_init(&bar.o_empty[1], 128);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bar.l_ready[s], 128);
+      mbar_init(&bar.l_empty[s], 128);
+    }
     abort_flag = 0;
     fence_mbarrier_init();
   }
@@ -456,20 +465,17 @@ __global__ void __launch_bounds__(kThreads, 1) hca_attn_kernel(const __grid_cons
         ++it;
       }
     }
-  } else {
-    // ------------------------------------------------------------ softmax + epilogue
+  } else if (warp >= kEpilogueWarp0) {
+    // ------------------------------------------------------------ epilogue
+    // Runs beside the softmax warps: while it reads out and stores one O half, they already
+    // reload P for the next half or run the next row tile's softmax.
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;  // row of the tile == TMEM lane
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const bool store_issuer = r == 0;
-    uint8_t* scratch = p.scratch + (size_t)blockIdx.x * p.J_max * kScratchTileBytes;
-    uint32_t g = 0, it = 0, ec = 0;  // key tiles, O halves, staged stores
-    // s_full[b] completes once per phase-A key tile on S buffer b (phase B issues no QK^T), so
-    // its parity is tracked per buffer here rather than derived from the key-tile counter
-    uint32_t s_par = 0;
+    uint32_t it = 0, ec = 0, tl = 0;  // O halves, staged stores, row tiles
     bool ok = true;
 
-    // O half (TMEM) -> bf16 -> two 8 KB staging buffers -> TMA tensor store; then release O
     // O half (TMEM) -> normalised bf16 in registers, 128 columns at a time, each 128 columns
     // released to the MMA warp as soon as they are read -> two 8 KB staging buffers -> TMA
     // tensor stores.  With split key ranges the unit's unnormalised fp32 O rows go to part_o.
@@ -532,7 +538,34 @@ __global__ void __launch_bounds__(kThreads, 1) hca_attn_kernel(const __grid_cons
       ++it;
     };
 
-    for (int T = blockIdx.x; ok && T < p.total_units; T += gridDim.x) {
+    for (int T = blockIdx.x; ok && T < p.total_units; T += gridDim.x, ++tl) {
+      TileSet ts;
+      ts.init(T, p);
+      if (ts.J > p.J_max) break;
+      const bool row_valid = ts.tok0 + r / p.g < p.Lq;
+      ok = mbar_wait(&bar.l_ready[tl & 1], (tl >> 1) & 1, &abort_flag, p.err);
+      if (!ok) break;
+      const float inv_l = inv_l_sh[tl & 1][r];
+      epilogue(ts, 0, inv_l, T, row_valid);
+      if (!ok) break;
+      epilogue(ts, kDHalf, inv_l, T, row_valid);
+      if (!ok) break;
+      mbar_arrive(&bar.l_empty[tl & 1]);
+    }
+    if (store_issuer) bulk_wait_group0();
+  } else {
+    // ------------------------------------------------------------ softmax and P reloads
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;  // row of the tile == TMEM lane
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    uint8_t* scratch = p.scratch + (size_t)blockIdx.x * p.J_max * kScratchTileBytes;
+    uint32_t g = 0, tl = 0;  // key tiles, row tiles
+    // s_full[b] completes once per phase-A key tile on S buffer b (phase B issues no QK^T), so
+    // its parity is tracked per buffer here rather than derived from the key-tile counter
+    uint32_t s_par = 0;
+    bool ok = true;
+
+    for (int T = blockIdx.x; ok && T < p.total_units; T += gridDim.x, ++tl) {
       TileSet ts;
       ts.init(T, p);
       if (ts.J > p.J_max) break;
@@ -669,8 +702,13 @@ __global__ void __launch_bounds__(kThreads, 1) hca_attn_kernel(const __grid_cons
       } else if (p.lse && row_valid) {
         p.lse[((size_t)ts.b * p.Lq + tok) * p.Hq + h] = (m_ref + __log2f(l_run)) * 0.69314718055994531f;
       }
-      epilogue(ts, 0, inv_l, T, row_valid);
-      if (!ok) break;
+      // hand 1/l to the epilogue warps (their buffer of two row tiles ago must be consumed)
+      if (tl >= 2) {
+        ok = mbar_wait(&bar.l_empty[tl & 1], ((tl >> 1) - 1) & 1, &abort_flag, p.err);
+        if (!ok) break;
+      }
+      inv_l_sh[tl & 1][r] = inv_l;
+      mbar_arrive(&bar.l_ready[tl & 1]);
       g += ts.J;
       // ---- phase B: reload P_j into the S buffers, apply the same rescales
       for (int j = 0; ok && j < ts.J; ++j) {
@@ -712,10 +750,8 @@ __global__ void __launch_bounds__(kThreads, 1) hca_attn_kernel(const __grid_cons
         mbar_arrive(&bar.p_ready[gs & 1]);
       }
       if (!ok) break;
-      epilogue(ts, kDHalf, inv_l, T, row_valid);
       g += ts.J;
     }
-    if (store_issuer) bulk_wait_group0();
   }
 
   tc_fence_before();
