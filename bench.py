@@ -115,26 +115,52 @@ def job_throughput(ms_per_step_max: float, world: int, tokens_per_rank: int = No
 # ----------------------------------------------------------------------------- clocks
 
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    """nvidia-smi every 20 ms with host timestamps; stop() keeps the samples taken inside the
+    window marked by begin()/end() (the timed region)."""
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, device_index):
         self.dev = device_index
         self.proc = None
+        self.t0 = self.t1 = None
         import tempfile
 
         fd, self.path = tempfile.mkstemp(prefix=f"hcadsa_clocks_gpu{device_index}_", suffix=".csv")
         os.close(fd)
 
-    def start(self):
+    def start(self, ready_timeout_s=5.0):
         try:
             self.fh = open(self.path, "w")
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                          "--format=csv,noheader,nounits", "-lms", "20"],
                                          stdout=self.fh, stderr=subprocess.DEVNULL)
         except (OSError, FileNotFoundError):
             self.proc = None
+            return
+        t_end = time.time() + ready_timeout_s  # the first sample is there before timing starts
+        while time.time() < t_end and self.proc.poll() is None:
+            if os.path.getsize(self.path) > 0:
+                break
+            time.sleep(0.01)
+
+    def begin(self):
+        self.t0 = time.time()
+
+    def end(self):
+        self.t1 = time.time()
+
+    @staticmethod
+    def _stamp(text):
+        import datetime
+
+        for fmt in ("%Y/%m/%d %H:%M:%S.%f", "%Y/%m/%d %H:%M:%S"):
+            try:
+                return datetime.datetime.strptime(text, fmt).timestamp()
+            except ValueError:
+                pass
+        return None
 
     def stop(self):
         if self.proc is None:
@@ -145,24 +171,31 @@ class ClockSampler:
         except subprocess.TimeoutExpired:
             self.proc.kill()
         self.fh.close()
-        sm, mx, reasons = [], [], set()
+        rows = []
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for line in open(self.path):
             f = [x.strip() for x in line.split(",")]
-            if len(f) < 9:
+            if len(f) < 10:
                 continue
             try:
-                sm.append(float(f[1]))
-                mx.append(float(f[2]))
+                rows.append((self._stamp(f[0]), float(f[2]), float(f[3]), f[6:10]))
             except ValueError:
                 continue
-            for n, v in zip(names, f[5:9]):
+        if not rows:
+            return None
+        window = "timed region"
+        inside = [r for r in rows if r[0] is not None and self.t0 is not None and self.t1 is not None
+                  and self.t0 - 0.02 <= r[0] <= self.t1 + 0.02]
+        if not inside:  # no sample fell inside (a very short region): report the nearest ones
+            window = "around the timed region"
+            inside = rows
+        reasons = set()
+        for r in inside:
+            for n, v in zip(names, r[3]):
                 if v.lower() == "active":
                     reasons.add(n)
-        if not sm:
-            return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "samples": len(sm),
-                "reasons": sorted(reasons)}
+        return {"sm_mhz": statistics.median(r[1] for r in inside), "sm_max_mhz": max(r[2] for r in inside),
+                "samples": len(inside), "window": window, "reasons": sorted(reasons)}
 
 
 # ----------------------------------------------------------------------------- our arm
@@ -384,8 +417,9 @@ def ours(args):
     clocks = ClockSampler(local)
     if dist:
         dist.barrier()
-    torch.cuda.synchronize()
     clocks.start()
+    torch.cuda.synchronize()
+    clocks.begin()
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     t_start.record()
@@ -393,6 +427,7 @@ def ours(args):
         st.run(evs[i])
     t_end.record()
     torch.cuda.synchronize()
+    clocks.end()
     if dist:
         dist.barrier()
     clk = clocks.stop()

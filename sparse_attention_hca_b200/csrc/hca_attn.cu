@@ -19,17 +19,20 @@
 //     TMEM and runs only O[:, 256:512] += P_j V_j[:, 256:512] with the same rescales, so the
 //     second half costs no QK^T and no exponentials, and Q's buffer is free to take the
 //     next tile's Q while phase B runs.
-//   * warp 0: TMA producer (Q per tile; K and V in units of 128 d-columns (two 16 KB chunks)
-//     through a ring of two such groups, in exactly the order the MMA warp consumes them; key
-//     tiles of at most 32 keys use 32-row boxes); warp 1: TMEM allocation and the single
+//   * warp 0: TMA producer (Q per tile; K and V through a ring of two 32 KB groups, in exactly
+//     the order the MMA warp consumes them: a K group is 128 d-columns of a key tile (two 16 KB
+//     chunks of 128 rows), a V group 64 keys x one 256-column half of d_v (four 8 KB chunks);
+//     key tiles of at most 32 keys use 32-row boxes); warp 1: TMEM allocation and the single
 //     MMA-issuing thread.  One barrier wait per group: a wait costs the issuing thread a few
-//     hundred cycles, which only ~500 cycles of queued MMA work (8 MMAs of N = 128) hide;
-//     warps 2-5: softmax, one thread per row (TMEM lane), and the epilogues, which stage O
-//     through shared memory (64-byte swizzle, two 8 KB buffers) into TMA tensor stores.
+//     hundred cycles, which only ~500 cycles of queued MMA work hide (8 QK^T MMAs of N = 128,
+//     or 4 PV MMAs of N = 256); warps 2-5: softmax and the P reloads, one thread per row (TMEM
+//     lane); warps 6-9: the epilogues, which read each O half out of TMEM, hand it back to the
+//     MMA warp and stage it through shared memory (64-byte swizzle, four 8 KB boxes) into TMA
+//     tensor stores, while the softmax warps go on with the next half or row tile.
 //   * S_j accumulates over eight 64-wide d chunks (SS MMA, K-major operands, 128B swizzle).
 //     P_j is written in place over S_j in TMEM and PV runs as a TS MMA (A = P from TMEM,
-//     B = V, MN-major, N = 128 over the group's two chunks).  Online softmax with a lazy rescale: the reference max only
-//     moves when the tile max exceeds it by 2^8.
+//     B = V, MN-major, N = 256 over a V group's four chunks).  Online softmax with a lazy
+//     rescale: the reference max only moves when the tile max exceeds it by 2^8.
 //   * Key tiles: compressed entries [0, n_c(t_last)) in tiles of 128, then the window
 //     band [max(0, t_first-W+1), t_last] in tiles of 128; per-row visibility is one
 //     column interval per tile.  The band of 128/g tokens is 128/g + W - 1 keys long, so with
@@ -68,12 +71,15 @@ constexpr int kChunkBytes = 128 * 128;  // 128 rows x 64 bf16
 constexpr int kSmallChunkBytes = kSmallRows * 128;
 constexpr int kQChunks = kD / 64;      // 8
 constexpr int kVChunks = kDHalf / 64;  // 4
+constexpr int kVRows = 64;             // keys per V ring group (4 chunks of 64 keys x 64 columns)
+constexpr int kVChunkBytes = kVRows * 128;
 constexpr int kQBytes = kQChunks * kChunkBytes;
-constexpr int kOutCols = 32;                  // O columns per staged store
+constexpr int kOutCols = 32;                  // O columns per TMA store box
 constexpr int kOutBufBytes = 128 * kOutCols * 2;  // 8 KB
+constexpr int kOutBufs = 4;                       // staging: 128 columns of O in four boxes
 constexpr int kGroupBytes = 2 * kChunkBytes;
 constexpr int kSmemBytes = kQBytes + kMaxGroups * kGroupBytes + 1024;
-static_assert(kGroups * kGroupBytes + 2 * kOutBufBytes <= kMaxGroups * kGroupBytes, "staging fits the third group");
+static_assert(kGroups * kGroupBytes + kOutBufs * kOutBufBytes <= kMaxGroups * kGroupBytes, "staging fits the third group");
 constexpr int kThreads = 320;
 constexpr int kSoftmaxWarp0 = 2;   // warps 2-5: softmax and P reloads
 constexpr int kEpilogueWarp0 = 6;  // warps 6-9: O read-out and stores
@@ -99,12 +105,15 @@ struct Params {
   int* err;
 };
 
-// Q and O, then K and V over {compressed entries, window} x {128-row box, 32-row box}.
+// Q and O, then K and V over {compressed entries, window} x box heights, and the two boxes of
+// each half of a merged key tile.
 struct Maps {
   CUtensorMap q;
-  CUtensorMap o;            // box 32 columns x 128 rows, 64-byte swizzle (stores)
-  CUtensorMap kv[2][2][2];  // [0 = K, 1 = V][0 = compressed, 1 = window][0 = 128 rows, 1 = 32 rows]
-  CUtensorMap merge[2][2];  // [0 = K, 1 = V][0 = window 16 rows, 1 = compressed 112 rows]
+  CUtensorMap o;          // box 32 columns x 128 rows, 64-byte swizzle (stores)
+  CUtensorMap k[2][2];    // [0 = compressed, 1 = window][0 = 128 rows, 1 = 32 rows]
+  CUtensorMap v[2][2];    // [0 = compressed, 1 = window][0 = 64 rows, 1 = 32 rows]
+  CUtensorMap kmerge[2];  // [0 = window 16 rows, 1 = compressed 112 rows]
+  CUtensorMap vmerge[2];  // [0 = window 16 rows, 1 = compressed 48 rows]
 };
 
 __device__ __forceinline__ int n_compressed(int t, int W, int blk) {
@@ -285,37 +294,67 @@ __global__ void __launch_bounds__(kThreads, 1) hca_attn_kernel(const __grid_cons
       const uint32_t ngroups = p.split_mode ? kMaxGroups : kGroups;
       uint32_t grp = 0, gph = 0;  // next ring group to fill and the phase of its use
       bool ok = true;
-      // two 64-column chunks (columns col .. col+127 of key tile kt; kv 0 = K, 1 = V) into the
-      // next ring group
-      auto load_unit = [&](int kv, const KeyTile& kt, int col, int hk, int b) {
+      auto next_group = [&]() {
+        if (++grp == ngroups) {
+          grp = 0;
+          gph ^= 1;
+        }
+      };
+      // K: all rows of key tile kt x columns col .. col+127 (two 16 KB chunks) into the next group
+      auto load_k = [&](const KeyTile& kt, int col, int hk, int b) {
         ok = mbar_wait(&bar.empty[grp], gph ^ 1, &abort_flag, p.err);
         if (ok) {
           uint8_t* dst = sRing + grp * kGroupBytes;
-          if (kt.kind == 2) {  // 16 window rows, then 112 entry rows: both boxes fill the slot
+          if (kt.kind == 2) {  // 16 window rows, then 112 entry rows: both boxes fill the chunk
             mbar_arrive_expect_tx(&bar.full[grp], 2 * kChunkBytes);
             for (int cc = 0; cc < 2; ++cc) {
-              tma_load_4d(dst + cc * kChunkBytes, &maps.merge[kv][0], &bar.full[grp], col + cc * 64, hk,
+              tma_load_4d(dst + cc * kChunkBytes, &maps.kmerge[0], &bar.full[grp], col + cc * 64, hk,
                           kt.wstart - p.win_start, b);
-              tma_load_4d(dst + cc * kChunkBytes + kMergeWinRows * 128, &maps.merge[kv][1], &bar.full[grp],
+              tma_load_4d(dst + cc * kChunkBytes + kMergeWinRows * 128, &maps.kmerge[1], &bar.full[grp],
                           col + cc * 64, hk, kt.start, b);
             }
           } else {
             const int small = kt.n <= kSmallRows ? 1 : 0;
-            const CUtensorMap* m = &maps.kv[kv][kt.kind][small];
+            const CUtensorMap* m = &maps.k[kt.kind][small];
             const int row0 = kt.kind ? kt.start - p.win_start : kt.start;
             mbar_arrive_expect_tx(&bar.full[grp], 2 * (small ? kSmallChunkBytes : kChunkBytes));
             tma_load_4d(dst, m, &bar.full[grp], col, hk, row0, b);
             tma_load_4d(dst + kChunkBytes, m, &bar.full[grp], col + 64, hk, row0, b);
           }
         }
-        if (++grp == ngroups) {
-          grp = 0;
-          gph ^= 1;
+        next_group();
+      };
+      // V: rows [64 gi, 64 gi + 64) of key tile kt x columns col0 .. col0+255 (four 8 KB chunks)
+      // into the next group
+      auto load_vgroup = [&](const KeyTile& kt, int gi, int col0, int hk, int b) {
+        ok = mbar_wait(&bar.empty[grp], gph ^ 1, &abort_flag, p.err);
+        if (ok) {
+          uint8_t* dst = sRing + grp * kGroupBytes;
+          if (kt.kind == 2 && gi == 0) {  // 16 window rows, then 48 entry rows
+            mbar_arrive_expect_tx(&bar.full[grp], kVChunks * kVChunkBytes);
+            for (int c = 0; c < kVChunks; ++c) {
+              tma_load_4d(dst + c * kVChunkBytes, &maps.vmerge[0], &bar.full[grp], col0 + c * 64, hk,
+                          kt.wstart - p.win_start, b);
+              tma_load_4d(dst + c * kVChunkBytes + kMergeWinRows * 128, &maps.vmerge[1], &bar.full[grp],
+                          col0 + c * 64, hk, kt.start, b);
+            }
+          } else {
+            // tile row r of a merged tile (r >= 16) holds entry start + r - 16
+            const int kind = kt.kind == 1 ? 1 : 0;
+            const int small = kt.n <= kSmallRows ? 1 : 0;
+            const int row0 = (kt.kind == 1 ? kt.start - p.win_start : kt.start) + gi * kVRows -
+                             (kt.kind == 2 ? kMergeWinRows : 0);
+            mbar_arrive_expect_tx(&bar.full[grp], kVChunks * (small ? kSmallRows : kVRows) * 128);
+            for (int c = 0; c < kVChunks; ++c)
+              tma_load_4d(dst + c * kVChunkBytes, &maps.v[kind][small], &bar.full[grp], col0 + c * 64, hk, row0, b);
+          }
         }
+        next_group();
       };
       auto load_v = [&](const TileSet& ts, int j, int col0) {
         const KeyTile kt = ts.get(j);
-        for (int c = 0; ok && c < kVChunks; c += 2) load_unit(1, kt, col0 + c * 64, ts.hk, ts.b);
+        const int ngv = kt.n > kVRows ? 2 : 1;
+        for (int gi = 0; ok && gi < ngv; ++gi) load_vgroup(kt, gi, col0, ts.hk, ts.b);
       };
       if (blockIdx.x < p.total_units) {
         TileSet t0;
@@ -333,7 +372,7 @@ __global__ void __launch_bounds__(kThreads, 1) hca_attn_kernel(const __grid_cons
         for (int step = 0; ok && step <= ts.J; ++step) {
           if (step < ts.J) {
             const KeyTile kt = ts.get(step);
-            for (int c = 0; ok && c < kQChunks; c += 2) load_unit(0, kt, c * 64, ts.hk, ts.b);
+            for (int c = 0; ok && c < kQChunks; c += 2) load_k(kt, c * 64, ts.hk, ts.b);
           }
           if (ok && step >= 1) load_v(ts, step - 1, 0);
         }
@@ -369,29 +408,31 @@ __global__ void __launch_bounds__(kThreads, 1) hca_attn_kernel(const __grid_cons
       uint32_t g = 0;       // key tiles of all earlier phases
       uint32_t it = 0;      // O halves
       bool ok = true;
-      // N = 128: one PV MMA covers both 64-column chunks of a ring group (LBO = one slot)
-      const uint32_t idesc_pv = idesc_bf16_f32(128, 128, false, true);
+      // N = 256: one PV MMA covers the whole O half, the four 64-column chunks of a V group
+      // (LBO = one 8 KB chunk); its 64 keys take four MMAs of K = 16
+      const uint32_t idesc_pv = idesc_bf16_f32(128, kDHalf, false, true);
       // descriptors of the ring groups and of Q; the start-address field counts 16-byte units
       const uint64_t dq0 = smem_desc_sw128(sQa, 16, 1024);
       const uint64_t dk0 = smem_desc_sw128(sRa, 16, 1024);
-      const uint64_t dv0 = smem_desc_sw128(sRa, kChunkBytes, 1024);
+      const uint64_t dv0 = smem_desc_sw128(sRa, kVChunkBytes, 1024);
       constexpr uint64_t kGroupDesc = kGroupBytes >> 4;  // group offset in descriptor units
-      // PV of key tile j (global counter gj) into the O half; V from two ring groups
+      // PV of key tile j (global counter gj) into the O half; V from one group per 64 keys
       auto pv = [&](const KeyTile& kt, int j, uint32_t gj) {
         const uint32_t tP = tmem + kDHalf + (gj & 1) * kKeyTile;
-        const int nk = kt.n / 16;
-        for (int vu = 0; ok && vu < kVChunks / 2; ++vu, next_group()) {
-          if (j == 0) {  // the previous O half's epilogue must have read these 128 columns
-            ok = mbar_wait(&bar.o_empty[vu], (it & 1) ^ 1, &abort_flag, p.err);
-            if (!ok) break;
-          }
+        if (j == 0) {  // the previous O half's epilogue must have read all of it
+          for (int hh = 0; ok && hh < 2; ++hh) ok = mbar_wait(&bar.o_empty[hh], (it & 1) ^ 1, &abort_flag, p.err);
+          if (!ok) return;
+        }
+        const int ngv = kt.n > kVRows ? 2 : 1;
+        for (int gi = 0; ok && gi < ngv; ++gi, next_group()) {
           ok = mbar_wait(&bar.full[grp], gph, &abort_flag, p.err);
           if (!ok) break;
           tc_fence_after();
           const uint64_t db = dv0 + grp * kGroupDesc;
-          for (int kk = 0; kk < nk; ++kk)
-            mma_ts(tmem + vu * 128, tP + kk * 8, db + (uint64_t)(kk * (2048 >> 4)), idesc_pv,
-                   (j > 0 || kk > 0) ? 1u : 0u);
+          const int nk = min(kVRows, kt.n - gi * kVRows) / 16;
+          for (int kk = 0; kk < nk; ++kk)  // P columns of keys 64 gi + 16 kk .. +15 (bf16 pairs)
+            mma_ts(tmem, tP + (gi * 4 + kk) * 8, db + (uint64_t)(kk * (2048 >> 4)), idesc_pv,
+                   (j > 0 || gi > 0 || kk > 0) ? 1u : 0u);
           mma_commit(&bar.empty[grp]);
         }
       };
@@ -473,7 +514,7 @@ __global__ void __launch_bounds__(kThreads, 1) hca_attn_kernel(const __grid_cons
     const int r = quarter * 32 + lane;  // row of the tile == TMEM lane
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const bool store_issuer = r == 0;
-    uint32_t it = 0, ec = 0, tl = 0;  // O halves, staged stores, row tiles
+    uint32_t it = 0, tl = 0;  // O halves, row tiles
     bool ok = true;
 
     // O half (TMEM) -> normalised bf16 in registers, 128 columns at a time, each 128 columns
@@ -503,38 +544,50 @@ __global__ void __launch_bounds__(kThreads, 1) hca_attn_kernel(const __grid_cons
         ++it;
         return;
       }
+      // O half -> normalised bf16 -> staging (128 columns = four 32-column SW64 boxes) -> TMA
+      // tensor stores.  Columns [0,128) go to the staging while [128,256) are read, so O returns
+      // to the MMA warp after 256 columns of TMEM loads while only 128 are held in registers.
+      uint32_t ob[64];
+      auto read_o = [&](int c0) {  // 16 columns per load keeps ob + v within the register budget
 #pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        uint32_t ob[64];
+        for (int oc = 0; oc < 128; oc += 16) {
+          uint32_t v[16];
+          tmem_ld16(tmem + lane_off + c0 + oc, v);
+          tmem_wait_ld_regs16(v);
 #pragma unroll
-        for (int oc = 0; oc < 128; oc += 32) {
-          uint32_t v[32];
-          tmem_ld32_nowait(tmem + lane_off + hh * 128 + oc, v);
-          tmem_wait_ld_regs(v);
-#pragma unroll
-          for (int i = 0; i < 16; ++i)
+          for (int i = 0; i < 8; ++i)
             ob[oc / 2 + i] = pack_bf16x2(__uint_as_float(v[2 * i]) * inv_l, __uint_as_float(v[2 * i + 1]) * inv_l);
         }
-        tc_fence_before();
-        mbar_arrive(&bar.o_empty[hh]);
+      };
+      auto stage_o = [&]() {  // the stores that last read the staging must be done with it
+        if (store_issuer) bulk_wait_group_read0();
+        softmax_bar_sync();
 #pragma unroll
-        for (int oc = 0; oc < 128; oc += kOutCols) {
-          uint8_t* buf = sOut + (ec & 1) * kOutBufBytes;
-          if (store_issuer && ec >= 2) bulk_wait_group_read1();  // the store from this buffer has read it
-          softmax_bar_sync();
+        for (int q = 0; q < kOutBufs; ++q)
 #pragma unroll
           for (int i = 0; i < 4; ++i)  // 64-byte swizzle: 16-byte unit i of row r at unit i ^ ((r >> 1) & 3)
-            *reinterpret_cast<uint4*>(buf + r * 64 + ((i ^ ((r >> 1) & 3)) * 16)) =
-                make_uint4(ob[oc / 2 + 4 * i], ob[oc / 2 + 4 * i + 1], ob[oc / 2 + 4 * i + 2], ob[oc / 2 + 4 * i + 3]);
-          fence_proxy_async_smem();
-          softmax_bar_sync();
-          if (store_issuer) {
-            tma_store_4d(&maps.o, buf, col0 + hh * 128 + oc, ts.hk * p.g, ts.tok0, ts.b);
-            bulk_commit_group();
-          }
-          ++ec;
+            *reinterpret_cast<uint4*>(sOut + q * kOutBufBytes + r * 64 + ((i ^ ((r >> 1) & 3)) * 16)) =
+                make_uint4(ob[q * 16 + 4 * i], ob[q * 16 + 4 * i + 1], ob[q * 16 + 4 * i + 2], ob[q * 16 + 4 * i + 3]);
+        fence_proxy_async_smem();
+      };
+      auto store_o = [&](int c0) {
+        softmax_bar_sync();
+        if (store_issuer) {
+#pragma unroll
+          for (int q = 0; q < kOutBufs; ++q)
+            tma_store_4d(&maps.o, sOut + q * kOutBufBytes, col0 + c0 + q * kOutCols, ts.hk * p.g, ts.tok0, ts.b);
+          bulk_commit_group();
         }
-      }
+      };
+      read_o(0);
+      stage_o();
+      read_o(128);
+      tc_fence_before();
+      mbar_arrive(&bar.o_empty[0]);
+      mbar_arrive(&bar.o_empty[1]);
+      store_o(0);
+      stage_o();
+      store_o(128);
       ++it;
     };
 
@@ -949,24 +1002,23 @@ extern "C" hcadsa_status hca_attn_fwd(const hcadsa_bf16* Q, const hcadsa_bf16* K
   Maps maps;
   if (!make_map_4d(&maps.q, Q, kD, Hq, Lq, B, 64, g, G.TT, 128)) return HCADSA_ERR_CUDA;
   if (!make_map_4d(&maps.o, O, kD, Hq, Lq, B, kOutCols, g, G.TT, 64)) return HCADSA_ERR_CUDA;
-  for (int kv = 0; kv < 2; ++kv) {
-    const hcadsa_bf16* win = kv ? Vw : Kw;
-    const hcadsa_bf16* ent = n_c > 0 ? (kv ? Vc : Kc) : win;  // no query sees an entry without n_c > 0
-    const int ent_rows = n_c > 0 ? n_c : n_w;
-    if (!make_map_4d(&maps.merge[kv][0], win, kD, Hkv, n_w, B, 64, 1, kMergeWinRows, 128)) return HCADSA_ERR_CUDA;
-    if (!make_map_4d(&maps.merge[kv][1], ent, kD, Hkv, ent_rows, B, 64, 1, kMergeEntRows, 128))
+  {
+    // entries of the merged tiles exist only when n_c > 0; otherwise those maps are never read
+    const hcadsa_bf16* KcM = n_c > 0 ? Kc : Kw;
+    const hcadsa_bf16* VcM = n_c > 0 ? Vc : Vw;
+    const int rows_c = n_c > 0 ? n_c : n_w;
+    if (!make_map_4d(&maps.kmerge[0], Kw, kD, Hkv, n_w, B, 64, 1, kMergeWinRows, 128) ||
+        !make_map_4d(&maps.kmerge[1], KcM, kD, Hkv, rows_c, B, 64, 1, kMergeEntRows, 128) ||
+        !make_map_4d(&maps.vmerge[0], Vw, kD, Hkv, n_w, B, 64, 1, kMergeWinRows, 128) ||
+        !make_map_4d(&maps.vmerge[1], VcM, kD, Hkv, rows_c, B, 64, 1, kVRows - kMergeWinRows, 128))
       return HCADSA_ERR_CUDA;
-  }
-  for (int small = 0; small < 2; ++small) {
-    const int rows = small ? kSmallRows : 128;
-    if (!make_map_4d(&maps.kv[0][1][small], Kw, kD, Hkv, n_w, B, 64, 1, rows, 128)) return HCADSA_ERR_CUDA;
-    if (!make_map_4d(&maps.kv[1][1][small], Vw, kD, Hkv, n_w, B, 64, 1, rows, 128)) return HCADSA_ERR_CUDA;
-    if (n_c > 0) {
-      if (!make_map_4d(&maps.kv[0][0][small], Kc, kD, Hkv, n_c, B, 64, 1, rows, 128)) return HCADSA_ERR_CUDA;
-      if (!make_map_4d(&maps.kv[1][0][small], Vc, kD, Hkv, n_c, B, 64, 1, rows, 128)) return HCADSA_ERR_CUDA;
-    } else {  // no query sees an entry: these maps are never read
-      maps.kv[0][0][small] = maps.kv[0][1][small];
-      maps.kv[1][0][small] = maps.kv[1][1][small];
+    for (int small = 0; small < 2; ++small) {
+      const int krows = small ? kSmallRows : kKeyTile, vrows = small ? kSmallRows : kVRows;
+      if (!make_map_4d(&maps.k[1][small], Kw, kD, Hkv, n_w, B, 64, 1, krows, 128) ||
+          !make_map_4d(&maps.v[1][small], Vw, kD, Hkv, n_w, B, 64, 1, vrows, 128) ||
+          !make_map_4d(&maps.k[0][small], KcM, kD, Hkv, rows_c, B, 64, 1, krows, 128) ||
+          !make_map_4d(&maps.v[0][small], VcM, kD, Hkv, rows_c, B, 64, 1, vrows, 128))
+        return HCADSA_ERR_CUDA;
     }
   }
   Params p;
