@@ -255,7 +255,7 @@ class Step:
         if ev: ev[4].record()
 
 
-def run_decode(hd, device, iters=5):
+def run_decode(hd, device, iters=20):
     """Batch 32 single-token queries at t = 1,048,575: HCA layer and DSA layer, HBM-bound."""
     B, t = DEC.B, DEC.t
     g = torch.Generator(device=device)

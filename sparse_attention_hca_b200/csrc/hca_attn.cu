@@ -647,10 +647,10 @@ __global__ void __launch_bounds__(kThreads, 1) hca_attn_kernel(const __grid_cons
           lo2 = max(ws_t - kt.wstart, 0);
           hi2 = min(t + 1 - kt.wstart, kt.wn);
         }
-        if (!row_valid) {  // padding rows see nothing
-          hi = lo;
-          hi2 = lo2;
-        }
+        // Padding rows (tokens past Lq: a partial last tile, 7 of the 8 token slots of a decode
+        // tile) keep the last token's intervals.  Their Q rows are TMA zero fill, so their scores
+        // are 0 and their P finite, and nothing of theirs is stored; an empty interval would only
+        // push their warps off the all-visible fast paths below.
         const uint32_t tS = tmem + lane_off + kDHalf + (gs & 1) * kKeyTile;
         ok = mbar_wait(&bar.s_full[gs & 1], (s_par >> (gs & 1)) & 1, &abort_flag, p.err);
         if (!ok) break;
