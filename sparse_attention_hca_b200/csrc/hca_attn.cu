@@ -125,6 +125,17 @@ __device__ __forceinline__ int window_start(int t, int W) {
   return s > 0 ? s : 0;
 }
 
+// tcgen05.wait::ld naming the 16 destination registers of the loads it completes, so the
+// compiler cannot move their uses above the wait
+__device__ __forceinline__ void tmem_wait_ld_regs16(uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.wait::ld.sync.aligned;"
+      : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+        "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15])
+      :
+      : "memory");
+}
+
 __device__ __forceinline__ void softmax_bar_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_group_read1() {
   asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
