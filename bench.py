@@ -521,8 +521,15 @@ def reference(args):
 
 def only_kernel(args):
     """Runs one library kernel alone at sequence length --seq-len (profiling driver): W warm-up
-    and K timed launches; prints a small JSON record (not the benchmark contract line)."""
+    and K timed launches; prints a small JSON record (not the benchmark contract line).
+    --only decode runs the decode step instead."""
     import sparse_attention_hca_b200 as hd
+
+    if args.only == "decode":
+        out = run_decode(hd, torch.device("cuda", 0), iters=max(1, args.steps))
+        hd.hcadsa_check_device_error()
+        print(json.dumps(out))
+        return
 
     global L
     L = args.seq_len
@@ -559,8 +566,9 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", choices=["compress", "hca_attn", "index_topk", "dsa_attn"],
-                    help="profiling driver: run one kernel alone at --seq-len")
+    ap.add_argument("--only", choices=["compress", "hca_attn", "index_topk", "dsa_attn", "decode"],
+                    help="profiling driver: run one kernel alone at --seq-len, or the decode step "
+                         "(B = 32 at t = 1,048,575; --steps timed steps after 3 warm-up steps)")
     ap.add_argument("--seq-len", type=int, default=L)
     args = ap.parse_args()
     if args.only:

@@ -825,49 +825,49 @@ __global__ void __launch_bounds__(kThreads, 1) hca_attn_kernel(const __grid_cons
 
 // Split key ranges: row r of row tile T gathers its units' partial results,
 //     M = max_s m_s,  w_s = 2^(m_s - M),  O = sum_s w_s O_s / sum_s w_s l_s,
-// (m_s in log2 units, O_s and l_s relative to 2^m_s) and writes O (bf16) and lse.
-// One warp per row (8 rows per CTA, blockIdx.y = row group) and 128-column slice (blockIdx.z),
-// 4 columns per lane.
+// (m_s in log2 units, O_s and l_s relative to 2^m_s; units with l_s = 0 saw no key and drop
+// out) and writes O (bf16) and lse.  One warp per row (8 rows per CTA, blockIdx.y = row
+// group) and 128-column slice (blockIdx.z), 4 columns per lane.  A row tile has at most 64
+// units: lane i reads the (m, l) of units i and i + 32 in one round, the warp reduces M and
+// L, and the O loads of all units are independent of one another.
 __global__ void __launch_bounds__(256) hca_combine_kernel(const Params p, uint16_t* __restrict__ O) {
   const int T = blockIdx.x;
   const int bh = T / p.n_tiles, tile = T % p.n_tiles;
   const int b = bh / p.Hkv, hk = bh % p.Hkv;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  {
-    const int r = blockIdx.y * 8 + warp;
-    const int tok = tile * p.TT + r / p.g;
-    if (tok >= p.Lq) return;
-    const int h = hk * p.g + r % p.g;
-    float M = -INFINITY;
-    const int U0 = first_unit(T, p), S = n_splits(T, p);
-    for (int sp = 0; sp < S; ++sp) M = fmaxf(M, p.part_ml[((size_t)U0 + sp) * 128 + r].x);
-    float L = 0.0f;
-    for (int sp = 0; sp < S; ++sp) {
-      const float2 ml = p.part_ml[((size_t)U0 + sp) * 128 + r];
-      L += ml.y > 0.0f ? exp2f(ml.x - M) * ml.y : 0.0f;
-    }
-    const float inv_L = L > 0.0f ? 1.0f / L : 0.0f;
-    uint16_t* orow = O + (((size_t)b * p.Lq + tok) * p.Hq + h) * kD;
-    {
-      const int c = blockIdx.z * 128 + lane * 4;  // this CTA's 128-column slice of the row
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int sp = 0; sp < S; ++sp) {
-        const size_t U = (size_t)U0 + sp;
-        const float2 ml = p.part_ml[U * 128 + r];
-        if (!(ml.y > 0.0f)) continue;
-        const float w = exp2f(ml.x - M);
-        const float4 o = *reinterpret_cast<const float4*>(p.part_o + (U * 128 + r) * kD + c);
-        acc.x += w * o.x;
-        acc.y += w * o.y;
-        acc.z += w * o.z;
-        acc.w += w * o.w;
-      }
-      *reinterpret_cast<uint2*>(orow + c) =
-          make_uint2(pack_bf16x2(acc.x * inv_L, acc.y * inv_L), pack_bf16x2(acc.z * inv_L, acc.w * inv_L));
-    }
-    if (blockIdx.z == 0 && lane == 0 && p.lse)
-      p.lse[((size_t)b * p.Lq + tok) * p.Hq + h] = (M + __log2f(L)) * 0.69314718055994531f;
+  const int r = blockIdx.y * 8 + warp;
+  const int tok = tile * p.TT + r / p.g;
+  if (tok >= p.Lq) return;
+  const int h = hk * p.g + r % p.g;
+  const int U0 = first_unit(T, p), S = n_splits(T, p);
+  float2 ml0 = make_float2(-INFINITY, 0.0f), ml1 = make_float2(-INFINITY, 0.0f);
+  if (lane < S) ml0 = p.part_ml[((size_t)U0 + lane) * 128 + r];
+  if (lane + 32 < S) ml1 = p.part_ml[((size_t)U0 + lane + 32) * 128 + r];
+  float M = fmaxf(ml0.y > 0.0f ? ml0.x : -INFINITY, ml1.y > 0.0f ? ml1.x : -INFINITY);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  const float w0 = ml0.y > 0.0f ? exp2f(ml0.x - M) : 0.0f;
+  const float w1 = ml1.y > 0.0f ? exp2f(ml1.x - M) : 0.0f;
+  float L = w0 * ml0.y + w1 * ml1.y;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+  const float inv_L = L > 0.0f ? 1.0f / L : 0.0f;
+  uint16_t* orow = O + (((size_t)b * p.Lq + tok) * p.Hq + h) * kD;
+  const int c = blockIdx.z * 128 + lane * 4;  // this CTA's 128-column slice of the row
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+  for (int sp = 0; sp < S; ++sp) {  // every unit wrote its valid rows (zeros where it saw no key)
+    const float w = __shfl_sync(0xffffffffu, sp < 32 ? w0 : w1, sp & 31);
+    const float4 o = *reinterpret_cast<const float4*>(p.part_o + (((size_t)U0 + sp) * 128 + r) * kD + c);
+    acc.x += w * o.x;
+    acc.y += w * o.y;
+    acc.z += w * o.z;
+    acc.w += w * o.w;
   }
+  *reinterpret_cast<uint2*>(orow + c) =
+      make_uint2(pack_bf16x2(acc.x * inv_L, acc.y * inv_L), pack_bf16x2(acc.z * inv_L, acc.w * inv_L));
+  if (blockIdx.z == 0 && lane == 0 && p.lse)
+    p.lse[((size_t)b * p.Lq + tok) * p.Hq + h] = (M + __log2f(L)) * 0.69314718055994531f;
 }
 
 bool make_map_4d(CUtensorMap* m, const void* base, int d, int heads, int rows, int B, int box_cols, int box_heads,
@@ -949,7 +949,7 @@ hcadsa_status geometry(Geometry* G, int B, int Lq, int q_offset, int Hq, int Hkv
       splits = J_min;
       extra = 0;
     }
-    if (splits > 64) {
+    if (splits + (extra ? 1 : 0) > 64) {  // the combine pass takes at most 64 units per row tile
       splits = 64;
       extra = 0;
     }

@@ -245,6 +245,27 @@ def test_hca_decode_uneven_splits(hd):
     np.testing.assert_allclose(lse.reshape(B, Hq).cpu().numpy(), ref_lse, atol=2e-2, rtol=0)
 
 
+@pytest.mark.parametrize("B", [1, 2])
+def test_hca_decode_many_units(hd, B):
+    """One or two sequences at t = 1,048,575: 65 key tiles per row tile, split over the SMs
+    into the maximum of 64 units per row tile, so the combine pass gathers units 32-63 too."""
+    d, Hq, blk, W, t = 512, 16, 128, 128, 1048575
+    n_c = (t + 1) // blk - 1  # entries the query needs (8191), as a decode cache holds them
+    ws = t - W + 1
+    Kc = synth.normal_bf16((B, n_c, 1, d), 1.0, 61, "K")
+    Vc = synth.normal_bf16((B, n_c, 1, d), 1.0, 61, "V")
+    Kw = synth.normal_bf16((B, W, 1, d), 1.0, 62, "K")
+    Vw = synth.normal_bf16((B, W, 1, d), 1.0, 62, "V")
+    Q = synth.normal_bf16((B, 1, Hq, d), 1.0, 63, "Q")
+    O, lse = hd.hca_attn_fwd(Q.cuda(), Kc.cuda(), Vc.cuda(), Kw.cuda(), Vw.cuda(), win_start=ws, q_offset=t,
+                             return_lse=True)
+    no_device_error(hd)
+    ref, ref_lse = oracle.hca_attn(bits(Q), bits(Kc), bits(Vc), bits(Kw), bits(Vw), win_start=ws, q_offset=t,
+                                   with_lse=True)
+    print(check_attn(O.reshape(B, Hq, d), ref, f"hca decode B={B} t=1M"))
+    np.testing.assert_allclose(lse.reshape(B, Hq).cpu().numpy(), ref_lse, atol=2e-2, rtol=0)
+
+
 # ------------------------------------------------------------------ DSA indexer + top-k
 
 def _dsa_cfg(name, L, B=1, k=2048, sigma=None):
