@@ -62,9 +62,9 @@ constexpr int kKeyTile = 128;
 constexpr int kSmallRows = 32;  // TMA box height for key tiles of at most 32 keys
 constexpr int kMergeWinRows = 16;                       // window keys at the head of a merged tile
 constexpr int kMergeEntRows = kKeyTile - kMergeWinRows;  // compressed entries after them
-// Ring: groups of two 16 KB chunk slots (128 d-columns of a key tile).  Two groups, plus a third
-// in the epilogue staging area when key ranges are split (those epilogues write fp32 partials
-// straight to global memory, and their K/V stream from HBM, where depth pays).
+// Ring: 32 KB groups (a K group: two 16 KB chunks of 128 rows; a V group: four 8 KB chunks of 64
+// rows).  Two groups; the third group's space is the epilogue's staging area, or a third group
+// when key ranges are split (those epilogues write fp32 partials straight to global memory).
 constexpr int kGroups = 2;
 constexpr int kMaxGroups = 3;
 constexpr int kChunkBytes = 128 * 128;  // 128 rows x 64 bf16
@@ -528,9 +528,8 @@ __global__ void __launch_bounds__(kThreads, 1) hca_attn_kernel(const __grid_cons
     uint32_t it = 0, tl = 0;  // O halves, row tiles
     bool ok = true;
 
-    // O half (TMEM) -> normalised bf16 in registers, 128 columns at a time, each 128 columns
-    // released to the MMA warp as soon as they are read -> two 8 KB staging buffers -> TMA
-    // tensor stores.  With split key ranges the unit's unnormalised fp32 O rows go to part_o.
+    // One O half per call.  With split key ranges the unit's unnormalised fp32 O rows go
+    // straight to part_o; otherwise they are normalised, staged and stored (below).
     auto epilogue = [&](const TileSet& ts, int col0, float inv_l, int U, bool row_valid) {
       ok = mbar_wait(&bar.o_full, it & 1, &abort_flag, p.err);
       if (!ok) return;
