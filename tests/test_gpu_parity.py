@@ -245,6 +245,28 @@ def test_hca_decode_uneven_splits(hd):
     np.testing.assert_allclose(lse.reshape(B, Hq).cpu().numpy(), ref_lse, atol=2e-2, rtol=0)
 
 
+def test_hca_chunked_prefill(hd):
+    """A prefill chunk: 1500 query tokens at positions 4000..5499 of two sequences, over the
+    entries stored so far and a window buffer that starts at the first query's window (many
+    row tiles: the unsplit path, with merged key tiles at an offset)."""
+    d, Hq, blk, W, B, Lq, t0 = 512, 16, 128, 128, 2, 1500, 4000
+    t_last = t0 + Lq - 1
+    n_c = (t_last - W + 1) // blk
+    ws = t0 - W + 1
+    Kc = synth.normal_bf16((B, n_c, 1, d), 1.0, 71, "K")
+    Vc = synth.normal_bf16((B, n_c, 1, d), 1.0, 71, "V")
+    Kw = synth.normal_bf16((B, t_last + 1 - ws, 1, d), 1.0, 72, "K")
+    Vw = synth.normal_bf16((B, t_last + 1 - ws, 1, d), 1.0, 72, "V")
+    Q = synth.normal_bf16((B, Lq, Hq, d), 1.0, 73, "Q")
+    O, lse = hd.hca_attn_fwd(Q.cuda(), Kc.cuda(), Vc.cuda(), Kw.cuda(), Vw.cuda(), win_start=ws, q_offset=t0,
+                             return_lse=True)
+    no_device_error(hd)
+    ref, ref_lse = oracle.hca_attn(bits(Q), bits(Kc), bits(Vc), bits(Kw), bits(Vw), win_start=ws, q_offset=t0,
+                                   with_lse=True)
+    print(check_attn(O.reshape(B * Lq, Hq, d), ref, "hca chunked prefill"))
+    np.testing.assert_allclose(lse.reshape(B * Lq, Hq).cpu().numpy(), ref_lse, atol=2e-2, rtol=0)
+
+
 @pytest.mark.parametrize("B", [1, 2])
 def test_hca_decode_many_units(hd, B):
     """One or two sequences at t = 1,048,575: 65 key tiles per row tile, split over the SMs
@@ -348,6 +370,20 @@ def test_topk_decode_many_rows_split_select(hd):
     q = torch.randint(-8, 9, (B, Lq, 4, 64), generator=g).to(torch.int8)
     kk = torch.randint(-8, 9, (B, t0 + Lq, 64), generator=g).to(torch.int8)
     w = torch.tensor([2, 1, 4, 3], dtype=torch.int32)
+    idx = hd.dsa_index_topk(q.cuda(), kk.cuda(), w.cuda(), k, q_offset=t0)
+    no_device_error(hd)
+    ref = oracle.dsa_topk(q.numpy(), kk.numpy(), w.numpy(), k, q_offset=t0)
+    assert np.array_equal(idx.cpu().numpy().reshape(B * Lq, k), ref)
+
+
+def test_topk_chunked_prefill(hd):
+    """A prefill chunk: 600 query rows at positions 3000..3599 over 3600 keys (the tiled scorer
+    and single-block selection with a query offset), bit-exact on every row."""
+    B, Lq, t0, k = 2, 600, 3000, 2048
+    g = torch.Generator().manual_seed(43)
+    q = torch.randint(-8, 9, (B, Lq, 4, 64), generator=g).to(torch.int8)
+    kk = torch.randint(-8, 9, (B, t0 + Lq, 64), generator=g).to(torch.int8)
+    w = torch.tensor([3, 1, 2, 4], dtype=torch.int32)
     idx = hd.dsa_index_topk(q.cuda(), kk.cuda(), w.cuda(), k, q_offset=t0)
     no_device_error(hd)
     ref = oracle.dsa_topk(q.numpy(), kk.numpy(), w.numpy(), k, q_offset=t0)
