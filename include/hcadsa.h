@@ -110,10 +110,12 @@ hcadsa_status hca_compress_kv(const hcadsa_bf16* K, const hcadsa_bf16* V, const 
  * where #tiles = B * Hkv * ceil(Lq / (128 / (Hq/Hkv))) row tiles and J_max =
  * ceil(n_c(t_last)/128) + floor((128/(Hq/Hkv) + W + 126) / 128) key tiles.  #units =
  * #tiles, except when #tiles <= #SMs/2: then every row tile's key tiles are split over
- * several CTAs (#units <= #SMs, at most 64 per row tile, each with at least one key tile),
- * and the workspace also holds each unit's partial result, 128 * (512*4 + 8) bytes per
- * unit, for the combine pass.  The workspace holds no state between calls; concurrent
- * calls need separate workspaces.
+ * several CTAs (#units <= #SMs, at most 64 per row tile, each with at least one key tile;
+ * when all row tiles have the same number of key tiles, as in decode, each of #SMs CTAs
+ * takes an equal share of all of them and #units = #SMs + #tiles record slots), and the
+ * workspace also holds each unit's partial result, 128 * (512*4 + 8) bytes per unit, for
+ * the combine pass.  The workspace holds no state between calls; concurrent calls need
+ * separate workspaces.
  */
 size_t hca_attn_fwd_workspace_size(int B, int Lq, int q_offset, int Hq, int Hkv, int d, int n_c, int blk,
                                    int W);

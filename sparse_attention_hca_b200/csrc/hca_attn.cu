@@ -95,7 +95,10 @@ struct Params {
   int splits;       // work units per row tile (key tiles split among them) ...
   int split_extra;  // ... plus one more for the first split_extra row tiles
   int split_mode;   // units write partial results for the combine pass
-  int total_units;  // total_tiles * splits + split_extra
+  int total_units;  // total_tiles * splits + split_extra (stream_k: record slots, grid + total_tiles)
+  int stream_k;     // split mode with equal row tiles: CTA c takes key tiles [c*Jtot/G, (c+1)*Jtot/G)
+  int J_all;        // stream_k: key tiles of every row tile (Jtot = total_tiles * J_all)
+  int sk_grid;      // stream_k: G, the attention kernel's grid
   int J_max;        // key tiles of the longest row tile (scratch capacity)
   float scale_log2;
   float* lse;
@@ -152,8 +155,51 @@ struct KeyTile {
 __host__ __device__ inline int first_unit(int T, const Params& p) { return T * p.splits + min(T, p.split_extra); }
 __host__ __device__ inline int n_splits(int T, const Params& p) { return p.splits + (T < p.split_extra ? 1 : 0); }
 
+// Stream-K split (every row tile has J_all key tiles): all row tiles' key tiles laid end to end,
+// Jtot = total_tiles * J_all of them, and CTA c takes [c*Jtot/G, (c+1)*Jtot/G).  Its piece of row
+// tile T is the unit with record index c + T (unique: both grow along the key-tile order), so a
+// CTA's units are consecutive records and so are a row tile's: CTAs c_first(T) .. c_last(T), the
+// ones holding the row tile's first and last key tiles.
+// (The host enables it only while Jtot * (G + 1) < 2^31, so 32-bit arithmetic is exact.)
+__host__ __device__ inline int sk_cta_start(int c, const Params& p) {
+  return (int)((unsigned)c * (unsigned)(p.total_tiles * p.J_all) / (unsigned)p.sk_grid);
+}
+__host__ __device__ inline int sk_cta_of(int x, const Params& p) {  // CTA holding global key tile x
+  return (int)(((unsigned)(x + 1) * (unsigned)p.sk_grid - 1u) / (unsigned)(p.total_tiles * p.J_all));
+}
+
+// The units (record indices) this CTA processes: first, first + step, ... below end, with
+// step = 1 (stream_k) or gridDim.x.  With stream_k the CTA also keeps its key-tile range
+// [lo, hi).  Kept in shared memory (set once at kernel start) and read where needed, so the
+// per-unit loops do not hold them in registers.
+struct UnitInfo {
+  int first, end;   // units
+  int js_first;     // stream_k: first key tile of the first unit (later units start at 0)
+  int je_last;      // stream_k: end key tile of the last unit (earlier units end at J_all)
+};
+__device__ __forceinline__ UnitInfo unit_info(const Params& p) {
+  UnitInfo u;
+  if (p.stream_k) {
+    const int lo = sk_cta_start(blockIdx.x, p), hi = sk_cta_start(blockIdx.x + 1, p);
+    const int T0 = lo / p.J_all, T1 = (hi - 1) / p.J_all;
+    u.first = (int)blockIdx.x + T0;
+    u.end = (int)blockIdx.x + T1 + 1;
+    u.js_first = lo - T0 * p.J_all;
+    u.je_last = hi - T1 * p.J_all;
+  } else {
+    u.first = (int)blockIdx.x;
+    u.end = p.total_units;
+    u.js_first = 0;
+    u.je_last = 0;
+  }
+  return u;
+}
+__device__ __forceinline__ int unit_step(const Params& p) { return p.stream_k ? 1 : (int)gridDim.x; }
+__shared__ UnitInfo s_units;  // this CTA's units, set once by thread 0 at kernel start
+
 // The key tiles of one work unit: split s of row tile T (S = n_splits(T) units from
-// first_unit(T)) takes the row tile's key tiles [s*Jt/S, (s+1)*Jt/S).
+// first_unit(T)) takes the row tile's key tiles [s*Jt/S, (s+1)*Jt/S); with stream_k, unit
+// c + T of CTA c takes the row tile's share of [c*Jtot/G, (c+1)*Jtot/G).
 struct TileSet {
   int b, hk, tok0;  // batch, kv head, first token (relative to q_offset)
   int J_c, J;       // number of compressed tiles of the row tile, key tiles of this unit
@@ -164,9 +210,27 @@ struct TileSet {
   int w_part;       // keys of the band beyond its whole 128-key tiles (1..128)
   int merged;       // 1: the band's first w_part keys share the last compressed tile
   __device__ void init(int U, const Params& p) {
-    const int big = p.split_extra * (p.splits + 1);  // units of the row tiles with an extra split
-    const int T = U < big ? U / (p.splits + 1) : p.split_extra + (U - big) / p.splits;
-    const int split = U - first_unit(T, p), S = n_splits(T, p);
+    int T, split = 0, S = 1;
+    if (p.stream_k) {
+      T = U - (int)blockIdx.x;
+    } else {
+      const int big = p.split_extra * (p.splits + 1);  // units of the row tiles with an extra split
+      T = U < big ? U / (p.splits + 1) : p.split_extra + (U - big) / p.splits;
+      split = U - first_unit(T, p);
+      S = n_splits(T, p);
+    }
+    init_tile(T, p);
+    const int Jt = J;
+    if (p.stream_k) {  // Jt == J_all
+      js = U == s_units.first ? s_units.js_first : 0;
+      J = (U == s_units.end - 1 ? s_units.je_last : Jt) - js;
+    } else {
+      js = split * Jt / S;
+      J = (split + 1) * Jt / S - js;
+    }
+  }
+  // row tile T: everything but the key-tile range of the unit (J = all of the row tile's tiles)
+  __device__ __forceinline__ void init_tile(int T, const Params& p) {
     const int bh = T / p.n_tiles, tile = T % p.n_tiles;
     b = bh / p.Hkv;
     hk = bh % p.Hkv;
@@ -179,9 +243,8 @@ struct TileSet {
     const int n_wt = (w_span + kKeyTile - 1) / kKeyTile;
     w_part = w_span - (n_wt - 1) * kKeyTile;
     merged = J_c >= 1 && n_wt >= 2 && w_part <= kMergeWinRows && nc_hi - (J_c - 1) * kKeyTile <= kMergeEntRows;
-    const int Jt = J_c + n_wt - merged;
-    js = split * Jt / S;
-    J = (split + 1) * Jt / S - js;
+    J = J_c + n_wt - merged;
+    js = 0;
   }
   __device__ KeyTile get(int jl) const {
     KeyTile kt;
@@ -255,7 +318,7 @@ __device__ __forceinline__ void rescale_o(uint32_t t_row, float alpha) {
   tmem_wait_st();
 }
 
-__global__ void __launch_bounds__(kThreads, 1) hca_attn_kernel(const __grid_constant__ Maps maps, const Params p) {
+__global__ void __launch_bounds__(kThreads, 1) hca_attn_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;
@@ -263,6 +326,7 @@ __global__ void __launch_bounds__(kThreads, 1) hca_attn_kernel(const __grid_cons
   uint8_t* sOut = sRing + kGroups * kGroupBytes;
   __shared__ Barriers bar;
   __shared__ float inv_l_sh[2][128];  // 1/l per row (1 in split mode), double-buffered by row tile
+  UnitInfo& ui = s_units;
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_flag;
 
@@ -287,6 +351,7 @@ __global__ void __launch_bounds__(kThreads, 1) hca_attn_kernel(const __grid_cons
       mbar_init(&bar.l_empty[s], 128);
     }
     abort_flag = 0;
+    ui = unit_info(p);
     fence_mbarrier_init();
   }
   if (warp == 1) {
@@ -367,15 +432,15 @@ __global__ void __launch_bounds__(kThreads, 1) hca_attn_kernel(const __grid_cons
         const int ngv = kt.n > kVRows ? 2 : 1;
         for (int gi = 0; ok && gi < ngv; ++gi) load_vgroup(kt, gi, col0, ts.hk, ts.b);
       };
-      if (blockIdx.x < p.total_units) {
+      if (ui.first < ui.end) {
         TileSet t0;
-        t0.init(blockIdx.x, p);
+        t0.init(ui.first, p);
         mbar_arrive_expect_tx(&bar.q_full, kQBytes);
         for (int c = 0; c < kQChunks; ++c)
           tma_load_4d(sQ + c * kChunkBytes, &maps.q, &bar.q_full, c * 64, t0.hk * p.g, t0.tok0, t0.b);
       }
       uint32_t tcount = 0;
-      for (int T = blockIdx.x; ok && T < p.total_units; T += gridDim.x, ++tcount) {
+      for (int T = ui.first; ok && T < ui.end; T += unit_step(p), ++tcount) {
         TileSet ts;
         ts.init(T, p);
         if (ts.J > p.J_max) break;
@@ -389,8 +454,8 @@ __global__ void __launch_bounds__(kThreads, 1) hca_attn_kernel(const __grid_cons
         }
         if (!ok) break;
         // the next tile's Q, once this tile's last S MMA has read the buffer
-        const int Tn = T + gridDim.x;
-        if (Tn < p.total_units) {
+        const int Tn = T + unit_step(p);
+        if (Tn < ui.end) {
           TileSet tn;
           tn.init(Tn, p);
           ok = mbar_wait(&bar.q_empty, tcount & 1, &abort_flag, p.err);
@@ -447,7 +512,7 @@ __global__ void __launch_bounds__(kThreads, 1) hca_attn_kernel(const __grid_cons
           mma_commit(&bar.empty[grp]);
         }
       };
-      for (int T = blockIdx.x; ok && T < p.total_units; T += gridDim.x, ++tcount) {
+      for (int T = ui.first; ok && T < ui.end; T += unit_step(p), ++tcount) {
         TileSet ts;
         ts.init(T, p);
         if (ts.J > p.J_max) {
@@ -601,7 +666,7 @@ __global__ void __launch_bounds__(kThreads, 1) hca_attn_kernel(const __grid_cons
       ++it;
     };
 
-    for (int T = blockIdx.x; ok && T < p.total_units; T += gridDim.x, ++tl) {
+    for (int T = ui.first; ok && T < ui.end; T += unit_step(p), ++tl) {
       TileSet ts;
       ts.init(T, p);
       if (ts.J > p.J_max) break;
@@ -628,7 +693,7 @@ __global__ void __launch_bounds__(kThreads, 1) hca_attn_kernel(const __grid_cons
     uint32_t s_par = 0;
     bool ok = true;
 
-    for (int T = blockIdx.x; ok && T < p.total_units; T += gridDim.x, ++tl) {
+    for (int T = ui.first; ok && T < ui.end; T += unit_step(p), ++tl) {
       TileSet ts;
       ts.init(T, p);
       if (ts.J > p.J_max) break;
@@ -838,7 +903,15 @@ __global__ void __launch_bounds__(256) hca_combine_kernel(const Params p, uint16
   const int tok = tile * p.TT + r / p.g;
   if (tok >= p.Lq) return;
   const int h = hk * p.g + r % p.g;
-  const int U0 = first_unit(T, p), S = n_splits(T, p);
+  int U0, S;
+  if (p.stream_k) {
+    const int cf = sk_cta_of(T * p.J_all, p), cl = sk_cta_of((T + 1) * p.J_all - 1, p);
+    U0 = cf + T;
+    S = cl - cf + 1;
+  } else {
+    U0 = first_unit(T, p);
+    S = n_splits(T, p);
+  }
   float2 ml0 = make_float2(-INFINITY, 0.0f), ml1 = make_float2(-INFINITY, 0.0f);
   if (lane < S) ml0 = p.part_ml[((size_t)U0 + lane) * 128 + r];
   if (lane + 32 < S) ml1 = p.part_ml[((size_t)U0 + lane + 32) * 128 + r];
@@ -892,6 +965,7 @@ int num_sms() {
 // shapes the kernel does not take, HCADSA_ERR_CUDA if the device cannot be queried.
 struct Geometry {
   int g, TT, n_tiles, total_tiles, splits, split_extra, total_units, grid, J_max;
+  int stream_k, J_all;  // stream-K split of equal row tiles (see sk_cta_start)
   size_t scratch_bytes;   // probability tiles: grid * J_max * kScratchTileBytes
   size_t part_bytes;      // split mode: unnormalised O rows and (max, sum) of every unit
   size_t workspace_bytes;
@@ -932,12 +1006,34 @@ hcadsa_status geometry(Geometry* G, int B, int Lq, int q_offset, int Hq, int Hkv
   // Few row tiles (decode: one token per sequence) leave most SMs idle: split every row tile's
   // key tiles into `splits` units (each unit keeps at least one key tile) and combine after.
   long long splits = 1, extra = 0;
+  int stream_k = 0;
+  long long J_all = 0;
   if (2 * total <= sms) {
-    long long J_min = J_max;
+    long long J_min = J_max, J_hi = 0;
     for (long long t = 0; t < n_tiles; ++t) {
       const long long tok0 = t * TT, tok_hi = (tok0 + TT < Lq ? tok0 + TT : Lq) - 1;
       const long long J = host_tile_J(q_offset, tok0, tok_hi, W, blk);
       J_min = J < J_min ? J : J_min;
+      J_hi = J > J_hi ? J : J_hi;
+    }
+    // Equal row tiles (decode: one token per sequence, all at the same position): stream-K, every
+    // CTA an equal share of all key tiles, as long as each CTA gets one and no row tile is split
+    // into more than 64 units (the combine pass's limit).  Units per row tile otherwise differ by
+    // one (13 against 16.25 key tiles per unit at B = 32, t = 1M).
+    if (J_min == J_hi && total * J_min >= sms && total * J_min * (sms + 1) < 2147483647LL) {
+      Params q{};
+      q.total_tiles = (int)total;
+      q.J_all = (int)J_min;
+      q.sk_grid = sms;
+      int S_max = 0;
+      for (long long T = 0; T < total; ++T) {
+        const int S = sk_cta_of((int)((T + 1) * J_min - 1), q) - sk_cta_of((int)(T * J_min), q) + 1;
+        S_max = S > S_max ? S : S_max;
+      }
+      if (S_max <= 64) {
+        stream_k = 1;
+        J_all = J_min;
+      }
     }
     // one unit per SM: sms / total units per row tile, one more for the first sms % total
     // (two units per SM balance the key tiles better but measured slower at B = 32, t = 1M:
@@ -957,10 +1053,19 @@ hcadsa_status geometry(Geometry* G, int B, int Lq, int q_offset, int Hq, int Hkv
   G->TT = TT;
   G->n_tiles = (int)n_tiles;
   G->total_tiles = (int)total;
-  G->splits = (int)splits;
-  G->split_extra = (int)extra;
-  G->total_units = (int)(total * splits + extra);
-  G->grid = G->total_units < sms ? G->total_units : sms;
+  G->stream_k = stream_k;
+  G->J_all = (int)J_all;
+  if (stream_k) {  // records c + T: at most sms + total of them
+    G->splits = 1;
+    G->split_extra = 0;
+    G->total_units = (int)(sms + total);
+    G->grid = sms;
+  } else {
+    G->splits = (int)splits;
+    G->split_extra = (int)extra;
+    G->total_units = (int)(total * splits + extra);
+    G->grid = G->total_units < sms ? G->total_units : sms;
+  }
   G->J_max = (int)J_max;
   G->scratch_bytes = (size_t)G->grid * (size_t)J_max * kScratchTileBytes;
   G->part_bytes = G->total_units > G->total_tiles ? (size_t)G->total_units * 128 * (kD * 4 + 8) : 0;
@@ -1048,6 +1153,9 @@ extern "C" hcadsa_status hca_attn_fwd(const hcadsa_bf16* Q, const hcadsa_bf16* K
   p.split_extra = G.split_extra;
   p.split_mode = G.total_units > G.total_tiles ? 1 : 0;
   p.total_units = G.total_units;
+  p.stream_k = G.stream_k;
+  p.J_all = G.J_all;
+  p.sk_grid = G.grid;
   p.J_max = G.J_max;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.lse = lse;

@@ -226,8 +226,9 @@ def test_hca_split_key_ranges(hd):
 
 
 def test_hca_decode_uneven_splits(hd):
-    """32 sequences at t = 200000: the key tiles of the 32 row tiles are split over the SMs
-    unevenly (some row tiles get one more unit) and recombined."""
+    """32 sequences at t = 200000: 32 equal row tiles of 14 key tiles, so every CTA takes an
+    equal share of all 448 key tiles laid end to end (stream-K), and row tiles are recombined
+    from the pieces of 4-6 CTAs."""
     d, Hq, blk, W, B, t = 512, 16, 128, 128, 32, 200000
     n_c = (t + 1) // blk
     ws = t - W + 1
@@ -265,6 +266,26 @@ def test_hca_chunked_prefill(hd):
                                    with_lse=True)
     print(check_attn(O.reshape(B * Lq, Hq, d), ref, "hca chunked prefill"))
     np.testing.assert_allclose(lse.reshape(B * Lq, Hq).cpu().numpy(), ref_lse, atol=2e-2, rtol=0)
+
+
+def test_hca_decode_stream_k_short_rows(hd):
+    """70 sequences at t = 20000 (3 key tiles each, 210 in all): with stream-K most CTAs take
+    one or two key tiles, often the end of one row tile and the start of the next."""
+    d, Hq, blk, W, B, t = 512, 16, 128, 128, 70, 20000
+    n_c = (t - W + 1) // blk
+    ws = t - W + 1
+    Kc = synth.normal_bf16((B, n_c, 1, d), 1.0, 81, "K")
+    Vc = synth.normal_bf16((B, n_c, 1, d), 1.0, 81, "V")
+    Kw = synth.normal_bf16((B, W, 1, d), 1.0, 82, "K")
+    Vw = synth.normal_bf16((B, W, 1, d), 1.0, 82, "V")
+    Q = synth.normal_bf16((B, 1, Hq, d), 1.0, 83, "Q")
+    O, lse = hd.hca_attn_fwd(Q.cuda(), Kc.cuda(), Vc.cuda(), Kw.cuda(), Vw.cuda(), win_start=ws, q_offset=t,
+                             return_lse=True)
+    no_device_error(hd)
+    ref, ref_lse = oracle.hca_attn(bits(Q), bits(Kc), bits(Vc), bits(Kw), bits(Vw), win_start=ws, q_offset=t,
+                                   with_lse=True)
+    print(check_attn(O.reshape(B, Hq, d), ref, "hca decode stream-K short rows"))
+    np.testing.assert_allclose(lse.reshape(B, Hq).cpu().numpy(), ref_lse, atol=2e-2, rtol=0)
 
 
 @pytest.mark.parametrize("B", [1, 2])
