@@ -85,7 +85,7 @@ hcadsa_status hcadsa_selftest_bounded_wait(unsigned timeout_us, hcadsa_stream st
 
 /*
  * HCA block compression.  Source: mirrorspeed / besthub sections cited above
- * ("every 128 tokens are compressed into one cache entry").  Compressor form
+ * (the cache keeps one entry per 128 tokens).  Compressor form
  * (the pages leave it open): entry j of head h, channel c is
  *     acc = 0; for i in 0..blk-1: acc = fma(w[i], X[b, blk*j + i, h, c], acc)
  *     Xc[b, j, h, c] = bf16_round_nearest_even(acc)
@@ -121,9 +121,9 @@ size_t hca_attn_fwd_workspace_size(int B, int Lq, int q_offset, int Hq, int Hkv,
                                    int W);
 
 /*
- * HCA attention forward.  Source: the sections cited above ("attention is
- * computed only on the compressed entries plus a recent short uncompressed
- * window"; 512-wide heads).  Visible set of a query at position t (reading of
+ * HCA attention forward.  Source: the sections cited above (a query attends to
+ * the compressed entries and to a short window of the latest raw tokens, and to
+ * nothing else; 512-wide heads).  Visible set of a query at position t (reading of
  * the pages, which do not say how the two parts meet):
  *     raw window  s in [max(0, t-W+1), t]
  *     entries     j in [0, n_c(t)),  n_c(t) = max(0, floor((t-W+1)/blk))
@@ -159,9 +159,9 @@ size_t dsa_index_topk_workspace_size(int B, int Lq, int q_offset, int Lk, int k)
 
 /*
  * DSA indexer + per-query top-k.  Source: mirrorspeed / besthub sections cited
- * above ("a lightweight indexer ... scores historical positions for each
- * query ... core attention is computed only on the top-k positions with the
- * highest scores").  Indexer form (left open by the pages):
+ * above (a small scoring network rates every earlier position for each query,
+ * and attention then covers only the k best-rated positions).  Indexer form
+ * (left open by the pages):
  *     score[t, s] = sum_j w_idx[j] * sum_c q_idx[b, r, j, c] * k_idx[b, s, c]
  * exact in int32.  Candidates of a query at t are the positions s <= t with
  * s < Lk (its own position included).  The k candidates with the largest

@@ -82,7 +82,7 @@ void oracle_bf16_to_f32(const uint16_t* x, float* y, long n) {
 /* HCA block compression                                               */
 /* ------------------------------------------------------------------ */
 
-/* [P1]/[P3]: "every 128 tokens are compressed into one cache entry".
+/* [P1]/[P3]: the cache keeps one entry per 128 tokens.
  * Entry j of head h, channel c:
  *     acc = 0;  for i = 0 .. blk-1:  acc = fma(w[i], X[blk*j + i, h, c], acc)
  *     Xc[j, h, c] = bf16_rne(acc)
@@ -111,8 +111,8 @@ int oracle_hca_compress(const uint16_t* X, const float* w, uint16_t* Xc,
 /* HCA visible set                                                     */
 /* ------------------------------------------------------------------ */
 
-/* [P1]/[P3]/[P5]: a query attends to "the compressed entries plus a recent
- * short uncompressed window".  Reading taken (the pages do not say how the two
+/* [P1]/[P3]/[P5]: a query attends to the compressed entries and to a short
+ * window of the latest raw tokens.  Reading taken (the pages do not say how the two
  * meet):
  *   window   = raw positions s with  max(0, t-W+1) <= s <= t
  *   entries  = blocks j whose every position lies before the window start,
@@ -230,8 +230,8 @@ int oracle_hca_attn(const uint16_t* Q, const uint16_t* Kc, const uint16_t* Vc, i
 /* DSA lightning indexer                                               */
 /* ------------------------------------------------------------------ */
 
-/* [P1]/[P3]: "a lightweight indexer to score historical positions for each
- * query".  Form fixed by the problem statement:
+/* [P1]/[P3]: a small scoring network rates every earlier position for each
+ * query.  Form fixed by the problem statement:
  *   score[t, s] = sum_j w_idx[j] * sum_c q_idx[t, j, c] * k_idx[s, c]
  * exact in integers.  Writes the scores of query row (b, r) against key
  * positions 0 .. n-1 into out[0 .. n-1]. */
@@ -271,8 +271,8 @@ static int ascending_int32(const void* a, const void* b) {
   return (x > y) - (x < y);
 }
 
-/* [P1]/[P3]: "core attention is computed only on the top-k positions with the
- * highest scores".  Candidates of a query at t are the positions 0 .. t
+/* [P1]/[P3]: attention covers only the k positions with the best scores.
+ * Candidates of a query at t are the positions 0 .. t
  * (the query's own position included; reading needed so that k >= t+1 gives
  * dense causal attention), restricted to s < Lk.  All candidates are sorted by
  * (score descending, position ascending); the first min(k, count) are kept and

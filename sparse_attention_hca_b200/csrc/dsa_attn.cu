@@ -1,8 +1,8 @@
 // dsa_attn.cu -- DSA sparse attention forward on sm_100a (tcgen05 + TMEM + TMA gather).
 //
 // Method: the mirrorspeed page, section "Hybrid sparse attention, 1/7 full context
-// access": in the MLA layers "the core attention is computed only on the top-k
-// positions with the highest scores"; MLA heads are 256 wide (ai-club.cn page,
+// access": in the MLA layers each query attends only to the k positions its indexer
+// scored highest; MLA heads are 256 wide (ai-club.cn page,
 // section "混合注意力（MLA + HCA）").  All 64 query heads of a token share one K/V
 // head (the MLA latent reading) and the token's index row.
 //

@@ -1,8 +1,8 @@
 // dsa_indexer.cu -- DSA lightning indexer and per-query top-k selection.
 //
-// The pages ("Hybrid sparse attention, 1/7 full context access", mirrorspeed and
-// besthub pages) describe "a lightweight indexer to score historical positions for
-// each query" whose top-k positions receive attention.  The indexer form this library
+// The pages (section "Hybrid sparse attention, 1/7 full context access" of the mirrorspeed
+// page, and the besthub page) describe a small scoring network that rates every earlier
+// position for each query; attention then covers only the best-rated k.  The indexer form this library
 // fixes: score[t,s] = sum_j w_idx[j] * <q_idx[t,j,:], k_idx[s,:]>, exact int32, over
 // candidates s <= t; top-k by (score desc, position asc), written ascending, -1 padded.
 //

@@ -1,9 +1,9 @@
 // hca_attn.cu -- HCA attention forward on sm_100a (tcgen05 + TMEM + TMA).
 //
 // Method: the mirrorspeed page, section "Hybrid sparse attention, 1/7 full context
-// access" (and the besthub page, "Core Architectural Innovations", item 1): every 128
-// tokens are compressed into one cache entry and a query attends over the compressed
-// entries plus a recent uncompressed window; HCA heads are 512 wide (ai-club.cn page,
+// access" (and the besthub page, "Core Architectural Innovations", item 1): the cache
+// keeps one entry per 128 tokens, and a query attends to those entries together with the
+// latest raw tokens; HCA heads are 512 wide (ai-club.cn page,
 // section "混合注意力（MLA + HCA）").  Visible set of a query at t (this library's
 // reading): raw positions [max(0,t-W+1), t] and entries j < n_c(t) = max(0,(t-W+1)/blk).
 //
