@@ -520,7 +520,7 @@ def reference(args):
 
 
 def only_kernel(args):
-    """Runs one library kernel alone at sequence length --seq-len (profiling driver): W warm-up
+    """Runs one library kernel alone at sequence length --seq-len (profiling mode): W warm-up
     and K timed launches; prints a small JSON record (not the benchmark contract line).
     --only decode runs the decode step instead."""
     import sparse_attention_hca_b200 as hd
@@ -567,7 +567,7 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--only", choices=["compress", "hca_attn", "index_topk", "dsa_attn", "decode"],
-                    help="profiling driver: run one kernel alone at --seq-len, or the decode step "
+                    help="profiling mode: run one kernel alone at --seq-len, or the decode step "
                          "(B = 32 at t = 1,048,575; --steps timed steps after 3 warm-up steps)")
     ap.add_argument("--seq-len", type=int, default=L)
     args = ap.parse_args()
