@@ -1,4 +1,5 @@
-"""CPU oracle for the hybrid sparse attention forward (HCA + MLA-DSA).
+"""CPU oracle for the hybrid sparse attention forward (HCA + MLA-DSA), and for the
+gradients of its attention and compression steps (backward pass).
 
 TEST INFRASTRUCTURE ONLY: the test suite, the smoke check and the benchmark's
 CPU-baseline leg are the only callers.  The product path (the CUDA library and
@@ -10,7 +11,8 @@ Every function evaluates the definitions stated in ``oracle.c``; the pins that
 tie those definitions to the pages and to independent mathematics are in
 ``tests/test_oracle_pins.py``.  Parity status of each function: pinned (see the
 pin tests), except the large-configuration attention values, which are pinned
-only through the special cases and invariants the tests check.
+only through the special cases and invariants the tests check.  The backward
+functions are pinned to torch fp64 autograd and to closed forms.
 """
 from __future__ import annotations
 
@@ -69,6 +71,13 @@ def _load():
             lib.oracle_dsa_topk.restype = I
             lib.oracle_dsa_attn.argtypes = [P, P, P, P, I, I, I, I, I, I, D, P, I, P, P]
             lib.oracle_dsa_attn.restype = I
+            lib.oracle_hca_attn_bwd.argtypes = [P, P, P, I, P, P, I, I, P, I, I, I, I, I, I, I, I, D,
+                                                P, P, P, P, P]
+            lib.oracle_hca_attn_bwd.restype = I
+            lib.oracle_dsa_attn_bwd.argtypes = [P, P, P, P, P, I, I, I, I, I, I, D, P, P, P]
+            lib.oracle_dsa_attn_bwd.restype = I
+            lib.oracle_hca_compress_bwd.argtypes = [P, P, P, I, I, I, I, I, P, P]
+            lib.oracle_hca_compress_bwd.restype = I
             _lib = lib
     return _lib
 
@@ -203,3 +212,78 @@ def dsa_attn(Q, K, V, idx_rows, *, scale=None, rows=None, with_lse=False):
                                  float(scale), _ptr(rows), rows.size, _ptr(O), _ptr(lse))
     _check(st, "dsa_attn")
     return (O, lse) if with_lse else O
+
+
+# ---------------------------------------------------------------- backward pass
+
+
+def hca_attn_bwd(Q, Kc, Vc, Kw, Vw, dO, *, win_start=0, q_offset=0, blk=128, W=128, scale=None):
+    """Gradients of sum(O * dO) for hca_attn over every query row.
+
+    Q [B,Lq,Hq,d], Kc/Vc [B,n_c,Hkv,d], Kw/Vw [B,n_w,Hkv,d] bf16 bits; dO [B,Lq,Hq,d] fp64.
+    Returns fp64 (dQ, dKc, dVc, dKw, dVw) shaped like their inputs (dKc/dVc None when n_c = 0)."""
+    Q = _c(Q, np.uint16)
+    Kw = _c(Kw, np.uint16)
+    Vw = _c(Vw, np.uint16)
+    dO = _c(dO, np.float64)
+    B, Lq, Hq, d = Q.shape
+    n_w, Hkv = Kw.shape[1], Kw.shape[2]
+    assert dO.shape == Q.shape
+    if Kc is None or Kc.shape[1] == 0:
+        n_c, Kc_, Vc_, dKc, dVc = 0, None, None, None, None
+    else:
+        Kc_, Vc_ = _c(Kc, np.uint16), _c(Vc, np.uint16)
+        n_c = Kc_.shape[1]
+        dKc = np.empty(Kc_.shape, np.float64)
+        dVc = np.empty(Kc_.shape, np.float64)
+    if scale is None:
+        scale = float(np.float32(1.0 / np.sqrt(d)))
+    dQ = np.empty(Q.shape, np.float64)
+    dKw = np.empty(Kw.shape, np.float64)
+    dVw = np.empty(Kw.shape, np.float64)
+    st = _load().oracle_hca_attn_bwd(_ptr(Q), _ptr(Kc_), _ptr(Vc_), n_c, _ptr(Kw), _ptr(Vw), win_start,
+                                     n_w, _ptr(dO), B, Lq, q_offset, Hq, Hkv, d, blk, W, float(scale),
+                                     _ptr(dQ), _ptr(dKc), _ptr(dVc), _ptr(dKw), _ptr(dVw))
+    _check(st, "hca_attn_bwd")
+    return dQ, dKc, dVc, dKw, dVw
+
+
+def dsa_attn_bwd(Q, K, V, idx, dO, *, scale=None):
+    """Gradients of sum(O * dO) for dsa_attn over every query row.
+
+    Q [B,Lq,Hq,d], K/V [B,Lk,d] bf16 bits; idx [B,Lq,k] int32 (-1 padding); dO [B,Lq,Hq,d]
+    fp64.  Returns fp64 (dQ, dK, dV)."""
+    Q = _c(Q, np.uint16)
+    K = _c(K, np.uint16)
+    V = _c(V, np.uint16)
+    dO = _c(dO, np.float64)
+    idx = _c(idx, np.int32)
+    B, Lq, Hq, d = Q.shape
+    Lk = K.shape[1]
+    k = idx.shape[-1]
+    assert idx.size == B * Lq * k and dO.shape == Q.shape
+    if scale is None:
+        scale = float(np.float32(1.0 / np.sqrt(d)))
+    dQ = np.empty(Q.shape, np.float64)
+    dK = np.empty((B, Lk, d), np.float64)
+    dV = np.empty((B, Lk, d), np.float64)
+    st = _load().oracle_dsa_attn_bwd(_ptr(Q), _ptr(K), _ptr(V), _ptr(idx), _ptr(dO), B, Lq, Lk, Hq, d, k,
+                                     float(scale), _ptr(dQ), _ptr(dK), _ptr(dV))
+    _check(st, "dsa_attn_bwd")
+    return dQ, dK, dV
+
+
+def hca_compress_bwd(X, w, dXc, blk):
+    """Adjoint of the compressor as the exact linear map Xc[j] = sum_i w[i] X[blk*j + i].
+
+    X [B,L,H,d] bf16 bits, w [blk] fp32, dXc [B,L//blk,H,d] fp64 -> (dX [B,L,H,d], dw [blk]) fp64."""
+    X = _c(X, np.uint16)
+    w = _c(w, np.float32)
+    dXc = _c(dXc, np.float64)
+    B, L, H, d = X.shape
+    assert w.shape == (blk,) and dXc.shape == (B, L // blk, H, d)
+    dX = np.empty(X.shape, np.float64)
+    dw = np.empty(blk, np.float64)
+    st = _load().oracle_hca_compress_bwd(_ptr(X), _ptr(w), _ptr(dXc), B, L, H, d, blk, _ptr(dX), _ptr(dw))
+    _check(st, "hca_compress_bwd")
+    return dX, dw

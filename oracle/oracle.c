@@ -1,6 +1,7 @@
 /*
  * oracle.c -- plain, slow, obviously-correct CPU statement of the hybrid
- * sparse attention forward (HCA + MLA-DSA).
+ * sparse attention forward (HCA + MLA-DSA), and of the gradients of its
+ * attention and compression steps (the backward pass, at the end).
  *
  * TEST INFRASTRUCTURE ONLY.  Nothing in the product path links, loads or
  * calls this file; only the test suite, the smoke check and the benchmark's
@@ -365,4 +366,208 @@ int oracle_dsa_attn(const uint16_t* Q, const uint16_t* K, const uint16_t* V, con
     free(s_buf);
   }
   return status;
+}
+
+/* ================================================================== */
+/* Backward pass (gradients of a scalar loss through O)                */
+/* ================================================================== */
+
+/* Gradient of one query row of attend_row.  With s_i = scale <q, k_i>,
+ * p = softmax(s) and O = sum_i p_i v_i, a loss with dL/dO = dO gives
+ *   dL/dv_i = p_i dO
+ *   dL/ds_i = p_i (<dO, v_i> - <dO, O>)
+ *   dL/dq   = scale sum_i dL/ds_i k_i,   dL/dk_i = scale dL/ds_i q.
+ * Keys and values are given by element offsets into K/V (bf16) so that the
+ * key and value gradients land at the same offsets of dK/dV (fp64, added to).
+ * dq (d doubles) is added to as well.  p_buf holds n doubles. */
+static void attend_row_bwd(const uint16_t* q, const uint16_t* K, const uint16_t* V, const long* offs, int n,
+                           int d, double scale, const double* dO, double* p_buf, double* dq, double* dK,
+                           double* dV) {
+  if (n == 0) return;
+  double m = -INFINITY;
+  for (int i = 0; i < n; ++i) {
+    double dot = 0.0;
+    for (int c = 0; c < d; ++c) dot += (double)bf16_bits_to_float(q[c]) * (double)bf16_bits_to_float(K[offs[i] + c]);
+    p_buf[i] = scale * dot;
+    if (p_buf[i] > m) m = p_buf[i];
+  }
+  double l = 0.0;
+  for (int i = 0; i < n; ++i) {
+    p_buf[i] = exp(p_buf[i] - m);
+    l += p_buf[i];
+  }
+  for (int i = 0; i < n; ++i) p_buf[i] /= l;
+  /* <dO, O> = sum_i p_i <dO, v_i> */
+  double dO_O = 0.0;
+  for (int i = 0; i < n; ++i) {
+    double dp = 0.0;
+    for (int c = 0; c < d; ++c) dp += dO[c] * (double)bf16_bits_to_float(V[offs[i] + c]);
+    dO_O += p_buf[i] * dp;
+  }
+  for (int i = 0; i < n; ++i) {
+    double dp = 0.0;
+    for (int c = 0; c < d; ++c) dp += dO[c] * (double)bf16_bits_to_float(V[offs[i] + c]);
+    const double ds = p_buf[i] * (dp - dO_O);
+    for (int c = 0; c < d; ++c) {
+      dV[offs[i] + c] += p_buf[i] * dO[c];
+      dq[c] += scale * ds * (double)bf16_bits_to_float(K[offs[i] + c]);
+      dK[offs[i] + c] += scale * ds * (double)bf16_bits_to_float(q[c]);
+    }
+  }
+}
+
+/* Backward of oracle_hca_attn over every query row: dO is [B, Lq, Hq, d]
+ * fp64; dQ [B, Lq, Hq, d], dKc/dVc [B, n_c, Hkv, d], dKw/dVw [B, n_w, Hkv, d]
+ * are fp64 and overwritten.  The visible set, head mapping and scale are those
+ * of the forward.  Serial (keys are shared between rows and heads). */
+int oracle_hca_attn_bwd(const uint16_t* Q, const uint16_t* Kc, const uint16_t* Vc, int n_c,
+                        const uint16_t* Kw, const uint16_t* Vw, int win_start, int n_w, const double* dO,
+                        int B, int Lq, int q_offset, int Hq, int Hkv, int d, int blk, int W, double scale,
+                        double* dQ, double* dKc, double* dVc, double* dKw, double* dVw) {
+  if (!Q || !Kw || !Vw || !dO || !dQ || !dKw || !dVw || Hq <= 0 || Hkv <= 0 || Hq % Hkv || d <= 0 ||
+      blk <= 0 || W <= 0 || B < 0 || Lq < 0 || n_c < 0 || n_w < 0)
+    return ORACLE_ERR_ARG;
+  if (n_c > 0 && (!Kc || !Vc || !dKc || !dVc)) return ORACLE_ERR_ARG;
+  const int group = Hq / Hkv;
+  memset(dQ, 0, sizeof(double) * (size_t)B * Lq * Hq * d);
+  if (n_c > 0) {
+    memset(dKc, 0, sizeof(double) * (size_t)B * n_c * Hkv * d);
+    memset(dVc, 0, sizeof(double) * (size_t)B * n_c * Hkv * d);
+  }
+  memset(dKw, 0, sizeof(double) * (size_t)B * n_w * Hkv * d);
+  memset(dVw, 0, sizeof(double) * (size_t)B * n_w * Hkv * d);
+  long* offs_c = (long*)malloc(sizeof(long) * (size_t)(n_c + 1));
+  long* offs_w = (long*)malloc(sizeof(long) * (size_t)(n_w + 1));
+  double* p_buf = (double*)malloc(sizeof(double) * (size_t)(n_c + n_w + 1));
+  double* dq_tmp = (double*)malloc(sizeof(double) * (size_t)d);
+  int status = ORACLE_OK;
+  for (int b = 0; b < B && status == ORACLE_OK; ++b)
+    for (int r = 0; r < Lq && status == ORACLE_OK; ++r) {
+      const int t = q_offset + r;
+      const int ws = oracle_hca_window_start(t, W);
+      const int nc_t = oracle_hca_n_compressed(t, W, blk);
+      if (nc_t > n_c || ws < win_start || t - win_start >= n_w) {
+        status = ORACLE_ERR_RANGE;
+        break;
+      }
+      for (int h = 0; h < Hq; ++h) {
+        const int hk = h / group;
+        int n_cv = 0, n_wv = 0;
+        for (int j = 0; j < nc_t; ++j) offs_c[n_cv++] = (((long)b * n_c + j) * Hkv + hk) * (long)d;
+        for (int s = ws; s <= t; ++s) offs_w[n_wv++] = (((long)b * n_w + (s - win_start)) * Hkv + hk) * (long)d;
+        const long qo = (((long)b * Lq + r) * Hq + h) * (long)d;
+        /* the row's keys: its entries, then its window (one softmax over both, as in the
+         * forward); the same steps as attend_row_bwd, with two key tensors */
+        const int n = n_cv + n_wv;
+        if (n == 0) continue;
+        double m = -INFINITY;
+        for (int i = 0; i < n; ++i) {
+          const uint16_t* kr = i < n_cv ? Kc + offs_c[i] : Kw + offs_w[i - n_cv];
+          double dot = 0.0;
+          for (int c = 0; c < d; ++c) dot += (double)bf16_bits_to_float(Q[qo + c]) * (double)bf16_bits_to_float(kr[c]);
+          p_buf[i] = scale * dot;
+          if (p_buf[i] > m) m = p_buf[i];
+        }
+        double l = 0.0;
+        for (int i = 0; i < n; ++i) {
+          p_buf[i] = exp(p_buf[i] - m);
+          l += p_buf[i];
+        }
+        for (int i = 0; i < n; ++i) p_buf[i] /= l;
+        const double* g = dO + qo;
+        double dO_O = 0.0;
+        for (int i = 0; i < n; ++i) {
+          const uint16_t* vr = i < n_cv ? Vc + offs_c[i] : Vw + offs_w[i - n_cv];
+          double dp = 0.0;
+          for (int c = 0; c < d; ++c) dp += g[c] * (double)bf16_bits_to_float(vr[c]);
+          dO_O += p_buf[i] * dp;
+        }
+        for (int c = 0; c < d; ++c) dq_tmp[c] = 0.0;
+        for (int i = 0; i < n; ++i) {
+          const int entry = i < n_cv;
+          const long o = entry ? offs_c[i] : offs_w[i - n_cv];
+          const uint16_t* kr = (entry ? Kc : Kw) + o;
+          const uint16_t* vr = (entry ? Vc : Vw) + o;
+          double* dk = (entry ? dKc : dKw) + o;
+          double* dv = (entry ? dVc : dVw) + o;
+          double dp = 0.0;
+          for (int c = 0; c < d; ++c) dp += g[c] * (double)bf16_bits_to_float(vr[c]);
+          const double ds = p_buf[i] * (dp - dO_O);
+          for (int c = 0; c < d; ++c) {
+            dv[c] += p_buf[i] * g[c];
+            dq_tmp[c] += scale * ds * (double)bf16_bits_to_float(kr[c]);
+            dk[c] += scale * ds * (double)bf16_bits_to_float(Q[qo + c]);
+          }
+        }
+        for (int c = 0; c < d; ++c) dQ[qo + c] = dq_tmp[c];
+      }
+    }
+  free(offs_c);
+  free(offs_w);
+  free(p_buf);
+  free(dq_tmp);
+  return status;
+}
+
+/* Backward of oracle_dsa_attn over every query row: idx_rows is [B*Lq, k]
+ * (row b*Lq + r; entries < 0 are padding), dO [B, Lq, Hq, d] fp64; dQ
+ * [B, Lq, Hq, d], dK/dV [B, Lk, d] fp64, overwritten.  Serial. */
+int oracle_dsa_attn_bwd(const uint16_t* Q, const uint16_t* K, const uint16_t* V, const int32_t* idx_rows,
+                        const double* dO, int B, int Lq, int Lk, int Hq, int d, int k, double scale, double* dQ,
+                        double* dK, double* dV) {
+  if (!Q || !K || !V || !idx_rows || !dO || !dQ || !dK || !dV || B < 0 || Lq < 0 || Lk < 0 || Hq <= 0 ||
+      d <= 0 || k <= 0)
+    return ORACLE_ERR_ARG;
+  memset(dQ, 0, sizeof(double) * (size_t)B * Lq * Hq * d);
+  memset(dK, 0, sizeof(double) * (size_t)B * Lk * d);
+  memset(dV, 0, sizeof(double) * (size_t)B * Lk * d);
+  long* offs = (long*)malloc(sizeof(long) * (size_t)k);
+  double* p_buf = (double*)malloc(sizeof(double) * (size_t)k);
+  int status = ORACLE_OK;
+  for (int b = 0; b < B && status == ORACLE_OK; ++b)
+    for (int r = 0; r < Lq; ++r) {
+      int n = 0;
+      for (int m = 0; m < k; ++m) {
+        const int32_t s = idx_rows[((long)b * Lq + r) * k + m];
+        if (s < 0) continue;
+        if (s >= Lk) {
+          status = ORACLE_ERR_RANGE;
+          break;
+        }
+        offs[n++] = ((long)b * Lk + s) * (long)d;
+      }
+      if (status != ORACLE_OK) break;
+      for (int h = 0; h < Hq; ++h) {
+        const long qo = (((long)b * Lq + r) * Hq + h) * (long)d;
+        attend_row_bwd(Q + qo, K, V, offs, n, d, scale, dO + qo, p_buf, dQ + qo, dK, dV);
+      }
+    }
+  free(offs);
+  free(p_buf);
+  return status;
+}
+
+/* Backward of the compressor, taken as the exact linear map
+ *   Xc[b, j, h, c] = sum_i w[i] X[b, blk*j + i, h, c]
+ * (the forward's fp32 chain and bf16 rounding are not differentiated):
+ *   dX[b, blk*j + i, h, c] = w[i] dXc[b, j, h, c]   (0 for the partial tail block)
+ *   dw[i] = sum_{b, j, h, c} X[b, blk*j + i, h, c] dXc[b, j, h, c]
+ * dXc is [B, L/blk, H, d] fp64; dX [B, L, H, d] and dw [blk] fp64, overwritten. */
+int oracle_hca_compress_bwd(const uint16_t* X, const float* w, const double* dXc, int B, int L, int H, int d,
+                            int blk, double* dX, double* dw) {
+  if (!X || !w || !dXc || !dX || !dw || B < 0 || L < 0 || H <= 0 || d <= 0 || blk <= 0) return ORACLE_ERR_ARG;
+  const int n_c = L / blk;
+  memset(dX, 0, sizeof(double) * (size_t)B * L * H * d);
+  for (int i = 0; i < blk; ++i) dw[i] = 0.0;
+  for (int b = 0; b < B; ++b)
+    for (int j = 0; j < n_c; ++j)
+      for (int i = 0; i < blk; ++i)
+        for (int h = 0; h < H; ++h)
+          for (int c = 0; c < d; ++c) {
+            const long src = (((long)b * L + (long)blk * j + i) * H + h) * (long)d + c;
+            const double g = dXc[(((long)b * n_c + j) * H + h) * (long)d + c];
+            dX[src] = (double)w[i] * g;
+            dw[i] += (double)bf16_bits_to_float(X[src]) * g;
+          }
+  return ORACLE_OK;
 }

@@ -380,3 +380,140 @@ def test_dsa_attention_ignores_index_order_and_padding(oracle_mod):
     a = oracle_mod.dsa_attn(bits(inp["Q"]), bits(inp["K"]), bits(inp["V"]), idx)
     b = oracle_mod.dsa_attn(bits(inp["Q"]), bits(inp["K"]), bits(inp["V"]), shuffled)
     np.testing.assert_allclose(a, b, rtol=0, atol=1e-14)
+
+
+# ---------------------------------------------------------------- backward pass
+# The gradients are pinned to torch's fp64 autograd through an explicitly masked softmax
+# attention (the visible set enumerated from its definition, as above), to closed forms,
+# and, for the compressor, to autograd of the exact weighted block sum.
+
+def _masked_attention_grads(Q, Kall, Vall, mask, scale, dO):
+    """fp64 autograd of sum(O * dO) with O = softmax(scale q.k, masked) v; K/V [B,Lk,Hkv,d]
+    shared by the Hq/Hkv query heads of a group.  Returns dQ, dK, dV (numpy fp64)."""
+    q = Q.double().clone().requires_grad_(True)
+    k = Kall.double().clone().requires_grad_(True)
+    v = Vall.double().clone().requires_grad_(True)
+    g = q.shape[2] // k.shape[2]
+    kk = k.repeat_interleave(g, dim=2)
+    vv = v.repeat_interleave(g, dim=2)
+    s = scale * torch.einsum("bthc,bshc->bhts", q, kk)
+    s = s.masked_fill(~mask.view(1, 1, *mask.shape), float("-inf"))
+    p = torch.softmax(s, dim=-1)
+    o = torch.einsum("bhts,bshc->bthc", p, vv)
+    (o * torch.as_tensor(dO)).sum().backward()
+    return q.grad.numpy(), k.grad.numpy(), v.grad.numpy()
+
+
+def test_hca_attn_bwd_matches_autograd_over_entries_and_window(oracle_mod):
+    B, L, Hq, Hkv, d, blk, W, scale = 2, 45, 4, 2, 8, 4, 6, 0.4
+    inp = _hca_case(B, L, Hq, Hkv, d, 91, sigma=1.0)
+    Q, K, V = inp["Q"], inp["K"], inp["V"]
+    w = synth.uniform_f32((blk,), 0.0, 2.0 / blk, 91, "w").numpy()
+    Kc, Vc = oracle_mod.hca_compress(bits(K), w, blk), oracle_mod.hca_compress(bits(V), w, blk)
+    n_c = L // blk
+    dO = np.random.default_rng(92).standard_normal((B, L, Hq, d))
+    dQ, dKc, dVc, dKw, dVw = oracle_mod.hca_attn_bwd(bits(Q), Kc, Vc, bits(K), bits(V), dO, blk=blk, W=W,
+                                                     scale=scale)
+    Kall = torch.cat([from_bits(Kc), K], dim=1)
+    Vall = torch.cat([from_bits(Vc), V], dim=1)
+    mask = torch.zeros(L, n_c + L, dtype=torch.bool)
+    for t in range(L):
+        ws = max(0, t - W + 1)
+        for j in range(n_c):
+            mask[t, j] = (blk * j + blk - 1) < ws
+        for s in range(ws, t + 1):
+            mask[t, n_c + s] = True
+    rQ, rK, rV = _masked_attention_grads(Q, Kall, Vall, mask, scale, dO)
+    np.testing.assert_allclose(dQ, rQ, rtol=0, atol=1e-11)
+    np.testing.assert_allclose(dKc, rK[:, :n_c], rtol=0, atol=1e-11)
+    np.testing.assert_allclose(dVc, rV[:, :n_c], rtol=0, atol=1e-11)
+    np.testing.assert_allclose(dKw, rK[:, n_c:], rtol=0, atol=1e-11)
+    np.testing.assert_allclose(dVw, rV[:, n_c:], rtol=0, atol=1e-11)
+
+
+def test_hca_attn_bwd_decode_offset_matches_autograd(oracle_mod):
+    """One query per sequence at t = 300 over an entry cache and a window buffer that starts at
+    the window (q_offset and win_start both in play)."""
+    B, Hq, Hkv, d, blk, W, t = 2, 4, 1, 8, 16, 20, 300
+    n_c = (t - W + 1) // blk
+    ws = t - W + 1
+    g = torch.Generator().manual_seed(93)
+    Q = torch.randn(B, 1, Hq, d, generator=g).to(torch.bfloat16)
+    Kc = torch.randn(B, n_c, Hkv, d, generator=g).to(torch.bfloat16)
+    Vc = torch.randn(B, n_c, Hkv, d, generator=g).to(torch.bfloat16)
+    Kw = torch.randn(B, W, Hkv, d, generator=g).to(torch.bfloat16)
+    Vw = torch.randn(B, W, Hkv, d, generator=g).to(torch.bfloat16)
+    dO = np.random.default_rng(94).standard_normal((B, 1, Hq, d))
+    dQ, dKc, dVc, dKw, dVw = oracle_mod.hca_attn_bwd(bits(Q), bits(Kc), bits(Vc), bits(Kw), bits(Vw), dO,
+                                                     win_start=ws, q_offset=t, blk=blk, W=W, scale=0.3)
+    mask = torch.ones(1, n_c + W, dtype=torch.bool)  # every stored entry and window row is visible
+    rQ, rK, rV = _masked_attention_grads(Q, torch.cat([Kc, Kw], 1), torch.cat([Vc, Vw], 1), mask, 0.3, dO)
+    np.testing.assert_allclose(dQ, rQ, rtol=0, atol=1e-11)
+    np.testing.assert_allclose(np.concatenate([dKc, dKw], 1), rK, rtol=0, atol=1e-11)
+    np.testing.assert_allclose(np.concatenate([dVc, dVw], 1), rV, rtol=0, atol=1e-11)
+
+
+def test_hca_attn_bwd_closed_forms(oracle_mod):
+    """Token 0 sees only itself (p = 1): its dQ is 0 and its own V row receives dO.  With every
+    V row equal, O no longer depends on the scores, so dQ and all key gradients vanish."""
+    B, L, Hq, Hkv, d, blk, W = 1, 12, 2, 1, 4, 4, 5
+    inp = _hca_case(B, L, Hq, Hkv, d, 95, sigma=1.0)
+    Q, K, V = inp["Q"], inp["K"], inp["V"]
+    w = np.full(blk, 1.0 / blk, np.float32)
+    Kc, Vc = oracle_mod.hca_compress(bits(K), w, blk), oracle_mod.hca_compress(bits(V), w, blk)
+    dO = np.zeros((B, L, Hq, d))
+    dO[0, 0] = np.random.default_rng(96).standard_normal((Hq, d))
+    dQ, dKc, dVc, dKw, dVw = oracle_mod.hca_attn_bwd(bits(Q), Kc, Vc, bits(K), bits(V), dO, blk=blk, W=W)
+    assert np.all(dQ == 0.0) and np.all(dKc == 0.0) and np.all(dVc == 0.0)
+    np.testing.assert_allclose(dVw[0, 0, 0], dO[0, 0].sum(0), rtol=0, atol=1e-15)  # both heads share kv 0
+    assert np.all(dVw[0, 1:] == 0.0) and np.all(dKw == 0.0)
+    Vconst = torch.ones_like(V) * 0.75
+    Vc1 = oracle_mod.hca_compress(bits(Vconst), w, blk)  # entries of a constant row stay 0.75
+    dO = np.random.default_rng(97).standard_normal((B, L, Hq, d))
+    dQ, dKc, dVc, dKw, dVw = oracle_mod.hca_attn_bwd(bits(Q), Kc, Vc1, bits(K), bits(Vconst), dO, blk=blk, W=W)
+    assert np.abs(dQ).max() < 1e-14 and np.abs(dKc).max() < 1e-14 and np.abs(dKw).max() < 1e-14
+    # the value gradients still sum to the total dO of each kv head (softmax rows sum to 1)
+    np.testing.assert_allclose(dVc.sum((1,)) + dVw.sum((1,)), dO.sum(1).reshape(B, Hkv, Hq // Hkv, d).sum(2),
+                               rtol=0, atol=1e-12)
+
+
+def test_dsa_attn_bwd_matches_autograd_over_selection(oracle_mod):
+    B, L, Hq, d, k, scale = 2, 40, 4, 16, 7, 0.25
+    inp = _dsa_small(B, L, Hq, d, 98)
+    idx = oracle_mod.dsa_topk(inp["q_idx"].numpy(), inp["k_idx"].numpy(), inp["w_idx"].numpy(), k)
+    rng = np.random.default_rng(99)
+    idx = np.stack([rng.permutation(row) for row in idx]).reshape(B, L, k)  # order must not matter
+    dO = rng.standard_normal((B, L, Hq, d))
+    dQ, dK, dV = oracle_mod.dsa_attn_bwd(bits(inp["Q"]), bits(inp["K"]), bits(inp["V"]), idx, dO, scale=scale)
+    for b in range(B):
+        mask = torch.zeros(L, L, dtype=torch.bool)
+        for t in range(L):
+            for s in idx[b, t]:
+                if s >= 0:
+                    mask[t, s] = True
+        rQ, rK, rV = _masked_attention_grads(inp["Q"][b:b + 1], inp["K"][b:b + 1].unsqueeze(2),
+                                             inp["V"][b:b + 1].unsqueeze(2), mask, scale, dO[b:b + 1])
+        np.testing.assert_allclose(dQ[b:b + 1], rQ, rtol=0, atol=1e-11)
+        np.testing.assert_allclose(dK[b], rK[0, :, 0], rtol=0, atol=1e-11)
+        np.testing.assert_allclose(dV[b], rV[0, :, 0], rtol=0, atol=1e-11)
+
+
+def test_compress_bwd_matches_autograd_and_one_hot(oracle_mod):
+    B, L, H, d, blk = 2, 23, 3, 5, 4  # 5 complete blocks and a partial tail of 3 tokens
+    X = synth.normal_bf16((B, L, H, d), 1.0, 100, "K")
+    w = synth.uniform_f32((blk,), 0.0, 2.0 / blk, 100, "w").numpy()
+    n_c = L // blk
+    dXc = np.random.default_rng(101).standard_normal((B, n_c, H, d))
+    dX, dw = oracle_mod.hca_compress_bwd(bits(X), w, dXc, blk)
+    x = X.double().clone().requires_grad_(True)
+    wt = torch.as_tensor(w, dtype=torch.float64).clone().requires_grad_(True)
+    xc = torch.einsum("i,bjihc->bjhc", wt, x[:, : n_c * blk].reshape(B, n_c, blk, H, d))
+    (xc * torch.as_tensor(dXc)).sum().backward()
+    np.testing.assert_allclose(dX, x.grad.numpy(), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(dw, wt.grad.numpy(), rtol=1e-13, atol=1e-12)
+    assert np.all(dX[:, n_c * blk:] == 0.0)  # the partial tail block feeds no entry
+    onehot = np.zeros(blk, np.float32)
+    onehot[2] = 1.0
+    dX1, _ = oracle_mod.hca_compress_bwd(bits(X), onehot, dXc, blk)
+    np.testing.assert_array_equal(dX1[:, 2: n_c * blk: blk], dXc)  # row 2 of each block takes dXc
+    assert np.count_nonzero(dX1) == np.count_nonzero(dXc)
