@@ -116,6 +116,10 @@ def test_hca_tiny_all_rows(hd):
     # overhang shares that tile (merged tiles) or not, for 8- and 16-token row tiles
     (synth.HcaConfig("merge_blk16_L2400_hq16", B=1, L=2400, Hq=16, Hkv=1, blk=16, sigma=1.0), 128),
     (synth.HcaConfig("merge_g8_blk16_L2400_hq16_hkv2", B=1, L=2400, Hq=16, Hkv=2, blk=16, sigma=1.0), 128),
+    # 32 and 128 query heads per K/V head: row tiles of 4 tokens (band overhang 3, merged
+    # tiles) and of a single token
+    (synth.HcaConfig("g32_L700_hq32", B=1, L=700, Hq=32, Hkv=1, sigma=1.0), 128),
+    (synth.HcaConfig("g128_L300_hq128", B=1, L=300, Hq=128, Hkv=1, sigma=1.0), 128),
 ])
 def test_hca_stress(hd, cfg, W):
     O, lse, ref, ref_lse = _hca_gpu_and_oracle(hd, cfg, W=W)
