@@ -95,13 +95,35 @@ def _check(status: int, what: str):
         raise HcaDsaError(status, what)
 
 
-def _need(t, dtype, name):
-    if not t.is_cuda:
-        raise ValueError(f"{name} must be a CUDA tensor")
+def _need(t, dtype, name, shape=None):
+    """dtype, contiguity and (optionally) exact shape; the device is checked by _on_device."""
     if t.dtype != dtype:
         raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
+def _need_numel(t, n, name, what):
+    if t.numel() != n:
+        raise ValueError(f"{name} has {t.numel()} elements, expected {n} ({what})")
+
+
+def _on_device(*tensors):
+    """Every tensor must be a CUDA tensor on the current device: the library launches on the
+    current device's stream and reads the pointers there."""
+    cur = None
+    for t in tensors:
+        if t is None:
+            continue
+        if not t.is_cuda:
+            raise ValueError("every tensor must be a CUDA tensor")
+        if cur is None:
+            cur = torch.cuda.current_device()
+        if t.device.index != cur:
+            raise ValueError(f"tensor on {t.device}, but the current device is cuda:{cur}; "
+                             f"call under torch.cuda.device({t.device})")
 
 
 def _bf16(t):
@@ -115,13 +137,16 @@ def hcadsa_check_device_error(stream=None):
 
 def hca_compress_kv(K, V, w, blk: int = 128, *, Kc=None, Vc=None, stream=None):
     """K, V: [B, L, Hkv, d] bf16; w: [blk] fp32 -> Kc, Vc: [B, L // blk, Hkv, d] bf16."""
-    for t, n in ((K, "K"), (V, "V")):
-        _need(t, torch.bfloat16, n)
-    _need(w, torch.float32, "w")
+    _need(K, torch.bfloat16, "K")
     B, L, Hkv, d = K.shape
-    if V.shape != K.shape or w.numel() != blk:
-        raise ValueError("shape mismatch")
+    _need(V, torch.bfloat16, "V", K.shape)
+    _need(w, torch.float32, "w", (blk,))
     shape = (B, L // blk, Hkv, d)
+    if Kc is not None:
+        _need(Kc, torch.bfloat16, "Kc", shape)
+    if Vc is not None:
+        _need(Vc, torch.bfloat16, "Vc", shape)
+    _on_device(K, V, w, Kc, Vc)
     Kc = torch.empty(shape, dtype=torch.bfloat16, device=K.device) if Kc is None else Kc
     Vc = torch.empty(shape, dtype=torch.bfloat16, device=K.device) if Vc is None else Vc
     st = lib().hca_compress_kv(_ptr(K), _ptr(V), _ptr(w), _ptr(Kc), _ptr(Vc), B, L, Hkv, d, blk,
@@ -135,14 +160,23 @@ def hca_attn_fwd(Q, Kc, Vc, Kw, Vw, *, win_start: int = 0, q_offset: int = 0, bl
                  workspace=None, stream=None):
     """Q: [B, Lq, Hq, d]; Kc/Vc: [B, n_c, Hkv, d] (or None); Kw/Vw: [B, n_w, Hkv, d]."""
     _need(Q, torch.bfloat16, "Q")
-    _need(Kw, torch.bfloat16, "Kw")
-    _need(Vw, torch.bfloat16, "Vw")
     B, Lq, Hq, d = Q.shape
+    _need(Kw, torch.bfloat16, "Kw")
+    if Kw.dim() != 4 or Kw.shape[0] != B or Kw.shape[3] != d:
+        raise ValueError(f"Kw has shape {tuple(Kw.shape)}, expected [{B}, n_w, Hkv, {d}]")
     n_w, Hkv = Kw.shape[1], Kw.shape[2]
+    _need(Vw, torch.bfloat16, "Vw", Kw.shape)
     n_c = 0 if Kc is None else Kc.shape[1]
     if n_c:
-        _need(Kc, torch.bfloat16, "Kc")
-        _need(Vc, torch.bfloat16, "Vc")
+        _need(Kc, torch.bfloat16, "Kc", (B, n_c, Hkv, d))
+        _need(Vc, torch.bfloat16, "Vc", (B, n_c, Hkv, d))
+    if O is not None:
+        _need(O, torch.bfloat16, "O", Q.shape)
+    if lse is not None:
+        _need(lse, torch.float32, "lse", (B, Lq, Hq))
+    if workspace is not None and not workspace.is_contiguous():
+        raise ValueError("workspace must be contiguous")
+    _on_device(Q, Kw, Vw, Kc if n_c else None, Vc if n_c else None, O, lse, workspace)
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     O = torch.empty_like(Q) if O is None else O
@@ -166,14 +200,27 @@ def dsa_index_topk_workspace_size(B, Lq, q_offset, Lk, k) -> int:
     return lib().dsa_index_topk_workspace_size(B, Lq, q_offset, Lk, k)
 
 
+def _check_index_args(q_idx, k_idx, w_idx, k, idx):
+    _need(q_idx, torch.int8, "q_idx")
+    B, Lq, H_idx, d_idx = q_idx.shape
+    _need(k_idx, torch.int8, "k_idx")
+    if k_idx.shape[0] != B or k_idx.shape[-1] != d_idx:
+        raise ValueError(f"k_idx has shape {tuple(k_idx.shape)}, expected [{B}, Lk, {d_idx}]")
+    Lk = k_idx.shape[1]
+    _need_numel(k_idx, B * Lk * d_idx, "k_idx", f"[{B}, {Lk}, {d_idx}]")
+    _need(w_idx, torch.int32, "w_idx", (H_idx,))
+    if idx is not None:
+        _need(idx, torch.int32, "idx", (B, Lq, k))
+    return B, Lq, H_idx, d_idx, Lk
+
+
 def dsa_index_topk(q_idx, k_idx, w_idx, k: int, *, q_offset: int = 0, idx=None, workspace=None,
                    stream=None):
     """q_idx: [B, Lq, 4, 64] int8; k_idx: [B, Lk, 64] int8; w_idx: [4] int32 -> idx [B, Lq, k] int32."""
-    _need(q_idx, torch.int8, "q_idx")
-    _need(k_idx, torch.int8, "k_idx")
-    _need(w_idx, torch.int32, "w_idx")
-    B, Lq, H_idx, d_idx = q_idx.shape
-    Lk = k_idx.shape[1]
+    B, Lq, H_idx, d_idx, Lk = _check_index_args(q_idx, k_idx, w_idx, k, idx)
+    if workspace is not None and not workspace.is_contiguous():
+        raise ValueError("workspace must be contiguous")
+    _on_device(q_idx, k_idx, w_idx, idx, workspace)
     idx = torch.empty((B, Lq, k), dtype=torch.int32, device=q_idx.device) if idx is None else idx
     ws_bytes = dsa_index_topk_workspace_size(B, Lq, q_offset, Lk, k)
     if workspace is None:
@@ -189,11 +236,8 @@ def dsa_index_topk_noalloc(q_idx, k_idx, w_idx, k: int, *, q_offset: int = 0, id
     """dsa_index_topk for callers that cannot allocate device memory: the score rows go to a
     fixed 64 MiB array inside the library (see include/hcadsa.h for its limits and sharing).
     The output tensor is still the caller's; pass ``idx`` to avoid allocating it here."""
-    _need(q_idx, torch.int8, "q_idx")
-    _need(k_idx, torch.int8, "k_idx")
-    _need(w_idx, torch.int32, "w_idx")
-    B, Lq, H_idx, d_idx = q_idx.shape
-    Lk = k_idx.shape[1]
+    B, Lq, H_idx, d_idx, Lk = _check_index_args(q_idx, k_idx, w_idx, k, idx)
+    _on_device(q_idx, k_idx, w_idx, idx)
     idx = torch.empty((B, Lq, k), dtype=torch.int32, device=q_idx.device) if idx is None else idx
     st = lib().dsa_index_topk_noalloc(_ptr(q_idx), _ptr(k_idx), _ptr(w_idx), _ptr(idx), B, Lq, q_offset, Lk,
                                       H_idx, d_idx, k, _stream(stream))
@@ -205,12 +249,22 @@ def dsa_sparse_attn_fwd(Q, K, V, idx, *, scale: float | None = None, O=None, lse
                         return_lse=False, stream=None):
     """Q: [B, Lq, 64, 256]; K, V: [B, Lk, 256]; idx: [B, Lq, k] int32 -> O [B, Lq, 64, 256]."""
     _need(Q, torch.bfloat16, "Q")
-    _need(K, torch.bfloat16, "K")
-    _need(V, torch.bfloat16, "V")
-    _need(idx, torch.int32, "idx")
     B, Lq, Hq, d = Q.shape
+    _need(K, torch.bfloat16, "K")  # [B, Lk, d] (a [B, Lk, 1, d] view of one shared head is accepted)
+    if K.shape[0] != B or K.shape[-1] != d:
+        raise ValueError(f"K has shape {tuple(K.shape)}, expected [{B}, Lk, {d}]")
     Lk = K.shape[1]
+    _need_numel(K, B * Lk * d, "K", f"[{B}, {Lk}, {d}]: one shared K/V head")
+    _need(V, torch.bfloat16, "V", K.shape)
+    _need(idx, torch.int32, "idx")
+    if idx.dim() != 3 or idx.shape[0] != B or idx.shape[1] != Lq:
+        raise ValueError(f"idx has shape {tuple(idx.shape)}, expected [{B}, {Lq}, k]")
     k = idx.shape[-1]
+    if O is not None:
+        _need(O, torch.bfloat16, "O", Q.shape)
+    if lse is not None:
+        _need(lse, torch.float32, "lse", (B, Lq, Hq))
+    _on_device(Q, K, V, idx, O, lse)
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     O = torch.empty_like(Q) if O is None else O
