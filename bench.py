@@ -415,9 +415,9 @@ def ours(args):
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
     clocks = ClockSampler(local)
+    clocks.start()  # waits for its first sample, so it runs before the barrier that opens timing
     if dist:
         dist.barrier()
-    clocks.start()
     torch.cuda.synchronize()
     clocks.begin()
     t_start = torch.cuda.Event(enable_timing=True)
