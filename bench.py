@@ -200,29 +200,44 @@ class ClockSampler:
 
 # ----------------------------------------------------------------------------- our arm
 
+class _Draw:
+    """Seeded draws on the device with torch's generator (same laws as synth, other values);
+    each tensor has its own id, so a layer's inputs do not depend on which others are drawn."""
+
+    def __init__(self, device, seed):
+        self.device, self.seed = device, seed
+        self.g = torch.Generator(device=device)
+
+    def normal(self, shape, sigma, tid):
+        self.g.manual_seed(self.seed * 1000 + tid)
+        return (torch.randn(*shape, generator=self.g, device=self.device) * sigma).to(torch.bfloat16)
+
+    def ints(self, shape, lo, hi, tid, dtype):
+        self.g.manual_seed(self.seed * 1000 + tid)
+        return torch.randint(lo, hi + 1, shape, generator=self.g, device=self.device, dtype=torch.int64).to(dtype)
+
+    def uniform(self, n, hi, tid):
+        self.g.manual_seed(self.seed * 1000 + tid)
+        return torch.rand(n, generator=self.g, device=self.device) * hi
+
+
+def make_hca_inputs(device, seed):
+    d, sh = _Draw(device, seed), 1 / math.sqrt(HCA.d)
+    return {"hQ": d.normal((1, L, HCA.Hq, HCA.d), sh, 1), "hK": d.normal((1, L, HCA.Hkv, HCA.d), sh, 2),
+            "hV": d.normal((1, L, HCA.Hkv, HCA.d), sh, 3), "w": d.uniform(HCA.blk, 2.0 / HCA.blk, 4)}
+
+
+def make_dsa_inputs(device, seed):
+    d, sd = _Draw(device, seed), 1 / math.sqrt(DSA.d)
+    return {"dQ": d.normal((1, L, DSA.Hq, DSA.d), sd, 11), "dK": d.normal((1, L, DSA.d), sd, 12),
+            "dV": d.normal((1, L, DSA.d), sd, 13),
+            "q_idx": d.ints((1, L, 4, 64), -8, 8, 15, torch.int8), "k_idx": d.ints((1, L, 64), -8, 8, 16, torch.int8),
+            "w_idx": d.ints((4,), 1, 4, 17, torch.int32)}
+
+
 def make_inputs(device, seed):
-    """Bench inputs drawn on the device with torch's generator (same laws as synth, other values)."""
-    g = torch.Generator(device=device)
-
-    def normal(shape, sigma, tid):
-        g.manual_seed(seed * 1000 + tid)
-        return (torch.randn(*shape, generator=g, device=device) * sigma).to(torch.bfloat16)
-
-    def ints(shape, lo, hi, tid, dtype):
-        g.manual_seed(seed * 1000 + tid)
-        return torch.randint(lo, hi + 1, shape, generator=g, device=device, dtype=torch.int64).to(dtype)
-
-    sh, sd = 1 / math.sqrt(HCA.d), 1 / math.sqrt(DSA.d)
-    g.manual_seed(seed * 1000 + 4)
-    w = torch.rand(HCA.blk, generator=g, device=device) * (2.0 / HCA.blk)
-    return {
-        "hQ": normal((1, L, HCA.Hq, HCA.d), sh, 1), "hK": normal((1, L, HCA.Hkv, HCA.d), sh, 2),
-        "hV": normal((1, L, HCA.Hkv, HCA.d), sh, 3), "w": w,
-        "dQ": normal((1, L, DSA.Hq, DSA.d), sd, 11), "dK": normal((1, L, DSA.d), sd, 12),
-        "dV": normal((1, L, DSA.d), sd, 13),
-        "q_idx": ints((1, L, 4, 64), -8, 8, 15, torch.int8), "k_idx": ints((1, L, 64), -8, 8, 16, torch.int8),
-        "w_idx": ints((4,), 1, 4, 17, torch.int32),
-    }
+    """Bench inputs of both layers (see _Draw)."""
+    return {**make_hca_inputs(device, seed), **make_dsa_inputs(device, seed)}
 
 
 class Step:
@@ -534,17 +549,35 @@ def only_kernel(args):
     global L
     L = args.seq_len
     device = torch.device("cuda", 0)
-    x = make_inputs(device, seed=synth.SEED)
-    st = Step(hd, x, device)
-    st.run()
+    # only the selected kernel's layer is allocated (a profiled launch should hold a few GB at
+    # most; the top-k score workspace alone is 4 L^2 bytes)
+    if args.only in ("compress", "hca_attn"):
+        x = make_hca_inputs(device, seed=synth.SEED)
+        Kc = torch.empty((1, L // 128, 1, HCA.d), dtype=torch.bfloat16, device=device)
+        Vc = torch.empty_like(Kc)
+        hd.hca_compress_kv(x["hK"], x["hV"], x["w"], 128, Kc=Kc, Vc=Vc)
+        if args.only == "compress":
+            fn = lambda: hd.hca_compress_kv(x["hK"], x["hV"], x["w"], 128, Kc=Kc, Vc=Vc)  # noqa: E731
+        else:
+            hO = torch.empty_like(x["hQ"])
+            nb = hd.lib().hca_attn_fwd_workspace_size(1, L, 0, HCA.Hq, HCA.Hkv, HCA.d, L // 128, 128, 128)
+            hws = torch.empty(max(nb, 16), dtype=torch.uint8, device=device)
+            fn = lambda: hd.hca_attn_fwd(x["hQ"], Kc, Vc, x["hK"], x["hV"], O=hO, workspace=hws)  # noqa: E731
+    else:
+        x = make_dsa_inputs(device, seed=synth.SEED)
+        idx = torch.empty((1, L, DSA.k), dtype=torch.int32, device=device)
+        ws = torch.empty(hd.dsa_index_topk_workspace_size(1, L, 0, L, DSA.k), dtype=torch.uint8, device=device)
+        hd.dsa_index_topk(x["q_idx"], x["k_idx"], x["w_idx"], DSA.k, idx=idx, workspace=ws)
+        if args.only == "index_topk":
+            fn = lambda: hd.dsa_index_topk(x["q_idx"], x["k_idx"], x["w_idx"], DSA.k, idx=idx,  # noqa: E731
+                                           workspace=ws)
+        else:
+            torch.cuda.synchronize()
+            del ws  # the attention needs only the index rows
+            torch.cuda.empty_cache()
+            dO = torch.empty_like(x["dQ"])
+            fn = lambda: hd.dsa_sparse_attn_fwd(x["dQ"], x["dK"], x["dV"], idx, O=dO)  # noqa: E731
     torch.cuda.synchronize()
-    fn = {
-        "compress": lambda: hd.hca_compress_kv(x["hK"], x["hV"], x["w"], 128, Kc=st.Kc, Vc=st.Vc),
-        "hca_attn": lambda: hd.hca_attn_fwd(x["hQ"], st.Kc, st.Vc, x["hK"], x["hV"], O=st.hO, workspace=st.hws),
-        "index_topk": lambda: hd.dsa_index_topk(x["q_idx"], x["k_idx"], x["w_idx"], DSA.k, idx=st.idx,
-                                                workspace=st.ws),
-        "dsa_attn": lambda: hd.dsa_sparse_attn_fwd(x["dQ"], x["dK"], x["dV"], st.idx, O=st.dO),
-    }[args.only]
     for _ in range(args.warmup):
         fn()
     torch.cuda.synchronize()
