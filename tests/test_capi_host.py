@@ -77,6 +77,9 @@ def test_hca_attn_argument_errors(lib):
     assert call(O=MISALIGNED) == -3
     assert call(n_w=1000) == -2          # window of the last query not stored
     assert call(n_c=6) == -2             # entries of the last query not stored
+    assert call(ws=1, n_w=1023) == -2    # the window buffer starts after the first query's window
+    assert call(q0=-1) == -2
+    assert call(lse=ctypes.c_void_p(FAKE.value + 2)) == -3   # lse must be 4-byte aligned
     assert call(Lq=0) == 0
 
 
