@@ -186,9 +186,14 @@ class ClockSampler:
         window = "timed region"
         inside = [r for r in rows if r[0] is not None and self.t0 is not None and self.t1 is not None
                   and self.t0 - 0.02 <= r[0] <= self.t1 + 0.02]
-        if not inside:  # no sample fell inside (a very short region): report the nearest ones
-            window = "around the timed region"
-            inside = rows
+        if not inside and self.t0 is not None and self.t1 is not None:
+            # no sample fell inside (a very short region): the two samples nearest to it in time
+            window = "nearest samples to the timed region"
+            stamped = [r for r in rows if r[0] is not None]
+            dist = lambda r: max(self.t0 - r[0], r[0] - self.t1, 0.0)  # noqa: E731
+            inside = sorted(stamped, key=dist)[:2]
+        if not inside:
+            return None
         reasons = set()
         for r in inside:
             for n, v in zip(names, r[3]):
@@ -333,6 +338,56 @@ def run_decode(hd, device, iters=20):
     return out
 
 
+def run_hca_131k(hd, device, peaks, iters=10):
+    """The HCA long-context prefill configuration (B = 1, L = 131072, 16 query heads on one K/V
+    head, d = 512, 1024 compressed entries): compression and attention timed with CUDA events
+    after 3 warm-up runs (median of `iters`), with its own clock record."""
+    Lh = synth.HCA_131K.L
+    d = _Draw(device, synth.SEED)
+    sh = 1 / math.sqrt(HCA.d)
+    Q = d.normal((1, Lh, HCA.Hq, HCA.d), sh, 21)
+    K = d.normal((1, Lh, HCA.Hkv, HCA.d), sh, 22)
+    V = d.normal((1, Lh, HCA.Hkv, HCA.d), sh, 23)
+    w = d.uniform(HCA.blk, 2.0 / HCA.blk, 24)
+    Kc = torch.empty((1, Lh // 128, 1, HCA.d), dtype=torch.bfloat16, device=device)
+    Vc = torch.empty_like(Kc)
+    O = torch.empty_like(Q)
+    nb = hd.lib().hca_attn_fwd_workspace_size(1, Lh, 0, HCA.Hq, HCA.Hkv, HCA.d, Lh // 128, 128, 128)
+    ws = torch.empty(max(nb, 16), dtype=torch.uint8, device=device)
+
+    def step(ev=None):
+        if ev: ev[0].record()
+        hd.hca_compress_kv(K, V, w, 128, Kc=Kc, Vc=Vc)
+        if ev: ev[1].record()
+        hd.hca_attn_fwd(Q, Kc, Vc, K, V, O=O, workspace=ws)
+        if ev: ev[2].record()
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(device.index or 0)
+    clocks.start()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(iters)]
+    clocks.begin()
+    for i in range(iters):
+        step(evs[i])
+    torch.cuda.synchronize()
+    clocks.end()
+    clk = clocks.stop()
+    comp_ms = statistics.median(e[0].elapsed_time(e[1]) for e in evs)
+    attn_ms = statistics.median(e[1].elapsed_time(e[2]) for e in evs)
+    flop = 4.0 * HCA.d * HCA.Hq * hca_visible_keys_per_head(Lh)
+    comp_bytes = 2 * (Lh * HCA.Hkv * HCA.d * 2) + 2 * ((Lh // 128) * HCA.Hkv * HCA.d * 2) + 128 * 4
+    tf = flop / (attn_ms * 1e-3) / 1e12
+    gbs = comp_bytes / (comp_ms * 1e-3) / 1e9
+    del Q, K, V, O, ws
+    torch.cuda.empty_cache()
+    return {"workload": "hca_prefill_L131072_hq16_hkv1_d512 (B=1)", "iters": iters,
+            "compress_us": comp_ms * 1e3, "compress_gbs": gbs, "compress_pct_hbm": 100 * gbs / peaks["hbm_gbs"],
+            "attn_ms": attn_ms, "attn_tflops": tf, "attn_pct_bf16": 100 * tf / peaks["bf16_tflops"],
+            "algorithmic_flop": flop, "tokens_per_s": Lh / ((comp_ms + attn_ms) * 1e-3), "clocks": clk}
+
+
 def e2e_measure(hd, x, device, steps):
     """Same step through the C ABI with host buffers: H2D of every input from pinned memory and
     D2H of both layer outputs inside the timed region."""
@@ -401,7 +456,9 @@ def cpu_sample(n_hca=12288, n_dsa=3072):
         "value": 1.0 / per_token, "unit": "tokens/s", "cores": cores, "kind": "oracle",
         "sample": (f"full compression of the L={L} sequence; HCA attention (16 heads) for {n_hca} and DSA "
                    f"top-{DSA.k} + attention (64 heads) for {n_dsa} query tokens spread evenly over [0, {L}); "
-                   f"tokens/s = 1 / (compress/L + HCA per row + DSA per row)"),
+                   f"tokens/s extrapolated from the sample's per-token cost = 1 / (compress/L + HCA per row "
+                   f"+ DSA per row)"),
+        "extrapolated": True,
         "sample_seconds": t_comp + t_hca + t_dsa,
     }
 
@@ -454,12 +511,20 @@ def ours(args):
     peaks = load_peaks()
     hca_tf = HCA_FLOP / (hca_ms * 1e-3) / 1e12
     dsa_tf = DSA_FLOP / (dsa_ms * 1e-3) / 1e12
+    # The timed region is well under a second at full clock, so the denominator is the burst
+    # peak (a cuBLAS bf16 GEMM timed alone); the sustained figure was taken over seconds under
+    # the power cap at ~1.34 GHz and is reported beside it for context only.
+    peak_b = peaks["bf16_tflops"]
     peak_s = peaks["bf16_tflops_sustained"]
 
     decode = None
     e2e = None
+    hca131 = None
     if rank == 0 and not args.no_decode:
         decode = run_decode(hd, device)
+        hd.hcadsa_check_device_error()
+    if rank == 0 and not args.no_131k:
+        hca131 = run_hca_131k(hd, device, peaks)
         hd.hcadsa_check_device_error()
     e2e_ms, h2d, d2h = e2e_measure(hd, x, device, steps=max(2, min(args.steps, 4)))
     e2e_ms = max_over_ranks(e2e_ms, dist, device)
@@ -481,27 +546,31 @@ def ours(args):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic (seeded; Q/K/V ~N(0,1)/sqrt(d) bf16, int8 indexer U[-8,8], weights U[1,4], w~U(0,2/128))",
-        "config": {"workload": WORKLOAD, "global_batch": world, "seq_len": L, "parallelism": f"replicas{world}",
-                   "l2": "inputs larger than L2 (1.5 GiB of Q per step), no flush"},
+        "config": bench_config(world),
         "layers": {
             "hca": {"compress_us": comp_ms * 1e3, "compress_gbs": COMPRESS_BYTES / (comp_ms * 1e-3) / 1e9,
-                    "attn_ms": hca_ms, "attn_tflops": hca_tf, "attn_pct_bf16_sustained": 100 * hca_tf / peak_s,
+                    "compress_pct_hbm": 100 * COMPRESS_BYTES / (comp_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                    "attn_ms": hca_ms, "attn_tflops": hca_tf, "attn_pct_bf16": 100 * hca_tf / peak_b,
                     "layer_tokens_per_s": L / ((comp_ms + hca_ms) * 1e-3)},
             "dsa": {"index_topk_ms": idx_ms, "attn_ms": dsa_ms, "attn_tflops": dsa_tf,
-                    "attn_pct_bf16_sustained": 100 * dsa_tf / peak_s,
+                    "attn_pct_bf16": 100 * dsa_tf / peak_b,
                     "layer_tokens_per_s": L / ((idx_ms + dsa_ms) * 1e-3)},
             "algorithmic_flop": {"hca_attn": HCA_FLOP, "dsa_attn": DSA_FLOP},
+            "peak_note": f"percentages of the burst bf16 peak {peak_b} TFLOP/s and of {peaks['hbm_gbs']} GB/s "
+                         f"({peaks['src']})",
         },
         "roofline": {"kernel": "dsa_sparse_attn_fwd", "bound": "tensor", "achieved": dsa_tf,
-                     "peak": peak_s, "unit": "TFLOP/s", "frac": dsa_tf / peak_s,
-                     "peak_kind": f"bf16_tflops_sustained ({peaks['src']})",
-                     "frac_of_burst_peak": dsa_tf / peaks["bf16_tflops"], "traffic": traffic,
+                     "peak": peak_b, "unit": "TFLOP/s", "frac": dsa_tf / peak_b,
+                     "peak_kind": f"bf16_tflops, burst ({peaks['src']}): the kernel runs for ~10 ms at a time "
+                                  "inside a sub-second timed region at full clock",
+                     "frac_of_sustained_peak": dsa_tf / peak_s, "traffic": traffic,
                      "units_per_launch": f"{DSA_KEYS} visible keys x 64 heads x 4*256 flop"},
         "cpu_baseline": cpu,
         "e2e": e2e,
         "gpu_launches": Step.N_KERNELS * args.steps,
         "clocks": clk,
         "decode": decode,
+        "hca_131k": hca131,
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -510,25 +579,36 @@ def ours(args):
         dist.destroy_process_group()
 
 
+def bench_config(world):
+    """The workload description both arms print (the reference arm runs the same workload)."""
+    return {"workload": WORKLOAD, "global_batch": world, "seq_len": L, "parallelism": f"replicas{world}",
+            "l2": "inputs larger than L2 (1.5 GiB of Q per step), no flush"}
+
+
 def reference(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    per = []
+    per, secs = [], []
     cpu = None
     for _ in range(args.warmup):
         cpu_sample(n_hca=256, n_dsa=32)
     for _ in range(args.steps):
         cpu = cpu_sample(n_hca=1024, n_dsa=128)
         per.append(cpu["value"])
+        secs.append(cpu["sample_seconds"])
     v = statistics.median(per)
     cpu["value"] = v
+    # Each timed step is the bounded row sample (what ms_per_step reports); value is the tokens/s
+    # of the whole workload extrapolated from the sample's per-token cost.
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * L / v, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "global_batch": 1, "seq_len": L, "parallelism": "host cores"},
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * statistics.mean(secs),
+        "ms_per_full_step_extrapolated": 1e3 * L / v, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (same laws as the GPU arm); value extrapolated from a bounded row sample",
+        "config": bench_config(world),
         "cpu_baseline": cpu,
         "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }), flush=True)
@@ -599,6 +679,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-131k", action="store_true", help="skip the L = 131072 HCA block")
     ap.add_argument("--only", choices=["compress", "hca_attn", "index_topk", "dsa_attn", "decode"],
                     help="profiling mode: run one kernel alone at --seq-len, or the decode step "
                          "(B = 32 at t = 1,048,575; --steps timed steps after 3 warm-up steps)")

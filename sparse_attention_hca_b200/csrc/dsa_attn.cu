@@ -1,4 +1,5 @@
-// dsa_attn.cu -- DSA sparse attention forward on sm_100a (tcgen05 + TMEM + TMA gather).
+// dsa_attn.cu -- DSA sparse attention forward on sm_100a (tcgen05 + TMEM; K/V rows gathered
+// with cp.async, Q loaded by TMA).
 //
 // Method: the mirrorspeed page, section "Hybrid sparse attention, 1/7 full context
 // access": in the MLA layers each query attends only to the k positions its indexer

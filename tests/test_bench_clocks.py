@@ -45,10 +45,14 @@ def test_only_samples_inside_the_timed_region_count():
 
 
 def test_short_region_reports_the_nearest_samples():
+    """Only the two samples closest in time to the region stand in for it; idle samples further
+    away (here a low-clock one with a throttle reason) are left out."""
     t0 = time.time()
-    rec = _sampler(t0, [(0.0, 1965, False), (0.5, 1900, False)], 0.2, 0.21).stop()
-    assert rec["window"] == "around the timed region"
+    rows = [(0.0, 300, True), (0.15, 1965, False), (0.26, 1950, False), (0.9, 345, True)]
+    rec = _sampler(t0, rows, 0.2, 0.21).stop()
+    assert rec["window"] == "nearest samples to the timed region"
     assert rec["samples"] == 2
+    assert rec["sm_mhz"] == 1957.5 and rec["reasons"] == []
 
 
 def test_no_nvidia_smi_gives_no_record():

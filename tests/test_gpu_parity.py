@@ -182,6 +182,7 @@ def test_hca_32k_sampled(hd):
     rows = _sample_rows(cfg.L, extra=(8191, 16384, 32000))
     O, lse, ref, ref_lse = _hca_gpu_and_oracle(hd, cfg, rows=rows)
     print(check_attn(O, ref, "hca 32k sampled"))
+    np.testing.assert_allclose(lse.cpu().numpy(), ref_lse, atol=2e-3, rtol=0)
 
 
 def test_hca_131k_sampled(hd):
@@ -189,6 +190,7 @@ def test_hca_131k_sampled(hd):
     rows = _sample_rows(cfg.L, extra=(65536, 100000, 131000))
     O, lse, ref, ref_lse = _hca_gpu_and_oracle(hd, cfg, rows=rows)
     print(check_attn(O, ref, "hca 131k sampled"))
+    np.testing.assert_allclose(lse.cpu().numpy(), ref_lse, atol=2e-3, rtol=0)
 
 
 @pytest.mark.parametrize("B,t", [(2, 5000), (3, 130)])
@@ -428,32 +430,36 @@ def test_topk_32k_sampled_rows(hd):
 
 # ------------------------------------------------------------------ DSA sparse attention
 
-def _dsa_attn_case(hd, cfg, rows, sigma_tag=""):
-    """GPU attention fed the ORACLE's index rows for the sampled queries."""
+def _dsa_attn_case(hd, cfg, rows):
+    """GPU attention fed the ORACLE's index rows for the sampled queries; returns the GPU and
+    oracle outputs and log-sum-exps of those rows."""
     inp = synth.dsa_inputs(cfg)
     idx_o = oracle.dsa_topk(inp["q_idx"].numpy(), inp["k_idx"].numpy(), inp["w_idx"].numpy(), cfg.k, rows=rows)
     Qs = inp["Q"].reshape(cfg.B * cfg.L, 1, cfg.Hq, cfg.d)[torch.as_tensor(rows)]   # one query per sequence row
     # every sampled row becomes its own "token" of a batch-1 call over the key sequence of its batch
-    outs = []
+    outs, lses = [], []
     for b in range(cfg.B):
         sel = (rows // cfg.L) == b
         if not sel.any():
             continue
         q_b = Qs[torch.as_tensor(np.nonzero(sel)[0])].reshape(1, -1, cfg.Hq, cfg.d)
-        O = hd.dsa_sparse_attn_fwd(q_b.cuda(), inp["K"][b:b + 1].cuda(), inp["V"][b:b + 1].cuda(),
-                                   torch.as_tensor(idx_o[sel]).reshape(1, -1, cfg.k).cuda())
+        O, lse = hd.dsa_sparse_attn_fwd(q_b.cuda(), inp["K"][b:b + 1].cuda(), inp["V"][b:b + 1].cuda(),
+                                        torch.as_tensor(idx_o[sel]).reshape(1, -1, cfg.k).cuda(), return_lse=True)
         outs.append(O.reshape(-1, cfg.Hq, cfg.d))
+        lses.append(lse.reshape(-1, cfg.Hq))
     no_device_error(hd)
-    ref = oracle.dsa_attn(bits(inp["Q"]), bits(inp["K"]), bits(inp["V"]), idx_o, rows=rows)
-    return torch.cat(outs), ref
+    ref, ref_lse = oracle.dsa_attn(bits(inp["Q"]), bits(inp["K"]), bits(inp["V"]), idx_o, rows=rows, with_lse=True)
+    return torch.cat(outs), torch.cat(lses), ref, ref_lse
 
 
 @pytest.mark.parametrize("L,k,sigma", [(3000, 2048, None), (2000, 256, 1.0), (300, 2048, 1.0), (500, 100, 2.0)])
 def test_dsa_attn_against_oracle(hd, L, k, sigma):
     cfg = _dsa_cfg("dsa", L, k=k, sigma=sigma)
     rows = _sample_rows(L, extra=(k - 1, k, k + 1, L - 3))
-    O, ref = _dsa_attn_case(hd, cfg, rows)
+    O, lse, ref, ref_lse = _dsa_attn_case(hd, cfg, rows)
     print(check_attn(O, ref, f"dsa L={L} k={k} sigma={sigma}", value_scale=sigma or 1.0))
+    # natural-log log-sum-exp of the selected scores, per head (the backward consumes it)
+    np.testing.assert_allclose(lse.cpu().numpy(), ref_lse, atol=2e-3 * max(1.0, (sigma or 1.0) ** 2), rtol=0)
 
 
 def test_dsa_pipeline_32k_sampled(hd):
@@ -462,14 +468,15 @@ def test_dsa_pipeline_32k_sampled(hd):
     inp = synth.dsa_inputs(cfg)
     dev = {k: v.cuda() for k, v in inp.items()}
     idx = hd.dsa_index_topk(dev["q_idx"], dev["k_idx"], dev["w_idx"], cfg.k)
-    O = hd.dsa_sparse_attn_fwd(dev["Q"], dev["K"], dev["V"], idx)
+    O, lse = hd.dsa_sparse_attn_fwd(dev["Q"], dev["K"], dev["V"], idx, return_lse=True)
     no_device_error(hd)
     rows = _sample_rows(cfg.L, extra=(2047, 2048, 20000))
     idx_o = oracle.dsa_topk(inp["q_idx"].numpy(), inp["k_idx"].numpy(), inp["w_idx"].numpy(), cfg.k, rows=rows)
     r = torch.as_tensor(rows, device="cuda")
     assert np.array_equal(idx.reshape(cfg.L, cfg.k)[r].cpu().numpy(), idx_o)
-    ref = oracle.dsa_attn(bits(inp["Q"]), bits(inp["K"]), bits(inp["V"]), idx_o, rows=rows)
+    ref, ref_lse = oracle.dsa_attn(bits(inp["Q"]), bits(inp["K"]), bits(inp["V"]), idx_o, rows=rows, with_lse=True)
     print(check_attn(O.reshape(cfg.L, cfg.Hq, cfg.d)[r], ref, "dsa 32k pipeline"))
+    np.testing.assert_allclose(lse.reshape(cfg.L, cfg.Hq)[r].cpu().numpy(), ref_lse, atol=2e-3, rtol=0)
 
 
 def test_dsa_padding_and_order(hd):
@@ -488,6 +495,92 @@ def test_dsa_padding_and_order(hd):
     no_device_error(hd)
     ref = oracle.dsa_attn(bits(inp["Q"]), bits(inp["K"]), bits(inp["V"]), idx)
     print(check_attn(O, ref, "dsa padded/shuffled"))
+
+
+def test_dsa_all_padding_rows_and_lse(hd):
+    """Rows whose index list holds no valid entry (all -1) give O = 0 and lse = -inf, the
+    oracle's empty-set case; their neighbours (partly padded, shuffled) still match the oracle
+    in O and lse."""
+    cfg = _dsa_cfg("allpad", 300, k=256, sigma=1.0)
+    inp = synth.dsa_inputs(cfg)
+    rng = np.random.default_rng(17)
+    idx = np.full((cfg.L, cfg.k), -1, np.int32)
+    empty = {0, 1, 5, 128, 129, 200, 299}
+    for t in range(cfg.L):
+        if t in empty:
+            continue
+        n = min(cfg.k, t + 1, int(rng.integers(1, cfg.k + 1)))
+        idx[t, rng.choice(cfg.k, size=n, replace=False)] = rng.choice(t + 1, size=n, replace=False)
+    O, lse = hd.dsa_sparse_attn_fwd(inp["Q"].cuda(), inp["K"].cuda(), inp["V"].cuda(),
+                                    torch.as_tensor(idx).reshape(1, cfg.L, cfg.k).cuda(), return_lse=True)
+    no_device_error(hd)
+    ref, ref_lse = oracle.dsa_attn(bits(inp["Q"]), bits(inp["K"]), bits(inp["V"]), idx, with_lse=True)
+    O = O.reshape(cfg.L, cfg.Hq, cfg.d)
+    lse = lse.reshape(cfg.L, cfg.Hq).cpu().numpy()
+    e = sorted(empty)
+    assert torch.count_nonzero(O[e]).item() == 0
+    assert np.all(np.isneginf(lse[e])) and np.all(np.isneginf(ref_lse[e]))
+    assert np.all(ref[e] == 0.0)
+    keep = np.array([t for t in range(cfg.L) if t not in empty])
+    print(check_attn(O[torch.as_tensor(keep, device="cuda")], ref[keep], "dsa all-padding neighbours"))
+    np.testing.assert_allclose(lse[keep], ref_lse[keep], atol=2e-3, rtol=0)
+
+
+def test_dsa_index_out_of_range_is_reported(hd):
+    """An index entry >= Lk is a caller error the host cannot see: the kernel skips it (no read
+    outside K/V), records HCADSA_ERR_DEVICE_BOUNDS, and the row is the attention over its other
+    entries."""
+    cfg = _dsa_cfg("oob", 260, k=128, sigma=1.0)
+    inp = synth.dsa_inputs(cfg)
+    rows = np.array([10, 129, 259], np.int64)
+    idx_o = oracle.dsa_topk(inp["q_idx"].numpy(), inp["k_idx"].numpy(), inp["w_idx"].numpy(), cfg.k, rows=rows)
+    bad = idx_o.copy()
+    bad[0, 3] = cfg.L          # one past the end
+    bad[1, 0] = cfg.L + 12345  # far past the end
+    bad[2, 127] = 2 ** 30
+    q = inp["Q"].reshape(cfg.L, cfg.Hq, cfg.d)[torch.as_tensor(rows)].reshape(1, len(rows), cfg.Hq, cfg.d)
+    hd.hcadsa_check_device_error()  # start from a clear error word
+    O = hd.dsa_sparse_attn_fwd(q.cuda(), inp["K"].cuda(), inp["V"].cuda(),
+                               torch.as_tensor(bad).reshape(1, len(rows), cfg.k).cuda())
+    with pytest.raises(hd.HcaDsaError) as e:
+        hd.hcadsa_check_device_error()
+    assert e.value.status == -8
+    hd.hcadsa_check_device_error()  # reading the word cleared it
+    skipped = np.where(bad >= cfg.L, -1, bad)
+    qb = bits(inp["Q"]).reshape(cfg.L, cfg.Hq, cfg.d)[rows].reshape(1, len(rows), cfg.Hq, cfg.d)
+    ref = oracle.dsa_attn(qb, bits(inp["K"]), bits(inp["V"]), skipped)
+    print(check_attn(O.reshape(len(rows), cfg.Hq, cfg.d), ref, "dsa out-of-range entries skipped"))
+
+
+def test_dsa_decode_1m_batch32_sampled(hd):
+    """The benchmarked decode call exactly: 32 sequences, one query each at t = 1,048,575, top-2048
+    and sparse attention in one launch each; top-k (bit-exact), O and lse checked against the
+    oracle on 4 of the 32 sequences.  Inputs are drawn on the device with torch's seeded generator
+    (the same laws as the synthetic generators; 34 GB of caches) and copied to the host for the
+    oracle."""
+    cfg = synth.DECODE_1M
+    B, t, Lk = cfg.B, cfg.t, cfg.t + 1
+    dev = torch.device("cuda")
+    seed = 91
+    q_idx = synth.randint((B, 1, 4, 64), -8, 8, seed, "q_idx", torch.int8, dev)
+    k_idx = synth.randint((B, Lk, 64), -8, 8, seed, "k_idx", torch.int8, dev)
+    w_idx = synth.randint((4,), 1, 4, seed, "w_idx", torch.int32, dev)
+    Q = synth.normal_bf16((B, 1, 64, 256), 1.0, seed, "Q", dev)
+    K = synth.normal_bf16((B, Lk, 256), 1.0, seed, "K", dev)
+    V = synth.normal_bf16((B, Lk, 256), 1.0, seed, "V", dev)
+    idx = hd.dsa_index_topk(q_idx, k_idx, w_idx, cfg.k, q_offset=t)
+    O, lse = hd.dsa_sparse_attn_fwd(Q, K, V, idx, return_lse=True)
+    no_device_error(hd)
+    for b in (0, 7, 19, 31):
+        sl = slice(b, b + 1)
+        idx_o = oracle.dsa_topk(q_idx[sl].cpu().numpy(), k_idx[sl].cpu().numpy(), w_idx.cpu().numpy(), cfg.k,
+                                q_offset=t)
+        assert np.array_equal(idx[b].cpu().numpy(), idx_o), f"sequence {b}"
+        ref, ref_lse = oracle.dsa_attn(bits(Q[sl]), bits(K[sl]), bits(V[sl]), idx_o, with_lse=True)
+        print(check_attn(O[b].reshape(1, 64, 256), ref, f"dsa decode B=32 sequence {b}"))
+        np.testing.assert_allclose(lse[b].reshape(1, 64).cpu().numpy(), ref_lse, atol=2e-3, rtol=0)
+    del K, V, k_idx
+    torch.cuda.empty_cache()
 
 
 def test_dsa_decode_1m_sampled_batch(hd):

@@ -5,7 +5,7 @@ device memory, callers with no workspace allocator).
 dsa_index_topk_noalloc keeps its score rows in a fixed array inside the library.  Its GPU
 test compares it, through the C ABI, against dsa_index_topk (which uses a caller workspace)
 on two calls in a row with different inputs, so a second call that saw stale scratch from
-the first would show.  This file sorts last so a stop-at-first-failure run has already run
+the first would show, and checks sampled rows of both against the CPU oracle.  This file sorts last so a stop-at-first-failure run has already run
 every other test; the test also passes on its own in a fresh process.
 """
 import ctypes
@@ -14,6 +14,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 import synth
 
 
@@ -71,3 +72,10 @@ def test_noalloc_matches_workspace_entry_on_two_calls_in_a_row():
         # top-k indices: the tolerance of every top-k test here is bit-exact
         assert torch.equal(got, ref)
         assert (got[..., 0] >= 0).all()
+        # ... and both equal the oracle on sampled rows (the two entries share their scoring
+        # kernels, so the comparison above alone would not see a scoring fault)
+        rows = np.unique(np.linspace(0, c["B"] * c["Lq"] - 1, 12).astype(np.int64))
+        want = oracle.dsa_topk(q.cpu().numpy(), kk.cpu().numpy(), w.cpu().numpy(), c["k"], q_offset=c["q_offset"],
+                               rows=rows)
+        flat = got.reshape(c["B"] * c["Lq"], c["k"])[torch.as_tensor(rows, device="cuda")].cpu().numpy()
+        assert np.array_equal(flat, want)
