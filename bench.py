@@ -338,6 +338,61 @@ def run_decode(hd, device, iters=20):
     return out
 
 
+def csa_keys_per_head(L, k=2048, blk=4):
+    return sum(min(k, (t + 1) // blk) for t in range(L))
+
+
+def run_csa(hd, device, peaks, iters=10):
+    """The CSA layer (compressed sparse attention, the pages' comparison point) at the MLA-DSA
+    layer's size: B = 1, L = 32768, K/V compressed 4:1 (8192 entries, d = 256), indexer + top-2048
+    over the complete blocks, sparse attention of 64 heads over the selected entries.  CUDA events
+    per kernel, median of `iters` after 3 warm-up runs."""
+    Lc, blk, k = L, 4, DSA.k
+    n_c = Lc // blk
+    d = _Draw(device, synth.SEED)
+    sd = 1 / math.sqrt(DSA.d)
+    Q = d.normal((1, Lc, DSA.Hq, DSA.d), sd, 31)
+    K = d.normal((1, Lc, 1, DSA.d), sd, 32)
+    V = d.normal((1, Lc, 1, DSA.d), sd, 33)
+    w4 = d.uniform(blk, 2.0 / blk, 34)
+    q_idx = d.ints((1, Lc, 4, 64), -8, 8, 35, torch.int8)
+    kc_idx = d.ints((1, n_c, 64), -8, 8, 36, torch.int8)
+    w_idx = d.ints((4,), 1, 4, 37, torch.int32)
+    Kc = torch.empty((1, n_c, 1, DSA.d), dtype=torch.bfloat16, device=device)
+    Vc = torch.empty_like(Kc)
+    idx = torch.empty((1, Lc, k), dtype=torch.int32, device=device)
+    ws = torch.empty(max(hd.lib().csa_index_topk_workspace_size(1, Lc, 0, n_c, k, blk), 16), dtype=torch.uint8,
+                     device=device)
+    O = torch.empty_like(Q)
+
+    def step(ev=None):
+        if ev: ev[0].record()
+        hd.hca_compress_kv(K, V, w4, blk, Kc=Kc, Vc=Vc)
+        if ev: ev[1].record()
+        hd.csa_index_topk(q_idx, kc_idx, w_idx, k, blk, idx=idx, workspace=ws)
+        if ev: ev[2].record()
+        hd.dsa_sparse_attn_fwd(Q, Kc.view(1, n_c, DSA.d), Vc.view(1, n_c, DSA.d), idx, O=O)
+        if ev: ev[3].record()
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(iters)]
+    for i in range(iters):
+        step(evs[i])
+    torch.cuda.synchronize()
+    ms = [statistics.median(e[i].elapsed_time(e[i + 1]) for e in evs) for i in range(3)]
+    flop = 4.0 * DSA.d * DSA.Hq * csa_keys_per_head(Lc, k, blk)
+    comp_bytes = 2 * (Lc * DSA.d * 2) + 2 * (n_c * DSA.d * 2) + blk * 4
+    tf = flop / (ms[2] * 1e-3) / 1e12
+    del Q, K, V, O, idx, Kc, Vc
+    torch.cuda.empty_cache()
+    return {"workload": "csa_prefill_L32768_h64_d256_blk4_k2048 (B=1; 8192 entries)", "iters": iters,
+            "compress_us": ms[0] * 1e3, "compress_gbs": comp_bytes / (ms[0] * 1e-3) / 1e9,
+            "index_topk_ms": ms[1], "attn_ms": ms[2], "attn_tflops": tf, "attn_pct_bf16": 100 * tf / peaks["bf16_tflops"],
+            "algorithmic_flop": flop, "layer_tokens_per_s": Lc / (sum(ms) * 1e-3)}
+
+
 def run_hca_131k(hd, device, peaks, iters=10):
     """The HCA long-context prefill configuration (B = 1, L = 131072, 16 query heads on one K/V
     head, d = 512, 1024 compressed entries): compression and attention timed with CUDA events
@@ -526,6 +581,10 @@ def ours(args):
     if rank == 0 and not args.no_131k:
         hca131 = run_hca_131k(hd, device, peaks)
         hd.hcadsa_check_device_error()
+    csa = None
+    if rank == 0 and not args.no_csa:
+        csa = run_csa(hd, device, peaks)
+        hd.hcadsa_check_device_error()
     e2e_ms, h2d, d2h = e2e_measure(hd, x, device, steps=max(2, min(args.steps, 4)))
     e2e_ms = max_over_ranks(e2e_ms, dist, device)
     e2e = {"value": job_throughput(e2e_ms, world), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
@@ -571,6 +630,7 @@ def ours(args):
         "clocks": clk,
         "decode": decode,
         "hca_131k": hca131,
+        "csa": csa,
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -680,6 +740,7 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-131k", action="store_true", help="skip the L = 131072 HCA block")
+    ap.add_argument("--no-csa", action="store_true", help="skip the CSA layer block")
     ap.add_argument("--only", choices=["compress", "hca_attn", "index_topk", "dsa_attn", "decode"],
                     help="profiling mode: run one kernel alone at --seq-len, or the decode step "
                          "(B = 32 at t = 1,048,575; --steps timed steps after 3 warm-up steps)")

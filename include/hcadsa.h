@@ -149,11 +149,15 @@ hcadsa_status hca_attn_fwd(const hcadsa_bf16* Q, const hcadsa_bf16* Kc, const hc
                            float scale, void* workspace, size_t workspace_bytes, hcadsa_stream stream);
 
 /*
- * Size in bytes of the workspace dsa_index_topk needs: the int32 indexer score rows,
- *     B * Lq * round_up(min(q_offset + Lq, Lk), 128) * 4 bytes,
- * plus, for few query rows over many keys (B*Lq <= 64, Lq < 64 and at least 32768 keys: the
- * decode shape, where the selection is spread over all SMs), per row 16 + 2048*4 + 8192*8
- * bytes of selection state (score range, histogram, candidate list).
+ * Size in bytes of the workspace dsa_index_topk needs.
+ *   - Lq >= 64 query rows per sequence (prefill, chunked prefill): B * 512 bytes -- the
+ *     per-channel min and max of k_idx.  Scoring and selection run fused on the tensor cores
+ *     and keep no score matrix, so the workspace does not grow with the sequence.
+ *   - Lq < 64 (decode shapes): the int32 indexer score rows,
+ *         B * Lq * round_up(min(q_offset + Lq, Lk), 128) * 4 bytes
+ *     (4 MiB per row at 1M keys), plus, for few query rows over many keys (B*Lq <= 64 and at
+ *     least 32768 keys, where the selection is spread over all SMs), per row 16 + 2048*4 +
+ *     8192*8 bytes of selection state (score range, histogram, candidate list).
  */
 size_t dsa_index_topk_workspace_size(int B, int Lq, int q_offset, int Lk, int k);
 
@@ -180,6 +184,32 @@ size_t dsa_index_topk_workspace_size(int B, int Lq, int q_offset, int Lk, int k)
 hcadsa_status dsa_index_topk(const int8_t* q_idx, const int8_t* k_idx, const int32_t* w_idx, int32_t* idx,
                              void* ws, size_t ws_bytes, int B, int Lq, int q_offset, int Lk, int H_idx, int d_idx,
                              int k, hcadsa_stream stream);
+
+/*
+ * CSA selection: indexer + per-query top-k over compressed entries.  Source: the mirrorspeed
+ * page, section "Hybrid sparse attention, 1/7 full context access" (and the besthub page,
+ * "Core Architectural Innovations"): the alternative the pages compare HCA + MLA against,
+ * compressed sparse attention, compresses the history 4:1 and then selects sparsely.  Reading
+ * taken (the pages give no more): entry j summarises tokens blk*j .. blk*j + blk - 1 (made by
+ * hca_compress_kv with block size blk), carries its own indexer key kc_idx[j], and becomes a
+ * candidate of the query at t once its block is complete:
+ *     candidates of t = entries j < min(floor((t + 1) / blk), n_c)      (no raw window)
+ * Scores, tie rule and output as in dsa_index_topk (entry numbers instead of positions).  The
+ * CSA layer is then hca_compress_kv(blk) -> csa_index_topk -> dsa_sparse_attn_fwd over the
+ * compressed K/V (a query with no complete block gets O = 0, lse = -inf).
+ *
+ *   q_idx  : [B, Lq, H_idx, d_idx] int8
+ *   kc_idx : [B, n_c, d_idx] int8      (one indexer key per compressed entry)
+ *   w_idx  : [H_idx] int32 (device)
+ *   idx    : [B, Lq, k] int32          (written: ascending entry numbers, -1 padded)
+ *   ws     : workspace of csa_index_topk_workspace_size(...) bytes
+ * Requirements and errors as dsa_index_topk; blk >= 1 (HCADSA_ERR_SHAPE otherwise).  With
+ * blk = 1 it is dsa_index_topk over n_c positions.
+ */
+size_t csa_index_topk_workspace_size(int B, int Lq, int q_offset, int n_c, int k, int blk);
+hcadsa_status csa_index_topk(const int8_t* q_idx, const int8_t* kc_idx, const int32_t* w_idx, int32_t* idx,
+                             void* ws, size_t ws_bytes, int B, int Lq, int q_offset, int n_c, int H_idx, int d_idx,
+                             int k, int blk, hcadsa_stream stream);
 
 /*
  * DSA indexer + top-k without any device allocation by anyone.  The pages have no

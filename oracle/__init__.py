@@ -69,6 +69,10 @@ def _load():
             lib.oracle_dsa_scores.restype = I
             lib.oracle_dsa_topk.argtypes = [P, P, P, I, I, I, I, I, I, I, P, I, P]
             lib.oracle_dsa_topk.restype = I
+            lib.oracle_csa_n_candidates.argtypes = [I, I, I]
+            lib.oracle_csa_n_candidates.restype = I
+            lib.oracle_csa_topk.argtypes = [P, P, P, I, I, I, I, I, I, I, I, P, I, P]
+            lib.oracle_csa_topk.restype = I
             lib.oracle_dsa_attn.argtypes = [P, P, P, P, I, I, I, I, I, I, D, P, I, P, P]
             lib.oracle_dsa_attn.restype = I
             lib.oracle_hca_attn_bwd.argtypes = [P, P, P, I, P, P, I, I, P, I, I, I, I, I, I, I, I, D,
@@ -189,6 +193,27 @@ def dsa_topk(q_idx, k_idx, w_idx, k, *, q_offset=0, rows=None):
     st = _load().oracle_dsa_topk(_ptr(q_idx), _ptr(k_idx), _ptr(w_idx), B, Lq, q_offset, Lk, H_idx,
                                  d_idx, k, _ptr(rows), rows.size, _ptr(out))
     _check(st, "dsa_topk")
+    return out
+
+
+def csa_n_candidates(t: int, blk: int, n_c: int) -> int:
+    return _load().oracle_csa_n_candidates(t, blk, n_c)
+
+
+def csa_topk(q_idx, kc_idx, w_idx, k, blk, *, q_offset=0, rows=None):
+    """CSA selection over compressed entries: q_idx [B,Lq,H_idx,d_idx] int8, kc_idx [B,n_c,d_idx]
+    int8 (one indexer key per entry), w_idx [H_idx] int32; the query at t sees the entries
+    j < floor((t+1)/blk).  Returns idx [n_rows, k] int32: ascending entry numbers, -1 padded."""
+    q_idx = _c(q_idx, np.int8)
+    kc_idx = _c(kc_idx, np.int8)
+    w_idx = _c(w_idx, np.int32)
+    B, Lq, H_idx, d_idx = q_idx.shape
+    n_c = kc_idx.shape[1]
+    rows = _rows(rows, B * Lq)
+    out = np.empty((rows.size, k), np.int32)
+    st = _load().oracle_csa_topk(_ptr(q_idx), _ptr(kc_idx), _ptr(w_idx), B, Lq, q_offset, n_c, H_idx, d_idx,
+                                 k, blk, _ptr(rows), rows.size, _ptr(out))
+    _check(st, "csa_topk")
     return out
 
 

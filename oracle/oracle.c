@@ -317,6 +317,61 @@ int oracle_dsa_topk(const int8_t* q_idx, const int8_t* k_idx, const int32_t* w_i
 }
 
 /* ------------------------------------------------------------------ */
+/* CSA: top-k over compressed entries                                  */
+/* ------------------------------------------------------------------ */
+
+/* [P1] "Hybrid sparse attention, 1/7 full context access" (and [P3] item 1)
+ * name the alternative the pages compare against: CSA, which compresses the
+ * history 4:1 and then selects sparsely.  Reading taken here (the pages give
+ * no more): the entries are the compressor's output for blocks of blk tokens
+ * (the HCA compressor form with a blk-long weight vector), each entry has its
+ * own indexer key, and a query at t may select entry j once the block it
+ * summarises is complete, blk*(j+1) <= t+1, i.e. j < floor((t+1)/blk).  No
+ * raw window.  Selection as in DSA: the k entries with the largest (score,
+ * -j), written ascending, -1 padded.
+ * kc_idx is [B, n_c, d_idx] (one key per entry); idx_out [n_rows, k]. */
+int oracle_csa_n_candidates(int t, int blk, int n_c) {
+  if (blk <= 0 || t < 0) return 0;
+  const int n = (t + 1) / blk;
+  return n < n_c ? n : n_c;
+}
+
+int oracle_csa_topk(const int8_t* q_idx, const int8_t* kc_idx, const int32_t* w_idx,
+                    int B, int Lq, int q_offset, int n_c, int H_idx, int d_idx, int k, int blk,
+                    const int64_t* rows, int n_rows, int32_t* idx_out) {
+  if (!q_idx || !kc_idx || !w_idx || !rows || !idx_out || k <= 0 || n_c < 0 || blk <= 0) return ORACLE_ERR_ARG;
+  int status = ORACLE_OK;
+#pragma omp parallel
+  {
+    int64_t* sc = (int64_t*)malloc(sizeof(int64_t) * (size_t)(n_c + 1));
+    scored_pos* cand = (scored_pos*)malloc(sizeof(scored_pos) * (size_t)(n_c + 1));
+#pragma omp for schedule(dynamic, 1)
+    for (int i = 0; i < n_rows; ++i) {
+      const int b = (int)(rows[i] / Lq), r = (int)(rows[i] % Lq);
+      const int n = oracle_csa_n_candidates(q_offset + r, blk, n_c);
+      if (oracle_dsa_scores(q_idx, kc_idx, w_idx, B, Lq, n_c, H_idx, d_idx, b, r, n, sc) != ORACLE_OK) {
+#pragma omp atomic write
+        status = ORACLE_ERR_RANGE;
+        continue;
+      }
+      for (int j = 0; j < n; ++j) {
+        cand[j].score = sc[j];
+        cand[j].pos = j;
+      }
+      qsort(cand, (size_t)n, sizeof(scored_pos), by_score_then_position);
+      const int keep = n < k ? n : k;
+      int32_t* out = idx_out + (long)i * k;
+      for (int m = 0; m < keep; ++m) out[m] = cand[m].pos;
+      qsort(out, (size_t)keep, sizeof(int32_t), ascending_int32);
+      for (int m = keep; m < k; ++m) out[m] = -1;
+    }
+    free(sc);
+    free(cand);
+  }
+  return status;
+}
+
+/* ------------------------------------------------------------------ */
 /* DSA sparse attention                                                */
 /* ------------------------------------------------------------------ */
 

@@ -9,6 +9,7 @@ Functions (same names as the C ABI):
     hca_compress_kv(K, V, w, blk=128)                 -> (Kc, Vc)
     hca_attn_fwd(Q, Kc, Vc, Kw, Vw, ...)              -> O  (or (O, lse))
     dsa_index_topk(q_idx, k_idx, w_idx, k, ...)       -> idx
+    csa_index_topk(q_idx, kc_idx, w_idx, k, blk, ...) -> idx (over compressed entries)
     dsa_sparse_attn_fwd(Q, K, V, idx, ...)            -> O  (or (O, lse))
     hcadsa_check_device_error()                       -> raises on a recorded device error
 """
@@ -69,6 +70,10 @@ def lib() -> ctypes.CDLL:
             L.dsa_index_topk_workspace_size.restype = S
             L.dsa_index_topk.argtypes = [P, P, P, P, P, S, I, I, I, I, I, I, I, P]
             L.dsa_index_topk.restype = I
+            L.csa_index_topk_workspace_size.argtypes = [I, I, I, I, I, I]
+            L.csa_index_topk_workspace_size.restype = S
+            L.csa_index_topk.argtypes = [P, P, P, P, P, S, I, I, I, I, I, I, I, I, P]
+            L.csa_index_topk.restype = I
             L.dsa_index_topk_noalloc_max_scratch_bytes.argtypes = []
             L.dsa_index_topk_noalloc_max_scratch_bytes.restype = S
             L.dsa_index_topk_noalloc.argtypes = [P, P, P, P, I, I, I, I, I, I, I, P]
@@ -229,6 +234,26 @@ def dsa_index_topk(q_idx, k_idx, w_idx, k: int, *, q_offset: int = 0, idx=None, 
                               workspace.numel() * workspace.element_size(), B, Lq, q_offset, Lk, H_idx,
                               d_idx, k, _stream(stream))
     _check(st, "dsa_index_topk")
+    return idx
+
+
+def csa_index_topk(q_idx, kc_idx, w_idx, k: int, blk: int = 4, *, q_offset: int = 0, idx=None, workspace=None,
+                   stream=None):
+    """q_idx: [B, Lq, 4, 64] int8; kc_idx: [B, n_c, 64] int8 (one key per compressed entry);
+    w_idx: [4] int32 -> idx [B, Lq, k] int32 (entry numbers; the query at t sees the entries of
+    complete blocks, j < (t + 1) // blk)."""
+    B, Lq, H_idx, d_idx, n_c = _check_index_args(q_idx, kc_idx, w_idx, k, idx)
+    if workspace is not None and not workspace.is_contiguous():
+        raise ValueError("workspace must be contiguous")
+    _on_device(q_idx, kc_idx, w_idx, idx, workspace)
+    idx = torch.empty((B, Lq, k), dtype=torch.int32, device=q_idx.device) if idx is None else idx
+    ws_bytes = lib().csa_index_topk_workspace_size(B, Lq, q_offset, n_c, k, blk)
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=q_idx.device)
+    st = lib().csa_index_topk(_ptr(q_idx), _ptr(kc_idx), _ptr(w_idx), _ptr(idx), _ptr(workspace),
+                              workspace.numel() * workspace.element_size(), B, Lq, q_offset, n_c, H_idx, d_idx,
+                              k, blk, _stream(stream))
+    _check(st, "csa_index_topk")
     return idx
 
 

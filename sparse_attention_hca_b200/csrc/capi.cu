@@ -37,6 +37,18 @@ int* device_error_ptr() {
 
 bool encode_tmap_bf16_swizzle(CUtensorMap* map, int rank, void* base, const uint64_t* dims,
                               const uint64_t* strides_bytes, const uint32_t* box, int swizzle_bytes) {
+  return encode_tmap_typed(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, base, dims, strides_bytes, box,
+                           swizzle_bytes);
+}
+
+bool encode_tmap_u8_swizzle(CUtensorMap* map, int rank, void* base, const uint64_t* dims,
+                            const uint64_t* strides_bytes, const uint32_t* box, int swizzle_bytes) {
+  return encode_tmap_typed(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, rank, base, dims, strides_bytes, box,
+                           swizzle_bytes);
+}
+
+bool encode_tmap_typed(CUtensorMap* map, CUtensorMapDataType dtype, int rank, void* base, const uint64_t* dims,
+                       const uint64_t* strides_bytes, const uint32_t* box, int swizzle_bytes) {
   CUtensorMapSwizzle sw;
   switch (swizzle_bytes) {
     case 0: sw = CU_TENSOR_MAP_SWIZZLE_NONE; break;
@@ -66,7 +78,7 @@ bool encode_tmap_bf16_swizzle(CUtensorMap* map, int rank, void* base, const uint
     es[i] = 1;
     if (i + 1 < rank) st[i] = strides_bytes[i];
   }
-  const CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, base, d, st, bx, es,
+  const CUresult r = g_encode(map, dtype, (cuuint32_t)rank, base, d, st, bx, es,
                               CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;

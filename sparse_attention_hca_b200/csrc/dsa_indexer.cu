@@ -48,10 +48,18 @@ constexpr int kBRow = kDIdx + 16;          // padded bytes per key row in smem
 
 __host__ __device__ inline long long round_up(long long x, long long m) { return (x + m - 1) / m * m; }
 
+// Candidates of the query at position t: keys s < min((t + 1) / ratio, Lk).  ratio = 1 is DSA
+// (every position up to and including t); ratio = blk is CSA over compressed entries (an entry
+// is a candidate once its block of blk tokens is complete).
+__host__ __device__ inline int n_cand(long long t, int ratio, int Lk) {
+  long long n = (t + 1) / ratio;
+  if (n > Lk) n = Lk;
+  return n < 0 ? 0 : (int)n;
+}
+
 // Row stride (in int32 scores) of the workspace score matrix.
-__host__ __device__ inline long long score_row_stride(int Lq, int q_offset, int Lk) {
-  long long n_max = (long long)q_offset + Lq;  // candidates of the last query
-  if (n_max > Lk) n_max = Lk;
+__host__ __device__ inline long long score_row_stride(int Lq, int q_offset, int Lk, int ratio) {
+  long long n_max = n_cand((long long)q_offset + Lq - 1, ratio, Lk);  // candidates of the last query
   if (n_max < 1) n_max = 1;
   return round_up(n_max, kKTile);
 }
@@ -66,8 +74,8 @@ struct RowSel {
   int n_cand, pad;  // candidates appended (may exceed kCandCap: overflow)
   unsigned int hist[kHistBins];
 };
-__host__ __device__ inline bool use_split_select(int B, int Lq, int q_offset, int Lk) {
-  return (long long)B * Lq <= kSplitRowsMax && Lq < 64 && score_row_stride(Lq, q_offset, Lk) >= kSplitMinKeys;
+__host__ __device__ inline bool use_split_select(int B, int Lq, int q_offset, int Lk, int ratio) {
+  return (long long)B * Lq <= kSplitRowsMax && Lq < 64 && score_row_stride(Lq, q_offset, Lk, ratio) >= kSplitMinKeys;
 }
 // bytes after the score rows: RowSel per row, then kCandCap (u, position) pairs per row
 __host__ __device__ inline long long split_select_bytes(int rows) {
@@ -212,11 +220,12 @@ __global__ void __launch_bounds__(kStreamThreads) score_stream_kernel(const int8
                                                                      const int8_t* __restrict__ k_idx,
                                                                      const int32_t* __restrict__ w_idx,
                                                                      int32_t* __restrict__ scores, int Lq,
-                                                                     int q_offset, int Lk, long long row_stride,
+                                                                     int q_offset, int Lk, int ratio,
+                                                                     long long row_stride,
                                                                      RowSel* __restrict__ rowsel) {
   const int row = blockIdx.y;
   const int b = row / Lq, r = row % Lq;
-  const int n = min(q_offset + r + 1, Lk);
+  const int n = n_cand((long long)q_offset + r, ratio, Lk);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int part = lane & 3;  // 16-byte slice of the key
   int q[kHIdx][4];
@@ -558,12 +567,12 @@ __device__ void select_row(const int* __restrict__ row_g, int* row_s, int n, int
 
 __global__ void __launch_bounds__(kSelThreads) select_kernel(const int32_t* __restrict__ scores,
                                                               int32_t* __restrict__ idx, int Lq, int q_offset,
-                                                              int Lk, int k, long long row_stride) {
+                                                              int Lk, int ratio, int k, long long row_stride) {
   extern __shared__ __align__(16) int sel_row[];
   __shared__ SelShared sh;
   const int row = blockIdx.x;
   const int r = row % Lq;
-  const int n = max(0, min(q_offset + r + 1, Lk));
+  const int n = n_cand((long long)q_offset + r, ratio, Lk);
   int32_t* out = idx + (size_t)row * k;
   if (n <= k) {
     for (int i = threadIdx.x; i < k; i += kSelThreads) out[i] = i < n ? i : -1;
@@ -599,9 +608,10 @@ __device__ __forceinline__ int hist_shift(unsigned range) {
 }
 
 __global__ void __launch_bounds__(256) hist_kernel(const int32_t* __restrict__ scores, RowSel* __restrict__ rs,
-                                                   int Lq, int q_offset, int Lk, int k, long long row_stride) {
+                                                   int Lq, int q_offset, int Lk, int ratio, int k,
+                                                   long long row_stride) {
   const int row = blockIdx.y, r = row % Lq;
-  const int n = max(0, min(q_offset + r + 1, Lk));
+  const int n = n_cand((long long)q_offset + r, ratio, Lk);
   const int c0 = blockIdx.x * kSplitChunk;
   if (n <= k || c0 >= n) return;
   __shared__ unsigned int h[kHistBins];
@@ -674,10 +684,10 @@ __device__ __forceinline__ void threshold_bin(const unsigned int* __restrict__ h
 }
 
 __global__ void __launch_bounds__(256) candidates_kernel(const int32_t* __restrict__ scores, RowSel* __restrict__ rs,
-                                                         int2* __restrict__ cand, int Lq, int q_offset, int Lk, int k,
-                                                         long long row_stride) {
+                                                         int2* __restrict__ cand, int Lq, int q_offset, int Lk,
+                                                         int ratio, int k, long long row_stride) {
   const int row = blockIdx.y, r = row % Lq;
-  const int n = max(0, min(q_offset + r + 1, Lk));
+  const int n = n_cand((long long)q_offset + r, ratio, Lk);
   const int c0 = blockIdx.x * kSplitChunk;
   if (n <= k || c0 >= n) return;
   const int tid = threadIdx.x, lane = tid & 31;
@@ -751,11 +761,11 @@ __global__ void __launch_bounds__(kSelThreads) finalize_kernel(const int32_t* __
                                                                const RowSel* __restrict__ rs,
                                                                const int2* __restrict__ cand,
                                                                int32_t* __restrict__ idx, int Lq, int q_offset,
-                                                               int Lk, int k, long long row_stride) {
+                                                               int Lk, int ratio, int k, long long row_stride) {
   extern __shared__ __align__(16) int sel_row[];
   __shared__ SelShared sh;
   const int row = blockIdx.x, r = row % Lq;
-  const int n = max(0, min(q_offset + r + 1, Lk));
+  const int n = n_cand((long long)q_offset + r, ratio, Lk);
   int32_t* out = idx + (size_t)row * k;
   if (n <= k) {
     for (int i = threadIdx.x; i < k; i += kSelThreads) out[i] = i < n ? i : -1;
@@ -809,82 +819,105 @@ __global__ void __launch_bounds__(kSelThreads) finalize_kernel(const int32_t* __
   for (int i = threadIdx.x; i < k; i += kSelThreads) out[i] = pos[i];
 }
 
+// Calls with at least this many query rows per sequence take the fused path (one CTA per 128
+// query rows); fewer rows (decode) use the streaming scorer and the score rows.
+constexpr int kFusedMinRows = 64;
+
 // int32 score rows of a call (the workspace part both entry points need)
-size_t score_rows_bytes(int B, int Lq, int q_offset, int Lk) {
-  return (size_t)B * (size_t)Lq * (size_t)score_row_stride(Lq, q_offset, Lk) * sizeof(int32_t);
+size_t score_rows_bytes(int B, int Lq, int q_offset, int Lk, int ratio) {
+  return (size_t)B * (size_t)Lq * (size_t)score_row_stride(Lq, q_offset, Lk, ratio) * sizeof(int32_t);
 }
 
-}  // namespace
-}  // namespace hcadsa
-
-extern "C" size_t dsa_index_topk_workspace_size(int B, int Lq, int q_offset, int Lk, int k) {
-  using namespace hcadsa;
-  (void)k;
-  if (B <= 0 || Lq <= 0 || Lk <= 0 || q_offset < 0) return 0;
-  size_t bytes = score_rows_bytes(B, Lq, q_offset, Lk);
-  if (use_split_select(B, Lq, q_offset, Lk)) bytes += (size_t)split_select_bytes(B * Lq);
+// Workspace of an indexer + top-k call (both the DSA and the CSA entry points).
+size_t index_topk_workspace(int B, int Lq, int q_offset, int Lk, int ratio) {
+  if (B <= 0 || Lq <= 0 || Lk <= 0 || q_offset < 0 || ratio <= 0) return 0;
+  if (Lq >= kFusedMinRows) return topk_fused_workspace_bytes(B);  // no score rows at all
+  size_t bytes = score_rows_bytes(B, Lq, q_offset, Lk, ratio);
+  if (use_split_select(B, Lq, q_offset, Lk, ratio)) bytes += (size_t)split_select_bytes(B * Lq);
   return bytes;
 }
 
-extern "C" hcadsa_status dsa_index_topk(const int8_t* q_idx, const int8_t* k_idx, const int32_t* w_idx,
-                                        int32_t* idx, void* ws, size_t ws_bytes, int B, int Lq, int q_offset,
-                                        int Lk, int H_idx, int d_idx, int k, hcadsa_stream stream) {
-  using namespace hcadsa;
+// Indexer + top-k with candidates s < min((t + 1) / ratio, Lk) for the query at t.
+hcadsa_status index_topk(const int8_t* q_idx, const int8_t* k_idx, const int32_t* w_idx, int32_t* idx, void* ws,
+                         size_t ws_bytes, int B, int Lq, int q_offset, int Lk, int H_idx, int d_idx, int k,
+                         int ratio, hcadsa_stream stream) {
   if (!q_idx || !k_idx || !w_idx || !idx) return HCADSA_ERR_NULL;
-  if (B < 0 || Lq < 0 || Lk < 0 || q_offset < 0 || k <= 0) return HCADSA_ERR_SHAPE;
+  if (B < 0 || Lq < 0 || Lk < 0 || q_offset < 0 || k <= 0 || ratio <= 0) return HCADSA_ERR_SHAPE;
   if (H_idx != kHIdx || d_idx != kDIdx || k > 4096) return HCADSA_ERR_UNSUPPORTED;
   if ((long long)q_offset + Lq > 2147483647LL - 1 || (long long)B * Lq > 2147483647LL) return HCADSA_ERR_UNSUPPORTED;
   if (!aligned16(q_idx) || !aligned16(k_idx) || !aligned16(w_idx) || !aligned16(idx)) return HCADSA_ERR_ALIGN;
   if (B == 0 || Lq == 0) return HCADSA_OK;
   cudaStream_t s = as_stream(stream);
-  const bool need_scores = (long long)q_offset + Lq > k && Lk > k;  // some row has more than k candidates
-  const long long stride = score_row_stride(Lq, q_offset, Lk);
-  const bool split = need_scores && use_split_select(B, Lq, q_offset, Lk);
-  const int rows = B * Lq;
-  RowSel* rowsel = split ? reinterpret_cast<RowSel*>(static_cast<char*>(ws) + score_rows_bytes(B, Lq, q_offset, Lk))
-                         : nullptr;
-  int2* cand = split ? reinterpret_cast<int2*>(rowsel + rows) : nullptr;
+  // some row has more than k candidates
+  const bool need_scores = Lk > 0 && n_cand((long long)q_offset + Lq - 1, ratio, Lk) > k;
   if (need_scores) {
     if (!ws) return HCADSA_ERR_WORKSPACE;
     if (!aligned16(ws)) return HCADSA_ERR_ALIGN;
-    if (ws_bytes < dsa_index_topk_workspace_size(B, Lq, q_offset, Lk, k)) return HCADSA_ERR_WORKSPACE;
+    if (ws_bytes < index_topk_workspace(B, Lq, q_offset, Lk, ratio)) return HCADSA_ERR_WORKSPACE;
+  }
+  if (need_scores && Lq >= kFusedMinRows)  // many query rows: the fused tensor-core path (dsa_topk_tc.cu)
+    return launch_topk_fused(q_idx, k_idx, w_idx, idx, ws, B, Lq, q_offset, Lk, k, ratio, s);
+  const long long stride = score_row_stride(Lq, q_offset, Lk, ratio);
+  const bool split = need_scores && use_split_select(B, Lq, q_offset, Lk, ratio);
+  const int rows = B * Lq;
+  RowSel* rowsel =
+      split ? reinterpret_cast<RowSel*>(static_cast<char*>(ws) + score_rows_bytes(B, Lq, q_offset, Lk, ratio))
+            : nullptr;
+  int2* cand = split ? reinterpret_cast<int2*>(rowsel + rows) : nullptr;
+  if (need_scores) {
     int32_t* scores = static_cast<int32_t*>(ws);
     if (split) rowsel_init_kernel<<<(unsigned)(B * Lq), 256, 0, s>>>(rowsel);
-    if (Lq >= 64) {
-      const long long n_max = stride;
-      dim3 grid((unsigned)((n_max + kKeyTilesPerCta * kKTile - 1) / (kKeyTilesPerCta * kKTile)),
-                (unsigned)((Lq + kQTile - 1) / kQTile), (unsigned)B);
-      if (grid.y > 65535u || grid.z > 65535u) return HCADSA_ERR_UNSUPPORTED;
-      const int smem_tiled = kQTile * kARow + 2 * kKTile * kBRow;
-      if (cudaFuncSetAttribute(score_tiled_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_tiled) !=
-          cudaSuccess)
-        return HCADSA_ERR_CUDA;
-      score_tiled_kernel<<<grid, 256, smem_tiled, s>>>(q_idx, k_idx, w_idx, scores, Lq, q_offset, Lk, stride);
-    } else {
-      const long long n_max = stride;
-      dim3 grid((unsigned)((n_max + kStreamKeysPerCta - 1) / kStreamKeysPerCta), (unsigned)(B * Lq));
-      if (grid.y > 65535u) return HCADSA_ERR_UNSUPPORTED;
-      score_stream_kernel<<<grid, kStreamThreads, 0, s>>>(q_idx, k_idx, w_idx, scores, Lq, q_offset, Lk, stride,
-                                                           rowsel);
-    }
+    dim3 grid((unsigned)((stride + kStreamKeysPerCta - 1) / kStreamKeysPerCta), (unsigned)(B * Lq));
+    if (grid.y > 65535u) return HCADSA_ERR_UNSUPPORTED;
+    score_stream_kernel<<<grid, kStreamThreads, 0, s>>>(q_idx, k_idx, w_idx, scores, Lq, q_offset, Lk, ratio, stride,
+                                                         rowsel);
     if (cudaGetLastError() != cudaSuccess) return HCADSA_ERR_CUDA;
   }
   const int smem = kSelSmemCap * (int)sizeof(int);
   if (split) {
     int32_t* scores = static_cast<int32_t*>(ws);
     const dim3 grid((unsigned)((stride + kSplitChunk - 1) / kSplitChunk), (unsigned)rows);
-    hist_kernel<<<grid, 256, 0, s>>>(scores, rowsel, Lq, q_offset, Lk, k, stride);
-    candidates_kernel<<<grid, 256, 0, s>>>(scores, rowsel, cand, Lq, q_offset, Lk, k, stride);
+    hist_kernel<<<grid, 256, 0, s>>>(scores, rowsel, Lq, q_offset, Lk, ratio, k, stride);
+    candidates_kernel<<<grid, 256, 0, s>>>(scores, rowsel, cand, Lq, q_offset, Lk, ratio, k, stride);
     if (cudaFuncSetAttribute(finalize_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
       return HCADSA_ERR_CUDA;
-    finalize_kernel<<<(unsigned)rows, kSelThreads, smem, s>>>(scores, rowsel, cand, idx, Lq, q_offset, Lk, k, stride);
+    finalize_kernel<<<(unsigned)rows, kSelThreads, smem, s>>>(scores, rowsel, cand, idx, Lq, q_offset, Lk, ratio, k,
+                                                              stride);
     return launch_status();
   }
   if (cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return HCADSA_ERR_CUDA;
   select_kernel<<<(unsigned)(B * Lq), kSelThreads, smem, s>>>(need_scores ? static_cast<int32_t*>(ws) : nullptr,
-                                                              idx, Lq, q_offset, Lk, k, stride);
+                                                              idx, Lq, q_offset, Lk, ratio, k, stride);
   return launch_status();
+}
+
+}  // namespace
+}  // namespace hcadsa
+
+extern "C" size_t dsa_index_topk_workspace_size(int B, int Lq, int q_offset, int Lk, int k) {
+  (void)k;
+  return hcadsa::index_topk_workspace(B, Lq, q_offset, Lk, 1);
+}
+
+extern "C" hcadsa_status dsa_index_topk(const int8_t* q_idx, const int8_t* k_idx, const int32_t* w_idx,
+                                        int32_t* idx, void* ws, size_t ws_bytes, int B, int Lq, int q_offset,
+                                        int Lk, int H_idx, int d_idx, int k, hcadsa_stream stream) {
+  return hcadsa::index_topk(q_idx, k_idx, w_idx, idx, ws, ws_bytes, B, Lq, q_offset, Lk, H_idx, d_idx, k, 1, stream);
+}
+
+extern "C" size_t csa_index_topk_workspace_size(int B, int Lq, int q_offset, int n_c, int k, int blk) {
+  (void)k;
+  if (blk <= 0) return 0;
+  return hcadsa::index_topk_workspace(B, Lq, q_offset, n_c, blk);
+}
+
+extern "C" hcadsa_status csa_index_topk(const int8_t* q_idx, const int8_t* kc_idx, const int32_t* w_idx,
+                                        int32_t* idx, void* ws, size_t ws_bytes, int B, int Lq, int q_offset,
+                                        int n_c, int H_idx, int d_idx, int k, int blk, hcadsa_stream stream) {
+  if (blk <= 0) return HCADSA_ERR_SHAPE;
+  return hcadsa::index_topk(q_idx, kc_idx, w_idx, idx, ws, ws_bytes, B, Lq, q_offset, n_c, H_idx, d_idx, k, blk,
+                            stream);
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -933,9 +966,9 @@ extern "C" hcadsa_status dsa_index_topk_noalloc(const int8_t* q_idx, const int8_
   if (!aligned16(q_idx) || !aligned16(k_idx) || !aligned16(w_idx) || !aligned16(idx)) return HCADSA_ERR_ALIGN;
   if (B == 0 || Lq == 0) return HCADSA_OK;
   const bool need_scores = (long long)q_offset + Lq > k && Lk > k;
-  const long long stride = score_row_stride(Lq, q_offset, Lk);
+  const long long stride = score_row_stride(Lq, q_offset, Lk, 1);
   // size check first: a call that does not fit is refused before any CUDA call
-  if (need_scores && score_rows_bytes(B, Lq, q_offset, Lk) > kNoAllocScratchBytes) return HCADSA_ERR_WORKSPACE;
+  if (need_scores && score_rows_bytes(B, Lq, q_offset, Lk, 1) > kNoAllocScratchBytes) return HCADSA_ERR_WORKSPACE;
   cudaStream_t s = as_stream(stream);
   int32_t* scores = nullptr;
   if (need_scores) {
@@ -953,7 +986,7 @@ extern "C" hcadsa_status dsa_index_topk_noalloc(const int8_t* q_idx, const int8_
     } else {
       dim3 grid((unsigned)((stride + kStreamKeysPerCta - 1) / kStreamKeysPerCta), (unsigned)(B * Lq));
       if (grid.y > 65535u) return HCADSA_ERR_UNSUPPORTED;
-      score_stream_kernel<<<grid, kStreamThreads, 0, s>>>(q_idx, k_idx, w_idx, scores, Lq, q_offset, Lk, stride,
+      score_stream_kernel<<<grid, kStreamThreads, 0, s>>>(q_idx, k_idx, w_idx, scores, Lq, q_offset, Lk, 1, stride,
                                                            nullptr);
     }
     if (cudaGetLastError() != cudaSuccess) return HCADSA_ERR_CUDA;
@@ -961,6 +994,6 @@ extern "C" hcadsa_status dsa_index_topk_noalloc(const int8_t* q_idx, const int8_
   const int smem = kSelSmemCap * (int)sizeof(int);
   if (cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return HCADSA_ERR_CUDA;
-  select_kernel<<<(unsigned)(B * Lq), kSelThreads, smem, s>>>(scores, idx, Lq, q_offset, Lk, k, stride);
+  select_kernel<<<(unsigned)(B * Lq), kSelThreads, smem, s>>>(scores, idx, Lq, q_offset, Lk, 1, k, stride);
   return launch_status();
 }

@@ -5,7 +5,8 @@
 // page -- only say that 128 tokens become one entry).
 //
 // The work is a pure HBM stream.  Persistent CTAs walk work units (tensor, batch, block,
-// 256-channel column group).  One thread streams each unit's rows into a 3-stage ring of
+// 256-channel column group; for blocks shorter than 128 tokens a unit takes 128 / blk
+// consecutive blocks, so a box is never mostly unused).  One thread streams each unit's rows into a 3-stage ring of
 // shared-memory boxes (TMA, up to 128 rows x 256 channels = 64 KB per box) so plenty of
 // bytes are in flight per SM; four warps then run the sequential FMA chains from shared
 // memory, two channels per thread, rows in ascending order -- exactly the fixed
@@ -34,6 +35,8 @@ struct Params {
   uint16_t* Vc;
   int* err;
   int B, L, row_elems, n_c, blk, col_groups, n_units;
+  int bpu;       // blocks per unit: 128 / blk consecutive blocks share one 128-row box when blk < 128
+  int n_groups;  // block groups per batch: ceil(n_c / bpu)
 };
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -65,8 +68,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int cg = u % p.col_groups;
         const int rest = u / p.col_groups;
         const int tensor = rest & 1;
-        const int bj = rest >> 1;  // b * n_c + j
-        const int b = bj / p.n_c, j = bj % p.n_c;
+        const int bg = rest >> 1;  // b * n_groups + block group
+        const int b = bg / p.n_groups, j = (bg % p.n_groups) * p.bpu;  // first block of the unit
         const int row0 = b * p.L + j * p.blk;
         for (int bx = 0; bx < boxes_per_unit; ++bx, ++q) {
           const uint32_t st = q % kStages;
@@ -86,7 +89,31 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int cg = u % p.col_groups;
     const int rest = u / p.col_groups;
     const int tensor = rest & 1;
-    const int bj = rest >> 1;
+    const int bg = rest >> 1;
+    const int b = bg / p.n_groups, j0 = (bg % p.n_groups) * p.bpu;
+    const int gcol = cg * kCols + col;
+    uint16_t* dst_base = (tensor ? p.Vc : p.Kc) + (size_t)b * p.n_c * p.row_elems + gcol;
+    if (p.bpu > 1) {
+      // one box holds bpu whole blocks: each block's chain over its blk rows, in order
+      const uint32_t st = q % kStages;
+      if (!mbar_wait(&full[st], (q / kStages) & 1, &abort_flag, p.err)) return;
+      const uint32_t* box = reinterpret_cast<const uint32_t*>(ring + st * kBoxBytes) + threadIdx.x;
+      const int nb = min(p.bpu, p.n_c - j0);
+      for (int jj = 0; jj < nb; ++jj) {
+        float a0 = 0.0f, a1 = 0.0f;
+        const uint32_t* rows = box + jj * p.blk * (kCols / 2);
+        for (int i = 0; i < p.blk; ++i) {
+          const uint32_t x = rows[i * (kCols / 2)];
+          a0 = fmaf(sw[i], __uint_as_float(x << 16), a0);
+          a1 = fmaf(sw[i], __uint_as_float(x & 0xFFFF0000u), a1);
+        }
+        if (gcol < p.row_elems)
+          *reinterpret_cast<uint32_t*>(dst_base + (size_t)(j0 + jj) * p.row_elems) = pack_bf16x2(a0, a1);
+      }
+      mbar_arrive(&empty[st]);
+      ++q;
+      continue;
+    }
     float a0 = 0.0f, a1 = 0.0f;
     for (int bx = 0; bx < boxes_per_unit; ++bx, ++q) {
       const uint32_t st = q % kStages;
@@ -102,11 +129,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       mbar_arrive(&empty[st]);
     }
-    const int gcol = cg * kCols + col;
-    if (gcol < p.row_elems) {
-      uint16_t* dst = (tensor ? p.Vc : p.Kc) + (size_t)bj * p.row_elems + gcol;
-      *reinterpret_cast<uint32_t*>(dst) = pack_bf16x2(a0, a1);
-    }
+    if (gcol < p.row_elems) *reinterpret_cast<uint32_t*>(dst_base + (size_t)j0 * p.row_elems) = pack_bf16x2(a0, a1);
   }
 }
 
@@ -139,7 +162,10 @@ extern "C" hcadsa_status hca_compress_kv(const hcadsa_bf16* K, const hcadsa_bf16
   const long long rows = (long long)B * L;
   if (row_elems > (1LL << 24) || rows > 2147483647LL) return HCADSA_ERR_UNSUPPORTED;
   const long long col_groups = (row_elems + kCols - 1) / kCols;
-  const long long n_units = 2LL * B * n_c * col_groups;
+  // short blocks (blk < 128) are batched: 128 / blk consecutive blocks per 128-row box
+  const int bpu = blk < kBoxRows ? kBoxRows / blk : 1;
+  const long long n_groups = (n_c + bpu - 1) / bpu;
+  const long long n_units = 2LL * B * n_groups * col_groups;
   if (n_units > 2147483647LL) return HCADSA_ERR_UNSUPPORTED;
   // [rows, row_elems] bf16, box = 128 rows x 256 channels, no swizzle; box parts past the last
   // row or the last channel are zero-filled and never stored
@@ -161,6 +187,8 @@ extern "C" hcadsa_status hca_compress_kv(const hcadsa_bf16* K, const hcadsa_bf16
   p.blk = blk;
   p.col_groups = (int)col_groups;
   p.n_units = (int)n_units;
+  p.bpu = bpu;
+  p.n_groups = (int)n_groups;
   if (cudaFuncSetAttribute(hca_compress_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) !=
       cudaSuccess)
     return HCADSA_ERR_CUDA;

@@ -28,6 +28,21 @@ bool encode_tmap_bf16(CUtensorMap* map, int rank, void* base, const uint64_t* di
 bool encode_tmap_bf16_swizzle(CUtensorMap* map, int rank, void* base, const uint64_t* dims,
                               const uint64_t* strides_bytes, const uint32_t* box, int swizzle_bytes);
 
+// Same for 8-bit integer tensors (element = 1 byte), and for any driver data type.
+bool encode_tmap_u8_swizzle(CUtensorMap* map, int rank, void* base, const uint64_t* dims,
+                            const uint64_t* strides_bytes, const uint32_t* box, int swizzle_bytes);
+bool encode_tmap_typed(CUtensorMap* map, CUtensorMapDataType dtype, int rank, void* base, const uint64_t* dims,
+                       const uint64_t* strides_bytes, const uint32_t* box, int swizzle_bytes);
+
+// Indexer + exact top-k of many query rows in one fused kernel (dsa_topk_tc.cu): scores on the
+// int8 tensor cores, selection by per-row histograms, no score matrix.  Candidates of the query
+// at position t are the keys s < min((t + 1) / ratio, Lk).  `kstat` is workspace for
+// topk_fused_workspace_bytes(B) bytes.  Enqueues on `s`; returns a status before launch.
+size_t topk_fused_workspace_bytes(int B);
+hcadsa_status launch_topk_fused(const int8_t* q_idx, const int8_t* k_idx, const int32_t* w_idx, int32_t* idx,
+                                void* kstat, int B, int Lq, int q_offset, int Lk, int k, int ratio,
+                                cudaStream_t s);
+
 // Records the message of a failed CUDA call for hcadsa_last_error_string().
 void record_cuda_error(cudaError_t e);
 

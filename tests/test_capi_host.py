@@ -98,7 +98,12 @@ def test_dsa_argument_errors(lib):
 
 
 def test_workspace_size_queries(lib):
-    assert lib.dsa_index_topk_workspace_size(1, 32768, 0, 32768, 2048) == 32768 * 32768 * 4
+    # 64 or more query rows per sequence: the fused indexer + selection keeps no score rows, only
+    # the per-channel min / max of k_idx (2 x 64 int32 per sequence) -- at 32K as at 131K
+    assert lib.dsa_index_topk_workspace_size(1, 32768, 0, 32768, 2048) == 2 * 64 * 4
+    assert lib.dsa_index_topk_workspace_size(3, 131072, 0, 131072, 2048) == 3 * 2 * 64 * 4
+    # fewer rows (decode shapes) keep their int32 score rows: 63 rows over 5000 keys
+    assert lib.dsa_index_topk_workspace_size(1, 63, 4937, 5000, 2048) == 63 * 5120 * 4
     # few rows over many keys add the multi-CTA selection state: per row 16 bytes + a 2048-bin
     # histogram + 8192 (score, position) candidates
     assert lib.dsa_index_topk_workspace_size(2, 1, 1048575, 1048576, 2048) == 2 * 1048576 * 4 + 2 * (

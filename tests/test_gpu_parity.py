@@ -428,6 +428,37 @@ def test_topk_32k_sampled_rows(hd):
     assert np.array_equal(got, ref)
 
 
+def test_topk_131k_sampled_rows(hd):
+    """The long-context prefill length through the fused indexer + selection (no score matrix:
+    the workspace is 512 bytes), bit-exact on sampled rows."""
+    cfg = synth.DsaConfig("topk131k", B=1, L=131072, Hq=64)
+    g = torch.Generator().manual_seed(131)
+    q = torch.randint(-8, 9, (1, cfg.L, 4, 64), generator=g).to(torch.int8)
+    kk = torch.randint(-8, 9, (1, cfg.L, 64), generator=g).to(torch.int8)
+    w = torch.tensor([2, 4, 1, 3], dtype=torch.int32)
+    assert hd.dsa_index_topk_workspace_size(1, cfg.L, 0, cfg.L, cfg.k) == 512
+    idx = hd.dsa_index_topk(q.cuda(), kk.cuda(), w.cuda(), cfg.k)
+    no_device_error(hd)
+    rows = _sample_rows(cfg.L, extra=(2047, 2048, 65535, 65536, 100000, 131071))
+    ref = oracle.dsa_topk(q.numpy(), kk.numpy(), w.numpy(), cfg.k, rows=rows)
+    got = idx.reshape(cfg.L, cfg.k)[torch.as_tensor(rows, device="cuda")].cpu().numpy()
+    assert np.array_equal(got, ref)
+
+
+def test_topk_ragged_batches_offset_odd_k(hd):
+    """Three sequences, 300 query rows each at positions 1000..1299 (a ragged last tile of 44
+    rows), k = 77 (rows not 16-byte aligned: scalar stores), bit-exact on every row."""
+    B, Lq, t0, k = 3, 300, 1000, 77
+    g = torch.Generator().manual_seed(77)
+    q = torch.randint(-8, 9, (B, Lq, 4, 64), generator=g).to(torch.int8)
+    kk = torch.randint(-8, 9, (B, t0 + Lq, 64), generator=g).to(torch.int8)
+    w = torch.tensor([1, 3, 2, 4], dtype=torch.int32)
+    idx = hd.dsa_index_topk(q.cuda(), kk.cuda(), w.cuda(), k, q_offset=t0)
+    no_device_error(hd)
+    ref = oracle.dsa_topk(q.numpy(), kk.numpy(), w.numpy(), k, q_offset=t0)
+    assert np.array_equal(idx.cpu().numpy().reshape(B * Lq, k), ref)
+
+
 # ------------------------------------------------------------------ DSA sparse attention
 
 def _dsa_attn_case(hd, cfg, rows):

@@ -341,6 +341,86 @@ def test_dsa_topk_decode_offset_equals_prefill_row(oracle_mod):
     assert np.array_equal(pre, dec)
 
 
+# ---------------------------------------------------------------- CSA (top-k over compressed entries)
+
+@pytest.mark.parametrize("blk", [1, 4, 7])
+def test_csa_candidates_match_block_completion_enumeration(oracle_mod, blk):
+    """Entry j (tokens blk*j .. blk*j + blk - 1) is a candidate of the query at t exactly when its
+    last token is at or before t; the stored entries cap the count."""
+    for n_c in (3, 1000):
+        for t in range(200):
+            want = sum(1 for j in range(n_c) if blk * j + blk - 1 <= t)
+            assert oracle_mod.csa_n_candidates(t, blk, n_c) == want
+
+
+@pytest.mark.parametrize("blk,k", [(4, 1), (4, 9), (3, 30)])
+def test_csa_topk_matches_brute_force_sort_over_complete_blocks(oracle_mod, blk, k):
+    B, L, H_idx, d_idx = 2, 90, 2, 3
+    n_c = L // blk
+    g = torch.Generator().manual_seed(211 + blk + k)
+    q = torch.randint(-1, 2, (B, L, H_idx, d_idx), generator=g).to(torch.int8).numpy()
+    kc = torch.randint(-1, 2, (B, n_c, d_idx), generator=g).to(torch.int8).numpy()
+    w = np.array([2, 1], np.int32)
+    idx = oracle_mod.csa_topk(q, kc, w, k, blk)
+    sc = np.einsum("j,btjc,bsc->bts", w.astype(np.int64), q.astype(np.int64), kc.astype(np.int64))
+    for b in range(B):
+        for t in range(L):
+            n = min((t + 1) // blk, n_c)
+            assert idx[b * L + t].tolist() == _brute_topk(sc[b, t, :n], k)
+
+
+def test_csa_with_block_one_is_dsa(oracle_mod):
+    """blk = 1 makes every position its own entry: the CSA candidates are DSA's (0 .. t)."""
+    inp = _dsa_small(2, 120, 1, 8, 213)
+    q, kk, w = inp["q_idx"].numpy(), inp["k_idx"].numpy(), inp["w_idx"].numpy()
+    assert np.array_equal(oracle_mod.csa_topk(q, kk, w, 17, 1), oracle_mod.dsa_topk(q, kk, w, 17))
+    assert np.array_equal(oracle_mod.csa_topk(q[:, 100:], kk, w, 17, 1, q_offset=100),
+                          oracle_mod.dsa_topk(q[:, 100:], kk, w, 17, q_offset=100))
+
+
+def test_csa_layer_with_identity_compressor_and_large_k_is_dense_causal(oracle_mod):
+    """The whole CSA chain -- compress (blk = 1, w = [1]), select over complete blocks with
+    k >= L, attend over the selected entries -- is dense causal attention (torch fp64 SDPA)."""
+    B, L, Hq, d = 1, 40, 4, 16
+    inp = _dsa_small(B, L, Hq, d, 215)
+    K4 = bits(inp["K"]).reshape(B, L, 1, d)
+    V4 = bits(inp["V"]).reshape(B, L, 1, d)
+    one = np.ones(1, np.float32)
+    Kc = oracle_mod.hca_compress(K4, one, 1).reshape(B, L, d)
+    Vc = oracle_mod.hca_compress(V4, one, 1).reshape(B, L, d)
+    idx = oracle_mod.csa_topk(inp["q_idx"].numpy(), inp["k_idx"].numpy(), inp["w_idx"].numpy(), 64, 1)
+    O = oracle_mod.dsa_attn(bits(inp["Q"]), Kc, Vc, idx, scale=0.25)
+    ref = sdpa_ref(inp["Q"], inp["K"].unsqueeze(2), inp["V"].unsqueeze(2),
+                   torch.ones(L, L, dtype=torch.bool).tril(), 0.25).reshape(B * L, Hq, d)
+    np.testing.assert_allclose(O, ref, rtol=0, atol=1e-12)
+
+
+def test_csa_attention_over_4to1_entries_matches_masked_sdpa(oracle_mod):
+    """4:1 entries, top-5 of the complete blocks: attention over the selected entries equals SDPA
+    over the compressed keys with the selection as the mask (a query with no complete block sees
+    nothing: O = 0)."""
+    B, L, Hq, d, blk, k = 1, 64, 2, 16, 4, 5
+    n_c = L // blk
+    inp = _dsa_small(B, L, Hq, d, 217)
+    w4 = np.array([0.125, 0.25, 0.375, 0.25], np.float32)
+    Kc = oracle_mod.hca_compress(bits(inp["K"]).reshape(B, L, 1, d), w4, blk).reshape(B, n_c, d)
+    Vc = oracle_mod.hca_compress(bits(inp["V"]).reshape(B, L, 1, d), w4, blk).reshape(B, n_c, d)
+    kc_idx = torch.randint(-8, 9, (B, n_c, 64), generator=torch.Generator().manual_seed(219)).to(torch.int8)
+    idx = oracle_mod.csa_topk(inp["q_idx"].numpy(), kc_idx.numpy(), inp["w_idx"].numpy(), k, blk)
+    O = oracle_mod.dsa_attn(bits(inp["Q"]), Kc, Vc, idx, scale=0.25)
+    mask = torch.zeros(L, n_c, dtype=torch.bool)
+    for t in range(L):
+        for j in idx[t]:
+            if j >= 0:
+                assert blk * j + blk - 1 <= t
+                mask[t, j] = True
+    Kt, Vt = from_bits(Kc).view(B, n_c, 1, d), from_bits(Vc).view(B, n_c, 1, d)
+    seen = mask.any(1)
+    ref = sdpa_ref(inp["Q"][:, seen], Kt, Vt, mask[seen], 0.25).reshape(-1, Hq, d)
+    np.testing.assert_allclose(O[seen.numpy()], ref, rtol=0, atol=1e-12)
+    assert np.all(O[~seen.numpy()] == 0.0) and (~seen).sum() == blk - 1
+
+
 # ---------------------------------------------------------------- DSA attention
 
 def test_dsa_attention_with_large_k_is_dense_causal(oracle_mod):
