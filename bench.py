@@ -393,6 +393,78 @@ def run_csa(hd, device, peaks, iters=10):
             "algorithmic_flop": flop, "layer_tokens_per_s": Lc / (sum(ms) * 1e-3)}
 
 
+def run_gate_vha(hd, device, peaks, iters=10, H=16, dv=512, rq=1024, r=4):
+    """The fused output gate + virtual-head mix on the HCA layer's output (L = 32768, 16 heads of
+    512, query latent 1024, mix rank 4): a tensor-core GEMM (M = tokens, N = H * dv, K = rq) with
+    the epilogue reading O and writing Y.  CUDA events, median of `iters` after 3 warm-up runs."""
+    d = _Draw(device, synth.SEED)
+    O = d.normal((1, L, H, dv), 0.05, 41)
+    cq = d.normal((1, L, rq), 1.0, 42)
+    Wg = d.normal((H * dv, rq), 1 / math.sqrt(rq), 43)
+    U = d.uniform(H * r, 0.5, 44).view(H, r) - 0.25
+    V = d.uniform(H * r, 0.5, 45).view(H, r) - 0.25
+    Y = torch.empty_like(O)
+    for _ in range(3):
+        hd.attn_gate_vha_fwd(O, cq, Wg, U, V, Y=Y)
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(iters)]
+    for i in range(iters):
+        evs[i][0].record()
+        hd.attn_gate_vha_fwd(O, cq, Wg, U, V, Y=Y)
+        evs[i][1].record()
+    torch.cuda.synchronize()
+    ms = statistics.median(e[0].elapsed_time(e[1]) for e in evs)
+    flop = 2.0 * L * H * dv * rq
+    hbm = 2 * (2 * L * H * dv) + 2 * L * rq + 2 * H * dv * rq
+    tf = flop / (ms * 1e-3) / 1e12
+    del O, cq, Wg, Y
+    torch.cuda.empty_cache()
+    return {"workload": f"gate_vha_L{L}_h{H}_dv{dv}_rq{rq}_r{r} (B=1)", "iters": iters, "ms": ms,
+            "tflops": tf, "pct_bf16": 100 * tf / peaks["bf16_tflops"], "gbs": hbm / (ms * 1e-3) / 1e9,
+            "pct_hbm": 100 * hbm / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], "algorithmic_flop": flop,
+            "algorithmic_bytes": hbm}
+
+
+def run_hca_latent(hd, device, peaks, iters=10):
+    """HCA layer prefill with FlashMask-4's head shape (qk 576 / v 512, values = the latent part of
+    the keys) at L = 32768, 16 query heads on one K/V head: compression of the 576-wide keys and
+    the attention, CUDA events, median of `iters` after 3 warm-up runs."""
+    dqk, dv = 576, 512
+    d = _Draw(device, synth.SEED)
+    sh = 1 / math.sqrt(dqk)
+    Q = d.normal((1, L, HCA.Hq, dqk), sh, 51)
+    K = d.normal((1, L, HCA.Hkv, dqk), sh, 52)
+    w = d.uniform(HCA.blk, 2.0 / HCA.blk, 54)
+    Kc = torch.empty((1, L // 128, 1, dqk), dtype=torch.bfloat16, device=device)
+    O = torch.empty((1, L, HCA.Hq, dv), dtype=torch.bfloat16, device=device)
+    nb = hd.lib().hca_attn_fwd_latent_workspace_size(1, L, 0, HCA.Hq, HCA.Hkv, dqk, dv, L // 128, 128, 128)
+    ws = torch.empty(max(nb, 16), dtype=torch.uint8, device=device)
+
+    def step(ev=None):
+        if ev: ev[0].record()
+        hd.hca_compress_kv(K, K, w, 128, Kc=Kc, Vc=Kc)
+        if ev: ev[1].record()
+        hd.hca_attn_fwd_latent(Q, Kc, K, O=O, workspace=ws)
+        if ev: ev[2].record()
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(iters)]
+    for i in range(iters):
+        step(evs[i])
+    torch.cuda.synchronize()
+    comp_ms = statistics.median(e[0].elapsed_time(e[1]) for e in evs)
+    attn_ms = statistics.median(e[1].elapsed_time(e[2]) for e in evs)
+    flop = 2.0 * (dqk + dv) * HCA.Hq * hca_visible_keys_per_head(L)
+    tf = flop / (attn_ms * 1e-3) / 1e12
+    del Q, K, O, ws
+    torch.cuda.empty_cache()
+    return {"workload": f"hca_prefill_L{L}_hq16_hkv1_dqk576_dv512 (B=1, values = latent part of the keys)",
+            "iters": iters, "compress_us": comp_ms * 1e3, "attn_ms": attn_ms, "attn_tflops": tf,
+            "attn_pct_bf16": 100 * tf / peaks["bf16_tflops"], "algorithmic_flop": flop}
+
+
 def run_hca_131k(hd, device, peaks, iters=10):
     """The HCA long-context prefill configuration (B = 1, L = 131072, 16 query heads on one K/V
     head, d = 512, 1024 compressed entries): compression and attention timed with CUDA events
@@ -585,6 +657,14 @@ def ours(args):
     if rank == 0 and not args.no_csa:
         csa = run_csa(hd, device, peaks)
         hd.hcadsa_check_device_error()
+    gate = None
+    if rank == 0 and not args.no_gate:
+        gate = run_gate_vha(hd, device, peaks)
+        hd.hcadsa_check_device_error()
+    latent = None
+    if rank == 0 and not args.no_latent:
+        latent = run_hca_latent(hd, device, peaks)
+        hd.hcadsa_check_device_error()
     e2e_ms, h2d, d2h = e2e_measure(hd, x, device, steps=max(2, min(args.steps, 4)))
     e2e_ms = max_over_ranks(e2e_ms, dist, device)
     e2e = {"value": job_throughput(e2e_ms, world), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
@@ -631,6 +711,8 @@ def ours(args):
         "decode": decode,
         "hca_131k": hca131,
         "csa": csa,
+        "gate_vha": gate,
+        "hca_latent_576": latent,
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -677,7 +759,9 @@ def reference(args):
 def only_kernel(args):
     """Runs one library kernel alone at sequence length --seq-len (profiling mode): W warm-up
     and K timed launches; prints a small JSON record (not the benchmark contract line).
-    --only decode runs the decode step instead."""
+    --only decode runs the decode step instead; --only csa / gate_vha the CSA layer / the output
+    gate block at --seq-len."""
+    global L
     import sparse_attention_hca_b200 as hd
 
     if args.only == "decode":
@@ -685,12 +769,17 @@ def only_kernel(args):
         hd.hcadsa_check_device_error()
         print(json.dumps(out))
         return
+    if args.only in ("csa", "gate_vha", "hca_latent"):
+        L = args.seq_len
+        run = {"csa": run_csa, "gate_vha": run_gate_vha, "hca_latent": run_hca_latent}[args.only]
+        out = run(hd, torch.device("cuda", 0), load_peaks(), iters=max(1, args.steps))
+        hd.hcadsa_check_device_error()
+        print(json.dumps(out))
+        return
 
-    global L
     L = args.seq_len
     device = torch.device("cuda", 0)
-    # only the selected kernel's layer is allocated (a profiled launch should hold a few GB at
-    # most; the top-k score workspace alone is 4 L^2 bytes)
+    # only the selected kernel's layer is allocated (a profiled launch should hold a few GB at most)
     if args.only in ("compress", "hca_attn"):
         x = make_hca_inputs(device, seed=synth.SEED)
         Kc = torch.empty((1, L // 128, 1, HCA.d), dtype=torch.bfloat16, device=device)
@@ -741,7 +830,10 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-131k", action="store_true", help="skip the L = 131072 HCA block")
     ap.add_argument("--no-csa", action="store_true", help="skip the CSA layer block")
-    ap.add_argument("--only", choices=["compress", "hca_attn", "index_topk", "dsa_attn", "decode"],
+    ap.add_argument("--no-gate", action="store_true", help="skip the output gate + head mix block")
+    ap.add_argument("--no-latent", action="store_true", help="skip the qk 576 / v 512 HCA block")
+    ap.add_argument("--only", choices=["compress", "hca_attn", "index_topk", "dsa_attn", "decode", "csa", "gate_vha",
+                                       "hca_latent"],
                     help="profiling mode: run one kernel alone at --seq-len, or the decode step "
                          "(B = 32 at t = 1,048,575; --steps timed steps after 3 warm-up steps)")
     ap.add_argument("--seq-len", type=int, default=L)

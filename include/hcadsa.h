@@ -149,6 +149,28 @@ hcadsa_status hca_attn_fwd(const hcadsa_bf16* Q, const hcadsa_bf16* Kc, const hc
                            float scale, void* workspace, size_t workspace_bytes, hcadsa_stream stream);
 
 /*
+ * HCA attention with FlashMask-4's head shape: 576-wide scores, 512-wide values.  Source: the
+ * mirrorspeed page, section "More structural improvements, data, and infrastructure", and the
+ * ai-club.cn article, section "训练：Muon 优化器 + 自研注意力算子" (an attention operator for
+ * qk_head_dim 576 / v_head_dim 512, meant for HCA's 512-wide heads).  Reading taken (MLA-style
+ * shared latent): a key row is 576 wide -- the 512-wide latent and a 64-wide positional slice --
+ * and the value of a key is the first 512 columns of the same row, so the caches hold one
+ * tensor per part (entries Kc, raw window Kw) and no separate V.  Visible set, softmax, lse,
+ * layouts of Q/O/lse, workspace rules and errors as hca_attn_fwd, with
+ *   Q      : [B, Lq, Hq, 576] bf16         scores use all 576 columns
+ *   Kc, Kw : [B, n_c | n_w, Hkv, 576] bf16 (Kc may be NULL iff n_c == 0)
+ *   O      : [B, Lq, Hq, 512] bf16
+ * Requirements: dqk == 576, dv == 512 (HCADSA_ERR_UNSUPPORTED otherwise).  scale is usually
+ * 1/sqrt(576).  The workspace size is that of hca_attn_fwd with d = 512.
+ */
+size_t hca_attn_fwd_latent_workspace_size(int B, int Lq, int q_offset, int Hq, int Hkv, int dqk, int dv, int n_c,
+                                          int blk, int W);
+hcadsa_status hca_attn_fwd_latent(const hcadsa_bf16* Q, const hcadsa_bf16* Kc, int n_c, const hcadsa_bf16* Kw,
+                                  int win_start, int n_w, hcadsa_bf16* O, float* lse, int B, int Lq, int q_offset,
+                                  int Hq, int Hkv, int dqk, int dv, int blk, int W, float scale, void* workspace,
+                                  size_t workspace_bytes, hcadsa_stream stream);
+
+/*
  * Size in bytes of the workspace dsa_index_topk needs.
  *   - Lq >= 64 query rows per sequence (prefill, chunked prefill): B * 512 bytes -- the
  *     per-channel min and max of k_idx.  Scoring and selection run fused on the tensor cores
@@ -254,6 +276,54 @@ hcadsa_status dsa_index_topk_noalloc(const int8_t* q_idx, const int8_t* k_idx, c
 hcadsa_status dsa_sparse_attn_fwd(const hcadsa_bf16* Q, const hcadsa_bf16* K, const hcadsa_bf16* V,
                                   const int32_t* idx, hcadsa_bf16* O, float* lse, int B, int Lq, int Lk, int Hq,
                                   int d, int k, float scale, hcadsa_stream stream);
+
+/*
+ * Attention output gate + virtual-head mix, fused (tensor-core GEMM + epilogue).  Source: the
+ * mirrorspeed page, section "Hybrid sparse attention, 1/7 full context access" (last
+ * paragraph), and the besthub page, "Core Architectural Innovations": low-rank gated attention
+ * computes the output gate from the layer's low-rank query latent (a quarter of the hidden
+ * width); virtual head attention (VHA) mixes the heads with a light low-rank term beside an
+ * identity path and can be folded into the attention operator at inference.  Reading taken
+ * (the pages give no formulas): elementwise gate, mix applied per token and channel before it:
+ *     Ohat[t,h,c] = O[t,h,c] + sum_{m<r} U[h,m] * sum_h' V[h',m] * O[t,h',c]
+ *     Y[t,h,c]    = sigmoid(sum_i cq[t,i] * Wg[h*dv + c, i]) * Ohat[t,h,c]
+ *
+ *   O  : [B, L, H, dv] bf16   attention output (hca_attn_fwd / dsa_sparse_attn_fwd)
+ *   cq : [B, L, rq] bf16      low-rank query latent
+ *   Wg : [H*dv, rq] bf16      gate projection (row h*dv + c: head h, channel c)
+ *   U, V: [H, r] fp32 (device; may be NULL iff r == 0)
+ *   Y  : [B, L, H, dv] bf16   (written; must not alias O)
+ * Requirements: H in {16, 32, 64} (HCA: 16 heads of 512, DSA: 64 heads of 256); dv a multiple of
+ * 256 / H and of 8; rq a multiple of 64; 0 <= r <= 4.  HCADSA_ERR_UNSUPPORTED otherwise.
+ */
+hcadsa_status attn_gate_vha_fwd(const hcadsa_bf16* O, const hcadsa_bf16* cq, const hcadsa_bf16* Wg, const float* U,
+                                const float* V, hcadsa_bf16* Y, int B, int L, int H, int dv, int rq, int r,
+                                hcadsa_stream stream);
+
+/* ------------------------------------------------------------------ backward pass */
+
+/*
+ * Backward of the HCA compressor.  Source: the sections cited for hca_compress_kv (one cache
+ * entry per block of tokens); with the compressor form fixed there the map is linear,
+ *     Xc[b, j, h, c] = sum_i w[i] * X[b, blk*j + i, h, c],
+ * and its adjoint, for a gradient dXc of the entries, is
+ *     dX[b, blk*j + i, h, c] += w[i] * dXc[b, j, h, c]       (tail tokens past the last
+ *                                                              complete block get nothing)
+ *     dw[i]                  += sum_{b, j, h, c} dXc[b, j, h, c] * X[b, blk*j + i, h, c]
+ * (the bf16 rounding of the forward is not differentiated).  Both outputs are ADDED to, so the
+ * compressor's share of a key or value gradient can be added to the share of the raw window;
+ * zero them first for the compressor's share alone.  dw is summed with fp32 atomics (order not
+ * fixed: results can differ in the last bits between runs).
+ *
+ *   X   : [B, L, H, d] bf16       (the forward input, K or V)
+ *   w   : [blk] fp32
+ *   dXc : [B, L/blk, H, d] fp32
+ *   dX  : [B, L, H, d] fp32       (accumulated)
+ *   dw  : [blk] fp32              (accumulated)
+ * Requirements: d a multiple of 8, 1 <= blk <= 1024; X, dXc, dX 16-byte aligned.
+ */
+hcadsa_status hca_compress_bwd(const hcadsa_bf16* X, const float* w, const float* dXc, float* dX, float* dw, int B,
+                               int L, int H, int d, int blk, hcadsa_stream stream);
 
 #ifdef __cplusplus
 }

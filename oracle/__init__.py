@@ -65,6 +65,8 @@ def _load():
             lib.oracle_hca_attn.argtypes = [P, P, P, I, P, P, I, I, I, I, I, I, I, I, I, I,
                                             D, P, I, P, P]
             lib.oracle_hca_attn.restype = I
+            lib.oracle_hca_attn_latent.argtypes = [P, P, I, P, I, I, I, I, I, I, I, I, I, I, I, D, P, I, P, P]
+            lib.oracle_hca_attn_latent.restype = I
             lib.oracle_dsa_scores.argtypes = [P, P, P, I, I, I, I, I, I, I, I, P]
             lib.oracle_dsa_scores.restype = I
             lib.oracle_dsa_topk.argtypes = [P, P, P, I, I, I, I, I, I, I, P, I, P]
@@ -74,6 +76,8 @@ def _load():
             lib.oracle_csa_topk.argtypes = [P, P, P, I, I, I, I, I, I, I, I, P, I, P]
             lib.oracle_csa_topk.restype = I
             lib.oracle_dsa_attn.argtypes = [P, P, P, P, I, I, I, I, I, I, D, P, I, P, P]
+            lib.oracle_gate_vha.argtypes = [P, P, P, P, P, I, I, I, I, I, I, P]
+            lib.oracle_gate_vha.restype = I
             lib.oracle_dsa_attn.restype = I
             lib.oracle_hca_attn_bwd.argtypes = [P, P, P, I, P, P, I, I, P, I, I, I, I, I, I, I, I, D,
                                                 P, P, P, P, P]
@@ -166,6 +170,31 @@ def hca_attn(Q, Kc, Vc, Kw, Vw, *, win_start=0, q_offset=0, blk=128, W=128, scal
     return (O, lse) if with_lse else O
 
 
+def hca_attn_latent(Q, Kc, Kw, dv, *, win_start=0, q_offset=0, blk=128, W=128, scale=None, rows=None,
+                    with_lse=False):
+    """HCA attention with a shared latent: Q [B,Lq,Hq,dqk], Kc [B,n_c,Hkv,dqk] (or None), Kw
+    [B,n_w,Hkv,dqk] bf16 bits; the value of a key is the first dv columns of its row.  Returns O
+    [n_rows, Hq, dv] fp64 (and lse [n_rows, Hq])."""
+    Q = _c(Q, np.uint16)
+    Kw = _c(Kw, np.uint16)
+    B, Lq, Hq, dqk = Q.shape
+    n_w, Hkv = Kw.shape[1], Kw.shape[2]
+    if Kc is None or Kc.shape[1] == 0:
+        n_c, Kc_ = 0, None
+    else:
+        Kc_ = _c(Kc, np.uint16)
+        n_c = Kc_.shape[1]
+    if scale is None:
+        scale = float(np.float32(1.0 / np.sqrt(dqk)))
+    rows = _rows(rows, B * Lq)
+    O = np.empty((rows.size, Hq, dv), np.float64)
+    lse = np.empty((rows.size, Hq), np.float64) if with_lse else None
+    st = _load().oracle_hca_attn_latent(_ptr(Q), _ptr(Kc_), n_c, _ptr(Kw), win_start, n_w, B, Lq, q_offset, Hq, Hkv,
+                                        dqk, dv, blk, W, float(scale), _ptr(rows), rows.size, _ptr(O), _ptr(lse))
+    _check(st, "hca_attn_latent")
+    return (O, lse) if with_lse else O
+
+
 def dsa_scores(q_idx, k_idx, w_idx, b, r, n):
     q_idx = _c(q_idx, np.int8)
     k_idx = _c(k_idx, np.int8)
@@ -237,6 +266,28 @@ def dsa_attn(Q, K, V, idx_rows, *, scale=None, rows=None, with_lse=False):
                                  float(scale), _ptr(rows), rows.size, _ptr(O), _ptr(lse))
     _check(st, "dsa_attn")
     return (O, lse) if with_lse else O
+
+
+def gate_vha(O, cq, Wg, U, V):
+    """Attention epilogue: Y = sigmoid(cq . Wg^T) * (O + U (V^T O)) per token, channel by channel.
+
+    O [B,L,H,dv], cq [B,L,rq], Wg [H*dv, rq] (bf16 bits); U, V [H, r] fp32 (r may be 0).
+    Returns Y [B,L,H,dv] fp64."""
+    O = _c(O, np.uint16)
+    cq = _c(cq, np.uint16)
+    Wg = _c(Wg, np.uint16)
+    B, L, H, dv = O.shape
+    rq = cq.shape[-1]
+    assert cq.shape == (B, L, rq) and Wg.shape == (H * dv, rq)
+    U = _c(U, np.float32).reshape(H, -1)
+    V = _c(V, np.float32).reshape(H, -1)
+    r = U.shape[1]
+    assert V.shape == (H, r)
+    Y = np.empty((B, L, H, dv), np.float64)
+    st = _load().oracle_gate_vha(_ptr(O), _ptr(cq), _ptr(Wg), _ptr(U) if r else None, _ptr(V) if r else None,
+                                 B, L, H, dv, rq, r, _ptr(Y))
+    _check(st, "gate_vha")
+    return Y
 
 
 # ---------------------------------------------------------------- backward pass

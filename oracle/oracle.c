@@ -227,6 +227,74 @@ int oracle_hca_attn(const uint16_t* Q, const uint16_t* Kc, const uint16_t* Vc, i
   return status;
 }
 
+/* HCA attention with FlashMask-4's head shape ([P1] "More structural improvements, data, and
+ * infrastructure"; [P5] "训练：Muon 优化器 + 自研注意力算子": qk head dim 576, v head dim 512, for
+ * HCA's 512-wide heads).  Reading taken (MLA-style shared latent): a key row is dqk wide
+ * (the dv-wide latent plus a dqk - dv positional slice), and the value of a key is the first dv
+ * columns of the same row -- one cache tensor per part (entries Kc, window Kw), no separate V.
+ * Visible set, softmax and scale as oracle_hca_attn; scores over dqk, outputs over dv.
+ * O is [n_rows, Hq, dv] fp64; lse (nullable) [n_rows, Hq]. */
+int oracle_hca_attn_latent(const uint16_t* Q, const uint16_t* Kc, int n_c, const uint16_t* Kw, int win_start,
+                           int n_w, int B, int Lq, int q_offset, int Hq, int Hkv, int dqk, int dv, int blk, int W,
+                           double scale, const int64_t* rows, int n_rows, double* O, double* lse) {
+  if (!Q || !Kw || !rows || !O || Hq <= 0 || Hkv <= 0 || Hq % Hkv || dqk <= 0 || dv <= 0 || dv > dqk || blk <= 0 ||
+      W <= 0)
+    return ORACLE_ERR_ARG;
+  if (n_c > 0 && !Kc) return ORACLE_ERR_ARG;
+  const int group = Hq / Hkv;
+  int status = ORACLE_OK;
+#pragma omp parallel
+  {
+    const int max_keys = n_c + n_w;
+    const uint16_t** keys = (const uint16_t**)malloc(sizeof(void*) * (size_t)(max_keys + 1));
+    double* s_buf = (double*)malloc(sizeof(double) * (size_t)(max_keys + 1));
+#pragma omp for schedule(dynamic, 1)
+    for (int i = 0; i < n_rows; ++i) {
+      const int64_t flat = rows[i];
+      const int b = (int)(flat / Lq), r = (int)(flat % Lq);
+      const int t = q_offset + r;
+      const int ws = oracle_hca_window_start(t, W);
+      const int nc_t = oracle_hca_n_compressed(t, W, blk);
+      if (b < 0 || b >= B || nc_t > n_c || ws < win_start || t - win_start >= n_w) {
+#pragma omp atomic write
+        status = ORACLE_ERR_RANGE;
+        continue;
+      }
+      for (int h = 0; h < Hq; ++h) {
+        const int hk = h / group;
+        int n = 0;
+        for (int j = 0; j < nc_t; ++j) keys[n++] = Kc + (((long)b * n_c + j) * Hkv + hk) * (long)dqk;
+        for (int s = ws; s <= t; ++s) keys[n++] = Kw + (((long)b * n_w + (s - win_start)) * Hkv + hk) * (long)dqk;
+        const uint16_t* q = Q + (((long)b * Lq + r) * Hq + h) * (long)dqk;
+        double* out = O + ((long)i * Hq + h) * dv;
+        for (int c = 0; c < dv; ++c) out[c] = 0.0;
+        if (n == 0) {
+          if (lse) lse[(long)i * Hq + h] = -INFINITY;
+          continue;
+        }
+        double m = -INFINITY;
+        for (int e = 0; e < n; ++e) {
+          double dot = 0.0;
+          for (int c = 0; c < dqk; ++c) dot += (double)bf16_bits_to_float(q[c]) * (double)bf16_bits_to_float(keys[e][c]);
+          s_buf[e] = scale * dot;
+          if (s_buf[e] > m) m = s_buf[e];
+        }
+        double l = 0.0;
+        for (int e = 0; e < n; ++e) {
+          const double pe = exp(s_buf[e] - m);
+          l += pe;
+          for (int c = 0; c < dv; ++c) out[c] += pe * (double)bf16_bits_to_float(keys[e][c]);  // value = first dv columns
+        }
+        for (int c = 0; c < dv; ++c) out[c] /= l;
+        if (lse) lse[(long)i * Hq + h] = m + log(l);
+      }
+    }
+    free(keys);
+    free(s_buf);
+  }
+  return status;
+}
+
 /* ------------------------------------------------------------------ */
 /* DSA lightning indexer                                               */
 /* ------------------------------------------------------------------ */
@@ -421,6 +489,55 @@ int oracle_dsa_attn(const uint16_t* Q, const uint16_t* K, const uint16_t* V, con
     free(s_buf);
   }
   return status;
+}
+
+/* ------------------------------------------------------------------ */
+/* Output gate + virtual-head mix (the attention epilogue)              */
+/* ------------------------------------------------------------------ */
+
+/* [P1] "Hybrid sparse attention, 1/7 full context access", last paragraph, and
+ * [P3] "Core Architectural Innovations" (low-rank gated attention, VHA): the
+ * output gate is computed from the layer's low-rank query latent (a quarter of
+ * the hidden width), and VHA mixes the heads with a light low-rank term on top
+ * of an identity path.  Readings taken (the pages give no formulas): the gate
+ * is elementwise per head and channel, Z = c_q . W_g^T, and VHA acts on the
+ * attention output of one token, channel by channel, before the gate:
+ *   Ohat[t,h,c] = O[t,h,c] + sum_m U[h,m] sum_h' V[h',m] O[t,h',c]
+ *   Z[t,h,c]    = sum_i cq[t,i] Wg[h*dv + c, i]
+ *   Y[t,h,c]    = sigmoid(Z[t,h,c]) * Ohat[t,h,c]
+ * O [B,L,H,dv], cq [B,L,rq], Wg [H*dv, rq] bf16; U, V [H, r] fp32; Y fp64
+ * [B,L,H,dv].  Rows t are independent; OpenMP over them. */
+int oracle_gate_vha(const uint16_t* O, const uint16_t* cq, const uint16_t* Wg, const float* U, const float* V,
+                    int B, int L, int H, int dv, int rq, int r, double* Y) {
+  if (!O || !cq || !Wg || !Y || B < 0 || L < 0 || H <= 0 || dv <= 0 || rq <= 0 || r < 0 || (r > 0 && (!U || !V)))
+    return ORACLE_ERR_ARG;
+  const long rows = (long)B * L;
+#pragma omp parallel
+  {
+    double* proj = (double*)malloc(sizeof(double) * (size_t)(r > 0 ? r : 1) * (size_t)dv);
+#pragma omp for schedule(static)
+    for (long t = 0; t < rows; ++t) {
+      const uint16_t* o = O + t * (long)H * dv;
+      const uint16_t* q = cq + t * (long)rq;
+      for (int m = 0; m < r; ++m)
+        for (int c = 0; c < dv; ++c) {
+          double acc = 0.0;
+          for (int h2 = 0; h2 < H; ++h2) acc += (double)V[h2 * r + m] * (double)bf16_bits_to_float(o[h2 * dv + c]);
+          proj[m * dv + c] = acc;
+        }
+      for (int h = 0; h < H; ++h)
+        for (int c = 0; c < dv; ++c) {
+          double ohat = (double)bf16_bits_to_float(o[h * dv + c]);
+          for (int m = 0; m < r; ++m) ohat += (double)U[h * r + m] * proj[m * dv + c];
+          const uint16_t* wrow = Wg + ((long)h * dv + c) * rq;
+          double z = 0.0;
+          for (int i = 0; i < rq; ++i) z += (double)bf16_bits_to_float(q[i]) * (double)bf16_bits_to_float(wrow[i]);
+          Y[(t * H + h) * (long)dv + c] = ohat / (1.0 + exp(-z));
+        }
+    }
+    free(proj);
+  }
+  return ORACLE_OK;
 }
 
 /* ================================================================== */

@@ -8,9 +8,11 @@ tensors are not on a CUDA device, the calls raise.
 Functions (same names as the C ABI):
     hca_compress_kv(K, V, w, blk=128)                 -> (Kc, Vc)
     hca_attn_fwd(Q, Kc, Vc, Kw, Vw, ...)              -> O  (or (O, lse))
+    hca_attn_fwd_latent(Q, Kc, Kw, ...)               -> O  (qk 576 / v 512, values = latent part of K)
     dsa_index_topk(q_idx, k_idx, w_idx, k, ...)       -> idx
     csa_index_topk(q_idx, kc_idx, w_idx, k, blk, ...) -> idx (over compressed entries)
     dsa_sparse_attn_fwd(Q, K, V, idx, ...)            -> O  (or (O, lse))
+    attn_gate_vha_fwd(O, cq, Wg, U, V)                -> Y (output gate + virtual-head mix)
     hcadsa_check_device_error()                       -> raises on a recorded device error
 """
 from __future__ import annotations
@@ -66,6 +68,10 @@ def lib() -> ctypes.CDLL:
             L.hca_attn_fwd_workspace_size.restype = S
             L.hca_attn_fwd.argtypes = [P, P, P, I, P, P, I, I, P, P, I, I, I, I, I, I, I, I, F, P, S, P]
             L.hca_attn_fwd.restype = I
+            L.hca_attn_fwd_latent_workspace_size.argtypes = [I] * 10
+            L.hca_attn_fwd_latent_workspace_size.restype = S
+            L.hca_attn_fwd_latent.argtypes = [P, P, I, P, I, I, P, P, I, I, I, I, I, I, I, I, I, F, P, S, P]
+            L.hca_attn_fwd_latent.restype = I
             L.dsa_index_topk_workspace_size.argtypes = [I, I, I, I, I]
             L.dsa_index_topk_workspace_size.restype = S
             L.dsa_index_topk.argtypes = [P, P, P, P, P, S, I, I, I, I, I, I, I, P]
@@ -80,6 +86,10 @@ def lib() -> ctypes.CDLL:
             L.dsa_index_topk_noalloc.restype = I
             L.dsa_sparse_attn_fwd.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, F, P]
             L.dsa_sparse_attn_fwd.restype = I
+            L.attn_gate_vha_fwd.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, P]
+            L.attn_gate_vha_fwd.restype = I
+            L.hca_compress_bwd.argtypes = [P, P, P, P, P, I, I, I, I, I, P]
+            L.hca_compress_bwd.restype = I
             _lib = L
     return _lib
 
@@ -201,6 +211,46 @@ def hca_attn_fwd(Q, Kc, Vc, Kw, Vw, *, win_start: int = 0, q_offset: int = 0, bl
     return (O, lse) if return_lse else O
 
 
+def hca_attn_fwd_latent(Q, Kc, Kw, *, dv: int = 512, win_start: int = 0, q_offset: int = 0, blk: int = 128,
+                        W: int = 128, scale: float | None = None, O=None, lse=None, return_lse=False,
+                        workspace=None, stream=None):
+    """FlashMask-4's head shape: Q [B, Lq, Hq, 576]; Kc [B, n_c, Hkv, 576] (or None); Kw [B, n_w,
+    Hkv, 576]; the value of a key is the first dv = 512 columns of its row -> O [B, Lq, Hq, 512]."""
+    _need(Q, torch.bfloat16, "Q")
+    B, Lq, Hq, dqk = Q.shape
+    _need(Kw, torch.bfloat16, "Kw")
+    if Kw.dim() != 4 or Kw.shape[0] != B or Kw.shape[3] != dqk:
+        raise ValueError(f"Kw has shape {tuple(Kw.shape)}, expected [{B}, n_w, Hkv, {dqk}]")
+    n_w, Hkv = Kw.shape[1], Kw.shape[2]
+    n_c = 0 if Kc is None else Kc.shape[1]
+    if n_c:
+        _need(Kc, torch.bfloat16, "Kc", (B, n_c, Hkv, dqk))
+    if O is not None:
+        _need(O, torch.bfloat16, "O", (B, Lq, Hq, dv))
+    if lse is not None:
+        _need(lse, torch.float32, "lse", (B, Lq, Hq))
+    if workspace is not None and not workspace.is_contiguous():
+        raise ValueError("workspace must be contiguous")
+    _on_device(Q, Kw, Kc if n_c else None, O, lse, workspace)
+    if scale is None:
+        scale = 1.0 / math.sqrt(dqk)
+    O = torch.empty((B, Lq, Hq, dv), dtype=torch.bfloat16, device=Q.device) if O is None else O
+    if return_lse and lse is None:
+        lse = torch.empty((B, Lq, Hq), dtype=torch.float32, device=Q.device)
+    L = lib()
+    ws_bytes = L.hca_attn_fwd_latent_workspace_size(B, Lq, q_offset, Hq, Hkv, dqk, dv, n_c, blk, W)
+    if workspace is None:
+        if ws_bytes:
+            workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=Q.device)
+    else:
+        ws_bytes = workspace.numel() * workspace.element_size()
+    st = L.hca_attn_fwd_latent(_ptr(Q), _ptr(Kc) if n_c else None, n_c, _ptr(Kw), win_start, n_w, _ptr(O), _ptr(lse),
+                               B, Lq, q_offset, Hq, Hkv, dqk, dv, blk, W, float(scale), _ptr(workspace), ws_bytes,
+                               _stream(stream))
+    _check(st, "hca_attn_fwd_latent")
+    return (O, lse) if return_lse else O
+
+
 def dsa_index_topk_workspace_size(B, Lq, q_offset, Lk, k) -> int:
     return lib().dsa_index_topk_workspace_size(B, Lq, q_offset, Lk, k)
 
@@ -299,3 +349,51 @@ def dsa_sparse_attn_fwd(Q, K, V, idx, *, scale: float | None = None, O=None, lse
                                    Hq, d, k, float(scale), _stream(stream))
     _check(st, "dsa_sparse_attn_fwd")
     return (O, lse) if return_lse else O
+
+
+def attn_gate_vha_fwd(O, cq, Wg, U=None, V=None, *, Y=None, stream=None):
+    """O: [B, L, H, dv] bf16; cq: [B, L, rq] bf16; Wg: [H*dv, rq] bf16; U, V: [H, r] fp32 (or None)
+    -> Y = sigmoid(cq Wg^T) * (O + U (V^T O)) per token, [B, L, H, dv] bf16."""
+    _need(O, torch.bfloat16, "O")
+    B, L, H, dv = O.shape
+    _need(cq, torch.bfloat16, "cq")
+    if cq.dim() != 3 or cq.shape[0] != B or cq.shape[1] != L:
+        raise ValueError(f"cq has shape {tuple(cq.shape)}, expected [{B}, {L}, rq]")
+    rq = cq.shape[2]
+    _need(Wg, torch.bfloat16, "Wg", (H * dv, rq))
+    r = 0
+    if U is not None or V is not None:
+        if U is None or V is None:
+            raise ValueError("U and V go together")
+        _need(U, torch.float32, "U")
+        if U.dim() != 2 or U.shape[0] != H:
+            raise ValueError(f"U has shape {tuple(U.shape)}, expected [{H}, r]")
+        r = U.shape[1]
+        _need(V, torch.float32, "V", (H, r))
+    if Y is not None:
+        _need(Y, torch.bfloat16, "Y", O.shape)
+    _on_device(O, cq, Wg, U, V, Y)
+    Y = torch.empty_like(O) if Y is None else Y
+    st = lib().attn_gate_vha_fwd(_ptr(O), _ptr(cq), _ptr(Wg), _ptr(U) if r else None, _ptr(V) if r else None,
+                                 _ptr(Y), B, L, H, dv, rq, r, _stream(stream))
+    _check(st, "attn_gate_vha_fwd")
+    return Y
+
+
+def hca_compress_bwd(X, w, dXc, blk: int = 128, *, dX=None, dw=None, stream=None):
+    """Adjoint of hca_compress_kv: X [B, L, H, d] bf16, w [blk] fp32, dXc [B, L//blk, H, d] fp32 ->
+    (dX [B, L, H, d] fp32, dw [blk] fp32), both added to when given (zeros otherwise)."""
+    _need(X, torch.bfloat16, "X")
+    B, L, H, d = X.shape
+    _need(w, torch.float32, "w", (blk,))
+    _need(dXc, torch.float32, "dXc", (B, L // blk, H, d))
+    if dX is not None:
+        _need(dX, torch.float32, "dX", X.shape)
+    if dw is not None:
+        _need(dw, torch.float32, "dw", (blk,))
+    _on_device(X, w, dXc, dX, dw)
+    dX = torch.zeros(X.shape, dtype=torch.float32, device=X.device) if dX is None else dX
+    dw = torch.zeros(blk, dtype=torch.float32, device=X.device) if dw is None else dw
+    st = lib().hca_compress_bwd(_ptr(X), _ptr(w), _ptr(dXc), _ptr(dX), _ptr(dw), B, L, H, d, blk, _stream(stream))
+    _check(st, "hca_compress_bwd")
+    return dX, dw

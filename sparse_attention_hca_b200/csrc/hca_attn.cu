@@ -56,7 +56,7 @@
 namespace hcadsa {
 namespace {
 
-constexpr int kD = 512;
+constexpr int kD = 512;      // value width (and score width of the standard head shape)
 constexpr int kDHalf = 256;
 constexpr int kKeyTile = 128;
 constexpr int kSmallRows = 32;  // TMA box height for key tiles of at most 32 keys
@@ -69,17 +69,33 @@ constexpr int kGroups = 2;
 constexpr int kMaxGroups = 3;
 constexpr int kChunkBytes = 128 * 128;  // 128 rows x 64 bf16
 constexpr int kSmallChunkBytes = kSmallRows * 128;
-constexpr int kQChunks = kD / 64;      // 8
 constexpr int kVChunks = kDHalf / 64;  // 4
 constexpr int kVRows = 64;             // keys per V ring group (4 chunks of 64 keys x 64 columns)
 constexpr int kVChunkBytes = kVRows * 128;
-constexpr int kQBytes = kQChunks * kChunkBytes;
 constexpr int kOutCols = 32;                  // O columns per TMA store box
 constexpr int kOutBufBytes = 128 * kOutCols * 2;  // 8 KB
-constexpr int kOutBufs = 4;                       // staging: 128 columns of O in four boxes
 constexpr int kGroupBytes = 2 * kChunkBytes;
-constexpr int kSmemBytes = kQBytes + kMaxGroups * kGroupBytes + 1024;
-static_assert(kGroups * kGroupBytes + kOutBufs * kOutBufBytes <= kMaxGroups * kGroupBytes, "staging fits the third group");
+
+// Shared-memory plan per score width DQK (the value width is always 512):
+//   DQK = 512: Q 128 KB + two ring groups + a third 32 KB region that is the epilogue's staging
+//              (four 32-column boxes = 128 columns of O per round) or, with split key ranges, a
+//              third ring group.
+//   DQK = 576 (FlashMask-4's qk 576 / v 512 shape: 512-wide latent + 64-wide positional slice):
+//              Q 144 KB + two ring groups + a 16 KB staging area (two boxes = 64 columns per
+//              round); split key ranges keep two ring groups.  225 KB either way.
+template <int DQK>
+struct Shape {
+  static constexpr int kQChunks = DQK / 64;           // 8 or 9 chunks of 64 score columns
+  static constexpr int kQBytes = kQChunks * kChunkBytes;
+  static constexpr int kOutBufs = DQK == 512 ? 4 : 2;  // staging boxes per round
+  static constexpr int kMaxGroups = DQK == 512 ? 3 : 2;
+  static constexpr int kExtraBytes = DQK == 512 ? kGroupBytes : kOutBufs * kOutBufBytes;
+  static constexpr int kSmemBytes = kQBytes + kGroups * kGroupBytes + kExtraBytes + 1024;
+  static_assert(DQK == 512 || DQK == 576, "score width");
+  static_assert(kOutBufs * kOutBufBytes <= kExtraBytes, "staging fits its region");
+  static_assert((kMaxGroups - kGroups) * kGroupBytes <= kExtraBytes, "split-mode ring group fits");
+  static_assert(kSmemBytes <= 227 * 1024, "shared memory");
+};
 constexpr int kThreads = 320;
 constexpr int kSoftmaxWarp0 = 2;   // warps 2-5: softmax and P reloads
 constexpr int kEpilogueWarp0 = 6;  // warps 6-9: O read-out and stores
@@ -318,7 +334,13 @@ __device__ __forceinline__ void rescale_o(uint32_t t_row, float alpha) {
   tmem_wait_st();
 }
 
+template <int DQK>
 __global__ void __launch_bounds__(kThreads, 1) hca_attn_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Params p) {
+  using S = Shape<DQK>;
+  constexpr int kQChunks = S::kQChunks;
+  constexpr int kQBytes = S::kQBytes;
+  constexpr int kOutBufs = S::kOutBufs;
+  constexpr int kMaxGroups = S::kMaxGroups;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;
@@ -376,14 +398,15 @@ __global__ void __launch_bounds__(kThreads, 1) hca_attn_kernel(const __grid_cons
           gph ^= 1;
         }
       };
-      // K: all rows of key tile kt x columns col .. col+127 (two 16 KB chunks) into the next group
-      auto load_k = [&](const KeyTile& kt, int col, int hk, int b) {
+      // K: all rows of key tile kt x columns col .. col + 64 nch - 1 (nch = 2 16 KB chunks, or 1 for
+      // the last, odd chunk of a 576-wide score) into the next group
+      auto load_k = [&](const KeyTile& kt, int col, int hk, int b, int nch) {
         ok = mbar_wait(&bar.empty[grp], gph ^ 1, &abort_flag, p.err);
         if (ok) {
           uint8_t* dst = sRing + grp * kGroupBytes;
           if (kt.kind == 2) {  // 16 window rows, then 112 entry rows: both boxes fill the chunk
-            mbar_arrive_expect_tx(&bar.full[grp], 2 * kChunkBytes);
-            for (int cc = 0; cc < 2; ++cc) {
+            mbar_arrive_expect_tx(&bar.full[grp], nch * kChunkBytes);
+            for (int cc = 0; cc < nch; ++cc) {
               tma_load_4d(dst + cc * kChunkBytes, &maps.kmerge[0], &bar.full[grp], col + cc * 64, hk,
                           kt.wstart - p.win_start, b);
               tma_load_4d(dst + cc * kChunkBytes + kMergeWinRows * 128, &maps.kmerge[1], &bar.full[grp],
@@ -393,9 +416,9 @@ __global__ void __launch_bounds__(kThreads, 1) hca_attn_kernel(const __grid_cons
             const int small = kt.n <= kSmallRows ? 1 : 0;
             const CUtensorMap* m = &maps.k[kt.kind][small];
             const int row0 = kt.kind ? kt.start - p.win_start : kt.start;
-            mbar_arrive_expect_tx(&bar.full[grp], 2 * (small ? kSmallChunkBytes : kChunkBytes));
+            mbar_arrive_expect_tx(&bar.full[grp], nch * (small ? kSmallChunkBytes : kChunkBytes));
             tma_load_4d(dst, m, &bar.full[grp], col, hk, row0, b);
-            tma_load_4d(dst + kChunkBytes, m, &bar.full[grp], col + 64, hk, row0, b);
+            if (nch == 2) tma_load_4d(dst + kChunkBytes, m, &bar.full[grp], col + 64, hk, row0, b);
           }
         }
         next_group();
@@ -448,7 +471,7 @@ __global__ void __launch_bounds__(kThreads, 1) hca_attn_kernel(const __grid_cons
         for (int step = 0; ok && step <= ts.J; ++step) {
           if (step < ts.J) {
             const KeyTile kt = ts.get(step);
-            for (int c = 0; ok && c < kQChunks; c += 2) load_k(kt, c * 64, ts.hk, ts.b);
+            for (int c = 0; ok && c < kQChunks; c += 2) load_k(kt, c * 64, ts.hk, ts.b, kQChunks - c >= 2 ? 2 : 1);
           }
           if (ok && step >= 1) load_v(ts, step - 1, 0);
         }
@@ -541,11 +564,13 @@ __global__ void __launch_bounds__(kThreads, 1) hca_attn_kernel(const __grid_cons
               const uint64_t da = dq0 + (uint64_t)((c * kChunkBytes) >> 4);
               const uint64_t db = dk0 + grp * kGroupDesc;
 #pragma unroll
-              for (int cc = 0; cc < 2; ++cc)
+              for (int cc = 0; cc < 2; ++cc) {
+                if (kQChunks % 2 == 1 && c + cc >= kQChunks) break;  // the odd last chunk (576 wide)
 #pragma unroll
                 for (int k = 0; k < 4; ++k)
                   mma_ss(tS, da + (uint64_t)((cc * kChunkBytes + k * 32) >> 4),
                          db + (uint64_t)((cc * kChunkBytes + k * 32) >> 4), idesc, (c | cc | k) != 0);
+              }
               mma_commit(&bar.empty[grp]);
             }
             if (!ok) break;
@@ -634,15 +659,19 @@ __global__ void __launch_bounds__(kThreads, 1) hca_attn_kernel(const __grid_cons
             ob[oc / 2 + i] = pack_bf16x2(__uint_as_float(v[2 * i]) * inv_l, __uint_as_float(v[2 * i + 1]) * inv_l);
         }
       };
-      auto stage_o = [&]() {  // the stores that last read the staging must be done with it
+      // one staging round: the kOutBufs boxes of 32 columns starting at column 32 * kOutBufs * sub
+      // of the 128 held in ob
+      auto stage_o = [&](int sub) {  // the stores that last read the staging must be done with it
         if (store_issuer) bulk_wait_group_read0();
         softmax_bar_sync();
 #pragma unroll
         for (int q = 0; q < kOutBufs; ++q)
 #pragma unroll
-          for (int i = 0; i < 4; ++i)  // 64-byte swizzle: 16-byte unit i of row r at unit i ^ ((r >> 1) & 3)
+          for (int i = 0; i < 4; ++i) {  // 64-byte swizzle: 16-byte unit i of row r at unit i ^ ((r >> 1) & 3)
+            const int w = (sub * kOutBufs + q) * 16 + 4 * i;
             *reinterpret_cast<uint4*>(sOut + q * kOutBufBytes + r * 64 + ((i ^ ((r >> 1) & 3)) * 16)) =
-                make_uint4(ob[q * 16 + 4 * i], ob[q * 16 + 4 * i + 1], ob[q * 16 + 4 * i + 2], ob[q * 16 + 4 * i + 3]);
+                make_uint4(ob[w], ob[w + 1], ob[w + 2], ob[w + 3]);
+          }
         fence_proxy_async_smem();
       };
       auto store_o = [&](int c0) {
@@ -654,15 +683,31 @@ __global__ void __launch_bounds__(kThreads, 1) hca_attn_kernel(const __grid_cons
           bulk_commit_group();
         }
       };
-      read_o(0);
-      stage_o();
-      read_o(128);
-      tc_fence_before();
-      mbar_arrive(&bar.o_empty[0]);
-      mbar_arrive(&bar.o_empty[1]);
-      store_o(0);
-      stage_o();
-      store_o(128);
+      if constexpr (kOutBufs == 4) {  // one round per 128 columns
+        read_o(0);
+        stage_o(0);
+        read_o(128);
+        tc_fence_before();
+        mbar_arrive(&bar.o_empty[0]);
+        mbar_arrive(&bar.o_empty[1]);
+        store_o(0);
+        stage_o(0);
+        store_o(128);
+      } else {  // two rounds of 64 columns per 128 (smaller staging area)
+        read_o(0);
+        stage_o(0);
+        store_o(0);
+        stage_o(1);
+        store_o(64);
+        read_o(128);
+        tc_fence_before();
+        mbar_arrive(&bar.o_empty[0]);
+        mbar_arrive(&bar.o_empty[1]);
+        stage_o(0);
+        store_o(128);
+        stage_o(1);
+        store_o(192);
+      }
       ++it;
     };
 
@@ -942,12 +987,17 @@ __global__ void __launch_bounds__(256) hca_combine_kernel(const Params p, uint16
     p.lse[((size_t)b * p.Lq + tok) * p.Hq + h] = (M + __log2f(L)) * 0.69314718055994531f;
 }
 
-bool make_map_4d(CUtensorMap* m, const void* base, int d, int heads, int rows, int B, int box_cols, int box_heads,
-                 int box_rows, int swizzle) {
+// [B, rows, heads, pitch] bf16 tensor seen as its first d columns (d <= pitch)
+bool make_map_4d_pitch(CUtensorMap* m, const void* base, int d, int pitch, int heads, int rows, int B, int box_cols,
+                       int box_heads, int box_rows, int swizzle) {
   const uint64_t dims[4] = {(uint64_t)d, (uint64_t)heads, (uint64_t)rows, (uint64_t)B};
-  const uint64_t strides[3] = {(uint64_t)d * 2, (uint64_t)heads * d * 2, (uint64_t)rows * heads * d * 2};
+  const uint64_t strides[3] = {(uint64_t)pitch * 2, (uint64_t)heads * pitch * 2, (uint64_t)rows * heads * pitch * 2};
   const uint32_t box[4] = {(uint32_t)box_cols, (uint32_t)box_heads, (uint32_t)box_rows, 1};
   return encode_tmap_bf16_swizzle(m, 4, const_cast<void*>(base), dims, strides, box, swizzle);
+}
+bool make_map_4d(CUtensorMap* m, const void* base, int d, int heads, int rows, int B, int box_cols, int box_heads,
+                 int box_rows, int swizzle) {
+  return make_map_4d_pitch(m, base, d, d, heads, rows, B, box_cols, box_heads, box_rows, swizzle);
 }
 
 int num_sms() {
@@ -1084,12 +1134,15 @@ extern "C" size_t hca_attn_fwd_workspace_size(int B, int Lq, int q_offset, int H
   return G.workspace_bytes;
 }
 
-extern "C" hcadsa_status hca_attn_fwd(const hcadsa_bf16* Q, const hcadsa_bf16* Kc, const hcadsa_bf16* Vc, int n_c,
-                                      const hcadsa_bf16* Kw, const hcadsa_bf16* Vw, int win_start, int n_w,
-                                      hcadsa_bf16* O, float* lse, int B, int Lq, int q_offset, int Hq, int Hkv,
-                                      int d, int blk, int W, float scale, void* workspace, size_t workspace_bytes,
-                                      hcadsa_stream stream) {
-  using namespace hcadsa;
+namespace hcadsa {
+namespace {
+
+// Checks shared by both entry points; returns HCADSA_OK and the launch geometry when the call is
+// valid.  Score width dqk, value width kD (512).
+hcadsa_status check_call(const void* Q, const void* Kc, const void* Vc, int n_c, const void* Kw, const void* Vw,
+                         int win_start, int n_w, const void* O, const float* lse, int B, int Lq, int q_offset,
+                         int Hq, int Hkv, int blk, int W, const void* workspace, size_t workspace_bytes,
+                         Geometry* G) {
   if (!Q || !Kw || !Vw || !O) return HCADSA_ERR_NULL;
   if (n_c > 0 && (!Kc || !Vc)) return HCADSA_ERR_NULL;
   if (B < 0 || Lq < 0 || q_offset < 0 || Hq <= 0 || Hkv <= 0 || n_c < 0 || n_w < 0 || win_start < 0 || blk <= 0 ||
@@ -1097,7 +1150,7 @@ extern "C" hcadsa_status hca_attn_fwd(const hcadsa_bf16* Q, const hcadsa_bf16* K
     return HCADSA_ERR_SHAPE;
   if (Hq % Hkv != 0) return HCADSA_ERR_SHAPE;
   const int g = Hq / Hkv;
-  if (d != kD || g > 128 || 128 % g != 0) return HCADSA_ERR_UNSUPPORTED;
+  if (g > 128 || 128 % g != 0) return HCADSA_ERR_UNSUPPORTED;
   if (!aligned16(Q) || !aligned16(Kw) || !aligned16(Vw) || !aligned16(O) ||
       (n_c > 0 && (!aligned16(Kc) || !aligned16(Vc))) || (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
     return HCADSA_ERR_ALIGN;
@@ -1108,31 +1161,42 @@ extern "C" hcadsa_status hca_attn_fwd(const hcadsa_bf16* Q, const hcadsa_bf16* K
   const long long ws_first = t_first - W + 1 > 0 ? t_first - W + 1 : 0;
   const long long nc_last = t_last - W + 1 > 0 ? (t_last - W + 1) / blk : 0;
   if (ws_first < win_start || t_last - win_start >= n_w || nc_last > n_c) return HCADSA_ERR_SHAPE;
-  Geometry G;
-  const hcadsa_status gs = geometry(&G, B, Lq, q_offset, Hq, Hkv, d, blk, W);
+  const hcadsa_status gs = geometry(G, B, Lq, q_offset, Hq, Hkv, kD, blk, W);
   if (gs != HCADSA_OK) return gs;
-  if (!workspace || workspace_bytes < G.workspace_bytes) return HCADSA_ERR_WORKSPACE;
+  if (!workspace || workspace_bytes < G->workspace_bytes) return HCADSA_ERR_WORKSPACE;
   if (!aligned16(workspace)) return HCADSA_ERR_ALIGN;
+  return HCADSA_OK;
+}
 
+// Builds the tensor maps and launches.  Score width DQK; K rows are DQK wide, V rows are read as
+// the first kD columns of rows `vpitch` wide (vpitch = kD: separate V; vpitch = DQK: V is the
+// latent part of K).
+template <int DQK>
+hcadsa_status launch_hca(const hcadsa_bf16* Q, const hcadsa_bf16* Kc, const hcadsa_bf16* Vc, int n_c,
+                         const hcadsa_bf16* Kw, const hcadsa_bf16* Vw, int vpitch, int win_start, int n_w,
+                         hcadsa_bf16* O, float* lse, int B, int Lq, int q_offset, int Hq, int Hkv, int blk, int W,
+                         float scale, void* workspace, const Geometry& G, cudaStream_t stream) {
+  using S = Shape<DQK>;
+  const int g = Hq / Hkv;
   Maps maps;
-  if (!make_map_4d(&maps.q, Q, kD, Hq, Lq, B, 64, g, G.TT, 128)) return HCADSA_ERR_CUDA;
+  if (!make_map_4d(&maps.q, Q, DQK, Hq, Lq, B, 64, g, G.TT, 128)) return HCADSA_ERR_CUDA;
   if (!make_map_4d(&maps.o, O, kD, Hq, Lq, B, kOutCols, g, G.TT, 64)) return HCADSA_ERR_CUDA;
   {
     // entries of the merged tiles exist only when n_c > 0; otherwise those maps are never read
     const hcadsa_bf16* KcM = n_c > 0 ? Kc : Kw;
     const hcadsa_bf16* VcM = n_c > 0 ? Vc : Vw;
     const int rows_c = n_c > 0 ? n_c : n_w;
-    if (!make_map_4d(&maps.kmerge[0], Kw, kD, Hkv, n_w, B, 64, 1, kMergeWinRows, 128) ||
-        !make_map_4d(&maps.kmerge[1], KcM, kD, Hkv, rows_c, B, 64, 1, kMergeEntRows, 128) ||
-        !make_map_4d(&maps.vmerge[0], Vw, kD, Hkv, n_w, B, 64, 1, kMergeWinRows, 128) ||
-        !make_map_4d(&maps.vmerge[1], VcM, kD, Hkv, rows_c, B, 64, 1, kVRows - kMergeWinRows, 128))
+    if (!make_map_4d(&maps.kmerge[0], Kw, DQK, Hkv, n_w, B, 64, 1, kMergeWinRows, 128) ||
+        !make_map_4d(&maps.kmerge[1], KcM, DQK, Hkv, rows_c, B, 64, 1, kMergeEntRows, 128) ||
+        !make_map_4d_pitch(&maps.vmerge[0], Vw, kD, vpitch, Hkv, n_w, B, 64, 1, kMergeWinRows, 128) ||
+        !make_map_4d_pitch(&maps.vmerge[1], VcM, kD, vpitch, Hkv, rows_c, B, 64, 1, kVRows - kMergeWinRows, 128))
       return HCADSA_ERR_CUDA;
     for (int small = 0; small < 2; ++small) {
       const int krows = small ? kSmallRows : kKeyTile, vrows = small ? kSmallRows : kVRows;
-      if (!make_map_4d(&maps.k[1][small], Kw, kD, Hkv, n_w, B, 64, 1, krows, 128) ||
-          !make_map_4d(&maps.v[1][small], Vw, kD, Hkv, n_w, B, 64, 1, vrows, 128) ||
-          !make_map_4d(&maps.k[0][small], KcM, kD, Hkv, rows_c, B, 64, 1, krows, 128) ||
-          !make_map_4d(&maps.v[0][small], VcM, kD, Hkv, rows_c, B, 64, 1, vrows, 128))
+      if (!make_map_4d(&maps.k[1][small], Kw, DQK, Hkv, n_w, B, 64, 1, krows, 128) ||
+          !make_map_4d_pitch(&maps.v[1][small], Vw, kD, vpitch, Hkv, n_w, B, 64, 1, vrows, 128) ||
+          !make_map_4d(&maps.k[0][small], KcM, DQK, Hkv, rows_c, B, 64, 1, krows, 128) ||
+          !make_map_4d_pitch(&maps.v[0][small], VcM, kD, vpitch, Hkv, rows_c, B, 64, 1, vrows, 128))
         return HCADSA_ERR_CUDA;
     }
   }
@@ -1164,17 +1228,58 @@ extern "C" hcadsa_status hca_attn_fwd(const hcadsa_bf16* Q, const hcadsa_bf16* K
   p.part_ml = p.split_mode ? reinterpret_cast<float2*>(p.scratch + G.scratch_bytes + (size_t)G.total_units * 128 * kD * 4)
                            : nullptr;
   p.err = device_error_ptr();
-  if (cudaFuncSetAttribute(hca_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) != cudaSuccess)
+  if (cudaFuncSetAttribute(hca_attn_kernel<DQK>, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kSmemBytes) !=
+      cudaSuccess)
     return HCADSA_ERR_CUDA;
-  hca_attn_kernel<<<G.grid, kThreads, kSmemBytes, as_stream(stream)>>>(maps, p);
+  hca_attn_kernel<DQK><<<G.grid, kThreads, S::kSmemBytes, stream>>>(maps, p);
   if (p.split_mode) {
     const hcadsa_status st = launch_status();
     if (st != HCADSA_OK) return st;
     // only row groups holding a valid token: 8 rows per CTA
     const int valid_rows = Lq < G.TT ? Lq * g : 128;
-    hca_combine_kernel<<<dim3((unsigned)G.total_tiles, (unsigned)((valid_rows + 7) / 8), kD / 128), 256, 0,
-                         as_stream(stream)>>>(
+    hca_combine_kernel<<<dim3((unsigned)G.total_tiles, (unsigned)((valid_rows + 7) / 8), kD / 128), 256, 0, stream>>>(
         p, reinterpret_cast<uint16_t*>(O));
   }
   return launch_status();
+}
+
+}  // namespace
+}  // namespace hcadsa
+
+extern "C" hcadsa_status hca_attn_fwd(const hcadsa_bf16* Q, const hcadsa_bf16* Kc, const hcadsa_bf16* Vc, int n_c,
+                                      const hcadsa_bf16* Kw, const hcadsa_bf16* Vw, int win_start, int n_w,
+                                      hcadsa_bf16* O, float* lse, int B, int Lq, int q_offset, int Hq, int Hkv,
+                                      int d, int blk, int W, float scale, void* workspace, size_t workspace_bytes,
+                                      hcadsa_stream stream) {
+  using namespace hcadsa;
+  Geometry G;
+  if (d != kD && Q && Kw && Vw && O && (n_c == 0 || (Kc && Vc)) && B >= 0 && Lq >= 0 && Hq > 0 && Hkv > 0 &&
+      Hq % Hkv == 0)
+    return HCADSA_ERR_UNSUPPORTED;
+  const hcadsa_status st = check_call(Q, Kc, Vc, n_c, Kw, Vw, win_start, n_w, O, lse, B, Lq, q_offset, Hq, Hkv, blk,
+                                      W, workspace, workspace_bytes, &G);
+  if (st != HCADSA_OK || B == 0 || Lq == 0) return st;
+  return launch_hca<512>(Q, Kc, Vc, n_c, Kw, Vw, kD, win_start, n_w, O, lse, B, Lq, q_offset, Hq, Hkv, blk, W, scale,
+                         workspace, G, as_stream(stream));
+}
+
+extern "C" size_t hca_attn_fwd_latent_workspace_size(int B, int Lq, int q_offset, int Hq, int Hkv, int dqk, int dv,
+                                                     int n_c, int blk, int W) {
+  if (dqk != 576 || dv != 512) return 0;
+  return hca_attn_fwd_workspace_size(B, Lq, q_offset, Hq, Hkv, dv, n_c, blk, W);
+}
+
+extern "C" hcadsa_status hca_attn_fwd_latent(const hcadsa_bf16* Q, const hcadsa_bf16* Kc, int n_c,
+                                             const hcadsa_bf16* Kw, int win_start, int n_w, hcadsa_bf16* O,
+                                             float* lse, int B, int Lq, int q_offset, int Hq, int Hkv, int dqk, int dv,
+                                             int blk, int W, float scale, void* workspace, size_t workspace_bytes,
+                                             hcadsa_stream stream) {
+  using namespace hcadsa;
+  Geometry G;
+  const hcadsa_status st = check_call(Q, Kc, Kc, n_c, Kw, Kw, win_start, n_w, O, lse, B, Lq, q_offset, Hq, Hkv, blk,
+                                      W, workspace, workspace_bytes, &G);
+  if (st == HCADSA_OK && (dqk != 576 || dv != 512)) return HCADSA_ERR_UNSUPPORTED;
+  if (st != HCADSA_OK || B == 0 || Lq == 0) return st;
+  return launch_hca<576>(Q, Kc, Kc, n_c, Kw, Kw, 576, win_start, n_w, O, lse, B, Lq, q_offset, Hq, Hkv, blk, W,
+                         scale, workspace, G, as_stream(stream));
 }

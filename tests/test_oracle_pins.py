@@ -341,6 +341,59 @@ def test_dsa_topk_decode_offset_equals_prefill_row(oracle_mod):
     assert np.array_equal(pre, dec)
 
 
+# ---------------------------------------------------------------- qk 576 / v 512 (shared latent)
+
+def _sdpa_latent(Q, K, dv, mask, scale):
+    """torch fp64 SDPA with keys of width dqk and values = the first dv columns of the keys."""
+    q = Q.double().permute(0, 2, 1, 3)
+    k = K.double().permute(0, 2, 1, 3)
+    g = q.shape[1] // k.shape[1]
+    k = k.repeat_interleave(g, dim=1)
+    o = torch.nn.functional.scaled_dot_product_attention(q, k, k[..., :dv].contiguous(), attn_mask=mask, scale=scale)
+    return o.permute(0, 2, 1, 3).numpy()
+
+
+def test_hca_latent_wide_window_is_dense_causal_with_positional_slice(oracle_mod):
+    """W >= L: dense causal attention with 24-wide scores (16-wide latent + an 8-wide positional
+    slice that changes the scores) and values = the latent part of the keys (torch fp64 SDPA)."""
+    B, L, Hq, Hkv, dqk, dv = 2, 40, 4, 2, 24, 16
+    g = torch.Generator().manual_seed(601)
+    Q = torch.randn(B, L, Hq, dqk, generator=g).to(torch.bfloat16)
+    K = torch.randn(B, L, Hkv, dqk, generator=g).to(torch.bfloat16)
+    O, lse = oracle_mod.hca_attn_latent(bits(Q), None, bits(K), dv, W=L, scale=0.3, with_lse=True)
+    mask = torch.ones(L, L, dtype=torch.bool).tril()
+    np.testing.assert_allclose(O, _sdpa_latent(Q, K, dv, mask, 0.3).reshape(B * L, Hq, dv), rtol=0, atol=1e-12)
+    # the positional slice is part of the score: zeroing it changes the result
+    Q0 = Q.clone()
+    Q0[..., dv:] = 0
+    O0 = oracle_mod.hca_attn_latent(bits(Q0), None, bits(K), dv, W=L, scale=0.3)
+    assert np.abs(O0 - O).max() > 1e-3
+    s = 0.3 * K[1, :8, 1].double() @ Q[1, 7, 3].double()
+    assert abs(lse[L + 7, 3] - torch.logsumexp(s, 0).item()) < 1e-12
+
+
+def test_hca_latent_general_matches_masked_sdpa_over_entries_and_window(oracle_mod):
+    """Entries + window (W = 5, blk = 4) with shared-latent values against SDPA over [entries ||
+    window] with the visible set enumerated from its definition."""
+    B, L, Hq, dqk, dv, blk, W = 1, 37, 2, 24, 16, 4, 5
+    g = torch.Generator().manual_seed(603)
+    Q = torch.randn(B, L, Hq, dqk, generator=g).to(torch.bfloat16)
+    K = torch.randn(B, L, 1, dqk, generator=g).to(torch.bfloat16)
+    w = np.full(blk, 0.25, np.float32)
+    Kc = oracle_mod.hca_compress(bits(K), w, blk)
+    O = oracle_mod.hca_attn_latent(bits(Q), Kc, bits(K), dv, blk=blk, W=W, scale=0.2)
+    n_c = L // blk
+    Kall = torch.cat([from_bits(Kc).view(B, n_c, 1, dqk), K], dim=1)
+    mask = torch.zeros(L, n_c + L, dtype=torch.bool)
+    for t in range(L):
+        for j in range(n_c):
+            if blk * (j + 1) <= t - W + 1:
+                mask[t, j] = True
+        for s in range(max(0, t - W + 1), t + 1):
+            mask[t, n_c + s] = True
+    np.testing.assert_allclose(O, _sdpa_latent(Q, Kall, dv, mask, 0.2).reshape(L, Hq, dv), rtol=0, atol=1e-12)
+
+
 # ---------------------------------------------------------------- CSA (top-k over compressed entries)
 
 @pytest.mark.parametrize("blk", [1, 4, 7])
@@ -419,6 +472,68 @@ def test_csa_attention_over_4to1_entries_matches_masked_sdpa(oracle_mod):
     ref = sdpa_ref(inp["Q"][:, seen], Kt, Vt, mask[seen], 0.25).reshape(-1, Hq, d)
     np.testing.assert_allclose(O[seen.numpy()], ref, rtol=0, atol=1e-12)
     assert np.all(O[~seen.numpy()] == 0.0) and (~seen).sum() == blk - 1
+
+
+# ---------------------------------------------------------------- output gate + virtual-head mix
+
+def _gate_inputs(B, L, H, dv, rq, r, seed):
+    g = torch.Generator().manual_seed(seed)
+    O = (torch.randn(B, L, H, dv, generator=g) * 0.1).to(torch.bfloat16)
+    cq = torch.randn(B, L, rq, generator=g).to(torch.bfloat16)
+    Wg = (torch.randn(H * dv, rq, generator=g) / math.sqrt(rq)).to(torch.bfloat16)
+    U = (torch.randn(H, r, generator=g) * 0.3).numpy().astype(np.float32)
+    V = (torch.randn(H, r, generator=g) * 0.3).numpy().astype(np.float32)
+    return O, cq, Wg, U, V
+
+
+def test_gate_vha_zero_gate_weights_and_no_mix_halve_the_output(oracle_mod):
+    """W_g = 0 gives sigmoid(0) = 1/2 everywhere; U = 0 switches the mix off: Y = O / 2 exactly."""
+    O, cq, _, _, _ = _gate_inputs(2, 5, 4, 8, 16, 2, 401)
+    Wg = torch.zeros(4 * 8, 16, dtype=torch.bfloat16)
+    Y = oracle_mod.gate_vha(bits(O), bits(cq), bits(Wg), np.zeros((4, 2), np.float32), np.ones((4, 2), np.float32))
+    np.testing.assert_array_equal(Y, O.double().numpy() / 2)
+
+
+def test_gate_vha_without_mix_is_sigmoid_of_latent_projection(oracle_mod):
+    """No mix (rank 0): Y = sigmoid(cq W_g^T) * O, the gate through torch's fp64 matmul and sigmoid."""
+    B, L, H, dv, rq = 2, 6, 4, 8, 32
+    O, cq, Wg, _, _ = _gate_inputs(B, L, H, dv, rq, 1, 403)
+    Y = oracle_mod.gate_vha(bits(O), bits(cq), bits(Wg), np.zeros((H, 0), np.float32), np.zeros((H, 0), np.float32))
+    z = (cq.double().reshape(B * L, rq) @ Wg.double().t()).reshape(B, L, H, dv)
+    np.testing.assert_allclose(Y, (torch.sigmoid(z) * O.double()).numpy(), rtol=0, atol=1e-13)
+
+
+def test_gate_vha_mix_orientation_copies_one_head(oracle_mod):
+    """I + U V^T with U = [[1], [0]], V = [[-1], [1]] has rows [0, 1] and [0, 1]: both heads
+    become head 1 (U and V swapped would give [[0, 0], [1, 2]] instead)."""
+    B, L, H, dv, rq = 1, 3, 2, 8, 16
+    O, cq, _, _, _ = _gate_inputs(B, L, H, dv, rq, 1, 405)
+    Wg = torch.zeros(H * dv, rq, dtype=torch.bfloat16)
+    U = np.array([[1.0], [0.0]], np.float32)
+    V = np.array([[-1.0], [1.0]], np.float32)
+    Y = oracle_mod.gate_vha(bits(O), bits(cq), bits(Wg), U, V)
+    o = O.double().numpy()
+    np.testing.assert_array_equal(Y[:, :, 0], o[:, :, 1] / 2)
+    np.testing.assert_array_equal(Y[:, :, 1], o[:, :, 1] / 2)
+
+
+def test_gate_vha_full_rank_negative_identity_mix_cancels_the_output(oracle_mod):
+    """U V^T = -I (rank H) removes the identity path: Y = 0."""
+    O, cq, Wg, _, _ = _gate_inputs(1, 4, 3, 8, 16, 3, 407)
+    Y = oracle_mod.gate_vha(bits(O), bits(cq), bits(Wg), -np.eye(3, dtype=np.float32), np.eye(3, dtype=np.float32))
+    np.testing.assert_allclose(Y, 0.0, rtol=0, atol=1e-15)
+
+
+def test_gate_vha_mix_matches_matrix_form_per_channel(oracle_mod):
+    """With the gate fixed at 1/2, each token's output is (I + U V^T) applied to its H x dv block,
+    checked against a torch fp64 matrix product (heads mix, channels do not)."""
+    B, L, H, dv, rq, r = 2, 3, 16, 32, 16, 4
+    O, cq, _, U, V = _gate_inputs(B, L, H, dv, rq, r, 409)
+    Wg = torch.zeros(H * dv, rq, dtype=torch.bfloat16)
+    Y = oracle_mod.gate_vha(bits(O), bits(cq), bits(Wg), U, V)
+    M = torch.eye(H, dtype=torch.float64) + torch.from_numpy(U).double() @ torch.from_numpy(V).double().t()
+    ref = torch.einsum("hg,btgc->bthc", M, O.double()) / 2
+    np.testing.assert_allclose(Y, ref.numpy(), rtol=0, atol=1e-13)
 
 
 # ---------------------------------------------------------------- DSA attention
