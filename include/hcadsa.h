@@ -325,6 +325,33 @@ hcadsa_status attn_gate_vha_fwd(const hcadsa_bf16* O, const hcadsa_bf16* cq, con
 hcadsa_status hca_compress_bwd(const hcadsa_bf16* X, const float* w, const float* dXc, float* dX, float* dw, int B,
                                int L, int H, int d, int blk, hcadsa_stream stream);
 
+/*
+ * Backward of DSA sparse attention.  Source: the forward above (the mirrorspeed page, section
+ * "Hybrid sparse attention, 1/7 full context access": attention over the k selected positions;
+ * 64 heads of 256 on one shared K/V head).  For a loss with output gradient dO, with the
+ * forward's probabilities p[h, s] = exp(scale <Q[h], K[s]> - lse[h]) over the selected s:
+ *     D[h]    = <dO[h], O[h]>
+ *     dS[h,s] = p[h,s] (<dO[h], V[s]> - D[h])
+ *     dQ[h]   = scale sum_s dS[h,s] K[s]                      (written)
+ *     dK[s]  += scale sum_h dS[h,s] Q[h],  dV[s] += sum_h p[h,s] dO[h]   (ADDED to)
+ * P and dS enter the tensor cores as bf16; accumulation is fp32.  dK and dV are summed over
+ * tokens with fp32 atomics (order not fixed: results can differ in the last bits between
+ * runs); zero them first.  Padding entries (< 0) contribute nothing; an entry >= Lk is skipped
+ * and recorded as HCADSA_ERR_DEVICE_BOUNDS.
+ *
+ *   Q, O, dO : [B, Lq, Hq, d] bf16 (O and lse from dsa_sparse_attn_fwd)
+ *   K, V     : [B, Lk, d] bf16
+ *   idx      : [B, Lq, k] int32 (as for the forward)
+ *   lse      : [B, Lq, Hq] fp32, natural log
+ *   dQ       : [B, Lq, Hq, d] fp32 (written)
+ *   dK, dV   : [B, Lk, d] fp32 (accumulated)
+ * Requirements: d == 256, Hq == 64, 1 <= k <= 4096.
+ */
+hcadsa_status dsa_sparse_attn_bwd(const hcadsa_bf16* Q, const hcadsa_bf16* K, const hcadsa_bf16* V,
+                                  const int32_t* idx, const hcadsa_bf16* O, const hcadsa_bf16* dO, const float* lse,
+                                  float* dQ, float* dK, float* dV, int B, int Lq, int Lk, int Hq, int d, int k,
+                                  float scale, hcadsa_stream stream);
+
 #ifdef __cplusplus
 }
 #endif

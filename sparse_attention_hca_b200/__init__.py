@@ -90,6 +90,8 @@ def lib() -> ctypes.CDLL:
             L.attn_gate_vha_fwd.restype = I
             L.hca_compress_bwd.argtypes = [P, P, P, P, P, I, I, I, I, I, P]
             L.hca_compress_bwd.restype = I
+            L.dsa_sparse_attn_bwd.argtypes = [P, P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, F, P]
+            L.dsa_sparse_attn_bwd.restype = I
             _lib = L
     return _lib
 
@@ -397,3 +399,38 @@ def hca_compress_bwd(X, w, dXc, blk: int = 128, *, dX=None, dw=None, stream=None
     st = lib().hca_compress_bwd(_ptr(X), _ptr(w), _ptr(dXc), _ptr(dX), _ptr(dw), B, L, H, d, blk, _stream(stream))
     _check(st, "hca_compress_bwd")
     return dX, dw
+
+
+def dsa_sparse_attn_bwd(Q, K, V, idx, O, dO, lse, *, scale: float | None = None, dK=None, dV=None, stream=None):
+    """Gradients of the DSA sparse attention: Q, O, dO [B, Lq, 64, 256] bf16, K, V [B, Lk, 256] bf16,
+    idx [B, Lq, k] int32, lse [B, Lq, 64] fp32 (from the forward) -> (dQ [B, Lq, 64, 256] fp32,
+    dK, dV [B, Lk, 256] fp32; dK and dV are added to when given, zeros otherwise)."""
+    _need(Q, torch.bfloat16, "Q")
+    B, Lq, Hq, d = Q.shape
+    _need(K, torch.bfloat16, "K")
+    if K.shape[0] != B or K.shape[-1] != d:
+        raise ValueError(f"K has shape {tuple(K.shape)}, expected [{B}, Lk, {d}]")
+    Lk = K.shape[1]
+    _need_numel(K, B * Lk * d, "K", f"[{B}, {Lk}, {d}]")
+    _need(V, torch.bfloat16, "V", K.shape)
+    _need(idx, torch.int32, "idx")
+    if idx.dim() != 3 or idx.shape[0] != B or idx.shape[1] != Lq:
+        raise ValueError(f"idx has shape {tuple(idx.shape)}, expected [{B}, {Lq}, k]")
+    k = idx.shape[-1]
+    _need(O, torch.bfloat16, "O", Q.shape)
+    _need(dO, torch.bfloat16, "dO", Q.shape)
+    _need(lse, torch.float32, "lse", (B, Lq, Hq))
+    if dK is not None:
+        _need_numel(dK, B * Lk * d, "dK", "fp32 like K")
+    if dV is not None:
+        _need_numel(dV, B * Lk * d, "dV", "fp32 like V")
+    _on_device(Q, K, V, idx, O, dO, lse, dK, dV)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    dQ = torch.empty(Q.shape, dtype=torch.float32, device=Q.device)
+    dK = torch.zeros((B, Lk, d), dtype=torch.float32, device=Q.device) if dK is None else dK
+    dV = torch.zeros((B, Lk, d), dtype=torch.float32, device=Q.device) if dV is None else dV
+    st = lib().dsa_sparse_attn_bwd(_ptr(Q), _ptr(K), _ptr(V), _ptr(idx), _ptr(O), _ptr(dO), _ptr(lse), _ptr(dQ),
+                                   _ptr(dK), _ptr(dV), B, Lq, Lk, Hq, d, k, float(scale), _stream(stream))
+    _check(st, "dsa_sparse_attn_bwd")
+    return dQ, dK, dV
