@@ -465,6 +465,63 @@ def run_hca_latent(hd, device, peaks, iters=10):
             "attn_pct_bf16": 100 * tf / peaks["bf16_tflops"], "algorithmic_flop": flop}
 
 
+def run_backward(hd, device, peaks, iters=5):
+    """Backward kernels at the layer sizes of the step (L = 32768): the DSA sparse attention
+    backward (dQ, dK, dV from the forward's O and lse over the top-2048 selection of the step's
+    indexer) and the HCA compressor's adjoint (dX, dw for 512-wide keys, blocks of 128).  CUDA
+    events, median of `iters` after 3 warm-up runs.  Algorithmic units: 5 * 2 * 256 flop per
+    (query, head, selected key) (S, dP, dV, dK, dQ) and 2 KB of fp32 reductions into dK / dV per
+    (query, selected key)."""
+    x = make_dsa_inputs(device, synth.SEED)
+    idx = hd.dsa_index_topk(x["q_idx"], x["k_idx"], x["w_idx"], DSA.k)
+    O, lse = hd.dsa_sparse_attn_fwd(x["dQ"], x["dK"], x["dV"], idx, return_lse=True)
+    gO = _Draw(device, synth.SEED).normal(tuple(O.shape), 0.1, 61)
+    dK = torch.zeros((1, L, DSA.d), dtype=torch.float32, device=device)
+    dV = torch.zeros_like(dK)
+    for _ in range(3):
+        hd.dsa_sparse_attn_bwd(x["dQ"], x["dK"], x["dV"], idx, O, gO, lse, dK=dK, dV=dV)
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(iters)]
+    for i in range(iters):
+        evs[i][0].record()
+        hd.dsa_sparse_attn_bwd(x["dQ"], x["dK"], x["dV"], idx, O, gO, lse, dK=dK, dV=dV)
+        evs[i][1].record()
+    torch.cuda.synchronize()
+    ms = statistics.median(e[0].elapsed_time(e[1]) for e in evs)
+    keys = int((idx >= 0).sum().item())  # selected (query, key) pairs
+    del x, idx, O, lse, gO, dK, dV
+    torch.cuda.empty_cache()
+    flop = 10.0 * DSA.d * DSA.Hq * keys
+    red_bytes = 2.0 * 4 * DSA.d * keys
+    tf = flop / (ms * 1e-3) / 1e12
+    # compressor adjoint: X (bf16) read, dX (fp32) read + written, dXc (fp32) read
+    Xk = _Draw(device, synth.SEED).normal((1, L, HCA.Hkv, HCA.d), 1 / math.sqrt(HCA.d), 62)
+    w = _Draw(device, synth.SEED).uniform(HCA.blk, 2.0 / HCA.blk, 63)
+    dXc = _Draw(device, synth.SEED).normal((1, L // HCA.blk, HCA.Hkv, HCA.d), 1.0, 64).float()
+    dX = torch.zeros((1, L, HCA.Hkv, HCA.d), dtype=torch.float32, device=device)
+    dw = torch.zeros(HCA.blk, dtype=torch.float32, device=device)
+    for _ in range(3):
+        hd.hca_compress_bwd(Xk, w, dXc, HCA.blk, dX=dX, dw=dw)
+    torch.cuda.synchronize()
+    cevs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(iters)]
+    for i in range(iters):
+        cevs[i][0].record()
+        hd.hca_compress_bwd(Xk, w, dXc, HCA.blk, dX=dX, dw=dw)
+        cevs[i][1].record()
+    torch.cuda.synchronize()
+    cms = statistics.median(e[0].elapsed_time(e[1]) for e in cevs)
+    cbytes = L * HCA.Hkv * HCA.d * (2 + 4 + 4) + (L // HCA.blk) * HCA.Hkv * HCA.d * 4
+    del Xk, dXc, dX, dw
+    torch.cuda.empty_cache()
+    return {"workload": f"dsa_bwd_L{L}_h64_d256_k2048 + compress_bwd_L{L}_d512_blk128 (B=1)", "iters": iters,
+            "dsa_bwd_ms": ms, "dsa_bwd_tflops": tf, "dsa_bwd_pct_bf16": 100 * tf / peaks["bf16_tflops"],
+            "dsa_bwd_reduce_gbs": red_bytes / (ms * 1e-3) / 1e9, "dsa_bwd_algorithmic_flop": flop,
+            "dsa_bwd_reduce_bytes": red_bytes,
+            "compress_bwd_us": cms * 1e3, "compress_bwd_gbs": cbytes / (cms * 1e-3) / 1e9,
+            "compress_bwd_pct_hbm": 100 * cbytes / (cms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+            "compress_bwd_bytes": cbytes}
+
+
 def run_hca_131k(hd, device, peaks, iters=10):
     """The HCA long-context prefill configuration (B = 1, L = 131072, 16 query heads on one K/V
     head, d = 512, 1024 compressed entries): compression and attention timed with CUDA events
@@ -665,6 +722,10 @@ def ours(args):
     if rank == 0 and not args.no_latent:
         latent = run_hca_latent(hd, device, peaks)
         hd.hcadsa_check_device_error()
+    bwd = None
+    if rank == 0 and not args.no_bwd:
+        bwd = run_backward(hd, device, peaks)
+        hd.hcadsa_check_device_error()
     e2e_ms, h2d, d2h = e2e_measure(hd, x, device, steps=max(2, min(args.steps, 4)))
     e2e_ms = max_over_ranks(e2e_ms, dist, device)
     e2e = {"value": job_throughput(e2e_ms, world), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
@@ -713,6 +774,7 @@ def ours(args):
         "csa": csa,
         "gate_vha": gate,
         "hca_latent_576": latent,
+        "backward": bwd,
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -769,9 +831,10 @@ def only_kernel(args):
         hd.hcadsa_check_device_error()
         print(json.dumps(out))
         return
-    if args.only in ("csa", "gate_vha", "hca_latent"):
+    if args.only in ("csa", "gate_vha", "hca_latent", "backward"):
         L = args.seq_len
-        run = {"csa": run_csa, "gate_vha": run_gate_vha, "hca_latent": run_hca_latent}[args.only]
+        run = {"csa": run_csa, "gate_vha": run_gate_vha, "hca_latent": run_hca_latent,
+               "backward": run_backward}[args.only]
         out = run(hd, torch.device("cuda", 0), load_peaks(), iters=max(1, args.steps))
         hd.hcadsa_check_device_error()
         print(json.dumps(out))
@@ -832,8 +895,9 @@ def main():
     ap.add_argument("--no-csa", action="store_true", help="skip the CSA layer block")
     ap.add_argument("--no-gate", action="store_true", help="skip the output gate + head mix block")
     ap.add_argument("--no-latent", action="store_true", help="skip the qk 576 / v 512 HCA block")
+    ap.add_argument("--no-bwd", action="store_true", help="skip the backward block")
     ap.add_argument("--only", choices=["compress", "hca_attn", "index_topk", "dsa_attn", "decode", "csa", "gate_vha",
-                                       "hca_latent"],
+                                       "hca_latent", "backward"],
                     help="profiling mode: run one kernel alone at --seq-len, or the decode step "
                          "(B = 32 at t = 1,048,575; --steps timed steps after 3 warm-up steps)")
     ap.add_argument("--seq-len", type=int, default=L)

@@ -20,9 +20,12 @@
 //       dQ^T += K_g^T dS^T                       (A = K_g MN-major, B = dS^T MN-major, over all
 //                                                 tiles of the token, 2 x 64 TMEM columns)
 //     TMEM: S^T 64 + dP^T 64 + dK_g/dV_g 256 + dQ^T 128 = 512 columns.
-//   * dK_g / dV_g rows go to dK[s] / dV[s] with fp32 vector atomics (16 bytes per add): several
-//     tokens select the same key, in any order, so those two gradients are summed in fp32 in an
-//     order that is not fixed.  dQ is written once per token (fp32).
+//   * dK_g / dV_g rows go to dK[s] / dV[s] as bulk asynchronous reductions (cp.reduce.async.bulk
+//     add.f32, 256 bytes = 64 columns of one key per operation): each row thread stages its key's
+//     64 columns in its own padded shared-memory row (272-byte stride: conflict-free 16-byte
+//     stores) and hands the row to the bulk-copy unit, which adds whole lines in L2.  Several
+//     tokens select the same key, in any order, so dK and dV are summed in fp32 in an order that
+//     is not fixed.  dQ is written once per token (fp32).
 //   * Warps 0-5 gather the K and V rows of a tile with cp.async (one 512-byte row per warp
 //     instruction, 128B-swizzled), warp 6 allocates TMEM and issues every MMA, warps 7-10 are
 //     the row threads.  One tile is in flight at a time (the V tile's space holds P^T / dS^T).
@@ -52,10 +55,13 @@ constexpr int kProducerWarps = 6;
 constexpr int kMmaWarp = kProducerWarps;
 constexpr int kRowWarp0 = kProducerWarps + 1;
 constexpr int kThreads = 32 * (kProducerWarps + 1 + 4);
-// layout: Q | dO | K tile | V tile (later P^T, dS^T) | index row
+constexpr int kStageCols = 64;                     // fp32 columns per bulk reduction
+constexpr int kStageStride = kStageCols * 4 + 16;  // padded row: 16-byte stores conflict-free
+// layout (no static shared memory, so the dynamic window starts 1024-byte aligned):
+// Q | dO | K tile | V tile (later P^T, dS^T) | reduction staging | barriers and small arrays
 constexpr int kOffQ = 0, kOffDO = kQBytes, kOffK = 2 * kQBytes, kOffV = kOffK + kTileBytes;
-constexpr int kOffIdx = kOffV + kTileBytes;
-constexpr int kSmemBytes = kOffIdx + kMaxK * 4 + 1024;
+constexpr int kOffStage = kOffV + kTileBytes;
+constexpr int kOffMisc = kOffStage + kKeyTile * kStageStride;
 constexpr uint32_t kTmemS = 0, kTmemDP = 64, kTmemKV = 128, kTmemDQ = 384;
 
 struct Params {
@@ -73,7 +79,7 @@ struct Params {
   float scale, scale_log2;
 };
 
-struct __align__(8) Barriers {
+struct __align__(8) Misc {
   uint64_t q_full;    // Q and dO of the token landed (TMA)
   uint64_t k_full, v_full;  // the tile's K / V rows landed (192 producer-thread arrivals)
   uint64_t kv_empty;  // the tile's MMAs are done with the K and V (P^T, dS^T) tiles
@@ -82,7 +88,13 @@ struct __align__(8) Barriers {
   uint64_t dv_ready, dk_ready;  // dV_g / dK_g in TMEM
   uint64_t kv_read;   // the row threads have read the dK_g / dV_g region (twice per tile)
   uint64_t dq_full;   // dQ^T of the token is complete
+  uint32_t tmem_base;
+  int abort_flag;
+  uint32_t mask;      // bit j: tile j holds a valid entry
+  float lse2[kH], D[kH];
 };
+constexpr int kSmemBytes = kOffMisc + (int)sizeof(Misc);
+static_assert(kSmemBytes <= 232448, "shared memory");
 
 __device__ __forceinline__ bool idx_ok(int s, int Lk) { return s >= 0 && s < Lk; }
 
@@ -93,18 +105,27 @@ __device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
   asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+__device__ __forceinline__ void bulk_reduce_add_f32(float* dst, uint32_t src, uint32_t bytes) {
+  asm volatile("cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], %2;" ::"l"(dst), "r"(src),
+               "r"(bytes)
+               : "memory");
+}
 
 __global__ void __launch_bounds__(kThreads, 1)
     dsa_attn_bwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_do,
                         const Params p) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  int32_t* row = reinterpret_cast<int32_t*>(smem + kOffIdx);
-  __shared__ Barriers bar;
-  __shared__ uint32_t tmem_base_sh;
-  __shared__ int abort_flag;
-  __shared__ uint32_t s_mask;  // bit j: tile j holds a valid entry
-  __shared__ float s_lse2[kH], s_D[kH];
+  extern __shared__ __align__(1024) uint8_t smem[];
+  if (smem_u32(smem) & 1023u) {  // the swizzled tiles need 1024-byte alignment (uniform branch)
+    if (threadIdx.x == 0) raise_device_error(p.err, kErrDeviceBounds);
+    return;
+  }
+  Misc& bar = *reinterpret_cast<Misc*>(smem + kOffMisc);
+  uint32_t& tmem_base_sh = bar.tmem_base;
+  int& abort_flag = bar.abort_flag;
+  uint32_t& s_mask = bar.mask;
+  float* s_lse2 = bar.lse2;
+  float* s_D = bar.D;
+  const int32_t* row = p.idx + (size_t)blockIdx.x * p.k;  // the token's index row (global)
 
   const int tok = blockIdx.x;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -128,8 +149,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(&tmem_base_sh, 512);
     tmem_relinquish();
   }
-  // the token's index row, then which 128-entry tiles hold a valid entry
-  for (int e = threadIdx.x; e < k; e += kThreads) row[e] = p.idx[(size_t)tok * k + e];
+  // which 128-entry tiles of the index row hold a valid entry
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -276,6 +296,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     uint8_t* sP = smem + kOffV;
     uint8_t* sDS = smem + kOffV + kPBytes;
+    uint8_t* stage_row = smem + kOffStage + kl * kStageStride;
     uint32_t m = mask;
     for (int t = 0; t < J; ++t) {
       const int j = __ffs(m) - 1;
@@ -323,31 +344,42 @@ __global__ void __launch_bounds__(kThreads, 1)
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(&bar.p_ready);
-      // dV_g, then dK_g: this key's 256 values into dV[s] / dK[s]
+      // dV_g, then dK_g: this key's 256 values added to dV[s] / dK[s], 64 columns per bulk
+      // reduction through the thread's staging row
       for (int which = 0; which < 2; ++which) {
         ok = mbar_wait(which == 0 ? &bar.dv_ready : &bar.dk_ready, t & 1, &abort_flag, p.err) && ok;
         tc_fence_after();
         float* dst = (which == 0 ? p.dV : p.dK) + (kv_row0 + (size_t)(valid ? s_idx : 0)) * kD;
         const float f = which == 0 ? 1.0f : p.scale;
 #pragma unroll 1
-        for (int c0 = 0; c0 < kD; c0 += 32) {
-          uint32_t v[32];
-          tmem_ld32_nowait(tmem + lane_off + kTmemKV + c0, v);
-          tmem_wait_ld_regs(v);
-          if (c0 + 32 == kD) {  // the region may be rewritten once every row thread has read it
+        for (int c0 = 0; c0 < kD; c0 += kStageCols) {
+          uint32_t v0[32], v1[32];
+          tmem_ld32_nowait(tmem + lane_off + kTmemKV + c0, v0);
+          tmem_ld32_nowait(tmem + lane_off + kTmemKV + c0 + 32, v1);
+          tmem_wait_ld_regs2(v0, v1);
+          if (c0 + kStageCols == kD) {  // the region may be rewritten once every row thread has read it
             tc_fence_before();
             mbar_arrive(&bar.kv_read);
           }
           if (valid) {
+            bulk_wait_group_read0();  // this thread's previous reduction has read the row
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
-              atomicAdd(reinterpret_cast<float4*>(dst + c0) + i,
-                        make_float4(f * __uint_as_float(v[4 * i]), f * __uint_as_float(v[4 * i + 1]),
-                                    f * __uint_as_float(v[4 * i + 2]), f * __uint_as_float(v[4 * i + 3])));
+            for (int i = 0; i < 8; ++i) {
+              *reinterpret_cast<float4*>(stage_row + 16 * i) =
+                  make_float4(f * __uint_as_float(v0[4 * i]), f * __uint_as_float(v0[4 * i + 1]),
+                              f * __uint_as_float(v0[4 * i + 2]), f * __uint_as_float(v0[4 * i + 3]));
+              *reinterpret_cast<float4*>(stage_row + 128 + 16 * i) =
+                  make_float4(f * __uint_as_float(v1[4 * i]), f * __uint_as_float(v1[4 * i + 1]),
+                              f * __uint_as_float(v1[4 * i + 2]), f * __uint_as_float(v1[4 * i + 3]));
+            }
+            fence_proxy_async_smem();
+            bulk_reduce_add_f32(dst + c0, smem_u32(stage_row), kStageCols * 4);
+            bulk_commit_group();
           }
         }
       }
     }
+    bulk_wait_group0();  // every reduction of this thread has completed
     // dQ[h, d] = scale * dQ^T[d, h]: this thread's d rows kl and 128 + kl
     float* dq = p.dQ + (size_t)tok * kH * kD;
     if (J > 0) {
