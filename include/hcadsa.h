@@ -352,6 +352,45 @@ hcadsa_status dsa_sparse_attn_bwd(const hcadsa_bf16* Q, const hcadsa_bf16* K, co
                                   float* dQ, float* dK, float* dV, int B, int Lq, int Lk, int Hq, int d, int k,
                                   float scale, hcadsa_stream stream);
 
+/*
+ * Size in bytes of the workspace hca_attn_bwd needs: one fp32 per query row (D = <dO, O>) and
+ * the bf16 probability and score-gradient blocks of every (row tile, key tile) pair,
+ *     B*Lq*Hq*4 (rounded up to 256) + 2 * B*Hkv*n_rt*J * 128*128*2 bytes,
+ * n_rt = ceil(Lq / (128/(Hq/Hkv))) row tiles, J = ceil(n_c(t_last)/128) +
+ * ceil((128/(Hq/Hkv) + W - 1)/128) + 1 key tiles per row tile.  0 for unsupported sizes.
+ */
+size_t hca_attn_bwd_workspace_size(int B, int Lq, int q_offset, int Hq, int Hkv, int d, int n_c, int blk, int W);
+
+/*
+ * Backward of HCA attention.  Source: the forward above (the mirrorspeed page, section "Hybrid
+ * sparse attention, 1/7 full context access": one softmax over a query's visible compressed
+ * entries and raw window positions; 512-wide heads).  For output gradient dO, with the
+ * forward's probabilities p_s = exp(scale <q, k_s> - lse) over the visible set (same reading
+ * of the visible set as hca_attn_fwd):
+ *     D = <dO, O>,  dS_s = p_s (<dO, v_s> - D)
+ *     dQ  = scale sum_s dS_s k_s                                    (written)
+ *     dK_s += scale sum_rows dS_s q,  dV_s += sum_rows p_s dO       (ADDED to; entries s go to
+ *                                                                    dKc/dVc, window rows to dKw/dVw)
+ * P and dS enter the tensor cores as bf16; accumulation is fp32.  Several units add to the same
+ * dK / dV rows with fp32 reductions in no fixed order (last-bit differences between runs).
+ * The entry gradients dKc / dVc feed hca_compress_bwd to reach the raw keys and the weights.
+ *
+ *   Q, O, dO : [B, Lq, Hq, d] bf16 (O and lse from hca_attn_fwd)
+ *   Kc, Vc   : [B, n_c, Hkv, d] bf16 (NULL allowed iff n_c == 0), Kw, Vw: [B, n_w, Hkv, d] bf16
+ *   lse      : [B, Lq, Hq] fp32
+ *   dQ       : [B, Lq, Hq, d] fp32 (written)
+ *   dKc, dVc : [B, n_c, Hkv, d] fp32, dKw, dVw: [B, n_w, Hkv, d] fp32 (accumulated)
+ *   workspace: hca_attn_bwd_workspace_size(...) bytes, 16-byte aligned
+ * Requirements as hca_attn_fwd (d == 512, (Hq/Hkv) divides 128, windows inside the raw buffer,
+ * n_c(t) <= n_c): HCADSA_ERR_SHAPE / _UNSUPPORTED / _WORKSPACE / _ALIGN otherwise.
+ */
+hcadsa_status hca_attn_bwd(const hcadsa_bf16* Q, const hcadsa_bf16* Kc, const hcadsa_bf16* Vc, int n_c,
+                           const hcadsa_bf16* Kw, const hcadsa_bf16* Vw, int win_start, int n_w,
+                           const hcadsa_bf16* O, const hcadsa_bf16* dO, const float* lse, float* dQ, float* dKc,
+                           float* dVc, float* dKw, float* dVw, int B, int Lq, int q_offset, int Hq, int Hkv, int d,
+                           int blk, int W, float scale, void* workspace, size_t workspace_bytes,
+                           hcadsa_stream stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -92,6 +92,11 @@ def lib() -> ctypes.CDLL:
             L.hca_compress_bwd.restype = I
             L.dsa_sparse_attn_bwd.argtypes = [P, P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, F, P]
             L.dsa_sparse_attn_bwd.restype = I
+            L.hca_attn_bwd_workspace_size.argtypes = [I] * 9
+            L.hca_attn_bwd_workspace_size.restype = S
+            L.hca_attn_bwd.argtypes = [P, P, P, I, P, P, I, I, P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, F, P,
+                                       S, P]
+            L.hca_attn_bwd.restype = I
             _lib = L
     return _lib
 
@@ -434,3 +439,55 @@ def dsa_sparse_attn_bwd(Q, K, V, idx, O, dO, lse, *, scale: float | None = None,
                                    _ptr(dK), _ptr(dV), B, Lq, Lk, Hq, d, k, float(scale), _stream(stream))
     _check(st, "dsa_sparse_attn_bwd")
     return dQ, dK, dV
+
+
+def hca_attn_bwd(Q, Kc, Vc, Kw, Vw, O, dO, lse, *, win_start: int = 0, q_offset: int = 0, blk: int = 128,
+                 W: int = 128, scale: float | None = None, dKc=None, dVc=None, dKw=None, dVw=None, workspace=None,
+                 stream=None):
+    """Gradients of the HCA attention: Q, O, dO [B, Lq, Hq, 512] bf16, Kc/Vc [B, n_c, Hkv, 512] (or
+    None), Kw/Vw [B, n_w, Hkv, 512] bf16, lse [B, Lq, Hq] fp32 from the forward ->
+    (dQ fp32 like Q, dKc, dVc fp32 like Kc (None if n_c = 0), dKw, dVw fp32 like Kw); the key and
+    value gradients are added to when given, zeros otherwise."""
+    _need(Q, torch.bfloat16, "Q")
+    B, Lq, Hq, d = Q.shape
+    _need(Kw, torch.bfloat16, "Kw")
+    if Kw.dim() != 4 or Kw.shape[0] != B or Kw.shape[3] != d:
+        raise ValueError(f"Kw has shape {tuple(Kw.shape)}, expected [{B}, n_w, Hkv, {d}]")
+    n_w, Hkv = Kw.shape[1], Kw.shape[2]
+    _need(Vw, torch.bfloat16, "Vw", Kw.shape)
+    n_c = 0 if Kc is None else Kc.shape[1]
+    if n_c:
+        _need(Kc, torch.bfloat16, "Kc", (B, n_c, Hkv, d))
+        _need(Vc, torch.bfloat16, "Vc", (B, n_c, Hkv, d))
+    _need(O, torch.bfloat16, "O", Q.shape)
+    _need(dO, torch.bfloat16, "dO", Q.shape)
+    _need(lse, torch.float32, "lse", (B, Lq, Hq))
+    for t, n, shp in ((dKc, "dKc", (B, n_c, Hkv, d)), (dVc, "dVc", (B, n_c, Hkv, d)), (dKw, "dKw", Kw.shape),
+                      (dVw, "dVw", Kw.shape)):
+        if t is not None:
+            _need(t, torch.float32, n, shp)
+    if workspace is not None and not workspace.is_contiguous():
+        raise ValueError("workspace must be contiguous")
+    _on_device(Q, Kw, Vw, Kc if n_c else None, Vc if n_c else None, O, dO, lse, dKc, dVc, dKw, dVw, workspace)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    dev = Q.device
+    dQ = torch.empty(Q.shape, dtype=torch.float32, device=dev)
+    if n_c:
+        dKc = torch.zeros((B, n_c, Hkv, d), dtype=torch.float32, device=dev) if dKc is None else dKc
+        dVc = torch.zeros((B, n_c, Hkv, d), dtype=torch.float32, device=dev) if dVc is None else dVc
+    dKw = torch.zeros(tuple(Kw.shape), dtype=torch.float32, device=dev) if dKw is None else dKw
+    dVw = torch.zeros(tuple(Kw.shape), dtype=torch.float32, device=dev) if dVw is None else dVw
+    L = lib()
+    ws_bytes = L.hca_attn_bwd_workspace_size(B, Lq, q_offset, Hq, Hkv, d, n_c, blk, W)
+    if workspace is None:
+        if ws_bytes:
+            workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    else:
+        ws_bytes = workspace.numel() * workspace.element_size()
+    st = L.hca_attn_bwd(_ptr(Q), _ptr(Kc) if n_c else None, _ptr(Vc) if n_c else None, n_c, _ptr(Kw), _ptr(Vw),
+                        win_start, n_w, _ptr(O), _ptr(dO), _ptr(lse), _ptr(dQ), _ptr(dKc) if n_c else None,
+                        _ptr(dVc) if n_c else None, _ptr(dKw), _ptr(dVw), B, Lq, q_offset, Hq, Hkv, d, blk, W,
+                        float(scale), _ptr(workspace), ws_bytes, _stream(stream))
+    _check(st, "hca_attn_bwd")
+    return dQ, (dKc if n_c else None), (dVc if n_c else None), dKw, dVw

@@ -103,3 +103,94 @@ def test_dsa_attn_bwd_padding_rows(hd):
     assert torch.count_nonzero(got[0][0, empty]).item() == 0
     for g, r, what in zip(got, ref, ("dQ", "dK", "dV")):
         _check_grad(g, r, what)
+
+
+def _hca_bwd_gpu(hd, Q, Kc, Vc, Kw, Vw, dO, **kw):
+    """Forward (O, lse) then backward on the GPU, over the given cache tensors."""
+    dev = [t.cuda() if t is not None else None for t in (Q, Kc, Vc, Kw, Vw, dO)]
+    Qd, Kcd, Vcd, Kwd, Vwd, dOd = dev
+    O, lse = hd.hca_attn_fwd(Qd, Kcd, Vcd, Kwd, Vwd, return_lse=True, **kw)
+    out = hd.hca_attn_bwd(Qd, Kcd, Vcd, Kwd, Vwd, O, dOd, lse, **kw)
+    hd.hcadsa_check_device_error()
+    return out
+
+
+@pytest.mark.parametrize("B,L,Hq,Hkv,blk,W,sigma", [
+    (1, 600, 16, 1, 128, 128, None),   # the HCA layer's head grouping, 3 entries
+    (2, 700, 8, 2, 64, 96, 1.0),       # 4 heads per K/V head, two sequences, ragged last row tile
+    (1, 300, 2, 2, 16, 64, 1.0),       # one head per K/V head: 128-token row tiles, 3 window tiles
+    (1, 200, 128, 1, 32, 64, 1.0),     # 128 heads per K/V head: one-token row tiles
+    (1, 1200, 4, 1, 4, 128, 1.0),      # 268 entries: 3 entry tiles, dK/dV units over several chunks
+])
+def test_hca_attn_bwd_matches_oracle(hd, B, L, Hq, Hkv, blk, W, sigma):
+    """Every row and every key: dQ, dKc, dVc (compressed entries) and dKw, dVw (raw window keys)
+    against the oracle's fp64 gradients."""
+    cfg = synth.HcaConfig("hbwd", B=B, L=L, Hq=Hq, Hkv=Hkv, blk=blk, W=W, sigma=sigma)
+    x = synth.hca_inputs(cfg, seed=841 + L)
+    w = x["w"].numpy()
+    Kc = torch.as_tensor(oracle.hca_compress(bits(x["K"]), w, blk).view(np.int16)).view(torch.bfloat16)
+    Vc = torch.as_tensor(oracle.hca_compress(bits(x["V"]), w, blk).view(np.int16)).view(torch.bfloat16)
+    g = torch.Generator().manual_seed(842)
+    dO = (torch.randn(B, L, Hq, 512, generator=g) * 0.1).to(torch.bfloat16)
+    dQ, dKc, dVc, dKw, dVw = _hca_bwd_gpu(hd, x["Q"], Kc, Vc, x["K"], x["V"], dO, blk=blk, W=W)
+    ref = oracle.hca_attn_bwd(bits(x["Q"]), bits(Kc), bits(Vc), bits(x["K"]), bits(x["V"]), dO.double().numpy(),
+                              blk=blk, W=W)
+    for got, r, what in zip((dQ, dKc, dVc, dKw, dVw), ref, ("dQ", "dKc", "dVc", "dKw", "dVw")):
+        _check_grad(got, r, what)
+
+
+def test_hca_attn_bwd_chunk_at_offset(hd):
+    """A chunk of 300 query tokens at positions 4000..4299 of two sequences over the entries stored
+    so far and a window buffer that starts at the first query's window."""
+    d, Hq, blk, W, B, Lq, t0 = 512, 16, 128, 128, 2, 300, 4000
+    t_last = t0 + Lq - 1
+    n_c = (t_last - W + 1) // blk
+    ws = t0 - W + 1
+    Kc = synth.normal_bf16((B, n_c, 1, d), 1.0, 851, "K")
+    Vc = synth.normal_bf16((B, n_c, 1, d), 1.0, 851, "V")
+    Kw = synth.normal_bf16((B, t_last + 1 - ws, 1, d), 1.0, 852, "K")
+    Vw = synth.normal_bf16((B, t_last + 1 - ws, 1, d), 1.0, 852, "V")
+    Q = synth.normal_bf16((B, Lq, Hq, d), 1.0, 853, "Q")
+    g = torch.Generator().manual_seed(854)
+    dO = (torch.randn(B, Lq, Hq, d, generator=g) * 0.1).to(torch.bfloat16)
+    got = _hca_bwd_gpu(hd, Q, Kc, Vc, Kw, Vw, dO, win_start=ws, q_offset=t0)
+    ref = oracle.hca_attn_bwd(bits(Q), bits(Kc), bits(Vc), bits(Kw), bits(Vw), dO.double().numpy(), win_start=ws,
+                              q_offset=t0)
+    for gg, r, what in zip(got, ref, ("dQ", "dKc", "dVc", "dKw", "dVw")):
+        _check_grad(gg, r, what)
+
+
+def test_hca_attn_bwd_32k(hd):
+    """The HCA layer's size (L = 32768, 16 heads on one K/V head, 256 entries): dQ of sampled row
+    chunks against the oracle; the raw-key gradients of two window keys exactly (the oracle over
+    the W + 1 query rows that see them); and two sums that hold at any size: the value gradients
+    of all keys add up to the sum of dO over all rows (each row's probabilities sum to 1), and the
+    key gradients to ~0 (each row's dS sums to 0)."""
+    cfg = synth.HCA_32K
+    B, L, Hq, blk, W = cfg.B, cfg.L, cfg.Hq, cfg.blk, cfg.W
+    x = synth.hca_inputs(cfg, seed=861)
+    dev = {n: v.cuda() for n, v in x.items()}
+    Kc, Vc = hd.hca_compress_kv(dev["K"], dev["V"], dev["w"], blk)
+    g = torch.Generator(device="cuda").manual_seed(862)
+    dO = (torch.randn(B, L, Hq, 512, generator=g, device="cuda") * 0.1).to(torch.bfloat16)
+    O, lse = hd.hca_attn_fwd(dev["Q"], Kc, Vc, dev["K"], dev["V"], return_lse=True)
+    dQ, dKc, dVc, dKw, dVw = hd.hca_attn_bwd(dev["Q"], Kc, Vc, dev["K"], dev["V"], O, dO, lse)
+    hd.hcadsa_check_device_error()
+    Kc_h, Vc_h = bits(Kc), bits(Vc)
+    dO_h = dO.cpu()
+    Kb, Vb = bits(x["K"]), bits(x["V"])
+    for r0, n in ((0, 24), (16380, 24), (32744, 24)):
+        ref = oracle.hca_attn_bwd(bits(x["Q"][:, r0:r0 + n]), Kc_h, Vc_h, Kb, Vb,
+                                  dO_h[:, r0:r0 + n].double().numpy(), q_offset=r0)
+        _check_grad(dQ[:, r0:r0 + n], ref[0], f"dQ rows {r0}..")
+    s = 20000  # keys s and s + 1 are seen by the rows s .. s + W exactly
+    ref = oracle.hca_attn_bwd(bits(x["Q"][:, s:s + W + 1]), Kc_h, Vc_h, Kb, Vb,
+                              dO_h[:, s:s + W + 1].double().numpy(), q_offset=s)
+    _check_grad(dKw[:, s:s + 2], ref[3][:, s:s + 2], "dKw keys 20000, 20001")
+    _check_grad(dVw[:, s:s + 2], ref[4][:, s:s + 2], "dVw keys 20000, 20001")
+    sum_dv = (dVc.double().sum(dim=(0, 1, 2)) + dVw.double().sum(dim=(0, 1, 2))).cpu().numpy()
+    sum_do = dO.double().sum(dim=(0, 1, 2)).cpu().numpy()
+    assert np.abs(sum_dv - sum_do).max() <= 1e-2 * np.abs(sum_do).max() + 1e-3, np.abs(sum_dv - sum_do).max()
+    sum_dk = (dKc.double().sum(dim=(0, 1, 2)) + dKw.double().sum(dim=(0, 1, 2))).cpu().numpy()
+    abs_dk = (dKc.double().abs().sum(dim=(0, 1, 2)) + dKw.double().abs().sum(dim=(0, 1, 2))).cpu().numpy()
+    assert np.all(np.abs(sum_dk) <= 1e-2 * abs_dk), (np.abs(sum_dk) / abs_dk).max()
