@@ -468,7 +468,8 @@ def run_hca_latent(hd, device, peaks, iters=10):
 def run_backward(hd, device, peaks, iters=5):
     """Backward kernels at the layer sizes of the step (L = 32768): the DSA sparse attention
     backward (dQ, dK, dV from the forward's O and lse over the top-2048 selection of the step's
-    indexer) and the HCA compressor's adjoint (dX, dw for 512-wide keys, blocks of 128).  CUDA
+    indexer), the HCA compressor's adjoint (dX, dw for 512-wide keys, blocks of 128) and the HCA
+    attention backward (dQ, entry and window dK / dV; 5 * 2 * 512 flop per visible (row, key)).  CUDA
     events, median of `iters` after 3 warm-up runs.  Algorithmic units: 5 * 2 * 256 flop per
     (query, head, selected key) (S, dP, dV, dK, dQ) and 2 KB of fp32 reductions into dK / dV per
     (query, selected key)."""
@@ -513,13 +514,46 @@ def run_backward(hd, device, peaks, iters=5):
     cbytes = L * HCA.Hkv * HCA.d * (2 + 4 + 4) + (L // HCA.blk) * HCA.Hkv * HCA.d * 4
     del Xk, dXc, dX, dw
     torch.cuda.empty_cache()
-    return {"workload": f"dsa_bwd_L{L}_h64_d256_k2048 + compress_bwd_L{L}_d512_blk128 (B=1)", "iters": iters,
+    # HCA attention backward (prep, score blocks, dQ, dK/dV: four launches)
+    h = make_hca_inputs(device, synth.SEED)
+    Kc = torch.empty((1, L // HCA.blk, HCA.Hkv, HCA.d), dtype=torch.bfloat16, device=device)
+    Vc = torch.empty_like(Kc)
+    hd.hca_compress_kv(h["hK"], h["hV"], h["w"], HCA.blk, Kc=Kc, Vc=Vc)
+    hO, hlse = hd.hca_attn_fwd(h["hQ"], Kc, Vc, h["hK"], h["hV"], return_lse=True)
+    hgO = _Draw(device, synth.SEED).normal(tuple(hO.shape), 0.1, 65)
+    hws = torch.empty(hd.lib().hca_attn_bwd_workspace_size(1, L, 0, HCA.Hq, HCA.Hkv, HCA.d, L // HCA.blk, HCA.blk,
+                                                           HCA.W), dtype=torch.uint8, device=device)
+    grads = {}
+
+    def hbwd():
+        return hd.hca_attn_bwd(h["hQ"], Kc, Vc, h["hK"], h["hV"], hO, hgO, hlse, workspace=hws, **grads)
+
+    out = hbwd()
+    grads.update(dKc=out[1], dVc=out[2], dKw=out[3], dVw=out[4])
+    for _ in range(2):
+        hbwd()
+    torch.cuda.synchronize()
+    hevs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(iters)]
+    for i in range(iters):
+        hevs[i][0].record()
+        hbwd()
+        hevs[i][1].record()
+    torch.cuda.synchronize()
+    hms = statistics.median(e[0].elapsed_time(e[1]) for e in hevs)
+    hflop = 10.0 * HCA.d * HCA.Hq * hca_visible_keys_per_head(L)
+    htf = hflop / (hms * 1e-3) / 1e12
+    del h, Kc, Vc, hO, hlse, hgO, hws, grads, out
+    torch.cuda.empty_cache()
+    return {"workload": f"dsa_bwd_L{L}_h64_d256_k2048 + compress_bwd_L{L}_d512_blk128 + hca_bwd_L{L}_hq16_hkv1_d512 "
+                        "(B=1)", "iters": iters,
             "dsa_bwd_ms": ms, "dsa_bwd_tflops": tf, "dsa_bwd_pct_bf16": 100 * tf / peaks["bf16_tflops"],
             "dsa_bwd_reduce_gbs": red_bytes / (ms * 1e-3) / 1e9, "dsa_bwd_algorithmic_flop": flop,
             "dsa_bwd_reduce_bytes": red_bytes,
             "compress_bwd_us": cms * 1e3, "compress_bwd_gbs": cbytes / (cms * 1e-3) / 1e9,
             "compress_bwd_pct_hbm": 100 * cbytes / (cms * 1e-3) / 1e9 / peaks["hbm_gbs"],
-            "compress_bwd_bytes": cbytes}
+            "compress_bwd_bytes": cbytes,
+            "hca_bwd_ms": hms, "hca_bwd_tflops": htf, "hca_bwd_pct_bf16": 100 * htf / peaks["bf16_tflops"],
+            "hca_bwd_algorithmic_flop": hflop}
 
 
 def run_hca_131k(hd, device, peaks, iters=10):
