@@ -13,23 +13,26 @@
 // Kernel design (one CTA per token; the token's 128-key tiles in order):
 //   * Transposed like the forward, keys as M (128 per tile):
 //       S^T  = K_g Q^T,   dP^T = V_g dO^T        (SS, K-major, N = 64 heads, fp32 in TMEM)
-//     the four row warps (thread = key = TMEM lane) form P^T and dS^T (bf16) and write them,
+//     the four softmax warps (thread = key = TMEM lane) form P^T and dS^T (bf16) and write them,
 //     128B-swizzled, over the V tile (whose last reader was the dP^T MMA), then
 //       dV_g = P^T dO,    dK_g = dS^T Q          (A = P^T / dS^T K-major, B = dO / Q MN-major,
 //                                                 N = 256, one 256-column TMEM region in turn)
 //       dQ^T += K_g^T dS^T                       (A = K_g MN-major, B = dS^T MN-major, over all
 //                                                 tiles of the token, 2 x 64 TMEM columns)
 //     TMEM: S^T 64 + dP^T 64 + dK_g/dV_g 256 + dQ^T 128 = 512 columns.
+//   * MMA order per tile: S^T, dP^T | dV_g, dQ^T (the K tile is free) | dK_g (the V tile's space
+//     is free), so the next tile's K rows are gathered while dK_g waits for the read-out of dV_g.
 //   * dK_g / dV_g rows go to dK[s] / dV[s] as bulk asynchronous reductions (cp.reduce.async.bulk
-//     add.f32, 256 bytes = 64 columns of one key per operation): each row thread stages its key's
-//     64 columns in its own padded shared-memory row (272-byte stride: conflict-free 16-byte
-//     stores) and hands the row to the bulk-copy unit, which adds whole lines in L2.  Several
-//     tokens select the same key, in any order, so dK and dV are summed in fp32 in an order that
-//     is not fixed.  dQ is written once per token (fp32).
-//   * Warps 0-5 gather the K and V rows of a tile with cp.async (one 512-byte row per warp
-//     instruction, 128B-swizzled), warp 6 allocates TMEM and issues every MMA, warps 7-10 are
-//     the row threads.  One tile is in flight at a time (the V tile's space holds P^T / dS^T).
-//   * D[h] = <dO[h], O[h]> is computed at the token's start by the row threads.
+//     add.f32, 256 bytes = 64 columns of one key per operation): four reduction warps (thread =
+//     key) stage a key's 64 columns in their own padded shared-memory row (272-byte stride:
+//     conflict-free 16-byte stores) and hand the row to the bulk-copy unit, which adds whole
+//     lines in L2; the softmax warps meanwhile work on the next tile.  Several tokens select the
+//     same key, in any order, so dK and dV are summed in fp32 in an order that is not fixed.
+//     dQ is written once per token (fp32) by the softmax warps.
+//   * Warps 0-2 gather the K and V rows of a tile with cp.async (one 512-byte row per warp
+//     instruction, 128B-swizzled), warp 3 allocates TMEM and issues every MMA, warps 4-7 are the
+//     softmax warps, warps 8-11 the reduction warps.  One K and one V tile are resident.
+//   * D[h] = <dO[h], O[h]> is computed at the token's start by the softmax warps.
 // Every wait is bounded (the library's 2 s limit); on expiry the error word records a timeout
 // and every role leaves its loop.
 #include <cuda_bf16.h>
@@ -51,10 +54,11 @@ constexpr int kQChunkBytes = kH * 128;     // 64 heads x 64 bf16
 constexpr int kQBytes = 4 * kQChunkBytes;  // 32 KB
 constexpr int kPBytes = kKeyTile * 128;    // 128 keys x 64 heads bf16 (16 KB)
 constexpr int kMaxK = 4096;
-constexpr int kProducerWarps = 6;
+constexpr int kProducerWarps = 3;
 constexpr int kMmaWarp = kProducerWarps;
-constexpr int kRowWarp0 = kProducerWarps + 1;
-constexpr int kThreads = 32 * (kProducerWarps + 1 + 4);
+constexpr int kSoftWarp0 = kProducerWarps + 1;  // 4 warps: P^T, dS^T, D, the dQ epilogue
+constexpr int kRedWarp0 = kSoftWarp0 + 4;       // 4 warps: dV_g / dK_g read-out and reductions
+constexpr int kThreads = 32 * (kRedWarp0 + 4);
 constexpr int kStageCols = 64;                     // fp32 columns per bulk reduction
 constexpr int kStageStride = kStageCols * 4 + 16;  // padded row: 16-byte stores conflict-free
 // layout (no static shared memory, so the dynamic window starts 1024-byte aligned):
@@ -82,11 +86,12 @@ struct Params {
 struct __align__(8) Misc {
   uint64_t q_full;    // Q and dO of the token landed (TMA)
   uint64_t k_full, v_full;  // the tile's K / V rows landed (192 producer-thread arrivals)
-  uint64_t kv_empty;  // the tile's MMAs are done with the K and V (P^T, dS^T) tiles
+  uint64_t k_free;    // the tile's MMAs are done with the K tile (after dQ^T)
+  uint64_t v_free;    // ... and with the V tile's space (P^T, dS^T: after dK_g)
   uint64_t s_ready;   // S^T and dP^T are in TMEM
   uint64_t p_ready;   // P^T and dS^T are in shared memory (128 row threads)
   uint64_t dv_ready, dk_ready;  // dV_g / dK_g in TMEM
-  uint64_t kv_read;   // the row threads have read the dK_g / dV_g region (twice per tile)
+  uint64_t kv_read;   // the reduction warps have read the dK_g / dV_g region (twice per tile)
   uint64_t dq_full;   // dQ^T of the token is complete
   uint32_t tmem_base;
   int abort_flag;
@@ -134,7 +139,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&bar.q_full, 1);
     mbar_init(&bar.k_full, kProducerWarps * 32);
     mbar_init(&bar.v_full, kProducerWarps * 32);
-    mbar_init(&bar.kv_empty, 1);
+    mbar_init(&bar.k_free, 1);
+    mbar_init(&bar.v_free, 1);
     mbar_init(&bar.s_ready, 1);
     mbar_init(&bar.p_ready, 128);
     mbar_init(&bar.dv_ready, 1);
@@ -168,23 +174,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ producers (cp.async rows)
     const uint32_t sK = smem_u32(smem + kOffK), sV = smem_u32(smem + kOffV);
     const int chunk = lane >> 3, piece = lane & 7;
-    const int n_rows_w = (kKeyTile - warp + kProducerWarps - 1) / kProducerWarps;
+    const int n_rows_w = (kKeyTile - warp + kProducerWarps - 1) / kProducerWarps;  // 43 or 42
     bool ok = true;
     uint32_t m = mask;
     for (int t = 0; t < J && ok; ++t) {
       const int j = __ffs(m) - 1;
       m &= m - 1;
-      if (t > 0) {  // both tiles' space is free once the previous tile's MMAs are done
-        ok = __all_sync(0xffffffffu, mbar_wait(&bar.kv_empty, (t - 1) & 1, &abort_flag, p.err));
-        if (!ok) break;
-      }
       // lane l holds the K/V row of the warp's l-th and (32 + l)-th rows
       const int ea = j * kKeyTile + warp + kProducerWarps * lane;
       const int eb = j * kKeyTile + warp + kProducerWarps * (32 + lane);
-      const int sa = ea < k ? row[ea] : -1;
+      const int sa = (lane < n_rows_w && ea < k) ? row[ea] : -1;
       const int sb = (32 + lane < n_rows_w && eb < k) ? row[eb] : -1;
       const int ra = idx_ok(sa, Lk) ? sa : 0, rb = idx_ok(sb, Lk) ? sb : 0;
-      for (int part = 0; part < 2; ++part) {
+      for (int part = 0; part < 2 && ok; ++part) {
+        if (t > 0) {  // the previous tile's K (after dQ^T) / V space (after dK_g) is free
+          ok = __all_sync(0xffffffffu, mbar_wait(part == 0 ? &bar.k_free : &bar.v_free, (t - 1) & 1, &abort_flag,
+                                                 p.err));
+          if (!ok) break;
+        }
         const uint16_t* base = (part == 0 ? p.K : p.V) + kv_row0 * kD + lane * 8;
         const uint32_t dst0 = (part == 0 ? sK : sV) + chunk * kChunkBytes;
 #pragma unroll 4
@@ -233,8 +240,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         tc_fence_after();
         // dV_g = P^T dO (K = 64 heads): A = P^T rows of 64 heads; B = dO as [heads x d], d in
-        // four 64-wide groups 8 KB apart
-        if (t > 0) {  // the row threads have read the previous tile's dK_g
+        // four 64-wide groups 8 KB apart.  The region must have been read out (dK_g of t - 1).
+        if (t > 0) {
           ok = mbar_wait(&bar.kv_read, 1, &abort_flag, p.err);
           if (!ok) break;
           tc_fence_after();
@@ -244,31 +251,33 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_ss(tmem + kTmemKV, smem_desc_sw128(sP + kk * 32, 16, 1024),
                  smem_desc_sw128(sDO + kk * 2048, kQChunkBytes, 1024), idesc_kv, kk > 0);
         mma_commit(&bar.dv_ready);
-        ok = mbar_wait(&bar.kv_read, 0, &abort_flag, p.err);  // dV_g read out
-        if (!ok) break;
-        tc_fence_after();
-        // dK_g = dS^T Q (the scale is applied when it is added to dK)
-#pragma unroll
-        for (int kk = 0; kk < kH / 16; ++kk)
-          mma_ss(tmem + kTmemKV, smem_desc_sw128(sDS + kk * 32, 16, 1024),
-                 smem_desc_sw128(sQ + kk * 2048, kQChunkBytes, 1024), idesc_kv, kk > 0);
-        mma_commit(&bar.dk_ready);
-        // dQ^T += K_g^T dS^T: d in two halves of 128 rows (K chunks 2hv, 2hv+1), keys as K
+        // dQ^T += K_g^T dS^T: d in two halves of 128 rows (K chunks 2hv, 2hv+1), keys as K; the
+        // K tile is free once these are done
 #pragma unroll
         for (int hv = 0; hv < 2; ++hv)
 #pragma unroll
           for (int kk = 0; kk < kKeyTile / 16; ++kk)
             mma_ss(tmem + kTmemDQ + hv * kH, smem_desc_sw128(sK + hv * 2 * kChunkBytes + kk * 2048, kChunkBytes, 1024),
                    smem_desc_sw128(sDS + kk * 2048, kPBytes, 1024), idesc_q, (t > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(&bar.kv_empty);
+        mma_commit(&bar.k_free);
+        ok = mbar_wait(&bar.kv_read, 0, &abort_flag, p.err);  // dV_g read out
+        if (!ok) break;
+        tc_fence_after();
+        // dK_g = dS^T Q (the scale is applied when it is added to dK); then the V space is free
+#pragma unroll
+        for (int kk = 0; kk < kH / 16; ++kk)
+          mma_ss(tmem + kTmemKV, smem_desc_sw128(sDS + kk * 32, 16, 1024),
+                 smem_desc_sw128(sQ + kk * 2048, kQChunkBytes, 1024), idesc_kv, kk > 0);
+        mma_commit(&bar.dk_ready);
+        mma_commit(&bar.v_free);
         if (t == J - 1) mma_commit(&bar.dq_full);
       }
     }
-  } else {
-    // ------------------------------------------------------------ row threads
+  } else if (warp < kRedWarp0) {
+    // ------------------------------------------------------------ softmax warps (thread = key)
     const int quarter = warp & 3;
     const int kl = quarter * 32 + lane;  // key of a tile == TMEM lane; d row of dQ^T
-    const int tid = (warp - kRowWarp0) * 32 + lane;  // 0..127
+    const int tid = (warp - kSoftWarp0) * 32 + lane;  // 0..127
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     // D[h] = <dO[h], O[h]> and lse in log2 units; two threads per head, 128 columns each
     {
@@ -296,7 +305,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     uint8_t* sP = smem + kOffV;
     uint8_t* sDS = smem + kOffV + kPBytes;
-    uint8_t* stage_row = smem + kOffStage + kl * kStageStride;
     uint32_t m = mask;
     for (int t = 0; t < J; ++t) {
       const int j = __ffs(m) - 1;
@@ -344,8 +352,44 @@ __global__ void __launch_bounds__(kThreads, 1)
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(&bar.p_ready);
-      // dV_g, then dK_g: this key's 256 values added to dV[s] / dK[s], 64 columns per bulk
-      // reduction through the thread's staging row
+    }
+    // dQ[h, d] = scale * dQ^T[d, h]: this thread's d rows kl and 128 + kl
+    float* dq = p.dQ + (size_t)tok * kH * kD;
+    if (J > 0) {
+      ok = mbar_wait(&bar.dq_full, 0, &abort_flag, p.err) && ok;
+      tc_fence_after();
+    }
+#pragma unroll 1
+    for (int hv = 0; hv < 2; ++hv) {
+      uint32_t v0[32], v1[32];
+      if (J > 0) {
+        tmem_ld32_nowait(tmem + lane_off + kTmemDQ + hv * kH, v0);
+        tmem_ld32_nowait(tmem + lane_off + kTmemDQ + hv * kH + 32, v1);
+        tmem_wait_ld_regs2(v0, v1);
+      }
+#pragma unroll
+      for (int h = 0; h < kH; ++h) {
+        const float x = J > 0 ? __uint_as_float(h < 32 ? v0[h] : v1[h - 32]) * p.scale : 0.0f;
+        dq[(size_t)h * kD + hv * 128 + kl] = x;
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ reduction warps (thread = key)
+    // dV_g, then dK_g: this key's 256 values added to dV[s] / dK[s], 64 columns per bulk
+    // reduction through the thread's staging row, while the softmax warps and the tensor cores
+    // go on with the next tile
+    const int quarter = warp & 3;
+    const int kl = quarter * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    uint8_t* stage_row = smem + kOffStage + kl * kStageStride;
+    bool ok = true;
+    uint32_t m = mask;
+    for (int t = 0; t < J; ++t) {
+      const int j = __ffs(m) - 1;
+      m &= m - 1;
+      const int e = j * kKeyTile + kl;
+      const int s_idx = e < k ? row[e] : -1;
+      const bool valid = idx_ok(s_idx, Lk);
       for (int which = 0; which < 2; ++which) {
         ok = mbar_wait(which == 0 ? &bar.dv_ready : &bar.dk_ready, t & 1, &abort_flag, p.err) && ok;
         tc_fence_after();
@@ -357,7 +401,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld32_nowait(tmem + lane_off + kTmemKV + c0, v0);
           tmem_ld32_nowait(tmem + lane_off + kTmemKV + c0 + 32, v1);
           tmem_wait_ld_regs2(v0, v1);
-          if (c0 + kStageCols == kD) {  // the region may be rewritten once every row thread has read it
+          if (c0 + kStageCols == kD) {  // the region may be rewritten once every thread has read it
             tc_fence_before();
             mbar_arrive(&bar.kv_read);
           }
@@ -380,26 +424,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     bulk_wait_group0();  // every reduction of this thread has completed
-    // dQ[h, d] = scale * dQ^T[d, h]: this thread's d rows kl and 128 + kl
-    float* dq = p.dQ + (size_t)tok * kH * kD;
-    if (J > 0) {
-      ok = mbar_wait(&bar.dq_full, 0, &abort_flag, p.err) && ok;
-      tc_fence_after();
-    }
-#pragma unroll 1
-    for (int hv = 0; hv < 2; ++hv) {
-      uint32_t v0[32], v1[32];
-      if (J > 0) {
-        tmem_ld32_nowait(tmem + lane_off + kTmemDQ + hv * kH, v0);
-        tmem_ld32_nowait(tmem + lane_off + kTmemDQ + hv * kH + 32, v1);
-        tmem_wait_ld_regs2(v0, v1);
-      }
-#pragma unroll
-      for (int h = 0; h < kH; ++h) {
-        const float x = J > 0 ? __uint_as_float(h < 32 ? v0[h] : v1[h - 32]) * p.scale : 0.0f;
-        dq[(size_t)h * kD + hv * 128 + kl] = x;
-      }
-    }
   }
 
   tc_fence_before();

@@ -110,6 +110,8 @@ __device__ __forceinline__ int levels_for(uint32_t width) {
 }
 
 __device__ __forceinline__ void rows_bar() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+// Named barrier of the two row warps that share TMEM lane quarter q (ids 2..5).
+__device__ __forceinline__ void pair_bar(int q) { asm volatile("bar.sync %0, 64;" ::"r"(2 + q) : "memory"); }
 // Named barrier over the 256 row threads that also ANDs a predicate across them.
 __device__ __forceinline__ bool rows_bar_and(bool pred) {
   uint32_t r;
@@ -440,14 +442,54 @@ __global__ void __launch_bounds__(kThreads, 1)
         RowWriter wr;
         wr.init(out, vec);
         int eq_seen = 0, taken = 0;
+        // emit: bit i of gt / eq = key s0 + i is a candidate above / equal to the threshold
+        auto masks = [&](const int (&sc)[32], int s0, uint32_t& gt, uint32_t& eq) {
+          const int lim = n - s0;
+          gt = eq = 0u;
+          if (mode < 2 || lim <= 0) return;
+          uint32_t gt4[4] = {0u, 0u, 0u, 0u}, eq4[4] = {0u, 0u, 0u, 0u};  // four independent chains
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            gt4[i & 3] |= (uint32_t)(sc[i] > thr) << i;
+            eq4[i & 3] |= (uint32_t)(sc[i] == thr) << i;
+          }
+          const uint32_t inr = lim >= 32 ? 0xffffffffu : ((1u << lim) - 1u);
+          gt = (gt4[0] | gt4[1] | gt4[2] | gt4[3]) & inr;
+          eq = (eq4[0] | eq4[1] | eq4[2] | eq4[3]) & inr;
+        };
+        // emit, in key order: the keys above the threshold and the lowest-positioned equal ones
+        // until need_eq of them are in
+        auto take = [&](uint32_t gt, uint32_t eq, int s0) {
+          const int ne = __popc(eq);
+          if (eq_seen + ne > need_eq) {
+            uint32_t keep = 0, e = eq;
+            for (int q = eq_seen; q < need_eq; ++q) {
+              keep |= e & (0u - e);  // lowest remaining set bit
+              e &= e - 1;
+            }
+            eq = keep;
+          }
+          eq_seen += ne;
+          uint32_t sel = gt | eq;
+          while (sel && taken < k) {  // ascending positions
+            wr.put(s0 + __ffs(sel) - 1);
+            sel &= sel - 1;
+            ++taken;
+          }
+        };
         // the pass's work on 32 consecutive scores of this row, keys s0 .. s0 + 31
         auto consume = [&](const int (&sc)[32], int s0) {
           const int lim = n - s0;  // keys s0 + i with i < lim are candidates of the row
           if (!emit) {
             if (!done) {
-              if (pass == 0) {
-                // every score of the first level lies in [lo, hi]: count it (keys past the row's
-                // candidates go to the discard bin kBins), no branches
+              if (pass == 0 && lim >= 32) {
+                // every score lies in the exact bounds [lo, hi] and every key is a candidate:
+                // count it in its bin, nothing to check
+                uint32_t* hr = hist + r;
+#pragma unroll
+                for (int i = 0; i < 32; ++i) atomicAdd(hr + (((uint32_t)sc[i] - (uint32_t)lo) >> shift) * kRows, 1u);
+              } else if (pass == 0) {
+                // the row's last keys: those past its candidates go to the discard bin kBins
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
                   const uint32_t u = (uint32_t)sc[i] - (uint32_t)lo;
@@ -462,39 +504,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
               }
             }
-          } else if (mode >= 2 && lim > 0) {
-            // bit i: key s0 + i is above the threshold / equal to it (four independent chains)
-            uint32_t gt4[4] = {0u, 0u, 0u, 0u}, eq4[4] = {0u, 0u, 0u, 0u};
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              gt4[i & 3] |= (uint32_t)(sc[i] > thr) << i;
-              eq4[i & 3] |= (uint32_t)(sc[i] == thr) << i;
-            }
-            const uint32_t inr = lim >= 32 ? 0xffffffffu : ((1u << lim) - 1u);
-            const uint32_t gt = (gt4[0] | gt4[1] | gt4[2] | gt4[3]) & inr;
-            uint32_t eq = (eq4[0] | eq4[1] | eq4[2] | eq4[3]) & inr;
-            // equal scores are taken from the lowest positions until need_eq of them are in
-            const int ne = __popc(eq);
-            if (eq_seen + ne > need_eq) {
-              uint32_t keep = 0, e = eq;
-              for (int q = eq_seen; q < need_eq; ++q) {
-                keep |= e & (0u - e);  // lowest remaining set bit
-                e &= e - 1;
-              }
-              eq = keep;
-            }
-            eq_seen += ne;
-            uint32_t sel = gt | eq;
-            while (sel && taken < k) {  // ascending positions
-              wr.put(s0 + __ffs(sel) - 1);
-              sel &= sel - 1;
-              ++taken;
-            }
+          } else {
+            uint32_t gt, eq;
+            masks(sc, s0, gt, eq);
+            take(gt, eq, s0);
           }
         };
         // TMEM chunks of this pass: one per 256-key stage (single accumulator), or four of 64 keys
         const int chunks = single ? n_stages : n_stages * (kStageKeys / kSub);
-        const bool active = !emit || half == 0;  // the emit pass is half 0's alone (key order)
+        // the emit pass of per-head accumulators is half 0's alone (key order); with one
+        // accumulator half 1 forms the bit masks of the chunk's second 128 keys for half 0
+        const bool active = !emit || half == 0 || single;
         for (int c = 0; c < chunks; ++c, ++g) {
           const uint32_t buf = g % kBufs;
           ok = mbar_wait(&bar.tfull[buf], (g / kBufs) & 1, &abort_flag, p.err) && ok;
@@ -504,10 +524,44 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_arrive(&bar.tempty[buf]);
             continue;
           }
-          if (single) {
-            // 256 scores of keys c*256 .. c*256+255, 64 at a time: all four groups in the emit
-            // pass, groups 2 half .. 2 half + 1 in the histogram passes
-            const int q0 = emit ? 0 : 2 * half, q1 = emit ? 4 : 2 * half + 2;
+          if (single && emit) {
+            // 256 scores of keys c*256 .. c*256+255: half 0 takes keys 0..127 in order, half 1
+            // turns keys 128..255 into bit masks (shared memory, two buffers by chunk parity);
+            // the two warps of a lane quarter meet once per chunk, then half 0 takes the rest
+            uint32_t* mk = hist + (c & 1) * 8 * kRows + r;  // [buffer][word][row]
+#pragma unroll 1
+            for (int q = 2 * half; q < 2 * half + 2; ++q) {
+              uint32_t v0[32], v1[32];
+              const uint32_t ta = tmem + lane_off + buf * 256 + q * 64;
+              tmem_ld32_nowait(ta, v0);
+              tmem_ld32_nowait(ta + 32, v1);
+              tmem_wait_ld_regs2(v0, v1);
+              if (q == 2 * half + 1) {
+                tc_fence_before();
+                mbar_arrive(&bar.tempty[buf]);
+              }
+              const int s0 = c * kStageKeys + q * 64;
+              uint32_t gt0, eq0, gt1, eq1;
+              masks(reinterpret_cast<const int(&)[32]>(v0), s0, gt0, eq0);
+              masks(reinterpret_cast<const int(&)[32]>(v1), s0 + 32, gt1, eq1);
+              if (half == 0) {
+                take(gt0, eq0, s0);
+                take(gt1, eq1, s0 + 32);
+              } else {
+                const int w0 = (q - 2) * 2;
+                mk[w0 * kRows] = gt0;
+                mk[(w0 + 1) * kRows] = gt1;
+                mk[(4 + w0) * kRows] = eq0;
+                mk[(5 + w0) * kRows] = eq1;
+              }
+            }
+            pair_bar(quarter);
+            if (half == 0)
+#pragma unroll 1
+              for (int w4 = 0; w4 < 4; ++w4) take(mk[w4 * kRows], mk[(4 + w4) * kRows], c * kStageKeys + 128 + 32 * w4);
+          } else if (single) {
+            // 256 scores of keys c*256 .. c*256+255, 64 at a time: groups 2 half .. 2 half + 1
+            const int q0 = 2 * half, q1 = 2 * half + 2;
 #pragma unroll 1
             for (int q = q0; q < q1; ++q) {
               uint32_t v0[32], v1[32];
