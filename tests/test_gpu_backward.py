@@ -194,3 +194,51 @@ def test_hca_attn_bwd_32k(hd):
     sum_dk = (dKc.double().sum(dim=(0, 1, 2)) + dKw.double().sum(dim=(0, 1, 2))).cpu().numpy()
     abs_dk = (dKc.double().abs().sum(dim=(0, 1, 2)) + dKw.double().abs().sum(dim=(0, 1, 2))).cpu().numpy()
     assert np.all(np.abs(sum_dk) <= 1e-2 * abs_dk), (np.abs(sum_dk) / abs_dk).max()
+
+
+def test_dsa_attn_bwd_two_sequences(hd):
+    """Two sequences with their own K/V: gradients land in each sequence's own dK / dV rows."""
+    B, Lq, Lk, k = 2, 48, 1500, 512
+    cfg = synth.DsaConfig("bwdb2", B=B, L=Lk, Hq=64, k=k, sigma=1.0)
+    x = synth.dsa_inputs(cfg, seed=871)
+    Q = x["Q"][:, :Lq].contiguous()
+    idx = np.stack([_random_rows(Lq, Lk, k, 872 + b) for b in range(B)])
+    g = torch.Generator().manual_seed(873)
+    dO = (torch.randn(B, Lq, 64, 256, generator=g) * 0.1).to(torch.bfloat16)
+    Qd, Kd, Vd, idd = Q.cuda(), x["K"].cuda(), x["V"].cuda(), torch.as_tensor(idx).cuda()
+    O, lse = hd.dsa_sparse_attn_fwd(Qd, Kd, Vd, idd, return_lse=True)
+    got = hd.dsa_sparse_attn_bwd(Qd, Kd, Vd, idd, O, dO.cuda(), lse)
+    hd.hcadsa_check_device_error()
+    ref = oracle.dsa_attn_bwd(bits(Q), bits(x["K"]), bits(x["V"]), idx, dO.double().numpy())
+    for gg, r, what in zip(got, ref, ("dQ", "dK", "dV")):
+        _check_grad(gg, r, what)
+
+
+def test_dsa_attn_bwd_index_out_of_range_is_reported(hd):
+    """An index entry >= Lk: the backward skips it (no read or reduction outside K/V and dK/dV),
+    records HCADSA_ERR_DEVICE_BOUNDS, and the gradients are those of the other entries (the
+    forward skips the same entries)."""
+    Lq, Lk, k = 40, 600, 256
+    cfg = synth.DsaConfig("bwdoob", B=1, L=Lk, Hq=64, k=k, sigma=1.0)
+    x = synth.dsa_inputs(cfg, seed=881)
+    Q = x["Q"][:, :Lq].contiguous()
+    idx = _random_rows(Lq, Lk, k, 882)
+    bad = idx.copy()
+    bad[0, 5] = Lk
+    bad[7, 200] = Lk + 999
+    bad[39, 255] = 2 ** 30
+    g = torch.Generator().manual_seed(883)
+    dO = (torch.randn(1, Lq, 64, 256, generator=g) * 0.1).to(torch.bfloat16)
+    Qd, Kd, Vd = Q.cuda(), x["K"].cuda(), x["V"].cuda()
+    idd = torch.as_tensor(bad).reshape(1, Lq, k).cuda()
+    hd.hcadsa_check_device_error()  # start from a clear error word
+    O, lse = hd.dsa_sparse_attn_fwd(Qd, Kd, Vd, idd, return_lse=True)
+    got = hd.dsa_sparse_attn_bwd(Qd, Kd, Vd, idd, O, dO.cuda(), lse)
+    with pytest.raises(hd.HcaDsaError) as e:
+        hd.hcadsa_check_device_error()
+    assert e.value.status == -8
+    hd.hcadsa_check_device_error()  # reading the word cleared it
+    skipped = np.where(bad >= Lk, -1, bad).reshape(1, Lq, k)
+    ref = oracle.dsa_attn_bwd(bits(Q), bits(x["K"]), bits(x["V"]), skipped, dO.double().numpy())
+    for gg, r, what in zip(got, ref, ("dQ", "dK", "dV")):
+        _check_grad(gg, r, what)
