@@ -50,13 +50,14 @@ constexpr int kScoreStages = 3;
 constexpr int kScoreStageBytes = 4 * kChunkBytes;  // Q, dO, K, V chunks
 constexpr int kGemmStages = 2;
 constexpr int kGemmABytes = kTile * 64 * 2;        // 16 KB
-constexpr int kGemmBBytes = 64 * kD * 2;           // 64 KB: 64 K-rows x 512
-constexpr int kGemmStageBytes = kGemmABytes + kGemmBBytes;
-constexpr int kStageRow = kD / 2 * 4 + 16;         // epilogue staging row: 256 fp32 + pad
+constexpr int kGemmBHalfBytes = 64 * (kD / 2) * 2;  // 32 KB: 64 K-rows x 256 columns
+constexpr int kGemmStageBytes = kGemmABytes + 2 * kGemmBHalfBytes;  // whole 512 columns
+constexpr int kStageCols = 128;                    // epilogue: fp32 columns per bulk operation
+constexpr int kStageRow = kStageCols * 4 + 16;     // staging row: 128 fp32 + pad (conflict free)
 constexpr int kChunkRows = 16;                     // row tiles per dK / dV unit
 constexpr uint32_t kBlockElems = kTile * kTile;
 
-static_assert(kTile * kStageRow <= kGemmStages * kGemmStageBytes, "staging fits in the ring");
+static_assert(kTile * kStageRow <= kGemmStages * (kGemmABytes + kGemmBHalfBytes), "staging fits in the ring");
 
 // Geometry of one call (same for every (b, kv)).
 struct Geo {
@@ -319,7 +320,8 @@ struct GemmMaps {
 
 struct GemmParams {
   Geo G;
-  int mode;  // 0: dQ units (one per row tile); 1: dK / dV units (key tile x row-tile chunk)
+  int mode;  // 0: dQ units (one per row tile and 256-column half); 1: dK / dV units (key tile x
+             // row-tile chunk, all 512 columns)
   int bh, bt;
   float* dQ;   // [B, Lq, Hq, 512] fp32 (written)
   float* dKc;  // [B, n_c, Hkv, 512] fp32 (added to)
@@ -340,7 +342,7 @@ struct __align__(8) GemmBars {
 // chunk that see key tile kt (entries: kt < E_i; window: mlo <= m <= mhi).
 struct Unit {
   int bkv, b, kv;
-  int grad;     // dK / dV units: 0 = dK, 1 = dV
+  int grad;     // dK / dV units: 0 = dK, 1 = dV; dQ units: the 256-column half
   bool entry;   // dK / dV units: entry key tile (else a window key tile)
   int tile;     // dQ: row tile; dK / dV: entry tile e or window tile m
   int i0, i1;   // dK / dV: row-tile range of the chunk
@@ -349,6 +351,8 @@ struct Unit {
     entry = false;
     i0 = i1 = 0;
     if (mode == 0) {
+      grad = u & 1;
+      u >>= 1;
       tile = u % G.n_rt;
       bkv = u / G.n_rt;
     } else {
@@ -404,7 +408,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0) raise_device_error(p.err, kErrDeviceBounds);
     return;
   }
-  GemmBars& bar = *reinterpret_cast<GemmBars*>(smem + kGemmStages * kGemmStageBytes);
+  // dQ: one 256-column half per CTA (two CTAs per SM); dK / dV: both halves
+  const int nh = p.mode == 0 ? 1 : 2;
+  const int stage_bytes = kGemmABytes + nh * kGemmBHalfBytes;
+  GemmBars& bar = *reinterpret_cast<GemmBars*>(smem + kGemmStages * stage_bytes);
   const Geo& G = p.G;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   Unit U;
@@ -432,13 +439,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_mbarrier_init();
   }
   if (warp == 1) {
-    tmem_alloc(&bar.tmem_base, 512);
+    tmem_alloc(&bar.tmem_base, nh * 256);
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bar.tmem_base;
+  const int c_first = p.mode == 0 ? U.grad * 4 : 0;  // first 64-column box of B
 
   if (warp == 0) {
     if (lane == 0) {
@@ -467,13 +475,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int s = cnt % kGemmStages;
           ok = mbar_wait(&bar.empty[s], ((cnt / kGemmStages) & 1) ^ 1, &bar.abort_flag, p.err);
           if (!ok) break;
-          uint8_t* sa = smem + s * kGemmStageBytes;
+          uint8_t* sa = smem + s * stage_bytes;
           uint8_t* sb = sa + kGemmABytes;
-          mbar_arrive_expect_tx(&bar.full[s], kGemmStageBytes);
+          mbar_arrive_expect_tx(&bar.full[s], stage_bytes);
           if (p.mode == 0) {
             tma_load_2d(sa, &maps.dsK, &bar.full[s], hf * 64, row0);
-            for (int c = 0; c < kD / 64; ++c)
-              tma_load_4d(sb + c * 8192, mb, &bar.full[s], c * 64, U.kv, key0 + hf * 64, U.b);
+            for (int c = 0; c < 4; ++c)
+              tma_load_4d(sb + c * 8192, mb, &bar.full[s], (c_first + c) * 64, U.kv, key0 + hf * 64, U.b);
           } else {
             const CUtensorMap* ma = U.grad == 0 ? &maps.dsM : &maps.pM;
             tma_load_2d(sa, ma, &bar.full[s], 0, row0 + hf * 64);
@@ -497,13 +505,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           ok = mbar_wait(&bar.full[s], (cnt / kGemmStages) & 1, &bar.abort_flag, p.err);
           if (!ok) break;
           tc_fence_after();
-          const uint32_t sa = smem_u32(smem + s * kGemmStageBytes), sb = sa + kGemmABytes;
+          const uint32_t sa = smem_u32(smem + s * stage_bytes), sb = sa + kGemmABytes;
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
             const uint64_t da = p.mode == 0 ? smem_desc_sw128(sa + kk * 32, 16, 1024)
                                             : smem_desc_sw128(sa + kk * 2048, 8192, 1024);
-#pragma unroll
-            for (int n = 0; n < 2; ++n)
+            for (int n = 0; n < nh; ++n)
               mma_ss(tmem + n * 256, da, smem_desc_sw128(sb + n * 4 * 8192 + kk * 2048, 8192, 1024), idesc,
                      (jb | hf | kk) != 0 ? 1u : 0u);
           }
@@ -513,8 +520,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (ok) mma_commit(&bar.tfull);
     }
   } else {
-    // epilogue: thread = output row (TMEM lane); each 256-column half staged and handed to
-    // the bulk-copy unit as one 1 KB row
+    // epilogue: thread = output row (TMEM lane); 128 columns at a time staged and handed to the
+    // bulk-copy unit as one 512-byte row
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
@@ -538,14 +545,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       f = U.grad == 0 ? G.scale : 1.0f;
     }
     uint8_t* srow = smem + r * kStageRow;
+    const int col0 = p.mode == 0 ? U.grad * 256 : 0;  // output column of TMEM column 0
     if (ok) {
 #pragma unroll 1
-      for (int n = 0; n < 2; ++n) {
+      for (int n = 0; n < nh * 256; n += kStageCols) {
         if (n > 0) bulk_wait_group_read0();
 #pragma unroll 1
-        for (int c0 = 0; c0 < kD / 2; c0 += 32) {
+        for (int c0 = 0; c0 < kStageCols; c0 += 32) {
           uint32_t v[32];
-          tmem_ld32_nowait(tmem + lane_off + n * 256 + c0, v);
+          tmem_ld32_nowait(tmem + lane_off + n + c0, v);
           tmem_wait_ld_regs(v);
 #pragma unroll
           for (int q = 0; q < 8; ++q)
@@ -556,9 +564,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (dst) {
           fence_proxy_async_smem();
           if (p.mode == 0)
-            bulk_store(dst + n * 256, smem_u32(srow), kD / 2 * 4);
+            bulk_store(dst + col0 + n, smem_u32(srow), kStageCols * 4);
           else
-            bulk_reduce_add_f32(dst + n * 256, smem_u32(srow), kD / 2 * 4);
+            bulk_reduce_add_f32(dst + col0 + n, smem_u32(srow), kStageCols * 4);
           bulk_commit_group();
         }
       }
@@ -567,7 +575,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) tmem_dealloc(tmem, 512);
+  if (warp == 1) tmem_dealloc(tmem, nh * 256);
 }
 
 // ------------------------------------------------------------------------------------ host side
@@ -739,11 +747,12 @@ extern "C" hcadsa_status hca_attn_bwd(const hcadsa_bf16* Q, const hcadsa_bf16* K
   gp.dVw = dVw;
   gp.err = err;
   const int gemm_smem = kGemmStages * kGemmStageBytes + (int)sizeof(GemmBars);
+  const int gemm_smem_half = kGemmStages * (kGemmABytes + kGemmBHalfBytes) + (int)sizeof(GemmBars);
   if (cudaFuncSetAttribute(hca_bwd_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, gemm_smem) !=
       cudaSuccess)
     return launch_status();
-  gp.mode = 0;
-  hca_bwd_gemm_kernel<<<(unsigned)n_score, kThreads, gemm_smem, s>>>(gm, gp);
+  gp.mode = 0;  // two units per row tile (column halves), two CTAs per SM
+  hca_bwd_gemm_kernel<<<(unsigned)(2 * n_score), kThreads, gemm_smem_half, s>>>(gm, gp);
   st = launch_status();
   if (st != HCADSA_OK) return st;
   gp.mode = 1;
