@@ -242,3 +242,33 @@ def test_dsa_attn_bwd_index_out_of_range_is_reported(hd):
     ref = oracle.dsa_attn_bwd(bits(Q), bits(x["K"]), bits(x["V"]), skipped, dO.double().numpy())
     for gg, r, what in zip(got, ref, ("dQ", "dK", "dV")):
         _check_grad(gg, r, what)
+
+
+def test_dsa_attn_bwd_32k(hd):
+    """The MLA-DSA layer's size (L = 32768, 64 heads of 256, top-2048 from the fused indexer):
+    dQ of sampled query rows against the oracle (a row's dQ depends only on that row), and two
+    sums that hold at any size: the value gradients of all keys add up to the sum of dO over all
+    rows with a selection (each row's probabilities sum to 1), and the key gradients to ~0."""
+    cfg = synth.DSA_32K
+    B, L, k = cfg.B, cfg.L, cfg.k
+    x = synth.dsa_inputs(cfg, seed=891)
+    dev = {n: v.cuda() for n, v in x.items()}
+    idx = hd.dsa_index_topk(dev["q_idx"], dev["k_idx"], dev["w_idx"], k)
+    g = torch.Generator(device="cuda").manual_seed(892)
+    dO = (torch.randn(B, L, 64, 256, generator=g, device="cuda") * 0.1).to(torch.bfloat16)
+    O, lse = hd.dsa_sparse_attn_fwd(dev["Q"], dev["K"], dev["V"], idx, return_lse=True)
+    dQ, dK, dV = hd.dsa_sparse_attn_bwd(dev["Q"], dev["K"], dev["V"], idx, O, dO, lse)
+    hd.hcadsa_check_device_error()
+    rows = np.array([0, 1, 2047, 2048, 16385, 32767], np.int64)
+    r = torch.as_tensor(rows, device="cuda")
+    idx_rows = idx.reshape(L, k)[r].cpu().numpy().reshape(1, len(rows), k)
+    Qb = bits(x["Q"]).reshape(L, 64, 256)[rows].reshape(1, len(rows), 64, 256)
+    dO_rows = dO.reshape(L, 64, 256)[r].cpu().double().numpy().reshape(1, len(rows), 64, 256)
+    ref = oracle.dsa_attn_bwd(Qb, bits(x["K"]), bits(x["V"]), idx_rows, dO_rows)
+    _check_grad(dQ.reshape(L, 64, 256)[r], ref[0].reshape(len(rows), 64, 256), "dQ sampled rows")
+    sum_dv = dV.double().sum(dim=(0, 1)).cpu().numpy()
+    sum_do = dO.double().sum(dim=(0, 1, 2)).cpu().numpy()  # every row selects >= 1 key
+    assert np.abs(sum_dv - sum_do).max() <= 1e-2 * np.abs(sum_do).max() + 1e-3, np.abs(sum_dv - sum_do).max()
+    sum_dk = dK.double().sum(dim=(0, 1)).cpu().numpy()
+    abs_dk = dK.double().abs().sum(dim=(0, 1)).cpu().numpy()
+    assert np.all(np.abs(sum_dk) <= 1e-2 * abs_dk), (np.abs(sum_dk) / abs_dk).max()
