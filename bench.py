@@ -607,33 +607,63 @@ def run_hca_131k(hd, device, peaks, iters=10):
 
 
 def e2e_measure(hd, x, device, steps):
-    """Same step through the C ABI with host buffers: H2D of every input from pinned memory and
-    D2H of both layer outputs inside the timed region."""
+    """Same step through the C ABI with host buffers: every step copies all of its inputs from
+    pinned host memory to the device and both layer outputs back, inside the timed region.  The
+    steps are pipelined on three streams (host-to-device copies, compute, device-to-host
+    copies) over two sets of device buffers, so step i+1's inputs and step i-1's outputs cross
+    PCIe while step i computes; the timed region runs from the first input copy to the last
+    output copy."""
     host = {k: v.cpu().pin_memory() for k, v in x.items()}
-    dev = {k: torch.empty_like(v) for k, v in x.items()}
-    stp = Step(hd, dev, device)
-    out_h = torch.empty(x["hQ"].shape, dtype=torch.bfloat16).pin_memory()
-    out_d = torch.empty(x["dQ"].shape, dtype=torch.bfloat16).pin_memory()
+    bufs = []
+    for _ in range(2):
+        dev = {k: torch.empty_like(v) for k, v in x.items()}
+        bufs.append((dev, Step(hd, dev, device)))
+    outs = [(torch.empty(x["hQ"].shape, dtype=torch.bfloat16).pin_memory(),
+             torch.empty(x["dQ"].shape, dtype=torch.bfloat16).pin_memory()) for _ in range(2)]
     h2d = sum(v.numel() * v.element_size() for v in host.values())
-    d2h = out_h.numel() * 2 + out_d.numel() * 2
+    d2h = outs[0][0].numel() * 2 + outs[0][1].numel() * 2
+    s_in, s_cmp, s_out = torch.cuda.Stream(device), torch.cuda.Stream(device), torch.cuda.Stream(device)
+    ev = lambda: torch.cuda.Event()  # noqa: E731
+    in_done = [ev(), ev()]    # inputs of buffer b landed
+    cmp_done = [ev(), ev()]   # step on buffer b finished (inputs free, outputs ready)
+    out_done = [ev(), ev()]   # outputs of buffer b copied to the host
 
-    def one():
-        for k in host:
-            dev[k].copy_(host[k], non_blocking=True)
-        stp.run()
-        out_h.copy_(stp.hO, non_blocking=True)
-        out_d.copy_(stp.dO, non_blocking=True)
+    def run(n, e_start=None, e_end=None):
+        for i in range(n):
+            b = i & 1
+            dev, stp = bufs[b]
+            with torch.cuda.stream(s_in):
+                if i >= 2:
+                    s_in.wait_event(cmp_done[b])  # step i-2 no longer reads these inputs
+                if i == 0 and e_start is not None:
+                    e_start.record(s_in)
+                for k in host:
+                    dev[k].copy_(host[k], non_blocking=True)
+                in_done[b].record(s_in)
+            with torch.cuda.stream(s_cmp):
+                s_cmp.wait_event(in_done[b])
+                if i >= 2:
+                    s_cmp.wait_event(out_done[b])  # step i-2's outputs are on the host
+                stp.run()
+                cmp_done[b].record(s_cmp)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(cmp_done[b])
+                outs[b][0].copy_(stp.hO, non_blocking=True)
+                outs[b][1].copy_(stp.dO, non_blocking=True)
+                out_done[b].record(s_out)
+        if e_end is not None:
+            s_out.wait_stream(s_in)
+            s_out.wait_stream(s_cmp)
+            e_end.record(s_out)
 
-    one()
+    run(2)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(steps):
-        one()
-    e1.record()
+    run(steps, e0, e1)
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / steps
-    del dev, stp
+    del bufs
+    torch.cuda.empty_cache()
     return ms, h2d, d2h
 
 
@@ -760,7 +790,7 @@ def ours(args):
     if rank == 0 and not args.no_bwd:
         bwd = run_backward(hd, device, peaks)
         hd.hcadsa_check_device_error()
-    e2e_ms, h2d, d2h = e2e_measure(hd, x, device, steps=max(2, min(args.steps, 4)))
+    e2e_ms, h2d, d2h = e2e_measure(hd, x, device, steps=max(4, min(args.steps, 8)))
     e2e_ms = max_over_ranks(e2e_ms, dist, device)
     e2e = {"value": job_throughput(e2e_ms, world), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
            "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
