@@ -1276,6 +1276,9 @@ extern "C" hcadsa_status hca_attn_fwd_latent(const hcadsa_bf16* Q, const hcadsa_
                                              hcadsa_stream stream) {
   using namespace hcadsa;
   Geometry G;
+  if ((dqk != 576 || dv != 512) && Q && Kw && O && (n_c == 0 || Kc) && B >= 0 && Lq >= 0 && Hq > 0 && Hkv > 0 &&
+      Hq % Hkv == 0)
+    return HCADSA_ERR_UNSUPPORTED;  // before anything that needs the device, like hca_attn_fwd
   const hcadsa_status st = check_call(Q, Kc, Kc, n_c, Kw, Kw, win_start, n_w, O, lse, B, Lq, q_offset, Hq, Hkv, blk,
                                       W, workspace, workspace_bytes, &G);
   if (st == HCADSA_OK && (dqk != 576 || dv != 512)) return HCADSA_ERR_UNSUPPORTED;

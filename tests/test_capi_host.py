@@ -112,3 +112,64 @@ def test_workspace_size_queries(lib):
     # current device; unsupported shapes (and a machine with no device to size for) give 0
     assert lib.hca_attn_fwd_workspace_size(1, 32768, 0, 16, 1, 256, 256, 128, 128) == 0
     assert lib.hca_attn_fwd_workspace_size(1, 32768, 0, 16, 3, 512, 256, 128, 128) == 0
+
+
+def test_next_row_entry_argument_errors(lib):
+    """Gate + head mix, qk 576 / v 512 HCA, CSA selection: documented host-side errors."""
+    g = lib.attn_gate_vha_fwd
+    assert g(None, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 128, 16, 512, 1024, 4, None) == -1
+    assert g(FAKE, FAKE, FAKE, None, FAKE, FAKE, 1, 128, 16, 512, 1024, 4, None) == -1   # r > 0 needs U, V
+    assert g(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 128, 16, 512, 1024, -1, None) == -2
+    assert g(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 128, 12, 512, 1024, 4, None) == -4   # H not 16/32/64
+    assert g(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 128, 16, 512, 1000, 4, None) == -4   # rq % 64
+    assert g(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 128, 16, 512, 1024, 5, None) == -4   # rank > 4
+    assert g(FAKE, MISALIGNED, FAKE, FAKE, FAKE, FAKE, 1, 128, 16, 512, 1024, 4, None) == -3
+    assert lib.hca_attn_fwd_latent_workspace_size(1, 4096, 0, 16, 1, 512, 512, 31, 128, 128) == 0  # dqk != 576
+    la = lib.hca_attn_fwd_latent
+    assert la(FAKE, FAKE, 1, FAKE, 0, 256, FAKE, None, 1, 256, 0, 16, 1, 512, 512, 128, 128, 0.04, FAKE, 1 << 30,
+              None) == -4
+    c = lib.csa_index_topk
+    assert c(FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 30, 1, 64, 0, 16, 4, 64, 16, 0, None) == -2  # blk < 1
+
+
+def test_backward_argument_errors(lib):
+    """The three backward calls: documented host-side errors before anything is enqueued."""
+    d = lib.dsa_sparse_attn_bwd
+    args = [FAKE] * 10 + [1, 8, 8, 64, 256, 16, 0.0625, None]
+    assert d(*([None] + args[1:])) == -1
+    assert d(*(args[:13] + [32] + args[14:])) == -4        # Hq != 64
+    assert d(*(args[:14] + [512] + args[15:])) == -4       # d != 256
+    assert d(*(args[:15] + [5000] + args[16:])) == -4      # k > 4096
+    assert d(*(args[:15] + [0] + args[16:])) == -2         # k < 1
+    assert d(*(args[:7] + [MISALIGNED] + args[8:])) == -3  # dQ misaligned
+    h = lib.hca_attn_bwd
+    # Q, Kc, Vc, n_c, Kw, Vw, win_start, n_w, O, dO, lse, dQ, dKc, dVc, dKw, dVw,
+    # B, Lq, q_offset, Hq, Hkv, d, blk, W, scale, ws, ws_bytes, stream
+    base = [FAKE, FAKE, FAKE, 1, FAKE, FAKE, 0, 256, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+            1, 256, 0, 16, 1, 512, 128, 128, 0.04, FAKE, 1 << 40, None]
+
+    def call(**kw):
+        a = list(base)
+        pos = {"Q": 0, "n_w": 7, "Hq": 19, "Hkv": 20, "d": 21, "ws_bytes": 26, "dQ": 11, "win_start": 6}
+        for k, v in kw.items():
+            a[pos[k]] = v
+        return h(*a)
+
+    assert call(Q=None) == -1
+    assert call(d=256) == -4
+    assert call(Hq=16, Hkv=3) == -2
+    assert call(n_w=200) == -2                # the last query's window is past the raw buffer
+    assert call(win_start=5) == -2            # the first query's window starts before it
+    assert call(ws_bytes=1024) == -5
+    assert call(dQ=MISALIGNED) == -3
+    # one fp32 D per query row (256-rounded) + P and dS blocks: 4096 row tiles x (2 entry + 3
+    # window slots) x 2 x 32 KB at L = 32768, 16 heads on one K/V head
+    assert lib.hca_attn_bwd_workspace_size(1, 32768, 0, 16, 1, 512, 256, 128, 128) == \
+        32768 * 16 * 4 + 2 * 4096 * 5 * 128 * 128 * 2
+    assert lib.hca_attn_bwd_workspace_size(1, 32768, 0, 16, 1, 256, 256, 128, 128) == 0
+    cb = lib.hca_compress_bwd
+    assert cb(None, FAKE, FAKE, FAKE, FAKE, 1, 256, 1, 512, 128, None) == -1
+    assert cb(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 256, 1, 500, 128, None) == -4
+    assert cb(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 256, 1, 512, 2048, None) == -4
+    assert cb(FAKE, FAKE, FAKE, MISALIGNED, FAKE, 1, 256, 1, 512, 128, None) == -3
+    assert cb(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 100, 1, 512, 128, None) == 0  # no complete block: nothing to do
