@@ -61,7 +61,8 @@ constexpr int kQBytes = 2 * kQBoxBytes;       // 32 KB
 constexpr int kKStageBytes = kStageKeys * kDIdx;  // 16 KB
 constexpr int kHistBytes = (kBins + 1) * kRows * 4;  // 128.5 KB: 256 bins + a discard bin per row
 constexpr int kSmemBytes = kQBytes + kStages * kKStageBytes + kHistBytes + 1024;
-constexpr int kRowWarps = 8;                  // two warps per TMEM lane quarter (32 rows)
+constexpr int kRowWarps = 16;                 // four warps per TMEM lane quarter (32 rows)
+constexpr int kSubs = kRowWarps / 4;          // threads per query row
 constexpr int kRowThreads = kRowWarps * 32;
 constexpr int kThreads = 64 + kRowThreads;
 constexpr uint32_t kTmemCols = 512;           // two buffers of 256 columns: 256 keys, or 4 heads x 64 keys
@@ -109,16 +110,16 @@ __device__ __forceinline__ int levels_for(uint32_t width) {
   return lv;
 }
 
-__device__ __forceinline__ void rows_bar() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
-// Named barrier of the two row warps that share TMEM lane quarter q (ids 2..5).
-__device__ __forceinline__ void pair_bar(int q) { asm volatile("bar.sync %0, 64;" ::"r"(2 + q) : "memory"); }
+__device__ __forceinline__ void rows_bar() { asm volatile("bar.sync 1, 512;" ::: "memory"); }
+// Named barrier of the four row warps that share TMEM lane quarter q (ids 2..5).
+__device__ __forceinline__ void quad_bar(int q) { asm volatile("bar.sync %0, 128;" ::"r"(2 + q) : "memory"); }
 // Named barrier over the 256 row threads that also ANDs a predicate across them.
 __device__ __forceinline__ bool rows_bar_and(bool pred) {
   uint32_t r;
   asm volatile(
       "{\n\t.reg .pred p, q;\n\t"
       "setp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.and.pred q, 1, 256, p;\n\t"
+      "bar.red.and.pred q, 1, 512, p;\n\t"
       "selp.u32 %0, 1, 0, q;\n\t}"
       : "=r"(r)
       : "r"((uint32_t)pred)
@@ -300,16 +301,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else {
-    // ------------------------------------------------------------ two threads per query row
-    // Warps 2-5 (half 0) and 6-9 (half 1) both cover the tile's 128 rows (warp w reaches TMEM
-    // lanes 32 (w % 4) ..); in the histogram passes the two threads of a row split every chunk's
-    // keys, in the emit pass half 0 walks all keys in order.  Both keep the same row state
-    // (computed from the same inputs); only half 0 writes.
+    // ------------------------------------------------------------ four threads per query row
+    // Warps 2-5 (sub 0), 6-9, 10-13 and 14-17 (subs 1-3) each cover the tile's 128 rows (warp w
+    // reaches TMEM lanes 32 (w % 4) ..); in the histogram passes the four threads of a row take
+    // one 64-key group of every 256-key chunk each; in the emit pass sub 0 takes the keys in
+    // order, the other subs hand it bit masks of their groups.  All four keep the same row state
+    // (computed from the same inputs); only sub 0 writes.
     const int quarter = warp & 3;
-    const int half = (warp - 2) >> 2;
+    const int sub = (warp - 2) >> 2;
     const int r = quarter * 32 + lane;  // row of the tile == TMEM lane
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-    const int tid = half * kRows + r;   // 0 .. 255
+    const int tid = sub * kRows + r;    // 0 .. 511
     const int gr = r0 + r;
     const bool valid = gr < p.Lq;
     const int n = valid ? n_candidates((long long)p.q_offset + gr, p.ratio, p.Lk) : 0;
@@ -334,39 +336,39 @@ __global__ void __launch_bounds__(kThreads, 1)
       rows_bar();  // s_kstat complete
       // This row of the tile: 16-byte unit u of box pb, row r, holds bytes 16u .. 16u+15 of that
       // box's 128-byte row (heads 2 pb + (u >> 2), channels 16 (u & 3) ..) at unit u ^ (r & 7).
-      uint4 qv[2][8];
-#pragma unroll
-      for (int pb = 0; pb < 2; ++pb)
-#pragma unroll
-        for (int u = 0; u < 8; ++u)
-          qv[pb][u] = *reinterpret_cast<const uint4*>(sQ + pb * kQBoxBytes + r * 128 + ((u ^ (r & 7)) << 4));
-      // the weighted query q' = sum_j w_j q_j (exact int32); whether every w_j q_j fits int8
-      int qp[kDIdx];
-#pragma unroll
-      for (int c = 0; c < kDIdx; ++c) qp[c] = 0;
+      // The weighted query q' = sum_j w_j q_j (exact int32) is formed 16 channels at a time (the
+      // four heads' units of a channel group) and folded straight into the score bounds, so
+      // few registers are live; also: whether every w_j q_j fits int8.
+      auto q_unit = [&](int j, int cg) -> uint8_t* {
+        return sQ + (j >> 1) * kQBoxBytes + r * 128 + (((((j & 1) << 2) | cg) ^ (r & 7)) << 4);
+      };
       bool fits = true;
+      long long lo64 = 0, hi64 = 0;
+#pragma unroll 1
+      for (int cg = 0; cg < 4; ++cg) {
+        int qp[16];
 #pragma unroll
-      for (int pb = 0; pb < 2; ++pb)
+        for (int e = 0; e < 16; ++e) qp[e] = 0;
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const int j = pb * 2 + (u >> 2);
-          const int c0 = (u & 3) * 16;
-          const uint32_t wd[4] = {qv[pb][u].x, qv[pb][u].y, qv[pb][u].z, qv[pb][u].w};
+        for (int j = 0; j < kHIdx; ++j) {
+          const uint4 a = *reinterpret_cast<const uint4*>(q_unit(j, cg));
+          const uint32_t wd[4] = {a.x, a.y, a.z, a.w};
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
             const int x = w[j] * (int)(int8_t)(wd[e >> 2] >> (8 * (e & 3)));
-            qp[c0 + e] += x;
+            qp[e] += x;
             fits = fits && x >= -128 && x <= 127;
           }
         }
-      if (mode == 2) {
-        long long lo64 = 0, hi64 = 0;
 #pragma unroll
-        for (int c = 0; c < kDIdx; ++c) {
-          const long long a = (long long)qp[c] * s_kstat[c], z = (long long)qp[c] * s_kstat[kDIdx + c];
+        for (int e = 0; e < 16; ++e) {
+          const int c = cg * 16 + e;
+          const long long a = (long long)qp[e] * s_kstat[c], z = (long long)qp[e] * s_kstat[kDIdx + c];
           lo64 += a < z ? a : z;
           hi64 += a < z ? z : a;
         }
+      }
+      if (mode == 2) {
         // the true scores fit int32 (caller contract), so clamping keeps them inside [lo, hi]
         lo64 = lo64 < INT_MIN ? INT_MIN : lo64;
         hi64 = hi64 > INT_MAX ? INT_MAX : hi64;
@@ -385,14 +387,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       // When every row's w_j q_j fits int8, the tile is rewritten in place as w_j q_j, so that
       // summing the four heads' products in one accumulator gives the score directly (exact:
       // the int32 sum is order free).  Otherwise the MMA keeps one accumulator per head.
-      const bool single = rows_bar_and(fits);  // both halves have read the tile by now
-      if (single && half == 0) {
+      const bool single = rows_bar_and(fits);  // every sub has read the tile by now
+      if (single && sub == 0) {
 #pragma unroll
-        for (int pb = 0; pb < 2; ++pb)
-#pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            const int j = pb * 2 + (u >> 2);
-            uint32_t wd[4] = {qv[pb][u].x, qv[pb][u].y, qv[pb][u].z, qv[pb][u].w};
+        for (int j = 0; j < kHIdx; ++j)
+#pragma unroll 1
+          for (int cg = 0; cg < 4; ++cg) {
+            uint4* up = reinterpret_cast<uint4*>(q_unit(j, cg));
+            const uint4 a = *up;
+            uint32_t wd[4] = {a.x, a.y, a.z, a.w};
 #pragma unroll
             for (int e4 = 0; e4 < 4; ++e4) {
               uint32_t o = 0;
@@ -403,8 +406,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
               wd[e4] = o;
             }
-            *reinterpret_cast<uint4*>(sQ + pb * kQBoxBytes + r * 128 + ((u ^ (r & 7)) << 4)) =
-                make_uint4(wd[0], wd[1], wd[2], wd[3]);
+            *up = make_uint4(wd[0], wd[1], wd[2], wd[3]);
           }
         fence_proxy_async_smem();  // generic-proxy writes -> tensor-core operand reads
       }
@@ -418,12 +420,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         s_single = single ? 1 : 0;
         mbar_arrive(&bar.plan);
       }
-      if (!done && half == 0)
+      if (!done && sub == 0)
         for (int bb = 0; bb <= kBins; ++bb) hist[bb * kRows + r] = 0;
     }
 
     // rows with at most k candidates: every candidate, then -1
-    if (mode == 1 && half == 0) {
+    if (mode == 1 && sub == 0) {
       RowWriter wr;
       wr.init(out, vec);
       for (int s = 0; s < n; ++s) wr.put(s);
@@ -512,9 +514,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         };
         // TMEM chunks of this pass: one per 256-key stage (single accumulator), or four of 64 keys
         const int chunks = single ? n_stages : n_stages * (kStageKeys / kSub);
-        // the emit pass of per-head accumulators is half 0's alone (key order); with one
-        // accumulator half 1 forms the bit masks of the chunk's second 128 keys for half 0
-        const bool active = !emit || half == 0 || single;
+        // the emit pass of per-head accumulators is sub 0's alone (key order); with one
+        // accumulator subs 1-3 form the bit masks of the chunk's later 64-key groups for sub 0.
+        // Per-head accumulators (64 keys a chunk) split over subs 0 and 1 in the counting passes.
+        const bool active = single || (emit ? sub == 0 : sub < 2);
         for (int c = 0; c < chunks; ++c, ++g) {
           const uint32_t buf = g % kBufs;
           ok = mbar_wait(&bar.tfull[buf], (g / kBufs) & 1, &abort_flag, p.err) && ok;
@@ -525,87 +528,87 @@ __global__ void __launch_bounds__(kThreads, 1)
             continue;
           }
           if (single && emit) {
-            // 256 scores of keys c*256 .. c*256+255: half 0 takes keys 0..127 in order, half 1
-            // turns keys 128..255 into bit masks (shared memory, two buffers by chunk parity);
-            // the two warps of a lane quarter meet once per chunk, then half 0 takes the rest
-            uint32_t* mk = hist + (c & 1) * 8 * kRows + r;  // [buffer][word][row]
-#pragma unroll 1
-            for (int q = 2 * half; q < 2 * half + 2; ++q) {
-              uint32_t v0[32], v1[32];
-              const uint32_t ta = tmem + lane_off + buf * 256 + q * 64;
-              tmem_ld32_nowait(ta, v0);
-              tmem_ld32_nowait(ta + 32, v1);
-              tmem_wait_ld_regs2(v0, v1);
-              if (q == 2 * half + 1) {
+            // 256 scores of keys c*256 .. c*256+255: sub 0 takes keys 0..63 in order, subs 1-3
+            // turn their 64-key groups into bit masks (shared memory, two buffers by chunk
+            // parity); the four warps of a lane quarter meet once per chunk, then sub 0 takes the rest
+            uint32_t* mk = hist + (c & 1) * 12 * kRows + r;  // [buffer][word][row]
+            {
+              const uint32_t ta = tmem + lane_off + buf * 256 + sub * 64;
+              const int s0 = c * kStageKeys + sub * 64;
+              uint32_t gt0, eq0, gt1, eq1;
+              {
+                uint32_t v[32];
+                tmem_ld32_nowait(ta, v);
+                tmem_wait_ld_regs(v);
+                masks(reinterpret_cast<const int(&)[32]>(v), s0, gt0, eq0);
+              }
+              {
+                uint32_t v[32];
+                tmem_ld32_nowait(ta + 32, v);
+                tmem_wait_ld_regs(v);
                 tc_fence_before();
                 mbar_arrive(&bar.tempty[buf]);
+                masks(reinterpret_cast<const int(&)[32]>(v), s0 + 32, gt1, eq1);
               }
-              const int s0 = c * kStageKeys + q * 64;
-              uint32_t gt0, eq0, gt1, eq1;
-              masks(reinterpret_cast<const int(&)[32]>(v0), s0, gt0, eq0);
-              masks(reinterpret_cast<const int(&)[32]>(v1), s0 + 32, gt1, eq1);
-              if (half == 0) {
+              if (sub == 0) {
                 take(gt0, eq0, s0);
                 take(gt1, eq1, s0 + 32);
               } else {
-                const int w0 = (q - 2) * 2;
+                const int w0 = (sub - 1) * 2;
                 mk[w0 * kRows] = gt0;
                 mk[(w0 + 1) * kRows] = gt1;
-                mk[(4 + w0) * kRows] = eq0;
-                mk[(5 + w0) * kRows] = eq1;
+                mk[(6 + w0) * kRows] = eq0;
+                mk[(7 + w0) * kRows] = eq1;
               }
             }
-            pair_bar(quarter);
-            if (half == 0)
+            quad_bar(quarter);
+            if (sub == 0)
 #pragma unroll 1
-              for (int w4 = 0; w4 < 4; ++w4) take(mk[w4 * kRows], mk[(4 + w4) * kRows], c * kStageKeys + 128 + 32 * w4);
+              for (int w6 = 0; w6 < 6; ++w6) take(mk[w6 * kRows], mk[(6 + w6) * kRows], c * kStageKeys + 64 + 32 * w6);
           } else if (single) {
-            // 256 scores of keys c*256 .. c*256+255, 64 at a time: groups 2 half .. 2 half + 1
-            const int q0 = 2 * half, q1 = 2 * half + 2;
-#pragma unroll 1
-            for (int q = q0; q < q1; ++q) {
-              uint32_t v0[32], v1[32];
-              const uint32_t ta = tmem + lane_off + buf * 256 + q * 64;
-              tmem_ld32_nowait(ta, v0);
-              tmem_ld32_nowait(ta + 32, v1);
-              tmem_wait_ld_regs2(v0, v1);
-              if (q == q1 - 1) {  // this thread's part of the chunk is in registers or consumed
+            // 256 scores of keys c*256 .. c*256+255: this sub's 64-key group
+            {
+              const uint32_t ta = tmem + lane_off + buf * 256 + sub * 64;
+              {
+                uint32_t v[32];
+                tmem_ld32_nowait(ta, v);
+                tmem_wait_ld_regs(v);
+                consume(reinterpret_cast<const int(&)[32]>(v), c * kStageKeys + sub * 64);
+              }
+              {
+                uint32_t v[32];
+                tmem_ld32_nowait(ta + 32, v);
+                tmem_wait_ld_regs(v);
                 tc_fence_before();
                 mbar_arrive(&bar.tempty[buf]);
+                consume(reinterpret_cast<const int(&)[32]>(v), c * kStageKeys + sub * 64 + 32);
               }
-              int sc[32];
-#pragma unroll
-              for (int i = 0; i < 32; ++i) sc[i] = (int)v0[i];
-              consume(sc, c * kStageKeys + q * 64);
-#pragma unroll
-              for (int i = 0; i < 32; ++i) sc[i] = (int)v1[i];
-              consume(sc, c * kStageKeys + q * 64 + 32);
             }
           } else {
-            const int h0 = emit ? 0 : half, h1 = emit ? 2 : half + 1;
+            const int h0 = emit ? 0 : sub, h1 = emit ? 2 : sub + 1;
 #pragma unroll 1
             for (int h = h0; h < h1; ++h) {
-              uint32_t v0[32], v1[32], v2[32], v3[32];
               const uint32_t ta = tmem + lane_off + buf * 256 + h * 32;
-              tmem_ld32_nowait(ta + 0 * kSub, v0);
-              tmem_ld32_nowait(ta + 1 * kSub, v1);
-              tmem_ld32_nowait(ta + 2 * kSub, v2);
-              tmem_ld32_nowait(ta + 3 * kSub, v3);
-              tmem_wait_ld_regs2(v0, v1);
-              tmem_wait_ld_regs2(v2, v3);
+              int sc[32];
+#pragma unroll
+              for (int i = 0; i < 32; ++i) sc[i] = 0;
+#pragma unroll
+              for (int hd = 0; hd < kHIdx; ++hd) {  // one head's accumulator at a time
+                uint32_t v[32];
+                tmem_ld32_nowait(ta + hd * kSub, v);
+                tmem_wait_ld_regs(v);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) sc[i] += w[hd] * (int)v[i];
+              }
               if (h == h1 - 1) {
                 tc_fence_before();
                 mbar_arrive(&bar.tempty[buf]);
               }
-              int sc[32];
-#pragma unroll
-              for (int i = 0; i < 32; ++i)
-                sc[i] = w[0] * (int)v0[i] + w[1] * (int)v1[i] + w[2] * (int)v2[i] + w[3] * (int)v3[i];
               consume(sc, c * kSub + h * 32);
             }
           }
         }
-        if (!emit) rows_bar();  // both halves' counts of this level are in
+        if (!emit) rows_bar();  // every sub's counts of this level are in
         if (!emit && !done) {
           // the bin holding the rank-rem score of the interval, counted from the top (both
           // threads of the row read the same counts and reach the same state)
@@ -638,12 +641,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         if (!emit) {
-          rows_bar();  // both halves have read the counts
-          if (half == 0 && !done_before)
+          rows_bar();  // every sub has read the counts
+          if (sub == 0 && !done_before)
             for (int bb = 0; bb <= kBins; ++bb) hist[bb * kRows + r] = 0;
           rows_bar();  // cleared before the next level counts
         }
-        if (emit && mode >= 2 && half == 0) wr.flush();
+        if (emit && mode >= 2 && sub == 0) wr.flush();
       }
     }
   }
