@@ -528,43 +528,73 @@ __global__ void __launch_bounds__(kThreads, 1)
             continue;
           }
           if (single && emit) {
-            // 256 scores of keys c*256 .. c*256+255: sub 0 takes keys 0..63 in order, subs 1-3
-            // turn their 64-key groups into bit masks (shared memory, two buffers by chunk
-            // parity); the four warps of a lane quarter meet once per chunk, then sub 0 takes the rest
-            uint32_t* mk = hist + (c & 1) * 12 * kRows + r;  // [buffer][word][row]
+            // 256 scores of keys c*256 .. c*256+255: every sub forms the bit masks of its 64-key
+            // group and posts its (above, equal) counts (shared memory, two buffers by chunk
+            // parity); after the four warps of a lane quarter meet, each sub knows how many
+            // keys the earlier groups take and writes its own positions at that offset
+            uint32_t* cn = hist + (c & 1) * 4 * kRows + r;  // [buffer][sub][row]: gt | eq << 16
+            const uint32_t ta = tmem + lane_off + buf * 256 + sub * 64;
+            const int s0 = c * kStageKeys + sub * 64;
+            uint32_t gt0, eq0, gt1, eq1;
             {
-              const uint32_t ta = tmem + lane_off + buf * 256 + sub * 64;
-              const int s0 = c * kStageKeys + sub * 64;
-              uint32_t gt0, eq0, gt1, eq1;
-              {
-                uint32_t v[32];
-                tmem_ld32_nowait(ta, v);
-                tmem_wait_ld_regs(v);
-                masks(reinterpret_cast<const int(&)[32]>(v), s0, gt0, eq0);
+              uint32_t v[32];
+              tmem_ld32_nowait(ta, v);
+              tmem_wait_ld_regs(v);
+              masks(reinterpret_cast<const int(&)[32]>(v), s0, gt0, eq0);
+            }
+            {
+              uint32_t v[32];
+              tmem_ld32_nowait(ta + 32, v);
+              tmem_wait_ld_regs(v);
+              tc_fence_before();
+              mbar_arrive(&bar.tempty[buf]);
+              masks(reinterpret_cast<const int(&)[32]>(v), s0 + 32, gt1, eq1);
+            }
+            cn[sub * kRows] = (uint32_t)(__popc(gt0) + __popc(gt1)) | ((uint32_t)(__popc(eq0) + __popc(eq1)) << 16);
+            quad_bar(quarter);
+            int gt_before = 0, eq_before = 0, gt_tot = 0, eq_tot = 0;
+#pragma unroll
+            for (int s2 = 0; s2 < kSubs; ++s2) {
+              const uint32_t w2 = cn[s2 * kRows];
+              const int g2 = (int)(w2 & 0xFFFFu), e2 = (int)(w2 >> 16);
+              if (s2 < sub) {
+                gt_before += g2;
+                eq_before += e2;
               }
-              {
-                uint32_t v[32];
-                tmem_ld32_nowait(ta + 32, v);
-                tmem_wait_ld_regs(v);
-                tc_fence_before();
-                mbar_arrive(&bar.tempty[buf]);
-                masks(reinterpret_cast<const int(&)[32]>(v), s0 + 32, gt1, eq1);
+              gt_tot += g2;
+              eq_tot += e2;
+            }
+            // equal keys are taken in position order until need_eq of them are in
+            const int eq_room = max(0, need_eq - eq_seen);
+            const int eq_taken_before = min(eq_before, eq_room);
+            int eq_take = min(__popc(eq0) + __popc(eq1), eq_room - eq_taken_before);
+            int pos = taken + gt_before + eq_taken_before;
+            if (mode >= 2) {
+              // this group's selected keys, ascending: all above, the first eq_take equal ones
+              uint32_t sel0 = gt0, e = eq0;
+              while (e && eq_take > 0) {
+                sel0 |= e & (0u - e);
+                e &= e - 1;
+                --eq_take;
               }
-              if (sub == 0) {
-                take(gt0, eq0, s0);
-                take(gt1, eq1, s0 + 32);
-              } else {
-                const int w0 = (sub - 1) * 2;
-                mk[w0 * kRows] = gt0;
-                mk[(w0 + 1) * kRows] = gt1;
-                mk[(6 + w0) * kRows] = eq0;
-                mk[(7 + w0) * kRows] = eq1;
+              uint32_t sel1 = gt1;
+              e = eq1;
+              while (e && eq_take > 0) {
+                sel1 |= e & (0u - e);
+                e &= e - 1;
+                --eq_take;
+              }
+              while (sel0) {
+                out[pos++] = s0 + __ffs(sel0) - 1;
+                sel0 &= sel0 - 1;
+              }
+              while (sel1) {
+                out[pos++] = s0 + 32 + __ffs(sel1) - 1;
+                sel1 &= sel1 - 1;
               }
             }
-            quad_bar(quarter);
-            if (sub == 0)
-#pragma unroll 1
-              for (int w6 = 0; w6 < 6; ++w6) take(mk[w6 * kRows], mk[(6 + w6) * kRows], c * kStageKeys + 64 + 32 * w6);
+            taken += gt_tot + min(eq_tot, eq_room);
+            eq_seen += eq_tot;
           } else if (single) {
             // 256 scores of keys c*256 .. c*256+255: this sub's 64-key group
             {
@@ -646,7 +676,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int bb = 0; bb <= kBins; ++bb) hist[bb * kRows + r] = 0;
           rows_bar();  // cleared before the next level counts
         }
-        if (emit && mode >= 2 && sub == 0) wr.flush();
+        if (emit && mode >= 2 && sub == 0 && !single) wr.flush();
       }
     }
   }
