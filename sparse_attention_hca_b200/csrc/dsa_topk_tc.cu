@@ -14,10 +14,10 @@
 // int32 scores, so nothing but the selection state survives between passes:
 //   * Scores on the int8 tensor cores (tcgen05.mma kind::i8, M = 128 queries, K = 64 int8 per
 //     head in two K = 32 steps; A = the tile's q_idx (two 128-byte SW128 boxes, two heads
-//     each), B = a 256-key k_idx stage (SW64)).  When every w_j * q_j of the tile fits
+//     each), B = a 192-key k_idx stage (SW64)).  When every w_j * q_j of the tile fits
 //     int8 (the usual inputs: |w| <= 4, |q| <= 8), the row threads rewrite the tile in place as
 //     w_j * q_j and the four heads accumulate into ONE int32 accumulator, which is the score
-//     itself: eight N = 256 MMAs per 256-key stage (TMEM: two buffers of 256 columns).
+//     itself: eight N = 192 MMAs per 192-key stage (TMEM: two buffers of 256 columns).
 //     Otherwise each head keeps its own accumulator (four N = 64 accumulators per 64 keys, the
 //     same two 256-column buffers) and the thread of query row r (= TMEM lane r) weights them:
 //     score = sum_j w_j D_j[r, :].  Both are exact.  (One thread issues every MMA, and its
@@ -33,14 +33,19 @@
 //       thr to take (the lowest positions first).
 //     levels = 1 + ceil(s_1 / 8) for the widest row of the tile (s_1 = bits(hi - lo) - 8):
 //     two for the usual indexer inputs (scores within about +-2^14).
-//   * Last pass (emit): each row thread walks its keys in ascending order and writes the
-//     positions with score > thr and the first need_eq with score == thr -- exactly the k
-//     positions, already ascending.
+//   * Last pass (emit): the positions with score > thr and the first need_eq with score == thr
+//     -- exactly the k positions, ascending.  Each of a row's three threads forms the bit masks
+//     of its 64-key group of a stage and posts its (above, equal) counts; after the three warps
+//     of the lane quarter meet, each knows how many positions the earlier groups take (and how
+//     many equal keys are left) and writes its own at that offset.
 // Rows with at most k candidates write 0 .. n-1 and -1 padding without scores.  Tiles are
 // issued longest first (causal rows near the end of the sequence have the most keys).
 //
-// Warps: 0 = TMA producer (Q once, then the k_idx stages of 256 keys of every pass through a
-// 4-stage ring), 1 = TMEM allocation + the MMA-issuing thread, 2-5 = one thread per query row.
+// Warps: 0 = TMA producer (Q once, then the k_idx stages of 192 keys of every pass through a
+// 4-stage ring), 1 = TMEM allocation + the MMA-issuing thread, 2-13 = three threads per query
+// row (warp w reaches TMEM lanes 32 (w % 4) ..; each takes one 64-key group of every stage).
+// 14 warps keep 128 registers a thread (16 warps, four groups of a 256-key stage, capped them at
+// 96 and spilled: 1.19 against 1.14 ms at L = 32768).
 #include <climits>
 
 #include "host_common.h"
@@ -50,7 +55,7 @@ namespace hcadsa {
 namespace {
 
 constexpr int kRows = 128;                    // query rows per CTA (MMA M, TMEM lanes)
-constexpr int kStageKeys = 256;               // keys per k_idx stage (one N = 256 MMA per head and K step)
+constexpr int kStageKeys = 192;               // keys per k_idx stage (one N = 192 MMA per head and K step)
 constexpr int kSub = 64;                      // keys per MMA when each head has its own accumulator
 constexpr int kDIdx = 64;                     // indexer dim (int8 per head and key)
 constexpr int kHIdx = 4;                      // indexer heads
@@ -58,10 +63,10 @@ constexpr int kStages = 4;                    // k_idx stage ring
 constexpr int kBins = 256;                    // histogram bins per level (8 bits)
 constexpr int kQBoxBytes = kRows * 128;       // one SW128 box: 128 rows x (2 heads x 64 int8)
 constexpr int kQBytes = 2 * kQBoxBytes;       // 32 KB
-constexpr int kKStageBytes = kStageKeys * kDIdx;  // 16 KB
+constexpr int kKStageBytes = kStageKeys * kDIdx;  // 12 KB
 constexpr int kHistBytes = (kBins + 1) * kRows * 4;  // 128.5 KB: 256 bins + a discard bin per row
 constexpr int kSmemBytes = kQBytes + kStages * kKStageBytes + kHistBytes + 1024;
-constexpr int kRowWarps = 16;                 // four warps per TMEM lane quarter (32 rows)
+constexpr int kRowWarps = 12;                 // three warps per TMEM lane quarter (32 rows)
 constexpr int kSubs = kRowWarps / 4;          // threads per query row
 constexpr int kRowThreads = kRowWarps * 32;
 constexpr int kThreads = 64 + kRowThreads;
@@ -110,19 +115,19 @@ __device__ __forceinline__ int levels_for(uint32_t width) {
   return lv;
 }
 
-__device__ __forceinline__ void rows_bar() { asm volatile("bar.sync 1, 512;" ::: "memory"); }
-// Named barrier of the four row warps that share TMEM lane quarter q (ids 2..5).
-__device__ __forceinline__ void quad_bar(int q) { asm volatile("bar.sync %0, 128;" ::"r"(2 + q) : "memory"); }
+__device__ __forceinline__ void rows_bar() { asm volatile("bar.sync 1, %0;" ::"n"(kRowThreads) : "memory"); }
+// Named barrier of the row warps that share TMEM lane quarter q (ids 2..5).
+__device__ __forceinline__ void quad_bar(int q) { asm volatile("bar.sync %0, %1;" ::"r"(2 + q), "n"(kSubs * 32) : "memory"); }
 // Named barrier over the 256 row threads that also ANDs a predicate across them.
 __device__ __forceinline__ bool rows_bar_and(bool pred) {
   uint32_t r;
   asm volatile(
       "{\n\t.reg .pred p, q;\n\t"
       "setp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.and.pred q, 1, 512, p;\n\t"
+      "bar.red.and.pred q, 1, %2, p;\n\t"
       "selp.u32 %0, 1, 0, q;\n\t}"
       : "=r"(r)
-      : "r"((uint32_t)pred)
+      : "r"((uint32_t)pred), "n"(kRowThreads)
       : "memory");
   return r != 0;
 }
