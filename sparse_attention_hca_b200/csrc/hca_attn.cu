@@ -121,6 +121,8 @@ struct Params {
   uint8_t* scratch;  // gridDim.x * J_max * kScratchTileBytes
   float* part_o;     // split mode: [total_units][128][512] unnormalised O of each unit
   float2* part_ml;   // split mode: [total_units][128] (reference max in log2 units, row sum)
+  uint16_t* O;       // the output (stored directly by the epilogue when deep_ring)
+  int deep_ring;     // 512 shape, long rows: the staging region is a third ring group
   int* err;
 };
 
@@ -389,7 +391,7 @@ __global__ void __launch_bounds__(kThreads, 1) hca_attn_kernel(const __grid_cons
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       tma_prefetch_desc(&maps.q);
-      const uint32_t ngroups = p.split_mode ? kMaxGroups : kGroups;
+      const uint32_t ngroups = (p.split_mode || p.deep_ring) ? kMaxGroups : kGroups;
       uint32_t grp = 0, gph = 0;  // next ring group to fill and the phase of its use
       bool ok = true;
       auto next_group = [&]() {
@@ -495,7 +497,7 @@ __global__ void __launch_bounds__(kThreads, 1) hca_attn_kernel(const __grid_cons
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t sQa = smem_u32(sQ), sRa = smem_u32(sRing);
-      const uint32_t ngroups = p.split_mode ? kMaxGroups : kGroups;
+      const uint32_t ngroups = (p.split_mode || p.deep_ring) ? kMaxGroups : kGroups;
       uint32_t grp = 0, gph = 0;  // next ring group to consume and the phase of its use
       auto next_group = [&]() {
         if (++grp == ngroups) {
@@ -683,7 +685,30 @@ __global__ void __launch_bounds__(kThreads, 1) hca_attn_kernel(const __grid_cons
           bulk_commit_group();
         }
       };
-      if constexpr (kOutBufs == 4) {  // one round per 128 columns
+      if (kOutBufs == 4 && p.deep_ring) {
+        // long rows (many key tiles per row tile): the staging region is the ring's third group,
+        // so the rows go straight from registers to global memory (16-byte stores)
+        uint16_t* orow = nullptr;
+        {
+          const int tok_r = ts.tok0 + r / p.g;
+          if (row_valid)
+            orow = p.O + (((size_t)ts.b * p.Lq + tok_r) * p.Hq + ts.hk * p.g + r % p.g) * kD + col0;
+        }
+        auto store_row = [&](int c0) {
+          if (orow) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + c0);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) dst[i] = make_uint4(ob[4 * i], ob[4 * i + 1], ob[4 * i + 2], ob[4 * i + 3]);
+          }
+        };
+        read_o(0);
+        store_row(0);
+        read_o(128);
+        tc_fence_before();
+        mbar_arrive(&bar.o_empty[0]);
+        mbar_arrive(&bar.o_empty[1]);
+        store_row(128);
+      } else if constexpr (kOutBufs == 4) {  // one round per 128 columns
         read_o(0);
         stage_o(0);
         read_o(128);
@@ -1227,6 +1252,10 @@ hcadsa_status launch_hca(const hcadsa_bf16* Q, const hcadsa_bf16* Kc, const hcad
   p.part_o = p.split_mode ? reinterpret_cast<float*>(p.scratch + G.scratch_bytes) : nullptr;
   p.part_ml = p.split_mode ? reinterpret_cast<float2*>(p.scratch + G.scratch_bytes + (size_t)G.total_units * 128 * kD * 4)
                            : nullptr;
+  p.O = reinterpret_cast<uint16_t*>(O);
+  // a third ring group pays off once row tiles have many key tiles (long contexts); with few
+  // (L = 32768: 3-4) the TMA-stored epilogue is the better use of the region
+  p.deep_ring = (DQK == 512 && !p.split_mode && G.J_max >= 6) ? 1 : 0;
   p.err = device_error_ptr();
   if (cudaFuncSetAttribute(hca_attn_kernel<DQK>, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kSmemBytes) !=
       cudaSuccess)

@@ -120,6 +120,9 @@ def test_hca_tiny_all_rows(hd):
     # tiles) and of a single token
     (synth.HcaConfig("g32_L700_hq32", B=1, L=700, Hq=32, Hkv=1, sigma=1.0), 128),
     (synth.HcaConfig("g128_L300_hq128", B=1, L=300, Hq=128, Hkv=1, sigma=1.0), 128),
+    # 618 entries of 4 tokens: row tiles of 7 key tiles, the long-row ring (three groups,
+    # rows stored straight from registers)
+    (synth.HcaConfig("deep_ring_blk4_L2600_hq4", B=1, L=2600, Hq=4, Hkv=1, blk=4, sigma=1.0), 128),
 ])
 def test_hca_stress(hd, cfg, W):
     O, lse, ref, ref_lse = _hca_gpu_and_oracle(hd, cfg, W=W)
