@@ -8,27 +8,34 @@
 // head (the MLA latent reading) and the token's index row.
 //
 // Kernel design (persistent: one CTA per SM walks query tokens tok = blockIdx.x + i*gridDim.x):
-//   * The 64 heads of a token are too few rows for a full-rate M=128 tcgen05 tile, so the
-//     contraction is transposed: the 128 gathered keys of a tile are M.
-//       S^T[key, head]  = K_g (A, K-major, 128 x 256)  *  Q^T (B, K-major, 64 heads)
-//       O^T[dv, head]  += V_g^T (A, MN-major, 2 x 128 dv) * P^T (B, MN-major, 64 heads)
-//     TMEM: O^T double-buffered per token [0,128) / [128,256) so one token's epilogue
-//     overlaps the next token's MMAs; S^T double-buffered per tile [256,320) / [320,384).
+//   * The 64 heads of a token are the M of every MMA (M = 64: half of the datapath, so an
+//     instruction takes as long as its M = 128 twin, measured on B200):
+//       S  = Q (A, smem, K-major, 64 x 256) * K_g^T (B, smem, K-major, 128 gathered keys)
+//       O += P (A, TMEM, bf16)               * V_g (B, smem, MN-major, 256 d_v)
+//     P never touches shared memory: the softmax writes it as bf16 pairs over the first 64
+//     columns of its S tile, where the PV MMA reads it as the TMEM A operand.  Against the
+//     keys-as-M form (S^T = K_g Q^T, P^T staged in shared memory) this saves 48 KB of
+//     shared-memory traffic per 128-key tile and every per-head cross-thread reduction:
+//     a head is a TMEM lane, so its max and sum are two threads' business.
+//   * An M = 64 accumulator fills 16 of the 32 lanes of each lane quarter; the other 16 lanes
+//     hold a second one (lane offset 16).  Token i uses half i & 1 for everything: O at
+//     columns [0, 256) and two S tiles at [256, 384) / [384, 512).  A TS MMA needs A and D in
+//     the same half, which this keeps, and one token's epilogue overlaps the next token's MMAs
+//     in the other half.
 //   * Warps 0-5 gather K and V rows with cp.async: one warp instruction moves one whole
 //     512-byte row (lane l -> 16 bytes of 64-column chunk l/8), written 128B-swizzled into a
 //     ring of two 64 KB groups (4 chunk slots each); a group holds one K or one V tile, loaded
 //     in exactly the order warp 6 consumes them: K_0, K_1, V_0, K_2, V_1, ...  Completion is
 //     tracked with cp.async.mbarrier.arrive.noinc, one arrival per producer thread per tile, so
-//     the MMA thread waits once per tile (a wait costs the issuing thread a few hundred cycles,
-//     which only a whole tile of MMAs hides) and issues a proxy fence after it so the tensor
-//     core sees the generic-proxy writes.  (Measured on B200: this reaches ~105 GB/s per SM
-//     from L2, TMA tile::gather4 of 4 x 128 B rows ~16 GB/s.)
-//     Q (32 KB, TMA) is reloaded per token once the previous token's last S^T MMA is done.
-//   * Warp 6, lane 0 issues every MMA.  Warps 7-10: softmax (one thread per key = TMEM lane,
-//     64 head scores each; per-head row sums reduced across the warp every tile).  The first tile of a token sets the per-head reference max by a
-//     warp reduce-scatter + 4-warp combine; later tiles only check their scores against it and
-//     redo the reduction (and rescale O^T) when some score exceeds it by 2^8.  P^T rows go to
-//     shared memory; then the token's epilogue (normalise O^T, store O).
+//     the MMA thread waits once per tile and issues a proxy fence after it so the tensor core
+//     sees the generic-proxy writes.  (Measured on B200: this reaches ~105 GB/s per SM from L2,
+//     TMA tile::gather4 of 4 x 128 B rows ~16 GB/s.)
+//     Q (32 KB, TMA) is reloaded per token once the previous token's last S MMA is done.
+//   * Warp 6, lane 0 issues every MMA.  Warps 7-10: softmax.  Warp 7+q owns heads 16q..16q+15
+//     (TMEM lane quarter q); thread t of it holds head 16q + t%16 and keys 64(t/16)..+63 of a
+//     tile.  Online softmax per head with a lazy reference max: the first tile sets it, a later
+//     tile moves it (and rescales that head's O in TMEM) only when a score exceeds it by 2^8.
+//     Then the token's epilogue: O / l to bf16, and the log-sum-exp.
 //   * Index rows may hold padding (< 0) anywhere; a 128-entry tile without any valid entry
 //     is skipped, other invalid entries read row 0 and are masked.  Index rows are staged in
 //     shared memory (double buffer): the softmax warps prefetch token i+2's row with cp.async
@@ -53,18 +60,16 @@ constexpr int kChunkBytes = 128 * 128;     // 128 rows x 64 bf16
 constexpr int kRingSlots = 8;  // two groups of 4 slots: one K tile or one V tile per group
 constexpr int kQChunkBytes = kH * 128;     // 64 heads x 64 bf16
 constexpr int kQBytes = 4 * kQChunkBytes;  // 32 KB
-constexpr int kPBytes = kKeyTile * 128;    // 128 keys x 64 heads bf16
 constexpr int kMaxK = 4096;                // 32 tiles: one bit per tile in a 32-bit mask
 constexpr int kIdxBytes = kMaxK * 4;  // one index row
-constexpr int kSmemBytes = kQBytes + kRingSlots * kChunkBytes + 2 * kPBytes + 2 * kIdxBytes + 1024;
-// Gather throughput scales with the number of producer warps.  11 warps put 3 on some SM
-// sub-partitions (16K-entry register file each), which caps a thread at 168 registers; the
-// softmax keeps its per-head row sums reduced across the warp (2 per lane) to fit.
+constexpr int kSmemBytes = kQBytes + kRingSlots * kChunkBytes + 2 * kIdxBytes + 1024;
+// Gather throughput scales with the number of producer warps; 11 warps cap a thread at 168
+// registers, which the softmax (64 scores per thread) stays well inside.
 constexpr int kProducerWarps = 6;
 constexpr int kMmaWarp = kProducerWarps;
 constexpr int kSoftmaxWarp0 = kProducerWarps + 1;
 constexpr int kThreads = 32 * (kProducerWarps + 1 + 4);
-constexpr uint32_t kTmemS = 256;  // S^T buffers at columns 256 and 320
+constexpr uint32_t kTmemS = 256;  // S tiles at columns 256 and 384 of a token's half; O at 0
 constexpr float kLazyRescale = 8.0f;
 
 struct Params {
@@ -88,13 +93,7 @@ struct __align__(8) Barriers {
   uint64_t o_full[2];
   uint64_t o_empty[2];
   uint64_t idx_full[2];   // index row of a token landed (128 softmax-thread cp.async arrivals)
-  uint64_t idx_empty[2];  // producers (3 warps) and MMA warp are done with the row
-};
-
-struct SoftShared {
-  float wred[4][kH];
-  __align__(16) float m_ref[kH];
-  __align__(16) float alpha[kH];  // rescale factors; 1/l in the epilogue
+  uint64_t idx_empty[2];  // the producer warps and the MMA warp are done with the row
 };
 
 __device__ __forceinline__ bool idx_ok(int s, int Lk) { return s >= 0 && s < Lk; }
@@ -108,64 +107,84 @@ __device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
 }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
-// Bit j set iff tile j (entries [128j, 128j+128) of the row) holds a valid entry.  Whole warp;
-// `row` is the shared-memory copy of the index row.
-__device__ __forceinline__ uint32_t tile_mask_of_row(const int32_t* row, int k, int Lk, int lane) {
-  uint32_t mask = 0;
-  const int n_tiles = (k + kKeyTile - 1) / kKeyTile;
-  for (int j = 0; j < n_tiles; ++j) {
-    bool any = false;
+// Bit j set iff tile j (entries [128j, 128j+128) of the row) holds a valid entry; with
+// kAll, `all_valid` gets bit j iff all 128 entries of tile j are valid.  Whole warp; `row` is
+// the 16-byte aligned shared-memory copy of the index row.  Each lane reads its four entries of
+// a whole tile as one 16-byte word (a warp reads 512 contiguous bytes: no bank conflicts), eight
+// tiles' words in flight at a time, and sets one bit per tile; one reduction over the warp then
+// gives the mask.  This runs between the tokens of the MMA warp, while the tensor pipe only
+// has its queue left, so it has to be short.
+template <bool kAll>
+__device__ __forceinline__ uint32_t tile_mask_of_row(const int32_t* row, int k, int Lk, int lane,
+                                                     uint32_t* all_valid = nullptr) {
+  const int full = k / kKeyTile;
+  uint32_t bits = 0, all_bits = 0;
+  for (int j0 = 0; j0 < full; j0 += 8) {
+    int4 v[8];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {  // consecutive lanes read consecutive words: no bank conflicts
-      const int e = j * kKeyTile + q * 32 + lane;
-      if (e < k) any |= idx_ok(row[e], Lk);
+    for (int q = 0; q < 8; ++q)
+      v[q] = j0 + q < full ? *reinterpret_cast<const int4*>(row + (j0 + q) * kKeyTile + 4 * lane)
+                           : make_int4(-1, -1, -1, -1);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const bool a = idx_ok(v[q].x, Lk), b = idx_ok(v[q].y, Lk), c = idx_ok(v[q].z, Lk), d = idx_ok(v[q].w, Lk);
+      if (a | b | c | d) bits |= 1u << (j0 + q);
+      if (kAll && (a & b & c & d)) all_bits |= 1u << (j0 + q);
     }
-    if (__any_sync(0xffffffffu, any)) mask |= 1u << j;
   }
-  return mask;
+  if (full * kKeyTile < k) {  // the ragged last tile (never all-valid: it has fewer than 128 entries)
+    bool any = false;
+    for (int e = full * kKeyTile + lane; e < k; e += 32) any |= idx_ok(row[e], Lk);
+    if (any) bits |= 1u << full;
+  }
+  if (kAll) *all_valid = __reduce_and_sync(0xffffffffu, all_bits);
+  return __reduce_or_sync(0xffffffffu, bits);
 }
 
 __device__ __forceinline__ void cp_async4(uint32_t dst, const void* src) {
   asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
 }
 
-// Warp reduce-scatter of 64 per-lane values: afterwards lane l holds, in v[0] and v[1],
-// the reduction over all 32 lanes of heads 2l and 2l+1.
-template <bool kMax, int W>
-__device__ __forceinline__ void reduce_scatter_stage(float (&v)[64], int lane) {
-  constexpr int o = W / 4;  // lane offset: 16, 8, 4, 2, 1 for W = 64 .. 4
-  const bool upper = (lane & o) != 0;
-#pragma unroll
-  for (int i = 0; i < W / 2; ++i) {
-    const float send = upper ? v[i] : v[i + W / 2];
-    const float keep = upper ? v[i + W / 2] : v[i];
-    const float recv = __shfl_xor_sync(0xffffffffu, send, o);
-    v[i] = kMax ? fmaxf(keep, recv) : keep + recv;
-  }
+// Half-quarter TMEM access (.16x32bx2): threads 0-15 of the warp address lanes base + t at
+// columns [c, c + 32), threads 16-31 the same 16 lanes at columns [c + kOff, c + kOff + 32).
+template <int kOff>
+__device__ __forceinline__ void tmem_ld_half32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x32bx2.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32], %33;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]),
+        "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]),
+        "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr), "n"(kOff)
+      : "memory");
 }
-template <bool kMax>
-__device__ __forceinline__ void warp_reduce_scatter64(float (&v)[64], int lane) {
-  reduce_scatter_stage<kMax, 64>(v, lane);
-  reduce_scatter_stage<kMax, 32>(v, lane);
-  reduce_scatter_stage<kMax, 16>(v, lane);
-  reduce_scatter_stage<kMax, 8>(v, lane);
-  reduce_scatter_stage<kMax, 4>(v, lane);
+template <int kOff>
+__device__ __forceinline__ void tmem_st_half32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.16x32bx2.x32.b32 [%0], %1, "
+      "{%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,"
+      "%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32,%33};" ::"r"(taddr),
+      "n"(kOff), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]),
+      "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]),
+      "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+
+template <int kOff>
+__device__ __forceinline__ void tmem_st_half16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.16x32bx2.x16.b32 [%0], %1, "
+      "{%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17};" ::"r"(taddr),
+      "n"(kOff), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
 }
 
 __device__ __forceinline__ void softmax_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
-// Named barrier over the 128 softmax threads that also ORs a predicate across them.
-__device__ __forceinline__ bool softmax_bar_or(bool pred) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\t"
-      "setp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.or.pred q, 1, 128, p;\n\t"
-      "selp.u32 %0, 1, 0, q;\n\t}"
-      : "=r"(r)
-      : "r"((uint32_t)pred)
-      : "memory");
-  return r != 0;
-}
 
 // Softmax threads: once the producers and the MMA warp released buffer `buf` (used by local
 // token i), fetch the index row of token `next` into it with cp.async.
@@ -183,13 +202,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;
   uint8_t* sRing = smem + kQBytes;
-  uint8_t* sP = sRing + kRingSlots * kChunkBytes;
-  int32_t* sIdx = reinterpret_cast<int32_t*>(sP + 2 * kPBytes);  // [2][kMaxK]
+  int32_t* sIdx = reinterpret_cast<int32_t*>(sRing + kRingSlots * kChunkBytes);  // [2][kMaxK]
   __shared__ Barriers bar;
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_flag;
-  __shared__ SoftShared ss;
-
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   if (threadIdx.x == 0) {
     mbar_init(&bar.q_full, 1);
@@ -237,16 +253,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = __all_sync(0xffffffffu, mbar_wait(&bar.idx_full[buf], (i >> 1) & 1, &abort_flag, p.err));
       if (!ok) break;
       const int32_t* row = sIdx + buf * kMaxK;
-      const uint32_t mask = tile_mask_of_row(row, k, Lk, lane);
+      const uint32_t mask = tile_mask_of_row<false>(row, k, Lk, lane);
       if (!mask) {
         if (lane == 0) mbar_arrive(&bar.idx_empty[buf]);
         continue;
       }
       const int J = __popc(mask);
       const size_t kv_row0 = (size_t)(tok / p.Lq) * Lk;  // first K/V row of this token's batch
-      // warp w gathers tile rows w, w+3, w+6, ...: lane l holds the K/V row of the warp's
+      // warp w gathers tile rows w, w+6, w+12, ...: lane l holds the K/V row of the warp's
       // l-th row (ra) and (32+l)-th row (rb)
-      const int n_rows_w = (kKeyTile - warp + kProducerWarps - 1) / kProducerWarps;  // 43, 43, 42
+      const int n_rows_w = (kKeyTile - warp + kProducerWarps - 1) / kProducerWarps;  // 22 or 21
       int ra_prev = 0, rb_prev = 0, ra_cur = 0, rb_cur = 0;
       uint32_t m = mask;
       for (int step = 0; step <= J && ok; ++step) {
@@ -300,27 +316,28 @@ __global__ void __launch_bounds__(kThreads, 1)
     int it = 0;
     uint32_t g = 0;  // global tile counter
     bool ok = true;
-    const uint32_t sQa = smem_u32(sQ), sRa = smem_u32(sRing), sPa = smem_u32(sP);
-    const uint32_t idesc_s = idesc_bf16_f32(128, kH, false, false);
-    const uint32_t idesc_o = idesc_bf16_f32(128, kH, true, true);
+    const uint32_t sQa = smem_u32(sQ), sRa = smem_u32(sRing);
+    const uint32_t idesc_s = idesc_bf16_f32(kH, kKeyTile, false, false);  // S: M = 64 heads, N = 128 keys
+    const uint32_t idesc_o = idesc_bf16_f32(kH, kD, false, true);         // O: N = 256 d_v, V MN-major
     int i = 0;
     for (int tok = blockIdx.x; tok < p.n_tok && ok; tok += gridDim.x, ++i) {
       const int buf = i & 1;
       ok = __all_sync(0xffffffffu, mbar_wait(&bar.idx_full[buf], (i >> 1) & 1, &abort_flag, p.err));
       if (!ok) break;
-      const uint32_t mask = tile_mask_of_row(sIdx + buf * kMaxK, k, Lk, lane);
+      const uint32_t mask = tile_mask_of_row<false>(sIdx + buf * kMaxK, k, Lk, lane);
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar.idx_empty[buf]);  // only the mask was needed
       if (!mask) continue;
       const int J = __popc(mask);
-      const int ob = it & 1;
+      const int hf = it & 1;  // this token's TMEM half (lane offset 16 * hf)
       if (lane == 0) {
+        const uint32_t t_half = tmem + (static_cast<uint32_t>(16 * hf) << 16);
         ok = mbar_wait(&bar.q_full, it & 1, &abort_flag, p.err);
         tc_fence_after();
         for (int step = 0; step <= J && ok; ++step) {
           if (step < J) {
             const uint32_t gs = g + step;
-            const uint32_t tS = tmem + kTmemS + (gs & 1) * kH;
+            const uint32_t tS = t_half + kTmemS + (gs & 1) * kKeyTile;
             // one wait per K tile: every producer thread arrives once all of its row copies of
             // the tile (all 4 chunks) have landed
             ok = mbar_wait(&bar.full[u & 1], (u >> 1) & 1, &abort_flag, p.err);
@@ -328,14 +345,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             fence_proxy_async_smem();  // cp.async (generic proxy) writes -> tensor core reads
             tc_fence_after();
             {
-              const uint64_t da0 = smem_desc_sw128(sRa + (u & 1) * 4 * kChunkBytes, 16, 1024);
-              const uint64_t db0 = smem_desc_sw128(sQa, 16, 1024);
+              const uint64_t da0 = smem_desc_sw128(sQa, 16, 1024);
+              const uint64_t db0 = smem_desc_sw128(sRa + (u & 1) * 4 * kChunkBytes, 16, 1024);
 #pragma unroll
               for (int c = 0; c < 4; ++c)
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)  // descriptor start address field is in 16-byte units
-                  mma_ss(tS, da0 + (uint64_t)((c * kChunkBytes + kk * 32) >> 4),
-                         db0 + (uint64_t)((c * kQChunkBytes + kk * 32) >> 4), idesc_s, (c | kk) != 0);
+                  mma_ss(tS, da0 + (uint64_t)((c * kQChunkBytes + kk * 32) >> 4),
+                         db0 + (uint64_t)((c * kChunkBytes + kk * 32) >> 4), idesc_s, (c | kk) != 0);
             }
             mma_commit(&bar.empty[u & 1]);
             ++u;
@@ -345,34 +362,30 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (step >= 1) {
             const int j = step - 1;
             const uint32_t gj = g + j;
-            if (j == 0) {  // O^T buffer ob must have been drained by the epilogue of token it-2
-              ok = mbar_wait(&bar.o_empty[ob], ((it >> 1) & 1) ^ 1, &abort_flag, p.err);
+            if (j == 0) {  // O in this half must have been drained by the epilogue of token it-2
+              ok = mbar_wait(&bar.o_empty[hf], ((it >> 1) & 1) ^ 1, &abort_flag, p.err);
               if (!ok) break;
             }
             ok = mbar_wait(&bar.p_ready[gj & 1], (gj >> 1) & 1, &abort_flag, p.err);
             if (!ok) break;
             tc_fence_after();
-            const uint32_t pbase = sPa + (gj & 1) * kPBytes;
+            const uint32_t tP = t_half + kTmemS + (gj & 1) * kKeyTile;  // P: bf16 pairs, 64 columns
             ok = mbar_wait(&bar.full[u & 1], (u >> 1) & 1, &abort_flag, p.err);  // the whole V tile
             if (!ok) break;
             fence_proxy_async_smem();
             tc_fence_after();
             {
-              // V^T chunk pair (2hv, 2hv+1): M = 128 d_v rows, the pair's slots are LBO apart
-              const uint64_t da0 = smem_desc_sw128(sRa + (u & 1) * 4 * kChunkBytes, kChunkBytes, 1024);
-              const uint64_t db0 = smem_desc_sw128(pbase, kPBytes, 1024);
-              const uint32_t acc0 = j > 0 ? 1u : 0u;
+              // V as MN-major B: 64-d_v chunks one slot (LBO) apart, 8-key groups 1024 B apart;
+              // 16 keys (one MMA) are 2048 B of the slot, 16 keys of P are 8 TMEM columns
+              const uint64_t db0 = smem_desc_sw128(sRa + (u & 1) * 4 * kChunkBytes, kChunkBytes, 1024);
 #pragma unroll
-              for (int hv = 0; hv < 2; ++hv)
-#pragma unroll
-                for (int kk = 0; kk < kKeyTile / 16; ++kk)
-                  mma_ss(tmem + ob * 128 + hv * kH, da0 + (uint64_t)((hv * 2 * kChunkBytes + kk * 2048) >> 4),
-                         db0 + (uint64_t)((kk * 2048) >> 4), idesc_o, kk > 0 ? 1u : acc0);
+              for (int kk = 0; kk < kKeyTile / 16; ++kk)
+                mma_ts(t_half, tP + kk * 8, db0 + (uint64_t)((kk * 2048) >> 4), idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
             }
             mma_commit(&bar.empty[u & 1]);
             ++u;
             mma_commit(&bar.pv_done);
-            if (j == J - 1) mma_commit(&bar.o_full[ob]);
+            if (j == J - 1) mma_commit(&bar.o_full[hf]);
           }
         }
       }
@@ -383,15 +396,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ softmax + epilogue
-    const int sw = warp - kSoftmaxWarp0;  // 0..3
-    const int quarter = warp & 3;         // TMEM lane quarter this warp may access
-    const int kl = quarter * 32 + lane;   // key lane of a tile / d_v row of O^T
-    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-    const int tid = sw * 32 + lane;       // 0..127
+    const int quarter = warp & 3;  // TMEM lane quarter this warp may access: heads 16q..16q+15
+    const int kh = lane >> 4;      // keys 64kh..64kh+63 of a tile, d_v 128kh..128kh+127 of O
+    const int h = quarter * 16 + (lane & 15);
+    const int tid = (warp - kSoftmaxWarp0) * 32 + lane;  // 0..127
     int it = 0;
     uint32_t g = 0;
     bool ok = true;
-    // No early exit in this loop: the four softmax warps meet at named barriers, so after an
+    // No early exit in this loop: the four softmax warps meet at a named barrier, so after an
     // abort every thread keeps walking the same barrier sequence (waits then fail fast).
     const uint32_t sIdx_a = smem_u32(sIdx);
     // index rows of this CTA's first two tokens
@@ -407,7 +419,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int buf = i & 1;
       ok = mbar_wait(&bar.idx_full[buf], (i >> 1) & 1, &abort_flag, p.err) && ok;
       const int32_t* row = sIdx + buf * kMaxK;
-      const uint32_t mask = tile_mask_of_row(row, k, Lk, lane);
+      uint32_t all_valid = 0;
+      const uint32_t mask = tile_mask_of_row<true>(row, k, Lk, lane, &all_valid);
       uint16_t* obase = p.O + (size_t)tok * kH * kD;
       if (!mask) {  // no valid entry: O = 0, lse = -inf
         for (int e = tid; e < kH * kD / 8; e += 128) reinterpret_cast<uint4*>(obase)[e] = make_uint4(0, 0, 0, 0);
@@ -417,194 +430,130 @@ __global__ void __launch_bounds__(kThreads, 1)
         continue;
       }
       const int J = __popc(mask);
-      const int ob = it & 1;
-      if (tid < kH) ss.m_ref[tid] = -INFINITY;
-      float lsum0 = 0.0f, lsum1 = 0.0f;  // row sums of heads 2*lane, 2*lane+1 over this warp's keys
+      const int hf = it & 1;
+      const uint32_t t_lanes = tmem + (static_cast<uint32_t>(quarter * 32 + hf * 16) << 16);
+      float m_run = -INFINITY;  // reference max of head h (log2 units), same in both threads of the head
+      float l_run = 0.0f;       // sum of p over this thread's keys
       uint32_t m = mask;
       for (int jj = 0; jj < J; ++jj) {
         const int j = __ffs(m) - 1;
         m &= m - 1;
         const uint32_t gs = g + jj;
-        const int e = j * kKeyTile + kl;
-        const int s_idx = e < k ? row[e] : -1;
-        const bool valid = idx_ok(s_idx, Lk);
-        if (s_idx >= Lk) raise_device_error(p.err, kErrDeviceBounds);
+        // validity of this thread's 64 keys (bit i: entry j*128 + 64kh + i); whole valid tiles skip it
+        uint32_t v_lo = 0xffffffffu, v_hi = 0xffffffffu;
+        if (!((all_valid >> j) & 1u)) {
+          v_lo = v_hi = 0;
+          bool oob = false;
+          const int e0 = j * kKeyTile + kh * 64;
+#pragma unroll 4
+          for (int q4 = 0; q4 < 16; ++q4) {
+            const int4 w = *reinterpret_cast<const int4*>(row + e0 + 4 * q4);  // inside the row buffer
+            const int e = e0 + 4 * q4;
+            const int s0 = e < k ? w.x : -1, s1 = e + 1 < k ? w.y : -1;
+            const int s2 = e + 2 < k ? w.z : -1, s3 = e + 3 < k ? w.w : -1;
+            oob |= (s0 >= Lk) | (s1 >= Lk) | (s2 >= Lk) | (s3 >= Lk);
+            const uint32_t nib = (idx_ok(s0, Lk) ? 1u : 0u) | (idx_ok(s1, Lk) ? 2u : 0u) | (idx_ok(s2, Lk) ? 4u : 0u) |
+                                 (idx_ok(s3, Lk) ? 8u : 0u);
+            if (q4 < 8) v_lo |= nib << (4 * q4);
+            else v_hi |= nib << (4 * q4 - 32);
+          }
+          if (oob) raise_device_error(p.err, kErrDeviceBounds);
+        }
         ok = mbar_wait(&bar.s_full[gs & 1], (gs >> 1) & 1, &abort_flag, p.err) && ok;
         tc_fence_after();
-        const uint32_t tS = tmem + lane_off + kTmemS + (gs & 1) * kH;
-        uint8_t* prow = sP + (gs & 1) * kPBytes + kl * 128;
-        uint32_t u0[32], u1[32];  // scores, then p (fp32 bits)
-        tmem_ld32_nowait(tS, u0);
-        tmem_ld32_nowait(tS + 32, u1);
-        tmem_wait_ld_regs2(u0, u1);
-        // Speculative pass: P against the current per-head reference max, and whether any score
-        // exceeds it by more than 2^8 (then the tile is redone after a reduction).  The first
-        // tile of a token always takes the reduction path (its reference is still -inf).
-        bool over = jj == 0;
-        if (!over) {
+        const uint32_t tS = t_lanes + kTmemS + (gs & 1) * kKeyTile;
+        uint32_t sa[32], sb[32];  // scores of keys 64kh + [0, 32) and 64kh + [32, 64)
+        tmem_ld_half32<64>(tS, sa);
+        tmem_ld_half32<64>(tS + 32, sb);
+        tmem_wait_ld_regs2(sa, sb);
+        float mt = -INFINITY;
 #pragma unroll
-          for (int c8 = 0; c8 < 8; ++c8) {
-            const float4 ma = *reinterpret_cast<const float4*>(&ss.m_ref[c8 * 8]);
-            const float4 mb = *reinterpret_cast<const float4*>(&ss.m_ref[c8 * 8 + 4]);
-            const float mr[8] = {ma.x, ma.y, ma.z, ma.w, mb.x, mb.y, mb.z, mb.w};
-            uint32_t w4[4];
+        for (int x = 0; x < 32; ++x) {
+          if ((v_lo >> x) & 1u) mt = fmaxf(mt, __uint_as_float(sa[x]));
+          if ((v_hi >> x) & 1u) mt = fmaxf(mt, __uint_as_float(sb[x]));
+        }
+        mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 16));  // the tile's max of head h
+        const float xt = mt * p.scale_log2;
+        bool resc = false;
+        float alpha = 1.0f;
+        if (m_run == -INFINITY) {
+          m_run = xt;  // first tile of the token: its PV starts O from zero
+        } else if (xt > m_run + kLazyRescale) {
+          alpha = fast_exp2(m_run - xt);
+          m_run = xt;
+          resc = true;
+        }
+        l_run *= alpha;
+        // P = 2^(x - m_run) (0 for invalid keys) as bf16 pairs over the tile's first 64 columns:
+        // keys 64kh + [0, 64) -> columns 32kh + [0, 32), the A operand of this tile's PV MMA
+        // (the S values were all read above, by both halves of the warp)
+        {
+          uint32_t pw[16];
 #pragma unroll
-            for (int qq = 0; qq < 4; ++qq) {
-              const int h = c8 * 8 + 2 * qq;
-              uint32_t& r0 = h < 32 ? u0[h] : u1[h - 32];
-              uint32_t& r1 = h + 1 < 32 ? u0[h + 1] : u1[h + 1 - 32];
-              const float x0 = fmaf(__uint_as_float(r0), p.scale_log2, -mr[2 * qq]);
-              const float x1 = fmaf(__uint_as_float(r1), p.scale_log2, -mr[2 * qq + 1]);
-              over |= valid && (x0 > kLazyRescale || x1 > kLazyRescale);
-              const float p0 = valid ? fast_exp2(x0) : 0.0f;
-              const float p1 = valid ? fast_exp2(x1) : 0.0f;
-              r0 = __float_as_uint(p0);
-              r1 = __float_as_uint(p1);
-              w4[qq] = pack_bf16x2(p0, p1);
-            }
-            *reinterpret_cast<uint4*>(prow + ((c8 ^ (kl & 7)) << 4)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+          for (int x2 = 0; x2 < 16; ++x2) {
+            const int x = 2 * x2;
+            const float p0 = (v_lo >> x) & 1u ? fast_exp2(fmaf(__uint_as_float(sa[x]), p.scale_log2, -m_run)) : 0.0f;
+            const float p1 = (v_lo >> (x + 1)) & 1u ? fast_exp2(fmaf(__uint_as_float(sa[x + 1]), p.scale_log2, -m_run)) : 0.0f;
+            l_run += p0 + p1;
+            pw[x2] = pack_bf16x2(p0, p1);
+          }
+          tmem_st_half16<32>(tS, pw);  // columns 32kh + [0, 16)
+#pragma unroll
+          for (int x2 = 0; x2 < 16; ++x2) {
+            const int x = 2 * x2;
+            const float p0 = (v_hi >> x) & 1u ? fast_exp2(fmaf(__uint_as_float(sb[x]), p.scale_log2, -m_run)) : 0.0f;
+            const float p1 = (v_hi >> (x + 1)) & 1u ? fast_exp2(fmaf(__uint_as_float(sb[x + 1]), p.scale_log2, -m_run)) : 0.0f;
+            l_run += p0 + p1;
+            pw[x2] = pack_bf16x2(p0, p1);
+          }
+          tmem_st_half16<32>(tS + 16, pw);  // columns 32kh + [16, 32)
+        }
+        if (__any_sync(0xffffffffu, resc)) {
+          // O must hold every PV of this token up to tile jj-1 before it is rescaled (and this
+          // tile's PV, which waits for p_ready, comes after)
+          ok = mbar_wait(&bar.pv_done, (gs - 1) & 1, &abort_flag, p.err) && ok;
+          tc_fence_after();
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint32_t o[32];
+            tmem_ld_half32<128>(t_lanes + c * 32, o);
+            tmem_wait_ld_regs(o);
+#pragma unroll
+            for (int x = 0; x < 32; ++x) o[x] = __float_as_uint(__uint_as_float(o[x]) * alpha);
+            tmem_st_half32<128>(t_lanes + c * 32, o);
           }
         }
-        if (!softmax_bar_or(over)) {
-          float pv[kH];
-#pragma unroll
-          for (int h = 0; h < 32; ++h) {
-            pv[h] = __uint_as_float(u0[h]);
-            pv[32 + h] = __uint_as_float(u1[h]);
-          }
-          warp_reduce_scatter64<false>(pv, lane);
-          lsum0 += pv[0];
-          lsum1 += pv[1];
-        } else {
-          // reduction path: new per-head reference, rescale O^T if it moved, P from scratch
-          float red[kH];
-          {
-            uint32_t t0[32], t1[32];
-            tmem_ld32_nowait(tS, t0);
-            tmem_ld32_nowait(tS + 32, t1);
-            tmem_wait_ld_regs2(t0, t1);
-#pragma unroll
-            for (int h = 0; h < 32; ++h) {
-              red[h] = valid ? __uint_as_float(t0[h]) * p.scale_log2 : -INFINITY;
-              red[32 + h] = valid ? __uint_as_float(t1[h]) * p.scale_log2 : -INFINITY;
-            }
-          }
-          warp_reduce_scatter64<true>(red, lane);
-          ss.wred[sw][2 * lane] = red[0];
-          ss.wred[sw][2 * lane + 1] = red[1];
-          softmax_bar();
-          bool resc = false;
-          if (tid < kH) {
-            const float mt = fmaxf(fmaxf(ss.wred[0][tid], ss.wred[1][tid]), fmaxf(ss.wred[2][tid], ss.wred[3][tid]));
-            const float mo = ss.m_ref[tid];
-            float alpha = 1.0f, mn = mo;
-            if (mo == -INFINITY) {
-              mn = mt;
-            } else if (mt > mo + kLazyRescale) {
-              mn = mt;
-              alpha = fast_exp2(mo - mt);
-              resc = true;
-            }
-            ss.m_ref[tid] = mn;
-            ss.alpha[tid] = alpha;
-          }
-          if (softmax_bar_or(resc)) {
-            // O^T must hold every PV of this token up to tile jj-1 before it is rescaled
-            ok = mbar_wait(&bar.pv_done, (gs - 1) & 1, &abort_flag, p.err) && ok;
-            tc_fence_after();
-#pragma unroll
-            for (int hv = 0; hv < 2; ++hv) {
-#pragma unroll
-              for (int c = 0; c < 2; ++c) {
-                uint32_t u[32];
-                const uint32_t tO = tmem + lane_off + ob * 128 + hv * kH + c * 32;
-                tmem_ld32_nowait(tO, u);
-                tmem_wait_ld_regs(u);
-#pragma unroll
-                for (int h = 0; h < 32; ++h) u[h] = __float_as_uint(__uint_as_float(u[h]) * ss.alpha[c * 32 + h]);
-                tmem_st32(tO, u);
-              }
-            }
-            tmem_wait_st();
-            lsum0 *= ss.alpha[2 * lane];
-            lsum1 *= ss.alpha[2 * lane + 1];
-          }
-          tmem_ld32_nowait(tS, u0);
-          tmem_ld32_nowait(tS + 32, u1);
-          tmem_wait_ld_regs2(u0, u1);
-#pragma unroll
-          for (int c8 = 0; c8 < 8; ++c8) {
-            const float4 ma = *reinterpret_cast<const float4*>(&ss.m_ref[c8 * 8]);
-            const float4 mb = *reinterpret_cast<const float4*>(&ss.m_ref[c8 * 8 + 4]);
-            const float mr[8] = {ma.x, ma.y, ma.z, ma.w, mb.x, mb.y, mb.z, mb.w};
-            uint32_t w4[4];
-#pragma unroll
-            for (int qq = 0; qq < 4; ++qq) {
-              const int h = c8 * 8 + 2 * qq;
-              const uint32_t s0 = h < 32 ? u0[h] : u1[h - 32];
-              const uint32_t s1 = h + 1 < 32 ? u0[h + 1] : u1[h + 1 - 32];
-              float p0 = 0.0f, p1 = 0.0f;
-              if (valid) {
-                p0 = fast_exp2(fmaf(__uint_as_float(s0), p.scale_log2, -mr[2 * qq]));
-                p1 = fast_exp2(fmaf(__uint_as_float(s1), p.scale_log2, -mr[2 * qq + 1]));
-              }
-              (h < 32 ? u0[h] : u1[h - 32]) = __float_as_uint(p0);
-              (h + 1 < 32 ? u0[h + 1] : u1[h + 1 - 32]) = __float_as_uint(p1);
-              w4[qq] = pack_bf16x2(p0, p1);
-            }
-            *reinterpret_cast<uint4*>(prow + ((c8 ^ (kl & 7)) << 4)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
-          }
-          float pv[kH];
-#pragma unroll
-          for (int h = 0; h < 32; ++h) {
-            pv[h] = __uint_as_float(u0[h]);
-            pv[32 + h] = __uint_as_float(u1[h]);
-          }
-          warp_reduce_scatter64<false>(pv, lane);
-          lsum0 += pv[0];
-          lsum1 += pv[1];
-        }
-        fence_proxy_async_smem();
+        tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&bar.p_ready[gs & 1]);
       }
-      // ---- epilogue of this token
-      ss.wred[sw][2 * lane] = lsum0;
-      ss.wred[sw][2 * lane + 1] = lsum1;
-      softmax_bar();
-      if (tid < kH) {  // per-head row sum -> 1/l (kept in ss.alpha) and log-sum-exp
-        const float l = ss.wred[0][tid] + ss.wred[1][tid] + ss.wred[2][tid] + ss.wred[3][tid];
-        ss.alpha[tid] = 1.0f / l;
-        if (p.lse) p.lse[(size_t)tok * kH + tid] = (ss.m_ref[tid] + __log2f(l)) * 0.69314718055994531f;
-      }
-      softmax_bar();
-      ok = mbar_wait(&bar.o_full[ob], (it >> 1) & 1, &abort_flag, p.err) && ok;
+      // ---- epilogue of this token: head h, d_v 128kh..128kh+127
+      const float l = l_run + __shfl_xor_sync(0xffffffffu, l_run, 16);
+      const float inv = 1.0f / l;
+      if (p.lse && kh == 0) p.lse[(size_t)tok * kH + h] = (m_run + __log2f(l)) * 0.69314718055994531f;
+      ok = mbar_wait(&bar.o_full[hf], (it >> 1) & 1, &abort_flag, p.err) && ok;
       tc_fence_after();
       {
-        __nv_bfloat16* ob16 = reinterpret_cast<__nv_bfloat16*>(obase);
+        uint4* orow = reinterpret_cast<uint4*>(obase + (size_t)h * kD + kh * 128);
 #pragma unroll
-        for (int hv = 0; hv < 2; ++hv) {
-          const int dv = hv * 128 + kl;  // this lane's d_v row of O^T
-          uint32_t u0[32], u1[32];
-          tmem_ld32_nowait(tmem + lane_off + ob * 128 + hv * kH, u0);
-          tmem_ld32_nowait(tmem + lane_off + ob * 128 + hv * kH + 32, u1);
-          tmem_wait_ld_regs2(u0, u1);
+        for (int c = 0; c < 4; ++c) {
+          uint32_t o[32];
+          tmem_ld_half32<128>(t_lanes + c * 32, o);
+          tmem_wait_ld_regs(o);
 #pragma unroll
-          for (int h4 = 0; h4 < 16; ++h4) {
-            const float4 il = *reinterpret_cast<const float4*>(&ss.alpha[h4 * 4]);
-            const float inv[4] = {il.x, il.y, il.z, il.w};
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const int h = h4 * 4 + q;
-              const float o = __uint_as_float(h < 32 ? u0[h] : u1[h - 32]) * inv[q];
-              ob16[(size_t)h * kD + dv] = __float2bfloat16_rn(o);
-            }
+          for (int q = 0; q < 4; ++q) {
+            uint4 w;
+            w.x = pack_bf16x2(__uint_as_float(o[8 * q + 0]) * inv, __uint_as_float(o[8 * q + 1]) * inv);
+            w.y = pack_bf16x2(__uint_as_float(o[8 * q + 2]) * inv, __uint_as_float(o[8 * q + 3]) * inv);
+            w.z = pack_bf16x2(__uint_as_float(o[8 * q + 4]) * inv, __uint_as_float(o[8 * q + 5]) * inv);
+            w.w = pack_bf16x2(__uint_as_float(o[8 * q + 6]) * inv, __uint_as_float(o[8 * q + 7]) * inv);
+            orow[c * 4 + q] = w;
           }
         }
       }
       tc_fence_before();
-      mbar_arrive(&bar.o_empty[ob]);
-      softmax_bar();  // wred / m_ref are rewritten by the next token; the row has been read
+      mbar_arrive(&bar.o_empty[hf]);
+      softmax_bar();  // every softmax thread has read the row before it is refilled
       refill_idx_row(p, bar, sIdx_a, buf, i, tok + 2 * gridDim.x, tid, abort_flag, ok);
       g += J;
       ++it;
