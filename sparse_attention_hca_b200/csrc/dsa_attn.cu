@@ -30,7 +30,7 @@
 //     the MMA thread waits once per tile and issues a proxy fence after it so the tensor core
 //     sees the generic-proxy writes.  (Measured on B200: this reaches ~105 GB/s per SM from L2,
 //     TMA tile::gather4 of 4 x 128 B rows ~16 GB/s.)
-//     Q (32 KB, TMA) is reloaded per token once the previous token's last S MMA is done.
+//     Q (32 KB, TMA, double-buffered) is loaded as soon as the producers start a token.
 //   * Warp 6, lane 0 issues every MMA.  Warps 7-10: softmax.  Warp 7+q owns heads 16q..16q+15
 //     (TMEM lane quarter q); thread t of it holds head 16q + t%16 and keys 64(t/16)..+63 of a
 //     tile.  Online softmax per head with a lazy reference max: the first tile sets it, a later
@@ -62,7 +62,7 @@ constexpr int kQChunkBytes = kH * 128;     // 64 heads x 64 bf16
 constexpr int kQBytes = 4 * kQChunkBytes;  // 32 KB
 constexpr int kMaxK = 4096;                // 32 tiles: one bit per tile in a 32-bit mask
 constexpr int kIdxBytes = kMaxK * 4;  // one index row
-constexpr int kSmemBytes = kQBytes + kRingSlots * kChunkBytes + 2 * kIdxBytes + 1024;
+constexpr int kSmemBytes = 2 * kQBytes + kRingSlots * kChunkBytes + 2 * kIdxBytes + 1024;  // 225 KB
 // Gather throughput scales with the number of producer warps; 11 warps cap a thread at 168
 // registers, which the softmax (64 scores per thread) stays well inside.
 constexpr int kProducerWarps = 6;
@@ -84,7 +84,7 @@ struct Params {
 };
 
 struct __align__(8) Barriers {
-  uint64_t q_full, q_empty;
+  uint64_t q_full[2], q_empty[2];  // Q double buffer, by the count of tokens with work
   uint64_t full[2];   // ring group g holds a whole K or V tile (192 producer-thread arrivals)
   uint64_t empty[2];  // the MMAs that read group g have completed
   uint64_t s_full[2];
@@ -200,16 +200,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     dsa_attn_kernel(const __grid_constant__ CUtensorMap map_q, const Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sQ = smem;
-  uint8_t* sRing = smem + kQBytes;
+  uint8_t* sQ = smem;  // [2][kQBytes]
+  uint8_t* sRing = smem + 2 * kQBytes;
   int32_t* sIdx = reinterpret_cast<int32_t*>(sRing + kRingSlots * kChunkBytes);  // [2][kMaxK]
   __shared__ Barriers bar;
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_flag;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   if (threadIdx.x == 0) {
-    mbar_init(&bar.q_full, 1);
-    mbar_init(&bar.q_empty, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bar.q_full[s], 1);
+      mbar_init(&bar.q_empty[s], 1);
+    }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bar.full[s], kProducerWarps * 32);
       mbar_init(&bar.empty[s], 1);
@@ -259,6 +261,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         continue;
       }
       const int J = __popc(mask);
+      if (warp == 0) {
+        // Q of this token into its buffer, ahead of the token's first K tile: the buffer was last
+        // read by the S MMAs of token it-2
+        const int qb = it & 1;
+        ok = __all_sync(0xffffffffu, mbar_wait(&bar.q_empty[qb], ((it >> 1) & 1) ^ 1, &abort_flag, p.err));
+        if (ok && lane == 0) {
+          mbar_arrive_expect_tx(&bar.q_full[qb], kQBytes);
+          for (int c = 0; c < 4; ++c)
+            tma_load_3d(sQ + qb * kQBytes + c * kQChunkBytes, &map_q, &bar.q_full[qb], c * 64, 0, tok);
+        }
+      }
       const size_t kv_row0 = (size_t)(tok / p.Lq) * Lk;  // first K/V row of this token's batch
       // warp w gathers tile rows w, w+6, w+12, ...: lane l holds the K/V row of the warp's
       // l-th row (ra) and (32+l)-th row (rb)
@@ -292,15 +305,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           cp_async_arrive_noinc(&bar.full[u & 1]);
           ++u;
-          if (is_k && step == 0 && warp == 0) {
-            // Q of this token (after its first K tile is in flight), once the previous token's
-            // last S^T MMA no longer reads the buffer
-            ok = __all_sync(0xffffffffu, mbar_wait(&bar.q_empty, (it & 1) ^ 1, &abort_flag, p.err));
-            if (ok && lane == 0) {
-              mbar_arrive_expect_tx(&bar.q_full, kQBytes);
-              for (int c = 0; c < 4; ++c) tma_load_3d(sQ + c * kQChunkBytes, &map_q, &bar.q_full, c * 64, 0, tok);
-            }
-          }
         }
         ra_prev = ra_cur;
         rb_prev = rb_cur;
@@ -332,7 +336,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int hf = it & 1;  // this token's TMEM half (lane offset 16 * hf)
       if (lane == 0) {
         const uint32_t t_half = tmem + (static_cast<uint32_t>(16 * hf) << 16);
-        ok = mbar_wait(&bar.q_full, it & 1, &abort_flag, p.err);
+        const int qb = it & 1;
+        ok = mbar_wait(&bar.q_full[qb], (it >> 1) & 1, &abort_flag, p.err);
         tc_fence_after();
         for (int step = 0; step <= J && ok; ++step) {
           if (step < J) {
@@ -345,7 +350,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             fence_proxy_async_smem();  // cp.async (generic proxy) writes -> tensor core reads
             tc_fence_after();
             {
-              const uint64_t da0 = smem_desc_sw128(sQa, 16, 1024);
+              const uint64_t da0 = smem_desc_sw128(sQa + qb * kQBytes, 16, 1024);
               const uint64_t db0 = smem_desc_sw128(sRa + (u & 1) * 4 * kChunkBytes, 16, 1024);
 #pragma unroll
               for (int c = 0; c < 4; ++c)
@@ -357,7 +362,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mma_commit(&bar.empty[u & 1]);
             ++u;
             mma_commit(&bar.s_full[gs & 1]);
-            if (step == J - 1) mma_commit(&bar.q_empty);
+            if (step == J - 1) mma_commit(&bar.q_empty[qb]);
           }
           if (step >= 1) {
             const int j = step - 1;
@@ -466,13 +471,27 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld_half32<64>(tS, sa);
         tmem_ld_half32<64>(tS + 32, sb);
         tmem_wait_ld_regs2(sa, sb);
-        float mt = -INFINITY;
+        if (!((all_valid >> j) & 1u)) {  // partial tile: invalid keys score -inf, so their p is 0
 #pragma unroll
-        for (int x = 0; x < 32; ++x) {
-          if ((v_lo >> x) & 1u) mt = fmaxf(mt, __uint_as_float(sa[x]));
-          if ((v_hi >> x) & 1u) mt = fmaxf(mt, __uint_as_float(sb[x]));
+          for (int x = 0; x < 32; ++x) {
+            if (!((v_lo >> x) & 1u)) sa[x] = 0xff800000u;
+            if (!((v_hi >> x) & 1u)) sb[x] = 0xff800000u;
+          }
         }
-        mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 16));  // the tile's max of head h
+        float mt;
+        {
+          float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
+#pragma unroll
+          for (int x = 0; x < 32; x += 2) {
+            m0 = fmaxf(m0, __uint_as_float(sa[x]));
+            m1 = fmaxf(m1, __uint_as_float(sa[x + 1]));
+            m2 = fmaxf(m2, __uint_as_float(sb[x]));
+            m3 = fmaxf(m3, __uint_as_float(sb[x + 1]));
+          }
+          mt = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
+        }
+        mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 16));  // the tile's max of head h (finite:
+                                                                // a tile in the mask has a valid key)
         const float xt = mt * p.scale_log2;
         bool resc = false;
         float alpha = 1.0f;
@@ -489,24 +508,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         // (the S values were all read above, by both halves of the warp)
         {
           uint32_t pw[16];
+          float la = 0.0f, lb = 0.0f;
 #pragma unroll
           for (int x2 = 0; x2 < 16; ++x2) {
-            const int x = 2 * x2;
-            const float p0 = (v_lo >> x) & 1u ? fast_exp2(fmaf(__uint_as_float(sa[x]), p.scale_log2, -m_run)) : 0.0f;
-            const float p1 = (v_lo >> (x + 1)) & 1u ? fast_exp2(fmaf(__uint_as_float(sa[x + 1]), p.scale_log2, -m_run)) : 0.0f;
-            l_run += p0 + p1;
+            const float p0 = fast_exp2(fmaf(__uint_as_float(sa[2 * x2]), p.scale_log2, -m_run));
+            const float p1 = fast_exp2(fmaf(__uint_as_float(sa[2 * x2 + 1]), p.scale_log2, -m_run));
+            la += p0;
+            lb += p1;
             pw[x2] = pack_bf16x2(p0, p1);
           }
           tmem_st_half16<32>(tS, pw);  // columns 32kh + [0, 16)
 #pragma unroll
           for (int x2 = 0; x2 < 16; ++x2) {
-            const int x = 2 * x2;
-            const float p0 = (v_hi >> x) & 1u ? fast_exp2(fmaf(__uint_as_float(sb[x]), p.scale_log2, -m_run)) : 0.0f;
-            const float p1 = (v_hi >> (x + 1)) & 1u ? fast_exp2(fmaf(__uint_as_float(sb[x + 1]), p.scale_log2, -m_run)) : 0.0f;
-            l_run += p0 + p1;
+            const float p0 = fast_exp2(fmaf(__uint_as_float(sb[2 * x2]), p.scale_log2, -m_run));
+            const float p1 = fast_exp2(fmaf(__uint_as_float(sb[2 * x2 + 1]), p.scale_log2, -m_run));
+            la += p0;
+            lb += p1;
             pw[x2] = pack_bf16x2(p0, p1);
           }
           tmem_st_half16<32>(tS + 16, pw);  // columns 32kh + [16, 32)
+          l_run += la + lb;
         }
         if (__any_sync(0xffffffffu, resc)) {
           // O must hold every PV of this token up to tile jj-1 before it is rescaled (and this
