@@ -270,8 +270,10 @@ hcadsa_status dsa_index_topk_noalloc(const int8_t* q_idx, const int8_t* k_idx, c
  *   K, V: [B, Lk, d] bf16
  *   idx : [B, Lq, k] int32, entries in [0, Lk) or < 0
  *   O   : [B, Lq, Hq, d] bf16 (written); lse: [B, Lq, Hq] fp32 or NULL
- * Requirements: d == 256, Hq == 64, 1 <= k.  An entry >= Lk is skipped and
- * recorded as HCADSA_ERR_DEVICE_BOUNDS.
+ * Requirements: d == 256, Hq == 64, 1 <= k <= 4096 (HCADSA_ERR_UNSUPPORTED
+ * otherwise), scale > 0 (HCADSA_ERR_SHAPE otherwise: the kernel takes each tile's maximum
+ * over the unscaled scores).  An entry >= Lk is skipped and recorded as
+ * HCADSA_ERR_DEVICE_BOUNDS.
  */
 hcadsa_status dsa_sparse_attn_fwd(const hcadsa_bf16* Q, const hcadsa_bf16* K, const hcadsa_bf16* V,
                                   const int32_t* idx, hcadsa_bf16* O, float* lse, int B, int Lq, int Lk, int Hq,

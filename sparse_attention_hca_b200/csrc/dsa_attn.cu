@@ -608,7 +608,7 @@ extern "C" hcadsa_status dsa_sparse_attn_fwd(const hcadsa_bf16* Q, const hcadsa_
                                              int Hq, int d, int k, float scale, hcadsa_stream stream) {
   using namespace hcadsa;
   if (!Q || !K || !V || !idx || !O) return HCADSA_ERR_NULL;
-  if (B < 0 || Lq < 0 || Lk < 0 || k <= 0) return HCADSA_ERR_SHAPE;
+  if (B < 0 || Lq < 0 || Lk < 0 || k <= 0 || !(scale > 0.0f)) return HCADSA_ERR_SHAPE;
   if (d != kD || Hq != kH || k > kMaxK) return HCADSA_ERR_UNSUPPORTED;
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(idx) ||
       (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))

@@ -95,6 +95,9 @@ def test_dsa_argument_errors(lib):
     assert a(FAKE, FAKE, FAKE, FAKE, FAKE, None, 1, 8, 8, 32, 256, 16, 0.06, None) == -4
     assert a(FAKE, FAKE, FAKE, FAKE, FAKE, None, 1, 8, 8, 64, 512, 16, 0.06, None) == -4
     assert a(FAKE, FAKE, MISALIGNED, FAKE, FAKE, None, 1, 8, 8, 64, 256, 16, 0.06, None) == -3
+    assert a(FAKE, FAKE, FAKE, FAKE, FAKE, None, 1, 8, 8, 64, 256, 4097, 0.06, None) == -4  # k > 4096
+    assert a(FAKE, FAKE, FAKE, FAKE, FAKE, None, 1, 8, 8, 64, 256, 16, 0.0, None) == -2    # scale <= 0
+    assert a(FAKE, FAKE, FAKE, FAKE, FAKE, None, 1, 8, 8, 64, 256, 16, float("nan"), None) == -2
 
 
 def test_workspace_size_queries(lib):
