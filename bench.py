@@ -303,6 +303,9 @@ def run_decode(hd, device, iters=20):
     ws_start = t - DEC.W + 1
     hws = hd.lib().hca_attn_fwd_workspace_size(B, 1, t, 16, 1, 512, n_c, 128, DEC.W)
     hws = torch.empty(max(hws, 16), dtype=torch.uint8, device=device)
+    # the DSA attention of 32 tokens splits each token's key tiles over several CTAs
+    dws = torch.empty(max(hd.lib().dsa_sparse_attn_fwd_workspace_size(B, 1, DEC.k), 16), dtype=torch.uint8,
+                      device=device)
 
     def step(ev=None):
         if ev: ev[0].record()
@@ -310,7 +313,7 @@ def run_decode(hd, device, iters=20):
         if ev: ev[1].record()
         hd.dsa_index_topk(q_idx, k_idx, w_idx, DEC.k, q_offset=t, idx=idx, workspace=ws)
         if ev: ev[2].record()
-        hd.dsa_sparse_attn_fwd(dQ, K, V, idx, O=dO)
+        hd.dsa_sparse_attn_fwd(dQ, K, V, idx, O=dO, workspace=dws)
         if ev: ev[3].record()
 
     for _ in range(3):

@@ -280,6 +280,30 @@ hcadsa_status dsa_sparse_attn_fwd(const hcadsa_bf16* Q, const hcadsa_bf16* K, co
                                   int d, int k, float scale, hcadsa_stream stream);
 
 /*
+ * The same computation with a caller-provided workspace, for calls with few query rows
+ * (decode batches): when B*Lq is at most half the number of SMs of the current device, each
+ * row's key tiles (128 entries of its index row each) are divided among up to 8 CTAs, which
+ * write unnormalised fp32 partial outputs and per-head (max, sum) pairs to the workspace; a
+ * second kernel on the same stream merges them (the online-softmax merge) and writes O and
+ * lse.  Same arguments, requirements and result as dsa_sparse_attn_fwd (up to the rounding of
+ * the merge), plus:
+ *   workspace      : device memory of at least dsa_sparse_attn_fwd_workspace_size(B, Lq, k)
+ *                    bytes, 16-byte aligned; caller-owned, contents need no initialisation and
+ *                    are scratch after the call.  Calls that share a workspace must be
+ *                    serialised on one stream.
+ *   workspace_bytes: its size.  HCADSA_ERR_WORKSPACE if the call splits and the workspace is
+ *                    NULL or smaller, HCADSA_ERR_ALIGN if it is misaligned.
+ * dsa_sparse_attn_fwd_workspace_size returns 0 when the call does not split (then workspace
+ * may be NULL and the call runs exactly as dsa_sparse_attn_fwd), and for invalid shapes; it
+ * depends on the current device's SM count.
+ */
+size_t dsa_sparse_attn_fwd_workspace_size(int B, int Lq, int k);
+hcadsa_status dsa_sparse_attn_fwd_ws(const hcadsa_bf16* Q, const hcadsa_bf16* K, const hcadsa_bf16* V,
+                                     const int32_t* idx, hcadsa_bf16* O, float* lse, int B, int Lq, int Lk, int Hq,
+                                     int d, int k, float scale, void* workspace, size_t workspace_bytes,
+                                     hcadsa_stream stream);
+
+/*
  * Attention output gate + virtual-head mix, fused (tensor-core GEMM + epilogue).  Source: the
  * mirrorspeed page, section "Hybrid sparse attention, 1/7 full context access" (last
  * paragraph), and the besthub page, "Core Architectural Innovations": low-rank gated attention

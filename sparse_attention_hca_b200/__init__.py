@@ -86,6 +86,10 @@ def lib() -> ctypes.CDLL:
             L.dsa_index_topk_noalloc.restype = I
             L.dsa_sparse_attn_fwd.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, F, P]
             L.dsa_sparse_attn_fwd.restype = I
+            L.dsa_sparse_attn_fwd_workspace_size.argtypes = [I, I, I]
+            L.dsa_sparse_attn_fwd_workspace_size.restype = S
+            L.dsa_sparse_attn_fwd_ws.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, F, P, S, P]
+            L.dsa_sparse_attn_fwd_ws.restype = I
             L.attn_gate_vha_fwd.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, P]
             L.attn_gate_vha_fwd.restype = I
             L.hca_compress_bwd.argtypes = [P, P, P, P, P, I, I, I, I, I, P]
@@ -328,8 +332,12 @@ def dsa_index_topk_noalloc(q_idx, k_idx, w_idx, k: int, *, q_offset: int = 0, id
 
 
 def dsa_sparse_attn_fwd(Q, K, V, idx, *, scale: float | None = None, O=None, lse=None,
-                        return_lse=False, stream=None):
-    """Q: [B, Lq, 64, 256]; K, V: [B, Lk, 256]; idx: [B, Lq, k] int32 -> O [B, Lq, 64, 256]."""
+                        return_lse=False, split: bool = True, workspace=None, stream=None):
+    """Q: [B, Lq, 64, 256]; K, V: [B, Lk, 256]; idx: [B, Lq, k] int32 -> O [B, Lq, 64, 256].
+
+    With split (the default), calls with few query rows divide each row's key tiles among
+    several CTAs through a workspace (allocated here unless given); split=False always runs
+    one CTA per query row."""
     _need(Q, torch.bfloat16, "Q")
     B, Lq, Hq, d = Q.shape
     _need(K, torch.bfloat16, "K")  # [B, Lk, d] (a [B, Lk, 1, d] view of one shared head is accepted)
@@ -352,9 +360,24 @@ def dsa_sparse_attn_fwd(Q, K, V, idx, *, scale: float | None = None, O=None, lse
     O = torch.empty_like(Q) if O is None else O
     if return_lse and lse is None:
         lse = torch.empty((B, Lq, Hq), dtype=torch.float32, device=Q.device)
-    st = lib().dsa_sparse_attn_fwd(_ptr(Q), _ptr(K), _ptr(V), _ptr(idx), _ptr(O), _ptr(lse), B, Lq, Lk,
+    L = lib()
+    if not split:
+        st = L.dsa_sparse_attn_fwd(_ptr(Q), _ptr(K), _ptr(V), _ptr(idx), _ptr(O), _ptr(lse), B, Lq, Lk,
                                    Hq, d, k, float(scale), _stream(stream))
-    _check(st, "dsa_sparse_attn_fwd")
+        _check(st, "dsa_sparse_attn_fwd")
+        return (O, lse) if return_lse else O
+    ws_bytes = L.dsa_sparse_attn_fwd_workspace_size(B, Lq, k)
+    if workspace is None:
+        if ws_bytes:
+            workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=Q.device)
+    else:
+        if not workspace.is_contiguous():
+            raise ValueError("workspace must be contiguous")
+        _on_device(workspace)
+        ws_bytes = workspace.numel() * workspace.element_size()
+    st = L.dsa_sparse_attn_fwd_ws(_ptr(Q), _ptr(K), _ptr(V), _ptr(idx), _ptr(O), _ptr(lse), B, Lq, Lk, Hq, d, k,
+                                  float(scale), _ptr(workspace), ws_bytes, _stream(stream))
+    _check(st, "dsa_sparse_attn_fwd_ws")
     return (O, lse) if return_lse else O
 
 

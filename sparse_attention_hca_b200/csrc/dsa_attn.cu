@@ -43,6 +43,10 @@
 //     role waits on the index tensor in HBM.
 //   * Barrier phases continue across tokens: s_full/p_ready/pv_done are indexed by a global
 //     tile counter, q_full/q_empty/o_full/o_empty by a counter of tokens with work.
+//   * Few tokens (at most half as many as SMs: decode batches) split: the CTAs walk units
+//     (token, part), part p of S taking ranks [p J / S, (p+1) J / S) of the token's J tiles,
+//     write unnormalised fp32 O rows and per-head (max, sum) to a workspace, and
+//     dsa_combine_kernel merges a token's parts (the online-softmax merge) into O and lse.
 #include <cuda_bf16.h>
 
 #include <mutex>
@@ -81,6 +85,12 @@ struct Params {
   int* err;
   int n_tok, Lq, Lk, k;
   float scale_log2;
+  // Split mode (few tokens, split > 1): unit u = token u / split, part u % split of its key
+  // tiles; the unit's unnormalised O (fp32) and per-head (max, sum) go to ws_O / ws_ml and a
+  // combine pass writes O and lse.  split == 1: units are tokens and O is written directly.
+  int split, n_units;
+  float* ws_O;   // [n_units][64][256]
+  float* ws_ml;  // [n_units][2][64]: reference max (log2 units), then sum of p
 };
 
 struct __align__(8) Barriers {
@@ -141,6 +151,19 @@ __device__ __forceinline__ uint32_t tile_mask_of_row(const int32_t* row, int k, 
   return __reduce_or_sync(0xffffffffu, bits);
 }
 
+// The tiles of `mask` that part `part` of `split` takes: ranks [part J / split, (part+1) J / split)
+// of its J set bits, in ascending order.  Every role derives the same subset.
+__device__ __forceinline__ uint32_t part_of_mask(uint32_t mask, int part, int split) {
+  if (split == 1) return mask;
+  const int J = __popc(mask);
+  const int lo = part * J / split, hi = (part + 1) * J / split;
+  uint32_t out = 0;
+  int r = 0;
+  for (uint32_t m = mask; m; m &= m - 1, ++r)
+    if (r >= lo && r < hi) out |= m & (0u - m);
+  return out;
+}
+
 __device__ __forceinline__ void cp_async4(uint32_t dst, const void* src) {
   asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
 }
@@ -187,12 +210,13 @@ __device__ __forceinline__ void tmem_st_half16(uint32_t taddr, const uint32_t (&
 __device__ __forceinline__ void softmax_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
 // Softmax threads: once the producers and the MMA warp released buffer `buf` (used by local
-// token i), fetch the index row of token `next` into it with cp.async.
+// unit i), fetch the index row of unit `next`'s token into it with cp.async.
 __device__ __forceinline__ void refill_idx_row(const Params& p, Barriers& bar, uint32_t sIdx_a, int buf, int i,
                                                int next, int tid, volatile int& abort_flag, bool& ok) {
-  if (next >= p.n_tok) return;
+  if (next >= p.n_units) return;
   ok = mbar_wait(&bar.idx_empty[buf], (i >> 1) & 1, &abort_flag, p.err) && ok;
-  for (int e = tid; e < p.k; e += 128) cp_async4(sIdx_a + (buf * kMaxK + e) * 4, p.idx + (size_t)next * p.k + e);
+  const int32_t* src = p.idx + (size_t)(next / p.split) * p.k;
+  for (int e = tid; e < p.k; e += 128) cp_async4(sIdx_a + (buf * kMaxK + e) * 4, src + e);
   cp_async_arrive_noinc(&bar.idx_full[buf]);
 }
 
@@ -249,13 +273,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     int it = 0;  // tokens with work so far
     bool ok = true;
     const int chunk = lane >> 3, piece = lane & 7;
-    int i = 0;   // tokens of this CTA so far (index-row buffer i & 1)
-    for (int tok = blockIdx.x; tok < p.n_tok && ok; tok += gridDim.x, ++i) {
+    int i = 0;  // units of this CTA so far (index-row buffer i & 1)
+    for (int unit = blockIdx.x; unit < p.n_units && ok; unit += gridDim.x, ++i) {
+      const int tok = unit / p.split;
       const int buf = i & 1;
       ok = __all_sync(0xffffffffu, mbar_wait(&bar.idx_full[buf], (i >> 1) & 1, &abort_flag, p.err));
       if (!ok) break;
       const int32_t* row = sIdx + buf * kMaxK;
-      const uint32_t mask = tile_mask_of_row<false>(row, k, Lk, lane);
+      const uint32_t mask = part_of_mask(tile_mask_of_row<false>(row, k, Lk, lane), unit % p.split, p.split);
       if (!mask) {
         if (lane == 0) mbar_arrive(&bar.idx_empty[buf]);
         continue;
@@ -324,11 +349,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t idesc_s = idesc_bf16_f32(kH, kKeyTile, false, false);  // S: M = 64 heads, N = 128 keys
     const uint32_t idesc_o = idesc_bf16_f32(kH, kD, false, true);         // O: N = 256 d_v, V MN-major
     int i = 0;
-    for (int tok = blockIdx.x; tok < p.n_tok && ok; tok += gridDim.x, ++i) {
+    for (int unit = blockIdx.x; unit < p.n_units && ok; unit += gridDim.x, ++i) {
       const int buf = i & 1;
       ok = __all_sync(0xffffffffu, mbar_wait(&bar.idx_full[buf], (i >> 1) & 1, &abort_flag, p.err));
       if (!ok) break;
-      const uint32_t mask = tile_mask_of_row<false>(sIdx + buf * kMaxK, k, Lk, lane);
+      const uint32_t mask =
+          part_of_mask(tile_mask_of_row<false>(sIdx + buf * kMaxK, k, Lk, lane), unit % p.split, p.split);
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar.idx_empty[buf]);  // only the mask was needed
       if (!mask) continue;
@@ -411,27 +437,36 @@ __global__ void __launch_bounds__(kThreads, 1)
     // No early exit in this loop: the four softmax warps meet at a named barrier, so after an
     // abort every thread keeps walking the same barrier sequence (waits then fail fast).
     const uint32_t sIdx_a = smem_u32(sIdx);
-    // index rows of this CTA's first two tokens
+    // index rows of this CTA's first two units
     for (int i0 = 0; i0 < 2; ++i0) {
-      const int t0 = blockIdx.x + i0 * gridDim.x;
-      if (t0 < p.n_tok) {
-        for (int e = tid; e < k; e += 128) cp_async4(sIdx_a + (i0 * kMaxK + e) * 4, p.idx + (size_t)t0 * k + e);
+      const int u0 = blockIdx.x + i0 * gridDim.x;
+      if (u0 < p.n_units) {
+        const int32_t* src = p.idx + (size_t)(u0 / p.split) * k;
+        for (int e = tid; e < k; e += 128) cp_async4(sIdx_a + (i0 * kMaxK + e) * 4, src + e);
         cp_async_arrive_noinc(&bar.idx_full[i0]);
       }
     }
     int i = 0;
-    for (int tok = blockIdx.x; tok < p.n_tok; tok += gridDim.x, ++i) {
+    for (int unit = blockIdx.x; unit < p.n_units; unit += gridDim.x, ++i) {
+      const int tok = unit / p.split;
       const int buf = i & 1;
       ok = mbar_wait(&bar.idx_full[buf], (i >> 1) & 1, &abort_flag, p.err) && ok;
       const int32_t* row = sIdx + buf * kMaxK;
       uint32_t all_valid = 0;
-      const uint32_t mask = tile_mask_of_row<true>(row, k, Lk, lane, &all_valid);
+      const uint32_t mask = part_of_mask(tile_mask_of_row<true>(row, k, Lk, lane, &all_valid), unit % p.split, p.split);
       uint16_t* obase = p.O + (size_t)tok * kH * kD;
-      if (!mask) {  // no valid entry: O = 0, lse = -inf
-        for (int e = tid; e < kH * kD / 8; e += 128) reinterpret_cast<uint4*>(obase)[e] = make_uint4(0, 0, 0, 0);
-        if (p.lse && tid < kH) p.lse[(size_t)tok * kH + tid] = -INFINITY;
+      if (!mask) {
+        if (p.split > 1) {  // no tile in this part: an empty record for the combine pass
+          if (tid < kH) {
+            p.ws_ml[(size_t)unit * 2 * kH + tid] = -INFINITY;
+            p.ws_ml[(size_t)unit * 2 * kH + kH + tid] = 0.0f;
+          }
+        } else {  // no valid entry: O = 0, lse = -inf
+          for (int e = tid; e < kH * kD / 8; e += 128) reinterpret_cast<uint4*>(obase)[e] = make_uint4(0, 0, 0, 0);
+          if (p.lse && tid < kH) p.lse[(size_t)tok * kH + tid] = -INFINITY;
+        }
         softmax_bar();  // every softmax thread has read the row before it is refilled
-        refill_idx_row(p, bar, sIdx_a, buf, i, tok + 2 * gridDim.x, tid, abort_flag, ok);
+        refill_idx_row(p, bar, sIdx_a, buf, i, unit + 2 * gridDim.x, tid, abort_flag, ok);
         continue;
       }
       const int J = __popc(mask);
@@ -551,10 +586,26 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ---- epilogue of this token: head h, d_v 128kh..128kh+127
       const float l = l_run + __shfl_xor_sync(0xffffffffu, l_run, 16);
       const float inv = 1.0f / l;
-      if (p.lse && kh == 0) p.lse[(size_t)tok * kH + h] = (m_run + __log2f(l)) * 0.69314718055994531f;
+      if (p.split == 1 && p.lse && kh == 0) p.lse[(size_t)tok * kH + h] = (m_run + __log2f(l)) * 0.69314718055994531f;
       ok = mbar_wait(&bar.o_full[hf], (it >> 1) & 1, &abort_flag, p.err) && ok;
       tc_fence_after();
-      {
+      if (p.split > 1) {  // unnormalised fp32 O rows and (max, sum) of this part
+        if (kh == 0) {
+          p.ws_ml[(size_t)unit * 2 * kH + h] = m_run;
+          p.ws_ml[(size_t)unit * 2 * kH + kH + h] = l;
+        }
+        float4* orow = reinterpret_cast<float4*>(p.ws_O + ((size_t)unit * kH + h) * kD + kh * 128);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t o[32];
+          tmem_ld_half32<128>(t_lanes + c * 32, o);
+          tmem_wait_ld_regs(o);
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            orow[c * 8 + q] = make_float4(__uint_as_float(o[4 * q]), __uint_as_float(o[4 * q + 1]),
+                                          __uint_as_float(o[4 * q + 2]), __uint_as_float(o[4 * q + 3]));
+        }
+      } else {
         uint4* orow = reinterpret_cast<uint4*>(obase + (size_t)h * kD + kh * 128);
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
@@ -575,7 +626,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(&bar.o_empty[hf]);
       softmax_bar();  // every softmax thread has read the row before it is refilled
-      refill_idx_row(p, bar, sIdx_a, buf, i, tok + 2 * gridDim.x, tid, abort_flag, ok);
+      refill_idx_row(p, bar, sIdx_a, buf, i, unit + 2 * gridDim.x, tid, abort_flag, ok);
       g += J;
       ++it;
     }
@@ -600,21 +651,85 @@ int num_sms_current_device() {
   return cache[dev];
 }
 
-}  // namespace
-}  // namespace hcadsa
+// Split mode: O of a token = sum over its parts of 2^(m_p - M) O_p / sum of 2^(m_p - M) l_p,
+// M = max m_p over the parts with l_p > 0 (the same online-softmax merge the kernel does per
+// tile); lse = (M + log2 of the denominator) ln 2.  A token with no valid entry in any part
+// gets O = 0 and lse = -inf.  One CTA per token; thread t: head t / 4, d_v 64 (t % 4) .. +63.
+constexpr int kMaxSplit = 8;
 
-extern "C" hcadsa_status dsa_sparse_attn_fwd(const hcadsa_bf16* Q, const hcadsa_bf16* K, const hcadsa_bf16* V,
-                                             const int32_t* idx, hcadsa_bf16* O, float* lse, int B, int Lq, int Lk,
-                                             int Hq, int d, int k, float scale, hcadsa_stream stream) {
-  using namespace hcadsa;
+__global__ void __launch_bounds__(256) dsa_combine_kernel(const float* __restrict__ ws_O,
+                                                          const float* __restrict__ ws_ml, uint16_t* __restrict__ O,
+                                                          float* __restrict__ lse, int split) {
+  const int tok = blockIdx.x;
+  const int h = threadIdx.x >> 2, q4 = threadIdx.x & 3;
+  const size_t u0 = (size_t)tok * split;
+  float M = -INFINITY;
+  for (int s = 0; s < split; ++s) {
+    const float* ml = ws_ml + (u0 + s) * 2 * kH;
+    if (ml[kH + h] > 0.0f) M = fmaxf(M, ml[h]);
+  }
+  float acc[64];
+#pragma unroll
+  for (int x = 0; x < 64; ++x) acc[x] = 0.0f;
+  float den = 0.0f;
+  for (int s = 0; s < split; ++s) {
+    const float* ml = ws_ml + (u0 + s) * 2 * kH;
+    const float l = ml[kH + h];
+    if (!(l > 0.0f)) continue;  // a part without tiles left its O rows unwritten
+    const float w = exp2f(ml[h] - M);
+    den += w * l;
+    const float4* src = reinterpret_cast<const float4*>(ws_O + ((u0 + s) * kH + h) * kD + q4 * 64);
+#pragma unroll
+    for (int x = 0; x < 16; ++x) {
+      const float4 v = src[x];
+      acc[4 * x] = fmaf(w, v.x, acc[4 * x]);
+      acc[4 * x + 1] = fmaf(w, v.y, acc[4 * x + 1]);
+      acc[4 * x + 2] = fmaf(w, v.z, acc[4 * x + 2]);
+      acc[4 * x + 3] = fmaf(w, v.w, acc[4 * x + 3]);
+    }
+  }
+  const float inv = den > 0.0f ? 1.0f / den : 0.0f;
+  uint4* dst = reinterpret_cast<uint4*>(O + ((size_t)tok * kH + h) * kD + q4 * 64);
+#pragma unroll
+  for (int x = 0; x < 8; ++x) {
+    uint4 w;
+    w.x = pack_bf16x2(acc[8 * x] * inv, acc[8 * x + 1] * inv);
+    w.y = pack_bf16x2(acc[8 * x + 2] * inv, acc[8 * x + 3] * inv);
+    w.z = pack_bf16x2(acc[8 * x + 4] * inv, acc[8 * x + 5] * inv);
+    w.w = pack_bf16x2(acc[8 * x + 6] * inv, acc[8 * x + 7] * inv);
+    dst[x] = w;
+  }
+  if (lse && q4 == 0) lse[(size_t)tok * kH + h] = den > 0.0f ? (M + __log2f(den)) * 0.69314718055994531f : -INFINITY;
+}
+
+// Parts per token: only calls with at most half as many tokens as SMs split (decode batches),
+// into as many parts as fill the SMs, at most kMaxSplit and at most one per key tile.
+int split_of(int n_tok, int k, int sms) {
+  if (n_tok <= 0 || sms <= 0 || 2 * n_tok > sms) return 1;
+  const int n_tiles = (k + kKeyTile - 1) / kKeyTile;
+  int s = sms / n_tok;
+  if (s > kMaxSplit) s = kMaxSplit;
+  if (s > n_tiles) s = n_tiles;
+  return s < 1 ? 1 : s;
+}
+
+constexpr size_t kUnitWsBytes = (size_t)kH * kD * 4 + 2 * kH * 4;  // O rows + (max, sum) per unit
+
+hcadsa_status check_args(const hcadsa_bf16* Q, const hcadsa_bf16* K, const hcadsa_bf16* V, const int32_t* idx,
+                         hcadsa_bf16* O, float* lse, int B, int Lq, int Lk, int Hq, int d, int k, float scale) {
   if (!Q || !K || !V || !idx || !O) return HCADSA_ERR_NULL;
   if (B < 0 || Lq < 0 || Lk < 0 || k <= 0 || !(scale > 0.0f)) return HCADSA_ERR_SHAPE;
   if (d != kD || Hq != kH || k > kMaxK) return HCADSA_ERR_UNSUPPORTED;
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(idx) ||
       (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
     return HCADSA_ERR_ALIGN;
-  if (B == 0 || Lq == 0) return HCADSA_OK;
   if ((long long)B * Lq > 2147483647LL || (long long)B * Lk > 2147483647LL) return HCADSA_ERR_UNSUPPORTED;
+  return HCADSA_OK;
+}
+
+hcadsa_status launch(const hcadsa_bf16* Q, const hcadsa_bf16* K, const hcadsa_bf16* V, const int32_t* idx,
+                     hcadsa_bf16* O, float* lse, int B, int Lq, int Lk, int k, float scale, int split, float* ws,
+                     int sms, hcadsa_stream stream) {
   CUtensorMap mq;
   {
     const uint64_t dims[3] = {(uint64_t)kD, (uint64_t)kH, (uint64_t)B * Lq};
@@ -634,11 +749,60 @@ extern "C" hcadsa_status dsa_sparse_attn_fwd(const hcadsa_bf16* Q, const hcadsa_
   p.Lk = Lk;
   p.k = k;
   p.scale_log2 = scale * 1.4426950408889634f;
+  p.split = split;
+  p.n_units = p.n_tok * split;
+  p.ws_O = split > 1 ? ws : nullptr;
+  p.ws_ml = split > 1 ? ws + (size_t)p.n_units * kH * kD : nullptr;
   if (cudaFuncSetAttribute(dsa_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) != cudaSuccess)
     return HCADSA_ERR_CUDA;
+  const int grid = p.n_units < sms ? p.n_units : sms;
+  dsa_attn_kernel<<<grid, kThreads, kSmemBytes, as_stream(stream)>>>(mq, p);
+  if (split > 1) {
+    const hcadsa_status st = launch_status();
+    if (st != HCADSA_OK) return st;
+    dsa_combine_kernel<<<p.n_tok, 256, 0, as_stream(stream)>>>(p.ws_O, p.ws_ml, reinterpret_cast<uint16_t*>(O), lse,
+                                                               split);
+  }
+  return launch_status();
+}
+
+}  // namespace
+}  // namespace hcadsa
+
+extern "C" hcadsa_status dsa_sparse_attn_fwd(const hcadsa_bf16* Q, const hcadsa_bf16* K, const hcadsa_bf16* V,
+                                             const int32_t* idx, hcadsa_bf16* O, float* lse, int B, int Lq, int Lk,
+                                             int Hq, int d, int k, float scale, hcadsa_stream stream) {
+  using namespace hcadsa;
+  const hcadsa_status st = check_args(Q, K, V, idx, O, lse, B, Lq, Lk, Hq, d, k, scale);
+  if (st != HCADSA_OK) return st;
+  if (B == 0 || Lq == 0) return HCADSA_OK;
   const int sms = num_sms_current_device();
   if (sms <= 0) return HCADSA_ERR_CUDA;
-  const int grid = p.n_tok < sms ? p.n_tok : sms;
-  dsa_attn_kernel<<<grid, kThreads, kSmemBytes, as_stream(stream)>>>(mq, p);
-  return launch_status();
+  return launch(Q, K, V, idx, O, lse, B, Lq, Lk, k, scale, 1, nullptr, sms, stream);
+}
+
+extern "C" size_t dsa_sparse_attn_fwd_workspace_size(int B, int Lq, int k) {
+  using namespace hcadsa;
+  if (B <= 0 || Lq <= 0 || k <= 0 || k > kMaxK || (long long)B * Lq > 2147483647LL) return 0;
+  const int sms = num_sms_current_device();
+  const int split = split_of(B * Lq, k, sms);
+  return split > 1 ? (size_t)B * Lq * split * kUnitWsBytes : 0;
+}
+
+extern "C" hcadsa_status dsa_sparse_attn_fwd_ws(const hcadsa_bf16* Q, const hcadsa_bf16* K, const hcadsa_bf16* V,
+                                                const int32_t* idx, hcadsa_bf16* O, float* lse, int B, int Lq,
+                                                int Lk, int Hq, int d, int k, float scale, void* workspace,
+                                                size_t workspace_bytes, hcadsa_stream stream) {
+  using namespace hcadsa;
+  const hcadsa_status st = check_args(Q, K, V, idx, O, lse, B, Lq, Lk, Hq, d, k, scale);
+  if (st != HCADSA_OK) return st;
+  if (B == 0 || Lq == 0) return HCADSA_OK;
+  const int sms = num_sms_current_device();
+  if (sms <= 0) return HCADSA_ERR_CUDA;
+  const int split = split_of(B * Lq, k, sms);
+  if (split > 1) {
+    if (!workspace || workspace_bytes < (size_t)B * Lq * split * kUnitWsBytes) return HCADSA_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return HCADSA_ERR_ALIGN;
+  }
+  return launch(Q, K, V, idx, O, lse, B, Lq, Lk, k, scale, split, static_cast<float*>(workspace), sms, stream);
 }

@@ -98,6 +98,13 @@ def test_dsa_argument_errors(lib):
     assert a(FAKE, FAKE, FAKE, FAKE, FAKE, None, 1, 8, 8, 64, 256, 4097, 0.06, None) == -4  # k > 4096
     assert a(FAKE, FAKE, FAKE, FAKE, FAKE, None, 1, 8, 8, 64, 256, 16, 0.0, None) == -2    # scale <= 0
     assert a(FAKE, FAKE, FAKE, FAKE, FAKE, None, 1, 8, 8, 64, 256, 16, float("nan"), None) == -2
+    w = lib.dsa_sparse_attn_fwd_ws  # same argument checks before any device query or launch
+    assert w(FAKE, FAKE, FAKE, None, FAKE, None, 1, 8, 8, 64, 256, 16, 0.06, None, 0, None) == -1
+    assert w(FAKE, FAKE, FAKE, FAKE, FAKE, None, 1, 8, 8, 64, 128, 16, 0.06, None, 0, None) == -4
+    assert w(FAKE, FAKE, FAKE, FAKE, FAKE, None, 1, 8, 8, 64, 256, 16, -1.0, None, 0, None) == -2
+    assert w(FAKE, MISALIGNED, FAKE, FAKE, FAKE, None, 1, 8, 8, 64, 256, 16, 0.06, None, 0, None) == -3
+    assert lib.dsa_sparse_attn_fwd_workspace_size(1, 8, 0) == 0        # invalid k
+    assert lib.dsa_sparse_attn_fwd_workspace_size(1, 8, 4097) == 0     # unsupported k
 
 
 def test_workspace_size_queries(lib):

@@ -531,6 +531,32 @@ def test_dsa_padding_and_order(hd):
     print(check_attn(O, ref, "dsa padded/shuffled"))
 
 
+def test_dsa_forced_rescales(hd):
+    """Keys whose scale grows with their position and index rows in ascending order: later
+    128-entry tiles raise a head's running max by far more than the lazy-rescale threshold, so
+    that head's O row is rescaled in TMEM (while other heads of the same warp keep theirs); a
+    few padded entries in the middle of some rows mix partial tiles with fully valid ones."""
+    cfg = _dsa_cfg("ramp", 1500, k=1024, sigma=1.0)
+    inp = synth.dsa_inputs(cfg)
+    ramp = 1.0 + 6.0 * torch.arange(cfg.L, dtype=torch.float32) / cfg.L
+    K = (inp["K"].float() * ramp.view(1, -1, 1)).to(torch.bfloat16)
+    rng = np.random.default_rng(11)
+    idx = np.full((cfg.L, cfg.k), -1, np.int32)
+    for t in range(cfg.L):
+        n = min(cfg.k, t + 1)
+        idx[t, :n] = np.sort(rng.choice(t + 1, size=n, replace=False))
+        if t % 3 == 0 and n > 300:
+            idx[t, 200:210] = -1
+    O, lse = hd.dsa_sparse_attn_fwd(inp["Q"].cuda(), K.cuda(), inp["V"].cuda(),
+                                    torch.as_tensor(idx).reshape(1, cfg.L, cfg.k).cuda(), return_lse=True)
+    no_device_error(hd)
+    rows = _sample_rows(cfg.L, extra=(300, 1023, 1024, 1200, 1497))
+    ref, ref_lse = oracle.dsa_attn(bits(inp["Q"]), bits(K), bits(inp["V"]), idx[rows], rows=rows, with_lse=True)
+    r = torch.as_tensor(rows, device="cuda")
+    print(check_attn(O.reshape(cfg.L, cfg.Hq, cfg.d)[r], ref, "dsa forced rescales"))
+    np.testing.assert_allclose(lse.reshape(cfg.L, cfg.Hq)[r].cpu().numpy(), ref_lse, atol=2e-2, rtol=0)
+
+
 def test_dsa_all_padding_rows_and_lse(hd):
     """Rows whose index list holds no valid entry (all -1) give O = 0 and lse = -inf, the
     oracle's empty-set case; their neighbours (partly padded, shuffled) still match the oracle
@@ -558,6 +584,42 @@ def test_dsa_all_padding_rows_and_lse(hd):
     keep = np.array([t for t in range(cfg.L) if t not in empty])
     print(check_attn(O[torch.as_tensor(keep, device="cuda")], ref[keep], "dsa all-padding neighbours"))
     np.testing.assert_allclose(lse[keep], ref_lse[keep], atol=2e-3, rtol=0)
+
+
+def test_dsa_split_matches_oracle_and_unsplit(hd):
+    """Few query rows (a decode-sized call): each row's key tiles are divided among several CTAs
+    whose partial outputs the combine pass merges.  Rows with every entry valid, with entries in
+    only two tiles (most parts empty), with none (every part empty) and with scattered padding;
+    compared with the oracle and with the one-CTA-per-row path."""
+    Lk, n_q, k = 5000, 12, 2048
+    cfg = _dsa_cfg("split", Lk, k=k, sigma=1.0)
+    inp = synth.dsa_inputs(cfg)
+    assert hd.lib().dsa_sparse_attn_fwd_workspace_size(1, n_q, k) > 0  # this call splits
+    rng = np.random.default_rng(23)
+    idx = np.full((n_q, k), -1, np.int32)
+    for r in range(n_q):
+        if r == 3:
+            continue  # no valid entry
+        if r == 5:
+            idx[r, 700:790] = rng.choice(Lk, 90, replace=False)  # tiles 5 and 6 only
+            continue
+        idx[r] = rng.choice(Lk, k, replace=False)
+        if r == 8:
+            idx[r, rng.random(k) < 0.3] = -1
+    qpos = torch.as_tensor(rng.choice(Lk, n_q, replace=False))
+    q = inp["Q"].reshape(Lk, cfg.Hq, cfg.d)[qpos].reshape(1, n_q, cfg.Hq, cfg.d)
+    args = (q.cuda(), inp["K"].cuda(), inp["V"].cuda(), torch.as_tensor(idx).reshape(1, n_q, k).cuda())
+    O_s, lse_s = hd.dsa_sparse_attn_fwd(*args, return_lse=True)
+    O_u, lse_u = hd.dsa_sparse_attn_fwd(*args, return_lse=True, split=False)
+    no_device_error(hd)
+    ref, ref_lse = oracle.dsa_attn(bits(q), bits(inp["K"]), bits(inp["V"]), idx, with_lse=True)
+    for O, lse, name in ((O_s, lse_s, "split"), (O_u, lse_u, "one CTA per row")):
+        O = O.reshape(n_q, cfg.Hq, cfg.d)
+        lse = lse.reshape(n_q, cfg.Hq).cpu().numpy()
+        assert torch.count_nonzero(O[3]).item() == 0 and np.all(np.isneginf(lse[3]))
+        keep = [r for r in range(n_q) if r != 3]
+        print(check_attn(O[keep], ref[keep], f"dsa {name}, {n_q} rows"))
+        np.testing.assert_allclose(lse[keep], ref_lse[keep], atol=2e-3, rtol=0)
 
 
 def test_dsa_index_out_of_range_is_reported(hd):
