@@ -464,7 +464,7 @@ def test_topk_ragged_batches_offset_odd_k(hd):
 
 # ------------------------------------------------------------------ DSA sparse attention
 
-def _dsa_attn_case(hd, cfg, rows):
+def _dsa_attn_case(hd, cfg, rows, split=True):
     """GPU attention fed the ORACLE's index rows for the sampled queries; returns the GPU and
     oracle outputs and log-sum-exps of those rows."""
     inp = synth.dsa_inputs(cfg)
@@ -478,7 +478,8 @@ def _dsa_attn_case(hd, cfg, rows):
             continue
         q_b = Qs[torch.as_tensor(np.nonzero(sel)[0])].reshape(1, -1, cfg.Hq, cfg.d)
         O, lse = hd.dsa_sparse_attn_fwd(q_b.cuda(), inp["K"][b:b + 1].cuda(), inp["V"][b:b + 1].cuda(),
-                                        torch.as_tensor(idx_o[sel]).reshape(1, -1, cfg.k).cuda(), return_lse=True)
+                                        torch.as_tensor(idx_o[sel]).reshape(1, -1, cfg.k).cuda(), return_lse=True,
+                                        split=split)
         outs.append(O.reshape(-1, cfg.Hq, cfg.d))
         lses.append(lse.reshape(-1, cfg.Hq))
     no_device_error(hd)
@@ -486,7 +487,8 @@ def _dsa_attn_case(hd, cfg, rows):
     return torch.cat(outs), torch.cat(lses), ref, ref_lse
 
 
-@pytest.mark.parametrize("L,k,sigma", [(3000, 2048, None), (2000, 256, 1.0), (300, 2048, 1.0), (500, 100, 2.0)])
+@pytest.mark.parametrize("L,k,sigma", [(3000, 2048, None), (2000, 256, 1.0), (300, 2048, 1.0), (500, 100, 2.0),
+                                         (5000, 4096, 1.0)])
 def test_dsa_attn_against_oracle(hd, L, k, sigma):
     cfg = _dsa_cfg("dsa", L, k=k, sigma=sigma)
     rows = _sample_rows(L, extra=(k - 1, k, k + 1, L - 3))
@@ -494,6 +496,16 @@ def test_dsa_attn_against_oracle(hd, L, k, sigma):
     print(check_attn(O, ref, f"dsa L={L} k={k} sigma={sigma}", value_scale=sigma or 1.0))
     # natural-log log-sum-exp of the selected scores, per head (the backward consumes it)
     np.testing.assert_allclose(lse.cpu().numpy(), ref_lse, atol=2e-3 * max(1.0, (sigma or 1.0) ** 2), rtol=0)
+
+
+def test_dsa_attn_max_k_one_cta_per_row(hd):
+    """k = 4096, the largest index row (32 key tiles, every bit of the tile mask), with one CTA
+    per query row (the split path of the same rows is in test_dsa_attn_against_oracle)."""
+    cfg = _dsa_cfg("dsa", 5000, k=4096, sigma=1.0)
+    rows = _sample_rows(cfg.L, extra=(4095, 4096, 4097, 4998))
+    O, lse, ref, ref_lse = _dsa_attn_case(hd, cfg, rows, split=False)
+    print(check_attn(O, ref, "dsa k=4096 one CTA per row"))
+    np.testing.assert_allclose(lse.cpu().numpy(), ref_lse, atol=2e-3, rtol=0)
 
 
 def test_dsa_pipeline_32k_sampled(hd):
@@ -620,6 +632,27 @@ def test_dsa_split_matches_oracle_and_unsplit(hd):
         keep = [r for r in range(n_q) if r != 3]
         print(check_attn(O[keep], ref[keep], f"dsa {name}, {n_q} rows"))
         np.testing.assert_allclose(lse[keep], ref_lse[keep], atol=2e-3, rtol=0)
+
+
+def test_dsa_split_two_sequences(hd):
+    """The split path with a batch: 2 sequences of 3000 keys, 5 query rows each; every unit reads
+    the K/V rows of its own sequence."""
+    cfg = synth.DsaConfig("split2", B=2, L=3000, Hq=64, k=1024, sigma=1.0)
+    inp = synth.dsa_inputs(cfg)
+    n_q = 5
+    assert hd.lib().dsa_sparse_attn_fwd_workspace_size(cfg.B, n_q, cfg.k) > 0
+    rng = np.random.default_rng(29)
+    idx = np.stack([np.stack([rng.choice(cfg.L, cfg.k, replace=False) for _ in range(n_q)]) for _ in range(cfg.B)])
+    idx = idx.astype(np.int32)
+    idx[1, 2, 500:] = -1  # a short row in the second sequence
+    q = inp["Q"][:, :n_q].contiguous()
+    O, lse = hd.dsa_sparse_attn_fwd(q.cuda(), inp["K"].cuda(), inp["V"].cuda(), torch.as_tensor(idx).cuda(),
+                                    return_lse=True)
+    no_device_error(hd)
+    ref, ref_lse = oracle.dsa_attn(bits(q), bits(inp["K"]), bits(inp["V"]), idx.reshape(cfg.B * n_q, cfg.k),
+                                   with_lse=True)
+    print(check_attn(O.reshape(cfg.B * n_q, cfg.Hq, cfg.d), ref, "dsa split, two sequences"))
+    np.testing.assert_allclose(lse.reshape(cfg.B * n_q, cfg.Hq).cpu().numpy(), ref_lse, atol=2e-3, rtol=0)
 
 
 def test_dsa_index_out_of_range_is_reported(hd):
