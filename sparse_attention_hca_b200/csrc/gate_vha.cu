@@ -14,16 +14,24 @@
 // no data from other threads: 256 columns = all H heads x cw = 256 / H channels of one channel
 // block, so the thread that owns token t (TMEM lane t) holds every head of those channels and
 // mixes them in registers.
-//   * A = cq tile (128 tokens x 64 of K per stage, TMA, SW128); B = the 256 rows (h, c) of Wg
-//     for the channel block (a 3D TMA box {64, cw, H} over Wg viewed as [H][dv][rq], SW128).
-//   * Warp 0: TMA producer (4 stages of 48 KB); warp 1: TMEM allocation + the MMA thread
-//     (4 MMAs of M = 128, N = 256, K = 16 per stage, fp32 accumulator of 256 TMEM columns,
-//     double-buffered across tiles); warps 2-9: epilogue, two threads per token (each half of the
-//     channel block, every head; its O values loaded at once and kept in registers): the rank-r
-//     projections sum_h V[h,m] O[t,h,c] of its channels, then per head the mix, the sigmoid of
-//     the logit from TMEM and the bf16 store of Y.
-//   * Persistent CTAs walk the tiles (token tile, channel block); consecutive CTAs share the
-//     token tile, so the cq tile and Wg stay in L2.
+//   * CTA pairs (clusters of 2, tcgen05 cta_group::2): a pair computes 256 tokens x the 256 gate
+//     columns of a channel block with M = 256 MMAs.  Each CTA loads its own 128-token cq tile
+//     (A) and HALF of the Wg rows (B: heads [r H/2, (r+1) H/2) of the block, a 3D TMA box
+//     {64, cw, H/2} over Wg viewed as [H][dv][rq], SW128), so a stage is 32 KB instead of 48 KB
+//     and the operand traffic from L2 per output drops by a third -- with single-CTA 128 x 256
+//     tiles every tile re-read 768 KB of operands, and that stream from L2 was the bound.
+//     Both CTAs' TMA loads complete on the leader's (rank 0) barrier; the leader's thread
+//     issues every MMA and its commits reach the barriers of both CTAs (.multicast::cluster).
+//     Each CTA's TMEM holds its 128 tokens x 256 columns, so the epilogue is per CTA.
+//   * Warp 0: TMA producer (6 stages of 32 KB); warp 1: TMEM allocation (both CTAs) + the MMA
+//     thread (leader only: 4 MMAs of M = 256, N = 256, K = 16 per stage, fp32 accumulator of
+//     256 TMEM columns, double-buffered across tiles); warps 2-9: epilogue, two threads per
+//     token (each half of the channel block, every head; its O values loaded at once and kept in
+//     registers): the rank-r projections sum_h V[h,m] O[t,h,c] of its channels, then per head
+//     the mix, the sigmoid of the logit from TMEM and the bf16 store of Y.  An epilogue warp
+//     frees a TMEM buffer with one arrival on the leader's barrier.
+//   * Persistent pairs walk the pair tiles (token-tile pair, channel block); consecutive pairs
+//     share the token tiles, so the cq tiles and Wg stay in L2.
 #include <cuda_bf16.h>
 
 #include <mutex>
@@ -37,11 +45,12 @@ namespace {
 constexpr int kM = 128;      // tokens per tile
 constexpr int kN = 256;      // gate columns per tile (H heads x cw channels)
 constexpr int kKStep = 64;   // K per stage (one 128-byte swizzle row of bf16)
-constexpr int kStages = 4;
-constexpr int kABytes = kM * kKStep * 2;  // 16 KB
-constexpr int kBBytes = kN * kKStep * 2;  // 32 KB
+constexpr int kStages = 6;
+constexpr int kABytes = kM * kKStep * 2;        // 16 KB
+constexpr int kBBytes = (kN / 2) * kKStep * 2;  // 16 KB: this CTA's half of the 256 Wg rows
 constexpr int kStageBytes = kABytes + kBBytes;
 constexpr int kMaxR = 4;     // rank of the head mix
+static_assert(kMaxR == 4, "the mix reads the per-head U / V slots as one float4");
 constexpr int kMaxH = 64;
 constexpr int kSmemBytes = kStages * kStageBytes + 1024;
 constexpr int kEpiWarps = 8;  // two per TMEM lane quarter: each takes half of the tile's channels
@@ -53,7 +62,7 @@ struct Params {
   const float* V;
   uint16_t* Y;
   int* err;
-  int rows, H, dv, rq, r, cw, n_blocks, n_tiles;
+  int rows, H, dv, rq, r, cw, n_blocks, n_tiles;  // n_tiles: pair tiles (token-tile pair, block)
 };
 
 struct __align__(8) Barriers {
@@ -97,6 +106,55 @@ __device__ __forceinline__ void store_packed(uint16_t* p, const uint32_t (&w)[N 
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// The address of the same shared variable in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t cluster_addr(const void* p, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void arrive_cluster(uint32_t addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(addr) : "memory");
+}
+// TMA loads of a CTA pair: the data lands in this CTA's shared memory, the transaction bytes
+// complete on `bar` (a shared::cluster address, here the leader's barrier).
+__device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* map, uint32_t bar, int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];"
+      ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1)
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_3d_pair(void* dst, const CUtensorMap* map, uint32_t bar, int c0, int c1,
+                                                 int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];"
+      ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+// D[tmem] (+)= A * B over the pair (M = 256: each CTA's A rows and half of B's rows).
+__device__ __forceinline__ void mma_ss_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// Arrive once on `bar` in both CTAs of the pair when every earlier MMA of this thread is done.
+__device__ __forceinline__ void mma_commit_pair(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;"
+               ::"r"(smem_u32(bar)), "h"((uint16_t)3)
+               : "memory");
+}
+
 template <int CW>
 // 10 warps put three on two of the four SM sub-partitions (16K registers each): at most 168
 // registers per thread, which __launch_bounds__ makes the compiler respect
@@ -109,12 +167,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ Barriers bar;
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_flag;
-  __shared__ float sU[kMaxH * kMaxR], sV[kMaxH * kMaxR];
+  // U and V with kMaxR slots per head (zero past the rank), so the mix reads one float4 per head
+  __shared__ __align__(16) float sU[kMaxH * kMaxR];
+  __shared__ __align__(16) float sV[kMaxH * kMaxR];
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  for (int i = threadIdx.x; i < H * p.r; i += kThreads) {
-    sU[i] = p.U[i];
-    sV[i] = p.V[i];
+  const uint32_t rank = cluster_rank();          // 0: the leader, which issues the MMAs
+  const int pair = (int)blockIdx.x >> 1, n_pairs = (int)gridDim.x >> 1;
+  for (int i = threadIdx.x; i < H * kMaxR; i += kThreads) {
+    const int hq = i / kMaxR, q = i % kMaxR;
+    sU[i] = q < p.r ? p.U[hq * p.r + q] : 0.0f;
+    sV[i] = q < p.r ? p.V[hq * p.r + q] : 0.0f;
   }
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -123,17 +186,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bar.tfull[s], 1);
-      mbar_init(&bar.tempty[s], 32 * kEpiWarps);
+      mbar_init(&bar.tempty[s], 2 * kEpiWarps);  // the leader's copy: one arrival per epilogue warp of the pair
     }
     abort_flag = 0;
-    fence_mbarrier_init();
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  if (warp == 1) {
-    tmem_alloc(&tmem_base_sh, 512);
-    tmem_relinquish();
+  if (warp == 1) {  // the same warp in both CTAs, the same shared slot
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&tmem_base_sh)),
+                 "r"(512));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::);
   }
   tc_fence_before();
   __syncthreads();
+  cluster_sync();  // barriers and TMEM of both CTAs exist before any cross-CTA operation
   tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
   const int k_steps = p.rq / kKStep;
@@ -145,26 +210,28 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&map_b);
       uint32_t g = 0;
       bool ok = true;
-      for (int t = blockIdx.x; ok && t < p.n_tiles; t += gridDim.x) {
-        const int m = t / p.n_blocks, nb = t % p.n_blocks;
+      for (int t = pair; ok && t < p.n_tiles; t += n_pairs) {
+        const int m = 2 * (t / p.n_blocks) + (int)rank, nb = t % p.n_blocks;  // this CTA's token tile
         for (int ks = 0; ok && ks < k_steps; ++ks, ++g) {
           const uint32_t st = g % kStages;
+          // the slot is free in this CTA once the pair's MMAs that read it are done (multicast)
           ok = mbar_wait(&bar.empty[st], ((g / kStages) & 1) ^ 1, &abort_flag, p.err);
           if (!ok) break;
           uint8_t* sa = smem + st * kStageBytes;
-          mbar_arrive_expect_tx(&bar.full[st], kStageBytes);
-          tma_load_2d(sa, &map_a, &bar.full[st], ks * kKStep, m * kM);
-          tma_load_3d(sa + kABytes, &map_b, &bar.full[st], ks * kKStep, nb * CW, 0);
+          const uint32_t full_leader = cluster_addr(&bar.full[st], 0);
+          if (rank == 0) mbar_arrive_expect_tx(&bar.full[st], 2 * kStageBytes);  // both CTAs' bytes
+          tma_load_2d_pair(sa, &map_a, full_leader, ks * kKStep, m * kM);
+          tma_load_3d_pair(sa + kABytes, &map_b, full_leader, ks * kKStep, nb * CW, (int)rank * (H / 2));
         }
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(kM, kN, false, false);
+    if (lane == 0 && rank == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(2 * kM, kN, false, false);
       uint32_t g = 0, tl = 0;
       bool ok = true;
-      for (int t = blockIdx.x; ok && t < p.n_tiles; t += gridDim.x, ++tl) {
+      for (int t = pair; ok && t < p.n_tiles; t += n_pairs, ++tl) {
         const uint32_t buf = tl & 1;
         ok = mbar_wait(&bar.tempty[buf], ((tl >> 1) & 1) ^ 1, &abort_flag, p.err);
         if (!ok) break;
@@ -178,11 +245,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t da = smem_desc_sw128(sa, 16, 1024), db = smem_desc_sw128(sa + kABytes, 16, 1024);
 #pragma unroll
           for (int kk = 0; kk < kKStep / 16; ++kk)  // start address in 16-byte units: 32 bytes per K = 16
-            mma_ss(tmem + buf * kN, da + (uint64_t)(kk * 2), db + (uint64_t)(kk * 2), idesc, (ks | kk) != 0);
-          mma_commit(&bar.empty[st]);
+            mma_ss_pair(tmem + buf * kN, da + (uint64_t)(kk * 2), db + (uint64_t)(kk * 2), idesc, (ks | kk) != 0);
+          mma_commit_pair(&bar.empty[st]);
         }
         if (!ok) break;
-        mma_commit(&bar.tfull[buf]);
+        mma_commit_pair(&bar.tfull[buf]);
       }
     }
   } else {
@@ -193,11 +260,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int half = (warp - 2) >> 2;
     const int r = quarter * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-    const int R = p.r;
     uint32_t tl = 0;
     bool ok = true;
-    for (int t = blockIdx.x; t < p.n_tiles; t += gridDim.x, ++tl) {
-      const int m = t / p.n_blocks, nb = t % p.n_blocks;
+    for (int t = pair; t < p.n_tiles; t += n_pairs, ++tl) {
+      const int m = 2 * (t / p.n_blocks) + (int)rank, nb = t % p.n_blocks;
       const int token = m * kM + r;
       const bool valid = token < p.rows;
       const uint32_t buf = tl & 1;
@@ -216,17 +282,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int c = 0; c < CH; ++c) proj[q][c] = 0.0f;
       if (valid) {
 #pragma unroll
-        for (int h = 0; h < H; ++h)
+        for (int h = 0; h < H; ++h) {
+          const float4 v4 = *reinterpret_cast<const float4*>(&sV[h * kMaxR]);
+          const float vq[kMaxR] = {v4.x, v4.y, v4.z, v4.w};
 #pragma unroll
-          for (int q = 0; q < kMaxR; ++q)
-            if (q < R) {
-              const float vv = sV[h * R + q];
+          for (int c = 0; c < CH; c += 2) {
+            const float x0 = bf16_lo(ow[h][c / 2]), x1 = bf16_hi(ow[h][c / 2]);
 #pragma unroll
-              for (int c = 0; c < CH; c += 2) {
-                proj[q][c] = fmaf(vv, bf16_lo(ow[h][c / 2]), proj[q][c]);
-                proj[q][c + 1] = fmaf(vv, bf16_hi(ow[h][c / 2]), proj[q][c + 1]);
-              }
+            for (int q = 0; q < kMaxR; ++q) {  // slots past the rank hold 0: they add nothing
+              proj[q][c] = fmaf(vq[q], x0, proj[q][c]);
+              proj[q][c + 1] = fmaf(vq[q], x1, proj[q][c + 1]);
             }
+          }
+        }
       }
       ok = mbar_wait(&bar.tfull[buf], (tl >> 1) & 1, &abort_flag, p.err) && ok;
       tc_fence_after();
@@ -238,23 +306,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_wait_ld_regs(zr);
         if (c0 + 32 == kN) {  // every logit of the tile is in registers: the buffer may be reused
           tc_fence_before();
-          mbar_arrive(&bar.tempty[buf]);
+          __syncwarp();
+          if (lane == 0) arrive_cluster(cluster_addr(&bar.tempty[buf], 0));
         }
         if (!valid) continue;
 #pragma unroll
         for (int hh = 0; hh < 32 / CW; ++hh) {
           const int h = c0 / CW + hh;
+          const float4 u4 = *reinterpret_cast<const float4*>(&sU[h * kMaxR]);
+          const float uq[kMaxR] = {u4.x, u4.y, u4.z, u4.w};
           uint32_t yw[CH / 2];
 #pragma unroll
           for (int c = 0; c < CH; c += 2) {
             float o0 = bf16_lo(ow[h][c / 2]), o1 = bf16_hi(ow[h][c / 2]);
 #pragma unroll
-            for (int q = 0; q < kMaxR; ++q)
-              if (q < R) {
-                const float uu = sU[h * R + q];
-                o0 = fmaf(uu, proj[q][c], o0);
-                o1 = fmaf(uu, proj[q][c + 1], o1);
-              }
+            for (int q = 0; q < kMaxR; ++q) {
+              o0 = fmaf(uq[q], proj[q][c], o0);
+              o1 = fmaf(uq[q], proj[q][c + 1], o1);
+            }
             // this thread's logits: channel c of its half (both indices compile-time constants)
             const float z0 = __uint_as_float(half ? zr[hh * CW + CH + c] : zr[hh * CW + c]);
             const float z1 = __uint_as_float(half ? zr[hh * CW + CH + c + 1] : zr[hh * CW + c + 1]);
@@ -268,7 +337,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) tmem_dealloc(tmem, 512);
+  cluster_sync();  // no MMA of the pair and no cross-CTA arrival is pending any more
+  tc_fence_after();
+  if (warp == 1) asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512));
 }
 
 int sm_count() {
@@ -288,9 +359,21 @@ hcadsa_status launch(const CUtensorMap& ma, const CUtensorMap& mb, const Params&
       cudaSuccess)
     return launch_status();
   const int sms = sm_count();
-  if (sms <= 0) return HCADSA_ERR_CUDA;
-  const int grid = p.n_tiles < sms ? p.n_tiles : sms;
-  gate_vha_kernel<CW><<<grid, kThreads, kSmemBytes, s>>>(ma, mb, p);
+  if (sms < 2) return HCADSA_ERR_CUDA;
+  const int pairs = p.n_tiles < sms / 2 ? p.n_tiles : sms / 2;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * pairs, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, gate_vha_kernel<CW>, ma, mb, p) != cudaSuccess) return launch_status();
   return launch_status();
 }
 
@@ -312,7 +395,7 @@ extern "C" hcadsa_status attn_gate_vha_fwd(const hcadsa_bf16* O, const hcadsa_bf
   if (rows == 0) return HCADSA_OK;
   const int cw = kN / H;
   const long long n_blocks = dv / cw;
-  const long long n_tiles = (rows + kM - 1) / kM * n_blocks;
+  const long long n_tiles = ((rows + kM - 1) / kM + 1) / 2 * n_blocks;  // pair tiles
   if (rows > 2147483647LL || n_tiles > 2147483647LL || (long long)H * dv * rq > (1LL << 40))
     return HCADSA_ERR_UNSUPPORTED;
   CUtensorMap ma, mb;
@@ -325,7 +408,7 @@ extern "C" hcadsa_status attn_gate_vha_fwd(const hcadsa_bf16* O, const hcadsa_bf
   {
     const uint64_t dims[3] = {(uint64_t)rq, (uint64_t)dv, (uint64_t)H};
     const uint64_t strides[2] = {(uint64_t)rq * 2, (uint64_t)dv * rq * 2};
-    const uint32_t box[3] = {(uint32_t)kKStep, (uint32_t)cw, (uint32_t)H};
+    const uint32_t box[3] = {(uint32_t)kKStep, (uint32_t)cw, (uint32_t)(H / 2)};  // a CTA's half of the rows
     if (!encode_tmap_bf16(&mb, 3, const_cast<hcadsa_bf16*>(Wg), dims, strides, box, true)) return HCADSA_ERR_CUDA;
   }
   Params p;
