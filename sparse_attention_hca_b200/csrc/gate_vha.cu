@@ -106,6 +106,29 @@ __device__ __forceinline__ void store_packed(uint16_t* p, const uint32_t (&w)[N 
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
+// 16 TMEM lanes, N columns, twice (.16x32bx2): threads 0-15 of the warp read lanes base + t at
+// columns [c, c + N), threads 16-31 the same lanes at columns [c + kOff, c + kOff + N).
+template <int N, int kOff>
+__device__ __forceinline__ void tmem_ld_16x2(uint32_t taddr, uint32_t (&r)[N]) {
+  if constexpr (N == 8) {
+    asm volatile("tcgen05.ld.sync.aligned.16x32bx2.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8], %9;"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+                 : "r"(taddr), "n"(kOff)
+                 : "memory");
+  } else if constexpr (N == 4) {
+    asm volatile("tcgen05.ld.sync.aligned.16x32bx2.x4.b32 {%0,%1,%2,%3}, [%4], %5;"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(taddr), "n"(kOff)
+                 : "memory");
+  } else {
+    static_assert(N == 2, "x2, x4 or x8");
+    asm volatile("tcgen05.ld.sync.aligned.16x32bx2.x2.b32 {%0,%1}, [%2], %3;"
+                 : "=r"(r[0]), "=r"(r[1])
+                 : "r"(taddr), "n"(kOff)
+                 : "memory");
+  }
+}
+
 __device__ __forceinline__ uint32_t cluster_rank() {
   uint32_t r;
   asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
@@ -255,11 +278,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ------------------------------------------------------------ epilogue: two threads per token
     // Thread (token, half) owns channels half * CH .. + CH - 1 of the channel block, all heads.
+    // A token's two threads are lanes t and t + 16 of one warp (the warp covers 16 TMEM lanes
+    // of its quarter), so their O loads and Y stores fill whole 32-byte sectors per instruction.
     constexpr int CH = CW / 2;
     const int quarter = warp & 3;
-    const int half = (warp - 2) >> 2;
-    const int r = quarter * 32 + lane;
-    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const int wq = (warp - 2) >> 2;  // which 16 lanes of the quarter
+    const int half = lane >> 4;
+    const int r = quarter * 32 + wq * 16 + (lane & 15);
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32 + wq * 16) << 16;
     uint32_t tl = 0;
     bool ok = true;
     for (int t = pair; t < p.n_tiles; t += n_pairs, ++tl) {
@@ -298,21 +324,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       ok = mbar_wait(&bar.tfull[buf], (tl >> 1) & 1, &abort_flag, p.err) && ok;
       tc_fence_after();
-      // 32 TMEM columns = 32 / CW heads at a time: logits, mix, gate, store
+      // kHB heads at a time (32 logit registers): this thread's CH logits of each head, then the
+      // mix, the gate and the store
+      constexpr int kHB = 32 / CH;
+      static_assert(H % kHB == 0, "whole head batches");
 #pragma unroll
-      for (int c0 = 0; c0 < kN; c0 += 32) {
-        uint32_t zr[32];
-        tmem_ld32_nowait(tmem + lane_off + buf * kN + c0, zr);
-        tmem_wait_ld_regs(zr);
-        if (c0 + 32 == kN) {  // every logit of the tile is in registers: the buffer may be reused
+      for (int h0 = 0; h0 < H; h0 += kHB) {
+        uint32_t zr[kHB][CH];
+#pragma unroll
+        for (int hh = 0; hh < kHB; ++hh) tmem_ld_16x2<CH, CH>(tmem + lane_off + buf * kN + (h0 + hh) * CW, zr[hh]);
+        tmem_wait_ld_regs(reinterpret_cast<uint32_t(&)[32]>(zr));
+        if (h0 + kHB == H) {  // every logit of the tile is in registers: the buffer may be reused
           tc_fence_before();
           __syncwarp();
           if (lane == 0) arrive_cluster(cluster_addr(&bar.tempty[buf], 0));
         }
         if (!valid) continue;
 #pragma unroll
-        for (int hh = 0; hh < 32 / CW; ++hh) {
-          const int h = c0 / CW + hh;
+        for (int hh = 0; hh < kHB; ++hh) {
+          const int h = h0 + hh;
           const float4 u4 = *reinterpret_cast<const float4*>(&sU[h * kMaxR]);
           const float uq[kMaxR] = {u4.x, u4.y, u4.z, u4.w};
           uint32_t yw[CH / 2];
@@ -324,9 +354,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               o0 = fmaf(uq[q], proj[q][c], o0);
               o1 = fmaf(uq[q], proj[q][c + 1], o1);
             }
-            // this thread's logits: channel c of its half (both indices compile-time constants)
-            const float z0 = __uint_as_float(half ? zr[hh * CW + CH + c] : zr[hh * CW + c]);
-            const float z1 = __uint_as_float(half ? zr[hh * CW + CH + c + 1] : zr[hh * CW + c + 1]);
+            const float z0 = __uint_as_float(zr[hh][c]), z1 = __uint_as_float(zr[hh][c + 1]);
             yw[c / 2] = pack_bf16x2(sigmoidf(z0) * o0, sigmoidf(z1) * o1);
           }
           store_packed<CH>(p.Y + base + (size_t)h * p.dv, yw);
