@@ -288,18 +288,28 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32 + wq * 16) << 16;
     uint32_t tl = 0;
     bool ok = true;
-    for (int t = pair; t < p.n_tiles; t += n_pairs, ++tl) {
+    // this thread's row of a tile: whether it is a token, and where its O / Y values start
+    auto row_of = [&](int t, bool& v, size_t& b) {
       const int m = 2 * (t / p.n_blocks) + (int)rank, nb = t % p.n_blocks;
       const int token = m * kM + r;
-      const bool valid = token < p.rows;
-      const uint32_t buf = tl & 1;
-      const size_t base = ((size_t)(valid ? token : 0) * H) * p.dv + (size_t)nb * CW + half * CH;
-      // this thread's O values, every head at once (loads in flight together), kept for the mix
-      uint32_t ow[H][CH / 2];
-      if (valid) {
+      v = t < p.n_tiles && token < p.rows;
+      b = ((size_t)(v ? token : 0) * H) * p.dv + (size_t)nb * CW + half * CH;
+    };
+    // this thread's O values, every head; the next tile's are loaded head by head as soon as a
+    // head's mix has used them, so their latency overlaps the rest of the tile
+    uint32_t ow[H][CH / 2];
+    bool valid;
+    size_t base;
+    row_of(pair, valid, base);
+    if (valid) {
 #pragma unroll
-        for (int h = 0; h < H; ++h) load_packed<CH>(p.O + base + (size_t)h * p.dv, ow[h]);
-      }
+      for (int h = 0; h < H; ++h) load_packed<CH>(p.O + base + (size_t)h * p.dv, ow[h]);
+    }
+    for (int t = pair; t < p.n_tiles; t += n_pairs, ++tl) {
+      const uint32_t buf = tl & 1;
+      bool valid_n;
+      size_t base_n;
+      row_of(t + n_pairs, valid_n, base_n);
       // rank-r projections sum_h V[h,m] O[t,h,c] of this thread's channels
       float proj[kMaxR][CH];
 #pragma unroll
@@ -339,7 +349,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           __syncwarp();
           if (lane == 0) arrive_cluster(cluster_addr(&bar.tempty[buf], 0));
         }
-        if (!valid) continue;
+        if (!valid) {
+#pragma unroll
+          for (int hh = 0; hh < kHB; ++hh)
+            if (valid_n) load_packed<CH>(p.O + base_n + (size_t)(h0 + hh) * p.dv, ow[h0 + hh]);
+          continue;
+        }
 #pragma unroll
         for (int hh = 0; hh < kHB; ++hh) {
           const int h = h0 + hh;
@@ -358,8 +373,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             yw[c / 2] = pack_bf16x2(sigmoidf(z0) * o0, sigmoidf(z1) * o1);
           }
           store_packed<CH>(p.Y + base + (size_t)h * p.dv, yw);
+          if (valid_n) load_packed<CH>(p.O + base_n + (size_t)h * p.dv, ow[h]);  // head h is done
         }
       }
+      valid = valid_n;
+      base = base_n;
     }
   }
 
